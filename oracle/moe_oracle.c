@@ -1,0 +1,371 @@
+/*
+ * CPU oracle for the decode-time MoE layer with batch-aware expert
+ * re-routing.
+ *
+ * TEST INFRASTRUCTURE.  Only the test suite, the smoke check in
+ * __graft_entry__.py and the CPU-baseline / reference leg of bench.py may
+ * load this library.  The product library (libmoe_decode.so) never calls
+ * it, shares no source with it and has no fallback to it.
+ *
+ * Everything here is a plain, slow restatement of what the layer computes,
+ * in the order the definitions below state.  Build flags:
+ *   -O2 -ffp-contract=off -fno-fast-math  (no silent FMA contraction; every
+ *   fused multiply-add below is an explicit fmaf()).
+ *
+ * Sources (web pages; cited by title and section):
+ *  [R]   "Router Caching and Optimization", section "Analyzing Router
+ *        Inference Cost", steps 1-3: linear projection h = x W_g, softmax,
+ *        top-k selection.
+ *  [OEA] "Opportunistic Expert Activation: Batch-Aware Expert Routing for
+ *        Faster Decode Without Retraining", abstract and lay summary: each
+ *        token keeps its most important experts, then piggybacks on experts
+ *        already loaded for other tokens of the batch.
+ *  [XS]  "XShare: Collaborative in-Batch Expert Sharing for Faster MoE
+ *        Inference", AI summary and abstract: batch expert selection as a
+ *        modular optimisation (maximise the total gating score of the
+ *        selected experts), solved greedily.
+ *  [LX]  "Lynx: Enabling Efficient MoE Inference through Dynamic Batch-Aware
+ *        Expert Selection", section 1 (latency follows the number of distinct
+ *        experts the batch activates) and section 2.2 (every token keeps
+ *        k expert slots).
+ *
+ * Readings where the pages are silent (each one is also listed in the
+ * design notes):
+ *  - router in fp32 with a fixed summation order (canon_dot / canon_sum);
+ *  - exp is our own Cody-Waite range reduction plus a degree-7 Taylor
+ *    polynomial (exp_spec), so the probabilities are reproducible bit for bit;
+ *  - ranking is by logit, descending, ties to the lower expert index;
+ *  - OEA fills from the union of kept sets fixed before any fill, up to k
+ *    slots, short sets padded with (-1, 0);
+ *  - XShare scores sum each token's top-k gate probabilities, the budget is
+ *    min(M, |union of top-k sets|), ties to the lower index;
+ *  - gate weights are renormalised over the chosen set (all modes);
+ *  - the expert FFN is SwiGLU: down( silu(gate x) * (up x) ), in fp64.
+ *
+ * Pins: every function here is checked by tests that do not re-run it
+ * (see tests/test_oracle_*.py): exp_spec against libm within 2 ulp,
+ * canon_dot against an fp64 dot within the forward error bound, the routing
+ * against fp64 logits + a stable sort, OEA and XShare against their defining
+ * invariants and brute force over subsets, the FFN against a dense fp64
+ * torch restatement.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_MODE_NONE 0
+#define ORACLE_MODE_OEA 1
+#define ORACLE_MODE_XSHARE 2
+
+/* ---------------------------------------------------------------- exp ---
+ * exp_spec(x) for x in [-87, 0] (softmax arguments are l - max(l) <= 0).
+ * Cody-Waite: x = n ln2 + r with n = rint(x log2 e) and r computed in two
+ * fmaf steps from a split ln2 = LN2_HI + LN2_LO (LN2_HI holds the leading
+ * 15 significant bits of ln 2, LN2_LO the float nearest the remainder);
+ * exp(r) by the Taylor series to degree 7 in Horner form with fmaf;
+ * scaling by 2^n by adding n to the exponent field.  Returns +0 below -87.
+ */
+static const float LOG2E_F = 1.44269504088896341f;
+static const float LN2_HI = 0.693145751953125f;
+static const float LN2_LO = 1.42860682030941723212e-6f;
+
+static float f_from_bits(int32_t b) { float f; memcpy(&f, &b, 4); return f; }
+static int32_t bits_from_f(float f) { int32_t b; memcpy(&b, &f, 4); return b; }
+
+float oracle_exp_spec(float x)
+{
+    if (!(x >= -87.0f)) return 0.0f;
+    float n = rintf(x * LOG2E_F);
+    float r = fmaf(-n, LN2_HI, x);
+    r = fmaf(-n, LN2_LO, r);
+    /* Taylor coefficients 1/j!, each the float nearest the exact value */
+    float p = 1.0f / 5040.0f;
+    p = fmaf(p, r, 1.0f / 720.0f);
+    p = fmaf(p, r, 1.0f / 120.0f);
+    p = fmaf(p, r, 1.0f / 24.0f);
+    p = fmaf(p, r, 1.0f / 6.0f);
+    p = fmaf(p, r, 0.5f);
+    p = fmaf(p, r, 1.0f);
+    p = fmaf(p, r, 1.0f);
+    return f_from_bits(bits_from_f(p) + ((int32_t)n << 23));
+}
+
+void oracle_exp_spec_n(const float *x, float *y, int n)
+{
+    for (int i = 0; i < n; ++i) y[i] = oracle_exp_spec(x[i]);
+}
+
+/* ------------------------------------------------- canonical reductions ---
+ * The fp32 order both sides use.  32 partial sums ("lanes"); then a
+ * butterfly: for o = 16, 8, 4, 2, 1 every lane l adds lane l^o.  All lanes
+ * end equal (fp32 addition is commutative); lane 0 is the result. */
+static float butterfly32(float lane[32])
+{
+    for (int o = 16; o >= 1; o >>= 1) {
+        float nxt[32];
+        for (int l = 0; l < 32; ++l) nxt[l] = lane[l] + lane[l ^ o];
+        memcpy(lane, nxt, sizeof nxt);
+    }
+    return lane[0];
+}
+
+/* dot(a, b) over d (d % 8 == 0): lane l owns j = 256 c + 8 l + t for
+ * c = 0, 1, ... and t = 0..7, accumulated with fmaf from +0 in (c, t)
+ * ascending order; groups with j >= d are skipped. */
+float oracle_canon_dot(const float *a, const float *b, int d)
+{
+    float lane[32];
+    for (int l = 0; l < 32; ++l) {
+        float acc = 0.0f;
+        for (int c = 0; 256 * c < d; ++c) {
+            int j0 = 256 * c + 8 * l;
+            if (j0 >= d) continue;
+            for (int t = 0; t < 8; ++t) acc = fmaf(a[j0 + t], b[j0 + t], acc);
+        }
+        lane[l] = acc;
+    }
+    return butterfly32(lane);
+}
+
+/* sum of q[0..n): lane l adds q[l + 32 i] for i ascending, from +0. */
+float oracle_canon_sum(const float *q, int n)
+{
+    float lane[32];
+    for (int l = 0; l < 32; ++l) {
+        float acc = 0.0f;
+        for (int e = l; e < n; e += 32) acc = acc + q[e];
+        lane[l] = acc;
+    }
+    return butterfly32(lane);
+}
+
+/* ------------------------------------------------------------- ranking ---
+ * Expert a ranks before expert b for a token iff its logit is larger, or
+ * the logits are equal and a has the lower index. */
+static int ranks_before(const float *l, int a, int b)
+{
+    return l[a] > l[b] || (l[a] == l[b] && a < b);
+}
+
+/* order[0..E) = the token's experts in rank order (insertion sort). */
+static void token_order(const float *l, int E, int *order)
+{
+    for (int e = 0; e < E; ++e) {
+        int pos = e;
+        while (pos > 0 && ranks_before(l, e, order[pos - 1])) {
+            order[pos] = order[pos - 1];
+            --pos;
+        }
+        order[pos] = e;
+    }
+}
+
+/* Renormalise gate weights over a chosen set: w_s = p[e_s] / sum, the sum
+ * taken in fp32 over the slots in slot order from +0.  Slots with e < 0
+ * get w = 0. */
+static void renormalise(const float *p, const int *sel, int k, float *w)
+{
+    float s = 0.0f;
+    for (int j = 0; j < k; ++j)
+        if (sel[j] >= 0) s = s + p[sel[j]];
+    for (int j = 0; j < k; ++j) w[j] = sel[j] >= 0 ? p[sel[j]] / s : 0.0f;
+}
+
+/* ------------------------------------------------------------- router ---
+ * [R] steps 1-3.  logits[b][e] = canon_dot(x[b], Wg[e]) (+ bias[e]);
+ * probs[b] = softmax(logits[b]) with m = max, q = exp_spec(l - m),
+ * Z = canon_sum(q), p = q / Z; topk_idx[b] = the first k experts of the
+ * token's rank order; topk_w[b] = their probabilities renormalised over the
+ * k chosen (the same weights the NONE rule yields). */
+void oracle_route(const float *x, const float *Wg, const float *bias,
+                  int B, int d, int E, int k,
+                  float *logits, float *probs, int *topk_idx, float *topk_w)
+{
+    int *order = (int *)malloc(sizeof(int) * (size_t)E);
+    float *q = (float *)malloc(sizeof(float) * (size_t)E);
+    for (int b = 0; b < B; ++b) {
+        float *l = logits + (size_t)b * E;
+        for (int e = 0; e < E; ++e) {
+            float v = oracle_canon_dot(x + (size_t)b * d, Wg + (size_t)e * d, d);
+            l[e] = bias ? v + bias[e] : v;
+        }
+        float m = l[0];
+        for (int e = 1; e < E; ++e) m = l[e] > m ? l[e] : m;
+        for (int e = 0; e < E; ++e) q[e] = oracle_exp_spec(l[e] - m);
+        float Z = oracle_canon_sum(q, E);
+        float *p = probs + (size_t)b * E;
+        for (int e = 0; e < E; ++e) p[e] = q[e] / Z;
+        token_order(l, E, order);
+        for (int j = 0; j < k; ++j) topk_idx[(size_t)b * k + j] = order[j];
+        renormalise(p, topk_idx + (size_t)b * k, k, topk_w + (size_t)b * k);
+    }
+    free(order);
+    free(q);
+}
+
+/* ----------------------------------------------------------- reselect ---
+ * sel_idx[b][0..k) and sel_w[b][0..k) for one of three rules.
+ *   NONE   : the token's top-k (standard routing, [LX] section 1).
+ *   OEA    : [OEA].  K_b = first k0 of the order; U_kept = union of all
+ *            K_b, fixed before any fill; F_b = the first k - k0 experts of
+ *            the order that lie in U_kept and not in K_b; sel = K_b ++ F_b,
+ *            padded with -1 when U_kept \ K_b is short.
+ *   XSHARE : [XS].  T_b = top-k; U_base = union of T_b;
+ *            s_e = sum over b ascending of [e in T_b] p[b][e] (fp32, from
+ *            +0); M' = min(budget, |U_base|); S = the M' experts of U_base
+ *            with the largest s (ties to the lower index) -- the exact
+ *            maximiser of the modular objective sum_{e in S} s_e;
+ *            sel_b = the first k experts of the order that lie in S.
+ * Weights are renormalised over the chosen set in every mode. */
+void oracle_reselect(const float *logits, const float *probs,
+                     int B, int E, int k, int mode, int k0, int budget,
+                     int *sel_idx, float *sel_w)
+{
+    int *order = (int *)malloc(sizeof(int) * (size_t)B * E);
+    for (int b = 0; b < B; ++b) token_order(logits + (size_t)b * E, E, order + (size_t)b * E);
+    unsigned char *inset = (unsigned char *)calloc((size_t)E, 1);
+
+    if (mode == ORACLE_MODE_OEA) {
+        for (int b = 0; b < B; ++b)
+            for (int j = 0; j < k0; ++j) inset[order[(size_t)b * E + j]] = 1;   /* U_kept */
+        for (int b = 0; b < B; ++b) {
+            const int *ord = order + (size_t)b * E;
+            int *sel = sel_idx + (size_t)b * k;
+            int n = 0;
+            for (int j = 0; j < k0; ++j) sel[n++] = ord[j];
+            for (int j = k0; j < E && n < k; ++j)
+                if (inset[ord[j]]) sel[n++] = ord[j];
+            while (n < k) sel[n++] = -1;
+        }
+    } else if (mode == ORACLE_MODE_XSHARE) {
+        float *s = (float *)calloc((size_t)E, sizeof(float));
+        unsigned char *ubase = (unsigned char *)calloc((size_t)E, 1);
+        for (int b = 0; b < B; ++b)
+            for (int j = 0; j < k; ++j) ubase[order[(size_t)b * E + j]] = 1;
+        for (int e = 0; e < E; ++e) {
+            float acc = 0.0f;
+            for (int b = 0; b < B; ++b) {
+                int in_tb = 0;
+                for (int j = 0; j < k; ++j) in_tb |= order[(size_t)b * E + j] == e;
+                if (in_tb) acc = acc + probs[(size_t)b * E + e];
+            }
+            s[e] = acc;
+        }
+        int nbase = 0;
+        for (int e = 0; e < E; ++e) nbase += ubase[e];
+        int Mp = budget < nbase ? budget : nbase;
+        /* greedy: take the best remaining expert of U_base, M' times */
+        for (int t = 0; t < Mp; ++t) {
+            int best = -1;
+            for (int e = 0; e < E; ++e) {
+                if (!ubase[e] || inset[e]) continue;
+                if (best < 0 || s[e] > s[best]) best = e;   /* equal s keeps the lower index */
+            }
+            inset[best] = 1;
+        }
+        for (int b = 0; b < B; ++b) {
+            const int *ord = order + (size_t)b * E;
+            int *sel = sel_idx + (size_t)b * k;
+            int n = 0;
+            for (int j = 0; j < E && n < k; ++j)
+                if (inset[ord[j]]) sel[n++] = ord[j];
+            while (n < k) sel[n++] = -1;
+        }
+        free(s);
+        free(ubase);
+    } else {
+        for (int b = 0; b < B; ++b)
+            for (int j = 0; j < k; ++j) sel_idx[(size_t)b * k + j] = order[(size_t)b * E + j];
+    }
+    for (int b = 0; b < B; ++b)
+        renormalise(probs + (size_t)b * E, sel_idx + (size_t)b * k, k, sel_w + (size_t)b * k);
+    free(inset);
+    free(order);
+}
+
+/* -------------------------------------------------------------- lists ---
+ * Per-expert token lists.  active = experts with at least one assignment,
+ * ascending; offsets[i] = start of active[i]'s entries (offsets[n_active]
+ * = total pairs); entries of one expert in ascending token order.  Unused
+ * tail entries: active = -1, offsets = total, tok = -1, w = 0.
+ * Returns n_active. */
+int oracle_lists(const int *sel_idx, const float *sel_w, int B, int E, int k,
+                 int *active, int *offsets, int *tok, float *w)
+{
+    int n_active = 0, pos = 0;
+    for (int e = 0; e < E; ++e) {
+        int start = pos;
+        for (int b = 0; b < B; ++b)
+            for (int j = 0; j < k; ++j)
+                if (sel_idx[(size_t)b * k + j] == e) {
+                    tok[pos] = b;
+                    w[pos] = sel_w[(size_t)b * k + j];
+                    ++pos;
+                }
+        if (pos > start) {
+            active[n_active] = e;
+            offsets[n_active] = start;
+            ++n_active;
+        }
+    }
+    for (int i = n_active; i < E; ++i) active[i] = -1;
+    for (int i = n_active; i <= E; ++i) offsets[i] = pos;
+    for (int i = pos; i < B * k; ++i) { tok[i] = -1; w[i] = 0.0f; }
+    return n_active;
+}
+
+/* ---------------------------------------------------------------- FFN ---
+ * SwiGLU expert e on token x (fp64):  g_j = sum_i x_i Wgate[e][j][i],
+ * u_j = sum_i x_i Wup[e][j][i], h_j = silu(g_j) u_j with
+ * silu(z) = z / (1 + exp(-z)), o_i = sum_j Wdown[e][i][j] h_j.
+ * y[r] = sum over the token's slots (slot order) of w * o, for each token r
+ * listed in rows[0..n_rows) (all tokens when rows == NULL).  The bf16
+ * weights decode exactly to fp64.  Tokens are independent, so they may run
+ * on `threads` OpenMP threads without changing any result. */
+static double bf16_to_double(uint16_t h)
+{
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return (double)f;
+}
+
+void oracle_ffn(const float *x, const uint16_t *Wgate, const uint16_t *Wup,
+                const uint16_t *Wdown, int B, int d, int E, int k, int F,
+                const int *sel_idx, const float *sel_w,
+                const int *rows, int n_rows, int threads, double *y)
+{
+    (void)E;
+    int nr = rows ? n_rows : B;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(threads > 0 ? threads : 1)
+    for (int ri = 0; ri < nr; ++ri) {
+        int b = rows ? rows[ri] : ri;
+        double *yo = y + (size_t)ri * d;
+        double *h = (double *)malloc(sizeof(double) * (size_t)F);
+        for (int i = 0; i < d; ++i) yo[i] = 0.0;
+        for (int j = 0; j < k; ++j) {
+            int e = sel_idx[(size_t)b * k + j];
+            if (e < 0) continue;
+            double wt = (double)sel_w[(size_t)b * k + j];
+            const float *xb = x + (size_t)b * d;
+            for (int f = 0; f < F; ++f) {
+                const uint16_t *gr = Wgate + ((size_t)e * F + f) * d;
+                const uint16_t *ur = Wup + ((size_t)e * F + f) * d;
+                double g = 0.0, u = 0.0;
+                for (int i = 0; i < d; ++i) {
+                    g += (double)xb[i] * bf16_to_double(gr[i]);
+                    u += (double)xb[i] * bf16_to_double(ur[i]);
+                }
+                h[f] = g / (1.0 + exp(-g)) * u;
+            }
+            for (int i = 0; i < d; ++i) {
+                const uint16_t *dr = Wdown + ((size_t)e * d + i) * F;
+                double o = 0.0;
+                for (int f = 0; f < F; ++f) o += bf16_to_double(dr[f]) * h[f];
+                yo[i] += wt * o;
+            }
+        }
+        free(h);
+    }
+}

@@ -1,0 +1,264 @@
+"""Pins for the oracle's re-selection rules.
+
+OEA ("Opportunistic Expert Activation: Batch-Aware Expert Routing for
+Faster Decode Without Retraining", abstract and lay summary): checked
+against a declarative characterisation that determines the result
+uniquely (kept prefix, fills drawn from the union of kept sets, maximal
+fill count, and every skipped candidate ranked below every fill), plus the
+closed forms k0 = k (standard top-k) and B = 1 (only the kept experts).
+
+XShare ("XShare: Collaborative in-Batch Expert Sharing for Faster MoE
+Inference", AI summary and abstract): the chosen expert set is compared
+with an exhaustive search over all subsets of the batch union for the
+modular objective, plus the closed form budget >= |union| (standard top-k).
+
+Hand-derived cases (worked out in the comments) pin the fill order and the
+tie rules.
+"""
+import itertools
+
+import numpy as np
+import pytest
+
+import moe_synth as ms
+
+NONE, OEA, XSHARE = 0, 1, 2
+
+
+def _rank_order(logits):
+    B, E = logits.shape
+    idx = np.arange(E)
+    return np.stack([np.lexsort((idx, -logits[b].astype(np.float64))) for b in range(B)])
+
+
+def _random_router(rng, B, E, scale=1.5, skew=2.0):
+    logits = (rng.standard_normal((B, E)) * scale - skew * np.log1p(rng.permutation(E))).astype(np.float32)
+    p = np.exp(logits.astype(np.float64) - logits.max(1, keepdims=True))
+    probs = (p / p.sum(1, keepdims=True)).astype(np.float32)
+    return logits, probs
+
+
+def _check_weights(probs, sel, w):
+    for b in range(sel.shape[0]):
+        m = sel[b] >= 0
+        assert np.all(w[b, ~m] == 0)
+        pk = probs[b, sel[b, m]].astype(np.float64)
+        assert np.allclose(w[b, m], pk / pk.sum(), rtol=3e-7, atol=0)
+        assert abs(float(w[b, m].astype(np.float64).sum()) - 1.0) <= 1e-6
+
+
+def check_oea(logits, probs, sel, w, k, k0):
+    order = _rank_order(logits)
+    B = logits.shape[0]
+    kept = order[:, :k0]
+    u_kept = set(kept.ravel().tolist())
+    u_base = set(order[:, :k].ravel().tolist())
+    assert u_kept <= u_base
+    for b in range(B):
+        row = sel[b].tolist()
+        n = sum(1 for e in row if e >= 0)
+        assert all(e >= 0 for e in row[:n]) and all(e == -1 for e in row[n:])
+        chosen = row[:n]
+        assert len(set(chosen)) == n
+        assert chosen[:k0] == kept[b].tolist()                 # keeps its top-k0
+        fills = chosen[k0:]
+        cand = u_kept - set(kept[b].tolist())
+        assert set(fills) <= cand                              # only experts already loaded
+        assert len(fills) == min(k - k0, len(cand))            # as many as fit
+        rank = {e: r for r, e in enumerate(order[b].tolist())}
+        assert [rank[e] for e in fills] == sorted(rank[e] for e in fills)
+        rest = cand - set(fills)
+        if fills and rest:                                     # highest-ranked candidates
+            assert max(rank[e] for e in fills) < min(rank[e] for e in rest)
+    active = set(e for e in sel.ravel().tolist() if e >= 0)
+    assert active == u_kept
+    _check_weights(probs, sel, w)
+
+
+def _xshare_scores64(probs, order, k):
+    B, E = probs.shape
+    s = np.zeros(E)
+    for b in range(B):
+        for e in order[b, :k]:
+            s[e] += float(probs[b, e])
+    return s
+
+
+def check_xshare(logits, probs, sel, w, k, budget, brute=False):
+    order = _rank_order(logits)
+    B, E = logits.shape
+    u_base = sorted(set(order[:, :k].ravel().tolist()))
+    mp = min(budget, len(u_base))
+    S = sorted(set(e for e in sel.ravel().tolist() if e >= 0))
+    assert len(S) == mp and set(S) <= set(u_base)
+    for b in range(B):
+        row = sel[b].tolist()
+        assert all(e >= 0 for e in row) and len(set(row)) == k
+        want = [e for e in order[b].tolist() if e in set(S)][:k]
+        assert row == want
+    _check_weights(probs, sel, w)
+    if brute:
+        s = _xshare_scores64(probs, order, k)
+        got = s[S].sum()
+        best = max(s[list(c)].sum() for c in itertools.combinations(u_base, mp))
+        assert got >= best - 1e-6 * max(1.0, best)
+
+
+@pytest.mark.parametrize("seed", range(6))
+@pytest.mark.parametrize("k,k0", [(4, 1), (4, 2), (4, 3), (8, 2), (8, 4), (8, 6)])
+def test_oea_characterisation_random(oracle_lib, seed, k, k0):
+    rng = np.random.default_rng(100 * seed + 10 * k + k0)
+    B = int(rng.integers(1, 40))
+    E = int(rng.choice([16, 64, 128, 256]))
+    logits, probs = _random_router(rng, B, E)
+    sel, w = oracle_lib.reselect(logits, probs, k, OEA, k0=k0)
+    check_oea(logits, probs, sel, w, k, k0)
+
+
+@pytest.mark.parametrize("shape,B,k0", [("tiny", 4, 2), ("e64", 16, 4), ("q30b", 16, 2),
+                                        ("q30b", 16, 4), ("q30b", 64, 6), ("q235b", 16, 4)])
+def test_oea_characterisation_layers(oracle_lib, shape, B, k0):
+    S = ms.SHAPES[shape]
+    L = ms.make_weights(S, 0, experts=False)
+    x = ms.make_tokens(S, B, 0)
+    logits, probs, ti, tw = oracle_lib.route(x, L["Wg"], L["bias"], S.k)
+    sel, w = oracle_lib.reselect(logits, probs, S.k, OEA, k0=k0)
+    check_oea(logits, probs, sel, w, S.k, k0)
+    base = len(set(ti.ravel().tolist()))
+    n_act = len(set(e for e in sel.ravel().tolist() if e >= 0))
+    assert n_act <= base
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_oea_k0_equals_k_is_standard_topk(oracle_lib, seed):
+    rng = np.random.default_rng(seed)
+    logits, probs = _random_router(rng, 17, 128)
+    s_none, w_none = oracle_lib.reselect(logits, probs, 8, NONE)
+    s_oea, w_oea = oracle_lib.reselect(logits, probs, 8, OEA, k0=8)
+    assert np.array_equal(s_none, s_oea)
+    assert np.array_equal(w_none.view(np.uint32), w_oea.view(np.uint32))
+    assert np.array_equal(s_none, _rank_order(logits)[:, :8])
+
+
+def test_oea_batch_of_one_keeps_only_k0(oracle_lib):
+    rng = np.random.default_rng(3)
+    logits, probs = _random_router(rng, 1, 128)
+    for k0 in range(1, 9):
+        sel, w = oracle_lib.reselect(logits, probs, 8, OEA, k0=k0)
+        assert (sel >= 0).sum() == k0
+        assert sel[0, :k0].tolist() == _rank_order(logits)[0, :k0].tolist()
+
+
+def test_oea_hand_worked_example(oracle_lib):
+    # B=3, E=6, k=3, k0=1.  Rank orders:
+    #   token 0: 0 3 1 2 4 5   kept {0}
+    #   token 1: 1 0 5 2 3 4   kept {1}
+    #   token 2: 2 4 3 0 1 5   kept {2}
+    # U_kept = {0,1,2}.  Fills walk each order and take members of U_kept:
+    #   token 0: 3 no, 1 yes, 2 yes      -> [0, 1, 2]
+    #   token 1: 0 yes, 5 no, 2 yes      -> [1, 0, 2]
+    #   token 2: 4 no, 3 no, 0 yes, 1 yes -> [2, 0, 1]
+    # Standard top-3 would activate all 6 experts; OEA activates 3.
+    orders = [[0, 3, 1, 2, 4, 5], [1, 0, 5, 2, 3, 4], [2, 4, 3, 0, 1, 5]]
+    logits = np.zeros((3, 6), np.float32)
+    for b, o in enumerate(orders):
+        for r, e in enumerate(o):
+            logits[b, e] = 5.0 - r
+    p = np.exp(logits - logits.max(1, keepdims=True))
+    probs = (p / p.sum(1, keepdims=True)).astype(np.float32)
+    sel, w = oracle_lib.reselect(logits, probs, 3, OEA, k0=1)
+    assert sel.tolist() == [[0, 1, 2], [1, 0, 2], [2, 0, 1]]
+    sel_n, _ = oracle_lib.reselect(logits, probs, 3, NONE)
+    assert sel_n.tolist() == [[0, 3, 1], [1, 0, 5], [2, 4, 3]]
+
+
+def test_oea_short_sets_are_padded(oracle_lib):
+    # both tokens keep expert 0 (k0=1): U_kept = {0} leaves nothing to fill,
+    # so each token runs one expert with weight 1 and two empty slots.
+    logits = np.array([[9, 8, 7, 6, 5, 4], [9, 7, 8, 6, 5, 4]], np.float32)
+    p = np.exp(logits - 9)
+    probs = (p / p.sum(1, keepdims=True)).astype(np.float32)
+    sel, w = oracle_lib.reselect(logits, probs, 3, OEA, k0=1)
+    assert sel.tolist() == [[0, -1, -1], [0, -1, -1]]
+    assert w.tolist() == [[1.0, 0.0, 0.0], [1.0, 0.0, 0.0]]
+
+
+@pytest.mark.parametrize("seed", range(8))
+@pytest.mark.parametrize("budget", [4, 6, 8])
+def test_xshare_brute_force_tiny(oracle_lib, seed, budget):
+    # E=16, B=4, k=4: every subset of the batch union of size M' is tried
+    rng = np.random.default_rng(1000 + seed)
+    logits, probs = _random_router(rng, 4, 16, scale=1.0, skew=0.5)
+    sel, w = oracle_lib.reselect(logits, probs, 4, XSHARE, budget=budget)
+    check_xshare(logits, probs, sel, w, 4, budget, brute=True)
+
+
+def test_xshare_brute_force_tiny_layer(oracle_lib):
+    S = ms.SHAPES["tiny"]
+    L = ms.make_weights(S, 0, experts=False)
+    for seed in range(3):
+        x = ms.make_tokens(S, 4, seed)
+        logits, probs, ti, tw = oracle_lib.route(x, L["Wg"], L["bias"], S.k)
+        for budget in (4, 6, 8):
+            sel, w = oracle_lib.reselect(logits, probs, S.k, XSHARE, budget=budget)
+            check_xshare(logits, probs, sel, w, S.k, budget, brute=True)
+
+
+@pytest.mark.parametrize("budget", [24, 32, 48])
+def test_xshare_speculative_batch(oracle_lib, budget):
+    S = ms.SHAPES["q30b"]
+    L = ms.make_weights(S, 0, experts=False)
+    x = ms.make_tokens(S, 32, 0, kind="spec")
+    logits, probs, ti, tw = oracle_lib.route(x, L["Wg"], L["bias"], S.k)
+    sel, w = oracle_lib.reselect(logits, probs, S.k, XSHARE, budget=budget)
+    check_xshare(logits, probs, sel, w, S.k, budget)
+    assert len(set(sel.ravel().tolist())) <= min(budget, len(set(ti.ravel().tolist())))
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_xshare_large_budget_is_standard_topk(oracle_lib, seed):
+    rng = np.random.default_rng(50 + seed)
+    logits, probs = _random_router(rng, 16, 128)
+    s_none, w_none = oracle_lib.reselect(logits, probs, 8, NONE)
+    s_x, w_x = oracle_lib.reselect(logits, probs, 8, XSHARE, budget=128)
+    assert np.array_equal(s_none, s_x)
+    assert np.array_equal(w_none.view(np.uint32), w_x.view(np.uint32))
+
+
+def test_xshare_hand_worked_ties(oracle_lib):
+    # B=2, E=6, k=2.  p0 = [.3 .3 .1 .1 .1 .1], p1 = [.1 .1 .3 .3 .1 .1].
+    # T_0 = {0,1}, T_1 = {2,3} (equal logits go to the lower index).
+    # Scores s = [.3 .3 .3 .3 0 0]; budget 2 -> four-way tie -> S = {0, 1}.
+    # Token 1's order is 2 3 0 1 4 5, so within S it takes [0, 1].
+    p = np.array([[.3, .3, .1, .1, .1, .1], [.1, .1, .3, .3, .1, .1]], np.float32)
+    logits = np.log(p).astype(np.float32)
+    sel, w = oracle_lib.reselect(logits, p, 2, XSHARE, budget=2)
+    assert sel.tolist() == [[0, 1], [0, 1]]
+    assert np.allclose(w, 0.5)
+    sel3, _ = oracle_lib.reselect(logits, p, 2, XSHARE, budget=3)
+    assert sel3.tolist() == [[0, 1], [2, 0]]
+
+
+@pytest.mark.parametrize("mode,k0,budget", [(NONE, 0, 0), (OEA, 2, 0), (XSHARE, 0, 20)])
+def test_lists_reconstruct_selection(oracle_lib, mode, k0, budget):
+    rng = np.random.default_rng(7)
+    B, E, k = 23, 64, 8
+    logits, probs = _random_router(rng, B, E)
+    sel, w = oracle_lib.reselect(logits, probs, k, mode, k0=k0, budget=budget)
+    li = oracle_lib.lists(sel, w, E)
+    n = li["n_active"]
+    act = li["active"][:n]
+    assert np.all(np.diff(act) > 0) and np.all(li["active"][n:] == -1)
+    assert set(act.tolist()) == set(e for e in sel.ravel().tolist() if e >= 0)
+    off = li["offsets"]
+    total = int((sel >= 0).sum())
+    assert off[0] == 0 and off[n] == total and np.all(off[n:] == total)
+    rebuilt = {}
+    for i, e in enumerate(act.tolist()):
+        toks = li["tok"][off[i]:off[i + 1]]
+        assert np.all(np.diff(toks) > 0)
+        for j, t in enumerate(toks.tolist()):
+            rebuilt[(t, e)] = li["w"][off[i] + j]
+    want = {(b, int(sel[b, j])): w[b, j] for b in range(B) for j in range(k) if sel[b, j] >= 0}
+    assert rebuilt == want
+    assert np.all(li["tok"][total:] == -1) and np.all(li["w"][total:] == 0)
