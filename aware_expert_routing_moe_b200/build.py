@@ -1,0 +1,82 @@
+"""Builds libmoe_decode.so in-tree with nvcc for sm_100a.
+
+    python -m aware_expert_routing_moe_b200.build [--force] [--verbose-ptxas]
+
+Each .cu file under csrc/ is compiled with
+``-gencode arch=compute_100a,code=sm_100a -O3 -lineinfo`` and linked into one
+shared library next to this file (the CUDA runtime is linked statically, so
+the library needs only the NVIDIA driver at run time).
+"""
+from __future__ import annotations
+
+import argparse
+import os
+import shutil
+import subprocess
+import sys
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
+CSRC = os.path.join(HERE, "csrc")
+INCLUDE = os.path.join(ROOT, "include")
+LIB = os.path.join(HERE, "libmoe_decode.so")
+BUILD_DIR = os.path.join(ROOT, "_build")
+
+SOURCES = ["router.cu", "expert.cu", "abi.cu"]
+GENCODE = "arch=compute_100a,code=sm_100a"
+
+
+def nvcc_path() -> str:
+    p = shutil.which("nvcc")
+    if p:
+        return p
+    cand = "/usr/local/cuda/bin/nvcc"
+    if os.path.exists(cand):
+        return cand
+    raise RuntimeError("nvcc not found")
+
+
+def _inputs():
+    files = [os.path.join(CSRC, s) for s in SOURCES]
+    files += [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".h", ".cuh"))]
+    files.append(os.path.join(INCLUDE, "moe_decode.h"))
+    return files
+
+
+def up_to_date() -> bool:
+    if not os.path.exists(LIB):
+        return False
+    t = os.path.getmtime(LIB)
+    return all(os.path.getmtime(f) <= t for f in _inputs())
+
+
+def build(force: bool = False, ptxas_verbose: bool = False) -> str:
+    if not force and up_to_date():
+        return LIB
+    nvcc = nvcc_path()
+    os.makedirs(BUILD_DIR, exist_ok=True)
+    objs = []
+    common = [nvcc, "-gencode", GENCODE, "-O3", "-lineinfo", "-std=c++17",
+              "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC]
+    if ptxas_verbose:
+        common += ["-Xptxas", "-v"]
+    for s in SOURCES:
+        obj = os.path.join(BUILD_DIR, s.replace(".cu", ".o"))
+        subprocess.run(common + ["-c", os.path.join(CSRC, s), "-o", obj], check=True)
+        objs.append(obj)
+    tmp = LIB + f".tmp{os.getpid()}"
+    subprocess.run([nvcc, "-gencode", GENCODE, "-shared", "-o", tmp] + objs, check=True)
+    os.replace(tmp, LIB)
+    return LIB
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--force", action="store_true")
+    ap.add_argument("--verbose-ptxas", action="store_true")
+    args = ap.parse_args(argv)
+    print(build(force=args.force, ptxas_verbose=args.verbose_ptxas))
+
+
+if __name__ == "__main__":
+    sys.exit(main())

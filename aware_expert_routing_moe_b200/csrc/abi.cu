@@ -1,0 +1,293 @@
+// Host side of the C ABI declared in include/moe_decode.h: argument
+// validation, workspace layout, TMA descriptor encoding and launch chaining.
+// Nothing here allocates device memory; every failure is reported as a
+// status code before anything is enqueued.
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+constexpr size_t ALIGN = 256;
+
+size_t round_up(size_t v) { return (v + ALIGN - 1) / ALIGN * ALIGN; }
+
+// B, E, k: every entry point; d: all but moe_reselect; d_ff: the FFN paths.
+bool dims_ok_reselect(const moe_dims_t &d) {
+    if (d.B < 1 || d.B > B_MAX) return false;
+    if (d.k < 1 || d.k > K_MAX) return false;
+    if (d.E < d.k || d.E > E_MAX) return false;
+    return true;
+}
+
+bool dims_ok_route(const moe_dims_t &d) {
+    return dims_ok_reselect(d) && d.d >= D_MIN && d.d <= D_MAX && d.d % 64 == 0;
+}
+
+bool dims_ok(const moe_dims_t &d) {
+    return dims_ok_route(d) && d.d_ff >= F_MIN && d.d_ff <= F_MAX && d.d_ff % 64 == 0;
+}
+
+bool rule_ok(const moe_dims_t &d, const moe_reselect_t &r) {
+    switch (r.mode) {
+        case MOE_RESELECT_NONE: return true;
+        case MOE_RESELECT_OEA: return r.k0 >= 1 && r.k0 <= d.k;
+        case MOE_RESELECT_XSHARE: return r.budget >= d.k && r.budget <= d.E;
+        default: return false;
+    }
+}
+
+bool al16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool al256(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+
+moe_status_t check_lists(const moe_lists_t &l) {
+    if (!l.n_active || !l.active || !l.offsets || !l.tok || !l.w) return MOE_ERR_INVALID_ARG;
+    if (!al16(l.n_active) || !al16(l.active) || !al16(l.offsets) || !al16(l.tok) || !al16(l.w))
+        return MOE_ERR_MISALIGNED;
+    return MOE_OK;
+}
+
+moe_status_t check_ws(const moe_dims_t &d, void *ws, size_t ws_bytes) {
+    if (!ws) return MOE_ERR_WORKSPACE;
+    if (!al256(ws)) return MOE_ERR_MISALIGNED;
+    if (ws_bytes < ws_layout(d).total) return MOE_ERR_WORKSPACE;
+    return MOE_OK;
+}
+
+// The current device must be an sm_100 part (B200).  Cached per device.
+moe_status_t check_device() {
+    static int cached[64] = {0};  // 0 unknown, 1 ok, 2 unsupported
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
+    if (dev < 0 || dev >= 64) return MOE_ERR_UNSUPPORTED;
+    if (cached[dev] == 0) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return MOE_ERR_CUDA;
+        }
+        cached[dev] = (major == 10 && minor == 0) ? 1 : 2;
+    }
+    return cached[dev] == 1 ? MOE_OK : MOE_ERR_UNSUPPORTED;
+}
+
+moe_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// ---------------------------------------------------------- tensor maps --
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+        else
+            cudaGetLastError();
+    });
+    return fn;
+}
+
+// 2-D bf16 matrix [rows][cols] (row-major), boxes of box_rows x 64 columns
+// (128 bytes, the 128B swizzle span).  Out-of-range elements read as zero.
+bool encode_bf16_2d(CUtensorMap *map, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t gdim[2] = {cols, rows};
+    cuuint64_t gstride[1] = {cols * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t estride[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), gdim, gstride, box, estride,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool encode_expert_maps(ExpertMaps *m, const moe_dims_t &d, const uint16_t *Wgate, const uint16_t *Wup,
+                        const uint16_t *Wdown, const uint16_t *h) {
+    std::memset(m, 0, sizeof(*m));
+    const uint64_t E = d.E, F = d.d_ff, D = d.d;
+    return encode_bf16_2d(&m->gate, Wgate, E * F, D, 16) && encode_bf16_2d(&m->up, Wup, E * F, D, 16) &&
+           encode_bf16_2d(&m->down, Wdown, E * D, F, 64) &&
+           encode_bf16_2d(&m->h, h, static_cast<uint64_t>(d.B) * d.k, F, expert_ffn_h_rows());
+}
+
+template <typename T>
+T *seg(void *ws, size_t off) {
+    return reinterpret_cast<T *>(static_cast<unsigned char *>(ws) + off);
+}
+
+moe_lists_t ws_lists(void *ws, const WsLayout &L) {
+    moe_lists_t l;
+    l.n_active = seg<int32_t>(ws, L.n_active);
+    l.active = seg<int32_t>(ws, L.active);
+    l.offsets = seg<int32_t>(ws, L.offsets);
+    l.tok = seg<int32_t>(ws, L.tok);
+    l.w = seg<float>(ws, L.w);
+    return l;
+}
+
+}  // namespace
+
+WsLayout ws_layout(const moe_dims_t &d) {
+    WsLayout L;
+    size_t o = 0;
+    const size_t B = d.B, E = d.E, k = d.k, D = d.d, F = d.d_ff;
+    L.counters = o; o += round_up(sizeof(Counters));
+    L.logits = o;   o += round_up(B * E * 4);
+    L.probs = o;    o += round_up(B * E * 4);
+    L.sel_idx = o;  o += round_up(B * k * 4);
+    L.sel_w = o;    o += round_up(B * k * 4);
+    L.n_active = o; o += round_up(4);
+    L.active = o;   o += round_up(E * 4);
+    L.offsets = o;  o += round_up((E + 1) * 4);
+    L.tok = o;      o += round_up(B * k * 4);
+    L.w = o;        o += round_up(B * k * 4);
+    L.xb = o;       o += round_up(B * D * 2);
+    L.h = o;        o += round_up(B * k * F * 2);
+    L.total = o;
+    return L;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+size_t moe_workspace_bytes(moe_dims_t dims) {
+    if (!dims_ok(dims)) return 0;
+    return ws_layout(dims).total;
+}
+
+const char *moe_status_string(moe_status_t s) {
+    switch (s) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument (null pointer, dimension or rule parameter)";
+        case MOE_ERR_MISALIGNED: return "misaligned buffer (device buffers 16-byte, workspace 256-byte)";
+        case MOE_ERR_WORKSPACE: return "workspace missing or smaller than moe_workspace_bytes()";
+        case MOE_ERR_UNSUPPORTED: return "unsupported: outside the implemented limits or not an sm_100 device";
+        case MOE_ERR_CUDA: return "a CUDA call or kernel launch failed";
+        case MOE_ERR_INTERNAL: return "a kernel recorded an internal error (bounded wait expired or bad lists)";
+        default: return "unknown status";
+    }
+}
+
+moe_status_t moe_route(const float *x, const float *Wg, const float *bias, moe_dims_t dims, float *logits,
+                       float *probs, int32_t *topk_idx, float *topk_w, void *stream) {
+    if (!dims_ok_route(dims)) return MOE_ERR_INVALID_ARG;
+    if (!x || !Wg || !logits || !probs || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+    if (!al16(x) || !al16(Wg) || (bias && !al16(bias)) || !al16(logits) || !al16(probs) || !al16(topk_idx) ||
+        !al16(topk_w))
+        return MOE_ERR_MISALIGNED;
+    moe_status_t st = check_device();
+    if (st != MOE_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    st = from_cuda(launch_router_logits(x, Wg, bias, dims, logits, nullptr, nullptr, s));
+    if (st != MOE_OK) return st;
+    return from_cuda(launch_route_topk(logits, dims, probs, topk_idx, topk_w, s));
+}
+
+moe_status_t moe_reselect(const float *logits, const float *probs, moe_dims_t dims, moe_reselect_t rule,
+                          int32_t *sel_idx, float *sel_w, moe_lists_t lists, void *stream) {
+    if (!dims_ok_reselect(dims) || !rule_ok(dims, rule)) return MOE_ERR_INVALID_ARG;
+    if (!logits || !probs || !sel_idx || !sel_w) return MOE_ERR_INVALID_ARG;
+    moe_status_t st = check_lists(lists);
+    if (st != MOE_OK) return st;
+    if (!al16(logits) || !al16(probs) || !al16(sel_idx) || !al16(sel_w)) return MOE_ERR_MISALIGNED;
+    st = check_device();
+    if (st != MOE_OK) return st;
+    return from_cuda(launch_reselect(logits, const_cast<float *>(probs), false, dims, rule, sel_idx, sel_w, lists,
+                                     nullptr, nullptr, false, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_expert_ffn(const float *x, const uint16_t *Wgate, const uint16_t *Wup, const uint16_t *Wdown,
+                            moe_dims_t dims, moe_lists_t lists, float *y, void *ws, size_t ws_bytes,
+                            void *stream) {
+    if (!dims_ok(dims)) return MOE_ERR_INVALID_ARG;
+    if (!x || !Wgate || !Wup || !Wdown || !y) return MOE_ERR_INVALID_ARG;
+    moe_status_t st = check_lists(lists);
+    if (st != MOE_OK) return st;
+    if (!al16(x) || !al16(Wgate) || !al16(Wup) || !al16(Wdown) || !al16(y)) return MOE_ERR_MISALIGNED;
+    st = check_ws(dims, ws, ws_bytes);
+    if (st != MOE_OK) return st;
+    st = check_device();
+    if (st != MOE_OK) return st;
+    const WsLayout L = ws_layout(dims);
+    ExpertMaps maps;
+    if (!encode_expert_maps(&maps, dims, Wgate, Wup, Wdown, seg<uint16_t>(ws, L.h))) return MOE_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    Counters *ctr = seg<Counters>(ws, L.counters);
+    uint16_t *xb = seg<uint16_t>(ws, L.xb);
+    st = from_cuda(launch_ffn_prep(x, dims, xb, y, ctr, s));
+    if (st != MOE_OK) return st;
+    return from_cuda(launch_expert_ffn(maps, xb, dims, lists, y, seg<uint16_t>(ws, L.h), ctr, true, s));
+}
+
+moe_status_t moe_layer_decode(const float *x, const float *Wg, const float *bias, const uint16_t *Wgate,
+                              const uint16_t *Wup, const uint16_t *Wdown, moe_dims_t dims, moe_reselect_t rule,
+                              float *y, int32_t *sel_idx, float *sel_w, int32_t *n_active, void *ws,
+                              size_t ws_bytes, void *stream) {
+    if (!dims_ok(dims) || !rule_ok(dims, rule)) return MOE_ERR_INVALID_ARG;
+    if (!x || !Wg || !Wgate || !Wup || !Wdown || !y) return MOE_ERR_INVALID_ARG;
+    if (!al16(x) || !al16(Wg) || (bias && !al16(bias)) || !al16(Wgate) || !al16(Wup) || !al16(Wdown) ||
+        !al16(y) || (sel_idx && !al16(sel_idx)) || (sel_w && !al16(sel_w)) || (n_active && !al16(n_active)))
+        return MOE_ERR_MISALIGNED;
+    moe_status_t st = check_ws(dims, ws, ws_bytes);
+    if (st != MOE_OK) return st;
+    st = check_device();
+    if (st != MOE_OK) return st;
+    const WsLayout L = ws_layout(dims);
+    ExpertMaps maps;
+    if (!encode_expert_maps(&maps, dims, Wgate, Wup, Wdown, seg<uint16_t>(ws, L.h))) return MOE_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    Counters *ctr = seg<Counters>(ws, L.counters);
+    uint16_t *xb = seg<uint16_t>(ws, L.xb);
+    float *logits = seg<float>(ws, L.logits);
+    float *probs = seg<float>(ws, L.probs);
+    int32_t *si = sel_idx ? sel_idx : seg<int32_t>(ws, L.sel_idx);
+    float *sw = sel_w ? sel_w : seg<float>(ws, L.sel_w);
+    const moe_lists_t lists = ws_lists(ws, L);
+    st = from_cuda(launch_router_logits(x, Wg, bias, dims, logits, xb, y, s));
+    if (st != MOE_OK) return st;
+    st = from_cuda(launch_reselect(logits, probs, true, dims, rule, si, sw, lists, n_active, ctr, true, s));
+    if (st != MOE_OK) return st;
+    return from_cuda(launch_expert_ffn(maps, xb, dims, lists, y, seg<uint16_t>(ws, L.h), ctr, true, s));
+}
+
+moe_status_t moe_check_error(void *ws, size_t ws_bytes, void *stream) {
+    if (!ws || ws_bytes < sizeof(Counters)) return MOE_ERR_WORKSPACE;
+    if (!al256(ws)) return MOE_ERR_MISALIGNED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    Counters *ctr = seg<Counters>(ws, 0);
+    int32_t err = 0;
+    if (cudaMemcpyAsync(&err, &ctr->error, sizeof(err), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
+    if (err != 0) {
+        if (cudaMemsetAsync(&ctr->error, 0, sizeof(int32_t), s) != cudaSuccess ||
+            cudaStreamSynchronize(s) != cudaSuccess) {
+            cudaGetLastError();
+            return MOE_ERR_CUDA;
+        }
+        return MOE_ERR_INTERNAL;
+    }
+    return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,603 @@
+// Router and batch-aware re-selection kernels (sm_100a).
+//
+//  router_logits_kernel : logits = x Wg^T + bias in a fixed fp32 order
+//      ("Router Caching and Optimization", "Analyzing Router Inference Cost",
+//      step 1).  Optionally also writes x as bf16 for the expert kernel and
+//      zeroes y (the layer path).
+//  route_topk_kernel    : warp per token: softmax (step 2) + top-k (step 3)
+//      with a warp-shuffle reduction and register-resident keys.
+//  reselect_kernel      : one CTA for the whole batch: (softmax +) top-k,
+//      OEA / XShare re-selection, renormalised weights, per-expert token
+//      lists, and the reset of the expert kernel's counters.
+//
+// Every floating-point step that decides an index is written with explicit
+// round-to-nearest intrinsics (__fmaf_rn, __fadd_rn, __fsub_rn, __fdiv_rn)
+// so that no contraction or reassociation can change a result:
+//  - dot products: lane l accumulates elements j = 256 c + 8 l + t (c, t
+//    ascending) with fma from +0, then a butterfly over lanes xor 16..1;
+//  - softmax: m = max, q = exp(l - m) with the library's own exp, Z = lane
+//    sums over e = l + 32 i (i ascending) then the butterfly, p = q / Z;
+//  - rank order: logit descending, equal logits to the lower expert index.
+#include <climits>
+#include <cmath>
+
+#include <cuda_bf16.h>
+
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+constexpr unsigned FULL = 0xffffffffu;
+
+// exp(x) for x in [-87, 0]: Cody-Waite reduction x = n ln2 + r with
+// n = rint(x log2 e), ln2 split into a 15-significant-bit head and a float
+// tail; exp(r) by its Taylor series to degree 7 (Horner, fma); 2^n applied
+// to the exponent field.  +0 below -87.
+__device__ __forceinline__ float exp_own(float x) {
+    if (!(x >= -87.0f)) return 0.0f;
+    const float kLog2e = 1.44269504088896341f;
+    const float kLn2Hi = 0.693145751953125f;
+    const float kLn2Lo = 1.42860682030941723212e-6f;
+    const float n = rintf(__fmul_rn(x, kLog2e));
+    float r = __fmaf_rn(-n, kLn2Hi, x);
+    r = __fmaf_rn(-n, kLn2Lo, r);
+    float p = 1.0f / 5040.0f;
+    p = __fmaf_rn(p, r, 1.0f / 720.0f);
+    p = __fmaf_rn(p, r, 1.0f / 120.0f);
+    p = __fmaf_rn(p, r, 1.0f / 24.0f);
+    p = __fmaf_rn(p, r, 1.0f / 6.0f);
+    p = __fmaf_rn(p, r, 0.5f);
+    p = __fmaf_rn(p, r, 1.0f);
+    p = __fmaf_rn(p, r, 1.0f);
+    return __int_as_float(__float_as_int(p) + (static_cast<int>(n) << 23));
+}
+
+__device__ __forceinline__ float warp_butterfly_sum(float v) {
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) v = __fadd_rn(v, __shfl_xor_sync(FULL, v, o));
+    return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) v = fmaxf(v, __shfl_xor_sync(FULL, v, o));
+    return v;
+}
+
+// Rank key: a larger key ranks earlier (larger logit, then lower index).
+// Key 0 never occurs for a real expert and marks "no candidate".
+__device__ __forceinline__ unsigned long long rank_key(float v, int idx) {
+    v = (v == 0.0f) ? 0.0f : v;  // -0 and +0 compare equal
+    const unsigned u = __float_as_uint(v);
+    const unsigned ord = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    return (static_cast<unsigned long long>(ord) << 32) | static_cast<unsigned>(~static_cast<unsigned>(idx));
+}
+
+// One round of warp arg-max over the lane's candidate bits; the winner is
+// removed from the candidates.  Returns the expert index or -1.
+template <int NI>
+__device__ __forceinline__ int warp_take_best(const unsigned long long (&key)[NI], unsigned &cand,
+                                              int lane) {
+    unsigned long long best = 0ull;
+#pragma unroll
+    for (int i = 0; i < NI; ++i)
+        if ((cand >> i) & 1u) best = key[i] > best ? key[i] : best;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+        const unsigned long long other = __shfl_xor_sync(FULL, best, o);
+        best = other > best ? other : best;
+    }
+    if (best == 0ull) return -1;
+    const int idx = static_cast<int>(~static_cast<unsigned>(best & 0xffffffffull));
+    if ((idx & 31) == lane) cand &= ~(1u << (idx >> 5));
+    return idx;
+}
+
+// Value held by the owner lane of expert e, broadcast to the warp.
+template <int NI>
+__device__ __forceinline__ float warp_fetch(const float (&v)[NI], int e) {
+    float mine = 0.0f;
+#pragma unroll
+    for (int i = 0; i < NI; ++i)
+        if (i == (e >> 5)) mine = v[i];
+    return __shfl_sync(FULL, mine, e & 31);
+}
+
+template <int NI>
+__device__ __forceinline__ void load_row(const float *row, int E, int lane, float (&l)[NI]) {
+#pragma unroll
+    for (int i = 0; i < NI; ++i) {
+        const int e = lane + 32 * i;
+        l[i] = e < E ? row[e] : -INFINITY;
+    }
+}
+
+template <int NI>
+__device__ __forceinline__ unsigned valid_bits(int E, int lane) {
+    unsigned m = 0;
+#pragma unroll
+    for (int i = 0; i < NI; ++i)
+        if (lane + 32 * i < E) m |= 1u << i;
+    return m;
+}
+
+// Softmax of one token's logits held lane-distributed (e = lane + 32 i).
+template <int NI>
+__device__ __forceinline__ void token_softmax(const float (&l)[NI], int E, int lane, float (&p)[NI]) {
+    float m = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < NI; ++i)
+        if (lane + 32 * i < E) m = fmaxf(m, l[i]);
+    m = warp_max(m);
+    float q[NI];
+    float acc = 0.0f;
+#pragma unroll
+    for (int i = 0; i < NI; ++i) {
+        if (lane + 32 * i < E) {
+            q[i] = exp_own(__fsub_rn(l[i], m));
+            acc = __fadd_rn(acc, q[i]);
+        } else {
+            q[i] = 0.0f;
+        }
+    }
+    const float Z = warp_butterfly_sum(acc);
+#pragma unroll
+    for (int i = 0; i < NI; ++i) p[i] = (lane + 32 * i < E) ? __fdiv_rn(q[i], Z) : 0.0f;
+}
+
+// Gate weights renormalised over the chosen slots (slot order, fp32 from
+// +0); every lane computes the same values.
+__device__ __forceinline__ void renormalise(const int (&sel)[K_MAX], const float (&ps)[K_MAX], int k,
+                                            float (&w)[K_MAX]) {
+    float s = 0.0f;
+#pragma unroll
+    for (int j = 0; j < K_MAX; ++j)
+        if (j < k && sel[j] >= 0) s = __fadd_rn(s, ps[j]);
+#pragma unroll
+    for (int j = 0; j < K_MAX; ++j) w[j] = (j < k && sel[j] >= 0) ? __fdiv_rn(ps[j], s) : 0.0f;
+}
+
+// ------------------------------------------------------------------ K1 --
+// Warp w of block (bx, by) computes expert e = 8 bx + w for tokens
+// TB by .. TB by + TB - 1.  The eight warps of a block read the same token
+// rows, which stay in L1.
+template <int TB>
+__global__ void __launch_bounds__(256) router_logits_kernel(
+    const float *__restrict__ x, const float *__restrict__ Wg, const float *__restrict__ bias,
+    int B, int d, int E, float *__restrict__ logits, uint16_t *__restrict__ xb,
+    float *__restrict__ y_zero) {
+    if (xb != nullptr) {
+        // layer path: x -> bf16 copy for the expert kernel, y = 0
+        const int n4 = B * d / 4;
+        const int nthreads = gridDim.x * gridDim.y * blockDim.x;
+        for (int i = (blockIdx.y * gridDim.x + blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+             i += nthreads) {
+            const float4 v = __ldg(reinterpret_cast<const float4 *>(x) + i);
+            const unsigned lo = static_cast<unsigned>(__bfloat16_as_ushort(__float2bfloat16_rn(v.x))) |
+                                (static_cast<unsigned>(__bfloat16_as_ushort(__float2bfloat16_rn(v.y))) << 16);
+            const unsigned hi = static_cast<unsigned>(__bfloat16_as_ushort(__float2bfloat16_rn(v.z))) |
+                                (static_cast<unsigned>(__bfloat16_as_ushort(__float2bfloat16_rn(v.w))) << 16);
+            reinterpret_cast<uint2 *>(xb)[i] = make_uint2(lo, hi);
+            if (y_zero) reinterpret_cast<float4 *>(y_zero)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int e = blockIdx.x * 8 + warp;
+    const int b0 = blockIdx.y * TB;
+    if (e < E) {
+        float acc[TB];
+#pragma unroll
+        for (int t = 0; t < TB; ++t) acc[t] = 0.0f;
+        const float *wrow = Wg + static_cast<size_t>(e) * d;
+        for (int c = 0; 256 * c < d; ++c) {
+            const int j0 = 256 * c + 8 * lane;
+            if (j0 >= d) continue;
+            const float4 w0 = __ldg(reinterpret_cast<const float4 *>(wrow + j0));
+            const float4 w1 = __ldg(reinterpret_cast<const float4 *>(wrow + j0 + 4));
+#pragma unroll
+            for (int t = 0; t < TB; ++t) {
+                if (b0 + t < B) {
+                    const float *xr = x + static_cast<size_t>(b0 + t) * d + j0;
+                    const float4 x0 = __ldg(reinterpret_cast<const float4 *>(xr));
+                    const float4 x1 = __ldg(reinterpret_cast<const float4 *>(xr + 4));
+                    float a = acc[t];
+                    a = __fmaf_rn(x0.x, w0.x, a);
+                    a = __fmaf_rn(x0.y, w0.y, a);
+                    a = __fmaf_rn(x0.z, w0.z, a);
+                    a = __fmaf_rn(x0.w, w0.w, a);
+                    a = __fmaf_rn(x1.x, w1.x, a);
+                    a = __fmaf_rn(x1.y, w1.y, a);
+                    a = __fmaf_rn(x1.z, w1.z, a);
+                    a = __fmaf_rn(x1.w, w1.w, a);
+                    acc[t] = a;
+                }
+            }
+        }
+        float mine = 0.0f;
+#pragma unroll
+        for (int t = 0; t < TB; ++t) {
+            const float v = warp_butterfly_sum(acc[t]);
+            if (lane == t) mine = v;
+        }
+        if (lane < TB && b0 + lane < B) {
+            const float v = bias ? __fadd_rn(mine, __ldg(bias + e)) : mine;
+            logits[static_cast<size_t>(b0 + lane) * E + e] = v;
+        }
+    }
+    // let the dependent (re-selection) kernel become resident; it waits for
+    // this grid's completion before reading the logits
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ------------------------------------------------------------ route only --
+template <int NI>
+__global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict__ logits, int B, int E,
+                                                         int k, float *__restrict__ probs,
+                                                         int32_t *__restrict__ topk_idx,
+                                                         float *__restrict__ topk_w) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int b = blockIdx.x * 8 + warp;
+    if (b >= B) return;
+    float l[NI], p[NI];
+    load_row<NI>(logits + static_cast<size_t>(b) * E, E, lane, l);
+    token_softmax<NI>(l, E, lane, p);
+#pragma unroll
+    for (int i = 0; i < NI; ++i)
+        if (lane + 32 * i < E) probs[static_cast<size_t>(b) * E + lane + 32 * i] = p[i];
+    unsigned long long key[NI];
+#pragma unroll
+    for (int i = 0; i < NI; ++i) key[i] = rank_key(l[i], lane + 32 * i);
+    unsigned cand = valid_bits<NI>(E, lane);
+    int sel[K_MAX];
+    float ps[K_MAX], w[K_MAX];
+#pragma unroll
+    for (int j = 0; j < K_MAX; ++j) {
+        sel[j] = -1;
+        ps[j] = 0.0f;
+        if (j < k) {
+            sel[j] = warp_take_best<NI>(key, cand, lane);
+            ps[j] = warp_fetch<NI>(p, sel[j]);
+        }
+    }
+    renormalise(sel, ps, k, w);
+#pragma unroll
+    for (int j = 0; j < K_MAX; ++j)
+        if (j < k && lane == j) {
+            topk_idx[static_cast<size_t>(b) * k + j] = sel[j];
+            topk_w[static_cast<size_t>(b) * k + j] = w[j];
+        }
+}
+
+// -------------------------------------------------------------- reselect --
+struct ReselectArgs {
+    const float *logits;
+    float *probs;  // read, or written when fuse_softmax
+    int fuse_softmax;
+    int B, E, k, mode, k0, budget;
+    int32_t *sel_idx;
+    float *sel_w;
+    moe_lists_t lists;
+    int32_t *n_active_copy;
+    Counters *ctr;
+};
+
+// Inclusive scan over threads 0..255 (value 0 for t >= n); every thread of
+// the block must call it.  Returns the inclusive prefix, sets *total.
+__device__ int block_scan256(int v, int *wsum, int *total) {
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(FULL, incl, o);
+        if (lane >= o) incl += u;
+    }
+    if (warp < 8 && lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    if (t == 0) {
+        int run = 0;
+        for (int i = 0; i < 8; ++i) {
+            const int s = wsum[i];
+            wsum[i] = run;
+            run += s;
+        }
+        wsum[8] = run;
+    }
+    __syncthreads();
+    const int res = (warp < 8) ? incl + wsum[warp] : 0;
+    *total = wsum[8];
+    __syncthreads();
+    return res;
+}
+
+template <int NI>
+__global__ void __launch_bounds__(1024, 1) reselect_kernel(ReselectArgs a) {
+    // wait until the router's logits are complete and visible
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    // the expert kernel may become resident now; it waits for this grid
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const int B = a.B, E = a.E, k = a.k;
+    const int BW = (B + 31) >> 5;
+    int *T = reinterpret_cast<int *>(smem_raw);                  // [B][k]
+    int *SEL = T + B * k;                                          // [B][k]
+    float *SELW = reinterpret_cast<float *>(SEL + B * k);         // [B][k]
+    unsigned *ASSIGN = reinterpret_cast<unsigned *>(SELW + B * k);  // [E][BW]
+    unsigned *TMEMB = ASSIGN + E * BW;                              // [E][BW]
+    __shared__ float s_score[E_MAX];
+    __shared__ int s_off[E_MAX];
+    __shared__ unsigned ukept[E_MAX / 32], ubase[E_MAX / 32], sbits[E_MAX / 32];
+    __shared__ int wsum[9];
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (int i = tid; i < 2 * E * BW; i += blockDim.x) ASSIGN[i] = 0u;  // and TMEMB
+    if (tid < E_MAX / 32) ukept[tid] = ubase[tid] = sbits[tid] = 0u;
+    __syncthreads();
+
+    const int mode = a.mode;
+    // ---- phase 1: per token softmax (layer path) + first ranks
+    const int r1 = (mode == MOE_RESELECT_OEA) ? a.k0 : k;
+    for (int b = warp; b < B; b += 32) {
+        float l[NI], p[NI];
+        load_row<NI>(a.logits + static_cast<size_t>(b) * E, E, lane, l);
+        if (a.fuse_softmax) {
+            token_softmax<NI>(l, E, lane, p);
+#pragma unroll
+            for (int i = 0; i < NI; ++i)
+                if (lane + 32 * i < E) a.probs[static_cast<size_t>(b) * E + lane + 32 * i] = p[i];
+        } else {
+            load_row<NI>(a.probs + static_cast<size_t>(b) * E, E, lane, p);
+        }
+        unsigned long long key[NI];
+#pragma unroll
+        for (int i = 0; i < NI; ++i) key[i] = rank_key(l[i], lane + 32 * i);
+        unsigned cand = valid_bits<NI>(E, lane);
+        int sel[K_MAX];
+        float ps[K_MAX];
+#pragma unroll
+        for (int j = 0; j < K_MAX; ++j) {
+            sel[j] = -1;
+            ps[j] = 0.0f;
+            if (j < r1) {
+                sel[j] = warp_take_best<NI>(key, cand, lane);
+                ps[j] = warp_fetch<NI>(p, sel[j]);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < K_MAX; ++j)
+            if (j < r1 && lane == j) {
+                const int e = sel[j];
+                T[b * k + j] = e;
+                if (mode == MOE_RESELECT_OEA) atomicOr(&ukept[e >> 5], 1u << (e & 31));
+                if (mode == MOE_RESELECT_XSHARE) {
+                    atomicOr(&ubase[e >> 5], 1u << (e & 31));
+                    atomicOr(&TMEMB[e * BW + (b >> 5)], 1u << (b & 31));
+                }
+            }
+        if (mode == MOE_RESELECT_NONE) {
+            float w[K_MAX];
+            renormalise(sel, ps, k, w);
+#pragma unroll
+            for (int j = 0; j < K_MAX; ++j)
+                if (j < k && lane == j) {
+                    SEL[b * k + j] = sel[j];
+                    SELW[b * k + j] = w[j];
+                }
+        }
+    }
+    __syncthreads();
+
+    // ---- XShare: batch scores, budget, greedy set (= top-M' by score)
+    if (mode == MOE_RESELECT_XSHARE) {
+        if (tid < E) {
+            float s = 0.0f;
+            for (int b = 0; b < B; ++b)
+                if ((TMEMB[tid * BW + (b >> 5)] >> (b & 31)) & 1u)
+                    s = __fadd_rn(s, a.probs[static_cast<size_t>(b) * E + tid]);
+            s_score[tid] = s;
+        }
+        __syncthreads();
+        if (tid < E && ((ubase[tid >> 5] >> (tid & 31)) & 1u)) {
+            int nb = 0;
+            for (int i = 0; i < E_MAX / 32; ++i) nb += __popc(ubase[i]);
+            const int Mp = a.budget < nb ? a.budget : nb;
+            const float se = s_score[tid];
+            int rank = 0;
+            for (int e2 = 0; e2 < E; ++e2) {
+                if (!((ubase[e2 >> 5] >> (e2 & 31)) & 1u)) continue;
+                const float s2 = s_score[e2];
+                rank += (s2 > se || (s2 == se && e2 < tid)) ? 1 : 0;
+            }
+            if (rank < Mp) atomicOr(&sbits[tid >> 5], 1u << (tid & 31));
+        }
+        __syncthreads();
+    }
+
+    // ---- phase 2: OEA fills / XShare top-k within the batch set; weights
+    if (mode != MOE_RESELECT_NONE) {
+        for (int b = warp; b < B; b += 32) {
+            float l[NI], p[NI];
+            load_row<NI>(a.logits + static_cast<size_t>(b) * E, E, lane, l);
+            load_row<NI>(a.probs + static_cast<size_t>(b) * E, E, lane, p);
+            unsigned long long key[NI];
+#pragma unroll
+            for (int i = 0; i < NI; ++i) key[i] = rank_key(l[i], lane + 32 * i);
+            unsigned cand = 0;
+            const unsigned *bits = (mode == MOE_RESELECT_OEA) ? ukept : sbits;
+#pragma unroll
+            for (int i = 0; i < NI; ++i) {
+                const int e = lane + 32 * i;
+                if (e < E && ((bits[e >> 5] >> (e & 31)) & 1u)) cand |= 1u << i;
+            }
+            int sel[K_MAX];
+            float ps[K_MAX];
+            const int kk = (mode == MOE_RESELECT_OEA) ? a.k0 : 0;
+#pragma unroll
+            for (int j = 0; j < K_MAX; ++j) {
+                sel[j] = -1;
+                ps[j] = 0.0f;
+                if (j < kk) {
+                    const int e = T[b * k + j];
+                    sel[j] = e;
+                    if ((e & 31) == lane) cand &= ~(1u << (e >> 5));
+                    ps[j] = warp_fetch<NI>(p, e);
+                }
+            }
+            int stop = 0;
+#pragma unroll
+            for (int j = 0; j < K_MAX; ++j) {
+                if (j >= kk && j < k && !stop) {
+                    const int e = warp_take_best<NI>(key, cand, lane);
+                    if (e < 0) {
+                        stop = 1;
+                    } else {
+                        sel[j] = e;
+                        ps[j] = warp_fetch<NI>(p, e);
+                    }
+                }
+            }
+            float w[K_MAX];
+            renormalise(sel, ps, k, w);
+#pragma unroll
+            for (int j = 0; j < K_MAX; ++j)
+                if (j < k && lane == j) {
+                    SEL[b * k + j] = sel[j];
+                    SELW[b * k + j] = w[j];
+                }
+        }
+        __syncthreads();
+    }
+
+    // ---- phase 3: assignment bits, counts, active list, offsets
+    for (int i = tid; i < B * k; i += blockDim.x) {
+        const int e = SEL[i];
+        const int b = i / k;
+        if (e >= 0) atomicOr(&ASSIGN[e * BW + (b >> 5)], 1u << (b & 31));
+        a.sel_idx[i] = e;
+        a.sel_w[i] = SELW[i];
+    }
+    __syncthreads();
+    int cnt = 0;
+    if (tid < E)
+        for (int wd = 0; wd < BW; ++wd) cnt += __popc(ASSIGN[tid * BW + wd]);
+    int n_active = 0, total = 0;
+    const int flag = (tid < E && cnt > 0) ? 1 : 0;
+    const int rank_incl = block_scan256(flag, wsum, &n_active);
+    const int off_incl = block_scan256(tid < E ? cnt : 0, wsum, &total);
+    if (tid < E) {
+        s_off[tid] = off_incl - cnt;
+        if (flag) {
+            a.lists.active[rank_incl - 1] = tid;
+            a.lists.offsets[rank_incl - 1] = off_incl - cnt;
+        }
+    }
+    if (tid >= n_active && tid < E) a.lists.active[tid] = -1;
+    if (tid >= n_active && tid <= E) a.lists.offsets[tid] = total;
+    if (tid == 0) {
+        *a.lists.n_active = n_active;
+        if (a.n_active_copy) *a.n_active_copy = n_active;
+    }
+    __syncthreads();
+
+    // ---- phase 4: compaction (expert ascending, token ascending)
+    for (int i = tid; i < B * k; i += blockDim.x) {
+        const int e = SEL[i];
+        if (e < 0) continue;
+        const int b = i / k;
+        int before = 0;
+        for (int wd = 0; wd < (b >> 5); ++wd) before += __popc(ASSIGN[e * BW + wd]);
+        before += __popc(ASSIGN[e * BW + (b >> 5)] & ((1u << (b & 31)) - 1u));
+        const int pos = s_off[e] + before;
+        a.lists.tok[pos] = b;
+        a.lists.w[pos] = SELW[i];
+    }
+    for (int i = total + tid; i < B * k; i += blockDim.x) {
+        a.lists.tok[i] = -1;
+        a.lists.w[i] = 0.0f;
+    }
+    // ---- reset the expert kernel's counters (layer path)
+    if (a.ctr) {
+        if (tid == 0) a.ctr->ticket = 0;
+        for (int i = tid; i < E_MAX; i += blockDim.x) a.ctr->gu_done[i] = 0;
+    }
+}
+
+int ni_for(int E) { return E <= 32 ? 1 : E <= 64 ? 2 : E <= 128 ? 4 : 8; }
+
+}  // namespace
+
+cudaError_t launch_router_logits(const float *x, const float *Wg, const float *bias,
+                                 const moe_dims_t &d, float *logits, uint16_t *xb,
+                                 float *y_zero, cudaStream_t s) {
+    constexpr int TB = 8;
+    dim3 grid((d.E + 7) / 8, (d.B + TB - 1) / TB);
+    router_logits_kernel<TB><<<grid, 256, 0, s>>>(x, Wg, bias, d.B, d.d, d.E, logits, xb, y_zero);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_route_topk(const float *logits, const moe_dims_t &d, float *probs,
+                              int32_t *topk_idx, float *topk_w, cudaStream_t s) {
+    dim3 grid((d.B + 7) / 8);
+    switch (ni_for(d.E)) {
+        case 1: route_topk_kernel<1><<<grid, 256, 0, s>>>(logits, d.B, d.E, d.k, probs, topk_idx, topk_w); break;
+        case 2: route_topk_kernel<2><<<grid, 256, 0, s>>>(logits, d.B, d.E, d.k, probs, topk_idx, topk_w); break;
+        case 4: route_topk_kernel<4><<<grid, 256, 0, s>>>(logits, d.B, d.E, d.k, probs, topk_idx, topk_w); break;
+        default: route_topk_kernel<8><<<grid, 256, 0, s>>>(logits, d.B, d.E, d.k, probs, topk_idx, topk_w); break;
+    }
+    return cudaGetLastError();
+}
+
+template <int NI>
+static cudaError_t launch_reselect_ni(const ReselectArgs &a, size_t smem, bool pdl, cudaStream_t s) {
+    static bool configured = false;  // the attribute is per function; set it once
+    cudaError_t err = cudaSuccess;
+    if (!configured) {
+        err = cudaFuncSetAttribute(reselect_kernel<NI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   96 * 1024);
+        if (err != cudaSuccess) return err;
+        configured = true;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1);
+    cfg.blockDim = dim3(1024);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, reselect_kernel<NI>, a);
+}
+
+cudaError_t launch_reselect(const float *logits, float *probs, bool fuse_softmax,
+                            const moe_dims_t &d, const moe_reselect_t &r,
+                            int32_t *sel_idx, float *sel_w, const moe_lists_t &l,
+                            int32_t *n_active_copy, Counters *ctr, bool pdl, cudaStream_t s) {
+    ReselectArgs a;
+    a.logits = logits;
+    a.probs = probs;
+    a.fuse_softmax = fuse_softmax ? 1 : 0;
+    a.B = d.B;
+    a.E = d.E;
+    a.k = d.k;
+    a.mode = r.mode;
+    a.k0 = r.k0;
+    a.budget = r.budget;
+    a.sel_idx = sel_idx;
+    a.sel_w = sel_w;
+    a.lists = l;
+    a.n_active_copy = n_active_copy;
+    a.ctr = ctr;
+    const int BW = (d.B + 31) / 32;
+    const size_t smem = static_cast<size_t>(d.B) * d.k * 12 + static_cast<size_t>(d.E) * BW * 8;
+    switch (ni_for(d.E)) {
+        case 1: return launch_reselect_ni<1>(a, smem, pdl, s);
+        case 2: return launch_reselect_ni<2>(a, smem, pdl, s);
+        case 4: return launch_reselect_ni<4>(a, smem, pdl, s);
+        default: return launch_reselect_ni<8>(a, smem, pdl, s);
+    }
+}
+
+}  // namespace moe

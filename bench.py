@@ -1,0 +1,418 @@
+#!/usr/bin/env python
+"""Benchmark of the decode-time MoE layer with batch-aware expert re-routing.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload q30b_b16_oea4] [--no-extra]
+
+One step = one moe_layer_decode call (router GEMV + softmax + top-k,
+re-selection + token lists, grouped SwiGLU expert FFN with the weighted
+combine) on one decode batch, inputs resident in HBM.  Weights rotate over
+4 identical copies (each larger than the 126 MB L2) so no step reads
+weights another step left in L2.  Steps run as CUDA-graph replays of 4
+consecutive layer calls (one per copy); the graph keeps every kernel of
+every call.
+
+Printed (rank 0, one JSON line): value = algorithmic bytes of all ranks per
+second (activated experts x 3 d d_ff x 2 B + router weights + x + y), the
+roofline of the expert kernel (events around moe_expert_ffn), the oracle
+timed on the host cores (cpu_baseline), an end-to-end number through the
+Python API with host buffers (e2e), and the SM clocks sampled with NVML
+during the timed region.
+
+N > 1 (torchrun): every rank runs an independent replica of the layer on
+its own GPU (the layer is single-GPU; there is no data-path collective);
+timing is the max over ranks; scaling is weak.
+
+--impl reference times the CPU oracle on the host cores instead (rank 0
+only), each step a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import moe_synth as ms  # noqa: E402
+
+METRIC = "MoE-layer decode µs & achieved HBM GB/s (% of roofline) vs batch size"
+UNIT = "GB/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+ROTATE = 4
+
+WORKLOADS = {
+    "q30b_b16_oea4": dict(shape="q30b", B=16, mode=1, k0=4, budget=0, rule="OEA k0=4"),
+    "q30b_b16_none": dict(shape="q30b", B=16, mode=0, k0=0, budget=0, rule="NONE (standard top-8)"),
+    "q30b_b64_oea4": dict(shape="q30b", B=64, mode=1, k0=4, budget=0, rule="OEA k0=4"),
+    "q235b_b16_oea4": dict(shape="q235b", B=16, mode=1, k0=4, budget=0, rule="OEA k0=4"),
+    "spec_xshare32": dict(shape="q30b", B=32, mode=2, k0=0, budget=32, rule="XShare budget=32",
+                          kind="spec"),
+}
+
+# DRAM bytes (read + write) per launch of the expert kernel from an ncu
+# capture of the same workload (profiles/expert_ffn_q30b_b16.md); None until
+# captured for the current kernel.
+NCU_TRAFFIC = {}
+
+
+def workload_desc(w: dict) -> str:
+    S = ms.SHAPES[w["shape"]]
+    name = {"q30b": "Qwen3-30B-A3B-shaped", "q235b": "Qwen3-235B-A22B-shaped"}[w["shape"]]
+    extra = ", speculative batch of 8 requests x 4 drafts" if w.get("kind") == "spec" else ""
+    return (f"{name} MoE layer (d={S.d}, E={S.E}, k={S.k}, d_ff={S.F}, bf16 experts), "
+            f"decode batch B={w['B']}{extra}, {w['rule']}")
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def algorithmic_bytes(S, B, n_active):
+    experts = n_active * 3 * S.d * S.F * 2
+    router = S.E * S.d * 4 + S.E * 4
+    io = B * S.d * 4 * 2
+    return experts + router + io, experts + io
+
+
+# ------------------------------------------------------------- clocks --
+class ClockSampler:
+    """Polls SM clock and clock-event reasons with NVML while running."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index: int):
+        self.samples, self.reasons = [], 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+
+    def summary(self):
+        if self._nv is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"], "samples": 0}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------- reference --
+def run_reference(args, w, rank):
+    import oracle
+    if rank != 0:
+        return
+    S = ms.SHAPES[w["shape"]]
+    L = ms.make_weights(S, 0)
+    x = ms.make_tokens(S, w["B"], 0, kind=w.get("kind", "normal"))
+    cores = len(os.sched_getaffinity(0))
+    r0 = oracle.layer(x, L, S.k, w["mode"], w["k0"], w["budget"], rows=np.arange(1, dtype=np.int32),
+                      threads=cores)
+    n_active = r0["lists"]["n_active"]
+    total_bytes, _ = algorithmic_bytes(S, w["B"], n_active)
+    # size one step: route + re-select the whole batch, FFN for `rows` tokens
+    t0 = time.perf_counter()
+    oracle.layer(x, L, S.k, w["mode"], w["k0"], w["budget"], rows=np.arange(1, dtype=np.int32), threads=cores)
+    t_one = time.perf_counter() - t0
+    budget_s = 150.0 / max(1, args.steps + args.warmup)
+    rows = int(max(1, min(w["B"], budget_s / max(t_one, 1e-6))))
+    sel = np.arange(rows, dtype=np.int32)
+
+    def step():
+        oracle.layer(x, L, S.k, w["mode"], w["k0"], w["budget"], rows=sel, threads=cores)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    value = total_bytes * rows / w["B"] / dt / 1e9
+    sample = (f"per step: router + {w['rule']} for all {w['B']} tokens, expert FFN for {rows} of "
+              f"{w['B']} tokens; bytes scaled by {rows}/{w['B']}")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_desc(w), "n_active": n_active},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline(w, S, L, x, seconds=12.0):
+    import oracle
+    cores = len(os.sched_getaffinity(0))
+    n = 0
+    t0 = time.perf_counter()
+    nact = None
+    while True:
+        r = oracle.layer(x, L, S.k, w["mode"], w["k0"], w["budget"], threads=cores)
+        nact = r["lists"]["n_active"]
+        n += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = (time.perf_counter() - t0) / n
+    total, _ = algorithmic_bytes(S, w["B"], nact)
+    return {"value": total / dt / 1e9, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{n} full layer calls (all {w['B']} tokens), {dt * 1e3:.1f} ms each"}
+
+
+# ---------------------------------------------------------------- ours --
+def run_ours(args, w, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import aware_expert_routing_moe_b200 as moe
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    moe.load_library()
+    S = ms.SHAPES[w["shape"]]
+    B, mode, k0, budget = w["B"], w["mode"], w["k0"], w["budget"]
+    L = ms.make_weights(S, 0)
+    x_np = ms.make_tokens(S, B, 0, kind=w.get("kind", "normal"))
+    t = lambda a: torch.from_numpy(a).to(dev)
+    Wg, bias = t(L["Wg"]), t(L["bias"])
+    copies = [(t(L["Wgate"].view(np.int16)), t(L["Wup"].view(np.int16)), t(L["Wdown"].view(np.int16)))]
+    for _ in range(ROTATE - 1):
+        copies.append(tuple(c.clone() for c in copies[0]))
+    x = t(x_np)
+    ws = moe.new_workspace(B, S.d, S.E, S.k, S.F, dev)
+    y = torch.empty(B, S.d, dtype=torch.float32, device=dev)
+    nact_t = torch.zeros(4, dtype=torch.int32, device=dev)
+    s = torch.cuda.Stream(dev)
+
+    def layer(r):
+        g, u, dn = copies[r]
+        moe.moe_layer_decode(x, Wg, bias, g, u, dn, S.k, mode, k0, budget, ws=ws, y=y, n_active=nact_t)
+
+    with torch.cuda.stream(s):
+        for r in range(ROTATE):
+            layer(r)
+    s.synchronize()
+    if moe.moe_check_error(ws, s) != 0:
+        raise RuntimeError("device error word set during warm-up")
+    n_active = int(nact_t[0].item())
+    total_bytes, ffn_bytes = algorithmic_bytes(S, B, n_active)
+
+    # CUDA graphs: one with ROTATE consecutive layer calls, and single calls
+    g_all = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_all, stream=s):
+        for r in range(ROTATE):
+            layer(r)
+    g_one = []
+    for r in range(ROTATE):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            layer(r)
+        g_one.append(g)
+
+    def replay(nsteps):
+        full, rest = divmod(nsteps, ROTATE)
+        for _ in range(full):
+            g_all.replay()
+        for r in range(rest):
+            g_one[r].replay()
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local_rank])
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        tv = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(tv, op=dist.ReduceOp.MAX)
+        return float(tv.item())
+
+    def timed(fn, nsteps, sampler=None):
+        barrier()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(s):
+            e0.record(s)
+            fn(nsteps)
+            e1.record(s)
+        e1.synchronize()
+        torch.cuda.synchronize(dev)
+        barrier()
+        return max_over_ranks(e0.elapsed_time(e1))  # ms, all steps
+
+    # ---- main timed region: K graph-replayed layer calls
+    with torch.cuda.stream(s):
+        replay(args.warmup)
+    sampler = ClockSampler(local_rank)
+    with sampler:
+        ms_total = timed(replay, args.steps)
+    clocks = sampler.summary()
+    ms_step = ms_total / args.steps
+    value = world * total_bytes / (ms_step * 1e-3) / 1e9
+
+    # ---- the same calls launched one by one from Python (launch overhead)
+    def stream_calls(nsteps):
+        for i in range(nsteps):
+            layer(i % ROTATE)
+
+    with torch.cuda.stream(s):
+        stream_calls(args.warmup)
+    ms_stream = timed(stream_calls, args.steps) / args.steps
+
+    # ---- expert kernel alone (roofline): lists from the routed batch
+    logits, probs, _, _ = moe.moe_route(x, Wg, bias, S.k)
+    _, _, lists = moe.moe_reselect(logits, probs, S.k, mode, k0, budget)
+    torch.cuda.synchronize(dev)
+    g_ffn = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_ffn, stream=s):
+        for r in range(ROTATE):
+            gg, uu, dd = copies[r]
+            moe.moe_expert_ffn(x, gg, uu, dd, lists, S.k, ws, y=y)
+    nrep = max(1, args.steps // ROTATE)
+    with torch.cuda.stream(s):
+        for _ in range(max(1, args.warmup // ROTATE)):
+            g_ffn.replay()
+    ms_ffn = timed(lambda n: [g_ffn.replay() for _ in range(n)], nrep) / (nrep * ROTATE)
+    hbm_peak, peak_kind = measured_peaks()
+    ffn_gbs = ffn_bytes / (ms_ffn * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": ffn_gbs, "peak": hbm_peak, "unit": "GB/s",
+                "frac": ffn_gbs / hbm_peak, "traffic": NCU_TRAFFIC.get(args.workload),
+                "kernel": "moe_expert_ffn (input prep + grouped SwiGLU expert kernel)",
+                "peak_source": f"{peak_kind} HBM copy bandwidth",
+                "frac_of_nominal_8tbs": ffn_gbs / NOMINAL_HBM_GBS}
+
+    # ---- end to end through the Python API with pinned host buffers
+    x_host = torch.from_numpy(x_np).pin_memory()
+    y_host = torch.empty(B, S.d, dtype=torch.float32).pin_memory()
+    x_dev = torch.empty_like(x)
+    y_dev = torch.empty_like(y)
+
+    def e2e_calls(nsteps):
+        for i in range(nsteps):
+            g, u, dn = copies[i % ROTATE]
+            x_dev.copy_(x_host, non_blocking=True)
+            moe.moe_layer_decode(x_dev, Wg, bias, g, u, dn, S.k, mode, k0, budget, ws=ws, y=y_dev)
+            y_host.copy_(y_dev, non_blocking=True)
+
+    with torch.cuda.stream(s):
+        e2e_calls(args.warmup)
+    ms_e2e = timed(e2e_calls, args.steps) / args.steps
+    e2e = {"value": world * total_bytes / (ms_e2e * 1e-3) / 1e9, "unit": UNIT,
+           "h2d_bytes_per_step": B * S.d * 4, "d2h_bytes_per_step": B * S.d * 4,
+           "ms_per_step": ms_e2e}
+    if moe.moe_check_error(ws, s) != 0:
+        raise RuntimeError("device error word set during the benchmark")
+
+    extra = {}
+    if not args.no_extra and rank == 0 and world == 1:
+        extra["host_ms_per_call_python_launch"] = ms_stream
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": workload_desc(w), "B": B, "d": S.d, "E": S.E, "k": S.k, "d_ff": S.F,
+                   "rule": w["rule"], "n_active": n_active, "bytes_per_call": total_bytes,
+                   "parallelism": f"replicas x{world}",
+                   "l2": f"inputs larger than L2: {ROTATE} rotating weight copies of "
+                         f"{3 * S.E * S.d * S.F * 2 / 1e9:.2f} GB",
+                   "launch": "CUDA graph of 4 layer calls, PDL between the 3 kernels of a call"},
+        "us_per_call": ms_step * 1e3,
+        "frac_of_nominal_8tbs": (total_bytes / (ms_step * 1e-3) / 1e9) / NOMINAL_HBM_GBS,
+        "frac_of_measured_hbm": (total_bytes / (ms_step * 1e-3) / 1e9) / hbm_peak,
+        "stream_launch_us_per_call": ms_stream * 1e3,
+        "roofline": roofline,
+        "e2e": e2e,
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, S, L, x_np)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del g_all, g_one, g_ffn
+    torch.cuda.synchronize(dev)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="q30b_b16_oea4")
+    ap.add_argument("--no-extra", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w, rank)
+        return 0
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, w, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

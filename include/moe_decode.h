@@ -1,0 +1,183 @@
+/*
+ * moe_decode.h -- C ABI of libmoe_decode.so: the decode-time Mixture-of-
+ * Experts layer with batch-aware expert re-routing, for one NVIDIA B200
+ * (sm_100a).
+ *
+ * The layer (one call per MoE layer per decode step):
+ *   1. router: logits = x Wg^T + bias, softmax, top-k
+ *      ("Router Caching and Optimization", section "Analyzing Router
+ *      Inference Cost", steps 1-3);
+ *   2. batch-aware re-selection, which shrinks the set of experts the batch
+ *      activates: OEA piggybacking ("Opportunistic Expert Activation:
+ *      Batch-Aware Expert Routing for Faster Decode Without Retraining",
+ *      abstract) or XShare greedy selection under an expert budget ("XShare:
+ *      Collaborative in-Batch Expert Sharing for Faster MoE Inference",
+ *      abstract);
+ *   3. the SwiGLU FFN of every activated expert over its tokens, combined
+ *      with the renormalised gate weights; each activated expert's weights
+ *      are read from HBM once per call ("Lynx: Enabling Efficient MoE
+ *      Inference through Dynamic Batch-Aware Expert Selection", section 1:
+ *      decode latency follows the number of distinct activated experts).
+ *
+ * Conventions for every entry point
+ *  - Pointers named "device" are CUDA device pointers of the current
+ *    device; the caller allocates and frees every buffer.  The library never
+ *    allocates or frees device memory and keeps no device state between
+ *    calls other than what lives in the caller's workspace.
+ *  - All layouts are dense row-major (C order).  bf16 values are passed as
+ *    their uint16_t bit patterns.
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and runs asynchronously; no entry point synchronises except
+ *    moe_check_error.
+ *  - Arguments are validated on the host before anything is enqueued.  On
+ *    any error nothing is launched and the status says why.
+ *  - Device buffers must be 16-byte aligned, the workspace 256-byte aligned
+ *    (MOE_ERR_MISALIGNED otherwise).  The workspace must be zero-filled
+ *    once before its first use (e.g. cudaMemset); the library keeps it
+ *    consistent afterwards.  Calls that share one workspace must not
+ *    overlap in time on the device (same stream, or ordered by events).
+ *  - Limits: 1 <= B <= 256, 1 <= k <= 16, k <= E <= 256, d % 64 == 0,
+ *    64 <= d <= 16384, d_ff % 64 == 0, 64 <= d_ff <= 8192.  moe_route reads
+ *    B, d, E, k of the dims (d_ff is ignored); moe_reselect reads B, E, k.
+ *  - Inputs must be finite; NaN or Inf inputs give unspecified results.
+ *  - Nothing is thrown across the ABI.
+ */
+#ifndef MOE_DECODE_H
+#define MOE_DECODE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,  /* null pointer, bad dimension or rule parameter */
+    MOE_ERR_MISALIGNED = 2,   /* a buffer is not 16-byte aligned */
+    MOE_ERR_WORKSPACE = 3,    /* workspace missing or smaller than moe_workspace_bytes() */
+    MOE_ERR_UNSUPPORTED = 4,  /* valid but outside the implemented limits, or no sm_100 device */
+    MOE_ERR_CUDA = 5,         /* a CUDA runtime/driver call or a launch failed */
+    MOE_ERR_INTERNAL = 6      /* a kernel recorded an internal error (see moe_check_error) */
+} moe_status_t;
+
+/* Re-selection rules. */
+typedef enum {
+    MOE_RESELECT_NONE = 0,    /* standard top-k routing */
+    MOE_RESELECT_OEA = 1,     /* keep top-k0, fill from the batch union of kept sets */
+    MOE_RESELECT_XSHARE = 2   /* budgeted greedy batch selection, then top-k within it */
+} moe_reselect_mode_t;
+
+/* Layer dimensions: B tokens, hidden size d, E experts, top-k k,
+ * expert intermediate size d_ff. */
+typedef struct {
+    int32_t B, d, E, k, d_ff;
+} moe_dims_t;
+
+/* Re-selection rule: mode (moe_reselect_mode_t); k0 (OEA: 1 <= k0 <= k);
+ * budget (XShare: k <= budget <= E).  Unused fields are ignored. */
+typedef struct {
+    int32_t mode, k0, budget;
+} moe_reselect_t;
+
+/* Per-expert token lists (all device pointers, int32 / fp32):
+ *   n_active[1]   number of activated experts;
+ *   active[E]     activated expert ids, ascending; -1 past n_active;
+ *   offsets[E+1]  offsets[i] = first entry of active[i]; offsets[n_active]
+ *                 and every later entry = total (token, expert) pairs;
+ *   tok[B*k]      token of each entry; entries of one expert in ascending
+ *                 token order; -1 past the total;
+ *   w[B*k]        renormalised gate weight of each entry; 0 past the total. */
+typedef struct {
+    int32_t *n_active;
+    int32_t *active;
+    int32_t *offsets;
+    int32_t *tok;
+    float *w;
+} moe_lists_t;
+
+/* Bytes of device workspace every entry point below may use for `dims`
+ * (one size serves all of them).  Returns 0 if dims are invalid. */
+size_t moe_workspace_bytes(moe_dims_t dims);
+
+/* Router ("Router Caching and Optimization", "Analyzing Router Inference
+ * Cost", steps 1-3, computed in one pass per token as its "Kernel Fusion"
+ * section suggests).
+ *   x[B][d] fp32, Wg[E][d] fp32, bias[E] fp32 (device; bias may be NULL);
+ *   outputs (device): logits[B][E], probs[B][E] fp32, topk_idx[B][k] int32,
+ *   topk_w[B][k] fp32.
+ * logits[b][e] = dot(x[b], Wg[e]) + bias[e] in fp32 with a fixed summation
+ * order; probs = softmax(logits) with the library's own exp; topk_idx = the
+ * k largest logits, descending, equal logits to the lower expert index;
+ * topk_w = probs of those experts renormalised to sum 1.  Bit-reproducible
+ * (identical results for identical inputs on every call). */
+moe_status_t moe_route(const float *x, const float *Wg, const float *bias,
+                       moe_dims_t dims, float *logits, float *probs,
+                       int32_t *topk_idx, float *topk_w, void *stream);
+
+/* Batch-aware re-selection + per-expert token lists.
+ *   logits[B][E], probs[B][E] fp32 (device; as produced by moe_route);
+ *   outputs (device): sel_idx[B][k] int32 (chosen experts in rank order,
+ *   -1 in unused slots), sel_w[B][k] fp32 (gate weights renormalised over
+ *   the chosen set, 0 in unused slots), and `lists`.
+ * Rules (rank order = logit descending, ties to the lower index):
+ *   NONE   : the token's top-k.
+ *   OEA    : the token keeps its first k0 experts; the union of all kept
+ *            sets is formed; each token then fills up to k slots with the
+ *            highest-ranked experts of that union it does not yet hold
+ *            (fewer when the union is short).  Activated set = the union.
+ *   XSHARE : score s_e = sum over tokens whose top-k holds e of p[b][e]
+ *            (fp32, tokens ascending); the min(budget, |union of top-k|)
+ *            experts of that union with the largest scores (ties to the
+ *            lower index) form the batch set -- the greedy, exact for this
+ *            modular objective; each token takes its k highest-ranked
+ *            experts inside the set.
+ * Results are bit-exact and deterministic.  Needs no workspace. */
+moe_status_t moe_reselect(const float *logits, const float *probs,
+                          moe_dims_t dims, moe_reselect_t rule,
+                          int32_t *sel_idx, float *sel_w, moe_lists_t lists,
+                          void *stream);
+
+/* Grouped SwiGLU expert FFN with the weighted combine.
+ *   x[B][d] fp32; Wgate[E][d_ff][d], Wup[E][d_ff][d], Wdown[E][d][d_ff]
+ *   bf16 bits (device; nn.Linear out x in layout); lists as written by
+ *   moe_reselect (device, read only);
+ *   y[B][d] fp32 (device, overwritten):
+ *   y[t] = sum over (t, e, w) entries of w * Wdown[e] (silu(Wgate[e] x_t)
+ *          * (Wup[e] x_t)).
+ * Only the experts in `lists` are read, each once per call.  x and the
+ * SwiGLU activations are rounded to bf16 for the tensor cores; sums are
+ * fp32; the combine uses fp32 atomics (summation order not fixed).
+ * ws: device workspace of at least moe_workspace_bytes(dims) bytes. */
+moe_status_t moe_expert_ffn(const float *x, const uint16_t *Wgate,
+                            const uint16_t *Wup, const uint16_t *Wdown,
+                            moe_dims_t dims, moe_lists_t lists, float *y,
+                            void *ws, size_t ws_bytes, void *stream);
+
+/* The whole layer: moe_route -> moe_reselect -> moe_expert_ffn, chained on
+ * the device with no host round trip (the activated-expert count never
+ * leaves the GPU).  Arguments as above; y[B][d] is overwritten.
+ * sel_idx[B][k], sel_w[B][k] and n_active[1] are optional device outputs
+ * (NULL = not returned).  ws: device workspace of at least
+ * moe_workspace_bytes(dims) bytes. */
+moe_status_t moe_layer_decode(const float *x, const float *Wg, const float *bias,
+                              const uint16_t *Wgate, const uint16_t *Wup,
+                              const uint16_t *Wdown, moe_dims_t dims,
+                              moe_reselect_t rule, float *y, int32_t *sel_idx,
+                              float *sel_w, int32_t *n_active, void *ws,
+                              size_t ws_bytes, void *stream);
+
+/* Synchronises `stream`, then reads and clears the error word that kernels
+ * of earlier calls using this workspace may have set (a bounded wait that
+ * ran out).  Returns MOE_OK, MOE_ERR_INTERNAL or MOE_ERR_CUDA. */
+moe_status_t moe_check_error(void *ws, size_t ws_bytes, void *stream);
+
+/* Static description of a status code (never NULL). */
+const char *moe_status_string(moe_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_DECODE_H */

@@ -1,0 +1,136 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads,
+exports every function include/moe_decode.h declares, sizes workspaces,
+and rejects bad arguments with the documented status before touching CUDA.
+
+Every call below with fake addresses carries at least one argument that the
+host validation rejects, so none of them can reach a kernel launch."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import aware_expert_routing_moe_b200 as moe
+from aware_expert_routing_moe_b200 import Dims, Lists, Rule
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+OK, INVALID, MISALIGNED, WORKSPACE, UNSUPPORTED, CUDA, INTERNAL = range(7)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from aware_expert_routing_moe_b200 import build
+    build.build()
+    return moe.load_library()
+
+
+def _declared_functions():
+    with open(os.path.join(ROOT, "include", "moe_decode.h")) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_symbols():
+    assert _declared_functions() == sorted(moe.ABI_SYMBOLS)
+
+
+def test_library_exports_every_declared_function(lib):
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    seen = set()
+    for s in range(7):
+        txt = moe.moe_status_string(s)
+        assert txt and txt not in seen
+        seen.add(txt)
+    assert moe.moe_status_string(99) == "unknown status"
+
+
+def test_workspace_bytes(lib):
+    q30 = moe.moe_workspace_bytes(16, 2048, 128, 8, 768)
+    assert q30 > 0 and q30 % 256 == 0
+    # H scratch dominates: B*k*d_ff bf16
+    assert q30 >= 16 * 8 * 768 * 2
+    assert moe.moe_workspace_bytes(64, 2048, 128, 8, 768) > q30
+    assert moe.moe_workspace_bytes(16, 4096, 128, 8, 1536) > q30
+    for bad in [(0, 2048, 128, 8, 768), (257, 2048, 128, 8, 768), (16, 2048, 128, 0, 768),
+                (16, 2048, 128, 17, 768), (16, 2048, 7, 8, 768), (16, 2048, 257, 8, 768),
+                (16, 2000, 128, 8, 768), (16, 2048, 128, 8, 700), (16, 32, 128, 8, 768),
+                (16, 2048, 128, 8, 32)]:
+        assert moe.moe_workspace_bytes(*bad) == 0, bad
+
+
+A = 0x10000  # fake, 256-byte aligned address (never dereferenced)
+
+
+def _layer_call(lib, dims=Dims(16, 2048, 128, 8, 768), rule=Rule(1, 4, 0), x=A, Wg=A, bias=A, Wgate=A,
+                Wup=A, Wdown=A, y=A, sel=None, selw=None, nact=None, ws=A, ws_bytes=None):
+    if ws_bytes is None:
+        ws_bytes = lib.moe_workspace_bytes(dims) if lib.moe_workspace_bytes(dims) else 1 << 30
+    return lib.moe_layer_decode(x, Wg, bias, Wgate, Wup, Wdown, dims, rule, y, sel, selw, nact, ws,
+                                ws_bytes, None)
+
+
+def test_layer_decode_rejects_bad_arguments(lib):
+    small = lib.moe_workspace_bytes(Dims(16, 2048, 128, 8, 768)) - 256
+    assert _layer_call(lib, dims=Dims(0, 2048, 128, 8, 768)) == INVALID
+    assert _layer_call(lib, dims=Dims(16, 2048, 128, 8, 700)) == INVALID
+    assert _layer_call(lib, rule=Rule(1, 0, 0)) == INVALID          # k0 < 1
+    assert _layer_call(lib, rule=Rule(1, 9, 0)) == INVALID          # k0 > k
+    assert _layer_call(lib, rule=Rule(2, 0, 7)) == INVALID          # budget < k
+    assert _layer_call(lib, rule=Rule(2, 0, 129)) == INVALID        # budget > E
+    assert _layer_call(lib, rule=Rule(3, 0, 0)) == INVALID          # unknown rule
+    assert _layer_call(lib, x=None) == INVALID
+    assert _layer_call(lib, Wdown=None) == INVALID
+    assert _layer_call(lib, y=None) == INVALID
+    assert _layer_call(lib, x=A + 4) == MISALIGNED
+    assert _layer_call(lib, Wup=A + 8) == MISALIGNED
+    assert _layer_call(lib, bias=A + 2) == MISALIGNED
+    assert _layer_call(lib, sel=A + 4) == MISALIGNED
+    assert _layer_call(lib, ws=None) == WORKSPACE
+    assert _layer_call(lib, ws_bytes=small) == WORKSPACE
+    assert _layer_call(lib, ws=A + 16) == MISALIGNED                # workspace wants 256 B
+
+
+def test_route_and_reselect_reject_bad_arguments(lib):
+    d = Dims(16, 2048, 128, 8, 0)
+    assert lib.moe_route(None, A, None, d, A, A, A, A, None) == INVALID
+    assert lib.moe_route(A, A, None, Dims(16, 2000, 128, 8, 0), A, A, A, A, None) == INVALID
+    assert lib.moe_route(A, A, None, Dims(16, 2048, 4, 8, 0), A, A, A, A, None) == INVALID
+    assert lib.moe_route(A, A + 4, None, d, A, A, A, A, None) == MISALIGNED
+    lists = Lists(A, A, A, A, A)
+    assert lib.moe_reselect(A, A, d, Rule(1, 9, 0), A, A, lists, None) == INVALID
+    assert lib.moe_reselect(A, A, d, Rule(0, 0, 0), None, A, lists, None) == INVALID
+    assert lib.moe_reselect(A, A, d, Rule(0, 0, 0), A, A, Lists(A, None, A, A, A), None) == INVALID
+    assert lib.moe_reselect(A, A, d, Rule(0, 0, 0), A, A, Lists(A, A, A + 4, A, A), None) == MISALIGNED
+    assert lib.moe_reselect(A, A, Dims(300, 0, 128, 8, 0), Rule(0, 0, 0), A, A, lists, None) == INVALID
+
+
+def test_expert_ffn_rejects_bad_arguments(lib):
+    d = Dims(16, 2048, 128, 8, 768)
+    lists = Lists(A, A, A, A, A)
+    n = lib.moe_workspace_bytes(d)
+    assert lib.moe_expert_ffn(A, A, A, A, Dims(16, 2048, 128, 8, 0), lists, A, A, n, None) == INVALID
+    assert lib.moe_expert_ffn(A, None, A, A, d, lists, A, A, n, None) == INVALID
+    assert lib.moe_expert_ffn(A, A, A, A, d, Lists(None, A, A, A, A), A, A, n, None) == INVALID
+    assert lib.moe_expert_ffn(A, A, A, A + 2, d, lists, A, A, n, None) == MISALIGNED
+    assert lib.moe_expert_ffn(A, A, A, A, d, lists, A, A, n - 1, None) == WORKSPACE
+    assert lib.moe_check_error(None, 0, None) == WORKSPACE
+    assert lib.moe_check_error(A + 16, 4096, None) == MISALIGNED
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_valid_call_without_a_device_reports_cuda_error(lib):
+    # all arguments valid: validation passes, the device query fails cleanly
+    assert _layer_call(lib) == CUDA
+    assert lib.moe_route(A, A, None, Dims(16, 2048, 128, 8, 0), A, A, A, A, None) == CUDA
+
+
+def test_binding_raises_on_error(lib):
+    with pytest.raises(moe.MoeError) as ei:
+        moe._check(MISALIGNED, "x")
+    assert ei.value.status == MISALIGNED
