@@ -90,6 +90,24 @@ def algorithmic_bytes(S, B, n_active):
     return experts + router + io, experts + io
 
 
+# ------------------------------------------------------ multi-rank host --
+def max_over_ranks(v: float, world: int, device=None) -> float:
+    """Max of a per-rank timing over all ranks (every rank must call it)."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    tv = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(tv, op=dist.ReduceOp.MAX)
+    return float(tv.item())
+
+
+def aggregate_gbs(bytes_per_rank_step: int, world: int, ms_per_step: float) -> float:
+    """Whole-job GB/s: every rank moves the same bytes per step; the step
+    time is the max over ranks."""
+    return world * bytes_per_rank_step / (ms_per_step * 1e-3) / 1e9
+
+
 # ------------------------------------------------------------- clocks --
 class ClockSampler:
     """Polls SM clock and clock-event reasons with NVML while running."""
@@ -265,13 +283,6 @@ def run_ours(args, w, rank, world, local_rank):
         if world > 1:
             dist.barrier(device_ids=[local_rank])
 
-    def max_over_ranks(v):
-        if world == 1:
-            return v
-        tv = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(tv, op=dist.ReduceOp.MAX)
-        return float(tv.item())
-
     def timed(fn, nsteps, sampler=None):
         barrier()
         torch.cuda.synchronize(dev)
@@ -283,7 +294,7 @@ def run_ours(args, w, rank, world, local_rank):
         e1.synchronize()
         torch.cuda.synchronize(dev)
         barrier()
-        return max_over_ranks(e0.elapsed_time(e1))  # ms, all steps
+        return max_over_ranks(e0.elapsed_time(e1), world, dev)  # ms, all steps
 
     # ---- main timed region: K graph-replayed layer calls
     with torch.cuda.stream(s):
@@ -293,7 +304,7 @@ def run_ours(args, w, rank, world, local_rank):
         ms_total = timed(replay, args.steps)
     clocks = sampler.summary()
     ms_step = ms_total / args.steps
-    value = world * total_bytes / (ms_step * 1e-3) / 1e9
+    value = aggregate_gbs(total_bytes, world, ms_step)
 
     # ---- the same calls launched one by one from Python (launch overhead)
     def stream_calls(nsteps):
@@ -342,7 +353,7 @@ def run_ours(args, w, rank, world, local_rank):
     with torch.cuda.stream(s):
         e2e_calls(args.warmup)
     ms_e2e = timed(e2e_calls, args.steps) / args.steps
-    e2e = {"value": world * total_bytes / (ms_e2e * 1e-3) / 1e9, "unit": UNIT,
+    e2e = {"value": aggregate_gbs(total_bytes, world, ms_e2e), "unit": UNIT,
            "h2d_bytes_per_step": B * S.d * 4, "d2h_bytes_per_step": B * S.d * 4,
            "ms_per_step": ms_e2e}
     if moe.moe_check_error(ws, s) != 0:

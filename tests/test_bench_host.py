@@ -1,0 +1,67 @@
+"""Host-side logic of bench.py that needs no GPU: the N > 1 path's
+max-over-ranks timing and whole-job aggregation (world size 2 over gloo on
+CPU), the workload table and the algorithmic byte count."""
+import os
+import socket
+
+import pytest
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+import moe_synth as ms
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        t = bench.max_over_ranks(1.5 + rank, world, device="cpu")  # rank 1 is slower
+        out[rank] = t
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo_world2():
+    world = 2
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    out = ctx.Manager().dict()
+    mp.start_processes(_rank_main, args=(world, port, out), nprocs=world, join=True, start_method="spawn")
+    assert dict(out) == {0: 2.5, 1: 2.5}
+
+
+def test_aggregate_is_whole_job():
+    one = bench.aggregate_gbs(1_000_000, 1, 1.0)
+    assert one == pytest.approx(1.0)            # 1 MB per ms = 1 GB/s
+    assert bench.aggregate_gbs(1_000_000, 8, 1.0) == pytest.approx(8.0)
+    assert bench.max_over_ranks(3.0, 1) == 3.0
+
+
+def test_algorithmic_bytes_q30b():
+    S = ms.SHAPES["q30b"]
+    total, ffn = bench.algorithmic_bytes(S, 16, 15)
+    per_expert = 3 * 2048 * 768 * 2
+    assert per_expert == 9_437_184
+    assert ffn == 15 * per_expert + 2 * 16 * 2048 * 4
+    assert total == ffn + 128 * 2048 * 4 + 128 * 4
+
+
+def test_workloads_describe_real_shapes():
+    for name, w in bench.WORKLOADS.items():
+        desc = bench.workload_desc(w)
+        S = ms.SHAPES[w["shape"]]
+        assert f"d={S.d}" in desc and f"B={w['B']}" in desc, name
+
+
+def test_reference_arm_other_ranks_do_nothing(capsys):
+    class A:
+        steps, warmup, gpus = 3, 3, 2
+    bench.run_reference(A, bench.WORKLOADS["q30b_b16_oea4"], rank=1)
+    assert capsys.readouterr().out == ""
