@@ -21,14 +21,16 @@ __all__ = [
     "MOE_RESELECT_NONE", "MOE_RESELECT_OEA", "MOE_RESELECT_XSHARE", "MoeError",
     "Dims", "Rule", "Lists", "load_library", "library_path", "moe_workspace_bytes",
     "moe_status_string", "moe_route", "moe_reselect", "moe_expert_ffn", "moe_layer_decode",
-    "moe_check_error", "new_workspace", "alloc_lists", "ABI_SYMBOLS",
+    "moe_check_error", "moe_expert_ffn_noalloc", "new_workspace", "alloc_lists", "ABI_SYMBOLS",
+    "NOALLOC_SCRATCH_BYTES",
 ]
 
 MOE_RESELECT_NONE, MOE_RESELECT_OEA, MOE_RESELECT_XSHARE = 0, 1, 2
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_MISALIGNED", 3: "MOE_ERR_WORKSPACE",
           4: "MOE_ERR_UNSUPPORTED", 5: "MOE_ERR_CUDA", 6: "MOE_ERR_INTERNAL"}
 ABI_SYMBOLS = ("moe_workspace_bytes", "moe_route", "moe_reselect", "moe_expert_ffn",
-               "moe_layer_decode", "moe_check_error", "moe_status_string")
+               "moe_layer_decode", "moe_expert_ffn_noalloc", "moe_check_error", "moe_status_string")
+NOALLOC_SCRATCH_BYTES = 8 * 1024 * 1024
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libmoe_decode.so")
@@ -79,6 +81,8 @@ def load_library() -> ctypes.CDLL:
         lib.moe_expert_ffn.argtypes = [P, P, P, P, Dims, Lists, P, P, S, P]
         lib.moe_layer_decode.restype = ctypes.c_int
         lib.moe_layer_decode.argtypes = [P, P, P, P, P, P, Dims, Rule, P, P, P, P, P, S, P]
+        lib.moe_expert_ffn_noalloc.restype = ctypes.c_int
+        lib.moe_expert_ffn_noalloc.argtypes = [P, P, P, P, Dims, Lists, P, P]
         lib.moe_check_error.restype = ctypes.c_int
         lib.moe_check_error.argtypes = [P, S, P]
         _lib = lib
@@ -199,6 +203,20 @@ def moe_layer_decode(x, Wg, bias, Wgate, Wup, Wdown, k: int, mode: int, k0: int 
         Rule(mode, k0, budget), _ptr(y), _ptr(sel_idx), _ptr(sel_w), _ptr(n_active), _ptr(ws),
         ws.numel() * ws.element_size(), _stream(stream))
     _check(st, "moe_layer_decode")
+    return y
+
+
+def moe_expert_ffn_noalloc(x, Wgate, Wup, Wdown, lists: dict, k: int, y=None, stream=None):
+    """moe_expert_ffn without a workspace, for callers that cannot allocate
+    device memory: the library's static 8 MiB device scratch is used instead
+    (shared by all calls on a device; overlapping calls race).  -> y[B][d]."""
+    B, d = x.shape
+    E, F, _ = Wgate.shape
+    if y is None:
+        y = torch.empty(B, d, dtype=torch.float32, device=x.device)
+    st = load_library().moe_expert_ffn_noalloc(_ptr(x), _ptr(Wgate), _ptr(Wup), _ptr(Wdown),
+                                               Dims(B, d, E, k, F), _lists(lists), _ptr(y), _stream(stream))
+    _check(st, "moe_expert_ffn_noalloc")
     return y
 
 

@@ -116,15 +116,6 @@ bool encode_bf16_2d(CUtensorMap *map, const void *ptr, uint64_t rows, uint64_t c
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool encode_expert_maps(ExpertMaps *m, const moe_dims_t &d, const uint16_t *Wgate, const uint16_t *Wup,
-                        const uint16_t *Wdown, const uint16_t *h) {
-    std::memset(m, 0, sizeof(*m));
-    const uint64_t E = d.E, F = d.d_ff, D = d.d;
-    return encode_bf16_2d(&m->gate, Wgate, E * F, D, 16) && encode_bf16_2d(&m->up, Wup, E * F, D, 16) &&
-           encode_bf16_2d(&m->down, Wdown, E * D, F, 64) &&
-           encode_bf16_2d(&m->h, h, static_cast<uint64_t>(d.B) * d.k, F, expert_ffn_h_rows());
-}
-
 template <typename T>
 T *seg(void *ws, size_t off) {
     return reinterpret_cast<T *>(static_cast<unsigned char *>(ws) + off);
@@ -141,6 +132,15 @@ moe_lists_t ws_lists(void *ws, const WsLayout &L) {
 }
 
 }  // namespace
+
+bool encode_expert_maps(ExpertMaps *m, const moe_dims_t &d, const uint16_t *Wgate, const uint16_t *Wup,
+                        const uint16_t *Wdown, const uint16_t *h) {
+    std::memset(m, 0, sizeof(*m));
+    const uint64_t E = d.E, F = d.d_ff, D = d.d;
+    return encode_bf16_2d(&m->gate, Wgate, E * F, D, 16) && encode_bf16_2d(&m->up, Wup, E * F, D, 16) &&
+           encode_bf16_2d(&m->down, Wdown, E * D, F, 64) &&
+           encode_bf16_2d(&m->h, h, static_cast<uint64_t>(d.B) * d.k, F, expert_ffn_h_rows());
+}
 
 WsLayout ws_layout(const moe_dims_t &d) {
     WsLayout L;

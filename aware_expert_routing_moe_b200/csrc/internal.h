@@ -65,4 +65,8 @@ cudaError_t launch_expert_ffn(const ExpertMaps &maps, const uint16_t *xb,
                               uint16_t *h, Counters *ctr, bool pdl, cudaStream_t s);
 int expert_ffn_h_rows();   // row count of one H tile box (tokens per tile)
 
+// TMA descriptors of the expert kernel (weights and the H scratch at `h`).
+bool encode_expert_maps(ExpertMaps *m, const moe_dims_t &d, const uint16_t *Wgate, const uint16_t *Wup,
+                        const uint16_t *Wdown, const uint16_t *h);
+
 }  // namespace moe

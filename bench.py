@@ -389,6 +389,28 @@ def run_ours(args, w, rank, world, local_rank):
     torch.cuda.synchronize(dev)
 
 
+def run_profile_case(args, w):
+    """A small case for ncu captures: one weight copy (about 1.2 GB for the
+    Qwen3-30B shape, so the activated experts still exceed L2), `warmup`
+    layer calls, then `steps` more, launched from the stream, no timing."""
+    import torch
+    import aware_expert_routing_moe_b200 as moe
+    S = ms.SHAPES[w["shape"]]
+    B = w["B"]
+    L = ms.make_weights(S, 0)
+    t = lambda a: torch.from_numpy(a).cuda()
+    x = t(ms.make_tokens(S, B, 0, kind=w.get("kind", "normal")))
+    Wg, bias = t(L["Wg"]), t(L["bias"])
+    g, u, dn = (t(L[n].view(np.int16)) for n in ("Wgate", "Wup", "Wdown"))
+    ws = moe.new_workspace(B, S.d, S.E, S.k, S.F)
+    for _ in range(args.warmup + args.steps):
+        moe.moe_layer_decode(x, Wg, bias, g, u, dn, S.k, w["mode"], w["k0"], w["budget"], ws=ws)
+    torch.cuda.synchronize()
+    status = moe.moe_check_error(ws)
+    print(f"profile case {args.workload}: {args.warmup}+{args.steps} layer calls, status {status}")
+    return 0 if status == 0 else 1
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -398,6 +420,8 @@ def main(argv=None):
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="q30b_b16_oea4")
     ap.add_argument("--no-extra", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", action="store_true",
+                    help="small case for ncu: one weight copy, warmup + steps layer calls, no timing")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -405,6 +429,8 @@ def main(argv=None):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     w = WORKLOADS[args.workload]
+    if args.profile:
+        return run_profile_case(args, w)
     if args.impl == "reference":
         run_reference(args, w, rank)
         return 0

@@ -23,7 +23,8 @@
  *  - Pointers named "device" are CUDA device pointers of the current
  *    device; the caller allocates and frees every buffer.  The library never
  *    allocates or frees device memory and keeps no device state between
- *    calls other than what lives in the caller's workspace.
+ *    calls other than what lives in the caller's workspace (and, for
+ *    moe_expert_ffn_noalloc, its static scratch array).
  *  - All layouts are dense row-major (C order).  bf16 values are passed as
  *    their uint16_t bit patterns.
  *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
@@ -167,6 +168,44 @@ moe_status_t moe_layer_decode(const float *x, const float *Wg, const float *bias
                               moe_reselect_t rule, float *y, int32_t *sel_idx,
                               float *sel_w, int32_t *n_active, void *ws,
                               size_t ws_bytes, void *stream);
+
+/* moe_expert_ffn for callers that cannot allocate device memory.
+ * (The source pages have no counterpart to this entry point; it is a
+ * deployment convenience of this library.)
+ *
+ * Some callers have no workspace to pass and may not call cudaMalloc:
+ * plugins whose host framework hands them only inputs and outputs, code
+ * running where all device memory was reserved up front by the host
+ * application, and latency-critical paths that cannot afford the device
+ * synchronisation cudaMalloc/cudaFree may cause.  This entry point takes the
+ * same arguments as moe_expert_ffn minus the workspace, and allocates
+ * nothing: its scratch (the expert kernel's counters, x in bf16 and the
+ * SwiGLU activations) lives in a file-scope static device array of
+ * MOE_NOALLOC_SCRATCH_BYTES (8 MiB), which every GPU that loads the library
+ * holds until the process exits.  It calls no cudaMalloc, cudaFree or other
+ * allocating routine.
+ *
+ *  - Size limit: 1280 + B*d*2 + B*k*d_ff*2 bytes (the last two terms each
+ *    rounded up to a multiple of 256) must fit in MOE_NOALLOC_SCRATCH_BYTES;
+ *    larger dims return MOE_ERR_UNSUPPORTED before anything is enqueued.
+ *    The Qwen3-30B-A3B-shaped layer fits up to B = 256, the Qwen3-235B-
+ *    A22B-shaped one up to B = 255.
+ *  - Set-up: the first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current) and caches it; make
+ *    that first call before any stream capture begins.
+ *  - Sharing: all calls on a device use the same array, which keeps the
+ *    last call's contents; each call clears the counters that must start at
+ *    zero.  Calls that overlap in time on the GPU (for example on two
+ *    streams with no ordering between them) race on the array and give
+ *    wrong results: order them on one stream or with events.
+ *  - A bounded wait that expires inside the kernels is recorded in the
+ *    array but not reported; use moe_expert_ffn + moe_check_error to
+ *    diagnose such a failure. */
+#define MOE_NOALLOC_SCRATCH_BYTES (8u * 1024u * 1024u)
+moe_status_t moe_expert_ffn_noalloc(const float *x, const uint16_t *Wgate,
+                                    const uint16_t *Wup, const uint16_t *Wdown,
+                                    moe_dims_t dims, moe_lists_t lists, float *y,
+                                    void *stream);
 
 /* Synchronises `stream`, then reads and clears the error word that kernels
  * of earlier calls using this workspace may have set (a bounded wait that
