@@ -102,17 +102,35 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 2-D bf16 matrix [rows][cols] (row-major), boxes of box_rows x 64 columns
-// (128 bytes, the 128B swizzle span).  Out-of-range elements read as zero.
-bool encode_bf16_2d(CUtensorMap *map, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+// bf16 matrix [rows][cols] (row-major, cols % 64 == 0) seen as a 3-D tensor
+// (64-element column chunk, row, chunk index).  One box of box_rows rows and
+// box_chunks chunks lands in shared memory as box_chunks consecutive tiles of
+// [box_rows][64], each with the 128-byte swizzle.  Elements past the end of
+// the matrix read as zero.
+bool encode_bf16_chunked(CUtensorMap *map, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box_rows,
+                         uint32_t box_chunks) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t gdim[3] = {64, rows, cols / 64};
+    cuuint64_t gstride[2] = {cols * 2, 128};
+    cuuint32_t box[3] = {64, box_rows, box_chunks};
+    cuuint32_t estride[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), gdim, gstride, box, estride,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// bf16 matrix [rows][cols] for tile::gather4 loads: boxes of one row and
+// box_cols columns, no swizzle.
+bool encode_bf16_rows(CUtensorMap *map, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box_cols) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t gdim[2] = {cols, rows};
     cuuint64_t gstride[1] = {cols * 2};
-    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t box[2] = {box_cols, 1};
     cuuint32_t estride[2] = {1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), gdim, gstride, box, estride,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -134,12 +152,15 @@ moe_lists_t ws_lists(void *ws, const WsLayout &L) {
 }  // namespace
 
 bool encode_expert_maps(ExpertMaps *m, const moe_dims_t &d, const uint16_t *Wgate, const uint16_t *Wup,
-                        const uint16_t *Wdown, const uint16_t *h) {
+                        const uint16_t *Wdown, const uint16_t *h, const uint16_t *xb) {
     std::memset(m, 0, sizeof(*m));
     const uint64_t E = d.E, F = d.d_ff, D = d.d;
-    return encode_bf16_2d(&m->gate, Wgate, E * F, D, 16) && encode_bf16_2d(&m->up, Wup, E * F, D, 16) &&
-           encode_bf16_2d(&m->down, Wdown, E * D, F, 64) &&
-           encode_bf16_2d(&m->h, h, static_cast<uint64_t>(d.B) * d.k, F, expert_ffn_h_rows());
+    const uint32_t gu_chunks = expert_ffn_gu_chunks(d.d), d_chunks = expert_ffn_d_chunks(d.d_ff);
+    return encode_bf16_chunked(&m->gate, Wgate, E * F, D, expert_ffn_gu_rows(), gu_chunks) &&
+           encode_bf16_chunked(&m->up, Wup, E * F, D, expert_ffn_gu_rows(), gu_chunks) &&
+           encode_bf16_chunked(&m->down, Wdown, E * D, F, expert_ffn_d_rows(), d_chunks) &&
+           encode_bf16_chunked(&m->h, h, static_cast<uint64_t>(d.B) * d.k, F, expert_ffn_h_rows(), d_chunks) &&
+           encode_bf16_rows(&m->x, xb, static_cast<uint64_t>(d.B), D, gu_chunks * 64);
 }
 
 WsLayout ws_layout(const moe_dims_t &d) {
@@ -228,7 +249,8 @@ moe_status_t moe_expert_ffn(const float *x, const uint16_t *Wgate, const uint16_
     if (st != MOE_OK) return st;
     const WsLayout L = ws_layout(dims);
     ExpertMaps maps;
-    if (!encode_expert_maps(&maps, dims, Wgate, Wup, Wdown, seg<uint16_t>(ws, L.h))) return MOE_ERR_CUDA;
+    if (!encode_expert_maps(&maps, dims, Wgate, Wup, Wdown, seg<uint16_t>(ws, L.h), seg<uint16_t>(ws, L.xb)))
+        return MOE_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     Counters *ctr = seg<Counters>(ws, L.counters);
     uint16_t *xb = seg<uint16_t>(ws, L.xb);
@@ -252,7 +274,8 @@ moe_status_t moe_layer_decode(const float *x, const float *Wg, const float *bias
     if (st != MOE_OK) return st;
     const WsLayout L = ws_layout(dims);
     ExpertMaps maps;
-    if (!encode_expert_maps(&maps, dims, Wgate, Wup, Wdown, seg<uint16_t>(ws, L.h))) return MOE_ERR_CUDA;
+    if (!encode_expert_maps(&maps, dims, Wgate, Wup, Wdown, seg<uint16_t>(ws, L.h), seg<uint16_t>(ws, L.xb)))
+        return MOE_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     Counters *ctr = seg<Counters>(ws, L.counters);
     uint16_t *xb = seg<uint16_t>(ws, L.xb);

@@ -31,22 +31,24 @@
 namespace moe {
 namespace {
 
-constexpr int NCW = 4;                    // consumer warps
-constexpr int NTHREADS = (NCW + 1) * 32;  // + one producer warp
+constexpr int NCW = 8;                    // consumer warps
+constexpr int NTHREADS = (NCW + 2) * 32;  // + one producer warp + one signal warp
+constexpr int SIG_SLOTS = 4;              // gate/up completions queued for the signal warp
 constexpr int TN = 32;                    // tokens per tile
 constexpr int GU_ROWS = 16;               // rows of Wgate and of Wup per GU unit
-constexpr int GU_KC = 256;                // d elements per GU stage
+constexpr int GU_CHUNKS = 4;              // 64-column chunks of d per GU stage (at most)
 constexpr int D_ROWS = 64;                // rows of Wdown per D unit
-constexpr int D_KC = 128;                 // d_ff elements per D stage
+constexpr int D_CHUNKS = 2;               // 64-column chunks of d_ff per D stage (at most)
 constexpr int STAGES = 6;
 constexpr int W_BYTES = 16384;            // weight bytes per stage (both kinds)
-constexpr int XROW_BYTES = GU_KC * 2 + 16;  // padded token row of x in a GU stage
-constexpr int OP_BYTES = 17408;           // operand region: >= TN * XROW_BYTES, 1 KiB multiple
+constexpr int OP_BYTES = 16384;           // operand region: x rows or the H tile
 constexpr int SLOT_BYTES = W_BYTES + OP_BYTES;
-constexpr int PART_FLOATS = NCW * 2 * 16 * TN;  // GU partial sums for the epilogue
+constexpr int PART_FLOATS = (NCW / 2) * 2 * 16 * TN;  // GU partial sums for the epilogue
 constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * SLOT_BYTES + PART_FLOATS * 4 + 4096;
-static_assert(TN * XROW_BYTES <= OP_BYTES, "x tile does not fit");
-static_assert(2 * TN * 128 <= OP_BYTES, "H tile does not fit");
+static_assert(2 * GU_ROWS * 128 * GU_CHUNKS <= W_BYTES, "gate/up tiles do not fit");
+static_assert(D_ROWS * 128 * D_CHUNKS <= W_BYTES, "down tile does not fit");
+static_assert(TN * GU_CHUNKS * 128 <= OP_BYTES, "x rows do not fit");
+static_assert(TN * 128 * D_CHUNKS <= OP_BYTES, "H tile does not fit");
 static_assert(SLOT_BYTES % 1024 == 0, "slots must keep 1 KiB alignment for 128B swizzle");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
@@ -61,11 +63,16 @@ struct StageHdr {
 struct SharedCtl {
     unsigned long long full[STAGES];
     unsigned long long empty[STAGES];
+    unsigned long long sig_full[SIG_SLOTS];
+    unsigned long long sig_empty[SIG_SLOTS];
+    int sig_iact[SIG_SLOTS];
     StageHdr hdr[STAGES];
     volatile int abort_flag;
     volatile int consumed;
     int n_active, total_tiles;
     int tile_start[E_MAX + 1];
+    int act_e[E_MAX];       // active expert ids (copied once per CTA)
+    int off[E_MAX + 1];     // list offsets (copied once per CTA)
 };
 
 struct ExpertArgs {
@@ -108,22 +115,27 @@ __device__ __forceinline__ bool mbar_try_wait(unsigned long long *bar, unsigned 
         : "memory");
     return ok != 0;
 }
-__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int c0, int c1,
+// one box of a (chunk, row, chunk index) map: `nch` tiles of [rows][64]
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, int c0, int c1, int c2,
                                             unsigned long long *bar) {
     asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<unsigned long long>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<unsigned long long>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
         : "memory");
 }
-__device__ __forceinline__ void bulk_load(void *dst, const void *src, unsigned bytes,
-                                          unsigned long long *bar) {
+// four rows r0..r3 (any order) from column `col` of a one-row-box map
+__device__ __forceinline__ void tma_gather4(void *dst, const CUtensorMap *map, int col, int r0, int r1, int r2,
+                                            int r3, unsigned long long *bar) {
     asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            smem_u32(dst)),
-        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<unsigned long long>(map)), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3),
+        "r"(smem_u32(bar))
         : "memory");
 }
+__device__ __forceinline__ int gu_chunks_of(int d) { return min(GU_CHUNKS, d / 64); }
+__device__ __forceinline__ int d_chunks_of(int F) { return min(D_CHUNKS, F / 64); }
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<unsigned long long>(map)) : "memory");
 }
@@ -146,7 +158,13 @@ __device__ __forceinline__ int ld_acquire(const int *p) {
     asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
+__device__ __forceinline__ int ld_relaxed(const int *p) {
+    int v;
+    asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
 __device__ __forceinline__ void consumer_bar() { asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory"); }
+static_assert(NCW == 8, "the stage split below assumes eight consumer warps");
 
 // address of (row r, 16-byte chunk c) in a 128B-swizzled box with 128-byte rows
 __device__ __forceinline__ uint32_t swz(uint32_t base, int r, int c) {
@@ -175,137 +193,149 @@ __device__ bool wait_phase(unsigned long long *bar, unsigned parity, SharedCtl *
 }
 
 // ------------------------------------------------------------ producer --
+// The producer keeps one unit decoded ahead: while it issues the stages of
+// the current unit, the next ticket, the next unit's token indices (GU) or
+// its gate/up completion count (D) are already in flight, so no global
+// round trip sits between two stages.
 struct UnitInfo {
     int type, e, i_act, p0, n, row0, ns, need;
+    int tok;  // GU: token of this lane's x row (lane < n)
+    int dep;  // D (lane 0): gate/up units counted done when decoded
 };
 
-__device__ UnitInfo decode_unit(int u, const ExpertArgs &a, const SharedCtl *ctl) {
-    UnitInfo ui;
+__device__ __forceinline__ bool decode_unit(int u, int n_units, const ExpertArgs &a, const SharedCtl *ctl,
+                                            int lane, UnitInfo &ui) {
+    if (u >= n_units) return false;
     const int gu_per_tile = a.F / GU_ROWS;
     const int d_per_tile = a.d / D_ROWS;
     const int n_gu = ctl->total_tiles * gu_per_tile;
-    int tile, blk;
+    int per, v;
     if (u < n_gu) {
         ui.type = UNIT_GU;
-        tile = u / gu_per_tile;
-        blk = u % gu_per_tile;
-        ui.row0 = blk * GU_ROWS;
-        ui.ns = (a.d + GU_KC - 1) / GU_KC;
+        per = gu_per_tile;
+        v = u;
+        const int gk = 64 * gu_chunks_of(a.d);
+        ui.ns = (a.d + gk - 1) / gk;
     } else {
         ui.type = UNIT_D;
-        const int v = u - n_gu;
-        tile = v / d_per_tile;
-        blk = v % d_per_tile;
-        ui.row0 = blk * D_ROWS;
-        ui.ns = (a.F + D_KC - 1) / D_KC;
+        per = d_per_tile;
+        v = u - n_gu;
+        const int dk = 64 * d_chunks_of(a.F);
+        ui.ns = (a.F + dk - 1) / dk;
     }
-    // active expert owning this tile: largest i with tile_start[i] <= tile
+    // active expert owning this unit: largest i with tile_start[i] <= v / per
+    const int tile = v / per;
     int lo = 0, hi = ctl->n_active - 1;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
         if (ctl->tile_start[mid] <= tile) lo = mid; else hi = mid - 1;
     }
     const int i = lo;
-    const int tt = tile - ctl->tile_start[i];
-    const int off0 = __ldg(a.offsets + i), off1 = __ldg(a.offsets + i + 1);
+    // an expert's units: row block major, token tile minor, so the tiles of
+    // one weight block run back to back (a re-read then hits L2)
+    const int nt_i = ctl->tile_start[i + 1] - ctl->tile_start[i];
+    const int local = v - ctl->tile_start[i] * per;
+    const int blk = local / nt_i;
+    const int tt = local - blk * nt_i;
+    ui.row0 = blk * (ui.type == UNIT_GU ? GU_ROWS : D_ROWS);
     ui.i_act = i;
-    ui.e = __ldg(a.active + i);
-    ui.p0 = off0 + tt * TN;
-    ui.n = min(TN, off1 - ui.p0);
-    ui.need = (ctl->tile_start[i + 1] - ctl->tile_start[i]) * gu_per_tile;
-    return ui;
+    ui.e = ctl->act_e[i];
+    ui.p0 = ctl->off[i] + tt * TN;
+    ui.n = min(TN, ctl->off[i + 1] - ui.p0);
+    ui.need = nt_i * gu_per_tile;
+    ui.tok = (ui.type == UNIT_GU && lane < ui.n) ? __ldg(a.tok + ui.p0 + lane) : 0;
+    ui.dep = (ui.type == UNIT_D && lane == 0) ? ld_relaxed(&a.ctr->gu_done[i]) : 0;
+    return true;
 }
 
 __device__ void producer(const ExpertArgs &a, const ExpertMaps &m, SharedCtl *ctl, unsigned char *slots) {
     const int lane = threadIdx.x & 31;
     const int n_units = ctl->total_tiles * (a.F / GU_ROWS + a.d / D_ROWS);
+    int req = 0;
+    if (lane == 0) req = atomicAdd(&a.ctr->ticket, 1);
+    UnitInfo cur;
+    bool have = decode_unit(__shfl_sync(0xffffffffu, req, 0), n_units, a, ctl, lane, cur);
+    if (have && lane == 0) req = atomicAdd(&a.ctr->ticket, 1);
     int g = 0;  // stages issued
     bool ok = true;
-    for (;;) {
-        int u = 0;
-        if (lane == 0) u = atomicAdd(&a.ctr->ticket, 1);
-        u = __shfl_sync(0xffffffffu, u, 0);
-        if (u >= n_units) break;
-        const UnitInfo ui = decode_unit(u, a, ctl);
-        bool dep_ready = (ui.type == UNIT_GU);
-        for (int s = 0; s < ui.ns && ok; ++s, ++g) {
+    while (have && ok) {
+        UnitInfo nxt;
+        bool have_nxt = false;
+        for (int s = 0; s < cur.ns; ++s) {
             const int slot = g % STAGES;
-            if (g >= STAGES) {
-                if (!wait_phase(&ctl->empty[slot], ((g / STAGES) - 1) & 1, ctl, a.ctr, DEV_TIMEOUT_EMPTY)) {
-                    ok = false;
-                    break;
-                }
+            if (g >= STAGES &&
+                !wait_phase(&ctl->empty[slot], ((g / STAGES) - 1) & 1, ctl, a.ctr, DEV_TIMEOUT_EMPTY)) {
+                ok = false;
+                break;
             }
             unsigned char *wdst = slots + slot * SLOT_BYTES;
             unsigned char *odst = wdst + W_BYTES;
-            int kvalid, nbox;
-            unsigned bytes;
-            if (ui.type == UNIT_GU) {
-                const int k0 = s * GU_KC;
-                kvalid = min(GU_KC, a.d - k0);
-                nbox = kvalid / 64;
-                bytes = 2u * nbox * (GU_ROWS * 128) + static_cast<unsigned>(ui.n) * kvalid * 2u;
-            } else {
-                const int k0 = s * D_KC;
-                kvalid = min(D_KC, a.F - k0);
-                nbox = kvalid / 64;
-                bytes = nbox * (D_ROWS * 128u) + nbox * (TN * 128u);
-            }
+            const int gc = gu_chunks_of(a.d), dc = d_chunks_of(a.F);
+            const int nq = (cur.n + 3) >> 2;  // gather-by-four loads of x rows
+            const unsigned bytes = cur.type == UNIT_GU
+                                       ? 2u * gc * (GU_ROWS * 128) + static_cast<unsigned>(nq) * 4u * gc * 128u
+                                       : dc * (D_ROWS * 128u) + dc * (TN * 128u);
             if (lane == 0) {
                 StageHdr &h = ctl->hdr[slot];
-                h.type = ui.type;
-                h.e = ui.e;
-                h.i_act = ui.i_act;
-                h.p0 = ui.p0;
-                h.n = ui.n;
-                h.row0 = ui.row0;
+                h.type = cur.type;
+                h.e = cur.e;
+                h.i_act = cur.i_act;
+                h.p0 = cur.p0;
+                h.n = cur.n;
+                h.row0 = cur.row0;
                 h.s = s;
-                h.ns = ui.ns;
+                h.ns = cur.ns;
                 mbar_expect_tx(&ctl->full[slot], bytes);
             }
             __syncwarp();
-            if (ui.type == UNIT_GU) {
-                const int k0 = s * GU_KC;
-                const int grow = ui.e * a.F + ui.row0;
-                if (lane < nbox) {
-                    tma_load_2d(wdst + lane * (GU_ROWS * 128), &m.gate, k0 + 64 * lane, grow, &ctl->full[slot]);
-                    tma_load_2d(wdst + 8192 + lane * (GU_ROWS * 128), &m.up, k0 + 64 * lane, grow,
+            if (cur.type == UNIT_GU) {
+                const int grow = cur.e * a.F + cur.row0;
+                if (lane == 0) tma_load_3d(wdst, &m.gate, 0, grow, s * gc, &ctl->full[slot]);
+                if (lane == 1) tma_load_3d(wdst + 8192, &m.up, 0, grow, s * gc, &ctl->full[slot]);
+                // lane 2 + q loads the x rows of tokens 4q .. 4q + 3 (the last
+                // token repeated past n)
+                const int q = lane - 2;
+                int t4[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) t4[j] = __shfl_sync(0xffffffffu, cur.tok, min(4 * max(q, 0) + j, cur.n - 1));
+                if (q >= 0 && q < nq)
+                    tma_gather4(odst + q * 4 * gc * 128, &m.x, s * gc * 64, t4[0], t4[1], t4[2], t4[3],
                                 &ctl->full[slot]);
-                }
-                if (lane < ui.n) {
-                    const int t = __ldg(a.tok + ui.p0 + lane);
-                    bulk_load(odst + lane * XROW_BYTES, a.xb + static_cast<size_t>(t) * a.d + k0,
-                              static_cast<unsigned>(kvalid) * 2u, &ctl->full[slot]);
-                }
             } else {
-                const int k0 = s * D_KC;
-                if (lane < nbox)
-                    tma_load_2d(wdst + lane * (D_ROWS * 128), &m.down, k0 + 64 * lane, ui.e * a.d + ui.row0,
-                                &ctl->full[slot]);
-                if (!dep_ready) {
-                    // gate/up of this expert must be complete before its H is read
+                if (lane == 0) tma_load_3d(wdst, &m.down, 0, cur.e * a.d + cur.row0, s * dc, &ctl->full[slot]);
+                if (s == 0) {
+                    // this expert's gate/up units must be complete before H is read
                     if (lane == 0) {
-                        const unsigned long long t0 = global_ns();
-                        while (ld_acquire(&a.ctr->gu_done[ui.i_act]) < ui.need) {
-                            if (ctl->abort_flag) { ok = false; break; }
-                            if (global_ns() - t0 > WAIT_LIMIT_NS) {
-                                record_error(a.ctr, ctl, DEV_TIMEOUT_DEP);
-                                ok = false;
-                                break;
+                        int v = cur.dep;
+                        if (v < cur.need) {
+                            const unsigned long long t0 = global_ns();
+                            while ((v = ld_acquire(&a.ctr->gu_done[cur.i_act])) < cur.need) {
+                                if (ctl->abort_flag) { ok = false; break; }
+                                if (global_ns() - t0 > WAIT_LIMIT_NS) {
+                                    record_error(a.ctr, ctl, DEV_TIMEOUT_DEP);
+                                    ok = false;
+                                    break;
+                                }
+                                __nanosleep(64);
                             }
-                            __nanosleep(128);
+                        } else {
+                            asm volatile("fence.acq_rel.gpu;" ::: "memory");
                         }
                         asm volatile("fence.proxy.async.global;" ::: "memory");
                     }
                     ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-                    dep_ready = true;
                 }
-                if (ok && lane < nbox)
-                    tma_load_2d(odst + lane * (TN * 128), &m.h, k0 + 64 * lane, ui.p0, &ctl->full[slot]);
-                if (!ok) { ++g; break; }
+                if (ok && lane == 1) tma_load_3d(odst, &m.h, 0, cur.p0, s * dc, &ctl->full[slot]);
+            }
+            ++g;
+            if (!ok) break;
+            if (s == 0) {
+                have_nxt = decode_unit(__shfl_sync(0xffffffffu, req, 0), n_units, a, ctl, lane, nxt);
+                if (have_nxt && lane == 0) req = atomicAdd(&a.ctr->ticket, 1);
             }
         }
-        if (!ok) break;
+        cur = nxt;
+        have = have_nxt;
     }
     if (ok) {
         // end marker for the consumers
@@ -330,11 +360,11 @@ __device__ void producer(const ExpertArgs &a, const ExpertMaps &m, SharedCtl *ct
 
 // ------------------------------------------------------------ consumers --
 template <int NT>
-__device__ __forceinline__ void gu_stage(uint32_t wbase, uint32_t xbase, int kvalid, int warp, int lane,
+__device__ __forceinline__ void gu_stage(uint32_t wbase, uint32_t xbase, int xrow, int kvalid, int warp, int lane,
                                          float (&acc_g)[4][4], float (&acc_u)[4][4]) {
     const int nks = kvalid / 16;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < (GU_CHUNKS * 4) / NCW; ++q) {
         const int ks = warp + NCW * q;
         if (ks >= nks) break;
         const int box = ks >> 2;
@@ -348,7 +378,7 @@ __device__ __forceinline__ void gu_stage(uint32_t wbase, uint32_t xbase, int kva
         for (int np = 0; np < (NT + 1) / 2; ++np) {
             const int n = np * 16 + (lane & 7) + ((lane >> 4) << 3);
             uint32_t b0, b1, b2, b3;
-            ldsm_x4(xbase + n * XROW_BYTES + xk * 2, b0, b1, b2, b3);
+            ldsm_x4(xbase + n * xrow + xk * 2, b0, b1, b2, b3);
             mma_bf16(acc_g[2 * np], g0, g1, g2, g3, b0, b1);
             mma_bf16(acc_u[2 * np], u0, u1, u2, u3, b0, b1);
             if (2 * np + 1 < NT) {
@@ -364,10 +394,11 @@ __device__ __forceinline__ void d_stage(uint32_t wbase, uint32_t hbase, int kval
                                         float (&acc)[4][4]) {
     const int nks = kvalid / 16;
 #pragma unroll
-    for (int ks = 0; ks < D_KC / 16; ++ks) {
+    for (int q = 0; q < (D_CHUNKS * 4) / 2; ++q) {
+        const int ks = (warp >> 2) * ((D_CHUNKS * 4) / 2) + q;
         if (ks >= nks) break;
         const int box = ks >> 2;
-        const int r = warp * 16 + (lane & 15);
+        const int r = (warp & 3) * 16 + (lane & 15);
         const int chunk = ((ks & 3) << 1) + (lane >> 4);
         uint32_t a0, a1, a2, a3;
         ldsm_x4(swz(wbase + box * (D_ROWS * 128), r, chunk), a0, a1, a2, a3);
@@ -387,26 +418,59 @@ template <int NT>
 __device__ __forceinline__ void stage_dispatch(const StageHdr &h, uint32_t wbase, uint32_t obase, const ExpertArgs &a,
                                                int warp, int lane, float (&acc_g)[4][4], float (&acc_u)[4][4]) {
     if (h.type == UNIT_GU) {
-        gu_stage<NT>(wbase, obase, min(GU_KC, a.d - h.s * GU_KC), warp, lane, acc_g, acc_u);
+        const int gk = 64 * gu_chunks_of(a.d);
+        gu_stage<NT>(wbase, obase, gk * 2, min(gk, a.d - h.s * gk), warp, lane, acc_g, acc_u);
     } else {
-        d_stage<NT>(wbase, obase, min(D_KC, a.F - h.s * D_KC), warp, lane, acc_g);
+        const int dk = 64 * d_chunks_of(a.F);
+        d_stage<NT>(wbase, obase, min(dk, a.F - h.s * dk), warp, lane, acc_g);
     }
+}
+
+// Queue one gate/up completion (i >= 0) or the end marker (i < 0) for the
+// signal warp.  False if the CTA aborted.
+__device__ bool post_signal(SharedCtl *ctl, Counters *ctr, int q, int i) {
+    const int slot = q % SIG_SLOTS;
+    if (q >= SIG_SLOTS && !wait_phase(&ctl->sig_empty[slot], ((q / SIG_SLOTS) - 1) & 1, ctl, ctr, DEV_TIMEOUT_EMPTY))
+        return false;
+    ctl->sig_iact[slot] = i;
+    mbar_arrive(&ctl->sig_full[slot]);
+    return true;
 }
 
 __device__ void consumer(const ExpertArgs &a, SharedCtl *ctl, unsigned char *slots, float *part) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int ct = threadIdx.x;  // 0 .. NCW*32-1
     float acc_g[4][4], acc_u[4][4];
+    int tk[4][2];
+    float wk[4][2];
+    int nsig = 0;  // completions posted (thread 0)
+    const int row = lane >> 2, col = (lane & 3) * 2;
     for (int g = 0;; ++g) {
         const int slot = g % STAGES;
         if (!wait_phase(&ctl->full[slot], (g / STAGES) & 1, ctl, a.ctr, DEV_TIMEOUT_FULL)) return;
         const StageHdr h = ctl->hdr[slot];
-        if (h.type == UNIT_END) return;
+        if (h.type == UNIT_END) {
+            if (ct == 0) post_signal(ctl, a.ctr, nsig, -1);
+            return;
+        }
         if (h.s == 0) {
 #pragma unroll
             for (int j = 0; j < 4; ++j)
 #pragma unroll
                 for (int c = 0; c < 4; ++c) acc_g[j][c] = acc_u[j][c] = 0.0f;
+            if (h.type == UNIT_D) {
+                // tokens and gate weights this thread combines; used at the
+                // unit's last stage, loaded now so the latency is hidden
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        const int n = j * 8 + col + c;
+                        const bool v = n < h.n;
+                        tk[j][c] = v ? __ldg(a.tok + h.p0 + n) : 0;
+                        wk[j][c] = v ? __ldg(a.w + h.p0 + n) : 0.0f;
+                    }
+            }
         }
         const uint32_t wbase = smem_u32(slots + slot * SLOT_BYTES);
         const uint32_t obase = wbase + W_BYTES;
@@ -423,9 +487,9 @@ __device__ void consumer(const ExpertArgs &a, SharedCtl *ctl, unsigned char *slo
         if (h.s != h.ns - 1) continue;
 
         // ---- unit epilogue
-        const int row = lane >> 2, col = (lane & 3) * 2;
         if (h.type == UNIT_D) {
-            const int i_base = h.row0 + warp * 16 + row;
+            // each warp holds a k-half of a 16-row block: both halves add into y
+            const int i_base = h.row0 + (warp & 3) * 16 + row;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 if (j >= nt) break;
@@ -433,28 +497,41 @@ __device__ void consumer(const ExpertArgs &a, SharedCtl *ctl, unsigned char *slo
                 for (int c = 0; c < 4; ++c) {
                     const int n = j * 8 + col + (c & 1);
                     if (n < h.n) {
-                        const int pair = h.p0 + n;
-                        const int t = __ldg(a.tok + pair);
-                        const float wt = __ldg(a.w + pair);
                         const int i = i_base + ((c >> 1) << 3);
-                        atomicAdd(a.y + static_cast<size_t>(t) * a.d + i, wt * acc_g[j][c]);
+                        atomicAdd(a.y + static_cast<size_t>(tk[j][c & 1]) * a.d + i, wk[j][c & 1] * acc_g[j][c]);
                     }
                 }
             }
         } else {
-            // partial sums of this warp's k-steps -> shared, then reduce in a
-            // fixed warp order and apply silu(g) * u
-            float *pg = part + (warp * 2 + 0) * 16 * TN;
-            float *pu = part + (warp * 2 + 1) * 16 * TN;
+            // reduce the eight warps' k-slices in a fixed order (warp w + 4
+            // into warp w, then the four sums) and apply silu(g) * u
+            float *pg = part + ((warp & 3) * 2 + 0) * 16 * TN;
+            float *pu = part + ((warp & 3) * 2 + 1) * 16 * TN;
+            if (warp >= 4) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                if (j >= nt) break;
+                for (int j = 0; j < 4; ++j) {
+                    if (j >= nt) break;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const int r = row + ((c >> 1) << 3);
-                    const int n = j * 8 + col + (c & 1);
-                    pg[r * TN + n] = acc_g[j][c];
-                    pu[r * TN + n] = acc_u[j][c];
+                    for (int c = 0; c < 4; ++c) {
+                        const int r = row + ((c >> 1) << 3);
+                        const int n = j * 8 + col + (c & 1);
+                        pg[r * TN + n] = acc_g[j][c];
+                        pu[r * TN + n] = acc_u[j][c];
+                    }
+                }
+            }
+            consumer_bar();
+            if (warp < 4) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    if (j >= nt) break;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const int r = row + ((c >> 1) << 3);
+                        const int n = j * 8 + col + (c & 1);
+                        pg[r * TN + n] = acc_g[j][c] + pg[r * TN + n];
+                        pu[r * TN + n] = acc_u[j][c] + pu[r * TN + n];
+                    }
                 }
             }
             consumer_bar();
@@ -462,7 +539,7 @@ __device__ void consumer(const ExpertArgs &a, SharedCtl *ctl, unsigned char *slo
                 const int r = idx & 15, n = idx >> 4;
                 float gs = 0.0f, us = 0.0f;
 #pragma unroll
-                for (int wv = 0; wv < NCW; ++wv) {
+                for (int wv = 0; wv < NCW / 2; ++wv) {
                     gs += part[(wv * 2 + 0) * 16 * TN + r * TN + n];
                     us += part[(wv * 2 + 1) * 16 * TN + r * TN + n];
                 }
@@ -470,14 +547,28 @@ __device__ void consumer(const ExpertArgs &a, SharedCtl *ctl, unsigned char *slo
                 a.h[static_cast<size_t>(h.p0 + n) * a.F + h.row0 + r] =
                     __bfloat16_as_ushort(__float2bfloat16_rn(hv));
             }
-            __threadfence();
+            // H is read by other CTAs through TMA (the async proxy)
             asm volatile("fence.proxy.async.global;" ::: "memory");
             consumer_bar();
-            if (ct == 0) {
-                __threadfence();
-                atomicAdd(&a.ctr->gu_done[h.i_act], 1);
-            }
+            // the signal warp publishes the completion (fence + counter), so
+            // the consumers do not wait for it
+            if (ct == 0 && !post_signal(ctl, a.ctr, nsig++, h.i_act)) return;
         }
+    }
+}
+
+// Signal warp: turns queued gate/up completions into gu_done increments
+// visible to the whole GPU.
+__device__ void signaller(const ExpertArgs &a, SharedCtl *ctl) {
+    if ((threadIdx.x & 31) != 0) return;
+    for (int q = 0;; ++q) {
+        const int slot = q % SIG_SLOTS;
+        if (!wait_phase(&ctl->sig_full[slot], (q / SIG_SLOTS) & 1, ctl, a.ctr, DEV_TIMEOUT_FULL)) return;
+        const int i = ctl->sig_iact[slot];
+        mbar_arrive(&ctl->sig_empty[slot]);
+        if (i < 0) return;
+        __threadfence();
+        atomicAdd(&a.ctr->gu_done[i], 1);
     }
 }
 
@@ -496,6 +587,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             mbar_init(&ctl->full[s], 1);
             mbar_init(&ctl->empty[s], NCW);
         }
+        for (int s = 0; s < SIG_SLOTS; ++s) {
+            mbar_init(&ctl->sig_full[s], 1);
+            mbar_init(&ctl->sig_empty[s], 1);
+        }
         ctl->abort_flag = 0;
         ctl->consumed = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -505,6 +600,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         prefetch_tmap(&maps.up);
         prefetch_tmap(&maps.down);
         prefetch_tmap(&maps.h);
+        prefetch_tmap(&maps.x);
     }
     // everything above overlaps the re-selection kernel; the lists are read
     // only after it has completed
@@ -523,9 +619,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 const int v = __shfl_up_sync(0xffffffffu, incl, o);
                 if (lane >= o) incl += v;
             }
-            if (i < na) ctl->tile_start[i] = run + incl - nt;
+            if (i < na) {
+                ctl->tile_start[i] = run + incl - nt;
+                ctl->act_e[i] = __ldg(a.active + i);
+                ctl->off[i] = __ldg(a.offsets + i);
+            }
             run += __shfl_sync(0xffffffffu, incl, 31);
         }
+        if (lane == 0 && na >= 0 && na <= a.E) ctl->off[na] = __ldg(a.offsets + na);
         if (lane == 0) {
             ctl->tile_start[na] = run;
             ctl->n_active = na;
@@ -536,6 +637,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     __syncthreads();
     if (warp == NCW) {
         producer(a, maps, ctl, slots);
+    } else if (warp == NCW + 1) {
+        signaller(a, ctl);
     } else {
         consumer(a, ctl, slots, part);
     }
@@ -565,6 +668,10 @@ int g_num_sms[64] = {0};
 }  // namespace
 
 int expert_ffn_h_rows() { return TN; }
+int expert_ffn_gu_rows() { return GU_ROWS; }
+int expert_ffn_d_rows() { return D_ROWS; }
+int expert_ffn_gu_chunks(int d) { return d / 64 < GU_CHUNKS ? d / 64 : GU_CHUNKS; }
+int expert_ffn_d_chunks(int F) { return F / 64 < D_CHUNKS ? F / 64 : D_CHUNKS; }
 
 cudaError_t launch_ffn_prep(const float *x, const moe_dims_t &d, uint16_t *xb, float *y, Counters *ctr,
                             cudaStream_t s) {

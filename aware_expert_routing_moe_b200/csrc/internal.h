@@ -57,16 +57,24 @@ cudaError_t launch_reselect(const float *logits, float *probs, bool fuse_softmax
 cudaError_t launch_ffn_prep(const float *x, const moe_dims_t &d, uint16_t *xb, float *y,
                             Counters *ctr, cudaStream_t s);
 
+// TMA descriptors of the expert kernel: the three weight tensors and the H
+// scratch as (64-column chunk, row, chunk index) boxes, and x in bf16 as
+// single rows for gather-by-four loads.
 struct ExpertMaps {
-    CUtensorMap gate, up, down, h;
+    CUtensorMap gate, up, down, h, x;
 };
 cudaError_t launch_expert_ffn(const ExpertMaps &maps, const uint16_t *xb,
                               const moe_dims_t &d, const moe_lists_t &l, float *y,
                               uint16_t *h, Counters *ctr, bool pdl, cudaStream_t s);
-int expert_ffn_h_rows();   // row count of one H tile box (tokens per tile)
+int expert_ffn_h_rows();              // rows of one H box (tokens per tile)
+int expert_ffn_gu_rows();             // rows of Wgate / Wup per gate-up unit
+int expert_ffn_d_rows();              // rows of Wdown per down unit
+int expert_ffn_gu_chunks(int d);      // 64-column chunks of d per gate-up stage
+int expert_ffn_d_chunks(int d_ff);    // 64-column chunks of d_ff per down stage
 
-// TMA descriptors of the expert kernel (weights and the H scratch at `h`).
+// Builds the expert kernel's TMA descriptors (weights, H scratch at `h`,
+// bf16 x at `xb`).
 bool encode_expert_maps(ExpertMaps *m, const moe_dims_t &d, const uint16_t *Wgate, const uint16_t *Wup,
-                        const uint16_t *Wdown, const uint16_t *h);
+                        const uint16_t *Wdown, const uint16_t *h, const uint16_t *xb);
 
 }  // namespace moe

@@ -98,7 +98,7 @@ extern "C" moe_status_t moe_expert_ffn_noalloc(const float *x, const uint16_t *W
     uint16_t *xb = reinterpret_cast<uint16_t *>(scratch + L.xb);
     uint16_t *h = reinterpret_cast<uint16_t *>(scratch + L.h);
     ExpertMaps maps;
-    if (!encode_expert_maps(&maps, dims, Wgate, Wup, Wdown, h)) return MOE_ERR_CUDA;
+    if (!encode_expert_maps(&maps, dims, Wgate, Wup, Wdown, h, xb)) return MOE_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     // the prep kernel clears the ticket and the per-expert counters the
     // expert kernel needs at zero; x and H are fully rewritten each call

@@ -146,27 +146,60 @@ __device__ __forceinline__ void token_softmax(const float (&l)[NI], int E, int l
     for (int i = 0; i < NI; ++i) p[i] = (lane + 32 * i < E) ? __fdiv_rn(q[i], Z) : 0.0f;
 }
 
-// Gate weights renormalised over the chosen slots (slot order, fp32 from
-// +0); every lane computes the same values.
-__device__ __forceinline__ void renormalise(const int (&sel)[K_MAX], const float (&ps)[K_MAX], int k,
-                                            float (&w)[K_MAX]) {
+// Top-r of the candidate experts by rank key, r rounds of warp arg-max.
+// Lane 0 writes the winners to out[0..) and their probabilities to pout[0..)
+// (when pout != nullptr).  Stops early when no candidate is left; returns the
+// number found.
+template <int NI>
+__device__ int warp_select(const unsigned long long (&key)[NI], unsigned &cand, const float (&p)[NI], int r,
+                           int lane, int *out, float *pout) {
+    int n = 0;
+#pragma unroll 1
+    for (int j = 0; j < r; ++j) {
+        const int e = warp_take_best<NI>(key, cand, lane);
+        if (e < 0) break;
+        const float pe = warp_fetch<NI>(p, e);
+        if (lane == 0) {
+            out[j] = e;
+            if (pout) pout[j] = pe;
+        }
+        ++n;
+    }
+    __syncwarp();
+    return n;
+}
+
+// Gate weights renormalised over the chosen slots: sel[0..k) and their
+// probabilities pv[0..k) in shared memory (sel < 0 = empty slot); pv is
+// overwritten with the weights.  The sum runs in slot order from +0 (lane 0),
+// then lane j divides slot j.
+__device__ void renormalise_slots(const int *sel, float *pv, int k, int lane) {
     float s = 0.0f;
-#pragma unroll
-    for (int j = 0; j < K_MAX; ++j)
-        if (j < k && sel[j] >= 0) s = __fadd_rn(s, ps[j]);
-#pragma unroll
-    for (int j = 0; j < K_MAX; ++j) w[j] = (j < k && sel[j] >= 0) ? __fdiv_rn(ps[j], s) : 0.0f;
+    if (lane == 0) {
+#pragma unroll 1
+        for (int j = 0; j < k; ++j)
+            if (sel[j] >= 0) s = __fadd_rn(s, pv[j]);
+    }
+    s = __shfl_sync(FULL, s, 0);
+    __syncwarp();
+    if (lane < k) pv[lane] = sel[lane] >= 0 ? __fdiv_rn(pv[lane], s) : 0.0f;
+    __syncwarp();
 }
 
 // ------------------------------------------------------------------ K1 --
-// Warp w of block (bx, by) computes expert e = 8 bx + w for tokens
-// TB by .. TB by + TB - 1.  The eight warps of a block read the same token
-// rows, which stay in L1.
-template <int TB>
+// Block (bx, by) computes experts 8 bx .. 8 bx + 7 (one per warp) for the
+// tokens tb * by .. tb * by + tb - 1.  The block stages those token rows in
+// shared memory; each warp holds up to R_CH 256-column chunks of its Wg row
+// in registers (all loads issued before any use) and runs the fixed-order
+// fma chains against the shared rows.
+constexpr int R_TB = 4;  // tokens per block (at most)
+constexpr int R_CH = 8;  // 256-column chunks of a Wg row held at once
+
 __global__ void __launch_bounds__(256) router_logits_kernel(
     const float *__restrict__ x, const float *__restrict__ Wg, const float *__restrict__ bias,
-    int B, int d, int E, float *__restrict__ logits, uint16_t *__restrict__ xb,
+    int B, int d, int E, int tb, float *__restrict__ logits, uint16_t *__restrict__ xb,
     float *__restrict__ y_zero) {
+    extern __shared__ float4 xs4[];  // [tb][d / 4]
     if (xb != nullptr) {
         // layer path: x -> bf16 copy for the expert kernel, y = 0
         const int n4 = B * d / 4;
@@ -184,43 +217,61 @@ __global__ void __launch_bounds__(256) router_logits_kernel(
     }
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int e = blockIdx.x * 8 + warp;
-    const int b0 = blockIdx.y * TB;
+    const int b0 = blockIdx.y * tb;
+    const int nb = min(tb, B - b0);
+    const int d4 = d / 4;
+    {
+        const float4 *src = reinterpret_cast<const float4 *>(x) + static_cast<size_t>(b0) * d4;
+        for (int i = threadIdx.x; i < nb * d4; i += blockDim.x) xs4[i] = __ldg(src + i);
+    }
+    __syncthreads();
     if (e < E) {
-        float acc[TB];
+        float acc[R_TB];
 #pragma unroll
-        for (int t = 0; t < TB; ++t) acc[t] = 0.0f;
+        for (int t = 0; t < R_TB; ++t) acc[t] = 0.0f;
         const float *wrow = Wg + static_cast<size_t>(e) * d;
-        for (int c = 0; 256 * c < d; ++c) {
-            const int j0 = 256 * c + 8 * lane;
-            if (j0 >= d) continue;
-            const float4 w0 = __ldg(reinterpret_cast<const float4 *>(wrow + j0));
-            const float4 w1 = __ldg(reinterpret_cast<const float4 *>(wrow + j0 + 4));
+        const int nch = (d + 255) / 256;
+#pragma unroll 1
+        for (int c0 = 0; c0 < nch; c0 += R_CH) {
+            float4 w[R_CH][2];
 #pragma unroll
-            for (int t = 0; t < TB; ++t) {
-                if (b0 + t < B) {
-                    const float *xr = x + static_cast<size_t>(b0 + t) * d + j0;
-                    const float4 x0 = __ldg(reinterpret_cast<const float4 *>(xr));
-                    const float4 x1 = __ldg(reinterpret_cast<const float4 *>(xr + 4));
-                    float a = acc[t];
-                    a = __fmaf_rn(x0.x, w0.x, a);
-                    a = __fmaf_rn(x0.y, w0.y, a);
-                    a = __fmaf_rn(x0.z, w0.z, a);
-                    a = __fmaf_rn(x0.w, w0.w, a);
-                    a = __fmaf_rn(x1.x, w1.x, a);
-                    a = __fmaf_rn(x1.y, w1.y, a);
-                    a = __fmaf_rn(x1.z, w1.z, a);
-                    a = __fmaf_rn(x1.w, w1.w, a);
-                    acc[t] = a;
+            for (int cc = 0; cc < R_CH; ++cc) {
+                const int j0 = 256 * (c0 + cc) + 8 * lane;
+                if (c0 + cc < nch && j0 < d) {
+                    w[cc][0] = __ldg(reinterpret_cast<const float4 *>(wrow + j0));
+                    w[cc][1] = __ldg(reinterpret_cast<const float4 *>(wrow + j0 + 4));
                 }
+            }
+#pragma unroll
+            for (int t = 0; t < R_TB; ++t) {
+                if (t >= nb) break;
+                float a = acc[t];
+#pragma unroll
+                for (int cc = 0; cc < R_CH; ++cc) {
+                    const int j0 = 256 * (c0 + cc) + 8 * lane;
+                    if (c0 + cc < nch && j0 < d) {
+                        const float4 x0 = xs4[(t * d + j0) / 4];
+                        const float4 x1 = xs4[(t * d + j0) / 4 + 1];
+                        a = __fmaf_rn(x0.x, w[cc][0].x, a);
+                        a = __fmaf_rn(x0.y, w[cc][0].y, a);
+                        a = __fmaf_rn(x0.z, w[cc][0].z, a);
+                        a = __fmaf_rn(x0.w, w[cc][0].w, a);
+                        a = __fmaf_rn(x1.x, w[cc][1].x, a);
+                        a = __fmaf_rn(x1.y, w[cc][1].y, a);
+                        a = __fmaf_rn(x1.z, w[cc][1].z, a);
+                        a = __fmaf_rn(x1.w, w[cc][1].w, a);
+                    }
+                }
+                acc[t] = a;
             }
         }
         float mine = 0.0f;
 #pragma unroll
-        for (int t = 0; t < TB; ++t) {
+        for (int t = 0; t < R_TB; ++t) {
             const float v = warp_butterfly_sum(acc[t]);
             if (lane == t) mine = v;
         }
-        if (lane < TB && b0 + lane < B) {
+        if (lane < nb) {
             const float v = bias ? __fadd_rn(mine, __ldg(bias + e)) : mine;
             logits[static_cast<size_t>(b0 + lane) * E + e] = v;
         }
@@ -236,6 +287,8 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict
                                                          int k, float *__restrict__ probs,
                                                          int32_t *__restrict__ topk_idx,
                                                          float *__restrict__ topk_w) {
+    __shared__ int s_sel[8][K_MAX];
+    __shared__ float s_w[8][K_MAX];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int b = blockIdx.x * 8 + warp;
     if (b >= B) return;
@@ -249,24 +302,12 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict
 #pragma unroll
     for (int i = 0; i < NI; ++i) key[i] = rank_key(l[i], lane + 32 * i);
     unsigned cand = valid_bits<NI>(E, lane);
-    int sel[K_MAX];
-    float ps[K_MAX], w[K_MAX];
-#pragma unroll
-    for (int j = 0; j < K_MAX; ++j) {
-        sel[j] = -1;
-        ps[j] = 0.0f;
-        if (j < k) {
-            sel[j] = warp_take_best<NI>(key, cand, lane);
-            ps[j] = warp_fetch<NI>(p, sel[j]);
-        }
+    warp_select<NI>(key, cand, p, k, lane, s_sel[warp], s_w[warp]);
+    renormalise_slots(s_sel[warp], s_w[warp], k, lane);
+    if (lane < k) {
+        topk_idx[static_cast<size_t>(b) * k + lane] = s_sel[warp][lane];
+        topk_w[static_cast<size_t>(b) * k + lane] = s_w[warp][lane];
     }
-    renormalise(sel, ps, k, w);
-#pragma unroll
-    for (int j = 0; j < K_MAX; ++j)
-        if (j < k && lane == j) {
-            topk_idx[static_cast<size_t>(b) * k + j] = sel[j];
-            topk_w[static_cast<size_t>(b) * k + j] = w[j];
-        }
 }
 
 // -------------------------------------------------------------- reselect --
@@ -320,11 +361,11 @@ __global__ void __launch_bounds__(1024, 1) reselect_kernel(ReselectArgs a) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const int B = a.B, E = a.E, k = a.k;
     const int BW = (B + 31) >> 5;
-    int *T = reinterpret_cast<int *>(smem_raw);                  // [B][k]
-    int *SEL = T + B * k;                                          // [B][k]
-    float *SELW = reinterpret_cast<float *>(SEL + B * k);         // [B][k]
-    unsigned *ASSIGN = reinterpret_cast<unsigned *>(SELW + B * k);  // [E][BW]
-    unsigned *TMEMB = ASSIGN + E * BW;                              // [E][BW]
+    int *T = reinterpret_cast<int *>(smem_raw);                      // [B][k] first ranks
+    int *SEL = T + B * k;                                              // [B][k] chosen experts
+    float *SELW = reinterpret_cast<float *>(SEL + B * k);             // [B][k] p, then weights
+    unsigned *ASSIGN = reinterpret_cast<unsigned *>(SELW + B * k);    // [E][BW]
+    unsigned *TMEMB = ASSIGN + E * BW;                                  // [E][BW]
     __shared__ float s_score[E_MAX];
     __shared__ int s_off[E_MAX];
     __shared__ unsigned ukept[E_MAX / 32], ubase[E_MAX / 32], sbits[E_MAX / 32];
@@ -338,6 +379,7 @@ __global__ void __launch_bounds__(1024, 1) reselect_kernel(ReselectArgs a) {
     const int mode = a.mode;
     // ---- phase 1: per token softmax (layer path) + first ranks
     const int r1 = (mode == MOE_RESELECT_OEA) ? a.k0 : k;
+#pragma unroll 1
     for (int b = warp; b < B; b += 32) {
         float l[NI], p[NI];
         load_row<NI>(a.logits + static_cast<size_t>(b) * E, E, lane, l);
@@ -353,37 +395,19 @@ __global__ void __launch_bounds__(1024, 1) reselect_kernel(ReselectArgs a) {
 #pragma unroll
         for (int i = 0; i < NI; ++i) key[i] = rank_key(l[i], lane + 32 * i);
         unsigned cand = valid_bits<NI>(E, lane);
-        int sel[K_MAX];
-        float ps[K_MAX];
-#pragma unroll
-        for (int j = 0; j < K_MAX; ++j) {
-            sel[j] = -1;
-            ps[j] = 0.0f;
-            if (j < r1) {
-                sel[j] = warp_take_best<NI>(key, cand, lane);
-                ps[j] = warp_fetch<NI>(p, sel[j]);
+        warp_select<NI>(key, cand, p, r1, lane, T + b * k, mode == MOE_RESELECT_NONE ? SELW + b * k : nullptr);
+        if (lane < r1) {
+            const int e = T[b * k + lane];
+            if (mode == MOE_RESELECT_OEA) atomicOr(&ukept[e >> 5], 1u << (e & 31));
+            if (mode == MOE_RESELECT_XSHARE) {
+                atomicOr(&ubase[e >> 5], 1u << (e & 31));
+                atomicOr(&TMEMB[e * BW + (b >> 5)], 1u << (b & 31));
             }
+            if (mode == MOE_RESELECT_NONE) SEL[b * k + lane] = e;
         }
-#pragma unroll
-        for (int j = 0; j < K_MAX; ++j)
-            if (j < r1 && lane == j) {
-                const int e = sel[j];
-                T[b * k + j] = e;
-                if (mode == MOE_RESELECT_OEA) atomicOr(&ukept[e >> 5], 1u << (e & 31));
-                if (mode == MOE_RESELECT_XSHARE) {
-                    atomicOr(&ubase[e >> 5], 1u << (e & 31));
-                    atomicOr(&TMEMB[e * BW + (b >> 5)], 1u << (b & 31));
-                }
-            }
         if (mode == MOE_RESELECT_NONE) {
-            float w[K_MAX];
-            renormalise(sel, ps, k, w);
-#pragma unroll
-            for (int j = 0; j < K_MAX; ++j)
-                if (j < k && lane == j) {
-                    SEL[b * k + j] = sel[j];
-                    SELW[b * k + j] = w[j];
-                }
+            __syncwarp();
+            renormalise_slots(SEL + b * k, SELW + b * k, k, lane);
         }
     }
     __syncthreads();
@@ -392,6 +416,7 @@ __global__ void __launch_bounds__(1024, 1) reselect_kernel(ReselectArgs a) {
     if (mode == MOE_RESELECT_XSHARE) {
         if (tid < E) {
             float s = 0.0f;
+#pragma unroll 1
             for (int b = 0; b < B; ++b)
                 if ((TMEMB[tid * BW + (b >> 5)] >> (b & 31)) & 1u)
                     s = __fadd_rn(s, a.probs[static_cast<size_t>(b) * E + tid]);
@@ -404,6 +429,7 @@ __global__ void __launch_bounds__(1024, 1) reselect_kernel(ReselectArgs a) {
             const int Mp = a.budget < nb ? a.budget : nb;
             const float se = s_score[tid];
             int rank = 0;
+#pragma unroll 1
             for (int e2 = 0; e2 < E; ++e2) {
                 if (!((ubase[e2 >> 5] >> (e2 & 31)) & 1u)) continue;
                 const float s2 = s_score[e2];
@@ -416,6 +442,7 @@ __global__ void __launch_bounds__(1024, 1) reselect_kernel(ReselectArgs a) {
 
     // ---- phase 2: OEA fills / XShare top-k within the batch set; weights
     if (mode != MOE_RESELECT_NONE) {
+#pragma unroll 1
         for (int b = warp; b < B; b += 32) {
             float l[NI], p[NI];
             load_row<NI>(a.logits + static_cast<size_t>(b) * E, E, lane, l);
@@ -430,41 +457,25 @@ __global__ void __launch_bounds__(1024, 1) reselect_kernel(ReselectArgs a) {
                 const int e = lane + 32 * i;
                 if (e < E && ((bits[e >> 5] >> (e & 31)) & 1u)) cand |= 1u << i;
             }
-            int sel[K_MAX];
-            float ps[K_MAX];
             const int kk = (mode == MOE_RESELECT_OEA) ? a.k0 : 0;
-#pragma unroll
-            for (int j = 0; j < K_MAX; ++j) {
-                sel[j] = -1;
-                ps[j] = 0.0f;
-                if (j < kk) {
-                    const int e = T[b * k + j];
-                    sel[j] = e;
-                    if ((e & 31) == lane) cand &= ~(1u << (e >> 5));
-                    ps[j] = warp_fetch<NI>(p, e);
+#pragma unroll 1
+            for (int j = 0; j < kk; ++j) {  // kept experts first, in rank order
+                const int e = T[b * k + j];
+                if ((e & 31) == lane) cand &= ~(1u << (e >> 5));
+                const float pe = warp_fetch<NI>(p, e);
+                if (lane == 0) {
+                    SEL[b * k + j] = e;
+                    SELW[b * k + j] = pe;
                 }
             }
-            int stop = 0;
-#pragma unroll
-            for (int j = 0; j < K_MAX; ++j) {
-                if (j >= kk && j < k && !stop) {
-                    const int e = warp_take_best<NI>(key, cand, lane);
-                    if (e < 0) {
-                        stop = 1;
-                    } else {
-                        sel[j] = e;
-                        ps[j] = warp_fetch<NI>(p, e);
-                    }
-                }
+            __syncwarp();
+            const int nf = warp_select<NI>(key, cand, p, k - kk, lane, SEL + b * k + kk, SELW + b * k + kk);
+            if (lane >= kk + nf && lane < k) {
+                SEL[b * k + lane] = -1;
+                SELW[b * k + lane] = 0.0f;
             }
-            float w[K_MAX];
-            renormalise(sel, ps, k, w);
-#pragma unroll
-            for (int j = 0; j < K_MAX; ++j)
-                if (j < k && lane == j) {
-                    SEL[b * k + j] = sel[j];
-                    SELW[b * k + j] = w[j];
-                }
+            __syncwarp();
+            renormalise_slots(SEL + b * k, SELW + b * k, k, lane);
         }
         __syncthreads();
     }
@@ -530,9 +541,19 @@ int ni_for(int E) { return E <= 32 ? 1 : E <= 64 ? 2 : E <= 128 ? 4 : 8; }
 cudaError_t launch_router_logits(const float *x, const float *Wg, const float *bias,
                                  const moe_dims_t &d, float *logits, uint16_t *xb,
                                  float *y_zero, cudaStream_t s) {
-    constexpr int TB = 8;
-    dim3 grid((d.E + 7) / 8, (d.B + TB - 1) / TB);
-    router_logits_kernel<TB><<<grid, 256, 0, s>>>(x, Wg, bias, d.B, d.d, d.E, logits, xb, y_zero);
+    static bool configured = false;  // one GPU per process
+    if (!configured) {
+        const cudaError_t err = cudaFuncSetAttribute(router_logits_kernel,
+                                                     cudaFuncAttributeMaxDynamicSharedMemorySize, 192 * 1024);
+        if (err != cudaSuccess) return err;
+        configured = true;
+    }
+    // tokens per block: up to R_TB, and at most 160 KB of staged rows
+    int tb = R_TB;
+    while (tb > 1 && static_cast<size_t>(tb) * d.d * 4 > 160u * 1024u) --tb;
+    dim3 grid((d.E + 7) / 8, (d.B + tb - 1) / tb);
+    const size_t smem = static_cast<size_t>(tb) * d.d * 4;
+    router_logits_kernel<<<grid, 256, smem, s>>>(x, Wg, bias, d.B, d.d, d.E, tb, logits, xb, y_zero);
     return cudaGetLastError();
 }
 
