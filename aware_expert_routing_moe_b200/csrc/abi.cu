@@ -160,7 +160,9 @@ bool encode_expert_maps(ExpertMaps *m, const moe_dims_t &d, const uint16_t *Wgat
            encode_bf16_chunked(&m->up, Wup, E * F, D, expert_ffn_gu_rows(), gu_chunks) &&
            encode_bf16_chunked(&m->down, Wdown, E * D, F, expert_ffn_d_rows(), d_chunks) &&
            encode_bf16_chunked(&m->h, h, static_cast<uint64_t>(d.B) * d.k, F, expert_ffn_h_rows(), d_chunks) &&
-           encode_bf16_rows(&m->x, xb, static_cast<uint64_t>(d.B), D, gu_chunks * 64);
+           (expert_ffn_dense_batch(d.B)
+                ? encode_bf16_chunked(&m->x, xb, static_cast<uint64_t>(d.B), D, (d.B + 7) / 8 * 8, gu_chunks)
+                : encode_bf16_rows(&m->x, xb, static_cast<uint64_t>(d.B), D, expert_ffn_gather_cols(d.d)));
 }
 
 WsLayout ws_layout(const moe_dims_t &d) {

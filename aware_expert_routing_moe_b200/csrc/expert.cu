@@ -36,21 +36,37 @@ constexpr int NTHREADS = (NCW + 2) * 32;  // + one producer warp + one signal wa
 constexpr int SIG_SLOTS = 4;              // gate/up completions queued for the signal warp
 constexpr int TN = 32;                    // tokens per tile
 constexpr int GU_ROWS = 16;               // rows of Wgate and of Wup per GU unit
-constexpr int GU_CHUNKS = 4;              // 64-column chunks of d per GU stage (at most)
+constexpr int GU_CHUNKS = 8;              // 64-column chunks of d per GU stage (at most)
 constexpr int D_ROWS = 64;                // rows of Wdown per D unit
-constexpr int D_CHUNKS = 2;               // 64-column chunks of d_ff per D stage (at most)
-constexpr int STAGES = 6;
-constexpr int W_BYTES = 16384;            // weight bytes per stage (both kinds)
-constexpr int OP_BYTES = 16384;           // operand region: x rows or the H tile
-constexpr int SLOT_BYTES = W_BYTES + OP_BYTES;
-constexpr int PART_FLOATS = (NCW / 2) * 2 * 16 * TN;  // GU partial sums for the epilogue
-constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * SLOT_BYTES + PART_FLOATS * 4 + 4096;
+constexpr int D_CHUNKS = 4;               // 64-column chunks of d_ff per D stage (at most)
+constexpr int MAX_STAGES = 4;
+constexpr int W_BYTES = 32768;            // weight bytes per stage (both kinds)
+constexpr int UP_OFF = GU_ROWS * 128 * GU_CHUNKS;  // Wup tile after the Wgate tile
+constexpr int GATHER_COLS = 256;          // widest row box of a gather-by-four load
+// Two ring shapes: 4 stages with a 16 KB operand region (B <= 16), and 3
+// stages with 32 KB (larger batches).
+template <int ST, int OPB>
+struct Ring {
+    static constexpr int STAGES = ST;
+    static constexpr int OP_BYTES = OPB;
+    static constexpr int SLOT_BYTES = W_BYTES + OPB;
+};
+constexpr int PART_LD = TN + 1;                        // padded row of the epilogue buffer
+constexpr int PART_FLOATS = (NCW / 2) * 2 * 16 * PART_LD;  // GU partial sums for the epilogue
+template <class RG>
+constexpr int smem_bytes() {
+    return 1024 /*align slack*/ + RG::STAGES * RG::SLOT_BYTES + PART_FLOATS * 4 + 4096;
+}
+using RingSmallB = Ring<4, 16384>;
+using RingLargeB = Ring<3, 32768>;
 static_assert(2 * GU_ROWS * 128 * GU_CHUNKS <= W_BYTES, "gate/up tiles do not fit");
 static_assert(D_ROWS * 128 * D_CHUNKS <= W_BYTES, "down tile does not fit");
-static_assert(TN * GU_CHUNKS * 128 <= OP_BYTES, "x rows do not fit");
-static_assert(TN * 128 * D_CHUNKS <= OP_BYTES, "H tile does not fit");
-static_assert(SLOT_BYTES % 1024 == 0, "slots must keep 1 KiB alignment for 128B swizzle");
-static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+static_assert(16 * GU_CHUNKS * 128 <= RingSmallB::OP_BYTES, "dense x rows (B <= 16) do not fit");
+static_assert(TN * GU_CHUNKS * 128 <= RingLargeB::OP_BYTES, "x rows (32 tokens) do not fit");
+static_assert(TN * 128 * D_CHUNKS <= RingSmallB::OP_BYTES, "H tile does not fit");
+static_assert(RingSmallB::SLOT_BYTES % 1024 == 0 && RingLargeB::SLOT_BYTES % 1024 == 0,
+              "slots must keep 1 KiB alignment for 128B swizzle");
+static_assert(smem_bytes<RingSmallB>() <= 232448 && smem_bytes<RingLargeB>() <= 232448, "shared memory budget");
 
 constexpr unsigned long long WAIT_LIMIT_NS = 1000000000ull;  // 1 s
 
@@ -61,12 +77,12 @@ struct StageHdr {
 };
 
 struct SharedCtl {
-    unsigned long long full[STAGES];
-    unsigned long long empty[STAGES];
+    unsigned long long full[MAX_STAGES];
+    unsigned long long empty[MAX_STAGES];
     unsigned long long sig_full[SIG_SLOTS];
     unsigned long long sig_empty[SIG_SLOTS];
     int sig_iact[SIG_SLOTS];
-    StageHdr hdr[STAGES];
+    StageHdr hdr[MAX_STAGES];
     volatile int abort_flag;
     volatile int consumed;
     int n_active, total_tiles;
@@ -78,6 +94,9 @@ struct SharedCtl {
 struct ExpertArgs {
     const uint16_t *xb;
     int B, d, E, k, F;
+    int xbox;   // gather mode: columns per row box of the x map (<= GATHER_COLS)
+    int dense;  // B <= TN: every gate/up stage loads all B token rows in one box
+    int bpad;   // B rounded up to a multiple of 8 (dense mode)
     const int32_t *n_active, *active, *offsets, *tok;
     const float *w;
     float *y;
@@ -243,12 +262,17 @@ __device__ __forceinline__ bool decode_unit(int u, int n_units, const ExpertArgs
     ui.p0 = ctl->off[i] + tt * TN;
     ui.n = min(TN, ctl->off[i + 1] - ui.p0);
     ui.need = nt_i * gu_per_tile;
-    ui.tok = (ui.type == UNIT_GU && lane < ui.n) ? __ldg(a.tok + ui.p0 + lane) : 0;
-    ui.dep = (ui.type == UNIT_D && lane == 0) ? ld_relaxed(&a.ctr->gu_done[i]) : 0;
+    // both loads are unconditional (valid addresses) so that nothing waits
+    // for them here; their values are first used when the unit's first stage
+    // is issued
+    ui.tok = __ldg(a.tok + ui.p0 + min(lane, ui.n - 1));
+    ui.dep = ld_relaxed(&a.ctr->gu_done[i]);
     return true;
 }
 
+template <class RG>
 __device__ void producer(const ExpertArgs &a, const ExpertMaps &m, SharedCtl *ctl, unsigned char *slots) {
+    constexpr int STAGES = RG::STAGES;
     const int lane = threadIdx.x & 31;
     const int n_units = ctl->total_tiles * (a.F / GU_ROWS + a.d / D_ROWS);
     int req = 0;
@@ -268,13 +292,15 @@ __device__ void producer(const ExpertArgs &a, const ExpertMaps &m, SharedCtl *ct
                 ok = false;
                 break;
             }
-            unsigned char *wdst = slots + slot * SLOT_BYTES;
+            unsigned char *wdst = slots + slot * RG::SLOT_BYTES;
             unsigned char *odst = wdst + W_BYTES;
             const int gc = gu_chunks_of(a.d), dc = d_chunks_of(a.F);
             const int nq = (cur.n + 3) >> 2;  // gather-by-four loads of x rows
-            const unsigned bytes = cur.type == UNIT_GU
-                                       ? 2u * gc * (GU_ROWS * 128) + static_cast<unsigned>(nq) * 4u * gc * 128u
-                                       : dc * (D_ROWS * 128u) + dc * (TN * 128u);
+            const int nhalf = (gc * 64 + a.xbox - 1) / a.xbox;  // gather loads per four tokens
+            const unsigned xbytes = a.dense ? static_cast<unsigned>(gc) * a.bpad * 128u
+                                            : static_cast<unsigned>(nq) * nhalf * 4u * a.xbox * 2u;
+            const unsigned bytes = cur.type == UNIT_GU ? 2u * gc * (GU_ROWS * 128) + xbytes
+                                                       : dc * (D_ROWS * 128u) + dc * (TN * 128u);
             if (lane == 0) {
                 StageHdr &h = ctl->hdr[slot];
                 h.type = cur.type;
@@ -291,16 +317,23 @@ __device__ void producer(const ExpertArgs &a, const ExpertMaps &m, SharedCtl *ct
             if (cur.type == UNIT_GU) {
                 const int grow = cur.e * a.F + cur.row0;
                 if (lane == 0) tma_load_3d(wdst, &m.gate, 0, grow, s * gc, &ctl->full[slot]);
-                if (lane == 1) tma_load_3d(wdst + 8192, &m.up, 0, grow, s * gc, &ctl->full[slot]);
-                // lane 2 + q loads the x rows of tokens 4q .. 4q + 3 (the last
-                // token repeated past n)
-                const int q = lane - 2;
-                int t4[4];
+                if (lane == 1) tma_load_3d(wdst + UP_OFF, &m.up, 0, grow, s * gc, &ctl->full[slot]);
+                if (a.dense) {
+                    // all B token rows of this column range in one swizzled box
+                    if (lane == 2) tma_load_3d(odst, &m.x, 0, 0, s * gc, &ctl->full[slot]);
+                } else {
+                    // lane 2 + q loads the x rows of tokens 4q .. 4q + 3 (the
+                    // last token repeated past n)
+                    const int q = lane - 2;
+                    int t4[4];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) t4[j] = __shfl_sync(0xffffffffu, cur.tok, min(4 * max(q, 0) + j, cur.n - 1));
-                if (q >= 0 && q < nq)
-                    tma_gather4(odst + q * 4 * gc * 128, &m.x, s * gc * 64, t4[0], t4[1], t4[2], t4[3],
-                                &ctl->full[slot]);
+                    for (int j = 0; j < 4; ++j)
+                        t4[j] = __shfl_sync(0xffffffffu, cur.tok, min(4 * max(q, 0) + j, cur.n - 1));
+                    if (q >= 0 && q < nq)
+                        for (int hh = 0; hh < nhalf; ++hh)
+                            tma_gather4(odst + hh * (TN * a.xbox * 2) + q * 4 * a.xbox * 2, &m.x,
+                                        s * gc * 64 + hh * a.xbox, t4[0], t4[1], t4[2], t4[3], &ctl->full[slot]);
+                }
             } else {
                 if (lane == 0) tma_load_3d(wdst, &m.down, 0, cur.e * a.d + cur.row0, s * dc, &ctl->full[slot]);
                 if (s == 0) {
@@ -359,9 +392,12 @@ __device__ void producer(const ExpertArgs &a, const ExpertMaps &m, SharedCtl *ct
 }
 
 // ------------------------------------------------------------ consumers --
+// B operand rows: dense mode = token ids in a 128B-swizzled tile per 64
+// columns ([bpad][64] per chunk); otherwise the tile's gathered rows of
+// `xrow` bytes each.
 template <int NT>
-__device__ __forceinline__ void gu_stage(uint32_t wbase, uint32_t xbase, int xrow, int kvalid, int warp, int lane,
-                                         float (&acc_g)[4][4], float (&acc_u)[4][4]) {
+__device__ __forceinline__ void gu_stage(uint32_t wbase, uint32_t xbase, int xbox, int dense_tile, int kvalid, int warp,
+                                         int lane, float (&acc_g)[4][4], float (&acc_u)[4][4]) {
     const int nks = kvalid / 16;
 #pragma unroll
     for (int q = 0; q < (GU_CHUNKS * 4) / NCW; ++q) {
@@ -372,13 +408,17 @@ __device__ __forceinline__ void gu_stage(uint32_t wbase, uint32_t xbase, int xro
         const int r = lane & 15;
         uint32_t g0, g1, g2, g3, u0, u1, u2, u3;
         ldsm_x4(swz(wbase + box * (GU_ROWS * 128), r, chunk), g0, g1, g2, g3);
-        ldsm_x4(swz(wbase + 8192 + box * (GU_ROWS * 128), r, chunk), u0, u1, u2, u3);
+        ldsm_x4(swz(wbase + UP_OFF + box * (GU_ROWS * 128), r, chunk), u0, u1, u2, u3);
         const int xk = ks * 16 + ((lane >> 3) & 1) * 8;
+        const int xchunk = ((ks & 3) << 1) + ((lane >> 3) & 1);
 #pragma unroll
         for (int np = 0; np < (NT + 1) / 2; ++np) {
             const int n = np * 16 + (lane & 7) + ((lane >> 4) << 3);
             uint32_t b0, b1, b2, b3;
-            ldsm_x4(xbase + n * xrow + xk * 2, b0, b1, b2, b3);
+            // gather mode: x rows of xbox columns, one block of TN rows per xbox
+            ldsm_x4(dense_tile ? swz(xbase + box * dense_tile, n, xchunk)
+                               : xbase + (xk / xbox) * (TN * xbox * 2) + n * (xbox * 2) + (xk % xbox) * 2,
+                    b0, b1, b2, b3);
             mma_bf16(acc_g[2 * np], g0, g1, g2, g3, b0, b1);
             mma_bf16(acc_u[2 * np], u0, u1, u2, u3, b0, b1);
             if (2 * np + 1 < NT) {
@@ -419,7 +459,8 @@ __device__ __forceinline__ void stage_dispatch(const StageHdr &h, uint32_t wbase
                                                int warp, int lane, float (&acc_g)[4][4], float (&acc_u)[4][4]) {
     if (h.type == UNIT_GU) {
         const int gk = 64 * gu_chunks_of(a.d);
-        gu_stage<NT>(wbase, obase, gk * 2, min(gk, a.d - h.s * gk), warp, lane, acc_g, acc_u);
+        gu_stage<NT>(wbase, obase, a.xbox, a.dense ? a.bpad * 128 : 0, min(gk, a.d - h.s * gk), warp, lane, acc_g,
+                     acc_u);
     } else {
         const int dk = 64 * d_chunks_of(a.F);
         d_stage<NT>(wbase, obase, min(dk, a.F - h.s * dk), warp, lane, acc_g);
@@ -437,13 +478,16 @@ __device__ bool post_signal(SharedCtl *ctl, Counters *ctr, int q, int i) {
     return true;
 }
 
+template <class RG>
 __device__ void consumer(const ExpertArgs &a, SharedCtl *ctl, unsigned char *slots, float *part) {
+    constexpr int STAGES = RG::STAGES;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int ct = threadIdx.x;  // 0 .. NCW*32-1
     float acc_g[4][4], acc_u[4][4];
     int tk[4][2];
     float wk[4][2];
     int nsig = 0;  // completions posted (thread 0)
+    int gtok[2] = {0, 0};
     const int row = lane >> 2, col = (lane & 3) * 2;
     for (int g = 0;; ++g) {
         const int slot = g % STAGES;
@@ -458,6 +502,12 @@ __device__ void consumer(const ExpertArgs &a, SharedCtl *ctl, unsigned char *slo
             for (int j = 0; j < 4; ++j)
 #pragma unroll
                 for (int c = 0; c < 4; ++c) acc_g[j][c] = acc_u[j][c] = 0.0f;
+            if (h.type == UNIT_GU && a.dense) {
+                // epilogue elements ct and ct + NCW*32 read columns = token ids
+                const int n0 = ct >> 4, n1 = (ct + NCW * 32) >> 4;
+                gtok[0] = n0 < h.n ? __ldg(a.tok + h.p0 + n0) : 0;
+                gtok[1] = n1 < h.n ? __ldg(a.tok + h.p0 + n1) : 0;
+            }
             if (h.type == UNIT_D) {
                 // tokens and gate weights this thread combines; used at the
                 // unit's last stage, loaded now so the latency is hidden
@@ -472,9 +522,9 @@ __device__ void consumer(const ExpertArgs &a, SharedCtl *ctl, unsigned char *slo
                     }
             }
         }
-        const uint32_t wbase = smem_u32(slots + slot * SLOT_BYTES);
+        const uint32_t wbase = smem_u32(slots + slot * RG::SLOT_BYTES);
         const uint32_t obase = wbase + W_BYTES;
-        const int nt = (h.n + 7) >> 3;
+        const int nt = (h.type == UNIT_GU && a.dense) ? (a.bpad >> 3) : ((h.n + 7) >> 3);
         switch (nt) {
             case 1: stage_dispatch<1>(h, wbase, obase, a, warp, lane, acc_g, acc_u); break;
             case 2: stage_dispatch<2>(h, wbase, obase, a, warp, lane, acc_g, acc_u); break;
@@ -505,8 +555,8 @@ __device__ void consumer(const ExpertArgs &a, SharedCtl *ctl, unsigned char *slo
         } else {
             // reduce the eight warps' k-slices in a fixed order (warp w + 4
             // into warp w, then the four sums) and apply silu(g) * u
-            float *pg = part + ((warp & 3) * 2 + 0) * 16 * TN;
-            float *pu = part + ((warp & 3) * 2 + 1) * 16 * TN;
+            float *pg = part + ((warp & 3) * 2 + 0) * 16 * PART_LD;
+            float *pu = part + ((warp & 3) * 2 + 1) * 16 * PART_LD;
             if (warp >= 4) {
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
@@ -515,8 +565,8 @@ __device__ void consumer(const ExpertArgs &a, SharedCtl *ctl, unsigned char *slo
                     for (int c = 0; c < 4; ++c) {
                         const int r = row + ((c >> 1) << 3);
                         const int n = j * 8 + col + (c & 1);
-                        pg[r * TN + n] = acc_g[j][c];
-                        pu[r * TN + n] = acc_u[j][c];
+                        pg[r * PART_LD + n] = acc_g[j][c];
+                        pu[r * PART_LD + n] = acc_u[j][c];
                     }
                 }
             }
@@ -529,19 +579,21 @@ __device__ void consumer(const ExpertArgs &a, SharedCtl *ctl, unsigned char *slo
                     for (int c = 0; c < 4; ++c) {
                         const int r = row + ((c >> 1) << 3);
                         const int n = j * 8 + col + (c & 1);
-                        pg[r * TN + n] = acc_g[j][c] + pg[r * TN + n];
-                        pu[r * TN + n] = acc_u[j][c] + pu[r * TN + n];
+                        pg[r * PART_LD + n] = acc_g[j][c] + pg[r * PART_LD + n];
+                        pu[r * PART_LD + n] = acc_u[j][c] + pu[r * PART_LD + n];
                     }
                 }
             }
             consumer_bar();
-            for (int idx = ct; idx < 16 * h.n; idx += NCW * 32) {
+            for (int idx = ct, it = 0; idx < 16 * h.n; idx += NCW * 32, ++it) {
                 const int r = idx & 15, n = idx >> 4;
+                // accumulator column of pair n: its token (dense) or n
+                const int cn = a.dense ? (it == 0 ? gtok[0] : gtok[1]) : n;
                 float gs = 0.0f, us = 0.0f;
 #pragma unroll
                 for (int wv = 0; wv < NCW / 2; ++wv) {
-                    gs += part[(wv * 2 + 0) * 16 * TN + r * TN + n];
-                    us += part[(wv * 2 + 1) * 16 * TN + r * TN + n];
+                    gs += part[(wv * 2 + 0) * 16 * PART_LD + r * PART_LD + cn];
+                    us += part[(wv * 2 + 1) * 16 * PART_LD + r * PART_LD + cn];
                 }
                 const float hv = gs / (1.0f + __expf(-gs)) * us;
                 a.h[static_cast<size_t>(h.p0 + n) * a.F + h.row0 + r] =
@@ -572,13 +624,15 @@ __device__ void signaller(const ExpertArgs &a, SharedCtl *ctl) {
     }
 }
 
+template <class RG>
 __global__ void __launch_bounds__(NTHREADS, 1)
     expert_ffn_kernel(const __grid_constant__ ExpertMaps maps, const ExpertArgs a) {
+    constexpr int STAGES = RG::STAGES;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *base = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     unsigned char *slots = base;
-    float *part = reinterpret_cast<float *>(base + STAGES * SLOT_BYTES);
+    float *part = reinterpret_cast<float *>(base + STAGES * RG::SLOT_BYTES);
     SharedCtl *ctl = reinterpret_cast<SharedCtl *>(part + PART_FLOATS);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -636,11 +690,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     __syncthreads();
     if (warp == NCW) {
-        producer(a, maps, ctl, slots);
+        producer<RG>(a, maps, ctl, slots);
     } else if (warp == NCW + 1) {
         signaller(a, ctl);
     } else {
-        consumer(a, ctl, slots, part);
+        consumer<RG>(a, ctl, slots, part);
     }
 }
 
@@ -664,10 +718,16 @@ __global__ void __launch_bounds__(256) ffn_prep_kernel(const float *__restrict__
 }
 
 int g_num_sms[64] = {0};
+bool g_attr_small[64] = {false}, g_attr_large[64] = {false};
 
 }  // namespace
 
 int expert_ffn_h_rows() { return TN; }
+int expert_ffn_dense_batch(int B) { return B <= TN ? 1 : 0; }
+int expert_ffn_gather_cols(int d) {
+    const int w = 64 * expert_ffn_gu_chunks(d);
+    return w < GATHER_COLS ? w : GATHER_COLS;
+}
 int expert_ffn_gu_rows() { return GU_ROWS; }
 int expert_ffn_d_rows() { return D_ROWS; }
 int expert_ffn_gu_chunks(int d) { return d / 64 < GU_CHUNKS ? d / 64 : GU_CHUNKS; }
@@ -692,9 +752,17 @@ cudaError_t launch_expert_ffn(const ExpertMaps &maps, const uint16_t *xb, const 
         int n = 0;
         err = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
         if (err != cudaSuccess) return err;
-        err = cudaFuncSetAttribute(expert_ffn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-        if (err != cudaSuccess) return err;
         g_num_sms[dev] = n;
+    }
+    const bool small = d.B <= 16;
+    bool &configured = small ? g_attr_small[dev] : g_attr_large[dev];
+    if (!configured) {
+        err = small ? cudaFuncSetAttribute(expert_ffn_kernel<RingSmallB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           smem_bytes<RingSmallB>())
+                    : cudaFuncSetAttribute(expert_ffn_kernel<RingLargeB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           smem_bytes<RingLargeB>());
+        if (err != cudaSuccess) return err;
+        configured = true;
     }
     ExpertArgs a;
     a.xb = xb;
@@ -703,6 +771,9 @@ cudaError_t launch_expert_ffn(const ExpertMaps &maps, const uint16_t *xb, const 
     a.E = d.E;
     a.k = d.k;
     a.F = d.d_ff;
+    a.dense = d.B <= TN ? 1 : 0;
+    a.bpad = (d.B + 7) / 8 * 8;
+    a.xbox = expert_ffn_gather_cols(d.d);
     a.n_active = l.n_active;
     a.active = l.active;
     a.offsets = l.offsets;
@@ -714,14 +785,15 @@ cudaError_t launch_expert_ffn(const ExpertMaps &maps, const uint16_t *xb, const 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(g_num_sms[dev]);
     cfg.blockDim = dim3(NTHREADS);
-    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.dynamicSmemBytes = small ? smem_bytes<RingSmallB>() : smem_bytes<RingLargeB>();
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, expert_ffn_kernel, maps, a);
+    return small ? cudaLaunchKernelEx(&cfg, expert_ffn_kernel<RingSmallB>, maps, a)
+                 : cudaLaunchKernelEx(&cfg, expert_ffn_kernel<RingLargeB>, maps, a);
 }
 
 }  // namespace moe

@@ -67,6 +67,8 @@ cudaError_t launch_expert_ffn(const ExpertMaps &maps, const uint16_t *xb,
                               const moe_dims_t &d, const moe_lists_t &l, float *y,
                               uint16_t *h, Counters *ctr, bool pdl, cudaStream_t s);
 int expert_ffn_h_rows();              // rows of one H box (tokens per tile)
+int expert_ffn_dense_batch(int B);    // 1 if gate/up stages load all B token rows at once
+int expert_ffn_gather_cols(int d);    // columns of one x row box in gather mode
 int expert_ffn_gu_rows();             // rows of Wgate / Wup per gate-up unit
 int expert_ffn_d_rows();              // rows of Wdown per down unit
 int expert_ffn_gu_chunks(int d);      // 64-column chunks of d per gate-up stage

@@ -200,46 +200,56 @@ __global__ void __launch_bounds__(256) router_logits_kernel(
     int B, int d, int E, int tb, float *__restrict__ logits, uint16_t *__restrict__ xb,
     float *__restrict__ y_zero) {
     extern __shared__ float4 xs4[];  // [tb][d / 4]
-    if (xb != nullptr) {
-        // layer path: x -> bf16 copy for the expert kernel, y = 0
-        const int n4 = B * d / 4;
-        const int nthreads = gridDim.x * gridDim.y * blockDim.x;
-        for (int i = (blockIdx.y * gridDim.x + blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
-             i += nthreads) {
-            const float4 v = __ldg(reinterpret_cast<const float4 *>(x) + i);
-            const unsigned lo = static_cast<unsigned>(__bfloat16_as_ushort(__float2bfloat16_rn(v.x))) |
-                                (static_cast<unsigned>(__bfloat16_as_ushort(__float2bfloat16_rn(v.y))) << 16);
-            const unsigned hi = static_cast<unsigned>(__bfloat16_as_ushort(__float2bfloat16_rn(v.z))) |
-                                (static_cast<unsigned>(__bfloat16_as_ushort(__float2bfloat16_rn(v.w))) << 16);
-            reinterpret_cast<uint2 *>(xb)[i] = make_uint2(lo, hi);
-            if (y_zero) reinterpret_cast<float4 *>(y_zero)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-    }
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int e = blockIdx.x * 8 + warp;
     const int b0 = blockIdx.y * tb;
     const int nb = min(tb, B - b0);
-    const int d4 = d / 4;
+    const int nch = (d + 255) / 256;
+    const float *wrow = Wg + static_cast<size_t>(min(e, E - 1)) * d;
+    // first R_CH chunks of this warp's Wg row: issued before anything waits
+    float4 w[R_CH][2];
+#pragma unroll
+    for (int cc = 0; cc < R_CH; ++cc) {
+        const int j0 = 256 * cc + 8 * lane;
+        if (cc < nch && j0 < d) {
+            w[cc][0] = __ldg(reinterpret_cast<const float4 *>(wrow + j0));
+            w[cc][1] = __ldg(reinterpret_cast<const float4 *>(wrow + j0 + 4));
+        }
+    }
     {
-        const float4 *src = reinterpret_cast<const float4 *>(x) + static_cast<size_t>(b0) * d4;
-        for (int i = threadIdx.x; i < nb * d4; i += blockDim.x) xs4[i] = __ldg(src + i);
+        // stage the token rows: eight loads in flight per thread, then stores
+        const float4 *src = reinterpret_cast<const float4 *>(x) + static_cast<size_t>(b0) * (d / 4);
+        const int total4 = nb * (d / 4);
+#pragma unroll 1
+        for (int base = 0; base < total4; base += 8 * 256) {
+            float4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int i = base + u * 256 + static_cast<int>(threadIdx.x);
+                if (i < total4) v[u] = __ldg(src + i);
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int i = base + u * 256 + static_cast<int>(threadIdx.x);
+                if (i < total4) xs4[i] = v[u];
+            }
+        }
     }
     __syncthreads();
     if (e < E) {
         float acc[R_TB];
 #pragma unroll
         for (int t = 0; t < R_TB; ++t) acc[t] = 0.0f;
-        const float *wrow = Wg + static_cast<size_t>(e) * d;
-        const int nch = (d + 255) / 256;
 #pragma unroll 1
         for (int c0 = 0; c0 < nch; c0 += R_CH) {
-            float4 w[R_CH][2];
+            if (c0 > 0) {
 #pragma unroll
-            for (int cc = 0; cc < R_CH; ++cc) {
-                const int j0 = 256 * (c0 + cc) + 8 * lane;
-                if (c0 + cc < nch && j0 < d) {
-                    w[cc][0] = __ldg(reinterpret_cast<const float4 *>(wrow + j0));
-                    w[cc][1] = __ldg(reinterpret_cast<const float4 *>(wrow + j0 + 4));
+                for (int cc = 0; cc < R_CH; ++cc) {
+                    const int j0 = 256 * (c0 + cc) + 8 * lane;
+                    if (c0 + cc < nch && j0 < d) {
+                        w[cc][0] = __ldg(reinterpret_cast<const float4 *>(wrow + j0));
+                        w[cc][1] = __ldg(reinterpret_cast<const float4 *>(wrow + j0 + 4));
+                    }
                 }
             }
 #pragma unroll
@@ -274,6 +284,21 @@ __global__ void __launch_bounds__(256) router_logits_kernel(
         if (lane < nb) {
             const float v = bias ? __fadd_rn(mine, __ldg(bias + e)) : mine;
             logits[static_cast<size_t>(b0 + lane) * E + e] = v;
+        }
+    }
+    if (xb != nullptr) {
+        // layer path: x -> bf16 copy for the expert kernel, y = 0
+        const int n4 = B * d / 4;
+        const int nthreads = gridDim.x * gridDim.y * blockDim.x;
+        for (int i = (blockIdx.y * gridDim.x + blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+             i += nthreads) {
+            const float4 v = __ldg(reinterpret_cast<const float4 *>(x) + i);
+            const unsigned lo = static_cast<unsigned>(__bfloat16_as_ushort(__float2bfloat16_rn(v.x))) |
+                                (static_cast<unsigned>(__bfloat16_as_ushort(__float2bfloat16_rn(v.y))) << 16);
+            const unsigned hi = static_cast<unsigned>(__bfloat16_as_ushort(__float2bfloat16_rn(v.z))) |
+                                (static_cast<unsigned>(__bfloat16_as_ushort(__float2bfloat16_rn(v.w))) << 16);
+            reinterpret_cast<uint2 *>(xb)[i] = make_uint2(lo, hi);
+            if (y_zero) reinterpret_cast<float4 *>(y_zero)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
     }
     // let the dependent (re-selection) kernel become resident; it waits for
@@ -315,6 +340,7 @@ struct ReselectArgs {
     const float *logits;
     float *probs;  // read, or written when fuse_softmax
     int fuse_softmax;
+    int cache_rows;  // logits / probabilities kept in shared memory
     int B, E, k, mode, k0, budget;
     int32_t *sel_idx;
     float *sel_w;
@@ -351,6 +377,74 @@ __device__ int block_scan256(int v, int *wsum, int *total) {
     return res;
 }
 
+// Order-preserving unsigned image of a logit (larger logit -> larger value,
+// -0 and +0 equal); never 0 for a finite or infinite float.
+__device__ __forceinline__ unsigned ord_of(float v) {
+    v = (v == 0.0f) ? 0.0f : v;
+    const unsigned u = __float_as_uint(v);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float float_of_ord(unsigned o) {
+    return __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
+}
+
+// One round of warp arg-max over candidate bits with two hardware warp
+// reductions: the largest logit image, then, among lanes holding it, the
+// lowest expert index.  The winner leaves the candidates.  -1 if none.
+template <int NI>
+__device__ __forceinline__ int warp_argmax(const unsigned (&ord)[NI], unsigned &cand, int lane) {
+    unsigned bo = 0u, bl = 0u;  // this lane's best: logit image, ~index
+#pragma unroll
+    for (int i = 0; i < NI; ++i) {
+        if ((cand >> i) & 1u) {
+            const unsigned lo = ~static_cast<unsigned>(lane + 32 * i);
+            if (ord[i] > bo || (ord[i] == bo && lo > bl)) {
+                bo = ord[i];
+                bl = lo;
+            }
+        }
+    }
+    const unsigned H = __reduce_max_sync(FULL, bo);
+    if (H == 0u) return -1;
+    const unsigned Lw = __reduce_max_sync(FULL, bo == H ? bl : 0u);
+    const int idx = static_cast<int>(~Lw);
+    if ((idx & 31) == lane) cand &= ~(1u << (idx >> 5));
+    return idx;
+}
+
+// Softmax of one token (row lane-distributed: e = lane + 32 i), max by
+// warp reduction of logit images, sum in the canonical lane/butterfly order.
+template <int NI>
+__device__ __forceinline__ void token_softmax_r(const float (&l)[NI], const unsigned (&ord)[NI], int E, int lane,
+                                                float (&p)[NI]) {
+    unsigned om = 0u;
+#pragma unroll
+    for (int i = 0; i < NI; ++i)
+        if (lane + 32 * i < E) om = ord[i] > om ? ord[i] : om;
+    const float m = float_of_ord(__reduce_max_sync(FULL, om));
+    float q[NI];
+    float acc = 0.0f;
+#pragma unroll
+    for (int i = 0; i < NI; ++i) {
+        if (lane + 32 * i < E) {
+            q[i] = exp_own(__fsub_rn(l[i], m));
+            acc = __fadd_rn(acc, q[i]);
+        } else {
+            q[i] = 0.0f;
+        }
+    }
+    const float Z = warp_butterfly_sum(acc);
+#pragma unroll
+    for (int i = 0; i < NI; ++i) p[i] = (lane + 32 * i < E) ? __fdiv_rn(q[i], Z) : 0.0f;
+}
+
+// Records slot j of one token: every lane adds the winner's probability to
+// the running sum (slot order, from +0); lane j keeps it for its weight.
+__device__ __forceinline__ void take_slot(int j, float pe, int lane, float &sum, float &myp) {
+    sum = __fadd_rn(sum, pe);
+    if (lane == j) myp = pe;
+}
+
 template <int NI>
 __global__ void __launch_bounds__(1024, 1) reselect_kernel(ReselectArgs a) {
     // wait until the router's logits are complete and visible
@@ -361,11 +455,11 @@ __global__ void __launch_bounds__(1024, 1) reselect_kernel(ReselectArgs a) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const int B = a.B, E = a.E, k = a.k;
     const int BW = (B + 31) >> 5;
-    int *T = reinterpret_cast<int *>(smem_raw);                      // [B][k] first ranks
-    int *SEL = T + B * k;                                              // [B][k] chosen experts
-    float *SELW = reinterpret_cast<float *>(SEL + B * k);             // [B][k] p, then weights
-    unsigned *ASSIGN = reinterpret_cast<unsigned *>(SELW + B * k);    // [E][BW]
-    unsigned *TMEMB = ASSIGN + E * BW;                                  // [E][BW]
+    int *T = reinterpret_cast<int *>(smem_raw);                    // [B][k] first ranks
+    unsigned *ASSIGN = reinterpret_cast<unsigned *>(T + B * k);     // [E][BW] final assignment
+    unsigned *TMEMB = ASSIGN + E * BW;                                // [E][BW] top-k membership
+    float *PC = reinterpret_cast<float *>(TMEMB + E * BW);           // [B][E] probability cache
+    float *LC = PC + (a.cache_rows ? B * E : 0);                      // [B][E] logit cache
     __shared__ float s_score[E_MAX];
     __shared__ int s_off[E_MAX];
     __shared__ unsigned ukept[E_MAX / 32], ubase[E_MAX / 32], sbits[E_MAX / 32];
@@ -377,37 +471,56 @@ __global__ void __launch_bounds__(1024, 1) reselect_kernel(ReselectArgs a) {
     __syncthreads();
 
     const int mode = a.mode;
-    // ---- phase 1: per token softmax (layer path) + first ranks
+    float *prob_rows = a.cache_rows ? PC : a.probs;
+    const float *logit_rows = a.cache_rows ? LC : a.logits;
+
+    // ---- phase 1: softmax (layer path) and each token's first ranks
     const int r1 = (mode == MOE_RESELECT_OEA) ? a.k0 : k;
 #pragma unroll 1
     for (int b = warp; b < B; b += 32) {
         float l[NI], p[NI];
+        unsigned ord[NI];
         load_row<NI>(a.logits + static_cast<size_t>(b) * E, E, lane, l);
-        if (a.fuse_softmax) {
-            token_softmax<NI>(l, E, lane, p);
 #pragma unroll
-            for (int i = 0; i < NI; ++i)
-                if (lane + 32 * i < E) a.probs[static_cast<size_t>(b) * E + lane + 32 * i] = p[i];
+        for (int i = 0; i < NI; ++i) ord[i] = ord_of(l[i]);
+        if (a.fuse_softmax) {
+            token_softmax_r<NI>(l, ord, E, lane, p);
         } else {
             load_row<NI>(a.probs + static_cast<size_t>(b) * E, E, lane, p);
         }
-        unsigned long long key[NI];
 #pragma unroll
-        for (int i = 0; i < NI; ++i) key[i] = rank_key(l[i], lane + 32 * i);
-        unsigned cand = valid_bits<NI>(E, lane);
-        warp_select<NI>(key, cand, p, r1, lane, T + b * k, mode == MOE_RESELECT_NONE ? SELW + b * k : nullptr);
-        if (lane < r1) {
-            const int e = T[b * k + lane];
-            if (mode == MOE_RESELECT_OEA) atomicOr(&ukept[e >> 5], 1u << (e & 31));
-            if (mode == MOE_RESELECT_XSHARE) {
-                atomicOr(&ubase[e >> 5], 1u << (e & 31));
-                atomicOr(&TMEMB[e * BW + (b >> 5)], 1u << (b & 31));
+        for (int i = 0; i < NI; ++i) {
+            const int e = lane + 32 * i;
+            if (e < E) {
+                if (a.cache_rows) {
+                    LC[b * E + e] = l[i];
+                    PC[b * E + e] = p[i];
+                } else if (a.fuse_softmax) {
+                    a.probs[static_cast<size_t>(b) * E + e] = p[i];
+                }
             }
-            if (mode == MOE_RESELECT_NONE) SEL[b * k + lane] = e;
         }
-        if (mode == MOE_RESELECT_NONE) {
-            __syncwarp();
-            renormalise_slots(SEL + b * k, SELW + b * k, k, lane);
+        unsigned cand = valid_bits<NI>(E, lane);
+        float sum = 0.0f, myp = 0.0f;
+        int mye = -1;
+#pragma unroll 1
+        for (int j = 0; j < r1; ++j) {
+            const int e = warp_argmax<NI>(ord, cand, lane);
+            if (lane == j) mye = e;
+            if (mode == MOE_RESELECT_NONE) take_slot(j, warp_fetch<NI>(p, e), lane, sum, myp);
+        }
+        if (lane < r1) {
+            T[b * k + lane] = mye;
+            if (mode == MOE_RESELECT_OEA) atomicOr(&ukept[mye >> 5], 1u << (mye & 31));
+            if (mode == MOE_RESELECT_XSHARE) {
+                atomicOr(&ubase[mye >> 5], 1u << (mye & 31));
+                atomicOr(&TMEMB[mye * BW + (b >> 5)], 1u << (b & 31));
+            }
+        }
+        if (mode == MOE_RESELECT_NONE && lane < k) {
+            a.sel_idx[static_cast<size_t>(b) * k + lane] = mye;
+            a.sel_w[static_cast<size_t>(b) * k + lane] = __fdiv_rn(myp, sum);
+            atomicOr(&ASSIGN[mye * BW + (b >> 5)], 1u << (b & 31));
         }
     }
     __syncthreads();
@@ -415,12 +528,12 @@ __global__ void __launch_bounds__(1024, 1) reselect_kernel(ReselectArgs a) {
     // ---- XShare: batch scores, budget, greedy set (= top-M' by score)
     if (mode == MOE_RESELECT_XSHARE) {
         if (tid < E) {
-            float s = 0.0f;
+            float sc = 0.0f;
 #pragma unroll 1
             for (int b = 0; b < B; ++b)
                 if ((TMEMB[tid * BW + (b >> 5)] >> (b & 31)) & 1u)
-                    s = __fadd_rn(s, a.probs[static_cast<size_t>(b) * E + tid]);
-            s_score[tid] = s;
+                    sc = __fadd_rn(sc, prob_rows[static_cast<size_t>(b) * E + tid]);
+            s_score[tid] = sc;
         }
         __syncthreads();
         if (tid < E && ((ubase[tid >> 5] >> (tid & 31)) & 1u)) {
@@ -445,11 +558,11 @@ __global__ void __launch_bounds__(1024, 1) reselect_kernel(ReselectArgs a) {
 #pragma unroll 1
         for (int b = warp; b < B; b += 32) {
             float l[NI], p[NI];
-            load_row<NI>(a.logits + static_cast<size_t>(b) * E, E, lane, l);
-            load_row<NI>(a.probs + static_cast<size_t>(b) * E, E, lane, p);
-            unsigned long long key[NI];
+            unsigned ord[NI];
+            load_row<NI>(logit_rows + static_cast<size_t>(b) * E, E, lane, l);
+            load_row<NI>(prob_rows + static_cast<size_t>(b) * E, E, lane, p);
 #pragma unroll
-            for (int i = 0; i < NI; ++i) key[i] = rank_key(l[i], lane + 32 * i);
+            for (int i = 0; i < NI; ++i) ord[i] = ord_of(l[i]);
             unsigned cand = 0;
             const unsigned *bits = (mode == MOE_RESELECT_OEA) ? ukept : sbits;
 #pragma unroll
@@ -457,50 +570,46 @@ __global__ void __launch_bounds__(1024, 1) reselect_kernel(ReselectArgs a) {
                 const int e = lane + 32 * i;
                 if (e < E && ((bits[e >> 5] >> (e & 31)) & 1u)) cand |= 1u << i;
             }
+            float sum = 0.0f, myp = 0.0f;
+            int mye = -1;
             const int kk = (mode == MOE_RESELECT_OEA) ? a.k0 : 0;
 #pragma unroll 1
             for (int j = 0; j < kk; ++j) {  // kept experts first, in rank order
                 const int e = T[b * k + j];
                 if ((e & 31) == lane) cand &= ~(1u << (e >> 5));
-                const float pe = warp_fetch<NI>(p, e);
-                if (lane == 0) {
-                    SEL[b * k + j] = e;
-                    SELW[b * k + j] = pe;
-                }
+                if (lane == j) mye = e;
+                take_slot(j, warp_fetch<NI>(p, e), lane, sum, myp);
             }
-            __syncwarp();
-            const int nf = warp_select<NI>(key, cand, p, k - kk, lane, SEL + b * k + kk, SELW + b * k + kk);
-            if (lane >= kk + nf && lane < k) {
-                SEL[b * k + lane] = -1;
-                SELW[b * k + lane] = 0.0f;
+#pragma unroll 1
+            for (int j = kk; j < k; ++j) {
+                const int e = warp_argmax<NI>(ord, cand, lane);
+                if (e < 0) break;
+                if (lane == j) mye = e;
+                take_slot(j, warp_fetch<NI>(p, e), lane, sum, myp);
             }
-            __syncwarp();
-            renormalise_slots(SEL + b * k, SELW + b * k, k, lane);
+            if (lane < k) {
+                a.sel_idx[static_cast<size_t>(b) * k + lane] = mye;
+                a.sel_w[static_cast<size_t>(b) * k + lane] = mye >= 0 ? __fdiv_rn(myp, sum) : 0.0f;
+                if (mye >= 0) atomicOr(&ASSIGN[mye * BW + (b >> 5)], 1u << (b & 31));
+            }
         }
-        __syncthreads();
-    }
-
-    // ---- phase 3: assignment bits, counts, active list, offsets
-    for (int i = tid; i < B * k; i += blockDim.x) {
-        const int e = SEL[i];
-        const int b = i / k;
-        if (e >= 0) atomicOr(&ASSIGN[e * BW + (b >> 5)], 1u << (b & 31));
-        a.sel_idx[i] = e;
-        a.sel_w[i] = SELW[i];
     }
     __syncthreads();
+
+    // ---- phase 3: counts, active list, offsets (one scan of flag and count)
     int cnt = 0;
     if (tid < E)
         for (int wd = 0; wd < BW; ++wd) cnt += __popc(ASSIGN[tid * BW + wd]);
-    int n_active = 0, total = 0;
     const int flag = (tid < E && cnt > 0) ? 1 : 0;
-    const int rank_incl = block_scan256(flag, wsum, &n_active);
-    const int off_incl = block_scan256(tid < E ? cnt : 0, wsum, &total);
+    int tot = 0;
+    const int incl = block_scan256((flag << 16) | cnt, wsum, &tot);
+    const int n_active = tot >> 16, total = tot & 0xffff;
     if (tid < E) {
-        s_off[tid] = off_incl - cnt;
+        const int off = (incl & 0xffff) - cnt;
+        s_off[tid] = off;
         if (flag) {
-            a.lists.active[rank_incl - 1] = tid;
-            a.lists.offsets[rank_incl - 1] = off_incl - cnt;
+            a.lists.active[(incl >> 16) - 1] = tid;
+            a.lists.offsets[(incl >> 16) - 1] = off;
         }
     }
     if (tid >= n_active && tid < E) a.lists.active[tid] = -1;
@@ -513,15 +622,15 @@ __global__ void __launch_bounds__(1024, 1) reselect_kernel(ReselectArgs a) {
 
     // ---- phase 4: compaction (expert ascending, token ascending)
     for (int i = tid; i < B * k; i += blockDim.x) {
-        const int e = SEL[i];
-        if (e < 0) continue;
         const int b = i / k;
+        const int e = a.sel_idx[i];
+        if (e < 0) continue;
         int before = 0;
         for (int wd = 0; wd < (b >> 5); ++wd) before += __popc(ASSIGN[e * BW + wd]);
         before += __popc(ASSIGN[e * BW + (b >> 5)] & ((1u << (b & 31)) - 1u));
         const int pos = s_off[e] + before;
         a.lists.tok[pos] = b;
-        a.lists.w[pos] = SELW[i];
+        a.lists.w[pos] = a.sel_w[i];
     }
     for (int i = total + tid; i < B * k; i += blockDim.x) {
         a.lists.tok[i] = -1;
@@ -612,7 +721,10 @@ cudaError_t launch_reselect(const float *logits, float *probs, bool fuse_softmax
     a.n_active_copy = n_active_copy;
     a.ctr = ctr;
     const int BW = (d.B + 31) / 32;
-    const size_t smem = static_cast<size_t>(d.B) * d.k * 12 + static_cast<size_t>(d.E) * BW * 8;
+    const size_t base = static_cast<size_t>(d.B) * d.k * 4 + static_cast<size_t>(d.E) * BW * 8;
+    const size_t rows = static_cast<size_t>(d.B) * d.E * 8;
+    a.cache_rows = (base + rows <= 96u * 1024u) ? 1 : 0;
+    const size_t smem = base + (a.cache_rows ? rows : 0);
     switch (ni_for(d.E)) {
         case 1: return launch_reselect_ni<1>(a, smem, pdl, s);
         case 2: return launch_reselect_ni<2>(a, smem, pdl, s);
