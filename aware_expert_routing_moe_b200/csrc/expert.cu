@@ -262,11 +262,13 @@ __device__ __forceinline__ bool decode_unit(int u, int n_units, const ExpertArgs
     ui.p0 = ctl->off[i] + tt * TN;
     ui.n = min(TN, ctl->off[i + 1] - ui.p0);
     ui.need = nt_i * gu_per_tile;
-    // both loads are unconditional (valid addresses) so that nothing waits
-    // for them here; their values are first used when the unit's first stage
-    // is issued
-    ui.tok = __ldg(a.tok + ui.p0 + min(lane, ui.n - 1));
-    ui.dep = ld_relaxed(&a.ctr->gu_done[i]);
+    // prefetches, first used when the unit's first stage is issued: the token
+    // rows a gathered gate/up stage loads, and (acquire) how many gate/up
+    // units of this expert are already published
+    ui.tok = 0;
+    ui.dep = 0;
+    if (ui.type == UNIT_GU && !a.dense) ui.tok = __ldg(a.tok + ui.p0 + min(lane, ui.n - 1));
+    if (ui.type == UNIT_D && lane == 0) ui.dep = ld_acquire(&a.ctr->gu_done[i]);
     return true;
 }
 
@@ -275,11 +277,13 @@ __device__ void producer(const ExpertArgs &a, const ExpertMaps &m, SharedCtl *ct
     constexpr int STAGES = RG::STAGES;
     const int lane = threadIdx.x & 31;
     const int n_units = ctl->total_tiles * (a.F / GU_ROWS + a.d / D_ROWS);
-    int req = 0;
-    if (lane == 0) req = atomicAdd(&a.ctr->ticket, 1);
+    // units are dealt round robin: CTA c takes c, c + grid, c + 2 grid, ...
+    // (all CTAs start together when the lists are ready; every gate/up unit
+    // precedes every down unit in each CTA's sequence)
+    int next_u = blockIdx.x;
     UnitInfo cur;
-    bool have = decode_unit(__shfl_sync(0xffffffffu, req, 0), n_units, a, ctl, lane, cur);
-    if (have && lane == 0) req = atomicAdd(&a.ctr->ticket, 1);
+    bool have = decode_unit(next_u, n_units, a, ctl, lane, cur);
+    next_u += gridDim.x;
     int g = 0;  // stages issued
     bool ok = true;
     while (have && ok) {
@@ -339,6 +343,8 @@ __device__ void producer(const ExpertArgs &a, const ExpertMaps &m, SharedCtl *ct
                 if (s == 0) {
                     // this expert's gate/up units must be complete before H is read
                     if (lane == 0) {
+                        // the prefetched count was read with acquire semantics;
+                        // if it is short, poll (acquire) until complete
                         int v = cur.dep;
                         if (v < cur.need) {
                             const unsigned long long t0 = global_ns();
@@ -351,9 +357,8 @@ __device__ void producer(const ExpertArgs &a, const ExpertMaps &m, SharedCtl *ct
                                 }
                                 __nanosleep(64);
                             }
-                        } else {
-                            asm volatile("fence.acq_rel.gpu;" ::: "memory");
                         }
+                        // H was written through the generic proxy; it is read by TMA
                         asm volatile("fence.proxy.async.global;" ::: "memory");
                     }
                     ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -363,8 +368,8 @@ __device__ void producer(const ExpertArgs &a, const ExpertMaps &m, SharedCtl *ct
             ++g;
             if (!ok) break;
             if (s == 0) {
-                have_nxt = decode_unit(__shfl_sync(0xffffffffu, req, 0), n_units, a, ctl, lane, nxt);
-                if (have_nxt && lane == 0) req = atomicAdd(&a.ctr->ticket, 1);
+                have_nxt = decode_unit(next_u, n_units, a, ctl, lane, nxt);
+                next_u += gridDim.x;
             }
         }
         cur = nxt;
