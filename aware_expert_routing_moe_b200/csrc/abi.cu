@@ -134,6 +134,21 @@ bool encode_bf16_rows(CUtensorMap *map, const void *ptr, uint64_t rows, uint64_t
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// fp32 matrix [rows][cols] (cols % 32 == 0) seen as rows * cols / 32
+// lines of 32 floats; boxes of box_lines whole lines, 128-byte swizzle.
+// Lines past the end read as zero.
+bool encode_f32_lines(CUtensorMap *map, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box_lines) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t gdim[2] = {32, rows * (cols / 32)};
+    cuuint64_t gstride[1] = {128};
+    cuuint32_t box[2] = {32, box_lines};
+    cuuint32_t estride[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(ptr), gdim, gstride, box, estride,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <typename T>
 T *seg(void *ws, size_t off) {
     return reinterpret_cast<T *>(static_cast<unsigned char *>(ws) + off);
@@ -159,16 +174,26 @@ bool encode_expert_maps(ExpertMaps *m, const moe_dims_t &d, const uint16_t *Wgat
     return encode_bf16_chunked(&m->gate, Wgate, E * F, D, expert_ffn_gu_rows(), gu_chunks) &&
            encode_bf16_chunked(&m->up, Wup, E * F, D, expert_ffn_gu_rows(), gu_chunks) &&
            encode_bf16_chunked(&m->down, Wdown, E * D, F, expert_ffn_d_rows(), d_chunks) &&
-           encode_bf16_chunked(&m->h, h, static_cast<uint64_t>(d.B) * d.k, F, expert_ffn_h_rows(), d_chunks) &&
+           encode_bf16_chunked(&m->h, h,
+                               expert_ffn_dense_batch(d.B) ? static_cast<uint64_t>(active_slots(d)) * d.B
+                                                           : static_cast<uint64_t>(d.B) * d.k,
+                               F, expert_ffn_h_rows(d.B), d_chunks) &&
            (expert_ffn_dense_batch(d.B)
                 ? encode_bf16_chunked(&m->x, xb, static_cast<uint64_t>(d.B), D, (d.B + 7) / 8 * 8, gu_chunks)
                 : encode_bf16_rows(&m->x, xb, static_cast<uint64_t>(d.B), D, expert_ffn_gather_cols(d.d)));
 }
 
+bool encode_router_maps(RouterMaps *m, const moe_dims_t &d, const float *x, const float *Wg) {
+    std::memset(m, 0, sizeof(*m));
+    const uint32_t bl = static_cast<uint32_t>(router_box_lines(d.d));
+    return encode_f32_lines(&m->x, x, static_cast<uint64_t>(d.B), static_cast<uint64_t>(d.d), bl) &&
+           encode_f32_lines(&m->wg, Wg, static_cast<uint64_t>(d.E), static_cast<uint64_t>(d.d), bl);
+}
+
 WsLayout ws_layout(const moe_dims_t &d) {
     WsLayout L;
     size_t o = 0;
-    const size_t B = d.B, E = d.E, k = d.k, D = d.d, F = d.d_ff;
+    const size_t B = d.B, E = d.E, k = d.k, D = d.d;
     L.counters = o; o += round_up(sizeof(Counters));
     L.logits = o;   o += round_up(B * E * 4);
     L.probs = o;    o += round_up(B * E * 4);
@@ -180,7 +205,8 @@ WsLayout ws_layout(const moe_dims_t &d) {
     L.tok = o;      o += round_up(B * k * 4);
     L.w = o;        o += round_up(B * k * 4);
     L.xb = o;       o += round_up(B * D * 2);
-    L.h = o;        o += round_up(B * k * F * 2);
+    L.h = o;        o += round_up(h_scratch_bytes(d));
+    L.wd = o;       o += round_up(wd_bytes(d));
     L.total = o;
     return L;
 }
@@ -219,7 +245,9 @@ moe_status_t moe_route(const float *x, const float *Wg, const float *bias, moe_d
     moe_status_t st = check_device();
     if (st != MOE_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    st = from_cuda(launch_router_logits(x, Wg, bias, dims, logits, nullptr, nullptr, s));
+    RouterMaps rmaps;
+    if (!encode_router_maps(&rmaps, dims, x, Wg)) return MOE_ERR_CUDA;
+    st = from_cuda(launch_router_logits(rmaps, bias, dims, logits, s));
     if (st != MOE_OK) return st;
     return from_cuda(launch_route_topk(logits, dims, probs, topk_idx, topk_w, s));
 }
@@ -233,8 +261,8 @@ moe_status_t moe_reselect(const float *logits, const float *probs, moe_dims_t di
     if (!al16(logits) || !al16(probs) || !al16(sel_idx) || !al16(sel_w)) return MOE_ERR_MISALIGNED;
     st = check_device();
     if (st != MOE_OK) return st;
-    return from_cuda(launch_reselect(logits, const_cast<float *>(probs), false, dims, rule, sel_idx, sel_w, lists,
-                                     nullptr, nullptr, false, static_cast<cudaStream_t>(stream)));
+    return from_cuda(launch_reselect(logits, probs, dims, rule, sel_idx, sel_w, lists,
+                                     static_cast<cudaStream_t>(stream)));
 }
 
 moe_status_t moe_expert_ffn(const float *x, const uint16_t *Wgate, const uint16_t *Wup, const uint16_t *Wdown,
@@ -256,9 +284,10 @@ moe_status_t moe_expert_ffn(const float *x, const uint16_t *Wgate, const uint16_
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     Counters *ctr = seg<Counters>(ws, L.counters);
     uint16_t *xb = seg<uint16_t>(ws, L.xb);
-    st = from_cuda(launch_ffn_prep(x, dims, xb, y, ctr, s));
+    float *wd = expert_ffn_dense_batch(dims.B) ? seg<float>(ws, L.wd) : nullptr;
+    st = from_cuda(launch_ffn_prep(x, dims, xb, y, ctr, lists, wd, s));
     if (st != MOE_OK) return st;
-    return from_cuda(launch_expert_ffn(maps, xb, dims, lists, y, seg<uint16_t>(ws, L.h), ctr, true, s));
+    return from_cuda(launch_expert_ffn(maps, xb, dims, lists, y, seg<uint16_t>(ws, L.h), wd, ctr, false, 0, s));
 }
 
 moe_status_t moe_layer_decode(const float *x, const float *Wg, const float *bias, const uint16_t *Wgate,
@@ -278,6 +307,8 @@ moe_status_t moe_layer_decode(const float *x, const float *Wg, const float *bias
     ExpertMaps maps;
     if (!encode_expert_maps(&maps, dims, Wgate, Wup, Wdown, seg<uint16_t>(ws, L.h), seg<uint16_t>(ws, L.xb)))
         return MOE_ERR_CUDA;
+    RouterMaps rmaps;
+    if (!encode_router_maps(&rmaps, dims, x, Wg)) return MOE_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     Counters *ctr = seg<Counters>(ws, L.counters);
     uint16_t *xb = seg<uint16_t>(ws, L.xb);
@@ -286,11 +317,17 @@ moe_status_t moe_layer_decode(const float *x, const float *Wg, const float *bias
     int32_t *si = sel_idx ? sel_idx : seg<int32_t>(ws, L.sel_idx);
     float *sw = sel_w ? sel_w : seg<float>(ws, L.sel_w);
     const moe_lists_t lists = ws_lists(ws, L);
-    st = from_cuda(launch_router_logits(x, Wg, bias, dims, logits, xb, y, s));
+    // B <= 32: the expert kernel starts streaming as soon as the activated
+    // set is published (by the router for OEA and plain top-k, by the
+    // selection for XShare); larger batches start when the selection ends
+    const bool dense = expert_ffn_dense_batch(dims.B) != 0;
+    float *wd = dense ? seg<float>(ws, L.wd) : nullptr;
+    st = from_cuda(launch_layer_route(rmaps, x, bias, dims, rule, logits, xb, y, ctr, s));
     if (st != MOE_OK) return st;
-    st = from_cuda(launch_reselect(logits, probs, true, dims, rule, si, sw, lists, n_active, ctr, true, s));
+    st = from_cuda(launch_layer_select(logits, probs, dims, rule, si, sw, lists, n_active, ctr, wd, dense, s));
     if (st != MOE_OK) return st;
-    return from_cuda(launch_expert_ffn(maps, xb, dims, lists, y, seg<uint16_t>(ws, L.h), ctr, true, s));
+    return from_cuda(launch_expert_ffn(maps, xb, dims, lists, y, seg<uint16_t>(ws, L.h), wd, ctr, dense,
+                                       layer_pub_target(dims, rule), s));
 }
 
 moe_status_t moe_check_error(void *ws, size_t ws_bytes, void *stream) {

@@ -7,23 +7,32 @@
 // Expert Activation: Batch-Aware Expert Routing for Faster Decode Without
 // Retraining", abstract).
 //
-// Work units, handed out by an atomic ticket to persistent CTAs (one per SM):
+// Work units, dealt round robin to persistent CTAs (one per SM):
 //   GU unit (expert e, token tile, 16-row block of d_ff):
 //       g = Wgate[e][rows] x_t, u = Wup[e][rows] x_t over all of d,
-//       h = silu(g) * u -> H scratch (bf16, [pair][d_ff]);
+//       h = silu(g) * u -> H scratch (bf16);
 //   D unit (expert e, token tile, 64-row block of d):
 //       y[t][rows] += w_t * Wdown[e][rows] h_t over all of d_ff.
-// All GU units come before all D units in ticket order; a D unit's producer
-// waits (bounded) until its expert's GU units are counted done.
+// Every CTA takes all its GU units before its D units; a D unit's producer
+// waits (bounded) until its expert's GU units are published done.
 //
-// Per CTA: one producer warp issues TMA tensor copies (128B-swizzled weight
-// boxes, H boxes) and bulk copies (token rows of x) into a ring of stages,
-// each guarded by a full/empty mbarrier pair; four consumer warps run
-// mma.sync m16n8k16 bf16 tiles with the weights as the 16-row A operand and
-// up to 32 tokens as the B operand (tokens padded to 8-column tiles), fp32
-// accumulation.  Every wait is bounded by a time limit; on expiry the CTA
-// records an error code in the workspace, drains its in-flight copies and
-// returns.
+// Dense mode (B <= 32): every unit works on all B tokens of the batch, so
+// gate/up stages load x for all tokens in one swizzled box, H is indexed by
+// (active slot, token), and the down epilogue weighs each token by a dense
+// [slot][B] weight matrix (0 for tokens that did not choose the expert).
+// Gate/up work then needs only the activated set, which the layer path's
+// selection publishes before it finishes the token lists: the kernel is
+// launched early and starts streaming on that signal.  Larger batches use
+// token tiles of up to 32 pairs, x rows gathered by four, and pair-indexed H.
+//
+// Per CTA: one producer warp issues TMA tensor copies (three-dimensional
+// boxes of 64-column chunks, 128-byte swizzle) into a ring of 32 KB weight
+// stages plus operand tiles, each guarded by a full/empty mbarrier pair;
+// eight consumer warps split every stage's k-steps and run mma.sync
+// m16n8k16 bf16 tiles (16 weight rows as A, tokens as B, fp32 accumulation);
+// a signal warp publishes gate/up completions.  Every wait is bounded by a
+// time limit; on expiry the CTA records an error code in the workspace,
+// drains its in-flight copies and returns.
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -53,9 +62,10 @@ struct Ring {
 };
 constexpr int PART_LD = TN + 1;                        // padded row of the epilogue buffer
 constexpr int PART_FLOATS = (NCW / 2) * 2 * 16 * PART_LD;  // GU partial sums for the epilogue
+constexpr int CTL_BYTES = 6144;  // reserved for SharedCtl (checked below)
 template <class RG>
 constexpr int smem_bytes() {
-    return 1024 /*align slack*/ + RG::STAGES * RG::SLOT_BYTES + PART_FLOATS * 4 + 4096;
+    return 1024 /*align slack*/ + RG::STAGES * RG::SLOT_BYTES + PART_FLOATS * 4 + CTL_BYTES;
 }
 using RingSmallB = Ring<4, 16384>;
 using RingLargeB = Ring<3, 32768>;
@@ -76,6 +86,14 @@ struct StageHdr {
     int type, e, i_act, p0, n, row0, s, ns;
 };
 
+// One work unit, decoded: kind, expert id and active index, first pair and
+// pair count of its token tile, first row, stage count, and (down units)
+// the gate/up units of its expert that must be published first.
+struct UnitRec {
+    int type, e, i_act, p0, n, row0, ns, need;
+};
+constexpr int UNIT_WINDOW = 32;  // units a producer decodes at once (one per lane)
+
 struct SharedCtl {
     unsigned long long full[MAX_STAGES];
     unsigned long long empty[MAX_STAGES];
@@ -86,17 +104,28 @@ struct SharedCtl {
     volatile int abort_flag;
     volatile int consumed;
     int n_active, total_tiles;
+    int last_cta;
     int tile_start[E_MAX + 1];
+    UnitRec urec[UNIT_WINDOW];  // the producer's decoded window of its own units
     int act_e[E_MAX];       // active expert ids (copied once per CTA)
     int off[E_MAX + 1];     // list offsets (copied once per CTA)
 };
+
+static_assert(sizeof(SharedCtl) <= CTL_BYTES, "SharedCtl does not fit its reservation");
 
 struct ExpertArgs {
     const uint16_t *xb;
     int B, d, E, k, F;
     int xbox;   // gather mode: columns per row box of the x map (<= GATHER_COLS)
-    int dense;  // B <= TN: every gate/up stage loads all B token rows in one box
+    // dense mode (B <= TN): every stage works on all B tokens; gate/up stages
+    // load all token rows of x in one box, H is token-indexed [slot][B][d_ff]
+    // and the down epilogue weighs tokens by wd[slot][B]
+    int dense;
     int bpad;   // B rounded up to a multiple of 8 (dense mode)
+    int hrows;  // rows of one H box (bpad in dense mode, TN otherwise)
+    int early;       // start when ctr->pubs[c].pub reaches pub_target, not at the previous kernel's end
+    int pub_target;
+    const float *wd;
     const int32_t *n_active, *active, *offsets, *tok;
     const float *w;
     float *y;
@@ -143,6 +172,22 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, i
         "l"(reinterpret_cast<unsigned long long>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
         : "memory");
 }
+// The same for a tensor read once per call (the expert weights): marked
+// evict-first in L2 so that the stream does not push out what the next call
+// reuses (router weights, code, the small per-call buffers).
+__device__ __forceinline__ unsigned long long evict_first_policy() {
+    unsigned long long p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ void tma_load_3d_stream(void *dst, const CUtensorMap *map, int c0, int c1, int c2,
+                                                   unsigned long long *bar, unsigned long long policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<unsigned long long>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar)), "l"(policy)
+        : "memory");
+}
 // four rows r0..r3 (any order) from column `col` of a one-row-box map
 __device__ __forceinline__ void tma_gather4(void *dst, const CUtensorMap *map, int col, int r0, int r1, int r2,
                                             int r3, unsigned long long *bar) {
@@ -177,11 +222,6 @@ __device__ __forceinline__ int ld_acquire(const int *p) {
     asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
-__device__ __forceinline__ int ld_relaxed(const int *p) {
-    int v;
-    asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
 __device__ __forceinline__ void consumer_bar() { asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory"); }
 static_assert(NCW == 8, "the stage split below assumes eight consumer warps");
 
@@ -213,18 +253,20 @@ __device__ bool wait_phase(unsigned long long *bar, unsigned parity, SharedCtl *
 
 // ------------------------------------------------------------ producer --
 // The producer keeps one unit decoded ahead: while it issues the stages of
-// the current unit, the next ticket, the next unit's token indices (GU) or
-// its gate/up completion count (D) are already in flight, so no global
-// round trip sits between two stages.
-struct UnitInfo {
-    int type, e, i_act, p0, n, row0, ns, need;
-    int tok;  // GU: token of this lane's x row (lane < n)
-    int dep;  // D (lane 0): gate/up units counted done when decoded
+// the current unit, the next unit's token indices (gathered gate/up) or its
+// gate/up completion count (down) are already in flight, so no global round
+// trip sits between two stages.
+struct UnitInfo : UnitRec {
+    int tok;  // GU, gather mode: token of this lane's x row (lane < n)
+    int dep;  // D (lane 0): gate/up units of the expert already published
 };
 
-__device__ __forceinline__ bool decode_unit(int u, int n_units, const ExpertArgs &a, const SharedCtl *ctl,
-                                            int lane, UnitInfo &ui) {
-    if (u >= n_units) return false;
+__device__ __forceinline__ void decode_rec(int u, int n_units, const ExpertArgs &a, const SharedCtl *ctl,
+                                           UnitRec &ui) {
+    if (u >= n_units) {
+        ui.type = UNIT_END;
+        return;
+    }
     const int gu_per_tile = a.F / GU_ROWS;
     const int d_per_tile = a.d / D_ROWS;
     const int n_gu = ctl->total_tiles * gu_per_tile;
@@ -262,13 +304,26 @@ __device__ __forceinline__ bool decode_unit(int u, int n_units, const ExpertArgs
     ui.p0 = ctl->off[i] + tt * TN;
     ui.n = min(TN, ctl->off[i + 1] - ui.p0);
     ui.need = nt_i * gu_per_tile;
-    // prefetches, first used when the unit's first stage is issued: the token
-    // rows a gathered gate/up stage loads, and (acquire) how many gate/up
-    // units of this expert are already published
+}
+
+// The j-th unit of this CTA's round-robin sequence (units blockIdx.x +
+// j * gridDim.x).  The producer's lanes decode UNIT_WINDOW units at a time
+// into shared memory; the prefetches of the unit's first stage are issued
+// here and first used when that stage is issued.
+__device__ bool fetch_unit(int j, int &win_base, int n_units, const ExpertArgs &a, SharedCtl *ctl, int lane,
+                           UnitInfo &ui) {
+    if (j >= win_base + UNIT_WINDOW) {
+        __syncwarp();
+        decode_rec(blockIdx.x + (j + lane) * gridDim.x, n_units, a, ctl, ctl->urec[lane]);
+        __syncwarp();
+        win_base = j;
+    }
+    static_cast<UnitRec &>(ui) = ctl->urec[j - win_base];
+    if (ui.type == UNIT_END) return false;
     ui.tok = 0;
     ui.dep = 0;
     if (ui.type == UNIT_GU && !a.dense) ui.tok = __ldg(a.tok + ui.p0 + min(lane, ui.n - 1));
-    if (ui.type == UNIT_D && lane == 0) ui.dep = ld_acquire(&a.ctr->gu_done[i]);
+    if (ui.type == UNIT_D && lane == 0) ui.dep = ld_acquire(&a.ctr->gu_done[ui.i_act]);
     return true;
 }
 
@@ -277,13 +332,13 @@ __device__ void producer(const ExpertArgs &a, const ExpertMaps &m, SharedCtl *ct
     constexpr int STAGES = RG::STAGES;
     const int lane = threadIdx.x & 31;
     const int n_units = ctl->total_tiles * (a.F / GU_ROWS + a.d / D_ROWS);
+    const unsigned long long policy = evict_first_policy();
     // units are dealt round robin: CTA c takes c, c + grid, c + 2 grid, ...
     // (all CTAs start together when the lists are ready; every gate/up unit
     // precedes every down unit in each CTA's sequence)
-    int next_u = blockIdx.x;
+    int j_next = 0, win_base = -UNIT_WINDOW;
     UnitInfo cur;
-    bool have = decode_unit(next_u, n_units, a, ctl, lane, cur);
-    next_u += gridDim.x;
+    bool have = fetch_unit(j_next++, win_base, n_units, a, ctl, lane, cur);
     int g = 0;  // stages issued
     bool ok = true;
     while (have && ok) {
@@ -304,7 +359,7 @@ __device__ void producer(const ExpertArgs &a, const ExpertMaps &m, SharedCtl *ct
             const unsigned xbytes = a.dense ? static_cast<unsigned>(gc) * a.bpad * 128u
                                             : static_cast<unsigned>(nq) * nhalf * 4u * a.xbox * 2u;
             const unsigned bytes = cur.type == UNIT_GU ? 2u * gc * (GU_ROWS * 128) + xbytes
-                                                       : dc * (D_ROWS * 128u) + dc * (TN * 128u);
+                                                       : dc * (D_ROWS * 128u) + dc * (a.hrows * 128u);
             if (lane == 0) {
                 StageHdr &h = ctl->hdr[slot];
                 h.type = cur.type;
@@ -320,8 +375,8 @@ __device__ void producer(const ExpertArgs &a, const ExpertMaps &m, SharedCtl *ct
             __syncwarp();
             if (cur.type == UNIT_GU) {
                 const int grow = cur.e * a.F + cur.row0;
-                if (lane == 0) tma_load_3d(wdst, &m.gate, 0, grow, s * gc, &ctl->full[slot]);
-                if (lane == 1) tma_load_3d(wdst + UP_OFF, &m.up, 0, grow, s * gc, &ctl->full[slot]);
+                if (lane == 0) tma_load_3d_stream(wdst, &m.gate, 0, grow, s * gc, &ctl->full[slot], policy);
+                if (lane == 1) tma_load_3d_stream(wdst + UP_OFF, &m.up, 0, grow, s * gc, &ctl->full[slot], policy);
                 if (a.dense) {
                     // all B token rows of this column range in one swizzled box
                     if (lane == 2) tma_load_3d(odst, &m.x, 0, 0, s * gc, &ctl->full[slot]);
@@ -339,7 +394,8 @@ __device__ void producer(const ExpertArgs &a, const ExpertMaps &m, SharedCtl *ct
                                         s * gc * 64 + hh * a.xbox, t4[0], t4[1], t4[2], t4[3], &ctl->full[slot]);
                 }
             } else {
-                if (lane == 0) tma_load_3d(wdst, &m.down, 0, cur.e * a.d + cur.row0, s * dc, &ctl->full[slot]);
+                if (lane == 0)
+                    tma_load_3d_stream(wdst, &m.down, 0, cur.e * a.d + cur.row0, s * dc, &ctl->full[slot], policy);
                 if (s == 0) {
                     // this expert's gate/up units must be complete before H is read
                     if (lane == 0) {
@@ -367,10 +423,7 @@ __device__ void producer(const ExpertArgs &a, const ExpertMaps &m, SharedCtl *ct
             }
             ++g;
             if (!ok) break;
-            if (s == 0) {
-                have_nxt = decode_unit(next_u, n_units, a, ctl, lane, nxt);
-                next_u += gridDim.x;
-            }
+            if (s == 0) have_nxt = fetch_unit(j_next++, win_base, n_units, a, ctl, lane, nxt);
         }
         cur = nxt;
         have = have_nxt;
@@ -435,7 +488,7 @@ __device__ __forceinline__ void gu_stage(uint32_t wbase, uint32_t xbase, int xbo
 }
 
 template <int NT>
-__device__ __forceinline__ void d_stage(uint32_t wbase, uint32_t hbase, int kvalid, int warp, int lane,
+__device__ __forceinline__ void d_stage(uint32_t wbase, uint32_t hbase, int hrows, int kvalid, int warp, int lane,
                                         float (&acc)[4][4]) {
     const int nks = kvalid / 16;
 #pragma unroll
@@ -452,7 +505,7 @@ __device__ __forceinline__ void d_stage(uint32_t wbase, uint32_t hbase, int kval
         for (int np = 0; np < (NT + 1) / 2; ++np) {
             const int n = np * 16 + (lane & 7) + ((lane >> 4) << 3);
             uint32_t b0, b1, b2, b3;
-            ldsm_x4(swz(hbase + box * (TN * 128), n, hchunk), b0, b1, b2, b3);
+            ldsm_x4(swz(hbase + box * (hrows * 128), n, hchunk), b0, b1, b2, b3);
             mma_bf16(acc[2 * np], a0, a1, a2, a3, b0, b1);
             if (2 * np + 1 < NT) mma_bf16(acc[2 * np + 1], a0, a1, a2, a3, b2, b3);
         }
@@ -468,7 +521,7 @@ __device__ __forceinline__ void stage_dispatch(const StageHdr &h, uint32_t wbase
                      acc_u);
     } else {
         const int dk = 64 * d_chunks_of(a.F);
-        d_stage<NT>(wbase, obase, min(dk, a.F - h.s * dk), warp, lane, acc_g);
+        d_stage<NT>(wbase, obase, a.hrows, min(dk, a.F - h.s * dk), warp, lane, acc_g);
     }
 }
 
@@ -492,7 +545,7 @@ __device__ void consumer(const ExpertArgs &a, SharedCtl *ctl, unsigned char *slo
     int tk[4][2];
     float wk[4][2];
     int nsig = 0;  // completions posted (thread 0)
-    int gtok[2] = {0, 0};
+    bool lists_ready = !a.early;
     const int row = lane >> 2, col = (lane & 3) * 2;
     for (int g = 0;; ++g) {
         const int slot = g % STAGES;
@@ -507,13 +560,22 @@ __device__ void consumer(const ExpertArgs &a, SharedCtl *ctl, unsigned char *slo
             for (int j = 0; j < 4; ++j)
 #pragma unroll
                 for (int c = 0; c < 4; ++c) acc_g[j][c] = acc_u[j][c] = 0.0f;
-            if (h.type == UNIT_GU && a.dense) {
-                // epilogue elements ct and ct + NCW*32 read columns = token ids
-                const int n0 = ct >> 4, n1 = (ct + NCW * 32) >> 4;
-                gtok[0] = n0 < h.n ? __ldg(a.tok + h.p0 + n0) : 0;
-                gtok[1] = n1 < h.n ? __ldg(a.tok + h.p0 + n1) : 0;
-            }
-            if (h.type == UNIT_D) {
+            if (h.type == UNIT_D && a.dense) {
+                // the dense weights are the selection's last output: in early
+                // mode wait for it to complete before the first down unit
+                if (!lists_ready) {
+                    asm volatile("griddepcontrol.wait;" ::: "memory");
+                    lists_ready = true;
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        const int t = j * 8 + col + c;
+                        tk[j][c] = t;
+                        wk[j][c] = t < a.B ? __ldcg(a.wd + static_cast<size_t>(h.i_act) * a.B + t) : 0.0f;
+                    }
+            } else if (h.type == UNIT_D) {
                 // tokens and gate weights this thread combines; used at the
                 // unit's last stage, loaded now so the latency is hidden
 #pragma unroll
@@ -551,7 +613,7 @@ __device__ void consumer(const ExpertArgs &a, SharedCtl *ctl, unsigned char *slo
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     const int n = j * 8 + col + (c & 1);
-                    if (n < h.n) {
+                    if (n < h.n && wk[j][c & 1] != 0.0f) {
                         const int i = i_base + ((c >> 1) << 3);
                         atomicAdd(a.y + static_cast<size_t>(tk[j][c & 1]) * a.d + i, wk[j][c & 1] * acc_g[j][c]);
                     }
@@ -590,10 +652,10 @@ __device__ void consumer(const ExpertArgs &a, SharedCtl *ctl, unsigned char *slo
                 }
             }
             consumer_bar();
-            for (int idx = ct, it = 0; idx < 16 * h.n; idx += NCW * 32, ++it) {
+            for (int idx = ct; idx < 16 * h.n; idx += NCW * 32) {
+                // column n: token n (dense mode) or the tile's pair n; H row p0 + n
                 const int r = idx & 15, n = idx >> 4;
-                // accumulator column of pair n: its token (dense) or n
-                const int cn = a.dense ? (it == 0 ? gtok[0] : gtok[1]) : n;
+                const int cn = n;
                 float gs = 0.0f, us = 0.0f;
 #pragma unroll
                 for (int wv = 0; wv < NCW / 2; ++wv) {
@@ -661,36 +723,108 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         prefetch_tmap(&maps.h);
         prefetch_tmap(&maps.x);
     }
-    // everything above overlaps the re-selection kernel; the lists are read
-    // only after it has completed
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    // everything above overlaps the selection.  Early mode: wait only until
+    // the activated set is published; otherwise until the previous kernel
+    // (selection or input preparation) has completed.
+    if (!a.early) asm volatile("griddepcontrol.wait;" ::: "memory");
     if (warp == NCW) {
-        // tile table: active expert i owns tiles [tile_start[i], tile_start[i+1])
-        const int na = *a.n_active;
-        int run = 0;
-        for (int base_i = 0; base_i < na; base_i += 32) {
-            const int i = base_i + lane;
-            int nt = 0;
-            if (i < na) nt = (__ldg(a.offsets + i + 1) - __ldg(a.offsets + i) + TN - 1) / TN;
-            int incl = nt;
+        if (a.early) {
+            // dense mode: one tile per active expert, taken from the published
+            // bit mask (ascending expert order, the order of the selection's
+            // active list); H rows of slot i start at i * B
+            bool ok = true;
+            uint4 m0 = make_uint4(0u, 0u, 0u, 0u), m1 = m0;
+            const PubLine *pl = &a.ctr->pubs[blockIdx.x % PUB_COPIES];
+            if (lane == 0) {
+                const unsigned long long t0 = global_ns();
+                while (ld_acquire(&pl->pub) < a.pub_target) {
+                    if (global_ns() - t0 > WAIT_LIMIT_NS) {
+                        record_error(a.ctr, ctl, DEV_TIMEOUT_DEP);
+                        ok = false;
+                        break;
+                    }
+                    __nanosleep(64);
+                }
+                if (ok) {
+                    m0 = __ldcg(reinterpret_cast<const uint4 *>(pl->mask));
+                    m1 = __ldcg(reinterpret_cast<const uint4 *>(pl->mask) + 1);
+                }
+            }
+            const unsigned mw[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+            unsigned word = 0u;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const unsigned v = __shfl_sync(0xffffffffu, mw[i], 0);
+                if (lane == i) word = v;
+            }
+            if (32 * lane >= a.E) word = 0u;
+            else if (a.E - 32 * lane < 32) word &= (1u << (a.E - 32 * lane)) - 1u;
+            int incl = __popc(word);
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const int v = __shfl_up_sync(0xffffffffu, incl, o);
                 if (lane >= o) incl += v;
             }
-            if (i < na) {
-                ctl->tile_start[i] = run + incl - nt;
-                ctl->act_e[i] = __ldg(a.active + i);
-                ctl->off[i] = __ldg(a.offsets + i);
+            int pos = incl - __popc(word);
+            while (word != 0u) {
+                const int bit = __ffs(word) - 1;
+                word &= word - 1u;
+                ctl->act_e[pos] = 32 * lane + bit;
+                ctl->tile_start[pos] = pos;
+                ctl->off[pos] = pos * a.B;
+                ++pos;
             }
-            run += __shfl_sync(0xffffffffu, incl, 31);
-        }
-        if (lane == 0 && na >= 0 && na <= a.E) ctl->off[na] = __ldg(a.offsets + na);
-        if (lane == 0) {
-            ctl->tile_start[na] = run;
-            ctl->n_active = na;
-            ctl->total_tiles = (na > 0 && na <= a.E) ? run : 0;
-            if (na < 0 || na > a.E) atomicCAS(&a.ctr->error, 0, DEV_BAD_LISTS);
+            const int na = __shfl_sync(0xffffffffu, incl, 31);
+            if (lane == 0) {
+                ctl->tile_start[na] = na;
+                ctl->off[na] = na * a.B;
+                ctl->n_active = na;
+                ctl->total_tiles = na;
+            }
+        } else if (a.dense) {
+            const int na = __ldcg(a.n_active);
+            // one tile per active expert; H rows of slot i start at i * B
+            for (int i = lane; i < na; i += 32) {
+                ctl->tile_start[i] = i;
+                ctl->act_e[i] = __ldcg(a.active + i);
+                ctl->off[i] = i * a.B;
+            }
+            if (lane == 0) {
+                const bool valid = na >= 0 && na <= a.E;
+                ctl->tile_start[valid ? na : 0] = valid ? na : 0;
+                ctl->off[valid ? na : 0] = (valid ? na : 0) * a.B;
+                ctl->n_active = valid ? na : 0;
+                ctl->total_tiles = (na > 0 && valid) ? na : 0;
+                if (!valid) atomicCAS(&a.ctr->error, 0, DEV_BAD_LISTS);
+            }
+        } else {
+            const int na = __ldcg(a.n_active);
+            // tile table: active expert i owns tiles [tile_start[i], tile_start[i+1])
+            int run = 0;
+            for (int base_i = 0; base_i < na; base_i += 32) {
+                const int i = base_i + lane;
+                int nt = 0;
+                if (i < na) nt = (__ldg(a.offsets + i + 1) - __ldg(a.offsets + i) + TN - 1) / TN;
+                int incl = nt;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += v;
+                }
+                if (i < na) {
+                    ctl->tile_start[i] = run + incl - nt;
+                    ctl->act_e[i] = __ldg(a.active + i);
+                    ctl->off[i] = __ldg(a.offsets + i);
+                }
+                run += __shfl_sync(0xffffffffu, incl, 31);
+            }
+            if (lane == 0 && na >= 0 && na <= a.E) ctl->off[na] = __ldg(a.offsets + na);
+            if (lane == 0) {
+                ctl->tile_start[na >= 0 && na <= a.E ? na : 0] = run;
+                ctl->n_active = na;
+                ctl->total_tiles = (na > 0 && na <= a.E) ? run : 0;
+                if (na < 0 || na > a.E) atomicCAS(&a.ctr->error, 0, DEV_BAD_LISTS);
+            }
         }
     }
     __syncthreads();
@@ -701,24 +835,64 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     } else {
         consumer<RG>(a, ctl, slots, part);
     }
+    // The last CTA to finish puts the call's counters back to zero (every
+    // CTA has read the published set and no gate/up count is awaited any
+    // more); the next call's first kernel starts after this grid completes.
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        ctl->last_cta = atomicAdd(&a.ctr->k3_exit, 1) == static_cast<int>(gridDim.x) - 1 ? 1 : 0;
+    }
+    __syncthreads();
+    if (ctl->last_cta) {
+        __threadfence();
+        for (int i = threadIdx.x; i < E_MAX; i += blockDim.x) a.ctr->gu_done[i] = 0;
+        for (int i = threadIdx.x; i < PUB_COPIES * (E_MAX / 32); i += blockDim.x)
+            a.ctr->pubs[i / (E_MAX / 32)].mask[i % (E_MAX / 32)] = 0u;
+        if (threadIdx.x < PUB_COPIES) a.ctr->pubs[threadIdx.x].pub = 0;
+        if (threadIdx.x == 0) a.ctr->k3_exit = 0;
+    }
 }
 
 // ------------------------------------------------------------------ prep --
-__global__ void __launch_bounds__(256) ffn_prep_kernel(const float *__restrict__ x, int n4, uint16_t *__restrict__ xb,
-                                                       float *__restrict__ y, Counters *ctr) {
-    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += gridDim.x * blockDim.x) {
-        const float4 v = __ldg(reinterpret_cast<const float4 *>(x) + i);
+struct PrepArgs {
+    const float *x;
+    int n4, B;
+    uint16_t *xb;
+    float *y;
+    Counters *ctr;
+    const int32_t *n_active, *offsets, *tok;
+    const float *w;
+    float *wd;  // dense weights [slot][B] (B <= 32), or null
+};
+
+__global__ void __launch_bounds__(256) ffn_prep_kernel(PrepArgs p) {
+    const int tid = blockIdx.x * blockDim.x + threadIdx.x, nthreads = gridDim.x * blockDim.x;
+    for (int i = tid; i < p.n4; i += nthreads) {
+        const float4 v = __ldg(reinterpret_cast<const float4 *>(p.x) + i);
         const unsigned lo = static_cast<unsigned>(__bfloat16_as_ushort(__float2bfloat16_rn(v.x))) |
                             (static_cast<unsigned>(__bfloat16_as_ushort(__float2bfloat16_rn(v.y))) << 16);
         const unsigned hi = static_cast<unsigned>(__bfloat16_as_ushort(__float2bfloat16_rn(v.z))) |
                             (static_cast<unsigned>(__bfloat16_as_ushort(__float2bfloat16_rn(v.w))) << 16);
-        reinterpret_cast<uint2 *>(xb)[i] = make_uint2(lo, hi);
-        reinterpret_cast<float4 *>(y)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        reinterpret_cast<uint2 *>(p.xb)[i] = make_uint2(lo, hi);
+        reinterpret_cast<float4 *>(p.y)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    if (blockIdx.x == 0) {
-        if (threadIdx.x == 0) ctr->ticket = 0;
-        for (int i = threadIdx.x; i < E_MAX; i += blockDim.x) ctr->gu_done[i] = 0;
+    if (p.wd) {
+        // wd[i][t] = weight of token t in active expert i's list, else 0:
+        // one warp per active expert (its list holds at most B <= 32 pairs)
+        const int na = *p.n_active;
+        const int lane = threadIdx.x & 31;
+        for (int i = tid >> 5; i < na; i += nthreads >> 5) {
+            const int j0 = p.offsets[i], n = p.offsets[i + 1] - j0;
+            const int t = lane < n ? p.tok[j0 + lane] : -1;
+            const float wv = lane < n ? p.w[j0 + lane] : 0.0f;
+            if (lane < p.B) p.wd[static_cast<size_t>(i) * p.B + lane] = 0.0f;
+            __syncwarp();
+            if (t >= 0) p.wd[static_cast<size_t>(i) * p.B + t] = wv;
+        }
     }
+    if (blockIdx.x == 0)
+        for (int i = threadIdx.x; i < E_MAX; i += blockDim.x) p.ctr->gu_done[i] = 0;
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
@@ -727,7 +901,7 @@ bool g_attr_small[64] = {false}, g_attr_large[64] = {false};
 
 }  // namespace
 
-int expert_ffn_h_rows() { return TN; }
+int expert_ffn_h_rows(int B) { return B <= TN ? (B + 7) / 8 * 8 : TN; }
 int expert_ffn_dense_batch(int B) { return B <= TN ? 1 : 0; }
 int expert_ffn_gather_cols(int d) {
     const int w = 64 * expert_ffn_gu_chunks(d);
@@ -739,16 +913,27 @@ int expert_ffn_gu_chunks(int d) { return d / 64 < GU_CHUNKS ? d / 64 : GU_CHUNKS
 int expert_ffn_d_chunks(int F) { return F / 64 < D_CHUNKS ? F / 64 : D_CHUNKS; }
 
 cudaError_t launch_ffn_prep(const float *x, const moe_dims_t &d, uint16_t *xb, float *y, Counters *ctr,
-                            cudaStream_t s) {
-    const int n4 = d.B * d.d / 4;
-    const int blocks = (n4 + 255) / 256 > 0 ? min((n4 + 255) / 256, 1024) : 1;
-    ffn_prep_kernel<<<blocks, 256, 0, s>>>(x, n4, xb, y, ctr);
+                            const moe_lists_t &l, float *wd, cudaStream_t s) {
+    PrepArgs p;
+    p.x = x;
+    p.n4 = d.B * d.d / 4;
+    p.B = d.B;
+    p.xb = xb;
+    p.y = y;
+    p.ctr = ctr;
+    p.n_active = l.n_active;
+    p.offsets = l.offsets;
+    p.tok = l.tok;
+    p.w = l.w;
+    p.wd = wd;
+    const int blocks = (p.n4 + 255) / 256 > 0 ? min((p.n4 + 255) / 256, 1024) : 1;
+    ffn_prep_kernel<<<blocks, 256, 0, s>>>(p);
     return cudaGetLastError();
 }
 
 cudaError_t launch_expert_ffn(const ExpertMaps &maps, const uint16_t *xb, const moe_dims_t &d,
-                              const moe_lists_t &l, float *y, uint16_t *h, Counters *ctr, bool pdl,
-                              cudaStream_t s) {
+                              const moe_lists_t &l, float *y, uint16_t *h, const float *wd, Counters *ctr, bool early,
+                              int pub_target, cudaStream_t s) {
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
@@ -778,7 +963,11 @@ cudaError_t launch_expert_ffn(const ExpertMaps &maps, const uint16_t *xb, const 
     a.F = d.d_ff;
     a.dense = d.B <= TN ? 1 : 0;
     a.bpad = (d.B + 7) / 8 * 8;
+    a.hrows = expert_ffn_h_rows(d.B);
     a.xbox = expert_ffn_gather_cols(d.d);
+    a.early = (early && a.dense) ? 1 : 0;
+    a.pub_target = pub_target;
+    a.wd = wd;
     a.n_active = l.n_active;
     a.active = l.active;
     a.offsets = l.offsets;
@@ -788,7 +977,11 @@ cudaError_t launch_expert_ffn(const ExpertMaps &maps, const uint16_t *xb, const 
     a.h = h;
     a.ctr = ctr;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(g_num_sms[dev]);
+    // early mode: one SM stays with the selection kernel, which runs beside
+    // this grid; the router blocks exit before the activated set is
+    // published, so all CTAs of this grid are resident when streaming starts
+    // (the round-robin deal assumes they start together)
+    cfg.gridDim = dim3(early && g_num_sms[dev] > 1 ? g_num_sms[dev] - 1 : g_num_sms[dev]);
     cfg.blockDim = dim3(NTHREADS);
     cfg.dynamicSmemBytes = small ? smem_bytes<RingSmallB>() : smem_bytes<RingLargeB>();
     cfg.stream = s;
@@ -796,7 +989,7 @@ cudaError_t launch_expert_ffn(const ExpertMaps &maps, const uint16_t *xb, const 
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = pdl ? 1 : 0;
+    cfg.numAttrs = 1;  // always chained to the previous kernel with programmatic dependent launch
     return small ? cudaLaunchKernelEx(&cfg, expert_ffn_kernel<RingSmallB>, maps, a)
                  : cudaLaunchKernelEx(&cfg, expert_ffn_kernel<RingLargeB>, maps, a);
 }

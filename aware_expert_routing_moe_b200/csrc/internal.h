@@ -17,13 +17,29 @@ constexpr int K_MAX = 16;
 constexpr int D_MIN = 64, D_MAX = 16384;
 constexpr int F_MIN = 64, F_MAX = 8192;
 
-// Counters the kernels share inside one workspace.
-struct Counters {
-    int32_t ticket;        // next work unit of the expert kernel
-    int32_t error;         // first error code a kernel recorded (0 = none)
-    int32_t pad[30];
-    int32_t gu_done[E_MAX];  // finished gate/up units per active-expert slot
+// Counters the kernels share inside one workspace.  They are zero between
+// calls: each user puts back what it changed (the router's last block of a
+// token group its count; the expert kernel's last CTA everything else).
+// One published copy of the activated set, alone in a 128-byte line.
+struct PubLine {
+    int32_t pub;                // token groups whose first ranks are in `mask`
+                                // (+1 once the selection published it, XShare)
+    int32_t pad0[3];
+    uint32_t mask[E_MAX / 32];  // the activated set, one bit per expert
+    int32_t pad1[20];
 };
+static_assert(sizeof(PubLine) == 128, "PubLine must fill one 128-byte line");
+constexpr int PUB_COPIES = 8;  // expert-kernel CTA c polls copy c % PUB_COPIES
+
+struct Counters {
+    int32_t error;     // first error code a kernel recorded (0 = none)
+    int32_t k3_exit;   // expert-kernel CTAs finished
+    int32_t pad0[30];
+    PubLine pubs[PUB_COPIES];   // layer path: the activated set, in copies
+    int32_t grp_done[B_MAX];    // router blocks finished, per token group
+    int32_t gu_done[E_MAX];     // finished gate/up units per active-expert slot
+};
+static_assert(sizeof(Counters) % 16 == 0, "Counters must keep 16-byte alignment");
 
 // Device error codes written into Counters::error.
 enum DeviceError : int32_t {
@@ -38,24 +54,64 @@ enum DeviceError : int32_t {
 struct WsLayout {
     size_t counters, logits, probs, sel_idx, sel_w;
     size_t n_active, active, offsets, tok, w;
-    size_t xb, h;
+    size_t xb, h, wd;
     size_t total;
 };
 
+// Activated-expert slots a call can have: min(E, B*k).
+inline int active_slots(const moe_dims_t &d) { return d.E < d.B * d.k ? d.E : d.B * d.k; }
+// Bytes of the expert kernel's H scratch: token-indexed [slot][B][d_ff]
+// when the batch is small enough for dense gate/up stages (B <= 32), else
+// pair-indexed [B*k][d_ff]; bf16.
+inline size_t h_scratch_bytes(const moe_dims_t &d) {
+    const size_t F = d.d_ff;
+    return d.B <= 32 ? static_cast<size_t>(active_slots(d)) * d.B * F * 2 : static_cast<size_t>(d.B) * d.k * F * 2;
+}
+// Bytes of the dense weight matrix [slot][B] fp32 (B <= 32 only).
+inline size_t wd_bytes(const moe_dims_t &d) {
+    return d.B <= 32 ? static_cast<size_t>(active_slots(d)) * d.B * 4 : 0;
+}
+
 WsLayout ws_layout(const moe_dims_t &d);
 
+// TMA descriptors of the router: x [B][d] and Wg [E][d] (fp32) seen as
+// columns of 128-byte lines, 128-byte swizzle, boxes of whole rows (at most
+// 256 lines).
+struct RouterMaps {
+    CUtensorMap x, wg;
+};
+bool encode_router_maps(RouterMaps *m, const moe_dims_t &d, const float *x, const float *Wg);
+// Lines per router box for `d` (the box of encode_router_maps).
+int router_box_lines(int d);
+
 // Launchers (enqueue only; arguments already validated).
-cudaError_t launch_router_logits(const float *x, const float *Wg, const float *bias,
-                                 const moe_dims_t &d, float *logits, uint16_t *xb,
-                                 float *y_zero, cudaStream_t s);
+cudaError_t launch_router_logits(const RouterMaps &maps, const float *bias, const moe_dims_t &d, float *logits,
+                                 cudaStream_t s);
 cudaError_t launch_route_topk(const float *logits, const moe_dims_t &d, float *probs,
                               int32_t *topk_idx, float *topk_w, cudaStream_t s);
-cudaError_t launch_reselect(const float *logits, float *probs, bool fuse_softmax,
-                            const moe_dims_t &d, const moe_reselect_t &r,
-                            int32_t *sel_idx, float *sel_w, const moe_lists_t &l,
-                            int32_t *n_active_copy, Counters *ctr, bool pdl, cudaStream_t s);
+cudaError_t launch_reselect(const float *logits, const float *probs, const moe_dims_t &d,
+                            const moe_reselect_t &r, int32_t *sel_idx, float *sel_w,
+                            const moe_lists_t &l, cudaStream_t s);
+// Layer path, first kernel: router GEMV; also writes x in bf16, zeroes y
+// and (OEA, no re-selection) publishes the activated set in
+// ctr->pubs for an expert kernel started early.
+cudaError_t launch_layer_route(const RouterMaps &maps, const float *x, const float *bias, const moe_dims_t &d,
+                               const moe_reselect_t &rule, float *logits, uint16_t *xb, float *y, Counters *ctr,
+                               cudaStream_t s);
+// Layer path, second kernel (chained with programmatic dependent launch):
+// softmax, selection, lists, and `wd` (B <= 32) the dense weights.  With
+// `early` the next kernel may launch at once, and in XShare the selection
+// publishes the batch set itself.
+cudaError_t launch_layer_select(const float *logits, float *probs, const moe_dims_t &d, const moe_reselect_t &rule,
+                                int32_t *sel_idx, float *sel_w, const moe_lists_t &l, int32_t *n_active_copy,
+                                Counters *ctr, float *wd, bool early, cudaStream_t s);
+// Value of every ctr->pubs[c].pub once the activated set of a layer call is
+// published.
+int layer_pub_target(const moe_dims_t &d, const moe_reselect_t &rule);
+// Standalone expert FFN: x -> bf16, y = 0, counters cleared and, for
+// B <= 32, the dense weights built from the lists.
 cudaError_t launch_ffn_prep(const float *x, const moe_dims_t &d, uint16_t *xb, float *y,
-                            Counters *ctr, cudaStream_t s);
+                            Counters *ctr, const moe_lists_t &l, float *wd, cudaStream_t s);
 
 // TMA descriptors of the expert kernel: the three weight tensors and the H
 // scratch as (64-column chunk, row, chunk index) boxes, and x in bf16 as
@@ -63,10 +119,14 @@ cudaError_t launch_ffn_prep(const float *x, const moe_dims_t &d, uint16_t *xb, f
 struct ExpertMaps {
     CUtensorMap gate, up, down, h, x;
 };
+// early (layer path, B <= 32): start when ctr->pubs[c].pub reaches
+// pub_target and take the activated set from its mask, instead of waiting for the
+// previous kernel; wd: dense weights (B <= 32).
 cudaError_t launch_expert_ffn(const ExpertMaps &maps, const uint16_t *xb,
                               const moe_dims_t &d, const moe_lists_t &l, float *y,
-                              uint16_t *h, Counters *ctr, bool pdl, cudaStream_t s);
-int expert_ffn_h_rows();              // rows of one H box (tokens per tile)
+                              uint16_t *h, const float *wd, Counters *ctr, bool early, int pub_target,
+                              cudaStream_t s);
+int expert_ffn_h_rows(int B);         // rows of one H box
 int expert_ffn_dense_batch(int B);    // 1 if gate/up stages load all B token rows at once
 int expert_ffn_gather_cols(int d);    // columns of one x row box in gather mode
 int expert_ffn_gu_rows();             // rows of Wgate / Wup per gate-up unit

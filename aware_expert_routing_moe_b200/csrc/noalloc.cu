@@ -26,7 +26,7 @@ unsigned char *g_scratch_addr[MAX_DEVICES] = {};
 size_t align256(size_t v) { return (v + 255) / 256 * 256; }
 
 struct NoallocLayout {
-    size_t counters, xb, h, total;
+    size_t counters, xb, h, wd, total;
 };
 
 NoallocLayout noalloc_layout(const moe_dims_t &d) {
@@ -34,7 +34,8 @@ NoallocLayout noalloc_layout(const moe_dims_t &d) {
     size_t o = 0;
     L.counters = o; o += align256(sizeof(Counters));
     L.xb = o;       o += align256(static_cast<size_t>(d.B) * d.d * 2);
-    L.h = o;        o += align256(static_cast<size_t>(d.B) * d.k * d.d_ff * 2);
+    L.h = o;        o += align256(h_scratch_bytes(d));
+    L.wd = o;       o += align256(wd_bytes(d));
     L.total = o;
     return L;
 }
@@ -97,12 +98,13 @@ extern "C" moe_status_t moe_expert_ffn_noalloc(const float *x, const uint16_t *W
     Counters *ctr = reinterpret_cast<Counters *>(scratch + L.counters);
     uint16_t *xb = reinterpret_cast<uint16_t *>(scratch + L.xb);
     uint16_t *h = reinterpret_cast<uint16_t *>(scratch + L.h);
+    float *wd = expert_ffn_dense_batch(dims.B) ? reinterpret_cast<float *>(scratch + L.wd) : nullptr;
     ExpertMaps maps;
     if (!encode_expert_maps(&maps, dims, Wgate, Wup, Wdown, h, xb)) return MOE_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // the prep kernel clears the ticket and the per-expert counters the
-    // expert kernel needs at zero; x and H are fully rewritten each call
-    if (launch_ffn_prep(x, dims, xb, y, ctr, s) != cudaSuccess) return MOE_ERR_CUDA;
-    if (launch_expert_ffn(maps, xb, dims, lists, y, h, ctr, true, s) != cudaSuccess) return MOE_ERR_CUDA;
+    // the prep kernel clears the per-expert counters the expert kernel needs
+    // at zero and rebuilds x, the dense weights and (in the kernel) H
+    if (launch_ffn_prep(x, dims, xb, y, ctr, lists, wd, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_expert_ffn(maps, xb, dims, lists, y, h, wd, ctr, false, 0, s) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;
 }

@@ -1,14 +1,15 @@
 // Router and batch-aware re-selection kernels (sm_100a).
 //
-//  router_logits_kernel : logits = x Wg^T + bias in a fixed fp32 order
+//  route_gemv_kernel    : logits = x Wg^T + bias in a fixed fp32 order
 //      ("Router Caching and Optimization", "Analyzing Router Inference Cost",
-//      step 1).  Optionally also writes x as bf16 for the expert kernel and
-//      zeroes y (the layer path).
+//      step 1).  In the layer path it also writes x as bf16 for the expert
+//      kernel, zeroes y and publishes the activated set as soon as every
+//      token's first ranks are known.
 //  route_topk_kernel    : warp per token: softmax (step 2) + top-k (step 3)
 //      with a warp-shuffle reduction and register-resident keys.
 //  reselect_kernel      : one CTA for the whole batch: (softmax +) top-k,
 //      OEA / XShare re-selection, renormalised weights, per-expert token
-//      lists, and the reset of the expert kernel's counters.
+//      lists and, for small batches, the dense weight matrix.
 //
 // Every floating-point step that decides an index is written with explicit
 // round-to-nearest intrinsics (__fmaf_rn, __fadd_rn, __fsub_rn, __fdiv_rn)
@@ -106,6 +107,17 @@ __device__ __forceinline__ float warp_fetch(const float (&v)[NI], int e) {
 
 template <int NI>
 __device__ __forceinline__ void load_row(const float *row, int E, int lane, float (&l)[NI]) {
+    // global rows written by other blocks or kernels: read through L2
+#pragma unroll
+    for (int i = 0; i < NI; ++i) {
+        const int e = lane + 32 * i;
+        l[i] = e < E ? __ldcg(row + e) : -INFINITY;
+    }
+}
+
+// A row in shared or global memory (generic load).
+template <int NI>
+__device__ __forceinline__ void load_row_any(const float *row, int E, int lane, float (&l)[NI]) {
 #pragma unroll
     for (int i = 0; i < NI; ++i) {
         const int e = lane + 32 * i;
@@ -186,126 +198,6 @@ __device__ void renormalise_slots(const int *sel, float *pv, int k, int lane) {
     __syncwarp();
 }
 
-// ------------------------------------------------------------------ K1 --
-// Block (bx, by) computes experts 8 bx .. 8 bx + 7 (one per warp) for the
-// tokens tb * by .. tb * by + tb - 1.  The block stages those token rows in
-// shared memory; each warp holds up to R_CH 256-column chunks of its Wg row
-// in registers (all loads issued before any use) and runs the fixed-order
-// fma chains against the shared rows.
-constexpr int R_TB = 4;  // tokens per block (at most)
-constexpr int R_CH = 8;  // 256-column chunks of a Wg row held at once
-
-__global__ void __launch_bounds__(256) router_logits_kernel(
-    const float *__restrict__ x, const float *__restrict__ Wg, const float *__restrict__ bias,
-    int B, int d, int E, int tb, float *__restrict__ logits, uint16_t *__restrict__ xb,
-    float *__restrict__ y_zero) {
-    extern __shared__ float4 xs4[];  // [tb][d / 4]
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int e = blockIdx.x * 8 + warp;
-    const int b0 = blockIdx.y * tb;
-    const int nb = min(tb, B - b0);
-    const int nch = (d + 255) / 256;
-    const float *wrow = Wg + static_cast<size_t>(min(e, E - 1)) * d;
-    // first R_CH chunks of this warp's Wg row: issued before anything waits
-    float4 w[R_CH][2];
-#pragma unroll
-    for (int cc = 0; cc < R_CH; ++cc) {
-        const int j0 = 256 * cc + 8 * lane;
-        if (cc < nch && j0 < d) {
-            w[cc][0] = __ldg(reinterpret_cast<const float4 *>(wrow + j0));
-            w[cc][1] = __ldg(reinterpret_cast<const float4 *>(wrow + j0 + 4));
-        }
-    }
-    {
-        // stage the token rows: eight loads in flight per thread, then stores
-        const float4 *src = reinterpret_cast<const float4 *>(x) + static_cast<size_t>(b0) * (d / 4);
-        const int total4 = nb * (d / 4);
-#pragma unroll 1
-        for (int base = 0; base < total4; base += 8 * 256) {
-            float4 v[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int i = base + u * 256 + static_cast<int>(threadIdx.x);
-                if (i < total4) v[u] = __ldg(src + i);
-            }
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int i = base + u * 256 + static_cast<int>(threadIdx.x);
-                if (i < total4) xs4[i] = v[u];
-            }
-        }
-    }
-    __syncthreads();
-    if (e < E) {
-        float acc[R_TB];
-#pragma unroll
-        for (int t = 0; t < R_TB; ++t) acc[t] = 0.0f;
-#pragma unroll 1
-        for (int c0 = 0; c0 < nch; c0 += R_CH) {
-            if (c0 > 0) {
-#pragma unroll
-                for (int cc = 0; cc < R_CH; ++cc) {
-                    const int j0 = 256 * (c0 + cc) + 8 * lane;
-                    if (c0 + cc < nch && j0 < d) {
-                        w[cc][0] = __ldg(reinterpret_cast<const float4 *>(wrow + j0));
-                        w[cc][1] = __ldg(reinterpret_cast<const float4 *>(wrow + j0 + 4));
-                    }
-                }
-            }
-#pragma unroll
-            for (int t = 0; t < R_TB; ++t) {
-                if (t >= nb) break;
-                float a = acc[t];
-#pragma unroll
-                for (int cc = 0; cc < R_CH; ++cc) {
-                    const int j0 = 256 * (c0 + cc) + 8 * lane;
-                    if (c0 + cc < nch && j0 < d) {
-                        const float4 x0 = xs4[(t * d + j0) / 4];
-                        const float4 x1 = xs4[(t * d + j0) / 4 + 1];
-                        a = __fmaf_rn(x0.x, w[cc][0].x, a);
-                        a = __fmaf_rn(x0.y, w[cc][0].y, a);
-                        a = __fmaf_rn(x0.z, w[cc][0].z, a);
-                        a = __fmaf_rn(x0.w, w[cc][0].w, a);
-                        a = __fmaf_rn(x1.x, w[cc][1].x, a);
-                        a = __fmaf_rn(x1.y, w[cc][1].y, a);
-                        a = __fmaf_rn(x1.z, w[cc][1].z, a);
-                        a = __fmaf_rn(x1.w, w[cc][1].w, a);
-                    }
-                }
-                acc[t] = a;
-            }
-        }
-        float mine = 0.0f;
-#pragma unroll
-        for (int t = 0; t < R_TB; ++t) {
-            const float v = warp_butterfly_sum(acc[t]);
-            if (lane == t) mine = v;
-        }
-        if (lane < nb) {
-            const float v = bias ? __fadd_rn(mine, __ldg(bias + e)) : mine;
-            logits[static_cast<size_t>(b0 + lane) * E + e] = v;
-        }
-    }
-    if (xb != nullptr) {
-        // layer path: x -> bf16 copy for the expert kernel, y = 0
-        const int n4 = B * d / 4;
-        const int nthreads = gridDim.x * gridDim.y * blockDim.x;
-        for (int i = (blockIdx.y * gridDim.x + blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
-             i += nthreads) {
-            const float4 v = __ldg(reinterpret_cast<const float4 *>(x) + i);
-            const unsigned lo = static_cast<unsigned>(__bfloat16_as_ushort(__float2bfloat16_rn(v.x))) |
-                                (static_cast<unsigned>(__bfloat16_as_ushort(__float2bfloat16_rn(v.y))) << 16);
-            const unsigned hi = static_cast<unsigned>(__bfloat16_as_ushort(__float2bfloat16_rn(v.z))) |
-                                (static_cast<unsigned>(__bfloat16_as_ushort(__float2bfloat16_rn(v.w))) << 16);
-            reinterpret_cast<uint2 *>(xb)[i] = make_uint2(lo, hi);
-            if (y_zero) reinterpret_cast<float4 *>(y_zero)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-    }
-    // let the dependent (re-selection) kernel become resident; it waits for
-    // this grid's completion before reading the logits
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-
 // ------------------------------------------------------------ route only --
 template <int NI>
 __global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict__ logits, int B, int E,
@@ -346,7 +238,16 @@ struct ReselectArgs {
     float *sel_w;
     moe_lists_t lists;
     int32_t *n_active_copy;
-    Counters *ctr;
+    Counters *ctr;  // layer path: the expert kernel's counters (else null)
+    // layer path, XShare, expert kernel started early: publish the batch
+    // set (every copy of ctr->pubs: mask, then pub + 1) as soon as it is known
+    int publish;
+    // let the dependent kernel launch before waiting for the previous one
+    // (the expert kernel started early); otherwise once that wait returns
+    int early_dependents;
+    // dense weights [active slot][B] (0 where a token does not use the
+    // expert), written when non-null
+    float *wd;
 };
 
 // Inclusive scan over threads 0..255 (value 0 for t >= n); every thread of
@@ -445,16 +346,24 @@ __device__ __forceinline__ void take_slot(int j, float pe, int lane, float &sum,
     if (lane == j) myp = pe;
 }
 
-template <int NI>
-__global__ void __launch_bounds__(1024, 1) reselect_kernel(ReselectArgs a) {
-    // wait until the router's logits are complete and visible
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    // the expert kernel may become resident now; it waits for this grid
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+// Dense weights of token b: wd[i][b] for every active slot i (0 unless the
+// token chose active[i]).  Lane j < k holds the token's slot j.
+__device__ void write_dense_weights(float *wd, int B, int b, int n_active, const int *s_rank, int mye, float myw,
+                                    int k, int lane) {
+    for (int i = lane; i < n_active; i += 32) wd[static_cast<size_t>(i) * B + b] = 0.0f;
+    __syncwarp();
+    if (lane < k && mye >= 0) wd[static_cast<size_t>(s_rank[mye]) * B + b] = myw;
+}
 
-    extern __shared__ __align__(16) unsigned char smem_raw[];
+// The batch-level selection, run by one block (any multiple of 32 threads,
+// at least 256): phase 1 per token (softmax in the layer path, first ranks),
+// XShare's batch set, phase 2 per token (OEA fills / XShare top-k, weights),
+// then the per-expert lists.  Every thread of the block must call it.
+template <int NI>
+__device__ void reselect_body(const ReselectArgs &a, unsigned char *smem_raw) {
     const int B = a.B, E = a.E, k = a.k;
     const int BW = (B + 31) >> 5;
+    const int nwarps = blockDim.x >> 5;
     int *T = reinterpret_cast<int *>(smem_raw);                    // [B][k] first ranks
     unsigned *ASSIGN = reinterpret_cast<unsigned *>(T + B * k);     // [E][BW] final assignment
     unsigned *TMEMB = ASSIGN + E * BW;                                // [E][BW] top-k membership
@@ -462,8 +371,10 @@ __global__ void __launch_bounds__(1024, 1) reselect_kernel(ReselectArgs a) {
     float *LC = PC + (a.cache_rows ? B * E : 0);                      // [B][E] logit cache
     __shared__ float s_score[E_MAX];
     __shared__ int s_off[E_MAX];
+    __shared__ int s_rank[E_MAX];  // expert -> active slot (publishing path)
     __shared__ unsigned ukept[E_MAX / 32], ubase[E_MAX / 32], sbits[E_MAX / 32];
     __shared__ int wsum[9];
+    __shared__ int s_nact;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     for (int i = tid; i < 2 * E * BW; i += blockDim.x) ASSIGN[i] = 0u;  // and TMEMB
@@ -473,11 +384,12 @@ __global__ void __launch_bounds__(1024, 1) reselect_kernel(ReselectArgs a) {
     const int mode = a.mode;
     float *prob_rows = a.cache_rows ? PC : a.probs;
     const float *logit_rows = a.cache_rows ? LC : a.logits;
+    const bool dense_w = a.wd != nullptr;
 
     // ---- phase 1: softmax (layer path) and each token's first ranks
     const int r1 = (mode == MOE_RESELECT_OEA) ? a.k0 : k;
 #pragma unroll 1
-    for (int b = warp; b < B; b += 32) {
+    for (int b = warp; b < B; b += nwarps) {
         float l[NI], p[NI];
         unsigned ord[NI];
         load_row<NI>(a.logits + static_cast<size_t>(b) * E, E, lane, l);
@@ -512,10 +424,8 @@ __global__ void __launch_bounds__(1024, 1) reselect_kernel(ReselectArgs a) {
         if (lane < r1) {
             T[b * k + lane] = mye;
             if (mode == MOE_RESELECT_OEA) atomicOr(&ukept[mye >> 5], 1u << (mye & 31));
-            if (mode == MOE_RESELECT_XSHARE) {
-                atomicOr(&ubase[mye >> 5], 1u << (mye & 31));
-                atomicOr(&TMEMB[mye * BW + (b >> 5)], 1u << (b & 31));
-            }
+            if (mode != MOE_RESELECT_OEA) atomicOr(&ubase[mye >> 5], 1u << (mye & 31));
+            if (mode == MOE_RESELECT_XSHARE) atomicOr(&TMEMB[mye * BW + (b >> 5)], 1u << (b & 31));
         }
         if (mode == MOE_RESELECT_NONE && lane < k) {
             a.sel_idx[static_cast<size_t>(b) * k + lane] = mye;
@@ -553,14 +463,49 @@ __global__ void __launch_bounds__(1024, 1) reselect_kernel(ReselectArgs a) {
         __syncthreads();
     }
 
+    // ---- the activated set is now fixed: OEA = union of kept sets, XShare =
+    // the batch set, NONE = union of top-k sets.  Map experts to active
+    // slots for the dense weights; in XShare with the expert kernel started
+    // early, publish the set (OEA and NONE sets are published by the router).
+    if (a.publish || dense_w) {
+        const unsigned *abits = (mode == MOE_RESELECT_OEA) ? ukept : (mode == MOE_RESELECT_XSHARE ? sbits : ubase);
+        if (warp == 0) {
+            const unsigned word = lane < E_MAX / 32 ? abits[lane] : 0u;
+            int incl = __popc(word);
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int u = __shfl_up_sync(FULL, incl, o);
+                if (lane >= o) incl += u;
+            }
+            if (a.publish)
+                for (int c = 0; c < PUB_COPIES; ++c)
+                    if (lane < E_MAX / 32) a.ctr->pubs[c].mask[lane] = word;
+            int pos = incl - __popc(word);
+            for (int bit = 0; bit < 32; ++bit) {
+                const int e = 32 * lane + bit;
+                if (e >= E) break;
+                s_rank[e] = ((word >> bit) & 1u) ? pos++ : -1;
+            }
+            const int na = __shfl_sync(FULL, incl, 31);
+            __syncwarp();
+            if (lane == 0) s_nact = na;
+            if (a.publish && lane < PUB_COPIES) {
+                __threadfence();
+                asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(&a.ctr->pubs[lane].pub), "r"(1)
+                             : "memory");
+            }
+        }
+        __syncthreads();
+    }
+
     // ---- phase 2: OEA fills / XShare top-k within the batch set; weights
     if (mode != MOE_RESELECT_NONE) {
 #pragma unroll 1
-        for (int b = warp; b < B; b += 32) {
+        for (int b = warp; b < B; b += nwarps) {
             float l[NI], p[NI];
             unsigned ord[NI];
-            load_row<NI>(logit_rows + static_cast<size_t>(b) * E, E, lane, l);
-            load_row<NI>(prob_rows + static_cast<size_t>(b) * E, E, lane, p);
+            load_row_any<NI>(logit_rows + static_cast<size_t>(b) * E, E, lane, l);
+            load_row_any<NI>(prob_rows + static_cast<size_t>(b) * E, E, lane, p);
 #pragma unroll
             for (int i = 0; i < NI; ++i) ord[i] = ord_of(l[i]);
             unsigned cand = 0;
@@ -587,11 +532,20 @@ __global__ void __launch_bounds__(1024, 1) reselect_kernel(ReselectArgs a) {
                 if (lane == j) mye = e;
                 take_slot(j, warp_fetch<NI>(p, e), lane, sum, myp);
             }
+            const float myw = mye >= 0 ? __fdiv_rn(myp, sum) : 0.0f;
             if (lane < k) {
                 a.sel_idx[static_cast<size_t>(b) * k + lane] = mye;
-                a.sel_w[static_cast<size_t>(b) * k + lane] = mye >= 0 ? __fdiv_rn(myp, sum) : 0.0f;
+                a.sel_w[static_cast<size_t>(b) * k + lane] = myw;
                 if (mye >= 0) atomicOr(&ASSIGN[mye * BW + (b >> 5)], 1u << (b & 31));
             }
+            if (dense_w) write_dense_weights(a.wd, B, b, s_nact, s_rank, mye, myw, k, lane);
+        }
+    } else if (dense_w) {
+#pragma unroll 1
+        for (int b = warp; b < B; b += nwarps) {
+            const int mye = lane < k ? a.sel_idx[static_cast<size_t>(b) * k + lane] : -1;
+            const float myw = lane < k ? a.sel_w[static_cast<size_t>(b) * k + lane] : 0.0f;
+            write_dense_weights(a.wd, B, b, s_nact, s_rank, mye, myw, k, lane);
         }
     }
     __syncthreads();
@@ -636,34 +590,388 @@ __global__ void __launch_bounds__(1024, 1) reselect_kernel(ReselectArgs a) {
         a.lists.tok[i] = -1;
         a.lists.w[i] = 0.0f;
     }
-    // ---- reset the expert kernel's counters (layer path)
-    if (a.ctr) {
-        if (tid == 0) a.ctr->ticket = 0;
-        for (int i = tid; i < E_MAX; i += blockDim.x) a.ctr->gu_done[i] = 0;
+}
+
+// moe_reselect: the selection alone (one block of 1024 threads).
+template <int NI>
+__global__ void __launch_bounds__(1024, 1) reselect_kernel(ReselectArgs a) {
+    if (a.early_dependents) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (!a.early_dependents) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    reselect_body<NI>(a, smem_raw);
+}
+
+// ------------------------------------------------------------ router GEMV --
+// logits = x Wg^T (+ bias).  Block (bx, by) computes experts
+// bx*epb .. bx*epb+epb-1 (one warp each) for tokens by*tpb .. by*tpb+tpb-1.
+// One thread first loads those Wg rows and token rows into shared memory
+// with TMA: each row is a column of 128-byte lines (32 floats) stored with
+// the 128-byte swizzle, so lane l's two 16-byte loads of its group of eight
+// columns 256 c + 8 l .. + 7 hit eight different bank quads in each
+// quarter-warp phase.  Each lane keeps eight chunks (2048 columns) of its Wg
+// row in registers at a time and runs the fixed-order fma chains of the
+// block's tokens against the token rows, the tokens' chains interleaved.
+//
+// Layer path (ctr != null): while the loads are in flight the blocks write
+// x in bf16 for the expert kernel and zero y.  The last block to finish for
+// a token group (a count per group, no waiting) ranks that group's tokens
+// and ORs their first r1 experts into every copy of ctr->pubs[].mask; every
+// group then adds 1 to each copy's pub with release semantics.  When a
+// copy's pub reaches the number of token groups its mask holds the
+// activated set (OEA: the union of the kept
+// top-k0 sets; no re-selection: the union of the top-k sets), which the
+// expert kernel, started early, reads without waiting for the rest of the
+// selection.
+struct GemvArgs {
+    const float *bias;
+    int B, d, E;
+    int epb, tpb;     // experts (= warps) and tokens per block; tpb <= 4
+    int row_bytes;    // shared-memory stride of one staged row (multiple of 1024)
+    int box_lines;    // 128-byte lines per TMA box
+    int boxes;        // boxes per row
+    float *logits;
+    const float *x;   // layer path: source of the bf16 copy
+    uint16_t *xb;     // layer path: x in bf16
+    float *y;         // layer path: zeroed
+    Counters *ctr;    // layer path only (else null)
+    int r1;           // first ranks per token in the published set (0: none)
+};
+
+constexpr int GEMV_TPB_MAX = 4;
+constexpr int GEMV_EPB_MAX = 4;
+constexpr size_t GEMV_SMEM_MAX = 160u * 1024u;
+constexpr unsigned long long GEMV_WAIT_LIMIT_NS = 1000000000ull;  // 1 s
+
+__device__ __forceinline__ unsigned smem_addr(const void *p) {
+    return static_cast<unsigned>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ unsigned long long now_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ bool bar_try_wait0(unsigned long long *bar) {
+    unsigned ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], 0;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar))
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ void tma_rows(void *dst, const CUtensorMap *map, int line, unsigned long long *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<unsigned long long>(map)), "r"(0), "r"(line), "r"(smem_addr(bar))
+        : "memory");
+}
+__device__ __forceinline__ float comp(const float4 &v, int u) {
+    return u == 0 ? v.x : u == 1 ? v.y : u == 2 ? v.z : v.w;
+}
+
+// Layer path: x -> bf16 copy for the expert kernel, y = 0 (grid-stride over
+// the blocks of the launch).
+__device__ void layer_prep(const float *__restrict__ x, int B, int d, uint16_t *__restrict__ xb,
+                           float *__restrict__ y) {
+    const int n4 = B * d / 4;
+    const int nblocks = gridDim.x * gridDim.y;
+    const int nthreads = nblocks * blockDim.x;
+    for (int i = (blockIdx.y * gridDim.x + blockIdx.x) * blockDim.x + threadIdx.x; i < n4; i += nthreads) {
+        const float4 v = __ldg(reinterpret_cast<const float4 *>(x) + i);
+        const unsigned lo = static_cast<unsigned>(__bfloat16_as_ushort(__float2bfloat16_rn(v.x))) |
+                            (static_cast<unsigned>(__bfloat16_as_ushort(__float2bfloat16_rn(v.y))) << 16);
+        const unsigned hi = static_cast<unsigned>(__bfloat16_as_ushort(__float2bfloat16_rn(v.z))) |
+                            (static_cast<unsigned>(__bfloat16_as_ushort(__float2bfloat16_rn(v.w))) << 16);
+        reinterpret_cast<uint2 *>(xb)[i] = make_uint2(lo, hi);
+        reinterpret_cast<float4 *>(y)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
+}
+
+// Dot products of one Wg row (wrow) with nb <= 4 token rows (xrows, stride
+// row_bytes), all in staged, swizzled shared memory.  FULL: every 256-column
+// chunk is complete (d % 256 == 0).
+template <bool FULL>
+__device__ __forceinline__ void gemv_rows(const unsigned char *wrow, const unsigned char *xrows, int row_bytes,
+                                          int d, int nb, int lane, float (&acc)[GEMV_TPB_MAX]) {
+    // byte offsets of this lane's two halves within a 1024-byte chunk: line
+    // lane / 4, 16-byte units 2 (lane % 4) and 2 (lane % 4) + 1, swizzled
+    const int line = lane >> 2;
+    const int o0 = line * 128 + (((2 * (lane & 3)) ^ line) << 4);
+    const int o1 = line * 128 + (((2 * (lane & 3) + 1) ^ line) << 4);
+    const int nch = (d + 255) >> 8;
+#pragma unroll 1
+    for (int c0 = 0; c0 < nch; c0 += 8) {
+        float4 w[8][2];
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+            const int c = c0 + cc;
+            if (c < nch && (FULL || 256 * c + 8 * lane < d)) {
+                w[cc][0] = *reinterpret_cast<const float4 *>(wrow + c * 1024 + o0);
+                w[cc][1] = *reinterpret_cast<const float4 *>(wrow + c * 1024 + o1);
+            }
+        }
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+            const int c = c0 + cc;
+            if (c >= nch) break;
+            if (!FULL && 256 * c + 8 * lane >= d) continue;
+            float4 xa[GEMV_TPB_MAX], xc[GEMV_TPB_MAX];
+#pragma unroll
+            for (int t = 0; t < GEMV_TPB_MAX; ++t) {
+                if (t < nb) {
+                    xa[t] = *reinterpret_cast<const float4 *>(xrows + t * row_bytes + c * 1024 + o0);
+                    xc[t] = *reinterpret_cast<const float4 *>(xrows + t * row_bytes + c * 1024 + o1);
+                } else {
+                    xa[t] = xc[t] = make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int t = 0; t < GEMV_TPB_MAX; ++t) acc[t] = __fmaf_rn(comp(xa[t], u), comp(w[cc][0], u), acc[t]);
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int t = 0; t < GEMV_TPB_MAX; ++t) acc[t] = __fmaf_rn(comp(xc[t], u), comp(w[cc][1], u), acc[t]);
+        }
+    }
+}
+
+template <int NI>
+__global__ void __launch_bounds__(32 * GEMV_EPB_MAX) route_gemv_kernel(const __grid_constant__ RouterMaps maps,
+                                                                       const GemvArgs g) {
+    extern __shared__ unsigned char gemv_smem[];
+    __shared__ __align__(8) unsigned long long s_bar;
+    __shared__ unsigned s_mask[E_MAX / 32];
+    __shared__ int s_last, s_fail;
+    // the next kernel (the selection) may become resident while this runs
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    unsigned char *rows = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(gemv_smem) + 1023) & ~static_cast<uintptr_t>(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int e0 = blockIdx.x * g.epb, b0 = blockIdx.y * g.tpb;
+    const int nb = min(g.tpb, g.B - b0), ne = min(g.epb, g.E - e0);
+    unsigned char *wrows = rows;                                 // [epb][row_bytes]
+    unsigned char *xrows = rows + g.epb * g.row_bytes;           // [tpb][row_bytes]
+    if (threadIdx.x == 0) {
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&s_bar)) : "memory");
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        s_fail = 0;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const unsigned bytes = static_cast<unsigned>((ne + nb) * g.boxes * g.box_lines * 128);
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(&s_bar)), "r"(bytes)
+                     : "memory");
+        const int lines = g.d >> 5;  // 128-byte lines per row
+        for (int r = 0; r < ne; ++r)
+            for (int bx = 0; bx < g.boxes; ++bx)
+                tma_rows(wrows + r * g.row_bytes + bx * g.box_lines * 128, &maps.wg,
+                         (e0 + r) * lines + bx * g.box_lines, &s_bar);
+        for (int r = 0; r < nb; ++r)
+            for (int bx = 0; bx < g.boxes; ++bx)
+                tma_rows(xrows + r * g.row_bytes + bx * g.box_lines * 128, &maps.x,
+                         (b0 + r) * lines + bx * g.box_lines, &s_bar);
+    }
+    if (g.ctr != nullptr) layer_prep(g.x, g.B, g.d, g.xb, g.y);  // overlaps the loads
+    if (!bar_try_wait0(&s_bar)) {
+        const unsigned long long t0 = now_ns();
+        while (!bar_try_wait0(&s_bar)) {
+            if (now_ns() - t0 > GEMV_WAIT_LIMIT_NS) {
+                s_fail = 1;
+                if (g.ctr != nullptr) atomicCAS(&g.ctr->error, 0, DEV_TIMEOUT_FULL);
+                break;
+            }
+        }
+    }
+    __syncthreads();
+
+    if (warp < ne && !s_fail) {
+        const int e = e0 + warp;
+        float acc[GEMV_TPB_MAX];
+#pragma unroll
+        for (int t = 0; t < GEMV_TPB_MAX; ++t) acc[t] = 0.0f;
+        if ((g.d & 255) == 0) gemv_rows<true>(wrows + warp * g.row_bytes, xrows, g.row_bytes, g.d, nb, lane, acc);
+        else gemv_rows<false>(wrows + warp * g.row_bytes, xrows, g.row_bytes, g.d, nb, lane, acc);
+        float mine = 0.0f;
+#pragma unroll
+        for (int t = 0; t < GEMV_TPB_MAX; ++t) {
+            const float v = warp_butterfly_sum(acc[t]);
+            if (lane == t) mine = v;
+        }
+        if (lane < nb) {
+            const float v = g.bias ? __fadd_rn(mine, __ldg(g.bias + e)) : mine;
+            g.logits[static_cast<size_t>(b0 + lane) * g.E + e] = v;
+        }
+    }
+    if (g.ctr == nullptr) return;
+
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        const int t = atomicAdd(&g.ctr->grp_done[blockIdx.y], 1);
+        s_last = (t == static_cast<int>(gridDim.x) - 1) ? 1 : 0;
+    }
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();  // see the other blocks' logits of this token group
+    if (threadIdx.x < E_MAX / 32) s_mask[threadIdx.x] = 0u;
+    if (threadIdx.x == 0) g.ctr->grp_done[blockIdx.y] = 0;
+    __syncthreads();
+    if (g.r1 > 0) {
+        const int nw = blockDim.x >> 5;
+#pragma unroll 1
+        for (int t = warp; t < nb; t += nw) {
+            float l[NI];
+            unsigned ord[NI];
+            load_row<NI>(g.logits + static_cast<size_t>(b0 + t) * g.E, g.E, lane, l);
+#pragma unroll
+            for (int i = 0; i < NI; ++i) ord[i] = ord_of(l[i]);
+            unsigned cand = valid_bits<NI>(g.E, lane);
+            int mye = -1;
+#pragma unroll 1
+            for (int j = 0; j < g.r1; ++j) {
+                const int e = warp_argmax<NI>(ord, cand, lane);
+                if (lane == j) mye = e;
+            }
+            if (lane < g.r1 && mye >= 0) atomicOr(&s_mask[mye >> 5], 1u << (mye & 31));
+        }
+        __syncthreads();
+        for (int i = threadIdx.x; i < PUB_COPIES * (E_MAX / 32); i += blockDim.x) {
+            const unsigned m = s_mask[i % (E_MAX / 32)];
+            if (m != 0u) atomicOr(&g.ctr->pubs[i / (E_MAX / 32)].mask[i % (E_MAX / 32)], m);
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x < PUB_COPIES) {
+        __threadfence();
+        asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(&g.ctr->pubs[threadIdx.x].pub), "r"(1)
+                     : "memory");
+    }
+}
+
+struct GemvShape {
+    int epb, tpb, row_bytes, box_lines, boxes;
+    size_t smem;
+};
+
+// Rows are staged in boxes of at most 256 lines (32 KB); a staged row takes
+// a multiple of 1024 bytes so that every row starts a swizzle period.
+// Tokens per block up to 4; experts per block up to 4, fewer when that
+// leaves fewer than 120 blocks (small batches); both cut back while the
+// staged rows exceed 160 KB.
+GemvShape gemv_shape(const moe_dims_t &d) {
+    GemvShape g;
+    const int lines = d.d / 32;
+    g.box_lines = router_box_lines(d.d);
+    g.boxes = (lines + g.box_lines - 1) / g.box_lines;
+    g.row_bytes = (g.boxes * g.box_lines * 128 + 1023) / 1024 * 1024;
+    g.tpb = d.B < GEMV_TPB_MAX ? d.B : GEMV_TPB_MAX;
+    g.epb = GEMV_EPB_MAX;
+    while (g.epb > 1 && ((d.E + g.epb - 1) / g.epb) * ((d.B + g.tpb - 1) / g.tpb) < 120) --g.epb;
+    while (static_cast<size_t>(g.tpb + g.epb) * g.row_bytes > GEMV_SMEM_MAX) {
+        if (g.tpb >= g.epb && g.tpb > 1) --g.tpb;
+        else if (g.epb > 1) --g.epb;
+        else break;
+    }
+    g.smem = static_cast<size_t>(g.tpb + g.epb) * g.row_bytes + 1024;  // + alignment slack
+    return g;
 }
 
 int ni_for(int E) { return E <= 32 ? 1 : E <= 64 ? 2 : E <= 128 ? 4 : 8; }
 
-}  // namespace
+size_t reselect_smem(const moe_dims_t &d, int *cache_rows) {
+    const int BW = (d.B + 31) / 32;
+    const size_t base = static_cast<size_t>(d.B) * d.k * 4 + static_cast<size_t>(d.E) * BW * 8;
+    const size_t rows = static_cast<size_t>(d.B) * d.E * 8;
+    *cache_rows = (base + rows <= 96u * 1024u) ? 1 : 0;
+    return base + (*cache_rows ? rows : 0);
+}
 
-cudaError_t launch_router_logits(const float *x, const float *Wg, const float *bias,
-                                 const moe_dims_t &d, float *logits, uint16_t *xb,
-                                 float *y_zero, cudaStream_t s) {
-    static bool configured = false;  // one GPU per process
+ReselectArgs make_reselect_args(const float *logits, float *probs, bool fuse_softmax, const moe_dims_t &d,
+                                const moe_reselect_t &r, int32_t *sel_idx, float *sel_w, const moe_lists_t &l,
+                                int32_t *n_active_copy) {
+    ReselectArgs a;
+    a.logits = logits;
+    a.probs = probs;
+    a.fuse_softmax = fuse_softmax ? 1 : 0;
+    a.B = d.B;
+    a.E = d.E;
+    a.k = d.k;
+    a.mode = r.mode;
+    a.k0 = r.k0;
+    a.budget = r.budget;
+    a.sel_idx = sel_idx;
+    a.sel_w = sel_w;
+    a.lists = l;
+    a.n_active_copy = n_active_copy;
+    a.ctr = nullptr;
+    a.publish = 0;
+    a.early_dependents = 0;
+    a.wd = nullptr;
+    a.cache_rows = 0;
+    return a;
+}
+
+template <int NI>
+cudaError_t launch_gemv_ni(const RouterMaps &maps, const GemvArgs &g, const GemvShape &sh, cudaStream_t s) {
+    static bool configured = false;  // the attribute is per function; set it once
     if (!configured) {
-        const cudaError_t err = cudaFuncSetAttribute(router_logits_kernel,
-                                                     cudaFuncAttributeMaxDynamicSharedMemorySize, 192 * 1024);
+        cudaError_t err = cudaFuncSetAttribute(route_gemv_kernel<NI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(GEMV_SMEM_MAX + 1024));
+        if (err != cudaSuccess) return err;
+        // same shared-memory carve-out as the expert kernel: an SM switching
+        // between the two needs no reconfiguration
+        err = cudaFuncSetAttribute(route_gemv_kernel<NI>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
         if (err != cudaSuccess) return err;
         configured = true;
     }
-    // tokens per block: up to R_TB, and at most 160 KB of staged rows
-    int tb = R_TB;
-    while (tb > 1 && static_cast<size_t>(tb) * d.d * 4 > 160u * 1024u) --tb;
-    dim3 grid((d.E + 7) / 8, (d.B + tb - 1) / tb);
-    const size_t smem = static_cast<size_t>(tb) * d.d * 4;
-    router_logits_kernel<<<grid, 256, smem, s>>>(x, Wg, bias, d.B, d.d, d.E, tb, logits, xb, y_zero);
+    const dim3 grid((g.E + sh.epb - 1) / sh.epb, (g.B + sh.tpb - 1) / sh.tpb);
+    route_gemv_kernel<NI><<<grid, 32 * sh.epb, sh.smem, s>>>(maps, g);
     return cudaGetLastError();
+}
+
+cudaError_t launch_gemv(const RouterMaps &maps, const GemvArgs &g, const GemvShape &sh, cudaStream_t s) {
+    switch (ni_for(g.E)) {
+        case 1: return launch_gemv_ni<1>(maps, g, sh, s);
+        case 2: return launch_gemv_ni<2>(maps, g, sh, s);
+        case 4: return launch_gemv_ni<4>(maps, g, sh, s);
+        default: return launch_gemv_ni<8>(maps, g, sh, s);
+    }
+}
+
+GemvArgs make_gemv_args(const float *bias, const moe_dims_t &d, const GemvShape &sh, float *logits) {
+    GemvArgs g;
+    g.bias = bias;
+    g.B = d.B;
+    g.d = d.d;
+    g.E = d.E;
+    g.epb = sh.epb;
+    g.tpb = sh.tpb;
+    g.row_bytes = sh.row_bytes;
+    g.box_lines = sh.box_lines;
+    g.boxes = sh.boxes;
+    g.logits = logits;
+    g.x = nullptr;
+    g.xb = nullptr;
+    g.y = nullptr;
+    g.ctr = nullptr;
+    g.r1 = 0;
+    return g;
+}
+
+}  // namespace
+
+int router_box_lines(int d) { return d / 32 <= 256 ? d / 32 : 256; }
+
+cudaError_t launch_router_logits(const RouterMaps &maps, const float *bias, const moe_dims_t &d, float *logits,
+                                 cudaStream_t s) {
+    const GemvShape sh = gemv_shape(d);
+    return launch_gemv(maps, make_gemv_args(bias, d, sh, logits), sh, s);
 }
 
 cudaError_t launch_route_topk(const float *logits, const moe_dims_t &d, float *probs,
@@ -679,14 +987,19 @@ cudaError_t launch_route_topk(const float *logits, const moe_dims_t &d, float *p
 }
 
 template <int NI>
-static cudaError_t launch_reselect_ni(const ReselectArgs &a, size_t smem, bool pdl, cudaStream_t s) {
+static cudaError_t launch_reselect_ni(const ReselectArgs &a, size_t smem, bool chained, cudaStream_t s) {
     static bool configured = false;  // the attribute is per function; set it once
-    cudaError_t err = cudaSuccess;
     if (!configured) {
-        err = cudaFuncSetAttribute(reselect_kernel<NI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   96 * 1024);
+        cudaError_t err =
+            cudaFuncSetAttribute(reselect_kernel<NI>, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
+        if (err != cudaSuccess) return err;
+        err = cudaFuncSetAttribute(reselect_kernel<NI>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
         if (err != cudaSuccess) return err;
         configured = true;
+    }
+    if (!chained) {
+        reselect_kernel<NI><<<1, 1024, smem, s>>>(a);
+        return cudaGetLastError();
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(1);
@@ -697,40 +1010,56 @@ static cudaError_t launch_reselect_ni(const ReselectArgs &a, size_t smem, bool p
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = pdl ? 1 : 0;
+    cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, reselect_kernel<NI>, a);
 }
 
-cudaError_t launch_reselect(const float *logits, float *probs, bool fuse_softmax,
-                            const moe_dims_t &d, const moe_reselect_t &r,
-                            int32_t *sel_idx, float *sel_w, const moe_lists_t &l,
-                            int32_t *n_active_copy, Counters *ctr, bool pdl, cudaStream_t s) {
-    ReselectArgs a;
-    a.logits = logits;
-    a.probs = probs;
-    a.fuse_softmax = fuse_softmax ? 1 : 0;
-    a.B = d.B;
-    a.E = d.E;
-    a.k = d.k;
-    a.mode = r.mode;
-    a.k0 = r.k0;
-    a.budget = r.budget;
-    a.sel_idx = sel_idx;
-    a.sel_w = sel_w;
-    a.lists = l;
-    a.n_active_copy = n_active_copy;
-    a.ctr = ctr;
-    const int BW = (d.B + 31) / 32;
-    const size_t base = static_cast<size_t>(d.B) * d.k * 4 + static_cast<size_t>(d.E) * BW * 8;
-    const size_t rows = static_cast<size_t>(d.B) * d.E * 8;
-    a.cache_rows = (base + rows <= 96u * 1024u) ? 1 : 0;
-    const size_t smem = base + (a.cache_rows ? rows : 0);
-    switch (ni_for(d.E)) {
-        case 1: return launch_reselect_ni<1>(a, smem, pdl, s);
-        case 2: return launch_reselect_ni<2>(a, smem, pdl, s);
-        case 4: return launch_reselect_ni<4>(a, smem, pdl, s);
-        default: return launch_reselect_ni<8>(a, smem, pdl, s);
+static cudaError_t launch_reselect_args(const ReselectArgs &a, size_t smem, bool chained, cudaStream_t s) {
+    switch (ni_for(a.E)) {
+        case 1: return launch_reselect_ni<1>(a, smem, chained, s);
+        case 2: return launch_reselect_ni<2>(a, smem, chained, s);
+        case 4: return launch_reselect_ni<4>(a, smem, chained, s);
+        default: return launch_reselect_ni<8>(a, smem, chained, s);
     }
+}
+
+cudaError_t launch_reselect(const float *logits, const float *probs, const moe_dims_t &d,
+                            const moe_reselect_t &r, int32_t *sel_idx, float *sel_w, const moe_lists_t &l,
+                            cudaStream_t s) {
+    ReselectArgs a = make_reselect_args(logits, const_cast<float *>(probs), false, d, r, sel_idx, sel_w, l,
+                                        nullptr);
+    const size_t smem = reselect_smem(d, &a.cache_rows);
+    return launch_reselect_args(a, smem, false, s);
+}
+
+int layer_pub_target(const moe_dims_t &d, const moe_reselect_t &rule) {
+    const GemvShape sh = gemv_shape(d);
+    return (d.B + sh.tpb - 1) / sh.tpb + (rule.mode == MOE_RESELECT_XSHARE ? 1 : 0);
+}
+
+cudaError_t launch_layer_route(const RouterMaps &maps, const float *x, const float *bias, const moe_dims_t &d,
+                               const moe_reselect_t &rule, float *logits, uint16_t *xb, float *y, Counters *ctr,
+                               cudaStream_t s) {
+    const GemvShape sh = gemv_shape(d);
+    GemvArgs g = make_gemv_args(bias, d, sh, logits);
+    g.x = x;
+    g.xb = xb;
+    g.y = y;
+    g.ctr = ctr;
+    g.r1 = rule.mode == MOE_RESELECT_OEA ? rule.k0 : (rule.mode == MOE_RESELECT_NONE ? d.k : 0);
+    return launch_gemv(maps, g, sh, s);
+}
+
+cudaError_t launch_layer_select(const float *logits, float *probs, const moe_dims_t &d, const moe_reselect_t &rule,
+                                int32_t *sel_idx, float *sel_w, const moe_lists_t &l, int32_t *n_active_copy,
+                                Counters *ctr, float *wd, bool early, cudaStream_t s) {
+    ReselectArgs a = make_reselect_args(logits, probs, true, d, rule, sel_idx, sel_w, l, n_active_copy);
+    a.ctr = ctr;
+    a.publish = (early && rule.mode == MOE_RESELECT_XSHARE) ? 1 : 0;
+    a.early_dependents = early ? 1 : 0;
+    a.wd = wd;
+    const size_t smem = reselect_smem(d, &a.cache_rows);
+    return launch_reselect_args(a, smem, true, s);
 }
 
 }  // namespace moe

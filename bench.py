@@ -238,7 +238,8 @@ def run_ours(args, w, rank, world, local_rank):
     x_np = ms.make_tokens(S, B, 0, kind=w.get("kind", "normal"))
     t = lambda a: torch.from_numpy(a).to(dev)
     Wg, bias = t(L["Wg"]), t(L["bias"])
-    copies = [(t(L["Wgate"].view(np.int16)), t(L["Wup"].view(np.int16)), t(L["Wdown"].view(np.int16)))]
+    # every rotation has its own copy of all layer weights (router included)
+    copies = [(t(L["Wgate"].view(np.int16)), t(L["Wup"].view(np.int16)), t(L["Wdown"].view(np.int16)), Wg)]
     for _ in range(ROTATE - 1):
         copies.append(tuple(c.clone() for c in copies[0]))
     x = t(x_np)
@@ -248,8 +249,8 @@ def run_ours(args, w, rank, world, local_rank):
     s = torch.cuda.Stream(dev)
 
     def layer(r):
-        g, u, dn = copies[r]
-        moe.moe_layer_decode(x, Wg, bias, g, u, dn, S.k, mode, k0, budget, ws=ws, y=y, n_active=nact_t)
+        g, u, dn, wg = copies[r]
+        moe.moe_layer_decode(x, wg, bias, g, u, dn, S.k, mode, k0, budget, ws=ws, y=y, n_active=nact_t)
 
     with torch.cuda.stream(s):
         for r in range(ROTATE):
@@ -322,7 +323,7 @@ def run_ours(args, w, rank, world, local_rank):
     g_ffn = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_ffn, stream=s):
         for r in range(ROTATE):
-            gg, uu, dd = copies[r]
+            gg, uu, dd, _ = copies[r]
             moe.moe_expert_ffn(x, gg, uu, dd, lists, S.k, ws, y=y)
     nrep = max(1, args.steps // ROTATE)
     with torch.cuda.stream(s):
@@ -345,9 +346,9 @@ def run_ours(args, w, rank, world, local_rank):
 
     def e2e_calls(nsteps):
         for i in range(nsteps):
-            g, u, dn = copies[i % ROTATE]
+            g, u, dn, wg = copies[i % ROTATE]
             x_dev.copy_(x_host, non_blocking=True)
-            moe.moe_layer_decode(x_dev, Wg, bias, g, u, dn, S.k, mode, k0, budget, ws=ws, y=y_dev)
+            moe.moe_layer_decode(x_dev, wg, bias, g, u, dn, S.k, mode, k0, budget, ws=ws, y=y_dev)
             y_host.copy_(y_dev, non_blocking=True)
 
     with torch.cuda.stream(s):
