@@ -60,9 +60,10 @@ WORKLOADS = {
 }
 
 # DRAM bytes (read + write) per launch of the expert kernel from an ncu
-# capture of the same workload (profiles/expert_ffn_q30b_b16.md); None until
-# captured for the current kernel.
-NCU_TRAFFIC = {}
+# capture of the same workload (profiles/expert_ffn_kernel_q30b_b16_oea4.md:
+# 141.83 MB read + 3.46 MB written); a workload without an entry reports
+# null.  Entries are dropped whenever the kernel changes.
+NCU_TRAFFIC = {"q30b_b16_oea4": 145285120}
 
 
 def workload_desc(w: dict) -> str:
@@ -370,8 +371,8 @@ def run_ours(args, w, rank, world, local_rank):
         "config": {"workload": workload_desc(w), "B": B, "d": S.d, "E": S.E, "k": S.k, "d_ff": S.F,
                    "rule": w["rule"], "n_active": n_active, "bytes_per_call": total_bytes,
                    "parallelism": f"replicas x{world}",
-                   "l2": f"inputs larger than L2: {ROTATE} rotating weight copies of "
-                         f"{3 * S.E * S.d * S.F * 2 / 1e9:.2f} GB",
+                   "l2": f"inputs larger than L2: {ROTATE} rotating copies of the layer weights "
+                         f"({3 * S.E * S.d * S.F * 2 / 1e9:.2f} GB of experts + the router each)",
                    "launch": "CUDA graph of 4 layer calls, PDL between the 3 kernels of a call"},
         "us_per_call": ms_step * 1e3,
         "frac_of_nominal_8tbs": (total_bytes / (ms_step * 1e-3) / 1e9) / NOMINAL_HBM_GBS,
