@@ -20,10 +20,12 @@
 // gate/up stages load x for all tokens in one swizzled box, H is indexed by
 // (active slot, token), and the down epilogue weighs each token by a dense
 // [slot][B] weight matrix (0 for tokens that did not choose the expert).
-// Gate/up work then needs only the activated set, which the layer path's
-// selection publishes before it finishes the token lists: the kernel is
-// launched early and starts streaming on that signal.  Larger batches use
-// token tiles of up to 32 pairs, x rows gathered by four, and pair-indexed H.
+// Gate/up work then needs only the activated set, which the layer path
+// publishes before the token lists exist (the router kernel for OEA and
+// plain top-k, the selection for XShare): the kernel is launched early,
+// reads the set from a published bit mask and starts streaming at once.
+// Larger batches use token tiles of up to 32 pairs, x rows gathered by four,
+// and pair-indexed H.
 //
 // Per CTA: one producer warp issues TMA tensor copies (three-dimensional
 // boxes of 64-column chunks, 128-byte swizzle) into a ring of 32 KB weight
@@ -32,7 +34,8 @@
 // m16n8k16 bf16 tiles (16 weight rows as A, tokens as B, fp32 accumulation);
 // a signal warp publishes gate/up completions.  Every wait is bounded by a
 // time limit; on expiry the CTA records an error code in the workspace,
-// drains its in-flight copies and returns.
+// drains its in-flight copies and returns.  The last CTA to finish puts the
+// workspace counters of the call back to zero.
 #include <cuda_bf16.h>
 
 #include "internal.h"
