@@ -609,9 +609,9 @@ __global__ void __launch_bounds__(1024, 1) reselect_kernel(ReselectArgs a) {
 // with TMA: each row is a column of 128-byte lines (32 floats) stored with
 // the 128-byte swizzle, so lane l's two 16-byte loads of its group of eight
 // columns 256 c + 8 l .. + 7 hit eight different bank quads in each
-// quarter-warp phase.  Each lane keeps eight chunks (2048 columns) of its Wg
-// row in registers at a time and runs the fixed-order fma chains of the
-// block's tokens against the token rows, the tokens' chains interleaved.
+// quarter-warp phase.  Each lane runs the fixed-order fma chains of the
+// block's tokens over its columns, chunk by chunk, the tokens' chains
+// interleaved.
 //
 // Layer path (ctr != null): while the loads are in flight the blocks write
 // x in bf16 for the expert kernel and zero y.  The last block to finish for
@@ -692,8 +692,10 @@ __device__ void layer_prep(const float *__restrict__ x, int B, int d, uint16_t *
 }
 
 // Dot products of one Wg row (wrow) with nb <= 4 token rows (xrows, stride
-// row_bytes), all in staged, swizzled shared memory.  FULL: every 256-column
-// chunk is complete (d % 256 == 0).
+// row_bytes), all in staged, swizzled shared memory.  One 256-column chunk
+// per iteration (a short loop body: this code runs once per call, so its
+// instruction fetch is on the critical path).  FULL: every chunk is
+// complete (d % 256 == 0).
 template <bool FULL>
 __device__ __forceinline__ void gemv_rows(const unsigned char *wrow, const unsigned char *xrows, int row_bytes,
                                           int d, int nb, int lane, float (&acc)[GEMV_TPB_MAX]) {
@@ -704,40 +706,28 @@ __device__ __forceinline__ void gemv_rows(const unsigned char *wrow, const unsig
     const int o1 = line * 128 + (((2 * (lane & 3) + 1) ^ line) << 4);
     const int nch = (d + 255) >> 8;
 #pragma unroll 1
-    for (int c0 = 0; c0 < nch; c0 += 8) {
-        float4 w[8][2];
+    for (int c = 0; c < nch; ++c) {
+        if (!FULL && 256 * c + 8 * lane >= d) continue;
+        const float4 w0 = *reinterpret_cast<const float4 *>(wrow + c * 1024 + o0);
+        const float4 w1 = *reinterpret_cast<const float4 *>(wrow + c * 1024 + o1);
+        float4 xa[GEMV_TPB_MAX], xc[GEMV_TPB_MAX];
 #pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-            const int c = c0 + cc;
-            if (c < nch && (FULL || 256 * c + 8 * lane < d)) {
-                w[cc][0] = *reinterpret_cast<const float4 *>(wrow + c * 1024 + o0);
-                w[cc][1] = *reinterpret_cast<const float4 *>(wrow + c * 1024 + o1);
+        for (int t = 0; t < GEMV_TPB_MAX; ++t) {
+            if (t < nb) {
+                xa[t] = *reinterpret_cast<const float4 *>(xrows + t * row_bytes + c * 1024 + o0);
+                xc[t] = *reinterpret_cast<const float4 *>(xrows + t * row_bytes + c * 1024 + o1);
+            } else {
+                xa[t] = xc[t] = make_float4(0.f, 0.f, 0.f, 0.f);
             }
         }
 #pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-            const int c = c0 + cc;
-            if (c >= nch) break;
-            if (!FULL && 256 * c + 8 * lane >= d) continue;
-            float4 xa[GEMV_TPB_MAX], xc[GEMV_TPB_MAX];
+        for (int u = 0; u < 4; ++u)
 #pragma unroll
-            for (int t = 0; t < GEMV_TPB_MAX; ++t) {
-                if (t < nb) {
-                    xa[t] = *reinterpret_cast<const float4 *>(xrows + t * row_bytes + c * 1024 + o0);
-                    xc[t] = *reinterpret_cast<const float4 *>(xrows + t * row_bytes + c * 1024 + o1);
-                } else {
-                    xa[t] = xc[t] = make_float4(0.f, 0.f, 0.f, 0.f);
-                }
-            }
+            for (int t = 0; t < GEMV_TPB_MAX; ++t) acc[t] = __fmaf_rn(comp(xa[t], u), comp(w0, u), acc[t]);
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
+        for (int u = 0; u < 4; ++u)
 #pragma unroll
-                for (int t = 0; t < GEMV_TPB_MAX; ++t) acc[t] = __fmaf_rn(comp(xa[t], u), comp(w[cc][0], u), acc[t]);
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-#pragma unroll
-                for (int t = 0; t < GEMV_TPB_MAX; ++t) acc[t] = __fmaf_rn(comp(xc[t], u), comp(w[cc][1], u), acc[t]);
-        }
+            for (int t = 0; t < GEMV_TPB_MAX; ++t) acc[t] = __fmaf_rn(comp(xc[t], u), comp(w1, u), acc[t]);
     }
 }
 

@@ -391,6 +391,95 @@ def run_ours(args, w, rank, world, local_rank):
     torch.cuda.synchronize(dev)
 
 
+SWEEP = {
+    # shape: [(B, mode, k0, budget, token kind)], the configurations the
+    # results table reports (one weight set per shape, ROTATE copies)
+    "tiny": [(4, 1, 2, 0, "normal"), (4, 0, 0, 0, "normal")],
+    "e64": [(16, 1, 4, 0, "normal"), (16, 0, 0, 0, "normal")],
+    "q30b": [(b, m, k0, 0, "normal") for b in (1, 4, 16, 32, 64) for (m, k0) in ((0, 0), (1, 4))]
+            + [(16, 1, k0, 0, "normal") for k0 in (2, 6, 8)]
+            + [(32, 0, 0, 0, "spec")] + [(32, 2, 0, m, "spec") for m in (24, 32, 48)],
+    "q235b": [(b, 1, 4, 0, "normal") for b in (1, 8, 16, 64)] + [(16, 0, 0, 0, "normal")],
+}
+
+
+def run_sweep(args):
+    """Times moe_layer_decode on every configuration of SWEEP (device time per
+    call over graph replays of ROTATE calls on rotating weight copies) and
+    the oracle on one call (1 thread and all host threads); one JSON line
+    per configuration."""
+    import torch
+    import aware_expert_routing_moe_b200 as moe
+    import oracle
+    dev = torch.device("cuda", 0)
+    moe.load_library()
+    cores = len(os.sched_getaffinity(0))
+    hbm_peak, _ = measured_peaks()
+    shapes = args.sweep.split(",") if args.sweep != "all" else list(SWEEP)
+    for shape in shapes:
+        S = ms.SHAPES[shape]
+        L = ms.make_weights(S, 0)
+        t = lambda a: torch.from_numpy(a).to(dev)
+        base = (t(L["Wgate"].view(np.int16)), t(L["Wup"].view(np.int16)), t(L["Wdown"].view(np.int16)), t(L["Wg"]))
+        copies = [base] + [tuple(c.clone() for c in base) for _ in range(ROTATE - 1)]
+        bias = t(L["bias"])
+        s = torch.cuda.Stream(dev)
+        for (B, mode, k0, budget, kind) in SWEEP[shape]:
+            x_np = ms.make_tokens(S, B, 0, kind=kind)
+            x = t(x_np)
+            ws = moe.new_workspace(B, S.d, S.E, S.k, S.F, dev)
+            y = torch.empty(B, S.d, dtype=torch.float32, device=dev)
+            nact_t = torch.zeros(4, dtype=torch.int32, device=dev)
+
+            def layer(r):
+                g, u, dn, wg = copies[r]
+                moe.moe_layer_decode(x, wg, bias, g, u, dn, S.k, mode, k0, budget, ws=ws, y=y, n_active=nact_t)
+
+            with torch.cuda.stream(s):
+                for r in range(ROTATE):
+                    layer(r)
+            s.synchronize()
+            g_all = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_all, stream=s):
+                for r in range(ROTATE):
+                    layer(r)
+            with torch.cuda.stream(s):
+                for _ in range(5):
+                    g_all.replay()
+            torch.cuda.synchronize(dev)
+            reps = max(args.steps // ROTATE, 5)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(s):
+                e0.record(s)
+                for _ in range(reps):
+                    g_all.replay()
+                e1.record(s)
+            e1.synchronize()
+            us = e0.elapsed_time(e1) * 1e3 / (reps * ROTATE)
+            if moe.moe_check_error(ws, s) != 0:
+                raise RuntimeError(f"device error word set: {shape} {B} {mode}")
+            n_active = int(nact_t[0].item())
+            total, _ = algorithmic_bytes(S, B, n_active)
+            gbs = total / (us * 1e-6) / 1e9
+            line = {"shape": shape, "B": B, "mode": ["NONE", "OEA", "XShare"][mode], "k0": k0, "budget": budget,
+                    "tokens": kind, "n_active": n_active, "us": us, "bytes": total, "GBps": gbs,
+                    "frac_8tbs": gbs / NOMINAL_HBM_GBS, "frac_measured": gbs / hbm_peak}
+            if not args.no_cpu_baseline:
+                ms_t = []
+                for th in (1, cores):
+                    t0 = time.perf_counter()
+                    oracle.layer(x_np, L, S.k, mode, k0, budget, threads=th)
+                    ms_t.append((time.perf_counter() - t0) * 1e3)
+                line["oracle_ms_1"] = ms_t[0]
+                line["oracle_ms_n"] = ms_t[1]
+                line["oracle_cores"] = cores
+            print(json.dumps(line), flush=True)
+            del g_all
+        del copies, base
+        torch.cuda.empty_cache()
+    return 0
+
+
 def run_profile_case(args, w):
     """A small case for ncu captures: one weight copy (about 1.2 GB for the
     Qwen3-30B shape, so the activated experts still exceed L2), `warmup`
@@ -422,6 +511,8 @@ def main(argv=None):
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="q30b_b16_oea4")
     ap.add_argument("--no-extra", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", default=None,
+                    help="time every results-table configuration of these shapes ('all' or a comma list)")
     ap.add_argument("--profile", action="store_true",
                     help="small case for ncu: one weight copy, warmup + steps layer calls, no timing")
     args = ap.parse_args(argv)
@@ -431,6 +522,8 @@ def main(argv=None):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     w = WORKLOADS[args.workload]
+    if args.sweep:
+        return run_sweep(args)
     if args.profile:
         return run_profile_case(args, w)
     if args.impl == "reference":
