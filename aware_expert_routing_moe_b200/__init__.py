@@ -30,7 +30,7 @@ STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_MISALIGNED", 3: "MO
           4: "MOE_ERR_UNSUPPORTED", 5: "MOE_ERR_CUDA", 6: "MOE_ERR_INTERNAL"}
 ABI_SYMBOLS = ("moe_workspace_bytes", "moe_route", "moe_reselect", "moe_expert_ffn",
                "moe_layer_decode", "moe_expert_ffn_noalloc", "moe_check_error", "moe_status_string")
-NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libmoe_decode.so")
@@ -208,7 +208,7 @@ def moe_layer_decode(x, Wg, bias, Wgate, Wup, Wdown, k: int, mode: int, k0: int 
 
 def moe_expert_ffn_noalloc(x, Wgate, Wup, Wdown, lists: dict, k: int, y=None, stream=None):
     """moe_expert_ffn without a workspace, for callers that cannot allocate
-    device memory: the library's static 16 MiB device scratch is used instead
+    device memory: the library's static 32 MiB device scratch is used instead
     (shared by all calls on a device; overlapping calls race).  -> y[B][d]."""
     B, d = x.shape
     E, F, _ = Wgate.shape

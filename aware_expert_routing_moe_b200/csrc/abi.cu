@@ -120,20 +120,6 @@ bool encode_bf16_chunked(CUtensorMap *map, const void *ptr, uint64_t rows, uint6
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// bf16 matrix [rows][cols] for tile::gather4 loads: boxes of one row and
-// box_cols columns, no swizzle.
-bool encode_bf16_rows(CUtensorMap *map, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box_cols) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t gdim[2] = {cols, rows};
-    cuuint64_t gstride[1] = {cols * 2};
-    cuuint32_t box[2] = {box_cols, 1};
-    cuuint32_t estride[2] = {1, 1};
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), gdim, gstride, box, estride,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // fp32 matrix [rows][cols] (cols % 32 == 0) seen as rows * cols / 32
 // lines of 32 floats; boxes of box_lines whole lines, 128-byte swizzle.
 // Lines past the end read as zero.
@@ -167,7 +153,7 @@ moe_lists_t ws_lists(void *ws, const WsLayout &L) {
 }  // namespace
 
 bool encode_expert_maps(ExpertMaps *m, const moe_dims_t &d, const uint16_t *Wgate, const uint16_t *Wup,
-                        const uint16_t *Wdown, const uint16_t *h, const uint16_t *xb) {
+                        const uint16_t *Wdown, const uint16_t *h, const uint16_t *x) {
     std::memset(m, 0, sizeof(*m));
     const uint64_t E = d.E, F = d.d_ff, D = d.d;
     const uint32_t gu_chunks = expert_ffn_gu_chunks(d.d), d_chunks = expert_ffn_d_chunks(d.d_ff);
@@ -179,8 +165,9 @@ bool encode_expert_maps(ExpertMaps *m, const moe_dims_t &d, const uint16_t *Wgat
                                                            : static_cast<uint64_t>(d.B) * d.k,
                                F, expert_ffn_h_rows(d.B), d_chunks) &&
            (expert_ffn_dense_batch(d.B)
-                ? encode_bf16_chunked(&m->x, xb, static_cast<uint64_t>(d.B), D, (d.B + 7) / 8 * 8, gu_chunks)
-                : encode_bf16_rows(&m->x, xb, static_cast<uint64_t>(d.B), D, expert_ffn_gather_cols(d.d)));
+                ? encode_bf16_chunked(&m->x, x, static_cast<uint64_t>(d.B), D, (d.B + 7) / 8 * 8, gu_chunks)
+                : encode_bf16_chunked(&m->x, x, static_cast<uint64_t>(d.B) * d.k, D, expert_ffn_h_rows(d.B),
+                                      gu_chunks));
 }
 
 bool encode_router_maps(RouterMaps *m, const moe_dims_t &d, const float *x, const float *Wg) {
@@ -205,6 +192,7 @@ WsLayout ws_layout(const moe_dims_t &d) {
     L.tok = o;      o += round_up(B * k * 4);
     L.w = o;        o += round_up(B * k * 4);
     L.xb = o;       o += round_up(B * D * 2);
+    L.xd = o;       o += round_up(xd_bytes(d));
     L.h = o;        o += round_up(h_scratch_bytes(d));
     L.wd = o;       o += round_up(wd_bytes(d));
     L.total = o;
@@ -278,16 +266,17 @@ moe_status_t moe_expert_ffn(const float *x, const uint16_t *Wgate, const uint16_
     st = check_device();
     if (st != MOE_OK) return st;
     const WsLayout L = ws_layout(dims);
+    const bool dense = expert_ffn_dense_batch(dims.B) != 0;
+    // the expert kernel's x: bf16 x (B <= 32) or the dispatched pair rows
+    uint16_t *xk = dense ? seg<uint16_t>(ws, L.xb) : seg<uint16_t>(ws, L.xd);
     ExpertMaps maps;
-    if (!encode_expert_maps(&maps, dims, Wgate, Wup, Wdown, seg<uint16_t>(ws, L.h), seg<uint16_t>(ws, L.xb)))
-        return MOE_ERR_CUDA;
+    if (!encode_expert_maps(&maps, dims, Wgate, Wup, Wdown, seg<uint16_t>(ws, L.h), xk)) return MOE_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     Counters *ctr = seg<Counters>(ws, L.counters);
-    uint16_t *xb = seg<uint16_t>(ws, L.xb);
-    float *wd = expert_ffn_dense_batch(dims.B) ? seg<float>(ws, L.wd) : nullptr;
-    st = from_cuda(launch_ffn_prep(x, dims, xb, y, ctr, lists, wd, s));
+    float *wd = dense ? seg<float>(ws, L.wd) : nullptr;
+    st = from_cuda(launch_ffn_prep(x, dims, dense ? xk : nullptr, dense ? nullptr : xk, y, ctr, lists, wd, false, s));
     if (st != MOE_OK) return st;
-    return from_cuda(launch_expert_ffn(maps, xb, dims, lists, y, seg<uint16_t>(ws, L.h), wd, ctr, false, 0, s));
+    return from_cuda(launch_expert_ffn(maps, xk, dims, lists, y, seg<uint16_t>(ws, L.h), wd, ctr, false, 0, s));
 }
 
 moe_status_t moe_layer_decode(const float *x, const float *Wg, const float *bias, const uint16_t *Wgate,
@@ -304,14 +293,15 @@ moe_status_t moe_layer_decode(const float *x, const float *Wg, const float *bias
     st = check_device();
     if (st != MOE_OK) return st;
     const WsLayout L = ws_layout(dims);
+    const bool dense = expert_ffn_dense_batch(dims.B) != 0;
+    // the expert kernel's x: bf16 x (B <= 32) or the dispatched pair rows
+    uint16_t *xk = dense ? seg<uint16_t>(ws, L.xb) : seg<uint16_t>(ws, L.xd);
     ExpertMaps maps;
-    if (!encode_expert_maps(&maps, dims, Wgate, Wup, Wdown, seg<uint16_t>(ws, L.h), seg<uint16_t>(ws, L.xb)))
-        return MOE_ERR_CUDA;
+    if (!encode_expert_maps(&maps, dims, Wgate, Wup, Wdown, seg<uint16_t>(ws, L.h), xk)) return MOE_ERR_CUDA;
     RouterMaps rmaps;
     if (!encode_router_maps(&rmaps, dims, x, Wg)) return MOE_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     Counters *ctr = seg<Counters>(ws, L.counters);
-    uint16_t *xb = seg<uint16_t>(ws, L.xb);
     float *logits = seg<float>(ws, L.logits);
     float *probs = seg<float>(ws, L.probs);
     int32_t *si = sel_idx ? sel_idx : seg<int32_t>(ws, L.sel_idx);
@@ -319,14 +309,18 @@ moe_status_t moe_layer_decode(const float *x, const float *Wg, const float *bias
     const moe_lists_t lists = ws_lists(ws, L);
     // B <= 32: the expert kernel starts streaming as soon as the activated
     // set is published (by the router for OEA and plain top-k, by the
-    // selection for XShare); larger batches start when the selection ends
-    const bool dense = expert_ffn_dense_batch(dims.B) != 0;
+    // selection for XShare).  Larger batches dispatch each pair's x row once
+    // the selection has built the lists, then stream.
     float *wd = dense ? seg<float>(ws, L.wd) : nullptr;
-    st = from_cuda(launch_layer_route(rmaps, x, bias, dims, rule, logits, xb, y, ctr, s));
+    st = from_cuda(launch_layer_route(rmaps, x, bias, dims, rule, logits, dense ? xk : nullptr, y, ctr, s));
     if (st != MOE_OK) return st;
     st = from_cuda(launch_layer_select(logits, probs, dims, rule, si, sw, lists, n_active, ctr, wd, dense, s));
     if (st != MOE_OK) return st;
-    return from_cuda(launch_expert_ffn(maps, xb, dims, lists, y, seg<uint16_t>(ws, L.h), wd, ctr, dense,
+    if (!dense) {
+        st = from_cuda(launch_ffn_prep(x, dims, nullptr, xk, nullptr, nullptr, lists, nullptr, true, s));
+        if (st != MOE_OK) return st;
+    }
+    return from_cuda(launch_expert_ffn(maps, xk, dims, lists, y, seg<uint16_t>(ws, L.h), wd, ctr, dense,
                                        layer_pub_target(dims, rule), s));
 }
 

@@ -24,8 +24,9 @@
 // publishes before the token lists exist (the router kernel for OEA and
 // plain top-k, the selection for XShare): the kernel is launched early,
 // reads the set from a published bit mask and starts streaming at once.
-// Larger batches use token tiles of up to 32 pairs, x rows gathered by four,
-// and pair-indexed H.
+// Larger batches use tiles of up to 32 (token, expert) pairs: the input
+// preparation copies each pair's x row (bf16) into a pair-indexed buffer in
+// the lists' order, so a tile's x rows are one swizzled box like H's.
 //
 // Per CTA: one producer warp issues TMA tensor copies (three-dimensional
 // boxes of 64-column chunks, 128-byte swizzle) into a ring of 32 KB weight
@@ -54,7 +55,6 @@ constexpr int D_CHUNKS = 4;               // 64-column chunks of d_ff per D stag
 constexpr int MAX_STAGES = 4;
 constexpr int W_BYTES = 32768;            // weight bytes per stage (both kinds)
 constexpr int UP_OFF = GU_ROWS * 128 * GU_CHUNKS;  // Wup tile after the Wgate tile
-constexpr int GATHER_COLS = 256;          // widest row box of a gather-by-four load
 // Two ring shapes: 4 stages with a 16 KB operand region (B <= 16), and 3
 // stages with 32 KB (larger batches).
 template <int ST, int OPB>
@@ -119,7 +119,6 @@ static_assert(sizeof(SharedCtl) <= CTL_BYTES, "SharedCtl does not fit its reserv
 struct ExpertArgs {
     const uint16_t *xb;
     int B, d, E, k, F;
-    int xbox;   // gather mode: columns per row box of the x map (<= GATHER_COLS)
     // dense mode (B <= TN): every stage works on all B tokens; gate/up stages
     // load all token rows of x in one box, H is token-indexed [slot][B][d_ff]
     // and the down epilogue weighs tokens by wd[slot][B]
@@ -191,16 +190,6 @@ __device__ __forceinline__ void tma_load_3d_stream(void *dst, const CUtensorMap 
         "l"(reinterpret_cast<unsigned long long>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar)), "l"(policy)
         : "memory");
 }
-// four rows r0..r3 (any order) from column `col` of a one-row-box map
-__device__ __forceinline__ void tma_gather4(void *dst, const CUtensorMap *map, int col, int r0, int r1, int r2,
-                                            int r3, unsigned long long *bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<unsigned long long>(map)), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3),
-        "r"(smem_u32(bar))
-        : "memory");
-}
 __device__ __forceinline__ int gu_chunks_of(int d) { return min(GU_CHUNKS, d / 64); }
 __device__ __forceinline__ int d_chunks_of(int F) { return min(D_CHUNKS, F / 64); }
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {
@@ -256,11 +245,9 @@ __device__ bool wait_phase(unsigned long long *bar, unsigned parity, SharedCtl *
 
 // ------------------------------------------------------------ producer --
 // The producer keeps one unit decoded ahead: while it issues the stages of
-// the current unit, the next unit's token indices (gathered gate/up) or its
-// gate/up completion count (down) are already in flight, so no global round
-// trip sits between two stages.
+// the current unit, the next unit's gate/up completion count (down units)
+// is already in flight, so no global round trip sits between two stages.
 struct UnitInfo : UnitRec {
-    int tok;  // GU, gather mode: token of this lane's x row (lane < n)
     int dep;  // D (lane 0): gate/up units of the expert already published
 };
 
@@ -323,9 +310,7 @@ __device__ bool fetch_unit(int j, int &win_base, int n_units, const ExpertArgs &
     }
     static_cast<UnitRec &>(ui) = ctl->urec[j - win_base];
     if (ui.type == UNIT_END) return false;
-    ui.tok = 0;
     ui.dep = 0;
-    if (ui.type == UNIT_GU && !a.dense) ui.tok = __ldg(a.tok + ui.p0 + min(lane, ui.n - 1));
     if (ui.type == UNIT_D && lane == 0) ui.dep = ld_acquire(&a.ctr->gu_done[ui.i_act]);
     return true;
 }
@@ -357,10 +342,8 @@ __device__ void producer(const ExpertArgs &a, const ExpertMaps &m, SharedCtl *ct
             unsigned char *wdst = slots + slot * RG::SLOT_BYTES;
             unsigned char *odst = wdst + W_BYTES;
             const int gc = gu_chunks_of(a.d), dc = d_chunks_of(a.F);
-            const int nq = (cur.n + 3) >> 2;  // gather-by-four loads of x rows
-            const int nhalf = (gc * 64 + a.xbox - 1) / a.xbox;  // gather loads per four tokens
-            const unsigned xbytes = a.dense ? static_cast<unsigned>(gc) * a.bpad * 128u
-                                            : static_cast<unsigned>(nq) * nhalf * 4u * a.xbox * 2u;
+            // x tile: all B token rows (dense mode) or the tile's TN pair rows
+            const unsigned xbytes = static_cast<unsigned>(gc) * (a.dense ? a.bpad : TN) * 128u;
             const unsigned bytes = cur.type == UNIT_GU ? 2u * gc * (GU_ROWS * 128) + xbytes
                                                        : dc * (D_ROWS * 128u) + dc * (a.hrows * 128u);
             if (lane == 0) {
@@ -380,22 +363,9 @@ __device__ void producer(const ExpertArgs &a, const ExpertMaps &m, SharedCtl *ct
                 const int grow = cur.e * a.F + cur.row0;
                 if (lane == 0) tma_load_3d_stream(wdst, &m.gate, 0, grow, s * gc, &ctl->full[slot], policy);
                 if (lane == 1) tma_load_3d_stream(wdst + UP_OFF, &m.up, 0, grow, s * gc, &ctl->full[slot], policy);
-                if (a.dense) {
-                    // all B token rows of this column range in one swizzled box
-                    if (lane == 2) tma_load_3d(odst, &m.x, 0, 0, s * gc, &ctl->full[slot]);
-                } else {
-                    // lane 2 + q loads the x rows of tokens 4q .. 4q + 3 (the
-                    // last token repeated past n)
-                    const int q = lane - 2;
-                    int t4[4];
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        t4[j] = __shfl_sync(0xffffffffu, cur.tok, min(4 * max(q, 0) + j, cur.n - 1));
-                    if (q >= 0 && q < nq)
-                        for (int hh = 0; hh < nhalf; ++hh)
-                            tma_gather4(odst + hh * (TN * a.xbox * 2) + q * 4 * a.xbox * 2, &m.x,
-                                        s * gc * 64 + hh * a.xbox, t4[0], t4[1], t4[2], t4[3], &ctl->full[slot]);
-                }
+                // x rows of this column range in one swizzled box: all B
+                // tokens (dense mode) or the tile's pairs of the dispatched x
+                if (lane == 2) tma_load_3d(odst, &m.x, 0, a.dense ? 0 : cur.p0, s * gc, &ctl->full[slot]);
             } else {
                 if (lane == 0)
                     tma_load_3d_stream(wdst, &m.down, 0, cur.e * a.d + cur.row0, s * dc, &ctl->full[slot], policy);
@@ -453,12 +423,11 @@ __device__ void producer(const ExpertArgs &a, const ExpertMaps &m, SharedCtl *ct
 }
 
 // ------------------------------------------------------------ consumers --
-// B operand rows: dense mode = token ids in a 128B-swizzled tile per 64
-// columns ([bpad][64] per chunk); otherwise the tile's gathered rows of
-// `xrow` bytes each.
+// B operand rows: a 128B-swizzled tile per 64 columns, x_tile bytes apart
+// ([rows][64] per chunk): token t in dense mode, the tile's pair n otherwise.
 template <int NT>
-__device__ __forceinline__ void gu_stage(uint32_t wbase, uint32_t xbase, int xbox, int dense_tile, int kvalid, int warp,
-                                         int lane, float (&acc_g)[4][4], float (&acc_u)[4][4]) {
+__device__ __forceinline__ void gu_stage(uint32_t wbase, uint32_t xbase, int x_tile, int kvalid, int warp, int lane,
+                                         float (&acc_g)[4][4], float (&acc_u)[4][4]) {
     const int nks = kvalid / 16;
 #pragma unroll
     for (int q = 0; q < (GU_CHUNKS * 4) / NCW; ++q) {
@@ -470,16 +439,12 @@ __device__ __forceinline__ void gu_stage(uint32_t wbase, uint32_t xbase, int xbo
         uint32_t g0, g1, g2, g3, u0, u1, u2, u3;
         ldsm_x4(swz(wbase + box * (GU_ROWS * 128), r, chunk), g0, g1, g2, g3);
         ldsm_x4(swz(wbase + UP_OFF + box * (GU_ROWS * 128), r, chunk), u0, u1, u2, u3);
-        const int xk = ks * 16 + ((lane >> 3) & 1) * 8;
         const int xchunk = ((ks & 3) << 1) + ((lane >> 3) & 1);
 #pragma unroll
         for (int np = 0; np < (NT + 1) / 2; ++np) {
             const int n = np * 16 + (lane & 7) + ((lane >> 4) << 3);
             uint32_t b0, b1, b2, b3;
-            // gather mode: x rows of xbox columns, one block of TN rows per xbox
-            ldsm_x4(dense_tile ? swz(xbase + box * dense_tile, n, xchunk)
-                               : xbase + (xk / xbox) * (TN * xbox * 2) + n * (xbox * 2) + (xk % xbox) * 2,
-                    b0, b1, b2, b3);
+            ldsm_x4(swz(xbase + box * x_tile, n, xchunk), b0, b1, b2, b3);
             mma_bf16(acc_g[2 * np], g0, g1, g2, g3, b0, b1);
             mma_bf16(acc_u[2 * np], u0, u1, u2, u3, b0, b1);
             if (2 * np + 1 < NT) {
@@ -520,8 +485,7 @@ __device__ __forceinline__ void stage_dispatch(const StageHdr &h, uint32_t wbase
                                                int warp, int lane, float (&acc_g)[4][4], float (&acc_u)[4][4]) {
     if (h.type == UNIT_GU) {
         const int gk = 64 * gu_chunks_of(a.d);
-        gu_stage<NT>(wbase, obase, a.xbox, a.dense ? a.bpad * 128 : 0, min(gk, a.d - h.s * gk), warp, lane, acc_g,
-                     acc_u);
+        gu_stage<NT>(wbase, obase, (a.dense ? a.bpad : TN) * 128, min(gk, a.d - h.s * gk), warp, lane, acc_g, acc_u);
     } else {
         const int dk = 64 * d_chunks_of(a.F);
         d_stage<NT>(wbase, obase, a.hrows, min(dk, a.F - h.s * dk), warp, lane, acc_g);
@@ -858,27 +822,57 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 }
 
 // ------------------------------------------------------------------ prep --
+// Input preparation of the expert kernel, chained before it:
+//  - x in bf16 [B][d] (dense mode) or, for larger batches, each pair's x
+//    row in bf16 at its list position p: xd[p] = x[tok[p]] (the dispatch);
+//  - y = 0 (standalone path; the layer path's router already zeroed it);
+//  - dense mode: the weight matrix wd[slot][B] from the lists;
+//  - the gate/up completion counts cleared (standalone path).
 struct PrepArgs {
     const float *x;
-    int n4, B;
-    uint16_t *xb;
-    float *y;
-    Counters *ctr;
+    int B, d;
+    uint16_t *xb;  // dense mode: x in bf16, or null
+    uint16_t *xd;  // larger batches: dispatched x rows, or null
+    float *y;      // zeroed when non-null
+    Counters *ctr; // gate/up counts cleared when non-null
     const int32_t *n_active, *offsets, *tok;
     const float *w;
     float *wd;  // dense weights [slot][B] (B <= 32), or null
 };
 
+__device__ __forceinline__ uint2 bf16x4(float4 v) {
+    const unsigned lo = static_cast<unsigned>(__bfloat16_as_ushort(__float2bfloat16_rn(v.x))) |
+                        (static_cast<unsigned>(__bfloat16_as_ushort(__float2bfloat16_rn(v.y))) << 16);
+    const unsigned hi = static_cast<unsigned>(__bfloat16_as_ushort(__float2bfloat16_rn(v.z))) |
+                        (static_cast<unsigned>(__bfloat16_as_ushort(__float2bfloat16_rn(v.w))) << 16);
+    return make_uint2(lo, hi);
+}
+
 __global__ void __launch_bounds__(256) ffn_prep_kernel(PrepArgs p) {
+    // the lists may come from the previous kernel (the layer path's selection)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int tid = blockIdx.x * blockDim.x + threadIdx.x, nthreads = gridDim.x * blockDim.x;
-    for (int i = tid; i < p.n4; i += nthreads) {
-        const float4 v = __ldg(reinterpret_cast<const float4 *>(p.x) + i);
-        const unsigned lo = static_cast<unsigned>(__bfloat16_as_ushort(__float2bfloat16_rn(v.x))) |
-                            (static_cast<unsigned>(__bfloat16_as_ushort(__float2bfloat16_rn(v.y))) << 16);
-        const unsigned hi = static_cast<unsigned>(__bfloat16_as_ushort(__float2bfloat16_rn(v.z))) |
-                            (static_cast<unsigned>(__bfloat16_as_ushort(__float2bfloat16_rn(v.w))) << 16);
-        reinterpret_cast<uint2 *>(p.xb)[i] = make_uint2(lo, hi);
-        reinterpret_cast<float4 *>(p.y)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    const int n4 = p.B * p.d / 4;
+    if (p.xb || p.y) {
+        for (int i = tid; i < n4; i += nthreads) {
+            const float4 v = __ldg(reinterpret_cast<const float4 *>(p.x) + i);
+            if (p.xb) reinterpret_cast<uint2 *>(p.xb)[i] = bf16x4(v);
+            if (p.y) reinterpret_cast<float4 *>(p.y)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
+    if (p.xd) {
+        // one thread per 4 columns of a pair row; rows of unused pairs skipped
+        const int na = *p.n_active;
+        const int total = (na > 0 && na <= 256) ? p.offsets[na] : 0;
+        const int q4 = p.d / 4;
+        for (int i = tid; i < total * q4; i += nthreads) {
+            const int pr = i / q4, c = i - pr * q4;
+            const int t = p.tok[pr];
+            if (t < 0 || t >= p.B) continue;
+            const float4 v = __ldg(reinterpret_cast<const float4 *>(p.x) + static_cast<size_t>(t) * q4 + c);
+            reinterpret_cast<uint2 *>(p.xd)[static_cast<size_t>(pr) * q4 + c] = bf16x4(v);
+        }
     }
     if (p.wd) {
         // wd[i][t] = weight of token t in active expert i's list, else 0:
@@ -894,9 +888,8 @@ __global__ void __launch_bounds__(256) ffn_prep_kernel(PrepArgs p) {
             if (t >= 0) p.wd[static_cast<size_t>(i) * p.B + t] = wv;
         }
     }
-    if (blockIdx.x == 0)
+    if (p.ctr && blockIdx.x == 0)
         for (int i = threadIdx.x; i < E_MAX; i += blockDim.x) p.ctr->gu_done[i] = 0;
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 int g_num_sms[64] = {0};
@@ -906,22 +899,19 @@ bool g_attr_small[64] = {false}, g_attr_large[64] = {false};
 
 int expert_ffn_h_rows(int B) { return B <= TN ? (B + 7) / 8 * 8 : TN; }
 int expert_ffn_dense_batch(int B) { return B <= TN ? 1 : 0; }
-int expert_ffn_gather_cols(int d) {
-    const int w = 64 * expert_ffn_gu_chunks(d);
-    return w < GATHER_COLS ? w : GATHER_COLS;
-}
 int expert_ffn_gu_rows() { return GU_ROWS; }
 int expert_ffn_d_rows() { return D_ROWS; }
 int expert_ffn_gu_chunks(int d) { return d / 64 < GU_CHUNKS ? d / 64 : GU_CHUNKS; }
 int expert_ffn_d_chunks(int F) { return F / 64 < D_CHUNKS ? F / 64 : D_CHUNKS; }
 
-cudaError_t launch_ffn_prep(const float *x, const moe_dims_t &d, uint16_t *xb, float *y, Counters *ctr,
-                            const moe_lists_t &l, float *wd, cudaStream_t s) {
+cudaError_t launch_ffn_prep(const float *x, const moe_dims_t &d, uint16_t *xb, uint16_t *xd, float *y,
+                            Counters *ctr, const moe_lists_t &l, float *wd, bool chained, cudaStream_t s) {
     PrepArgs p;
     p.x = x;
-    p.n4 = d.B * d.d / 4;
     p.B = d.B;
+    p.d = d.d;
     p.xb = xb;
+    p.xd = xd;
     p.y = y;
     p.ctr = ctr;
     p.n_active = l.n_active;
@@ -929,9 +919,22 @@ cudaError_t launch_ffn_prep(const float *x, const moe_dims_t &d, uint16_t *xb, f
     p.tok = l.tok;
     p.w = l.w;
     p.wd = wd;
-    const int blocks = (p.n4 + 255) / 256 > 0 ? min((p.n4 + 255) / 256, 1024) : 1;
-    ffn_prep_kernel<<<blocks, 256, 0, s>>>(p);
-    return cudaGetLastError();
+    const long long work = xd ? static_cast<long long>(d.B) * d.k * d.d / 4 : static_cast<long long>(d.B) * d.d / 4;
+    const int blocks = static_cast<int>(work / 256 + 1 < 1024 ? work / 256 + 1 : 1024);
+    if (!chained) {
+        ffn_prep_kernel<<<blocks, 256, 0, s>>>(p);
+        return cudaGetLastError();
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(blocks);
+    cfg.blockDim = dim3(256);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, ffn_prep_kernel, p);
 }
 
 cudaError_t launch_expert_ffn(const ExpertMaps &maps, const uint16_t *xb, const moe_dims_t &d,
@@ -967,7 +970,6 @@ cudaError_t launch_expert_ffn(const ExpertMaps &maps, const uint16_t *xb, const 
     a.dense = d.B <= TN ? 1 : 0;
     a.bpad = (d.B + 7) / 8 * 8;
     a.hrows = expert_ffn_h_rows(d.B);
-    a.xbox = expert_ffn_gather_cols(d.d);
     a.early = (early && a.dense) ? 1 : 0;
     a.pub_target = pub_target;
     a.wd = wd;

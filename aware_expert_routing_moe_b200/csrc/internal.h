@@ -54,7 +54,7 @@ enum DeviceError : int32_t {
 struct WsLayout {
     size_t counters, logits, probs, sel_idx, sel_w;
     size_t n_active, active, offsets, tok, w;
-    size_t xb, h, wd;
+    size_t xb, xd, h, wd;
     size_t total;
 };
 
@@ -66,6 +66,10 @@ inline int active_slots(const moe_dims_t &d) { return d.E < d.B * d.k ? d.E : d.
 inline size_t h_scratch_bytes(const moe_dims_t &d) {
     const size_t F = d.d_ff;
     return d.B <= 32 ? static_cast<size_t>(active_slots(d)) * d.B * F * 2 : static_cast<size_t>(d.B) * d.k * F * 2;
+}
+// Bytes of the dispatched x rows [B*k][d] bf16 (B > 32 only).
+inline size_t xd_bytes(const moe_dims_t &d) {
+    return d.B <= 32 ? 0 : static_cast<size_t>(d.B) * d.k * d.d * 2;
 }
 // Bytes of the dense weight matrix [slot][B] fp32 (B <= 32 only).
 inline size_t wd_bytes(const moe_dims_t &d) {
@@ -108,14 +112,17 @@ cudaError_t launch_layer_select(const float *logits, float *probs, const moe_dim
 // Value of every ctr->pubs[c].pub once the activated set of a layer call is
 // published.
 int layer_pub_target(const moe_dims_t &d, const moe_reselect_t &rule);
-// Standalone expert FFN: x -> bf16, y = 0, counters cleared and, for
-// B <= 32, the dense weights built from the lists.
-cudaError_t launch_ffn_prep(const float *x, const moe_dims_t &d, uint16_t *xb, float *y,
-                            Counters *ctr, const moe_lists_t &l, float *wd, cudaStream_t s);
+// Input preparation of the expert kernel (all pointers may be null, each
+// step is skipped then): x -> bf16 (xb, dense mode), each pair's x row ->
+// xd (larger batches), y = 0, gate/up counts cleared and, for B <= 32, the
+// dense weights built from the lists.  chained: launched with programmatic
+// dependent launch after the kernel that writes the lists.
+cudaError_t launch_ffn_prep(const float *x, const moe_dims_t &d, uint16_t *xb, uint16_t *xd, float *y,
+                            Counters *ctr, const moe_lists_t &l, float *wd, bool chained, cudaStream_t s);
 
-// TMA descriptors of the expert kernel: the three weight tensors and the H
-// scratch as (64-column chunk, row, chunk index) boxes, and x in bf16 as
-// single rows for gather-by-four loads.
+// TMA descriptors of the expert kernel: the three weight tensors, the H
+// scratch and the bf16 x rows (xb for B <= 32, the dispatched pair rows xd
+// above) as (64-column chunk, row, chunk index) boxes.
 struct ExpertMaps {
     CUtensorMap gate, up, down, h, x;
 };
@@ -128,15 +135,14 @@ cudaError_t launch_expert_ffn(const ExpertMaps &maps, const uint16_t *xb,
                               cudaStream_t s);
 int expert_ffn_h_rows(int B);         // rows of one H box
 int expert_ffn_dense_batch(int B);    // 1 if gate/up stages load all B token rows at once
-int expert_ffn_gather_cols(int d);    // columns of one x row box in gather mode
 int expert_ffn_gu_rows();             // rows of Wgate / Wup per gate-up unit
 int expert_ffn_d_rows();              // rows of Wdown per down unit
 int expert_ffn_gu_chunks(int d);      // 64-column chunks of d per gate-up stage
 int expert_ffn_d_chunks(int d_ff);    // 64-column chunks of d_ff per down stage
 
 // Builds the expert kernel's TMA descriptors (weights, H scratch at `h`,
-// bf16 x at `xb`).
+// bf16 x at `x`: xb [B][d] for B <= 32, xd [B*k][d] above).
 bool encode_expert_maps(ExpertMaps *m, const moe_dims_t &d, const uint16_t *Wgate, const uint16_t *Wup,
-                        const uint16_t *Wdown, const uint16_t *h, const uint16_t *xb);
+                        const uint16_t *Wdown, const uint16_t *h, const uint16_t *x);
 
 }  // namespace moe

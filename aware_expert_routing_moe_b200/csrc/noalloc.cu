@@ -26,14 +26,15 @@ unsigned char *g_scratch_addr[MAX_DEVICES] = {};
 size_t align256(size_t v) { return (v + 255) / 256 * 256; }
 
 struct NoallocLayout {
-    size_t counters, xb, h, wd, total;
+    size_t counters, xb, xd, h, wd, total;
 };
 
 NoallocLayout noalloc_layout(const moe_dims_t &d) {
     NoallocLayout L;
     size_t o = 0;
     L.counters = o; o += align256(sizeof(Counters));
-    L.xb = o;       o += align256(static_cast<size_t>(d.B) * d.d * 2);
+    L.xb = o;       o += align256(expert_ffn_dense_batch(d.B) ? static_cast<size_t>(d.B) * d.d * 2 : 0);
+    L.xd = o;       o += align256(xd_bytes(d));
     L.h = o;        o += align256(h_scratch_bytes(d));
     L.wd = o;       o += align256(wd_bytes(d));
     L.total = o;
@@ -96,15 +97,19 @@ extern "C" moe_status_t moe_expert_ffn_noalloc(const float *x, const uint16_t *W
     if (st != MOE_OK) return st;
 
     Counters *ctr = reinterpret_cast<Counters *>(scratch + L.counters);
-    uint16_t *xb = reinterpret_cast<uint16_t *>(scratch + L.xb);
+    const bool dense = expert_ffn_dense_batch(dims.B) != 0;
+    // the expert kernel's x: bf16 x (B <= 32) or the dispatched pair rows
+    uint16_t *xk = reinterpret_cast<uint16_t *>(scratch + (dense ? L.xb : L.xd));
     uint16_t *h = reinterpret_cast<uint16_t *>(scratch + L.h);
-    float *wd = expert_ffn_dense_batch(dims.B) ? reinterpret_cast<float *>(scratch + L.wd) : nullptr;
+    float *wd = dense ? reinterpret_cast<float *>(scratch + L.wd) : nullptr;
     ExpertMaps maps;
-    if (!encode_expert_maps(&maps, dims, Wgate, Wup, Wdown, h, xb)) return MOE_ERR_CUDA;
+    if (!encode_expert_maps(&maps, dims, Wgate, Wup, Wdown, h, xk)) return MOE_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     // the prep kernel clears the per-expert counters the expert kernel needs
     // at zero and rebuilds x, the dense weights and (in the kernel) H
-    if (launch_ffn_prep(x, dims, xb, y, ctr, lists, wd, s) != cudaSuccess) return MOE_ERR_CUDA;
-    if (launch_expert_ffn(maps, xb, dims, lists, y, h, wd, ctr, false, 0, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_ffn_prep(x, dims, dense ? xk : nullptr, dense ? nullptr : xk, y, ctr, lists, wd, false, s) !=
+        cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (launch_expert_ffn(maps, xk, dims, lists, y, h, wd, ctr, false, 0, s) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;
 }

@@ -673,8 +673,8 @@ __device__ __forceinline__ float comp(const float4 &v, int u) {
     return u == 0 ? v.x : u == 1 ? v.y : u == 2 ? v.z : v.w;
 }
 
-// Layer path: x -> bf16 copy for the expert kernel, y = 0 (grid-stride over
-// the blocks of the launch).
+// Layer path: x -> bf16 copy for the expert kernel (when xb is non-null),
+// y = 0 (grid-stride over the blocks of the launch).
 __device__ void layer_prep(const float *__restrict__ x, int B, int d, uint16_t *__restrict__ xb,
                            float *__restrict__ y) {
     const int n4 = B * d / 4;
@@ -686,7 +686,7 @@ __device__ void layer_prep(const float *__restrict__ x, int B, int d, uint16_t *
                             (static_cast<unsigned>(__bfloat16_as_ushort(__float2bfloat16_rn(v.y))) << 16);
         const unsigned hi = static_cast<unsigned>(__bfloat16_as_ushort(__float2bfloat16_rn(v.z))) |
                             (static_cast<unsigned>(__bfloat16_as_ushort(__float2bfloat16_rn(v.w))) << 16);
-        reinterpret_cast<uint2 *>(xb)[i] = make_uint2(lo, hi);
+        if (xb) reinterpret_cast<uint2 *>(xb)[i] = make_uint2(lo, hi);
         reinterpret_cast<float4 *>(y)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
 }

@@ -183,17 +183,17 @@ moe_status_t moe_layer_decode(const float *x, const float *Wg, const float *bias
  * same arguments as moe_expert_ffn minus the workspace, and allocates
  * nothing: its scratch (the expert kernel's counters, x in bf16 and the
  * SwiGLU activations) lives in a file-scope static device array of
- * MOE_NOALLOC_SCRATCH_BYTES (16 MiB), which every GPU that loads the library
+ * MOE_NOALLOC_SCRATCH_BYTES (32 MiB), which every GPU that loads the library
  * holds until the process exits.  It calls no cudaMalloc, cudaFree or other
  * allocating routine.
  *
- *  - Size limit: the scratch must fit in MOE_NOALLOC_SCRATCH_BYTES: about
- *    B*d*2 bytes of bf16 x plus the SwiGLU activations, which take
- *    min(E, B*k)*B*d_ff*2 bytes (+ min(E, B*k)*B*4 for dense weights) when
- *    B <= 32 and B*k*d_ff*2 bytes above, plus about 3 KB of counters, each
- *    part rounded up to 256 bytes.  Larger dims return MOE_ERR_UNSUPPORTED
- *    before anything is enqueued.  The Qwen3-30B-A3B- and Qwen3-235B-A22B-
- *    shaped layers fit for every B <= 256.
+ *  - Size limit: the scratch must fit in MOE_NOALLOC_SCRATCH_BYTES: when
+ *    B <= 32, B*d*2 bytes of bf16 x, min(E, B*k)*B*d_ff*2 bytes of SwiGLU
+ *    activations and min(E, B*k)*B*4 bytes of dense weights; above,
+ *    B*k*d*2 bytes of per-pair x rows and B*k*d_ff*2 bytes of activations;
+ *    plus about 3 KB of counters, each part rounded up to 256 bytes.  Larger
+ *    dims return MOE_ERR_UNSUPPORTED before anything is enqueued.  The
+ *    Qwen3-30B-A3B- and Qwen3-235B-A22B-shaped layers fit for every B <= 256.
  *  - Set-up: the first call on a device looks up the array's device address
  *    (cudaGetSymbolAddress, with that device current) and caches it; make
  *    that first call before any stream capture begins.
@@ -205,7 +205,7 @@ moe_status_t moe_layer_decode(const float *x, const float *Wg, const float *bias
  *  - A bounded wait that expires inside the kernels is recorded in the
  *    array but not reported; use moe_expert_ffn + moe_check_error to
  *    diagnose such a failure. */
-#define MOE_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+#define MOE_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
 moe_status_t moe_expert_ffn_noalloc(const float *x, const uint16_t *Wgate,
                                     const uint16_t *Wup, const uint16_t *Wdown,
                                     moe_dims_t dims, moe_lists_t lists, float *y,
