@@ -39,6 +39,12 @@
  *    slots, short sets padded with (-1, 0);
  *  - XShare scores sum each token's top-k gate probabilities, the budget is
  *    min(M, |union of top-k sets|), ties to the lower index;
+ *  - Lynx affinity binning: a token's confidence is the gap between the
+ *    probabilities of its two top-ranked experts; bins of width k/E,
+ *    min(32, ceil(E/k)) of them; expert scores sum 2^bin over the tokens
+ *    whose top-k holds the expert; the critical set is the shortest prefix
+ *    of the score order (at least k long) that holds every token's rank-0
+ *    expert; each token takes its first k experts inside it;
  *  - gate weights are renormalised over the chosen set (all modes);
  *  - the expert FFN is SwiGLU: down( silu(gate x) * (up x) ), in fp64.
  *
@@ -57,6 +63,7 @@
 #define ORACLE_MODE_NONE 0
 #define ORACLE_MODE_OEA 1
 #define ORACLE_MODE_XSHARE 2
+#define ORACLE_MODE_AFFINITY 3
 
 /* ---------------------------------------------------------------- exp ---
  * exp_spec(x) for x in [-87, 0] (softmax arguments are l - max(l) <= 0).
@@ -217,6 +224,16 @@ void oracle_route(const float *x, const float *Wg, const float *bias,
  *            with the largest s (ties to the lower index) -- the exact
  *            maximiser of the modular objective sum_{e in S} s_e;
  *            sel_b = the first k experts of the order that lie in S.
+ *   AFFINITY : [LX] section 2.2 (confidence analyzer, adaptive expert
+ *            scorer, expert remapper) and section 2.1 (rank-0 dominates).
+ *            c_b = p[b][r0] - p[b][r1] (fp32), r0, r1 the token's first two
+ *            experts; nb = min(32, ceil(E/k)) bins of width k/E: bin_b =
+ *            the largest j < nb with j*k <= c_b*E (fp32 product);
+ *            s_e = sum over b with e in T_b of 2^bin_b (exact integers);
+ *            U_base ordered by s descending, ties to the lower index;
+ *            M = max(k, 1 + the largest position of any r0(b) in that
+ *            order); S = its first M experts; sel_b = the first k experts
+ *            of the token's order that lie in S (always k of them).
  * Weights are renormalised over the chosen set in every mode. */
 void oracle_reselect(const float *logits, const float *probs,
                      int B, int E, int k, int mode, int k0, int budget,
@@ -274,6 +291,49 @@ void oracle_reselect(const float *logits, const float *probs,
         }
         free(s);
         free(ubase);
+    } else if (mode == ORACLE_MODE_AFFINITY) {
+        int nb = (E + k - 1) / k;
+        if (nb > 32) nb = 32;
+        long long *s = (long long *)calloc((size_t)E, sizeof(long long));
+        unsigned char *ubase = (unsigned char *)calloc((size_t)E, 1);
+        int *pos = (int *)malloc(sizeof(int) * (size_t)E);
+        for (int b = 0; b < B; ++b) {
+            const int *ord = order + (size_t)b * E;
+            const float *p = probs + (size_t)b * E;
+            float c = E > 1 ? p[ord[0]] - p[ord[1]] : p[ord[0]];
+            float cE = c * (float)E;
+            int bin = 0;
+            for (int j = nb - 1; j > 0; --j)
+                if ((float)(j * k) <= cE) { bin = j; break; }
+            for (int j = 0; j < k; ++j) {
+                s[ord[j]] += 1LL << bin;
+                ubase[ord[j]] = 1;
+            }
+        }
+        /* position of each expert of U_base in the score order */
+        for (int e = 0; e < E; ++e) {
+            pos[e] = 0;
+            if (!ubase[e]) continue;
+            for (int e2 = 0; e2 < E; ++e2)
+                if (ubase[e2] && (s[e2] > s[e] || (s[e2] == s[e] && e2 < e))) ++pos[e];
+        }
+        int M = k;
+        for (int b = 0; b < B; ++b) {
+            int r0 = order[(size_t)b * E];
+            if (pos[r0] + 1 > M) M = pos[r0] + 1;
+        }
+        for (int e = 0; e < E; ++e) inset[e] = ubase[e] && pos[e] < M;
+        for (int b = 0; b < B; ++b) {
+            const int *ord = order + (size_t)b * E;
+            int *sel = sel_idx + (size_t)b * k;
+            int n = 0;
+            for (int j = 0; j < E && n < k; ++j)
+                if (inset[ord[j]]) sel[n++] = ord[j];
+            while (n < k) sel[n++] = -1;
+        }
+        free(s);
+        free(ubase);
+        free(pos);
     } else {
         for (int b = 0; b < B; ++b)
             for (int j = 0; j < k; ++j) sel_idx[(size_t)b * k + j] = order[(size_t)b * E + j];

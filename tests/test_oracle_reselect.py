@@ -262,3 +262,107 @@ def test_lists_reconstruct_selection(oracle_lib, mode, k0, budget):
     want = {(b, int(sel[b, j])): w[b, j] for b in range(B) for j in range(k) if sel[b, j] >= 0}
     assert rebuilt == want
     assert np.all(li["tok"][total:] == -1) and np.all(li["w"][total:] == 0)
+
+
+# ------------------------------------------------------------------ Lynx --
+# Affinity binning ("Lynx: Enabling Efficient MoE Inference through Dynamic
+# Batch-Aware Expert Selection", sections 2.1-2.2): a confidence per token
+# from the gap of its top-ranked experts, bins fixed by k/E, exponentially
+# weighted expert scores, a minimal critical set, and every token keeping
+# exactly k experts inside it.  Pinned by invariants the reading fixes, the
+# closed forms B = 1 and identical tokens (standard top-k), and two
+# hand-worked cases.
+AFFINITY = 3
+
+
+def check_affinity(logits, probs, sel, w, k):
+    order = _rank_order(logits)
+    B = logits.shape[0]
+    u_base = set(order[:, :k].ravel().tolist())
+    S = set(sel.ravel().tolist())
+    assert -1 not in S                                  # exactly k per token
+    assert S <= u_base
+    assert len(S) >= k
+    assert {int(order[b, 0]) for b in range(B)} <= S    # rank-0 experts survive
+    for b in range(B):
+        inside = [int(e) for e in order[b] if int(e) in S][:k]
+        assert sel[b].tolist() == inside                # first k of its order in S
+    _check_weights(probs, sel, w)
+
+
+@pytest.mark.parametrize("seed", range(6))
+@pytest.mark.parametrize("B,E,k", [(4, 16, 4), (16, 128, 8), (32, 64, 8), (7, 256, 16)])
+def test_affinity_invariants_random(oracle_lib, seed, B, E, k):
+    rng = np.random.default_rng(300 + seed)
+    logits, probs = _random_router(rng, B, E)
+    sel, w = oracle_lib.reselect(logits, probs, k, AFFINITY)
+    check_affinity(logits, probs, sel, w, k)
+    # never more experts than standard routing activates
+    s_none, _ = oracle_lib.reselect(logits, probs, k, NONE)
+    assert len(set(sel.ravel().tolist())) <= len(set(s_none.ravel().tolist()))
+
+
+@pytest.mark.parametrize("shape,B", [("q30b", 16), ("q30b", 64), ("e64", 16)])
+def test_affinity_invariants_layers(oracle_lib, shape, B):
+    S = ms.SHAPES[shape]
+    L = ms.make_weights(S, 0, experts=False)
+    x = ms.make_tokens(S, B, 0)
+    logits, probs, ti, tw = oracle_lib.route(x, L["Wg"], L["bias"], S.k)
+    sel, w = oracle_lib.reselect(logits, probs, S.k, AFFINITY)
+    check_affinity(logits, probs, sel, w, S.k)
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_affinity_closed_forms_are_standard_topk(oracle_lib, seed):
+    rng = np.random.default_rng(80 + seed)
+    # one token: its k experts are the whole union, so the set cannot shrink
+    logits, probs = _random_router(rng, 1, 64)
+    s_none, w_none = oracle_lib.reselect(logits, probs, 8, NONE)
+    s_a, w_a = oracle_lib.reselect(logits, probs, 8, AFFINITY)
+    assert np.array_equal(s_none, s_a) and np.array_equal(w_none.view(np.uint32), w_a.view(np.uint32))
+    # identical tokens: the union is one token's top-k
+    logits5 = np.repeat(logits, 5, axis=0)
+    probs5 = np.repeat(probs, 5, axis=0)
+    s_none, w_none = oracle_lib.reselect(logits5, probs5, 8, NONE)
+    s_a, w_a = oracle_lib.reselect(logits5, probs5, 8, AFFINITY)
+    assert np.array_equal(s_none, s_a) and np.array_equal(w_none.view(np.uint32), w_a.view(np.uint32))
+
+
+def test_affinity_hand_worked_example(oracle_lib):
+    # E = 8, k = 2: 4 bins of width 2/8 on the gap c of the two top
+    # probabilities; bin = largest j < 4 with 2 j <= 8 c.
+    #  token 0: order 0 1 3 2 ..., c = .75 - .125 = .625, 8c = 5 -> bin 2 (weight 4)
+    #  token 1: order 1 2 0 3 ..., c = .3125 - .25 = .0625, 8c = .5 -> bin 0 (weight 1)
+    #  token 2: order 0 3 1 2 ..., c = .5 - .25 = .25, 8c = 2 -> bin 1 (weight 2: 2 <= 2 counts)
+    # scores (top-2 memberships): e0 = 4 + 2 = 6, e1 = 4 + 1 = 5, e2 = 1, e3 = 2
+    # score order e0 e1 e3 e2; rank-0 experts e0 e1 e0 sit at positions 0 1 0
+    # -> M = max(2, 2) = 2, S = {0, 1}; each token takes its first two in S.
+    logits = np.array([[8, 7, 1, 2, 0, -1, -2, -3],
+                       [5, 9, 8, 1, 0, -1, -2, -3],
+                       [9, 2, 1, 8, 0, -1, -2, -3]], np.float32)
+    probs = np.array([[.75, .125, .03125, .0625, 0, 0, 0, 0],
+                      [.125, .3125, .25, .0625, 0, 0, 0, 0],
+                      [.5, .125, .0625, .25, 0, 0, 0, 0]], np.float32)
+    sel, w = oracle_lib.reselect(logits, probs, 2, AFFINITY)
+    assert sel.tolist() == [[0, 1], [1, 0], [0, 1]]
+    expect = np.array([[.75 / .875, .125 / .875], [.3125 / .4375, .125 / .4375], [.5 / .625, .125 / .625]],
+                      np.float32)
+    assert np.allclose(w, expect, rtol=2e-7, atol=0)
+    # standard routing would activate four experts
+    s_none, _ = oracle_lib.reselect(logits, probs, 2, NONE)
+    assert sorted(set(s_none.ravel().tolist())) == [0, 1, 2, 3]
+
+
+def test_affinity_hand_worked_tie(oracle_lib):
+    # E = 8, k = 2, both tokens in bin 0 (zero gaps).
+    #  token 0: order 5 2 0 1 ...; token 1: order 2 6 7 5 ...
+    # scores e2 = 2, e5 = 1, e6 = 1: the tie e5/e6 goes to the lower index,
+    # so the order is e2 e5 e6 and the rank-0 experts (e5, e2) sit at 1, 0:
+    # M = 2, S = {2, 5}.  (The opposite tie rule would give S = {2, 6, 5}.)
+    logits = np.array([[4, 3, 8, 1, 0, 9, -1, -2],
+                       [0, -1, 9, -2, -3, 6, 8, 7]], np.float32)
+    probs = np.array([[.05, .04, .25, .02, .01, .25, 0, 0],
+                      [.01, 0, .25, 0, 0, .125, .25, .2]], np.float32)
+    sel, w = oracle_lib.reselect(logits, probs, 2, AFFINITY)
+    assert sel.tolist() == [[5, 2], [2, 5]]
+    assert np.allclose(w, [[.5, .5], [.25 / .375, .125 / .375]], rtol=2e-7, atol=0)
