@@ -8,7 +8,9 @@
 //  route_topk_kernel    : warp per token: softmax (step 2) + top-k (step 3)
 //      with a warp-shuffle reduction and register-resident keys.
 //  reselect_kernel      : one CTA for the whole batch: (softmax +) top-k,
-//      OEA / XShare re-selection, renormalised weights, per-expert token
+//      OEA / XShare / affinity-binning re-selection ("Lynx: Enabling
+//      Efficient MoE Inference through Dynamic Batch-Aware Expert
+//      Selection", section 2.2), renormalised weights, per-expert token
 //      lists and, for small batches, the dense weight matrix.
 //
 // Every floating-point step that decides an index is written with explicit
@@ -239,8 +241,9 @@ struct ReselectArgs {
     moe_lists_t lists;
     int32_t *n_active_copy;
     Counters *ctr;  // layer path: the expert kernel's counters (else null)
-    // layer path, XShare, expert kernel started early: publish the batch
-    // set (every copy of ctr->pubs: mask, then pub + 1) as soon as it is known
+    // layer path, XShare or affinity binning, expert kernel started early:
+    // publish the batch set (every copy of ctr->pubs: mask, then pub + 1)
+    // as soon as it is known
     int publish;
     // let the dependent kernel launch before waiting for the previous one
     // (the expert kernel started early); otherwise once that wait returns
@@ -372,13 +375,18 @@ __device__ void reselect_body(const ReselectArgs &a, unsigned char *smem_raw) {
     __shared__ float s_score[E_MAX];
     __shared__ int s_off[E_MAX];
     __shared__ int s_rank[E_MAX];  // expert -> active slot (publishing path)
-    __shared__ unsigned ukept[E_MAX / 32], ubase[E_MAX / 32], sbits[E_MAX / 32];
+    __shared__ unsigned ukept[E_MAX / 32], ubase[E_MAX / 32], sbits[E_MAX / 32], r0bits[E_MAX / 32];
+    __shared__ unsigned long long s_aff[E_MAX];  // affinity scores (exact integers)
+    __shared__ int s_pos[E_MAX];                 // position in the affinity score order
+    __shared__ int s_M;
     __shared__ int wsum[9];
     __shared__ int s_nact;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     for (int i = tid; i < 2 * E * BW; i += blockDim.x) ASSIGN[i] = 0u;  // and TMEMB
-    if (tid < E_MAX / 32) ukept[tid] = ubase[tid] = sbits[tid] = 0u;
+    if (tid < E_MAX / 32) ukept[tid] = ubase[tid] = sbits[tid] = r0bits[tid] = 0u;
+    for (int i = tid; i < E_MAX; i += blockDim.x) s_aff[i] = 0ull;
+    if (tid == 0) s_M = k;
     __syncthreads();
 
     const int mode = a.mode;
@@ -420,6 +428,25 @@ __device__ void reselect_body(const ReselectArgs &a, unsigned char *smem_raw) {
             const int e = warp_argmax<NI>(ord, cand, lane);
             if (lane == j) mye = e;
             if (mode == MOE_RESELECT_NONE) take_slot(j, warp_fetch<NI>(p, e), lane, sum, myp);
+        }
+        if (mode == MOE_RESELECT_AFFINITY) {
+            // confidence = gap of the two top probabilities, in bins of
+            // width k/E (min(32, ceil(E/k)) of them); each of the token's
+            // top-k experts scores 2^bin
+            const int r0 = __shfl_sync(FULL, mye, 0);
+            const int r1e = k >= 2 ? __shfl_sync(FULL, mye, 1) : warp_argmax<NI>(ord, cand, lane);
+            const float p0 = warp_fetch<NI>(p, r0);
+            const float c = r1e >= 0 ? __fsub_rn(p0, warp_fetch<NI>(p, r1e)) : p0;
+            const float cE = __fmul_rn(c, static_cast<float>(E));
+            const int nb = min(32, (E + k - 1) / k);
+            int bin = 0;
+            for (int j = nb - 1; j > 0; --j)
+                if (static_cast<float>(j * k) <= cE) {
+                    bin = j;
+                    break;
+                }
+            if (lane < k) atomicAdd(&s_aff[mye], 1ull << bin);
+            if (lane == 0) atomicOr(&r0bits[r0 >> 5], 1u << (r0 & 31));
         }
         if (lane < r1) {
             T[b * k + lane] = mye;
@@ -463,12 +490,35 @@ __device__ void reselect_body(const ReselectArgs &a, unsigned char *smem_raw) {
         __syncthreads();
     }
 
+    // ---- affinity binning: the critical set = the shortest prefix of the
+    // score order (score descending, ties to the lower index), at least k
+    // long, that holds every token's rank-0 expert
+    if (mode == MOE_RESELECT_AFFINITY) {
+        const bool in_base = tid < E && ((ubase[tid >> 5] >> (tid & 31)) & 1u);
+        if (in_base) {
+            const unsigned long long se = s_aff[tid];
+            int pos = 0;
+#pragma unroll 1
+            for (int e2 = 0; e2 < E; ++e2) {
+                if (!((ubase[e2 >> 5] >> (e2 & 31)) & 1u)) continue;
+                const unsigned long long s2 = s_aff[e2];
+                pos += (s2 > se || (s2 == se && e2 < tid)) ? 1 : 0;
+            }
+            s_pos[tid] = pos;
+            if ((r0bits[tid >> 5] >> (tid & 31)) & 1u) atomicMax(&s_M, pos + 1);
+        }
+        __syncthreads();
+        if (in_base && s_pos[tid] < s_M) atomicOr(&sbits[tid >> 5], 1u << (tid & 31));
+        __syncthreads();
+    }
+
     // ---- the activated set is now fixed: OEA = union of kept sets, XShare =
-    // the batch set, NONE = union of top-k sets.  Map experts to active
-    // slots for the dense weights; in XShare with the expert kernel started
-    // early, publish the set (OEA and NONE sets are published by the router).
+    // the batch set, affinity binning = the critical set, NONE = union of
+    // top-k sets.  Map experts to active slots for the dense weights; in
+    // XShare and affinity binning with the expert kernel started early,
+    // publish the set (OEA and NONE sets are published by the router).
     if (a.publish || dense_w) {
-        const unsigned *abits = (mode == MOE_RESELECT_OEA) ? ukept : (mode == MOE_RESELECT_XSHARE ? sbits : ubase);
+        const unsigned *abits = (mode == MOE_RESELECT_OEA) ? ukept : (mode == MOE_RESELECT_NONE ? ubase : sbits);
         if (warp == 0) {
             const unsigned word = lane < E_MAX / 32 ? abits[lane] : 0u;
             int incl = __popc(word);
@@ -1024,7 +1074,8 @@ cudaError_t launch_reselect(const float *logits, const float *probs, const moe_d
 
 int layer_pub_target(const moe_dims_t &d, const moe_reselect_t &rule) {
     const GemvShape sh = gemv_shape(d);
-    return (d.B + sh.tpb - 1) / sh.tpb + (rule.mode == MOE_RESELECT_XSHARE ? 1 : 0);
+    const bool sel_publishes = rule.mode == MOE_RESELECT_XSHARE || rule.mode == MOE_RESELECT_AFFINITY;
+    return (d.B + sh.tpb - 1) / sh.tpb + (sel_publishes ? 1 : 0);
 }
 
 cudaError_t launch_layer_route(const RouterMaps &maps, const float *x, const float *bias, const moe_dims_t &d,
@@ -1045,7 +1096,7 @@ cudaError_t launch_layer_select(const float *logits, float *probs, const moe_dim
                                 Counters *ctr, float *wd, bool early, cudaStream_t s) {
     ReselectArgs a = make_reselect_args(logits, probs, true, d, rule, sel_idx, sel_w, l, n_active_copy);
     a.ctr = ctr;
-    a.publish = (early && rule.mode == MOE_RESELECT_XSHARE) ? 1 : 0;
+    a.publish = (early && (rule.mode == MOE_RESELECT_XSHARE || rule.mode == MOE_RESELECT_AFFINITY)) ? 1 : 0;
     a.early_dependents = early ? 1 : 0;
     a.wd = wd;
     const size_t smem = reselect_smem(d, &a.cache_rows);

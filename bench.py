@@ -57,6 +57,7 @@ WORKLOADS = {
     "q235b_b16_oea4": dict(shape="q235b", B=16, mode=1, k0=4, budget=0, rule="OEA k0=4"),
     "spec_xshare32": dict(shape="q30b", B=32, mode=2, k0=0, budget=32, rule="XShare budget=32",
                           kind="spec"),
+    "q30b_b16_affinity": dict(shape="q30b", B=16, mode=3, k0=0, budget=0, rule="Lynx affinity binning"),
 }
 
 # DRAM bytes (read + write) per launch of the expert kernel from an ncu
@@ -398,7 +399,8 @@ SWEEP = {
     "e64": [(16, 1, 4, 0, "normal"), (16, 0, 0, 0, "normal")],
     "q30b": [(b, m, k0, 0, "normal") for b in (1, 4, 16, 32, 64) for (m, k0) in ((0, 0), (1, 4))]
             + [(16, 1, k0, 0, "normal") for k0 in (2, 6, 8)]
-            + [(32, 0, 0, 0, "spec")] + [(32, 2, 0, m, "spec") for m in (24, 32, 48)],
+            + [(32, 0, 0, 0, "spec")] + [(32, 2, 0, m, "spec") for m in (24, 32, 48)]
+            + [(16, 3, 0, 0, "normal"), (64, 3, 0, 0, "normal"), (32, 3, 0, 0, "spec")],
     "q235b": [(b, 1, 4, 0, "normal") for b in (1, 8, 16, 64)] + [(16, 0, 0, 0, "normal")],
 }
 
@@ -461,7 +463,7 @@ def run_sweep(args):
             n_active = int(nact_t[0].item())
             total, _ = algorithmic_bytes(S, B, n_active)
             gbs = total / (us * 1e-6) / 1e9
-            line = {"shape": shape, "B": B, "mode": ["NONE", "OEA", "XShare"][mode], "k0": k0, "budget": budget,
+            line = {"shape": shape, "B": B, "mode": ["NONE", "OEA", "XShare", "Affinity"][mode], "k0": k0, "budget": budget,
                     "tokens": kind, "n_active": n_active, "us": us, "bytes": total, "GBps": gbs,
                     "frac_8tbs": gbs / NOMINAL_HBM_GBS, "frac_measured": gbs / hbm_peak}
             if not args.no_cpu_baseline:

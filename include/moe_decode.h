@@ -69,7 +69,8 @@ typedef enum {
 typedef enum {
     MOE_RESELECT_NONE = 0,    /* standard top-k routing */
     MOE_RESELECT_OEA = 1,     /* keep top-k0, fill from the batch union of kept sets */
-    MOE_RESELECT_XSHARE = 2   /* budgeted greedy batch selection, then top-k within it */
+    MOE_RESELECT_XSHARE = 2,  /* budgeted greedy batch selection, then top-k within it */
+    MOE_RESELECT_AFFINITY = 3 /* Lynx affinity binning: confidence bins, critical set, remap */
 } moe_reselect_mode_t;
 
 /* Layer dimensions: B tokens, hidden size d, E experts, top-k k,
@@ -79,7 +80,18 @@ typedef struct {
 } moe_dims_t;
 
 /* Re-selection rule: mode (moe_reselect_mode_t); k0 (OEA: 1 <= k0 <= k);
- * budget (XShare: k <= budget <= E).  Unused fields are ignored. */
+ * budget (XShare: k <= budget <= E).  Unused fields are ignored.
+ *
+ * MOE_RESELECT_AFFINITY ("Lynx: Enabling Efficient MoE Inference through
+ * Dynamic Batch-Aware Expert Selection", sections 2.1-2.2; the page gives
+ * no formulas, this is the library's reading): a token's confidence c is
+ * the gap between the probabilities of its two top-ranked experts; bins
+ * have width k/E and there are min(32, ceil(E/k)) of them (bin = the
+ * largest j with j*k <= c*E in fp32); each expert scores the sum of 2^bin
+ * over the tokens whose top-k holds it; the critical set is the shortest
+ * prefix of the score order (descending, ties to the lower index), at
+ * least k long, that holds every token's top-ranked expert; every token
+ * keeps exactly k experts, its first k inside the critical set. */
 typedef struct {
     int32_t mode, k0, budget;
 } moe_reselect_t;

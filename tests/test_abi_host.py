@@ -86,7 +86,7 @@ def test_layer_decode_rejects_bad_arguments(lib):
     assert _layer_call(lib, rule=Rule(1, 9, 0)) == INVALID          # k0 > k
     assert _layer_call(lib, rule=Rule(2, 0, 7)) == INVALID          # budget < k
     assert _layer_call(lib, rule=Rule(2, 0, 129)) == INVALID        # budget > E
-    assert _layer_call(lib, rule=Rule(3, 0, 0)) == INVALID          # unknown rule
+    assert _layer_call(lib, rule=Rule(4, 0, 0)) == INVALID          # unknown rule
     assert _layer_call(lib, x=None) == INVALID
     assert _layer_call(lib, Wdown=None) == INVALID
     assert _layer_call(lib, y=None) == INVALID
@@ -130,6 +130,7 @@ def test_expert_ffn_rejects_bad_arguments(lib):
 def test_valid_call_without_a_device_reports_cuda_error(lib):
     # all arguments valid: validation passes, the device query fails cleanly
     assert _layer_call(lib) == CUDA
+    assert _layer_call(lib, rule=Rule(3, 0, 0)) == CUDA            # affinity binning: no parameters
     assert lib.moe_route(A, A, None, Dims(16, 2048, 128, 8, 0), A, A, A, A, None) == CUDA
 
 

@@ -19,7 +19,7 @@ from gpu_cases import assert_close_y, bits, device_layer, host_layer, shape
 
 pytestmark = pytest.mark.gpu
 
-NONE, OEA, XSHARE = 0, 1, 2
+NONE, OEA, XSHARE, AFFINITY = 0, 1, 2, 3
 THREADS = max(1, len(os.sched_getaffinity(0)))
 
 
@@ -86,7 +86,8 @@ def _check_reselect(logits, probs, k, mode, k0=0, budget=0):
 
 
 RESELECT_RULES = [(NONE, 0, 0), (OEA, 1, 0), (OEA, 2, 0), (OEA, 4, 0), (OEA, 6, 0), (OEA, 8, 0),
-                  (XSHARE, 0, 8), (XSHARE, 0, 24), (XSHARE, 0, 32), (XSHARE, 0, 48), (XSHARE, 0, 128)]
+                  (XSHARE, 0, 8), (XSHARE, 0, 24), (XSHARE, 0, 32), (XSHARE, 0, 48), (XSHARE, 0, 128),
+                  (AFFINITY, 0, 0)]
 
 
 @pytest.mark.parametrize("B", [1, 4, 16, 32, 64])
@@ -106,6 +107,7 @@ def test_reselect_speculative_batch(budget):
     x = _tokens("q30b", 32, 0, kind="spec")
     logits, probs, _, _ = oracle.route(x, L["Wg"], L["bias"], S.k)
     _check_reselect(logits, probs, S.k, XSHARE, budget=budget)
+    _check_reselect(logits, probs, S.k, AFFINITY)
 
 
 @pytest.mark.parametrize("seed", range(6))
@@ -118,7 +120,7 @@ def test_reselect_random_edges(seed):
         p = np.exp(logits.astype(np.float64) - logits.max(1, keepdims=True))
         probs = (p / p.sum(1, keepdims=True)).astype(np.float32)
         for mode, k0, budget in [(NONE, 0, 0), (OEA, 1, 0), (OEA, max(1, k // 2), 0), (OEA, k, 0),
-                                 (XSHARE, 0, k), (XSHARE, 0, min(E, 2 * k)), (XSHARE, 0, E)]:
+                                 (XSHARE, 0, k), (XSHARE, 0, min(E, 2 * k)), (XSHARE, 0, E), (AFFINITY, 0, 0)]:
             _check_reselect(logits, probs, k, mode, k0, budget)
 
 
@@ -153,6 +155,7 @@ LAYER_CASES = [
     ("min", 1, 0, NONE, 0, 0), ("min", 5, 0, OEA, 3, 0),
     ("ragged", 37, 0, NONE, 0, 0), ("ragged", 37, 0, OEA, 2, 0), ("ragged", 37, 0, XSHARE, 0, 10),
     ("maxek", 256, 0, NONE, 0, 0), ("maxek", 256, 0, OEA, 8, 0), ("maxek", 100, 0, XSHARE, 0, 40),
+    ("tiny", 4, 1, AFFINITY, 0, 0), ("ragged", 37, 0, AFFINITY, 0, 0), ("maxek", 256, 0, AFFINITY, 0, 0),
     ("e64", 16, 0, NONE, 0, 0), ("e64", 16, 0, OEA, 4, 0),
 ]
 
@@ -169,7 +172,8 @@ def test_layer_decode_parity_small(name, B, seed, mode, k0, budget):
 
 
 Q30_CASES = [(1, NONE, 0, 0), (1, OEA, 2, 0), (4, OEA, 4, 0), (16, NONE, 0, 0), (16, OEA, 2, 0),
-             (16, OEA, 4, 0), (16, OEA, 6, 0), (16, OEA, 8, 0), (16, XSHARE, 0, 16), (32, NONE, 0, 0),
+             (16, OEA, 4, 0), (16, OEA, 6, 0), (16, OEA, 8, 0), (16, XSHARE, 0, 16), (16, AFFINITY, 0, 0),
+             (64, AFFINITY, 0, 0), (32, NONE, 0, 0),
              (64, NONE, 0, 0), (64, OEA, 4, 0)]
 
 
