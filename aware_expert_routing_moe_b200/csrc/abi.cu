@@ -308,12 +308,12 @@ moe_status_t moe_layer_decode(const float *x, const float *Wg, const float *bias
     int32_t *si = sel_idx ? sel_idx : seg<int32_t>(ws, L.sel_idx);
     float *sw = sel_w ? sel_w : seg<float>(ws, L.sel_w);
     const moe_lists_t lists = ws_lists(ws, L);
-    // B <= 32: the expert kernel starts streaming as soon as the activated
-    // set is published (by the router for OEA and plain top-k, by the
-    // selection for XShare).  Larger batches dispatch each pair's x row once
-    // the selection has built the lists, then stream.
+    // B <= 32: the expert kernel starts streaming as soon as the router has
+    // published the activated set.  Larger batches dispatch each pair's x
+    // row once the selection has built the lists, then stream.
     float *wd = dense ? seg<float>(ws, L.wd) : nullptr;
-    st = from_cuda(launch_layer_route(rmaps, x, bias, dims, rule, logits, dense ? xk : nullptr, y, ctr, s));
+    st = from_cuda(launch_layer_route(rmaps, x, bias, dims, rule, logits, probs, dense ? xk : nullptr, y, ctr, dense,
+                                      s));
     if (st != MOE_OK) return st;
     st = from_cuda(launch_layer_select(logits, probs, dims, rule, si, sw, lists, n_active, ctr, wd, dense, s));
     if (st != MOE_OK) return st;

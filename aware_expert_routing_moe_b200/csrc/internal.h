@@ -38,6 +38,14 @@ struct Counters {
     PubLine pubs[PUB_COPIES];   // layer path: the activated set, in copies
     int32_t grp_done[B_MAX];    // router blocks finished, per token group
     int32_t gu_done[E_MAX];     // finished gate/up units per active-expert slot
+    // Batch-wide rules published by the router (XShare, affinity binning;
+    // B <= 32): each token group's contributions, cleared by the last group
+    int32_t grp_final;                 // token groups whose contributions are in
+    uint32_t ubase_bits[E_MAX / 32];   // union of the top-k sets
+    uint32_t r0_bits[E_MAX / 32];      // every token's rank-0 expert
+    int32_t pad2[15];
+    uint32_t memb[E_MAX];              // XShare: tokens (bit b) whose top-k holds the expert
+    unsigned long long aff_score[E_MAX];  // affinity binning: sum of 2^bin
 };
 static_assert(sizeof(Counters) % 16 == 0, "Counters must keep 16-byte alignment");
 
@@ -97,15 +105,15 @@ cudaError_t launch_reselect(const float *logits, const float *probs, const moe_d
                             const moe_reselect_t &r, int32_t *sel_idx, float *sel_w,
                             const moe_lists_t &l, cudaStream_t s);
 // Layer path, first kernel: router GEMV; also writes x in bf16, zeroes y
-// and (OEA, no re-selection) publishes the activated set in
-// ctr->pubs for an expert kernel started early.
+// and, with `early` (B <= 32), publishes the activated set in ctr->pubs for
+// the expert kernel started early (every rule: OEA and no re-selection per
+// token group, XShare and affinity binning once all groups are in).
 cudaError_t launch_layer_route(const RouterMaps &maps, const float *x, const float *bias, const moe_dims_t &d,
-                               const moe_reselect_t &rule, float *logits, uint16_t *xb, float *y, Counters *ctr,
-                               cudaStream_t s);
+                               const moe_reselect_t &rule, float *logits, float *probs, uint16_t *xb, float *y,
+                               Counters *ctr, bool early, cudaStream_t s);
 // Layer path, second kernel (chained with programmatic dependent launch):
 // softmax, selection, lists, and `wd` (B <= 32) the dense weights.  With
-// `early` the next kernel may launch at once, and in XShare the selection
-// publishes the batch set itself.
+// `early` the next kernel may launch at once.
 cudaError_t launch_layer_select(const float *logits, float *probs, const moe_dims_t &d, const moe_reselect_t &rule,
                                 int32_t *sel_idx, float *sel_w, const moe_lists_t &l, int32_t *n_active_copy,
                                 Counters *ctr, float *wd, bool early, cudaStream_t s);

@@ -241,10 +241,6 @@ struct ReselectArgs {
     moe_lists_t lists;
     int32_t *n_active_copy;
     Counters *ctr;  // layer path: the expert kernel's counters (else null)
-    // layer path, XShare or affinity binning, expert kernel started early:
-    // publish the batch set (every copy of ctr->pubs: mask, then pub + 1)
-    // as soon as it is known
-    int publish;
     // let the dependent kernel launch before waiting for the previous one
     // (the expert kernel started early); otherwise once that wait returns
     int early_dependents;
@@ -514,10 +510,8 @@ __device__ void reselect_body(const ReselectArgs &a, unsigned char *smem_raw) {
 
     // ---- the activated set is now fixed: OEA = union of kept sets, XShare =
     // the batch set, affinity binning = the critical set, NONE = union of
-    // top-k sets.  Map experts to active slots for the dense weights; in
-    // XShare and affinity binning with the expert kernel started early,
-    // publish the set (OEA and NONE sets are published by the router).
-    if (a.publish || dense_w) {
+    // top-k sets.  Map experts to active slots for the dense weights.
+    if (dense_w) {
         const unsigned *abits = (mode == MOE_RESELECT_OEA) ? ukept : (mode == MOE_RESELECT_NONE ? ubase : sbits);
         if (warp == 0) {
             const unsigned word = lane < E_MAX / 32 ? abits[lane] : 0u;
@@ -527,9 +521,6 @@ __device__ void reselect_body(const ReselectArgs &a, unsigned char *smem_raw) {
                 const int u = __shfl_up_sync(FULL, incl, o);
                 if (lane >= o) incl += u;
             }
-            if (a.publish)
-                for (int c = 0; c < PUB_COPIES; ++c)
-                    if (lane < E_MAX / 32) a.ctr->pubs[c].mask[lane] = word;
             int pos = incl - __popc(word);
             for (int bit = 0; bit < 32; ++bit) {
                 const int e = 32 * lane + bit;
@@ -537,13 +528,7 @@ __device__ void reselect_body(const ReselectArgs &a, unsigned char *smem_raw) {
                 s_rank[e] = ((word >> bit) & 1u) ? pos++ : -1;
             }
             const int na = __shfl_sync(FULL, incl, 31);
-            __syncwarp();
             if (lane == 0) s_nact = na;
-            if (a.publish && lane < PUB_COPIES) {
-                __threadfence();
-                asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(&a.ctr->pubs[lane].pub), "r"(1)
-                             : "memory");
-            }
         }
         __syncthreads();
     }
@@ -686,6 +671,10 @@ struct GemvArgs {
     float *y;         // layer path: zeroed
     Counters *ctr;    // layer path only (else null)
     int r1;           // first ranks per token in the published set (0: none)
+    // batch-wide rule whose set the router publishes (MOE_RESELECT_XSHARE or
+    // MOE_RESELECT_AFFINITY; 0: none) with its parameters; B <= 32
+    int batch_rule, k, budget;
+    float *probs;     // XShare: the tokens' probabilities, written here
 };
 
 constexpr int GEMV_TPB_MAX = 4;
@@ -781,13 +770,166 @@ __device__ __forceinline__ void gemv_rows(const unsigned char *wrow, const unsig
     }
 }
 
+// XShare and affinity binning need every token of the batch.  Each token
+// group's last block adds its tokens' contributions (top-k membership and,
+// for XShare, the probability rows; for affinity binning the 2^bin scores
+// and the rank-0 experts); the last group to do so computes the set with
+// the same definitions as the selection kernel, publishes it (the mask of
+// every copy, then one more count) and clears the contributions.  Called by
+// every thread of a group's last block; B <= 32.  `work`: the block's
+// staging area (at least 2 KB + 64 + B*E*4 bytes).
+template <int NI>
+__device__ void batch_rule_publish(const GemvArgs &g, int b0, int nb, unsigned *s_mask, int *s_M, float *s_xs,
+                                   int *s_flag, unsigned char *work) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    const int E = g.E, k = g.k;
+    Counters *ctr = g.ctr;
+#pragma unroll 1
+    for (int t = warp; t < nb; t += nw) {
+        const int b = b0 + t;
+        float l[NI], p[NI];
+        unsigned ord[NI];
+        load_row<NI>(g.logits + static_cast<size_t>(b) * E, E, lane, l);
+#pragma unroll
+        for (int i = 0; i < NI; ++i) ord[i] = ord_of(l[i]);
+        token_softmax_r<NI>(l, ord, E, lane, p);
+        if (g.batch_rule == MOE_RESELECT_XSHARE) {
+#pragma unroll
+            for (int i = 0; i < NI; ++i)
+                if (lane + 32 * i < E) g.probs[static_cast<size_t>(b) * E + lane + 32 * i] = p[i];
+        }
+        unsigned cand = valid_bits<NI>(E, lane);
+        int mye = -1;
+#pragma unroll 1
+        for (int j = 0; j < k; ++j) {
+            const int e = warp_argmax<NI>(ord, cand, lane);
+            if (lane == j) mye = e;
+        }
+        if (lane < k) atomicOr(&ctr->ubase_bits[mye >> 5], 1u << (mye & 31));
+        if (g.batch_rule == MOE_RESELECT_XSHARE) {
+            if (lane < k) atomicOr(&ctr->memb[mye], 1u << b);
+        } else {
+            const int r0 = __shfl_sync(FULL, mye, 0);
+            const int r1e = k >= 2 ? __shfl_sync(FULL, mye, 1) : warp_argmax<NI>(ord, cand, lane);
+            const float p0 = warp_fetch<NI>(p, r0);
+            const float c = r1e >= 0 ? __fsub_rn(p0, warp_fetch<NI>(p, r1e)) : p0;
+            const float cE = __fmul_rn(c, static_cast<float>(E));
+            const int nbins = min(32, (E + k - 1) / k);
+            int bin = 0;
+            for (int j = nbins - 1; j > 0; --j)
+                if (static_cast<float>(j * k) <= cE) {
+                    bin = j;
+                    break;
+                }
+            if (lane < k) atomicAdd(&ctr->aff_score[mye], 1ull << bin);
+            if (lane == 0) atomicOr(&ctr->r0_bits[r0 >> 5], 1u << (r0 & 31));
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        const int t = atomicAdd(&ctr->grp_final, 1);
+        *s_flag = (t == static_cast<int>(gridDim.y) - 1) ? 1 : 0;
+    }
+    __syncthreads();
+    if (!*s_flag) return;
+    __threadfence();  // see every group's contributions
+    // stage what the set depends on in shared memory (the block's staging
+    // area is free now): the union and rank-0 bit masks, and the scores
+    // (affinity binning) or the B x E probabilities (XShare)
+    unsigned *s_ub = reinterpret_cast<unsigned *>(work);        // [E_MAX / 32]
+    unsigned *s_r0 = s_ub + E_MAX / 32;                          // [E_MAX / 32]
+    unsigned long long *s_sc = reinterpret_cast<unsigned long long *>(s_r0 + E_MAX / 32);  // [E_MAX]
+    float *s_pr = reinterpret_cast<float *>(s_sc + E_MAX);      // [B][E]
+    if (threadIdx.x < E_MAX / 32) {
+        s_mask[threadIdx.x] = 0u;
+        s_ub[threadIdx.x] = __ldcg(&ctr->ubase_bits[threadIdx.x]);
+        s_r0[threadIdx.x] = __ldcg(&ctr->r0_bits[threadIdx.x]);
+    }
+    if (threadIdx.x == 0) *s_M = k;
+    if (g.batch_rule == MOE_RESELECT_XSHARE) {
+        for (int i = threadIdx.x; i < g.B * E; i += blockDim.x) s_pr[i] = __ldcg(g.probs + i);
+        for (int e = threadIdx.x; e < E; e += blockDim.x) s_sc[e] = __ldcg(&ctr->memb[e]);
+    } else {
+        for (int e = threadIdx.x; e < E; e += blockDim.x) s_sc[e] = __ldcg(&ctr->aff_score[e]);
+    }
+    __syncthreads();
+    int nbase = 0;
+    for (int i = 0; i < E_MAX / 32; ++i) nbase += __popc(s_ub[i]);
+    if (g.batch_rule == MOE_RESELECT_XSHARE) {
+        // s_e = sum over tokens b ascending holding e in their top-k of p[b][e]
+        for (int e = threadIdx.x; e < E; e += blockDim.x) {
+            const unsigned m = static_cast<unsigned>(s_sc[e]);
+            float sc = 0.0f;
+            for (int b = 0; b < g.B; ++b)
+                if ((m >> b) & 1u) sc = __fadd_rn(sc, s_pr[b * E + e]);
+            s_xs[e] = sc;
+        }
+        __syncthreads();
+        const int Mp = g.budget < nbase ? g.budget : nbase;
+        for (int e = threadIdx.x; e < E; e += blockDim.x) {
+            if (!((s_ub[e >> 5] >> (e & 31)) & 1u)) continue;
+            const float se = s_xs[e];
+            int rank = 0;
+            for (int e2 = 0; e2 < E; ++e2) {
+                if (!((s_ub[e2 >> 5] >> (e2 & 31)) & 1u)) continue;
+                const float s2 = s_xs[e2];
+                rank += (s2 > se || (s2 == se && e2 < e)) ? 1 : 0;
+            }
+            if (rank < Mp) atomicOr(&s_mask[e >> 5], 1u << (e & 31));
+        }
+    } else {
+        // the shortest prefix of the score order, at least k long, holding
+        // every rank-0 expert
+        int *pos_of = reinterpret_cast<int *>(s_xs);
+        for (int e = threadIdx.x; e < E; e += blockDim.x) {
+            pos_of[e] = E;
+            if (!((s_ub[e >> 5] >> (e & 31)) & 1u)) continue;
+            const unsigned long long se = s_sc[e];
+            int pos = 0;
+            for (int e2 = 0; e2 < E; ++e2) {
+                if (!((s_ub[e2 >> 5] >> (e2 & 31)) & 1u)) continue;
+                const unsigned long long s2 = s_sc[e2];
+                pos += (s2 > se || (s2 == se && e2 < e)) ? 1 : 0;
+            }
+            pos_of[e] = pos;
+            if ((s_r0[e >> 5] >> (e & 31)) & 1u) atomicMax(s_M, pos + 1);
+        }
+        __syncthreads();
+        for (int e = threadIdx.x; e < E; e += blockDim.x)
+            if (pos_of[e] < *s_M) atomicOr(&s_mask[e >> 5], 1u << (e & 31));
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < PUB_COPIES * (E_MAX / 32); i += blockDim.x) {
+        const unsigned m = s_mask[i % (E_MAX / 32)];
+        if (m != 0u) atomicOr(&ctr->pubs[i / (E_MAX / 32)].mask[i % (E_MAX / 32)], m);
+    }
+    // clear the contributions for the next call
+    for (int e = threadIdx.x; e < E_MAX; e += blockDim.x) {
+        ctr->memb[e] = 0u;
+        ctr->aff_score[e] = 0ull;
+    }
+    if (threadIdx.x < E_MAX / 32) {
+        ctr->ubase_bits[threadIdx.x] = 0u;
+        ctr->r0_bits[threadIdx.x] = 0u;
+    }
+    if (threadIdx.x == 0) ctr->grp_final = 0;
+    __syncthreads();
+    if (threadIdx.x < PUB_COPIES) {
+        __threadfence();
+        asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(&ctr->pubs[threadIdx.x].pub), "r"(1)
+                     : "memory");
+    }
+}
+
 template <int NI>
 __global__ void __launch_bounds__(32 * GEMV_EPB_MAX) route_gemv_kernel(const __grid_constant__ RouterMaps maps,
                                                                        const GemvArgs g) {
     extern __shared__ unsigned char gemv_smem[];
     __shared__ __align__(8) unsigned long long s_bar;
     __shared__ unsigned s_mask[E_MAX / 32];
-    __shared__ int s_last, s_fail;
+    __shared__ int s_last, s_fail, s_M;
+    __shared__ float s_xs[E_MAX];
     // the next kernel (the selection) may become resident while this runs
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     unsigned char *rows = reinterpret_cast<unsigned char *>(
@@ -886,6 +1028,7 @@ __global__ void __launch_bounds__(32 * GEMV_EPB_MAX) route_gemv_kernel(const __g
             if (m != 0u) atomicOr(&g.ctr->pubs[i / (E_MAX / 32)].mask[i % (E_MAX / 32)], m);
         }
     }
+    if (g.batch_rule != 0) batch_rule_publish<NI>(g, b0, nb, s_mask, &s_M, s_xs, &s_last, rows);
     __syncthreads();
     if (threadIdx.x < PUB_COPIES) {
         __threadfence();
@@ -919,6 +1062,10 @@ GemvShape gemv_shape(const moe_dims_t &d) {
         else break;
     }
     g.smem = static_cast<size_t>(g.tpb + g.epb) * g.row_bytes + 1024;  // + alignment slack
+    // a batch-wide rule (B <= 32) stages masks, scores and B x E
+    // probabilities in the same area
+    const size_t batch_area = 1024 + 64 + 8 * E_MAX + static_cast<size_t>(d.B) * d.E * 4;
+    if (d.B <= 32 && g.smem < batch_area) g.smem = batch_area;
     return g;
 }
 
@@ -950,7 +1097,6 @@ ReselectArgs make_reselect_args(const float *logits, float *probs, bool fuse_sof
     a.lists = l;
     a.n_active_copy = n_active_copy;
     a.ctr = nullptr;
-    a.publish = 0;
     a.early_dependents = 0;
     a.wd = nullptr;
     a.cache_rows = 0;
@@ -1001,6 +1147,10 @@ GemvArgs make_gemv_args(const float *bias, const moe_dims_t &d, const GemvShape 
     g.y = nullptr;
     g.ctr = nullptr;
     g.r1 = 0;
+    g.batch_rule = 0;
+    g.k = d.k;
+    g.budget = 0;
+    g.probs = nullptr;
     return g;
 }
 
@@ -1079,8 +1229,8 @@ int layer_pub_target(const moe_dims_t &d, const moe_reselect_t &rule) {
 }
 
 cudaError_t launch_layer_route(const RouterMaps &maps, const float *x, const float *bias, const moe_dims_t &d,
-                               const moe_reselect_t &rule, float *logits, uint16_t *xb, float *y, Counters *ctr,
-                               cudaStream_t s) {
+                               const moe_reselect_t &rule, float *logits, float *probs, uint16_t *xb, float *y,
+                               Counters *ctr, bool early, cudaStream_t s) {
     const GemvShape sh = gemv_shape(d);
     GemvArgs g = make_gemv_args(bias, d, sh, logits);
     g.x = x;
@@ -1088,6 +1238,10 @@ cudaError_t launch_layer_route(const RouterMaps &maps, const float *x, const flo
     g.y = y;
     g.ctr = ctr;
     g.r1 = rule.mode == MOE_RESELECT_OEA ? rule.k0 : (rule.mode == MOE_RESELECT_NONE ? d.k : 0);
+    const bool batch = rule.mode == MOE_RESELECT_XSHARE || rule.mode == MOE_RESELECT_AFFINITY;
+    g.batch_rule = (early && batch && d.B <= 32) ? rule.mode : 0;
+    g.budget = rule.budget;
+    g.probs = probs;
     return launch_gemv(maps, g, sh, s);
 }
 
@@ -1096,7 +1250,6 @@ cudaError_t launch_layer_select(const float *logits, float *probs, const moe_dim
                                 Counters *ctr, float *wd, bool early, cudaStream_t s) {
     ReselectArgs a = make_reselect_args(logits, probs, true, d, rule, sel_idx, sel_w, l, n_active_copy);
     a.ctr = ctr;
-    a.publish = (early && (rule.mode == MOE_RESELECT_XSHARE || rule.mode == MOE_RESELECT_AFFINITY)) ? 1 : 0;
     a.early_dependents = early ? 1 : 0;
     a.wd = wd;
     const size_t smem = reselect_smem(d, &a.cache_rows);

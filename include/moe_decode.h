@@ -203,7 +203,7 @@ moe_status_t moe_layer_decode(const float *x, const float *Wg, const float *bias
  *    B <= 32, B*d*2 bytes of bf16 x, min(E, B*k)*B*d_ff*2 bytes of SwiGLU
  *    activations and min(E, B*k)*B*4 bytes of dense weights; above,
  *    B*k*d*2 bytes of per-pair x rows and B*k*d_ff*2 bytes of activations;
- *    plus about 3 KB of counters, each part rounded up to 256 bytes.  Larger
+ *    plus about 7 KB of counters, each part rounded up to 256 bytes.  Larger
  *    dims return MOE_ERR_UNSUPPORTED before anything is enqueued.  The
  *    Qwen3-30B-A3B- and Qwen3-235B-A22B-shaped layers fit for every B <= 256.
  *  - Set-up: the first call on a device looks up the array's device address

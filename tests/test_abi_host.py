@@ -123,7 +123,7 @@ def test_expert_ffn_rejects_bad_arguments(lib):
     assert lib.moe_expert_ffn(A, A, A, A + 2, d, lists, A, A, n, None) == MISALIGNED
     assert lib.moe_expert_ffn(A, A, A, A, d, lists, A, A, n - 1, None) == WORKSPACE
     assert lib.moe_check_error(None, 0, None) == WORKSPACE
-    assert lib.moe_check_error(A + 16, 4096, None) == MISALIGNED
+    assert lib.moe_check_error(A + 16, 1 << 16, None) == MISALIGNED
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
