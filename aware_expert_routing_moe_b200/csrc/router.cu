@@ -288,6 +288,25 @@ __device__ __forceinline__ float float_of_ord(unsigned o) {
     return __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
 }
 
+// Sort keys of a batch-wide score order (score descending, ties to the
+// lower expert index), unique per expert; 0 marks a non-member.  Affinity
+// scores are exact integers below 2^44; XShare scores are non-negative
+// floats, whose bit patterns order like their values.
+__device__ __forceinline__ unsigned long long key_int_score(unsigned long long sc, int e) {
+    return (sc << 8) | static_cast<unsigned long long>(255 - e);
+}
+__device__ __forceinline__ unsigned long long key_float_score(float sc, int e) {
+    return (static_cast<unsigned long long>(__float_as_uint(sc)) << 32) | static_cast<unsigned>(~static_cast<unsigned>(e));
+}
+// Position of expert e in the score order of the members (keys > 0),
+// computed by one warp: the number of members with a larger key.
+__device__ __forceinline__ int warp_rank(const unsigned long long *key, int E, int e, int lane) {
+    const unsigned long long ke = key[e];
+    unsigned c = 0u;
+    for (int e2 = lane; e2 < E; e2 += 32) c += key[e2] > ke ? 1u : 0u;
+    return static_cast<int>(__reduce_add_sync(FULL, c));
+}
+
 // One round of warp arg-max over candidate bits with two hardware warp
 // reductions: the largest logit image, then, among lanes holding it, the
 // lowest expert index.  The winner leaves the candidates.  -1 if none.
@@ -469,19 +488,18 @@ __device__ void reselect_body(const ReselectArgs &a, unsigned char *smem_raw) {
             s_score[tid] = sc;
         }
         __syncthreads();
-        if (tid < E && ((ubase[tid >> 5] >> (tid & 31)) & 1u)) {
-            int nb = 0;
-            for (int i = 0; i < E_MAX / 32; ++i) nb += __popc(ubase[i]);
-            const int Mp = a.budget < nb ? a.budget : nb;
-            const float se = s_score[tid];
-            int rank = 0;
+        // rank the batch union by score (one warp per expert)
+        for (int e = tid; e < E; e += blockDim.x)
+            s_aff[e] = ((ubase[e >> 5] >> (e & 31)) & 1u) ? key_float_score(s_score[e], e) : 0ull;
+        __syncthreads();
+        int nbase = 0;
+        for (int i = 0; i < E_MAX / 32; ++i) nbase += __popc(ubase[i]);
+        const int Mp = a.budget < nbase ? a.budget : nbase;
 #pragma unroll 1
-            for (int e2 = 0; e2 < E; ++e2) {
-                if (!((ubase[e2 >> 5] >> (e2 & 31)) & 1u)) continue;
-                const float s2 = s_score[e2];
-                rank += (s2 > se || (s2 == se && e2 < tid)) ? 1 : 0;
-            }
-            if (rank < Mp) atomicOr(&sbits[tid >> 5], 1u << (tid & 31));
+        for (int e = warp; e < E; e += nwarps) {
+            if (s_aff[e] == 0ull) continue;
+            const int rank = warp_rank(s_aff, E, e, lane);
+            if (lane == 0 && rank < Mp) atomicOr(&sbits[e >> 5], 1u << (e & 31));
         }
         __syncthreads();
     }
@@ -490,21 +508,21 @@ __device__ void reselect_body(const ReselectArgs &a, unsigned char *smem_raw) {
     // score order (score descending, ties to the lower index), at least k
     // long, that holds every token's rank-0 expert
     if (mode == MOE_RESELECT_AFFINITY) {
-        const bool in_base = tid < E && ((ubase[tid >> 5] >> (tid & 31)) & 1u);
-        if (in_base) {
-            const unsigned long long se = s_aff[tid];
-            int pos = 0;
+        for (int e = tid; e < E; e += blockDim.x)
+            s_aff[e] = ((ubase[e >> 5] >> (e & 31)) & 1u) ? key_int_score(s_aff[e], e) : 0ull;
+        __syncthreads();
 #pragma unroll 1
-            for (int e2 = 0; e2 < E; ++e2) {
-                if (!((ubase[e2 >> 5] >> (e2 & 31)) & 1u)) continue;
-                const unsigned long long s2 = s_aff[e2];
-                pos += (s2 > se || (s2 == se && e2 < tid)) ? 1 : 0;
+        for (int e = warp; e < E; e += nwarps) {
+            if (s_aff[e] == 0ull) continue;
+            const int pos = warp_rank(s_aff, E, e, lane);
+            if (lane == 0) {
+                s_pos[e] = pos;
+                if ((r0bits[e >> 5] >> (e & 31)) & 1u) atomicMax(&s_M, pos + 1);
             }
-            s_pos[tid] = pos;
-            if ((r0bits[tid >> 5] >> (tid & 31)) & 1u) atomicMax(&s_M, pos + 1);
         }
         __syncthreads();
-        if (in_base && s_pos[tid] < s_M) atomicOr(&sbits[tid >> 5], 1u << (tid & 31));
+        for (int e = tid; e < E; e += blockDim.x)
+            if (s_aff[e] != 0ull && s_pos[e] < s_M) atomicOr(&sbits[e >> 5], 1u << (e & 31));
         __syncthreads();
     }
 
@@ -856,49 +874,36 @@ __device__ void batch_rule_publish(const GemvArgs &g, int b0, int nb, unsigned *
     __syncthreads();
     int nbase = 0;
     for (int i = 0; i < E_MAX / 32; ++i) nbase += __popc(s_ub[i]);
-    if (g.batch_rule == MOE_RESELECT_XSHARE) {
-        // s_e = sum over tokens b ascending holding e in their top-k of p[b][e]
-        for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    // sort keys of the batch union (0 for other experts), in place of the
+    // scores; XShare first sums each expert's probabilities (tokens ascending)
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        const bool member = (s_ub[e >> 5] >> (e & 31)) & 1u;
+        if (g.batch_rule == MOE_RESELECT_XSHARE) {
             const unsigned m = static_cast<unsigned>(s_sc[e]);
             float sc = 0.0f;
             for (int b = 0; b < g.B; ++b)
                 if ((m >> b) & 1u) sc = __fadd_rn(sc, s_pr[b * E + e]);
-            s_xs[e] = sc;
+            s_sc[e] = member ? key_float_score(sc, e) : 0ull;
+        } else {
+            s_sc[e] = member ? key_int_score(s_sc[e], e) : 0ull;
         }
-        __syncthreads();
-        const int Mp = g.budget < nbase ? g.budget : nbase;
-        for (int e = threadIdx.x; e < E; e += blockDim.x) {
-            if (!((s_ub[e >> 5] >> (e & 31)) & 1u)) continue;
-            const float se = s_xs[e];
-            int rank = 0;
-            for (int e2 = 0; e2 < E; ++e2) {
-                if (!((s_ub[e2 >> 5] >> (e2 & 31)) & 1u)) continue;
-                const float s2 = s_xs[e2];
-                rank += (s2 > se || (s2 == se && e2 < e)) ? 1 : 0;
-            }
-            if (rank < Mp) atomicOr(&s_mask[e >> 5], 1u << (e & 31));
-        }
-    } else {
-        // the shortest prefix of the score order, at least k long, holding
-        // every rank-0 expert
-        int *pos_of = reinterpret_cast<int *>(s_xs);
-        for (int e = threadIdx.x; e < E; e += blockDim.x) {
-            pos_of[e] = E;
-            if (!((s_ub[e >> 5] >> (e & 31)) & 1u)) continue;
-            const unsigned long long se = s_sc[e];
-            int pos = 0;
-            for (int e2 = 0; e2 < E; ++e2) {
-                if (!((s_ub[e2 >> 5] >> (e2 & 31)) & 1u)) continue;
-                const unsigned long long s2 = s_sc[e2];
-                pos += (s2 > se || (s2 == se && e2 < e)) ? 1 : 0;
-            }
-            pos_of[e] = pos;
-            if ((s_r0[e >> 5] >> (e & 31)) & 1u) atomicMax(s_M, pos + 1);
-        }
-        __syncthreads();
-        for (int e = threadIdx.x; e < E; e += blockDim.x)
-            if (pos_of[e] < *s_M) atomicOr(&s_mask[e >> 5], 1u << (e & 31));
     }
+    __syncthreads();
+    int *pos_of = reinterpret_cast<int *>(s_xs);
+    for (int e = warp; e < E; e += nw) {
+        if (s_sc[e] == 0ull) continue;
+        const int pos = warp_rank(s_sc, E, e, lane);
+        if (lane == 0) {
+            pos_of[e] = pos;
+            if (g.batch_rule == MOE_RESELECT_AFFINITY && ((s_r0[e >> 5] >> (e & 31)) & 1u)) atomicMax(s_M, pos + 1);
+        }
+    }
+    __syncthreads();
+    // XShare: the first min(budget, |union|); affinity binning: the shortest
+    // prefix, at least k long, holding every rank-0 expert
+    const int cut = g.batch_rule == MOE_RESELECT_XSHARE ? (g.budget < nbase ? g.budget : nbase) : *s_M;
+    for (int e = threadIdx.x; e < E; e += blockDim.x)
+        if (s_sc[e] != 0ull && pos_of[e] < cut) atomicOr(&s_mask[e >> 5], 1u << (e & 31));
     __syncthreads();
     for (int i = threadIdx.x; i < PUB_COPIES * (E_MAX / 32); i += blockDim.x) {
         const unsigned m = s_mask[i % (E_MAX / 32)];
