@@ -127,6 +127,10 @@ struct ExpertArgs {
     int hrows;  // rows of one H box (bpad in dense mode, TN otherwise)
     int early;       // start when ctr->pubs[c].pub reaches pub_target, not at the previous kernel's end
     int pub_target;
+    // host-computed unit geometry: gate/up and down units per tile, their
+    // stage counts, and the reciprocals of the unit counts (dense decode)
+    int gu_per_tile, d_per_tile, ns_gu, ns_d;
+    float inv_gu, inv_d;
     const float *wd;
     const int32_t *n_active, *active, *offsets, *tok;
     const float *w;
@@ -251,10 +255,36 @@ struct UnitInfo : UnitRec {
     int dep;  // D (lane 0): gate/up units of the expert already published
 };
 
+// q = floor(u / per) for 0 <= u < 2^22 from a float reciprocal, corrected
+// to the exact quotient.
+__device__ __forceinline__ int div_by(int u, int per, float inv) {
+    int q = __float2int_rz(__fmul_rn(static_cast<float>(u), inv));
+    if ((q + 1) * per <= u) ++q;
+    else if (q * per > u) --q;
+    return q;
+}
+
 __device__ __forceinline__ void decode_rec(int u, int n_units, const ExpertArgs &a, const SharedCtl *ctl,
                                            UnitRec &ui) {
     if (u >= n_units) {
         ui.type = UNIT_END;
+        return;
+    }
+    if (a.dense) {
+        // one tile per active expert: slot i's units are consecutive
+        const int n_gu = ctl->total_tiles * a.gu_per_tile;
+        const bool gu = u < n_gu;
+        const int v = gu ? u : u - n_gu;
+        const int per = gu ? a.gu_per_tile : a.d_per_tile;
+        const int i = div_by(v, per, gu ? a.inv_gu : a.inv_d);
+        ui.type = gu ? UNIT_GU : UNIT_D;
+        ui.ns = gu ? a.ns_gu : a.ns_d;
+        ui.row0 = (v - i * per) * (gu ? GU_ROWS : D_ROWS);
+        ui.i_act = i;
+        ui.e = ctl->act_e[i];
+        ui.p0 = i * a.B;
+        ui.n = a.B;
+        ui.need = a.gu_per_tile;
         return;
     }
     const int gu_per_tile = a.F / GU_ROWS;
@@ -972,6 +1002,15 @@ cudaError_t launch_expert_ffn(const ExpertMaps &maps, const uint16_t *xb, const 
     a.hrows = expert_ffn_h_rows(d.B);
     a.early = (early && a.dense) ? 1 : 0;
     a.pub_target = pub_target;
+    a.gu_per_tile = d.d_ff / GU_ROWS;
+    a.d_per_tile = d.d / D_ROWS;
+    {
+        const int gk = 64 * expert_ffn_gu_chunks(d.d), dk = 64 * expert_ffn_d_chunks(d.d_ff);
+        a.ns_gu = (d.d + gk - 1) / gk;
+        a.ns_d = (d.d_ff + dk - 1) / dk;
+    }
+    a.inv_gu = 1.0f / static_cast<float>(a.gu_per_tile);
+    a.inv_d = 1.0f / static_cast<float>(a.d_per_tile);
     a.wd = wd;
     a.n_active = l.n_active;
     a.active = l.active;
