@@ -37,6 +37,9 @@
 // time limit; on expiry the CTA records an error code in the workspace,
 // drains its in-flight copies and returns.  The last CTA to finish puts the
 // workspace counters of the call back to zero.
+#include <cstring>
+#include <mutex>
+
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -82,11 +85,13 @@ static_assert(RingSmallB::SLOT_BYTES % 1024 == 0 && RingLargeB::SLOT_BYTES % 102
 static_assert(smem_bytes<RingSmallB>() <= 232448 && smem_bytes<RingLargeB>() <= 232448, "shared memory budget");
 
 constexpr unsigned long long WAIT_LIMIT_NS = 1000000000ull;  // 1 s
+constexpr int SPLIT_TABLE_MAX = 256;  // tile counts covered by the split table
 
 enum : int { UNIT_GU = 0, UNIT_D = 1, UNIT_END = 2 };
 
 struct StageHdr {
     int type, e, i_act, p0, n, row0, s, ns;
+    int k;  // the stage's k-range (s, or k0 + s for a split down unit)
 };
 
 // One work unit, decoded: kind, expert id and active index, first pair and
@@ -94,6 +99,7 @@ struct StageHdr {
 // the gate/up units of its expert that must be published first.
 struct UnitRec {
     int type, e, i_act, p0, n, row0, ns, need;
+    int k0;  // first k-range (split down units; 0 otherwise)
 };
 constexpr int UNIT_WINDOW = 32;  // units a producer decodes at once (one per lane)
 
@@ -107,6 +113,7 @@ struct SharedCtl {
     volatile int abort_flag;
     volatile int consumed;
     int n_active, total_tiles;
+    int split;  // last-round down units cut into k-ranges
     int last_cta;
     int tile_start[E_MAX + 1];
     UnitRec urec[UNIT_WINDOW];  // the producer's decoded window of its own units
@@ -130,7 +137,9 @@ struct ExpertArgs {
     // host-computed unit geometry: gate/up and down units per tile, their
     // stage counts, and the reciprocals of the unit counts (dense decode)
     int gu_per_tile, d_per_tile, ns_gu, ns_d;
-    float inv_gu, inv_d;
+    float inv_gu, inv_d, inv_nsd;
+    // last-round down units to cut into k-ranges, per total tile count
+    unsigned char split_for[SPLIT_TABLE_MAX + 1];
     const float *wd;
     const int32_t *n_active, *active, *offsets, *tok;
     const float *w;
@@ -264,21 +273,45 @@ __device__ __forceinline__ int div_by(int u, int per, float inv) {
     return q;
 }
 
+// The unit sequence: all gate/up units, then the down units.  Units are
+// dealt round robin, so the last, partial round decides when the kernel
+// ends.  When that round holds only down units and cutting each of them
+// into its k-ranges (one stage each, their sums meet in y's atomic adds)
+// lowers the largest per-CTA stage count by two or more, the round is cut.
+struct UnitCounts {
+    int n_gu, d_main, split, total;  // split: down units cut into k-ranges
+};
+__device__ __forceinline__ UnitCounts unit_counts(const ExpertArgs &a, int total_tiles, int split) {
+    UnitCounts c;
+    c.n_gu = total_tiles * a.gu_per_tile;
+    c.split = split;
+    c.d_main = total_tiles * a.d_per_tile - split;
+    c.total = c.n_gu + c.d_main + split * a.ns_d;
+    return c;
+}
 __device__ __forceinline__ void decode_rec(int u, int n_units, const ExpertArgs &a, const SharedCtl *ctl,
                                            UnitRec &ui) {
     if (u >= n_units) {
         ui.type = UNIT_END;
         return;
     }
+    const UnitCounts uc = unit_counts(a, ctl->total_tiles, ctl->split);
+    ui.k0 = 0;
+    if (u >= uc.n_gu + uc.d_main) {
+        // a k-range of one of the last round's down units
+        const int j = u - uc.n_gu - uc.d_main;
+        const int q = div_by(j, a.ns_d, a.inv_nsd);
+        ui.k0 = j - q * a.ns_d;
+        u = uc.n_gu + uc.d_main + q;
+    }
     if (a.dense) {
         // one tile per active expert: slot i's units are consecutive
-        const int n_gu = ctl->total_tiles * a.gu_per_tile;
-        const bool gu = u < n_gu;
-        const int v = gu ? u : u - n_gu;
+        const bool gu = u < uc.n_gu;
+        const int v = gu ? u : u - uc.n_gu;
         const int per = gu ? a.gu_per_tile : a.d_per_tile;
         const int i = div_by(v, per, gu ? a.inv_gu : a.inv_d);
         ui.type = gu ? UNIT_GU : UNIT_D;
-        ui.ns = gu ? a.ns_gu : a.ns_d;
+        ui.ns = gu ? a.ns_gu : (ui.k0 > 0 || u - uc.n_gu >= uc.d_main ? 1 : a.ns_d);
         ui.row0 = (v - i * per) * (gu ? GU_ROWS : D_ROWS);
         ui.i_act = i;
         ui.e = ctl->act_e[i];
@@ -301,8 +334,7 @@ __device__ __forceinline__ void decode_rec(int u, int n_units, const ExpertArgs 
         ui.type = UNIT_D;
         per = d_per_tile;
         v = u - n_gu;
-        const int dk = 64 * d_chunks_of(a.F);
-        ui.ns = (a.F + dk - 1) / dk;
+        ui.ns = v >= uc.d_main ? 1 : a.ns_d;
     }
     // active expert owning this unit: largest i with tile_start[i] <= v / per
     const int tile = v / per;
@@ -349,7 +381,13 @@ template <class RG>
 __device__ void producer(const ExpertArgs &a, const ExpertMaps &m, SharedCtl *ctl, unsigned char *slots) {
     constexpr int STAGES = RG::STAGES;
     const int lane = threadIdx.x & 31;
-    const int n_units = ctl->total_tiles * (a.F / GU_ROWS + a.d / D_ROWS);
+    // host-computed per tile count: the producer's set-up code runs once per
+    // call on the critical path, so it does no arithmetic it can avoid
+    const int t = ctl->total_tiles;
+    const int split = t <= SPLIT_TABLE_MAX ? a.split_for[t] : 0;
+    if (lane == 0) ctl->split = split;
+    __syncwarp();
+    const int n_units = unit_counts(a, t, split).total;
     const unsigned long long policy = evict_first_policy();
     // units are dealt round robin: CTA c takes c, c + grid, c + 2 grid, ...
     // (all CTAs start together when the lists are ready; every gate/up unit
@@ -386,6 +424,7 @@ __device__ void producer(const ExpertArgs &a, const ExpertMaps &m, SharedCtl *ct
                 h.row0 = cur.row0;
                 h.s = s;
                 h.ns = cur.ns;
+                h.k = cur.k0 + s;
                 mbar_expect_tx(&ctl->full[slot], bytes);
             }
             __syncwarp();
@@ -398,7 +437,8 @@ __device__ void producer(const ExpertArgs &a, const ExpertMaps &m, SharedCtl *ct
                 if (lane == 2) tma_load_3d(odst, &m.x, 0, a.dense ? 0 : cur.p0, s * gc, &ctl->full[slot]);
             } else {
                 if (lane == 0)
-                    tma_load_3d_stream(wdst, &m.down, 0, cur.e * a.d + cur.row0, s * dc, &ctl->full[slot], policy);
+                    tma_load_3d_stream(wdst, &m.down, 0, cur.e * a.d + cur.row0, (cur.k0 + s) * dc, &ctl->full[slot],
+                                       policy);
                 if (s == 0) {
                     // this expert's gate/up units must be complete before H is read
                     if (lane == 0) {
@@ -422,7 +462,7 @@ __device__ void producer(const ExpertArgs &a, const ExpertMaps &m, SharedCtl *ct
                     }
                     ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
                 }
-                if (ok && lane == 1) tma_load_3d(odst, &m.h, 0, cur.p0, s * dc, &ctl->full[slot]);
+                if (ok && lane == 1) tma_load_3d(odst, &m.h, 0, cur.p0, (cur.k0 + s) * dc, &ctl->full[slot]);
             }
             ++g;
             if (!ok) break;
@@ -515,10 +555,10 @@ __device__ __forceinline__ void stage_dispatch(const StageHdr &h, uint32_t wbase
                                                int warp, int lane, float (&acc_g)[4][4], float (&acc_u)[4][4]) {
     if (h.type == UNIT_GU) {
         const int gk = 64 * gu_chunks_of(a.d);
-        gu_stage<NT>(wbase, obase, (a.dense ? a.bpad : TN) * 128, min(gk, a.d - h.s * gk), warp, lane, acc_g, acc_u);
+        gu_stage<NT>(wbase, obase, (a.dense ? a.bpad : TN) * 128, min(gk, a.d - h.k * gk), warp, lane, acc_g, acc_u);
     } else {
         const int dk = 64 * d_chunks_of(a.F);
-        d_stage<NT>(wbase, obase, a.hrows, min(dk, a.F - h.s * dk), warp, lane, acc_g);
+        d_stage<NT>(wbase, obase, a.hrows, min(dk, a.F - h.k * dk), warp, lane, acc_g);
     }
 }
 
@@ -922,6 +962,40 @@ __global__ void __launch_bounds__(256) ffn_prep_kernel(PrepArgs p) {
         for (int i = threadIdx.x; i < E_MAX; i += blockDim.x) p.ctr->gu_done[i] = 0;
 }
 
+// Host side of the last-round cut (see unit_counts): the largest per-CTA
+// stage count when consecutive slices of the unit sequence (start, length,
+// stages per unit) are dealt round robin over P CTAs.  Every CTA takes
+// floor(len / P) units of a slice and the len % P CTAs from start % P on
+// (cyclically) one more; the largest sum of extras is reached at the start
+// of one of the slices' extra runs.
+struct Slice {
+    long long start, len, w;
+};
+long long max_stages_host(const Slice *sl, int ns, long long P) {
+    long long base = 0, best = 0;
+    for (int i = 0; i < ns; ++i) base += sl[i].w * (sl[i].len / P);
+    for (int i = 0; i < ns; ++i) {
+        if (sl[i].len % P == 0) continue;
+        const long long c = sl[i].start % P;
+        long long extra = 0;
+        for (int j = 0; j < ns; ++j)
+            if (((c - sl[j].start % P) % P + P) % P < sl[j].len % P) extra += sl[j].w;
+        best = best > extra ? best : extra;
+    }
+    return base + best;
+}
+// Last-round down units to cut for `tiles` tiles: only when that round
+// holds down units alone and the cut lowers the largest stage count by two
+// or more (one stage does not pay for the extra epilogues, measured).
+int split_for_tiles(long long tiles, int gu_per_tile, int d_per_tile, int ns_gu, int ns_d, long long P) {
+    const long long n_gu = tiles * gu_per_tile, n_d = tiles * d_per_tile;
+    const long long r = (n_gu + n_d) % P;
+    if (ns_d <= 1 || r == 0 || r > n_d) return 0;
+    const Slice whole[2] = {{0, n_gu, ns_gu}, {n_gu, n_d, ns_d}};
+    const Slice cut[3] = {{0, n_gu, ns_gu}, {n_gu, n_d - r, ns_d}, {n_gu + n_d - r, r * ns_d, 1}};
+    return max_stages_host(cut, 3, P) + 2 <= max_stages_host(whole, 2, P) ? static_cast<int>(r) : 0;
+}
+
 int g_num_sms[64] = {0};
 bool g_attr_small[64] = {false}, g_attr_large[64] = {false};
 
@@ -1011,6 +1085,23 @@ cudaError_t launch_expert_ffn(const ExpertMaps &maps, const uint16_t *xb, const 
     }
     a.inv_gu = 1.0f / static_cast<float>(a.gu_per_tile);
     a.inv_d = 1.0f / static_cast<float>(a.d_per_tile);
+    a.inv_nsd = 1.0f / static_cast<float>(a.ns_d);
+    {
+        // cached per unit geometry and grid size (one GPU and shape at a time
+        // in practice; recomputed when either changes)
+        static std::mutex mu;
+        static int key[5] = {-1, -1, -1, -1, -1};
+        static unsigned char table[SPLIT_TABLE_MAX + 1];
+        const int grid = early && g_num_sms[dev] > 1 ? g_num_sms[dev] - 1 : g_num_sms[dev];
+        const int k[5] = {a.gu_per_tile, a.d_per_tile, a.ns_gu, a.ns_d, grid};
+        std::lock_guard<std::mutex> lock(mu);
+        if (std::memcmp(k, key, sizeof(k)) != 0) {
+            for (int t = 0; t <= SPLIT_TABLE_MAX; ++t)
+                table[t] = static_cast<unsigned char>(split_for_tiles(t, k[0], k[1], k[2], k[3], grid));
+            std::memcpy(key, k, sizeof(k));
+        }
+        std::memcpy(a.split_for, table, sizeof(table));
+    }
     a.wd = wd;
     a.n_active = l.n_active;
     a.active = l.active;
