@@ -138,3 +138,19 @@ def test_binding_raises_on_error(lib):
     with pytest.raises(moe.MoeError) as ei:
         moe._check(MISALIGNED, "x")
     assert ei.value.status == MISALIGNED
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_noalloc_size_limit(lib):
+    # the static scratch holds both model shapes at every batch size: valid
+    # dims pass the size check and only the device query fails here
+    lists = Lists(A, A, A, A, A)
+    for B in (1, 16, 32, 33, 64, 256):
+        for d, F in ((2048, 768), (4096, 1536)):
+            st = lib.moe_expert_ffn_noalloc(A, A, A, A, Dims(B, d, 128, 8, F), lists, A, None)
+            assert st == CUDA, (B, d, F, st)
+    # the largest dims do not fit: rejected before anything is enqueued
+    assert lib.moe_expert_ffn_noalloc(A, A, A, A, Dims(256, 16384, 256, 16, 8192), lists, A, None) == UNSUPPORTED
+    # invalid dims and misaligned buffers are reported first
+    assert lib.moe_expert_ffn_noalloc(A, A, A, A, Dims(257, 2048, 128, 8, 768), lists, A, None) == INVALID
+    assert lib.moe_expert_ffn_noalloc(A + 4, A, A, A, Dims(16, 2048, 128, 8, 768), lists, A, None) == MISALIGNED
