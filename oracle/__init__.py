@@ -20,7 +20,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "moe_oracle.c")
 _LIB = os.path.join(_HERE, "libmoe_oracle.so")
 
-MODE_NONE, MODE_OEA, MODE_XSHARE = 0, 1, 2
+MODE_NONE, MODE_OEA, MODE_XSHARE, MODE_AFFINITY, MODE_XSHARE_HIER = 0, 1, 2, 3, 4
 
 _lib = None
 
@@ -55,7 +55,7 @@ def _load():
         lib.oracle_route.restype = None
         lib.oracle_route.argtypes = [P, P, P, I, I, I, I, P, P, P, P]
         lib.oracle_reselect.restype = None
-        lib.oracle_reselect.argtypes = [P, P, I, I, I, I, I, I, P, P]
+        lib.oracle_reselect.argtypes = [P, P, I, I, I, I, I, I, I, P, P]
         lib.oracle_lists.restype = I
         lib.oracle_lists.argtypes = [P, P, I, I, I, P, P, P, P]
         lib.oracle_ffn.restype = None
@@ -117,15 +117,17 @@ def route(x, Wg, bias, k: int):
     return logits, probs, ti, tw
 
 
-def reselect(logits, probs, k: int, mode: int, k0: int = 0, budget: int = 0):
-    """-> sel_idx[B][k] int32 (-1 padded), sel_w[B][k] fp32."""
+def reselect(logits, probs, k: int, mode: int, k0: int = 0, budget: int = 0, group: int = 1):
+    """-> sel_idx[B][k] int32 (-1 padded), sel_w[B][k] fp32.  ``group``:
+    tokens per request (MODE_XSHARE_HIER only)."""
     lib = _load()
     logits = _c(logits, np.float32)
     probs = _c(probs, np.float32)
     B, E = logits.shape
     sel = np.empty((B, k), np.int32)
     w = np.empty((B, k), np.float32)
-    lib.oracle_reselect(_p(logits), _p(probs), B, E, k, mode, k0, budget, _p(sel), _p(w))
+    assert group >= 1
+    lib.oracle_reselect(_p(logits), _p(probs), B, E, k, mode, k0, budget, group, _p(sel), _p(w))
     return sel, w
 
 
@@ -167,11 +169,11 @@ def ffn(x, Wgate, Wup, Wdown, sel_idx, sel_w, rows=None, threads: int = 1) -> np
 
 
 def layer(x, L: dict, k: int, mode: int, k0: int = 0, budget: int = 0,
-          rows=None, threads: int = 1):
+          rows=None, threads: int = 1, group: int = 1):
     """Whole layer: route -> reselect -> lists -> FFN.  ``L`` holds the
     arrays of ``moe_synth.make_weights``."""
     logits, probs, ti, tw = route(x, L["Wg"], L.get("bias"), k)
-    sel, w = reselect(logits, probs, k, mode, k0, budget)
+    sel, w = reselect(logits, probs, k, mode, k0, budget, group)
     li = lists(sel, w, L["Wg"].shape[0])
     y = ffn(x, L["Wgate"], L["Wup"], L["Wdown"], sel, w, rows=rows, threads=threads)
     return {"logits": logits, "probs": probs, "topk_idx": ti, "topk_w": tw,

@@ -45,6 +45,12 @@
  *    whose top-k holds the expert; the critical set is the shortest prefix
  *    of the score order (at least k long) that holds every token's rank-0
  *    expert; each token takes its first k experts inside it;
+ *  - XShare's hierarchical selection for speculative batches: a request is
+ *    a run of `group` consecutive tokens (its drafts); each request first
+ *    picks the k experts with the largest request score (its tokens' top-k
+ *    gate probabilities summed), then the batch keeps the min(budget,
+ *    |picked|) picked experts with the largest batch score (the request
+ *    scores of the requests that picked the expert, summed);
  *  - gate weights are renormalised over the chosen set (all modes);
  *  - the expert FFN is SwiGLU: down( silu(gate x) * (up x) ), in fp64.
  *
@@ -52,8 +58,11 @@
  * (see tests/test_oracle_*.py): exp_spec against libm within 2 ulp,
  * canon_dot against an fp64 dot within the forward error bound, the routing
  * against fp64 logits + a stable sort, OEA and XShare against their defining
- * invariants and brute force over subsets, the FFN against a dense fp64
- * torch restatement.
+ * invariants and brute force over subsets, hierarchical XShare against its
+ * two closed forms (one token per request, one request per batch) and brute
+ * force over the subsets of both levels, affinity binning against its
+ * invariants, closed forms and hand-worked cases, the FFN against a dense
+ * fp64 torch restatement.
  */
 #include <math.h>
 #include <stdint.h>
@@ -64,6 +73,7 @@
 #define ORACLE_MODE_OEA 1
 #define ORACLE_MODE_XSHARE 2
 #define ORACLE_MODE_AFFINITY 3
+#define ORACLE_MODE_XSHARE_HIER 4
 
 /* ---------------------------------------------------------------- exp ---
  * exp_spec(x) for x in [-87, 0] (softmax arguments are l - max(l) <= 0).
@@ -212,7 +222,7 @@ void oracle_route(const float *x, const float *Wg, const float *bias,
 }
 
 /* ----------------------------------------------------------- reselect ---
- * sel_idx[b][0..k) and sel_w[b][0..k) for one of three rules.
+ * sel_idx[b][0..k) and sel_w[b][0..k) for one of five rules.
  *   NONE   : the token's top-k (standard routing, [LX] section 1).
  *   OEA    : [OEA].  K_b = first k0 of the order; U_kept = union of all
  *            K_b, fixed before any fill; F_b = the first k - k0 experts of
@@ -234,9 +244,21 @@ void oracle_route(const float *x, const float *Wg, const float *bias,
  *            M = max(k, 1 + the largest position of any r0(b) in that
  *            order); S = its first M experts; sel_b = the first k experts
  *            of the token's order that lie in S (always k of them).
+ *   XSHARE_HIER : [XS] abstract (speculative decoding: hierarchical,
+ *            correlation-aware selection).  Requests R_0, R_1, ... are runs
+ *            of `group` consecutive tokens (the last may be shorter).
+ *            Request level: s_r[e] = sum over b in R_r ascending of
+ *            [e in T_b] p[b][e] (fp32, from +0); P_r = the k experts with
+ *            the largest s_r > 0 (ties to the lower index).  Batch level:
+ *            C = union of the P_r; s[e] = sum over r ascending with e in
+ *            P_r of s_r[e] (fp32, from +0); M' = min(budget, |C|); S = the
+ *            M' experts of C with the largest s (ties to the lower index);
+ *            sel_b = the first k experts of the order that lie in S.
+ *            group = 1 is XSHARE; one request for the whole batch is
+ *            XSHARE with budget k.
  * Weights are renormalised over the chosen set in every mode. */
 void oracle_reselect(const float *logits, const float *probs,
-                     int B, int E, int k, int mode, int k0, int budget,
+                     int B, int E, int k, int mode, int k0, int budget, int group,
                      int *sel_idx, float *sel_w)
 {
     int *order = (int *)malloc(sizeof(int) * (size_t)B * E);
@@ -291,6 +313,63 @@ void oracle_reselect(const float *logits, const float *probs,
         }
         free(s);
         free(ubase);
+    } else if (mode == ORACLE_MODE_XSHARE_HIER) {
+        float *sr = (float *)malloc(sizeof(float) * (size_t)E);    /* request score */
+        float *s = (float *)calloc((size_t)E, sizeof(float));      /* batch score */
+        unsigned char *picked = (unsigned char *)malloc((size_t)E);
+        unsigned char *cand = (unsigned char *)calloc((size_t)E, 1);
+        int nreq = (B + group - 1) / group;
+        for (int r = 0; r < nreq; ++r) {
+            int b0 = r * group, b1 = b0 + group < B ? b0 + group : B;
+            for (int e = 0; e < E; ++e) {
+                float acc = 0.0f;
+                for (int b = b0; b < b1; ++b) {
+                    int in_tb = 0;
+                    for (int j = 0; j < k; ++j) in_tb |= order[(size_t)b * E + j] == e;
+                    if (in_tb) acc = acc + probs[(size_t)b * E + e];
+                }
+                sr[e] = acc;
+                picked[e] = 0;
+            }
+            /* the request's k best experts: take the best remaining one k times */
+            for (int t = 0; t < k; ++t) {
+                int best = -1;
+                for (int e = 0; e < E; ++e) {
+                    if (picked[e] || !(sr[e] > 0.0f)) continue;
+                    if (best < 0 || sr[e] > sr[best]) best = e;   /* equal scores keep the lower index */
+                }
+                if (best < 0) break;
+                picked[best] = 1;
+            }
+            for (int e = 0; e < E; ++e)
+                if (picked[e]) {
+                    s[e] = s[e] + sr[e];
+                    cand[e] = 1;
+                }
+        }
+        int ncand = 0;
+        for (int e = 0; e < E; ++e) ncand += cand[e];
+        int Mp = budget < ncand ? budget : ncand;
+        for (int t = 0; t < Mp; ++t) {
+            int best = -1;
+            for (int e = 0; e < E; ++e) {
+                if (!cand[e] || inset[e]) continue;
+                if (best < 0 || s[e] > s[best]) best = e;
+            }
+            inset[best] = 1;
+        }
+        for (int b = 0; b < B; ++b) {
+            const int *ord = order + (size_t)b * E;
+            int *sel = sel_idx + (size_t)b * k;
+            int n = 0;
+            for (int j = 0; j < E && n < k; ++j)
+                if (inset[ord[j]]) sel[n++] = ord[j];
+            while (n < k) sel[n++] = -1;
+        }
+        free(sr);
+        free(s);
+        free(picked);
+        free(cand);
     } else if (mode == ORACLE_MODE_AFFINITY) {
         int nb = (E + k - 1) / k;
         if (nb > 32) nb = 32;

@@ -12,6 +12,12 @@ Inference", AI summary and abstract): the chosen expert set is compared
 with an exhaustive search over all subsets of the batch union for the
 modular objective, plus the closed form budget >= |union| (standard top-k).
 
+XShare's hierarchical selection for speculative batches (same page,
+abstract): the closed forms group = 1 (plain XShare) and one request for the
+whole batch (plain XShare with budget k), an exhaustive search over the
+subsets at both levels on tiny batches, and a hand-worked case where the
+request level changes the batch set.
+
 Hand-derived cases (worked out in the comments) pin the fill order and the
 tie rules.
 """
@@ -22,7 +28,7 @@ import pytest
 
 import moe_synth as ms
 
-NONE, OEA, XSHARE = 0, 1, 2
+NONE, OEA, XSHARE, XSHARE_HIER = 0, 1, 2, 4
 
 
 def _rank_order(logits):
@@ -366,3 +372,169 @@ def test_affinity_hand_worked_tie(oracle_lib):
     sel, w = oracle_lib.reselect(logits, probs, 2, AFFINITY)
     assert sel.tolist() == [[5, 2], [2, 5]]
     assert np.allclose(w, [[.5, .5], [.25 / .375, .125 / .375]], rtol=2e-7, atol=0)
+
+
+# ---------------------------------------------------------------- XShare,
+# hierarchical: requests are runs of `group` consecutive tokens.
+
+def _hier_brute(probs, order, k, budget, group):
+    """Exhaustive restatement in fp64: each request's best k-subset of the
+    experts its tokens' top-k sets hold (by summed request score), then the
+    best min(budget, |picked|)-subset of the picked experts by batch score.
+    Returns the batch set and the smallest margin between the best and the
+    second-best subset seen at any level (near ties make the answer depend
+    on rounding, so callers require a clear margin)."""
+    B, E = probs.shape
+    s = np.zeros(E)
+    picked = set()
+    margin = np.inf
+
+    def best_two(pool, size, score):
+        vals = sorted((score[list(c)].sum(), c) for c in itertools.combinations(pool, size))
+        gap = vals[-1][0] - vals[-2][0] if len(vals) > 1 else np.inf
+        return set(vals[-1][1]), gap
+
+    for r0 in range(0, B, group):
+        sr = np.zeros(E)
+        for b in range(r0, min(B, r0 + group)):
+            for e in order[b, :k]:
+                sr[e] += float(probs[b, e])
+        pool = [e for e in range(E) if sr[e] > 0]
+        P, gap = best_two(pool, min(k, len(pool)), sr)
+        margin = min(margin, gap)
+        for e in P:
+            s[e] += sr[e]
+        picked |= P
+    pool = sorted(picked)
+    S, gap = best_two(pool, min(budget, len(pool)), s)
+    return S, min(margin, gap)
+
+
+def check_hier(logits, probs, sel, w, k, budget, group):
+    """Invariants that hold at any size: the activated set A is the batch
+    set (every member of it is in the top-k of some token that takes it),
+    A lies in the union of the top-k sets, |A| <= min(budget, requests * k),
+    each token takes its first k experts inside A, weights renormalised."""
+    order = _rank_order(logits)
+    B, E = logits.shape
+    nreq = -(-B // group)
+    u_base = set(order[:, :k].ravel().tolist())
+    A = set(e for e in sel.ravel().tolist() if e >= 0)
+    assert A <= u_base
+    assert k <= len(A) <= min(budget, nreq * k)
+    for b in range(B):
+        row = sel[b].tolist()
+        assert all(e >= 0 for e in row) and len(set(row)) == k
+        assert row == [e for e in order[b].tolist() if e in A][:k]
+    _check_weights(probs, sel, w)
+    return A
+
+
+@pytest.mark.parametrize("seed", range(4))
+@pytest.mark.parametrize("budget", [8, 12, 20, 128])
+def test_xshare_hier_one_token_per_request_is_xshare(oracle_lib, seed, budget):
+    rng = np.random.default_rng(300 + seed)
+    logits, probs = _random_router(rng, 19, 128)
+    s_x, w_x = oracle_lib.reselect(logits, probs, 8, XSHARE, budget=budget)
+    s_h, w_h = oracle_lib.reselect(logits, probs, 8, XSHARE_HIER, budget=budget, group=1)
+    assert np.array_equal(s_x, s_h)
+    assert np.array_equal(w_x.view(np.uint32), w_h.view(np.uint32))
+
+
+@pytest.mark.parametrize("seed", range(4))
+@pytest.mark.parametrize("group", [16, 17, 1000])
+def test_xshare_hier_one_request_is_xshare_with_budget_k(oracle_lib, seed, group):
+    # one request: its k picked experts are the batch's top-k by the summed
+    # score, so any budget >= k gives plain XShare with budget k
+    rng = np.random.default_rng(400 + seed)
+    logits, probs = _random_router(rng, 16, 64)
+    s_x, w_x = oracle_lib.reselect(logits, probs, 8, XSHARE, budget=8)
+    for budget in (8, 13, 64):
+        s_h, w_h = oracle_lib.reselect(logits, probs, 8, XSHARE_HIER, budget=budget, group=group)
+        assert np.array_equal(s_x, s_h)
+        assert np.array_equal(w_x.view(np.uint32), w_h.view(np.uint32))
+
+
+@pytest.mark.parametrize("seed", range(8))
+@pytest.mark.parametrize("B,group", [(4, 2), (6, 4), (6, 3), (5, 2)])
+@pytest.mark.parametrize("budget", [4, 6, 8])
+def test_xshare_hier_brute_force_tiny(oracle_lib, seed, B, group, budget):
+    # E=16, k=4: every k-subset at the request level and every subset of the
+    # picked experts at the batch level is tried
+    rng = np.random.default_rng(2000 + 10 * seed + B)
+    logits, probs = _random_router(rng, B, 16, scale=1.0, skew=0.5)
+    sel, w = oracle_lib.reselect(logits, probs, 4, XSHARE_HIER, budget=budget, group=group)
+    A = check_hier(logits, probs, sel, w, 4, budget, group)
+    S, margin = _hier_brute(probs, _rank_order(logits), 4, budget, group)
+    if margin > 1e-5:  # a clear optimum at every level
+        assert A == S
+    else:
+        pytest.skip("near tie")
+
+
+def test_xshare_hier_brute_force_has_clear_cases(oracle_lib):
+    # the brute-force comparison above must not be skipped wholesale
+    clear = 0
+    for seed in range(8):
+        for B, group in [(4, 2), (6, 4), (6, 3), (5, 2)]:
+            rng = np.random.default_rng(2000 + 10 * seed + B)
+            logits, probs = _random_router(rng, B, 16, scale=1.0, skew=0.5)
+            for budget in (4, 6, 8):
+                _, margin = _hier_brute(probs, _rank_order(logits), 4, budget, group)
+                clear += margin > 1e-5
+    assert clear >= 80
+
+
+@pytest.mark.parametrize("budget", [24, 32, 48])
+def test_xshare_hier_speculative_batch(oracle_lib, budget):
+    # 8 requests x 4 drafts on the Qwen3-30B-shaped router
+    S = ms.SHAPES["q30b"]
+    L = ms.make_weights(S, 0, experts=False)
+    x = ms.make_tokens(S, 32, 0, kind="spec")
+    logits, probs, ti, tw = oracle_lib.route(x, L["Wg"], L["bias"], S.k)
+    sel, w = oracle_lib.reselect(logits, probs, S.k, XSHARE_HIER, budget=budget, group=4)
+    check_hier(logits, probs, sel, w, S.k, budget, 4)
+
+
+def test_xshare_hier_hand_worked_example(oracle_lib):
+    # E=6, k=2, B=4 in two requests of two tokens (group=2).  Probabilities
+    # are dyadic, so every sum below is exact; logits = log2 p.
+    #   token 0: p = [.5 .25 .125 .0625 .03125 .03125]     T = {0, 1}
+    #   token 1: p = [.5 .03125 .375 .03125 .03125 .03125] T = {0, 2}
+    #   token 2: p = [.03125 .375 .03125 .5 .03125 .03125] T = {3, 1}
+    #   token 3: p = [.0625 .0625 .0625 .25 .5 .0625]      T = {4, 3}
+    # request 0 scores: e0 = 1, e1 = .25, e2 = .375   -> picks {0, 2}
+    # request 1 scores: e3 = .75, e1 = .375, e4 = .5  -> picks {3, 4}
+    # batch scores over the picks: e0 = 1, e3 = .75, e4 = .5, e2 = .375
+    #   budget 3 -> S = {0, 3, 4}; budget 4 (or more) -> S = {0, 2, 3, 4}.
+    # Flat XShare scores add e1 = .25 + .375 = .625 instead, so with budget 3
+    # it keeps {0, 3, 1}: the request level drops e1, which neither request
+    # ranks among its own two best.
+    # Each token then takes its first two experts inside S (order by p,
+    # equal p to the lower index): budget 3 -> [0 3] [0 3] [3 0] [4 3].
+    p = np.array([[.5, .25, .125, .0625, .03125, .03125],
+                  [.5, .03125, .375, .03125, .03125, .03125],
+                  [.03125, .375, .03125, .5, .03125, .03125],
+                  [.0625, .0625, .0625, .25, .5, .0625]], np.float32)
+    logits = np.log2(p).astype(np.float32)
+    sel, w = oracle_lib.reselect(logits, p, 2, XSHARE_HIER, budget=3, group=2)
+    assert sel.tolist() == [[0, 3], [0, 3], [3, 0], [4, 3]]
+    f = np.float32
+    expect = [[f(.5) / f(.5625), f(.0625) / f(.5625)], [f(.5) / f(.53125), f(.03125) / f(.53125)],
+              [f(.5) / f(.53125), f(.03125) / f(.53125)], [f(.5) / f(.75), f(.25) / f(.75)]]
+    assert np.array_equal(w, np.array(expect, np.float32))
+    sel4, _ = oracle_lib.reselect(logits, p, 2, XSHARE_HIER, budget=4, group=2)
+    assert sel4.tolist() == [[0, 2], [0, 2], [3, 0], [4, 3]]
+    flat, _ = oracle_lib.reselect(logits, p, 2, XSHARE, budget=3)
+    assert flat.tolist() == [[0, 1], [0, 1], [3, 1], [3, 0]]
+
+
+def test_xshare_hier_lists_reconstruct_selection(oracle_lib):
+    rng = np.random.default_rng(9)
+    B, E, k = 23, 64, 8
+    logits, probs = _random_router(rng, B, E)
+    sel, w = oracle_lib.reselect(logits, probs, k, XSHARE_HIER, budget=20, group=4)
+    li = oracle_lib.lists(sel, w, E)
+    n = li["n_active"]
+    assert set(li["active"][:n].tolist()) == set(sel.ravel().tolist())
+    assert li["offsets"][n] == B * k
