@@ -18,7 +18,8 @@ import os
 import torch
 
 __all__ = [
-    "MOE_RESELECT_NONE", "MOE_RESELECT_OEA", "MOE_RESELECT_XSHARE", "MoeError",
+    "MOE_RESELECT_NONE", "MOE_RESELECT_OEA", "MOE_RESELECT_XSHARE", "MOE_RESELECT_AFFINITY",
+    "MOE_RESELECT_XSHARE_HIER", "MoeError",
     "Dims", "Rule", "Lists", "load_library", "library_path", "moe_workspace_bytes",
     "moe_status_string", "moe_route", "moe_reselect", "moe_expert_ffn", "moe_layer_decode",
     "moe_check_error", "moe_expert_ffn_noalloc", "new_workspace", "alloc_lists", "ABI_SYMBOLS",
@@ -26,6 +27,7 @@ __all__ = [
 ]
 
 MOE_RESELECT_NONE, MOE_RESELECT_OEA, MOE_RESELECT_XSHARE = 0, 1, 2
+MOE_RESELECT_AFFINITY, MOE_RESELECT_XSHARE_HIER = 3, 4
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_MISALIGNED", 3: "MOE_ERR_WORKSPACE",
           4: "MOE_ERR_UNSUPPORTED", 5: "MOE_ERR_CUDA", 6: "MOE_ERR_INTERNAL"}
 ABI_SYMBOLS = ("moe_workspace_bytes", "moe_route", "moe_reselect", "moe_expert_ffn",
@@ -49,7 +51,8 @@ class Dims(ctypes.Structure):
 
 
 class Rule(ctypes.Structure):
-    _fields_ = [("mode", ctypes.c_int32), ("k0", ctypes.c_int32), ("budget", ctypes.c_int32)]
+    _fields_ = [("mode", ctypes.c_int32), ("k0", ctypes.c_int32), ("budget", ctypes.c_int32),
+                ("group", ctypes.c_int32)]
 
 
 class Lists(ctypes.Structure):
@@ -160,8 +163,9 @@ def moe_route(x, Wg, bias, k: int, out=None, stream=None):
 
 
 def moe_reselect(logits, probs, k: int, mode: int, k0: int = 0, budget: int = 0,
-                 out=None, lists=None, stream=None):
-    """-> (sel_idx[B][k], sel_w[B][k], lists dict)."""
+                 out=None, lists=None, stream=None, group: int = 1):
+    """-> (sel_idx[B][k], sel_w[B][k], lists dict).  ``group``: tokens per
+    request (hierarchical XShare)."""
     B, E = logits.shape
     if out is None:
         out = (torch.empty(B, k, dtype=torch.int32, device=logits.device),
@@ -169,7 +173,8 @@ def moe_reselect(logits, probs, k: int, mode: int, k0: int = 0, budget: int = 0,
     if lists is None:
         lists = alloc_lists(B, E, k, logits.device)
     sel, w = out
-    st = load_library().moe_reselect(_ptr(logits), _ptr(probs), Dims(B, 0, E, k, 0), Rule(mode, k0, budget),
+    st = load_library().moe_reselect(_ptr(logits), _ptr(probs), Dims(B, 0, E, k, 0),
+                                     Rule(mode, k0, budget, group),
                                      _ptr(sel), _ptr(w), _lists(lists), _stream(stream))
     _check(st, "moe_reselect")
     return sel, w, lists
@@ -189,7 +194,7 @@ def moe_expert_ffn(x, Wgate, Wup, Wdown, lists: dict, k: int, ws, y=None, stream
 
 
 def moe_layer_decode(x, Wg, bias, Wgate, Wup, Wdown, k: int, mode: int, k0: int = 0, budget: int = 0,
-                     ws=None, y=None, sel_idx=None, sel_w=None, n_active=None, stream=None):
+                     ws=None, y=None, sel_idx=None, sel_w=None, n_active=None, stream=None, group: int = 1):
     """Whole layer; -> y[B][d] fp32.  Optional device outputs sel_idx[B][k],
     sel_w[B][k], n_active[1] are filled when given."""
     B, d = x.shape
@@ -200,7 +205,7 @@ def moe_layer_decode(x, Wg, bias, Wgate, Wup, Wdown, k: int, mode: int, k0: int 
         y = torch.empty(B, d, dtype=torch.float32, device=x.device)
     st = load_library().moe_layer_decode(
         _ptr(x), _ptr(Wg), _ptr(bias), _ptr(Wgate), _ptr(Wup), _ptr(Wdown), Dims(B, d, E, k, F),
-        Rule(mode, k0, budget), _ptr(y), _ptr(sel_idx), _ptr(sel_w), _ptr(n_active), _ptr(ws),
+        Rule(mode, k0, budget, group), _ptr(y), _ptr(sel_idx), _ptr(sel_w), _ptr(n_active), _ptr(ws),
         ws.numel() * ws.element_size(), _stream(stream))
     _check(st, "moe_layer_decode")
     return y

@@ -37,6 +37,8 @@ bool rule_ok(const moe_dims_t &d, const moe_reselect_t &r) {
         case MOE_RESELECT_OEA: return r.k0 >= 1 && r.k0 <= d.k;
         case MOE_RESELECT_XSHARE: return r.budget >= d.k && r.budget <= d.E;
         case MOE_RESELECT_AFFINITY: return true;
+        case MOE_RESELECT_XSHARE_HIER:
+            return r.budget >= d.k && r.budget <= d.E && r.group >= 1 && r.group <= B_MAX;
         default: return false;
     }
 }

@@ -236,6 +236,7 @@ struct ReselectArgs {
     int fuse_softmax;
     int cache_rows;  // logits / probabilities kept in shared memory
     int B, E, k, mode, k0, budget;
+    int group;  // hierarchical XShare: tokens per request
     int32_t *sel_idx;
     float *sel_w;
     moe_lists_t lists;
@@ -387,6 +388,9 @@ __device__ void reselect_body(const ReselectArgs &a, unsigned char *smem_raw) {
     unsigned *TMEMB = ASSIGN + E * BW;                                // [E][BW] top-k membership
     float *PC = reinterpret_cast<float *>(TMEMB + E * BW);           // [B][E] probability cache
     float *LC = PC + (a.cache_rows ? B * E : 0);                      // [B][E] logit cache
+    // hierarchical XShare: bit r of word RPICK[e * BW + r / 32] = request r
+    // picked expert e (present only in that mode)
+    unsigned *RPICK = reinterpret_cast<unsigned *>(LC + (a.cache_rows ? B * E : 0));
     __shared__ float s_score[E_MAX];
     __shared__ int s_off[E_MAX];
     __shared__ int s_rank[E_MAX];  // expert -> active slot (publishing path)
@@ -467,7 +471,8 @@ __device__ void reselect_body(const ReselectArgs &a, unsigned char *smem_raw) {
             T[b * k + lane] = mye;
             if (mode == MOE_RESELECT_OEA) atomicOr(&ukept[mye >> 5], 1u << (mye & 31));
             if (mode != MOE_RESELECT_OEA) atomicOr(&ubase[mye >> 5], 1u << (mye & 31));
-            if (mode == MOE_RESELECT_XSHARE) atomicOr(&TMEMB[mye * BW + (b >> 5)], 1u << (b & 31));
+            if (mode == MOE_RESELECT_XSHARE || mode == MOE_RESELECT_XSHARE_HIER)
+                atomicOr(&TMEMB[mye * BW + (b >> 5)], 1u << (b & 31));
         }
         if (mode == MOE_RESELECT_NONE && lane < k) {
             a.sel_idx[static_cast<size_t>(b) * k + lane] = mye;
@@ -495,6 +500,69 @@ __device__ void reselect_body(const ReselectArgs &a, unsigned char *smem_raw) {
         int nbase = 0;
         for (int i = 0; i < E_MAX / 32; ++i) nbase += __popc(ubase[i]);
         const int Mp = a.budget < nbase ? a.budget : nbase;
+#pragma unroll 1
+        for (int e = warp; e < E; e += nwarps) {
+            if (s_aff[e] == 0ull) continue;
+            const int rank = warp_rank(s_aff, E, e, lane);
+            if (lane == 0 && rank < Mp) atomicOr(&sbits[e >> 5], 1u << (e & 31));
+        }
+        __syncthreads();
+    }
+
+    // ---- hierarchical XShare.  Request level (one warp per request, a run
+    // of `group` tokens): the request score of expert e sums the
+    // probabilities of the request's tokens whose top-k holds e (tokens
+    // ascending); the request picks its k best experts (score > 0; ties to
+    // the lower index).  Batch level: the batch score sums the request
+    // scores of the requests that picked e (requests ascending), and the
+    // batch set is the first min(budget, |picked|) picked experts by it.
+    if (mode == MOE_RESELECT_XSHARE_HIER) {
+        const int G = a.group;
+        const int nreq = (B + G - 1) / G;
+        for (int i = tid; i < E * BW; i += blockDim.x) RPICK[i] = 0u;
+        __syncthreads();
+#pragma unroll 1
+        for (int r = warp; r < nreq; r += nwarps) {
+            const int bb = r * G, be = min(B, bb + G);
+            unsigned o[NI];
+            unsigned cand = 0u;
+#pragma unroll
+            for (int i = 0; i < NI; ++i) {
+                const int e = lane + 32 * i;
+                float sc = 0.0f;
+                if (e < E)
+                    for (int b = bb; b < be; ++b)
+                        if ((TMEMB[e * BW + (b >> 5)] >> (b & 31)) & 1u)
+                            sc = __fadd_rn(sc, prob_rows[static_cast<size_t>(b) * E + e]);
+                o[i] = ord_of(sc);
+                if (sc > 0.0f) cand |= 1u << i;
+            }
+#pragma unroll 1
+            for (int j = 0; j < k; ++j) {
+                const int e = warp_argmax<NI>(o, cand, lane);
+                if (e < 0) break;
+                if ((e & 31) == lane) atomicOr(&RPICK[e * BW + (r >> 5)], 1u << (r & 31));
+            }
+        }
+        __syncthreads();
+        bool picked = false;
+        if (tid < E) {
+            float sc = 0.0f;
+#pragma unroll 1
+            for (int r = 0; r < nreq; ++r) {
+                if (!((RPICK[tid * BW + (r >> 5)] >> (r & 31)) & 1u)) continue;
+                picked = true;
+                float sr = 0.0f;
+                const int bb = r * G, be = min(B, bb + G);
+                for (int b = bb; b < be; ++b)
+                    if ((TMEMB[tid * BW + (b >> 5)] >> (b & 31)) & 1u)
+                        sr = __fadd_rn(sr, prob_rows[static_cast<size_t>(b) * E + tid]);
+                sc = __fadd_rn(sc, sr);
+            }
+            s_aff[tid] = picked ? key_float_score(sc, tid) : 0ull;
+        }
+        const int npicked = __syncthreads_count(picked ? 1 : 0);
+        const int Mp = a.budget < npicked ? a.budget : npicked;
 #pragma unroll 1
         for (int e = warp; e < E; e += nwarps) {
             if (s_aff[e] == 0ull) continue;
@@ -689,10 +757,11 @@ struct GemvArgs {
     float *y;         // layer path: zeroed
     Counters *ctr;    // layer path only (else null)
     int r1;           // first ranks per token in the published set (0: none)
-    // batch-wide rule whose set the router publishes (MOE_RESELECT_XSHARE or
-    // MOE_RESELECT_AFFINITY; 0: none) with its parameters; B <= 32
-    int batch_rule, k, budget;
-    float *probs;     // XShare: the tokens' probabilities, written here
+    // batch-wide rule whose set the router publishes (MOE_RESELECT_XSHARE,
+    // MOE_RESELECT_XSHARE_HIER or MOE_RESELECT_AFFINITY; 0: none) with its
+    // parameters; B <= 32
+    int batch_rule, k, budget, group;
+    float *probs;     // XShare rules: the tokens' probabilities, written here
 };
 
 constexpr int GEMV_TPB_MAX = 4;
@@ -788,10 +857,11 @@ __device__ __forceinline__ void gemv_rows(const unsigned char *wrow, const unsig
     }
 }
 
-// XShare and affinity binning need every token of the batch.  Each token
-// group's last block adds its tokens' contributions (top-k membership and,
-// for XShare, the probability rows; for affinity binning the 2^bin scores
-// and the rank-0 experts); the last group to do so computes the set with
+// The XShare rules and affinity binning need every token of the batch.
+// Each token group's last block adds its tokens' contributions (top-k
+// membership and, for XShare, the probability rows; for affinity binning
+// the 2^bin scores and the rank-0 experts); the last group to do so
+// computes the set with
 // the same definitions as the selection kernel, publishes it (the mask of
 // every copy, then one more count) and clears the contributions.  Called by
 // every thread of a group's last block; B <= 32.  `work`: the block's
@@ -801,6 +871,7 @@ __device__ void batch_rule_publish(const GemvArgs &g, int b0, int nb, unsigned *
                                    int *s_flag, unsigned char *work) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
     const int E = g.E, k = g.k;
+    const bool xs = g.batch_rule == MOE_RESELECT_XSHARE || g.batch_rule == MOE_RESELECT_XSHARE_HIER;
     Counters *ctr = g.ctr;
 #pragma unroll 1
     for (int t = warp; t < nb; t += nw) {
@@ -811,7 +882,7 @@ __device__ void batch_rule_publish(const GemvArgs &g, int b0, int nb, unsigned *
 #pragma unroll
         for (int i = 0; i < NI; ++i) ord[i] = ord_of(l[i]);
         token_softmax_r<NI>(l, ord, E, lane, p);
-        if (g.batch_rule == MOE_RESELECT_XSHARE) {
+        if (xs) {
 #pragma unroll
             for (int i = 0; i < NI; ++i)
                 if (lane + 32 * i < E) g.probs[static_cast<size_t>(b) * E + lane + 32 * i] = p[i];
@@ -824,7 +895,7 @@ __device__ void batch_rule_publish(const GemvArgs &g, int b0, int nb, unsigned *
             if (lane == j) mye = e;
         }
         if (lane < k) atomicOr(&ctr->ubase_bits[mye >> 5], 1u << (mye & 31));
-        if (g.batch_rule == MOE_RESELECT_XSHARE) {
+        if (xs) {
             if (lane < k) atomicOr(&ctr->memb[mye], 1u << b);
         } else {
             const int r0 = __shfl_sync(FULL, mye, 0);
@@ -865,7 +936,7 @@ __device__ void batch_rule_publish(const GemvArgs &g, int b0, int nb, unsigned *
         s_r0[threadIdx.x] = __ldcg(&ctr->r0_bits[threadIdx.x]);
     }
     if (threadIdx.x == 0) *s_M = k;
-    if (g.batch_rule == MOE_RESELECT_XSHARE) {
+    if (xs) {
         for (int i = threadIdx.x; i < g.B * E; i += blockDim.x) s_pr[i] = __ldcg(g.probs + i);
         for (int e = threadIdx.x; e < E; e += blockDim.x) s_sc[e] = __ldcg(&ctr->memb[e]);
     } else {
@@ -874,11 +945,66 @@ __device__ void batch_rule_publish(const GemvArgs &g, int b0, int nb, unsigned *
     __syncthreads();
     int nbase = 0;
     for (int i = 0; i < E_MAX / 32; ++i) nbase += __popc(s_ub[i]);
+    // hierarchical XShare, request level (one warp per request of `group`
+    // tokens): bit r of s_pick[e] = request r picked expert e, one of its k
+    // best by request score; s_r0 (unused by this rule) collects the picks
+    unsigned *s_pick = reinterpret_cast<unsigned *>(s_xs);  // [E_MAX]
+    const int G = g.group > 0 ? g.group : 1, nreq = (g.B + G - 1) / G;
+    if (g.batch_rule == MOE_RESELECT_XSHARE_HIER) {
+        for (int e = threadIdx.x; e < E_MAX; e += blockDim.x) s_pick[e] = 0u;
+        if (threadIdx.x < E_MAX / 32) s_r0[threadIdx.x] = 0u;
+        __syncthreads();
+#pragma unroll 1
+        for (int r = warp; r < nreq; r += nw) {
+            const int bb = r * G, be = min(g.B, bb + G);
+            unsigned o[NI];
+            unsigned cand = 0u;
+#pragma unroll
+            for (int i = 0; i < NI; ++i) {
+                const int e = lane + 32 * i;
+                float sc = 0.0f;
+                if (e < E) {
+                    const unsigned m = static_cast<unsigned>(s_sc[e]);
+                    for (int b = bb; b < be; ++b)
+                        if ((m >> b) & 1u) sc = __fadd_rn(sc, s_pr[b * E + e]);
+                }
+                o[i] = ord_of(sc);
+                if (sc > 0.0f) cand |= 1u << i;
+            }
+#pragma unroll 1
+            for (int j = 0; j < k; ++j) {
+                const int e = warp_argmax<NI>(o, cand, lane);
+                if (e < 0) break;
+                if ((e & 31) == lane) {
+                    atomicOr(&s_pick[e], 1u << r);
+                    atomicOr(&s_r0[e >> 5], 1u << (e & 31));
+                }
+            }
+        }
+        __syncthreads();
+        nbase = 0;
+        for (int i = 0; i < E_MAX / 32; ++i) nbase += __popc(s_r0[i]);
+    }
     // sort keys of the batch union (0 for other experts), in place of the
-    // scores; XShare first sums each expert's probabilities (tokens ascending)
+    // scores; XShare first sums each expert's probabilities (tokens
+    // ascending), its hierarchical form the request scores of the requests
+    // that picked the expert (requests ascending)
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         const bool member = (s_ub[e >> 5] >> (e & 31)) & 1u;
-        if (g.batch_rule == MOE_RESELECT_XSHARE) {
+        if (g.batch_rule == MOE_RESELECT_XSHARE_HIER) {
+            const unsigned m = static_cast<unsigned>(s_sc[e]);
+            const unsigned picks = s_pick[e];
+            float sc = 0.0f;
+            for (int r = 0; r < nreq; ++r) {
+                if (!((picks >> r) & 1u)) continue;
+                float sr = 0.0f;
+                const int bb = r * G, be = min(g.B, bb + G);
+                for (int b = bb; b < be; ++b)
+                    if ((m >> b) & 1u) sr = __fadd_rn(sr, s_pr[b * E + e]);
+                sc = __fadd_rn(sc, sr);
+            }
+            s_sc[e] = picks ? key_float_score(sc, e) : 0ull;
+        } else if (g.batch_rule == MOE_RESELECT_XSHARE) {
             const unsigned m = static_cast<unsigned>(s_sc[e]);
             float sc = 0.0f;
             for (int b = 0; b < g.B; ++b)
@@ -899,9 +1025,10 @@ __device__ void batch_rule_publish(const GemvArgs &g, int b0, int nb, unsigned *
         }
     }
     __syncthreads();
-    // XShare: the first min(budget, |union|); affinity binning: the shortest
-    // prefix, at least k long, holding every rank-0 expert
-    const int cut = g.batch_rule == MOE_RESELECT_XSHARE ? (g.budget < nbase ? g.budget : nbase) : *s_M;
+    // XShare: the first min(budget, |union|) (hierarchical: |picked|);
+    // affinity binning: the shortest prefix, at least k long, holding every
+    // rank-0 expert
+    const int cut = xs ? (g.budget < nbase ? g.budget : nbase) : *s_M;
     for (int e = threadIdx.x; e < E; e += blockDim.x)
         if (s_sc[e] != 0ull && pos_of[e] < cut) atomicOr(&s_mask[e >> 5], 1u << (e & 31));
     __syncthreads();
@@ -1076,9 +1203,10 @@ GemvShape gemv_shape(const moe_dims_t &d) {
 
 int ni_for(int E) { return E <= 32 ? 1 : E <= 64 ? 2 : E <= 128 ? 4 : 8; }
 
-size_t reselect_smem(const moe_dims_t &d, int *cache_rows) {
+size_t reselect_smem(const moe_dims_t &d, const moe_reselect_t &r, int *cache_rows) {
     const int BW = (d.B + 31) / 32;
-    const size_t base = static_cast<size_t>(d.B) * d.k * 4 + static_cast<size_t>(d.E) * BW * 8;
+    const size_t picks = r.mode == MOE_RESELECT_XSHARE_HIER ? static_cast<size_t>(d.E) * BW * 4 : 0;
+    const size_t base = static_cast<size_t>(d.B) * d.k * 4 + static_cast<size_t>(d.E) * BW * 8 + picks;
     const size_t rows = static_cast<size_t>(d.B) * d.E * 8;
     *cache_rows = (base + rows <= 96u * 1024u) ? 1 : 0;
     return base + (*cache_rows ? rows : 0);
@@ -1097,6 +1225,7 @@ ReselectArgs make_reselect_args(const float *logits, float *probs, bool fuse_sof
     a.mode = r.mode;
     a.k0 = r.k0;
     a.budget = r.budget;
+    a.group = r.mode == MOE_RESELECT_XSHARE_HIER ? r.group : 1;
     a.sel_idx = sel_idx;
     a.sel_w = sel_w;
     a.lists = l;
@@ -1155,6 +1284,7 @@ GemvArgs make_gemv_args(const float *bias, const moe_dims_t &d, const GemvShape 
     g.batch_rule = 0;
     g.k = d.k;
     g.budget = 0;
+    g.group = 1;
     g.probs = nullptr;
     return g;
 }
@@ -1223,13 +1353,14 @@ cudaError_t launch_reselect(const float *logits, const float *probs, const moe_d
                             cudaStream_t s) {
     ReselectArgs a = make_reselect_args(logits, const_cast<float *>(probs), false, d, r, sel_idx, sel_w, l,
                                         nullptr);
-    const size_t smem = reselect_smem(d, &a.cache_rows);
+    const size_t smem = reselect_smem(d, r, &a.cache_rows);
     return launch_reselect_args(a, smem, false, s);
 }
 
 int layer_pub_target(const moe_dims_t &d, const moe_reselect_t &rule) {
     const GemvShape sh = gemv_shape(d);
-    const bool sel_publishes = rule.mode == MOE_RESELECT_XSHARE || rule.mode == MOE_RESELECT_AFFINITY;
+    const bool sel_publishes = rule.mode == MOE_RESELECT_XSHARE || rule.mode == MOE_RESELECT_AFFINITY ||
+                               rule.mode == MOE_RESELECT_XSHARE_HIER;
     return (d.B + sh.tpb - 1) / sh.tpb + (sel_publishes ? 1 : 0);
 }
 
@@ -1243,9 +1374,11 @@ cudaError_t launch_layer_route(const RouterMaps &maps, const float *x, const flo
     g.y = y;
     g.ctr = ctr;
     g.r1 = rule.mode == MOE_RESELECT_OEA ? rule.k0 : (rule.mode == MOE_RESELECT_NONE ? d.k : 0);
-    const bool batch = rule.mode == MOE_RESELECT_XSHARE || rule.mode == MOE_RESELECT_AFFINITY;
+    const bool batch = rule.mode == MOE_RESELECT_XSHARE || rule.mode == MOE_RESELECT_AFFINITY ||
+                       rule.mode == MOE_RESELECT_XSHARE_HIER;
     g.batch_rule = (early && batch && d.B <= 32) ? rule.mode : 0;
     g.budget = rule.budget;
+    g.group = rule.mode == MOE_RESELECT_XSHARE_HIER ? rule.group : 1;
     g.probs = probs;
     return launch_gemv(maps, g, sh, s);
 }
@@ -1257,7 +1390,7 @@ cudaError_t launch_layer_select(const float *logits, float *probs, const moe_dim
     a.ctr = ctr;
     a.early_dependents = early ? 1 : 0;
     a.wd = wd;
-    const size_t smem = reselect_smem(d, &a.cache_rows);
+    const size_t smem = reselect_smem(d, rule, &a.cache_rows);
     return launch_reselect_args(a, smem, true, s);
 }
 

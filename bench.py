@@ -58,6 +58,8 @@ WORKLOADS = {
     "spec_xshare32": dict(shape="q30b", B=32, mode=2, k0=0, budget=32, rule="XShare budget=32",
                           kind="spec"),
     "q30b_b16_affinity": dict(shape="q30b", B=16, mode=3, k0=0, budget=0, rule="Lynx affinity binning"),
+    "spec_xshare_hier32": dict(shape="q30b", B=32, mode=4, k0=0, budget=32, group=4, kind="spec",
+                               rule="hierarchical XShare budget=32, 4 tokens per request"),
 }
 
 # DRAM bytes (read + write) per launch of the expert kernel from an ncu
@@ -172,20 +174,22 @@ def run_reference(args, w, rank):
     L = ms.make_weights(S, 0)
     x = ms.make_tokens(S, w["B"], 0, kind=w.get("kind", "normal"))
     cores = len(os.sched_getaffinity(0))
-    r0 = oracle.layer(x, L, S.k, w["mode"], w["k0"], w["budget"], rows=np.arange(1, dtype=np.int32),
+    r0 = oracle.layer(x, L, S.k, w["mode"], w["k0"], w["budget"], group=w.get("group", 1),
+                      rows=np.arange(1, dtype=np.int32),
                       threads=cores)
     n_active = r0["lists"]["n_active"]
     total_bytes, _ = algorithmic_bytes(S, w["B"], n_active)
     # size one step: route + re-select the whole batch, FFN for `rows` tokens
     t0 = time.perf_counter()
-    oracle.layer(x, L, S.k, w["mode"], w["k0"], w["budget"], rows=np.arange(1, dtype=np.int32), threads=cores)
+    oracle.layer(x, L, S.k, w["mode"], w["k0"], w["budget"], group=w.get("group", 1),
+                 rows=np.arange(1, dtype=np.int32), threads=cores)
     t_one = time.perf_counter() - t0
     budget_s = 150.0 / max(1, args.steps + args.warmup)
     rows = int(max(1, min(w["B"], budget_s / max(t_one, 1e-6))))
     sel = np.arange(rows, dtype=np.int32)
 
     def step():
-        oracle.layer(x, L, S.k, w["mode"], w["k0"], w["budget"], rows=sel, threads=cores)
+        oracle.layer(x, L, S.k, w["mode"], w["k0"], w["budget"], group=w.get("group", 1), rows=sel, threads=cores)
 
     for _ in range(args.warmup):
         step()
@@ -214,7 +218,7 @@ def cpu_baseline(w, S, L, x, seconds=12.0):
     t0 = time.perf_counter()
     nact = None
     while True:
-        r = oracle.layer(x, L, S.k, w["mode"], w["k0"], w["budget"], threads=cores)
+        r = oracle.layer(x, L, S.k, w["mode"], w["k0"], w["budget"], group=w.get("group", 1), threads=cores)
         nact = r["lists"]["n_active"]
         n += 1
         if time.perf_counter() - t0 >= seconds:
@@ -236,6 +240,7 @@ def run_ours(args, w, rank, world, local_rank):
     moe.load_library()
     S = ms.SHAPES[w["shape"]]
     B, mode, k0, budget = w["B"], w["mode"], w["k0"], w["budget"]
+    group = w.get("group", 1)
     L = ms.make_weights(S, 0)
     x_np = ms.make_tokens(S, B, 0, kind=w.get("kind", "normal"))
     t = lambda a: torch.from_numpy(a).to(dev)
@@ -252,7 +257,8 @@ def run_ours(args, w, rank, world, local_rank):
 
     def layer(r):
         g, u, dn, wg = copies[r]
-        moe.moe_layer_decode(x, wg, bias, g, u, dn, S.k, mode, k0, budget, ws=ws, y=y, n_active=nact_t)
+        moe.moe_layer_decode(x, wg, bias, g, u, dn, S.k, mode, k0, budget, ws=ws, y=y, n_active=nact_t,
+                             group=group)
 
     with torch.cuda.stream(s):
         for r in range(ROTATE):
@@ -350,7 +356,7 @@ def run_ours(args, w, rank, world, local_rank):
         for i in range(nsteps):
             g, u, dn, wg = copies[i % ROTATE]
             x_dev.copy_(x_host, non_blocking=True)
-            moe.moe_layer_decode(x_dev, wg, bias, g, u, dn, S.k, mode, k0, budget, ws=ws, y=y_dev)
+            moe.moe_layer_decode(x_dev, wg, bias, g, u, dn, S.k, mode, k0, budget, ws=ws, y=y_dev, group=group)
             y_host.copy_(y_dev, non_blocking=True)
 
     with torch.cuda.stream(s):
@@ -381,7 +387,9 @@ def run_ours(args, w, rank, world, local_rank):
         "stream_launch_us_per_call": ms_stream * 1e3,
         "roofline": roofline,
         "e2e": e2e,
-        "gpu_launches": 3 * args.steps,
+        # router, selection and expert kernels; batches above 32 tokens add
+        # the kernel that dispatches each pair's x row
+        "gpu_launches": (3 if B <= 32 else 4) * args.steps,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -393,14 +401,16 @@ def run_ours(args, w, rank, world, local_rank):
 
 
 SWEEP = {
-    # shape: [(B, mode, k0, budget, token kind)], the configurations the
-    # results table reports (one weight set per shape, ROTATE copies)
+    # shape: [(B, mode, k0, budget, token kind[, tokens per request])], the
+    # configurations the results table reports (one weight set per shape,
+    # ROTATE copies); mode 4 (hierarchical XShare) takes the request size
     "tiny": [(4, 1, 2, 0, "normal"), (4, 0, 0, 0, "normal")],
     "e64": [(16, 1, 4, 0, "normal"), (16, 0, 0, 0, "normal")],
     "q30b": [(b, m, k0, 0, "normal") for b in (1, 4, 16, 32, 64) for (m, k0) in ((0, 0), (1, 4))]
             + [(16, 1, k0, 0, "normal") for k0 in (2, 6, 8)]
             + [(32, 0, 0, 0, "spec")] + [(32, 2, 0, m, "spec") for m in (24, 32, 48)]
-            + [(16, 3, 0, 0, "normal"), (64, 3, 0, 0, "normal"), (32, 3, 0, 0, "spec")],
+            + [(16, 3, 0, 0, "normal"), (64, 3, 0, 0, "normal"), (32, 3, 0, 0, "spec")]
+            + [(32, 4, 0, m, "spec", 4) for m in (24, 32, 48)],
     "q235b": [(b, 1, 4, 0, "normal") for b in (1, 8, 16, 64)] + [(16, 0, 0, 0, "normal")],
 }
 
@@ -426,7 +436,9 @@ def run_sweep(args):
         copies = [base] + [tuple(c.clone() for c in base) for _ in range(ROTATE - 1)]
         bias = t(L["bias"])
         s = torch.cuda.Stream(dev)
-        for (B, mode, k0, budget, kind) in SWEEP[shape]:
+        for row in SWEEP[shape]:
+            B, mode, k0, budget, kind = row[:5]
+            group = row[5] if len(row) > 5 else 1
             x_np = ms.make_tokens(S, B, 0, kind=kind)
             x = t(x_np)
             ws = moe.new_workspace(B, S.d, S.E, S.k, S.F, dev)
@@ -435,7 +447,8 @@ def run_sweep(args):
 
             def layer(r):
                 g, u, dn, wg = copies[r]
-                moe.moe_layer_decode(x, wg, bias, g, u, dn, S.k, mode, k0, budget, ws=ws, y=y, n_active=nact_t)
+                moe.moe_layer_decode(x, wg, bias, g, u, dn, S.k, mode, k0, budget, ws=ws, y=y, n_active=nact_t,
+                                     group=group)
 
             with torch.cuda.stream(s):
                 for r in range(ROTATE):
@@ -463,14 +476,15 @@ def run_sweep(args):
             n_active = int(nact_t[0].item())
             total, _ = algorithmic_bytes(S, B, n_active)
             gbs = total / (us * 1e-6) / 1e9
-            line = {"shape": shape, "B": B, "mode": ["NONE", "OEA", "XShare", "Affinity"][mode], "k0": k0, "budget": budget,
-                    "tokens": kind, "n_active": n_active, "us": us, "bytes": total, "GBps": gbs,
-                    "frac_8tbs": gbs / NOMINAL_HBM_GBS, "frac_measured": gbs / hbm_peak}
+            line = {"shape": shape, "B": B, "mode": ["NONE", "OEA", "XShare", "Affinity", "XShareHier"][mode],
+                    "k0": k0, "budget": budget, "group": group, "tokens": kind, "n_active": n_active, "us": us,
+                    "bytes": total, "GBps": gbs, "frac_8tbs": gbs / NOMINAL_HBM_GBS,
+                    "frac_measured": gbs / hbm_peak}
             if not args.no_cpu_baseline:
                 ms_t = []
                 for th in (1, cores):
                     t0 = time.perf_counter()
-                    oracle.layer(x_np, L, S.k, mode, k0, budget, threads=th)
+                    oracle.layer(x_np, L, S.k, mode, k0, budget, threads=th, group=group)
                     ms_t.append((time.perf_counter() - t0) * 1e3)
                 line["oracle_ms_1"] = ms_t[0]
                 line["oracle_ms_n"] = ms_t[1]
@@ -497,7 +511,8 @@ def run_profile_case(args, w):
     g, u, dn = (t(L[n].view(np.int16)) for n in ("Wgate", "Wup", "Wdown"))
     ws = moe.new_workspace(B, S.d, S.E, S.k, S.F)
     for _ in range(args.warmup + args.steps):
-        moe.moe_layer_decode(x, Wg, bias, g, u, dn, S.k, w["mode"], w["k0"], w["budget"], ws=ws)
+        moe.moe_layer_decode(x, Wg, bias, g, u, dn, S.k, w["mode"], w["k0"], w["budget"], ws=ws,
+                             group=w.get("group", 1))
     torch.cuda.synchronize()
     status = moe.moe_check_error(ws)
     print(f"profile case {args.workload}: {args.warmup}+{args.steps} layer calls, status {status}")

@@ -70,7 +70,8 @@ typedef enum {
     MOE_RESELECT_NONE = 0,    /* standard top-k routing */
     MOE_RESELECT_OEA = 1,     /* keep top-k0, fill from the batch union of kept sets */
     MOE_RESELECT_XSHARE = 2,  /* budgeted greedy batch selection, then top-k within it */
-    MOE_RESELECT_AFFINITY = 3 /* Lynx affinity binning: confidence bins, critical set, remap */
+    MOE_RESELECT_AFFINITY = 3, /* Lynx affinity binning: confidence bins, critical set, remap */
+    MOE_RESELECT_XSHARE_HIER = 4 /* XShare per request, then under the batch budget */
 } moe_reselect_mode_t;
 
 /* Layer dimensions: B tokens, hidden size d, E experts, top-k k,
@@ -80,7 +81,8 @@ typedef struct {
 } moe_dims_t;
 
 /* Re-selection rule: mode (moe_reselect_mode_t); k0 (OEA: 1 <= k0 <= k);
- * budget (XShare: k <= budget <= E).  Unused fields are ignored.
+ * budget (both XShare rules: k <= budget <= E); group (hierarchical XShare:
+ * tokens per request, 1 <= group <= 256).  Unused fields are ignored.
  *
  * MOE_RESELECT_AFFINITY ("Lynx: Enabling Efficient MoE Inference through
  * Dynamic Batch-Aware Expert Selection", sections 2.1-2.2; the page gives
@@ -91,9 +93,22 @@ typedef struct {
  * over the tokens whose top-k holds it; the critical set is the shortest
  * prefix of the score order (descending, ties to the lower index), at
  * least k long, that holds every token's top-ranked expert; every token
- * keeps exactly k experts, its first k inside the critical set. */
+ * keeps exactly k experts, its first k inside the critical set.
+ *
+ * MOE_RESELECT_XSHARE_HIER ("XShare: Collaborative in-Batch Expert Sharing
+ * for Faster MoE Inference", abstract: hierarchical, correlation-aware
+ * selection for speculative decoding; the page gives no formulas, this is
+ * the library's reading): a request is a run of `group` consecutive tokens
+ * (a request's token and its drafts; the last run may be shorter).  Each
+ * request picks the k experts with the largest request score (its tokens'
+ * top-k gate probabilities summed, tokens ascending, fp32); an expert's
+ * batch score sums the request scores of the requests that picked it
+ * (requests ascending); the min(budget, |picked|) picked experts with the
+ * largest batch scores (ties to the lower index) form the batch set, and
+ * each token takes its k highest-ranked experts inside it.  group = 1 is
+ * MOE_RESELECT_XSHARE. */
 typedef struct {
-    int32_t mode, k0, budget;
+    int32_t mode, k0, budget, group;
 } moe_reselect_t;
 
 /* Per-expert token lists (all device pointers, int32 / fp32):
@@ -148,6 +163,7 @@ moe_status_t moe_route(const float *x, const float *Wg, const float *bias,
  *            lower index) form the batch set -- the greedy, exact for this
  *            modular objective; each token takes its k highest-ranked
  *            experts inside the set.
+ *   AFFINITY, XSHARE_HIER : as described at moe_reselect_t.
  * Results are bit-exact and deterministic.  Needs no workspace. */
 moe_status_t moe_reselect(const float *logits, const float *probs,
                           moe_dims_t dims, moe_reselect_t rule,

@@ -86,7 +86,11 @@ def test_layer_decode_rejects_bad_arguments(lib):
     assert _layer_call(lib, rule=Rule(1, 9, 0)) == INVALID          # k0 > k
     assert _layer_call(lib, rule=Rule(2, 0, 7)) == INVALID          # budget < k
     assert _layer_call(lib, rule=Rule(2, 0, 129)) == INVALID        # budget > E
-    assert _layer_call(lib, rule=Rule(4, 0, 0)) == INVALID          # unknown rule
+    assert _layer_call(lib, rule=Rule(5, 0, 0)) == INVALID          # unknown rule
+    assert _layer_call(lib, rule=Rule(4, 0, 16, 0)) == INVALID      # hierarchical: group < 1
+    assert _layer_call(lib, rule=Rule(4, 0, 16, 257)) == INVALID    # group > 256
+    assert _layer_call(lib, rule=Rule(4, 0, 7, 4)) == INVALID       # budget < k
+    assert _layer_call(lib, rule=Rule(4, 0, 129, 4)) == INVALID     # budget > E
     assert _layer_call(lib, x=None) == INVALID
     assert _layer_call(lib, Wdown=None) == INVALID
     assert _layer_call(lib, y=None) == INVALID
@@ -131,6 +135,8 @@ def test_valid_call_without_a_device_reports_cuda_error(lib):
     # all arguments valid: validation passes, the device query fails cleanly
     assert _layer_call(lib) == CUDA
     assert _layer_call(lib, rule=Rule(3, 0, 0)) == CUDA            # affinity binning: no parameters
+    assert _layer_call(lib, rule=Rule(4, 0, 16, 4)) == CUDA        # hierarchical XShare
+    assert _layer_call(lib, rule=Rule(4, 0, 128, 256)) == CUDA
     assert lib.moe_route(A, A, None, Dims(16, 2048, 128, 8, 0), A, A, A, A, None) == CUDA
 
 

@@ -19,7 +19,7 @@ from gpu_cases import assert_close_y, bits, device_layer, host_layer, shape
 
 pytestmark = pytest.mark.gpu
 
-NONE, OEA, XSHARE, AFFINITY = 0, 1, 2, 3
+NONE, OEA, XSHARE, AFFINITY, XSHARE_HIER = 0, 1, 2, 3, 4
 THREADS = max(1, len(os.sched_getaffinity(0)))
 
 
@@ -69,11 +69,11 @@ def test_route_without_bias_and_repeatable():
 
 
 # -------------------------------------------------------------- reselect --
-def _check_reselect(logits, probs, k, mode, k0=0, budget=0):
-    sel_ref, w_ref = oracle.reselect(logits, probs, k, mode, k0, budget)
+def _check_reselect(logits, probs, k, mode, k0=0, budget=0, group=1):
+    sel_ref, w_ref = oracle.reselect(logits, probs, k, mode, k0, budget, group)
     li_ref = oracle.lists(sel_ref, w_ref, logits.shape[1])
     sel, w, li = moe.moe_reselect(torch.from_numpy(logits).cuda(), torch.from_numpy(probs).cuda(), k, mode,
-                                  k0=k0, budget=budget)
+                                  k0=k0, budget=budget, group=group)
     torch.cuda.synchronize()
     assert np.array_equal(sel.cpu().numpy(), sel_ref)
     assert np.array_equal(bits(w), bits(w_ref))
@@ -100,6 +100,17 @@ def test_reselect_bit_exact_q30b(B, mode, k0, budget):
     _check_reselect(logits, probs, S.k, mode, k0, budget)
 
 
+@pytest.mark.parametrize("B", [1, 4, 16, 32, 64, 256])
+@pytest.mark.parametrize("group", [1, 3, 4, 256])
+@pytest.mark.parametrize("budget", [8, 24, 48])
+def test_reselect_xshare_hier_bit_exact_q30b(B, group, budget):
+    S = shape("q30b")
+    L = ms.make_weights(S, 0, experts=False)
+    x = _tokens("q30b", B, 0, kind="spec" if B % 8 == 0 else "normal")
+    logits, probs, _, _ = oracle.route(x, L["Wg"], L["bias"], S.k)
+    _check_reselect(logits, probs, S.k, XSHARE_HIER, budget=budget, group=group)
+
+
 @pytest.mark.parametrize("budget", [24, 32, 48])
 def test_reselect_speculative_batch(budget):
     S = shape("q30b")
@@ -108,6 +119,7 @@ def test_reselect_speculative_batch(budget):
     logits, probs, _, _ = oracle.route(x, L["Wg"], L["bias"], S.k)
     _check_reselect(logits, probs, S.k, XSHARE, budget=budget)
     _check_reselect(logits, probs, S.k, AFFINITY)
+    _check_reselect(logits, probs, S.k, XSHARE_HIER, budget=budget, group=4)
 
 
 @pytest.mark.parametrize("seed", range(6))
@@ -122,10 +134,12 @@ def test_reselect_random_edges(seed):
         for mode, k0, budget in [(NONE, 0, 0), (OEA, 1, 0), (OEA, max(1, k // 2), 0), (OEA, k, 0),
                                  (XSHARE, 0, k), (XSHARE, 0, min(E, 2 * k)), (XSHARE, 0, E), (AFFINITY, 0, 0)]:
             _check_reselect(logits, probs, k, mode, k0, budget)
+        for budget, group in [(k, 1), (min(E, 2 * k), 3), (E, 2), (min(E, 3 * k), B)]:
+            _check_reselect(logits, probs, k, XSHARE_HIER, budget=budget, group=group)
 
 
 # ------------------------------------------------------------------- FFN --
-def _run_layer(name, B, seed, mode, k0=0, budget=0, kind="normal"):
+def _run_layer(name, B, seed, mode, k0=0, budget=0, kind="normal", group=1):
     S = shape(name)
     L = host_layer(name, seed)
     D = device_layer(name, seed)
@@ -136,14 +150,14 @@ def _run_layer(name, B, seed, mode, k0=0, budget=0, kind="normal"):
     selw = torch.empty(B, S.k, dtype=torch.float32, device="cuda")
     nact = torch.empty(4, dtype=torch.int32, device="cuda")
     y = moe.moe_layer_decode(xd, D["Wg"], D["bias"], D["Wgate"], D["Wup"], D["Wdown"], S.k, mode, k0, budget,
-                             ws=ws, sel_idx=sel, sel_w=selw, n_active=nact)
+                             ws=ws, sel_idx=sel, sel_w=selw, n_active=nact, group=group)
     assert moe.moe_check_error(ws) == 0
     return S, L, x, y.cpu().numpy(), sel.cpu().numpy(), selw.cpu().numpy(), int(nact[0].item())
 
 
-def _oracle_layer(S, L, x, mode, k0, budget, rows):
+def _oracle_layer(S, L, x, mode, k0, budget, rows, group=1):
     logits, probs, _, _ = oracle.route(x, L["Wg"], L["bias"], S.k)
-    sel, w = oracle.reselect(logits, probs, S.k, mode, k0, budget)
+    sel, w = oracle.reselect(logits, probs, S.k, mode, k0, budget, group)
     li = oracle.lists(sel, w, S.E)
     y = oracle.ffn(x, L["Wgate"], L["Wup"], L["Wdown"], sel, w, rows=rows, threads=THREADS)
     return sel, w, li["n_active"], y
@@ -195,6 +209,25 @@ def test_layer_decode_parity_speculative(budget):
     sel_r, w_r, n_r, y_r = _oracle_layer(S, L, x, XSHARE, 0, budget, rows)
     assert np.array_equal(sel, sel_r) and n_act == n_r <= budget
     assert_close_y(y[rows], y_r, f"spec budget={budget}")
+
+
+HIER_LAYER_CASES = [("q30b", 16, 4, 16), ("q30b", 16, 3, 24), ("q30b", 32, 4, 24), ("q30b", 32, 4, 32),
+                    ("q30b", 32, 4, 48), ("q30b", 64, 4, 48), ("q30b", 1, 1, 8), ("tiny", 4, 2, 6),
+                    ("ragged", 37, 5, 10), ("maxek", 100, 8, 40), ("e64", 16, 4, 16)]
+
+
+@pytest.mark.parametrize("name,B,group,budget", HIER_LAYER_CASES)
+def test_layer_decode_parity_xshare_hier(name, B, group, budget):
+    # B <= 32: the router publishes the batch set and the expert kernel
+    # starts early; larger batches take the dispatch path
+    kind = "spec" if name == "q30b" and B % 8 == 0 else "normal"
+    S, L, x, y, sel, selw, n_act = _run_layer(name, B, 0, XSHARE_HIER, 0, budget, kind=kind, group=group)
+    rows = np.unique(np.linspace(0, B - 1, min(B, 6)).astype(np.int32))
+    sel_r, w_r, n_r, y_r = _oracle_layer(S, L, x, XSHARE_HIER, 0, budget, rows, group=group)
+    assert np.array_equal(sel, sel_r)
+    assert np.array_equal(bits(selw), bits(w_r))
+    assert n_act == n_r <= budget
+    assert_close_y(y[rows], y_r, f"{name} B={B} hierarchical group={group} budget={budget}")
 
 
 @pytest.mark.parametrize("B,mode,k0", [(1, OEA, 4), (16, NONE, 0), (16, OEA, 4), (64, OEA, 4)])
