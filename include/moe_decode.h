@@ -10,9 +10,11 @@
  *   2. batch-aware re-selection, which shrinks the set of experts the batch
  *      activates: OEA piggybacking ("Opportunistic Expert Activation:
  *      Batch-Aware Expert Routing for Faster Decode Without Retraining",
- *      abstract) or XShare greedy selection under an expert budget ("XShare:
- *      Collaborative in-Batch Expert Sharing for Faster MoE Inference",
- *      abstract);
+ *      abstract), XShare greedy selection under an expert budget, flat or
+ *      per request first ("XShare: Collaborative in-Batch Expert Sharing for
+ *      Faster MoE Inference", abstract), or Lynx affinity binning ("Lynx:
+ *      Enabling Efficient MoE Inference through Dynamic Batch-Aware Expert
+ *      Selection", section 2.2);
  *   3. the SwiGLU FFN of every activated expert over its tokens, combined
  *      with the renormalised gate weights; each activated expert's weights
  *      are read from HBM once per call ("Lynx: Enabling Efficient MoE
