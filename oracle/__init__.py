@@ -60,6 +60,10 @@ def _load():
         lib.oracle_lists.argtypes = [P, P, I, I, I, P, P, P, P]
         lib.oracle_ffn.restype = None
         lib.oracle_ffn.argtypes = [P, P, P, P, I, I, I, I, I, P, P, P, I, I, P]
+        lib.oracle_ffn_channels.restype = None
+        lib.oracle_ffn_channels.argtypes = [P, P, P, P, I, I, I, I, I, P, P, P, I, P, I, I, P, P]
+        lib.oracle_channel_sector_bytes.restype = ctypes.c_longlong
+        lib.oracle_channel_sector_bytes.argtypes = [P, P, I, I, I, I, I, I]
         _lib = lib
     return _lib
 
@@ -166,6 +170,44 @@ def ffn(x, Wgate, Wup, Wdown, sel_idx, sel_w, rows=None, threads: int = 1) -> np
     lib.oracle_ffn(_p(x), _p(Wgate), _p(Wup), _p(Wdown), B, d, E, k, F,
                    _p(sel_idx), _p(sel_w), rp, nr, int(threads), _p(y))
     return y
+
+
+def ffn_channels(x, Wgate, Wup, Wdown, sel_idx, sel_w, score, c: int, rows=None, threads: int = 1):
+    """Expert FFN with per-(token, slot) channel top-k: each pair keeps the
+    c channels with the largest ``score[b][s][f]`` (ties to the lower
+    index).  -> (y[len(rows) or B][d] fp64, keep[B][k][F] uint8)."""
+    lib = _load()
+    x = _c(x, np.float32)
+    Wgate = _c(Wgate, np.uint16)
+    Wup = _c(Wup, np.uint16)
+    Wdown = _c(Wdown, np.uint16)
+    sel_idx = _c(sel_idx, np.int32)
+    sel_w = _c(sel_w, np.float32)
+    score = _c(score, np.float32)
+    B, d = x.shape
+    E, F, _ = Wgate.shape
+    k = sel_idx.shape[1]
+    assert score.shape == (B, k, F) and 1 <= c <= F
+    if rows is None:
+        rp, nr = None, B
+    else:
+        rows = _c(rows, np.int32)
+        rp, nr = _p(rows), rows.size
+    y = np.empty((nr, d), np.float64)
+    keep = np.empty((B, k, F), np.uint8)
+    lib.oracle_ffn_channels(_p(x), _p(Wgate), _p(Wup), _p(Wdown), B, d, E, k, F, _p(sel_idx), _p(sel_w),
+                            _p(score), int(c), rp, nr, int(threads), _p(y), _p(keep))
+    return y, keep
+
+
+def channel_sector_bytes(keep, sel_idx, E: int, d: int, down_channel_major: bool = False) -> int:
+    """Expert-weight bytes one call reads under channel top-k, counted in
+    whole 32-byte sectors (see moe_oracle.c)."""
+    lib = _load()
+    keep = _c(keep, np.uint8)
+    sel_idx = _c(sel_idx, np.int32)
+    B, k, F = keep.shape
+    return int(lib.oracle_channel_sector_bytes(_p(keep), _p(sel_idx), B, E, k, d, F, int(down_channel_major)))
 
 
 def layer(x, L: dict, k: int, mode: int, k0: int = 0, budget: int = 0,

@@ -28,6 +28,10 @@
  *        Expert Selection", section 1 (latency follows the number of distinct
  *        experts the batch activates) and section 2.2 (every token keeps
  *        k expert slots).
+ *  [CS]  "Channel Selection for Mixture-of-Experts Decoding Needs No
+ *        Calibration Data", methodology: a channel selector is a score plus
+ *        a keep rule; top-k keeps each token's highest-scoring channels;
+ *        reads are counted in 32-byte sectors.
  *
  * Readings where the pages are silent (each one is also listed in the
  * design notes):
@@ -62,7 +66,9 @@
  * two closed forms (one token per request, one request per batch) and brute
  * force over the subsets of both levels, affinity binning against its
  * invariants, closed forms and hand-worked cases, the FFN against a dense
- * fp64 torch restatement.
+ * fp64 torch restatement, the channel top-k FFN against a torch restatement
+ * over the gathered channels, the dense FFN and complementarity, and its
+ * sector byte count against closed forms and brute force over addresses.
  */
 #include <math.h>
 #include <stdint.h>
@@ -507,4 +513,129 @@ void oracle_ffn(const float *x, const uint16_t *Wgate, const uint16_t *Wup,
         }
         free(h);
     }
+}
+
+/* ------------------------------------------------- channel top-k FFN ---
+ * [CS] "Channel Selection for Mixture-of-Experts Decoding Needs No
+ * Calibration Data", methodology: a channel selector is a score plus a
+ * keep rule, and the top-k keep rule takes each token's c highest-scoring
+ * channels.  Channel f of expert e is gate row f, up row f and down column
+ * f.  Only the keep rule and the sparse FFN are restated here: the scores
+ * come from the caller (any selector; the page's weight-derived reader is
+ * not part of this oracle).
+ * For each token r listed in rows[0..n_rows) (all tokens when rows ==
+ * NULL) and each slot s with e = sel_idx[b][s] >= 0:
+ *   K = the c channels with the largest score[b][s][f], equal scores to
+ *       the lower channel index (channel f is kept iff fewer than c
+ *       channels rank before it);
+ *   h_f = silu(g_f) u_f for f in K and 0 otherwise (g, u as in oracle_ffn);
+ *   o_i = sum over f ascending of Wdown[e][i][f] h_f;
+ *   y[r] = sum over the slots (slot order) of w o   (fp64).
+ * keep[b][s][f] (B x k x F bytes, may be NULL) receives 1 for the kept
+ * channels of every slot of every token (not only the listed rows), 0
+ * elsewhere and for empty slots. */
+void oracle_ffn_channels(const float *x, const uint16_t *Wgate, const uint16_t *Wup,
+                         const uint16_t *Wdown, int B, int d, int E, int k, int F,
+                         const int *sel_idx, const float *sel_w, const float *score, int c,
+                         const int *rows, int n_rows, int threads, double *y,
+                         unsigned char *keep)
+{
+    (void)E;
+    unsigned char *kp = (unsigned char *)calloc((size_t)B * k * F, 1);
+    for (int b = 0; b < B; ++b)
+        for (int s = 0; s < k; ++s) {
+            if (sel_idx[(size_t)b * k + s] < 0) continue;
+            const float *sc = score + ((size_t)b * k + s) * F;
+            unsigned char *m = kp + ((size_t)b * k + s) * F;
+            for (int f = 0; f < F; ++f) {
+                int before = 0;
+                for (int f2 = 0; f2 < F; ++f2)
+                    if (sc[f2] > sc[f] || (sc[f2] == sc[f] && f2 < f)) ++before;
+                m[f] = before < c;
+            }
+        }
+    if (keep) memcpy(keep, kp, (size_t)B * k * F);
+    int nr = rows ? n_rows : B;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(threads > 0 ? threads : 1)
+    for (int ri = 0; ri < nr; ++ri) {
+        int b = rows ? rows[ri] : ri;
+        double *yo = y + (size_t)ri * d;
+        double *h = (double *)malloc(sizeof(double) * (size_t)F);
+        for (int i = 0; i < d; ++i) yo[i] = 0.0;
+        for (int s = 0; s < k; ++s) {
+            int e = sel_idx[(size_t)b * k + s];
+            if (e < 0) continue;
+            double wt = (double)sel_w[(size_t)b * k + s];
+            const float *xb = x + (size_t)b * d;
+            const unsigned char *m = kp + ((size_t)b * k + s) * F;
+            for (int f = 0; f < F; ++f) {
+                h[f] = 0.0;
+                if (!m[f]) continue;
+                const uint16_t *gr = Wgate + ((size_t)e * F + f) * d;
+                const uint16_t *ur = Wup + ((size_t)e * F + f) * d;
+                double g = 0.0, u = 0.0;
+                for (int i = 0; i < d; ++i) {
+                    g += (double)xb[i] * bf16_to_double(gr[i]);
+                    u += (double)xb[i] * bf16_to_double(ur[i]);
+                }
+                h[f] = g / (1.0 + exp(-g)) * u;
+            }
+            for (int i = 0; i < d; ++i) {
+                const uint16_t *dr = Wdown + ((size_t)e * d + i) * F;
+                double o = 0.0;
+                for (int f = 0; f < F; ++f) o += bf16_to_double(dr[f]) * h[f];
+                yo[i] += wt * o;
+            }
+        }
+        free(h);
+    }
+    free(kp);
+}
+
+/* Bytes of expert weights one call reads when every activated expert reads
+ * only the union of its (token, slot) pairs' kept channels, every touched
+ * 32-byte sector charged in full ([CS], methodology: reads are counted in
+ * 32-byte sectors).  Addresses are byte offsets from each weight array's
+ * start, which is assumed 32-byte aligned.  Wgate and Wup are [E][F][d]
+ * (channel f's row: 2d contiguous bytes).  Wdown is [E][d][F] (channel f's
+ * column: one bf16 in each of d rows) unless down_channel_major, which
+ * charges it as [E][F][d] (the column contiguous).  Returns the bytes. */
+long long oracle_channel_sector_bytes(const unsigned char *keep, const int *sel_idx,
+                                      int B, int E, int k, int d, int F,
+                                      int down_channel_major)
+{
+    unsigned char *u = (unsigned char *)malloc((size_t)F);
+    long long sectors = 0;
+    for (int e = 0; e < E; ++e) {
+        memset(u, 0, (size_t)F);
+        int any = 0;
+        for (int b = 0; b < B; ++b)
+            for (int s = 0; s < k; ++s)
+                if (sel_idx[(size_t)b * k + s] == e) {
+                    const unsigned char *m = keep + ((size_t)b * k + s) * F;
+                    for (int f = 0; f < F; ++f) u[f] |= m[f];
+                    any = 1;
+                }
+        if (!any) continue;
+        for (int f = 0; f < F; ++f) {
+            if (!u[f]) continue;
+            /* gate and up rows (and the down column when channel-major) */
+            long long first = (((long long)e * F + f) * d * 2) / 32;
+            long long last = ((((long long)e * F + f) * d + d) * 2 - 1) / 32;
+            sectors += (down_channel_major ? 3 : 2) * (last - first + 1);
+        }
+        if (!down_channel_major) {
+            for (int i = 0; i < d; ++i) {
+                long long prev = -1;
+                for (int f = 0; f < F; ++f) {
+                    if (!u[f]) continue;
+                    long long sec = ((((long long)e * d + i) * F + f) * 2) / 32;
+                    if (sec != prev) ++sectors;   /* f ascending: sectors ascend */
+                    prev = sec;
+                }
+            }
+        }
+    }
+    free(u);
+    return sectors * 32;
 }
