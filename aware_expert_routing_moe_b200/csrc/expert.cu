@@ -996,8 +996,8 @@ int split_for_tiles(long long tiles, int gu_per_tile, int d_per_tile, int ns_gu,
     return max_stages_host(cut, 3, P) + 2 <= max_stages_host(whole, 2, P) ? static_cast<int>(r) : 0;
 }
 
-int g_num_sms[64] = {0};
-bool g_attr_small[64] = {false}, g_attr_large[64] = {false};
+int g_num_sms[MAX_DEVICES] = {0};
+bool g_attr_small[MAX_DEVICES] = {false}, g_attr_large[MAX_DEVICES] = {false};
 
 }  // namespace
 
@@ -1047,7 +1047,7 @@ cudaError_t launch_expert_ffn(const ExpertMaps &maps, const uint16_t *xb, const 
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
-    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (dev < 0 || dev >= MAX_DEVICES) return cudaErrorInvalidDevice;
     if (g_num_sms[dev] == 0) {
         int n = 0;
         err = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);

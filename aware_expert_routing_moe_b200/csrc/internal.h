@@ -29,6 +29,7 @@ struct PubLine {
     int32_t pad1[20];
 };
 static_assert(sizeof(PubLine) == 128, "PubLine must fill one 128-byte line");
+constexpr int MAX_DEVICES = 64;  // per-device host caches (attributes, SM counts)
 constexpr int PUB_COPIES = 8;  // expert-kernel CTA c polls copy c % PUB_COPIES
 
 struct Counters {

@@ -19,7 +19,6 @@ namespace {
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[MOE_NOALLOC_SCRATCH_BYTES];
 
-constexpr int MAX_DEVICES = 64;
 std::mutex g_scratch_mu;
 unsigned char *g_scratch_addr[MAX_DEVICES] = {};
 

@@ -1239,8 +1239,13 @@ ReselectArgs make_reselect_args(const float *logits, float *probs, bool fuse_sof
 
 template <int NI>
 cudaError_t launch_gemv_ni(const RouterMaps &maps, const GemvArgs &g, const GemvShape &sh, cudaStream_t s) {
-    static bool configured = false;  // the attribute is per function; set it once
-    if (!configured) {
+    // the attributes belong to the function on each device: set them once per device
+    static bool configured[MAX_DEVICES] = {};
+    int dev = 0;
+    cudaError_t derr = cudaGetDevice(&dev);
+    if (derr != cudaSuccess) return derr;
+    if (dev < 0 || dev >= MAX_DEVICES) return cudaErrorInvalidDevice;
+    if (!configured[dev]) {
         cudaError_t err = cudaFuncSetAttribute(route_gemv_kernel<NI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                static_cast<int>(GEMV_SMEM_MAX + 1024));
         if (err != cudaSuccess) return err;
@@ -1248,7 +1253,7 @@ cudaError_t launch_gemv_ni(const RouterMaps &maps, const GemvArgs &g, const Gemv
         // between the two needs no reconfiguration
         err = cudaFuncSetAttribute(route_gemv_kernel<NI>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
         if (err != cudaSuccess) return err;
-        configured = true;
+        configured[dev] = true;
     }
     const dim3 grid((g.E + sh.epb - 1) / sh.epb, (g.B + sh.tpb - 1) / sh.tpb);
     route_gemv_kernel<NI><<<grid, 32 * sh.epb, sh.smem, s>>>(maps, g);
@@ -1313,14 +1318,19 @@ cudaError_t launch_route_topk(const float *logits, const moe_dims_t &d, float *p
 
 template <int NI>
 static cudaError_t launch_reselect_ni(const ReselectArgs &a, size_t smem, bool chained, cudaStream_t s) {
-    static bool configured = false;  // the attribute is per function; set it once
-    if (!configured) {
+    // the attributes belong to the function on each device: set them once per device
+    static bool configured[MAX_DEVICES] = {};
+    int dev = 0;
+    cudaError_t derr = cudaGetDevice(&dev);
+    if (derr != cudaSuccess) return derr;
+    if (dev < 0 || dev >= MAX_DEVICES) return cudaErrorInvalidDevice;
+    if (!configured[dev]) {
         cudaError_t err =
             cudaFuncSetAttribute(reselect_kernel<NI>, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
         if (err != cudaSuccess) return err;
         err = cudaFuncSetAttribute(reselect_kernel<NI>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
         if (err != cudaSuccess) return err;
-        configured = true;
+        configured[dev] = true;
     }
     if (!chained) {
         reselect_kernel<NI><<<1, 1024, smem, s>>>(a);
