@@ -62,13 +62,13 @@ moe_status_t check_ws(const moe_dims_t &d, void *ws, size_t ws_bytes) {
 
 // The current device must be an sm_100 part (B200).  Cached per device.
 moe_status_t check_device() {
-    static int cached[64] = {0};  // 0 unknown, 1 ok, 2 unsupported
+    static int cached[MAX_DEVICES] = {0};  // 0 unknown, 1 ok, 2 unsupported
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) {
         cudaGetLastError();
         return MOE_ERR_CUDA;
     }
-    if (dev < 0 || dev >= 64) return MOE_ERR_UNSUPPORTED;
+    if (dev < 0 || dev >= MAX_DEVICES) return MOE_ERR_UNSUPPORTED;
     if (cached[dev] == 0) {
         int major = 0, minor = 0;
         if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
