@@ -21,8 +21,9 @@
 // (active slot, token), and the down epilogue weighs each token by a dense
 // [slot][B] weight matrix (0 for tokens that did not choose the expert).
 // Gate/up work then needs only the activated set, which the layer path
-// publishes before the token lists exist (the router kernel for OEA and
-// plain top-k, the selection for XShare): the kernel is launched early,
+// publishes before the token lists exist (the router kernel: per token
+// group for OEA and plain top-k, once every group is in for the batch-wide
+// rules): the kernel is launched early,
 // reads the set from a published bit mask and starts streaming at once.
 // Larger batches use tiles of up to 32 (token, expert) pairs: the input
 // preparation copies each pair's x row (bf16) into a pair-indexed buffer in

@@ -19,11 +19,13 @@ constexpr int F_MIN = 64, F_MAX = 8192;
 
 // Counters the kernels share inside one workspace.  They are zero between
 // calls: each user puts back what it changed (the router's last block of a
-// token group its count; the expert kernel's last CTA everything else).
+// token group its count, the router's last group the batch-wide rules'
+// contributions; the expert kernel's last CTA everything else).
 // One published copy of the activated set, alone in a 128-byte line.
 struct PubLine {
     int32_t pub;                // token groups whose first ranks are in `mask`
-                                // (+1 once the selection published it, XShare)
+                                // (+1 once the router's last group has added
+                                // a batch-wide rule's set)
     int32_t pad0[3];
     uint32_t mask[E_MAX / 32];  // the activated set, one bit per expert
     int32_t pad1[20];
@@ -39,13 +41,14 @@ struct Counters {
     PubLine pubs[PUB_COPIES];   // layer path: the activated set, in copies
     int32_t grp_done[B_MAX];    // router blocks finished, per token group
     int32_t gu_done[E_MAX];     // finished gate/up units per active-expert slot
-    // Batch-wide rules published by the router (XShare, affinity binning;
-    // B <= 32): each token group's contributions, cleared by the last group
+    // Batch-wide rules published by the router (XShare, hierarchical XShare,
+    // affinity binning; B <= 32): each token group's contributions, cleared
+    // by the last group
     int32_t grp_final;                 // token groups whose contributions are in
     uint32_t ubase_bits[E_MAX / 32];   // union of the top-k sets
     uint32_t r0_bits[E_MAX / 32];      // every token's rank-0 expert
     int32_t pad2[15];
-    uint32_t memb[E_MAX];              // XShare: tokens (bit b) whose top-k holds the expert
+    uint32_t memb[E_MAX];              // XShare rules: tokens (bit b) whose top-k holds the expert
     unsigned long long aff_score[E_MAX];  // affinity binning: sum of 2^bin
 };
 static_assert(sizeof(Counters) % 16 == 0, "Counters must keep 16-byte alignment");
@@ -108,7 +111,7 @@ cudaError_t launch_reselect(const float *logits, const float *probs, const moe_d
 // Layer path, first kernel: router GEMV; also writes x in bf16, zeroes y
 // and, with `early` (B <= 32), publishes the activated set in ctr->pubs for
 // the expert kernel started early (every rule: OEA and no re-selection per
-// token group, XShare and affinity binning once all groups are in).
+// token group, the batch-wide rules once all groups are in).
 cudaError_t launch_layer_route(const RouterMaps &maps, const float *x, const float *bias, const moe_dims_t &d,
                                const moe_reselect_t &rule, float *logits, float *probs, uint16_t *xb, float *y,
                                Counters *ctr, bool early, cudaStream_t s);

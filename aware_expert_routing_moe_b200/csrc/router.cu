@@ -8,10 +8,10 @@
 //  route_topk_kernel    : warp per token: softmax (step 2) + top-k (step 3)
 //      with a warp-shuffle reduction and register-resident keys.
 //  reselect_kernel      : one CTA for the whole batch: (softmax +) top-k,
-//      OEA / XShare / affinity-binning re-selection ("Lynx: Enabling
-//      Efficient MoE Inference through Dynamic Batch-Aware Expert
-//      Selection", section 2.2), renormalised weights, per-expert token
-//      lists and, for small batches, the dense weight matrix.
+//      OEA / XShare / hierarchical XShare / affinity-binning re-selection
+//      ("Lynx: Enabling Efficient MoE Inference through Dynamic Batch-Aware
+//      Expert Selection", section 2.2), renormalised weights, per-expert
+//      token lists and, for small batches, the dense weight matrix.
 //
 // Every floating-point step that decides an index is written with explicit
 // round-to-nearest intrinsics (__fmaf_rn, __fadd_rn, __fsub_rn, __fdiv_rn)
@@ -376,8 +376,9 @@ __device__ void write_dense_weights(float *wd, int B, int b, int n_active, const
 
 // The batch-level selection, run by one block (any multiple of 32 threads,
 // at least 256): phase 1 per token (softmax in the layer path, first ranks),
-// XShare's batch set, phase 2 per token (OEA fills / XShare top-k, weights),
-// then the per-expert lists.  Every thread of the block must call it.
+// the batch set of a batch-wide rule, phase 2 per token (OEA fills / top-k
+// within the batch set, weights), then the per-expert lists.  Every thread
+// of the block must call it.
 template <int NI>
 __device__ void reselect_body(const ReselectArgs &a, unsigned char *smem_raw) {
     const int B = a.B, E = a.E, k = a.k;
@@ -594,9 +595,10 @@ __device__ void reselect_body(const ReselectArgs &a, unsigned char *smem_raw) {
         __syncthreads();
     }
 
-    // ---- the activated set is now fixed: OEA = union of kept sets, XShare =
-    // the batch set, affinity binning = the critical set, NONE = union of
-    // top-k sets.  Map experts to active slots for the dense weights.
+    // ---- the activated set is now fixed: OEA = union of kept sets, XShare
+    // and hierarchical XShare = the batch set, affinity binning = the
+    // critical set, NONE = union of top-k sets.  Map experts to active slots
+    // for the dense weights.
     if (dense_w) {
         const unsigned *abits = (mode == MOE_RESELECT_OEA) ? ukept : (mode == MOE_RESELECT_NONE ? ubase : sbits);
         if (warp == 0) {
