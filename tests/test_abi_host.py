@@ -36,6 +36,41 @@ def test_header_declares_the_binding_symbols():
     assert _declared_functions() == sorted(moe.ABI_SYMBOLS)
 
 
+def _header_text():
+    with open(os.path.join(ROOT, "include", "moe_decode.h")) as f:
+        return re.sub(r"/\*.*?\*/", "", f.read(), flags=re.S)
+
+
+def test_binding_structs_and_constants_match_the_header():
+    text = _header_text()
+    # enum constants: status codes and re-selection modes
+    consts = {m.group(1): int(m.group(2)) for m in re.finditer(r"\b(MOE_[A-Z_]+)\s*=\s*(\d+)", text)}
+    status = {k: v for k, v in consts.items() if k.startswith("MOE_ERR") or k == "MOE_OK"}
+    assert {v: k for k, v in moe.STATUS.items()} == status
+    for name in ("MOE_RESELECT_NONE", "MOE_RESELECT_OEA", "MOE_RESELECT_XSHARE", "MOE_RESELECT_AFFINITY",
+                 "MOE_RESELECT_XSHARE_HIER"):
+        assert getattr(moe, name) == consts[name], name
+    assert sorted(k for k in consts if k.startswith("MOE_RESELECT_")) == sorted(
+        k for k in dir(moe) if k.startswith("MOE_RESELECT_"))
+    # struct fields, in order, all 32-bit integers (pointers for the lists)
+    def fields(tag):
+        body = re.search(r"typedef struct \{([^{}]*)\}\s*" + tag + r"\s*;", text).group(1)
+        names = []
+        for decl in body.split(";"):
+            decl = decl.strip()
+            if decl:
+                names += [n.strip().lstrip("*") for n in decl.split(None, 1)[1].split(",")]
+        return names
+    assert fields("moe_dims_t") == [f[0] for f in Dims._fields_]
+    assert fields("moe_reselect_t") == [f[0] for f in Rule._fields_]
+    assert fields("moe_lists_t") == [f[0] for f in Lists._fields_]
+    assert ctypes.sizeof(Rule) == 4 * len(Rule._fields_) and ctypes.sizeof(Dims) == 4 * len(Dims._fields_)
+    m = re.search(r"#define MOE_NOALLOC_SCRATCH_BYTES \((\d+)u? \* (\d+)u? \* (\d+)u?\)",
+                  open(os.path.join(ROOT, "include", "moe_decode.h")).read())
+    if m:
+        assert moe.NOALLOC_SCRATCH_BYTES == int(m.group(1)) * int(m.group(2)) * int(m.group(3))
+
+
 def test_library_exports_every_declared_function(lib):
     for name in _declared_functions():
         assert hasattr(lib, name), name
