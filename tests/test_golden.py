@@ -21,7 +21,7 @@ def test_oracle_matches_recorded_tiny_cases(oracle_lib):
         if seed not in layers:
             layers[seed] = (ms.make_weights(S, seed), ms.make_tokens(S, g["B"], seed))
         L, x = layers[seed]
-        r = oracle_lib.layer(x, L, S.k, c["mode"], k0=c["k0"], budget=c["budget"])
+        r = oracle_lib.layer(x, L, S.k, c["mode"], k0=c["k0"], budget=c["budget"], group=c.get("group", 1))
         assert r["logits"].view(np.uint32).ravel().tolist() == c["logits_bits"]
         assert r["probs"].view(np.uint32).ravel().tolist() == c["probs_bits"]
         assert r["sel_idx"].ravel().tolist() == c["sel_idx"]
