@@ -65,3 +65,26 @@ def test_reference_arm_other_ranks_do_nothing(capsys):
         steps, warmup, gpus = 3, 3, 2
     bench.run_reference(A, bench.WORKLOADS["q30b_b16_oea4"], rank=1)
     assert capsys.readouterr().out == ""
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="checks the no-device path")
+def test_every_timed_configuration_passes_host_validation():
+    # each bench workload and sweep row is a valid call: the library's host
+    # validation accepts it and only the (absent) device stops it
+    import aware_expert_routing_moe_b200 as moe
+    from aware_expert_routing_moe_b200 import Dims, Rule
+    from aware_expert_routing_moe_b200 import build
+    build.build()
+    lib = moe.load_library()
+    A = 0x10000
+    rows = [(w["shape"], w["B"], w["mode"], w["k0"], w["budget"], w.get("group", 1)) for w in bench.WORKLOADS.values()]
+    for shape, cfgs in bench.SWEEP.items():
+        rows += [(shape, r[0], r[1], r[2], r[3], r[5] if len(r) > 5 else 1) for r in cfgs]
+    for shape, B, mode, k0, budget, group in rows:
+        S = ms.SHAPES[shape]
+        dims = Dims(B, S.d, S.E, S.k, S.F)
+        nbytes = lib.moe_workspace_bytes(dims)
+        assert nbytes > 0, (shape, B)
+        st = lib.moe_layer_decode(A, A, A, A, A, A, dims, Rule(mode, k0, budget, group), A, None, None, None, A,
+                                  nbytes, None)
+        assert st == 5, (shape, B, mode, k0, budget, group, st)    # MOE_ERR_CUDA: validation passed
