@@ -621,8 +621,11 @@ __device__ void consumer(const ExpertArgs &a, SharedCtl *ctl, unsigned char *slo
 #pragma unroll
                     for (int c = 0; c < 2; ++c) {
                         const int n = j * 8 + col + c;
-                        const bool v = n < h.n;
-                        tk[j][c] = v ? __ldg(a.tok + h.p0 + n) : 0;
+                        const int t = n < h.n ? __ldg(a.tok + h.p0 + n) : 0;
+                        // a token outside the batch is skipped (and reported)
+                        const bool v = n < h.n && t >= 0 && t < a.B;
+                        if (n < h.n && !v) atomicCAS(&a.ctr->error, 0, DEV_BAD_LISTS);
+                        tk[j][c] = v ? t : 0;
                         wk[j][c] = v ? __ldg(a.w + h.p0 + n) : 0.0f;
                     }
             }
@@ -729,6 +732,29 @@ __device__ void signaller(const ExpertArgs &a, SharedCtl *ctl) {
     }
 }
 
+// n_active of caller-supplied lists, checked by the producer warp before
+// any list value is used as an index: 0 <= n_active <= min(E, B*k) (the H
+// and dense-weight slots), every active id an expert, and offsets
+// non-decreasing within [0, B*k] with at most B pairs per expert (a token
+// chooses an expert once).  Inconsistent lists record DEV_BAD_LISTS and
+// run as an empty call (n_active = 0).  Token ids are checked where they
+// are used.
+__device__ int checked_n_active(const ExpertArgs &a, int lane) {
+    const int na = __ldcg(a.n_active);
+    const int pairs = a.B * a.k;
+    bool bad = na < 0 || na > min(a.E, pairs);
+    if (!bad) {
+        for (int i = lane; i < na; i += 32) {
+            const int e = __ldcg(a.active + i);
+            const int o0 = __ldcg(a.offsets + i), o1 = __ldcg(a.offsets + i + 1);
+            bad = bad || e < 0 || e >= a.E || o0 < 0 || o1 < o0 || o1 > pairs || o1 - o0 > a.B;
+        }
+    }
+    bad = __any_sync(0xffffffffu, bad);
+    if (bad && lane == 0) atomicCAS(&a.ctr->error, 0, DEV_BAD_LISTS);
+    return bad ? 0 : na;
+}
+
 template <class RG>
 __global__ void __launch_bounds__(NTHREADS, 1)
     expert_ffn_kernel(const __grid_constant__ ExpertMaps maps, const ExpertArgs a) {
@@ -819,49 +845,49 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 ctl->n_active = na;
                 ctl->total_tiles = na;
             }
-        } else if (a.dense) {
-            const int na = __ldcg(a.n_active);
-            // one tile per active expert; H rows of slot i start at i * B
-            for (int i = lane; i < na; i += 32) {
-                ctl->tile_start[i] = i;
-                ctl->act_e[i] = __ldcg(a.active + i);
-                ctl->off[i] = i * a.B;
-            }
-            if (lane == 0) {
-                const bool valid = na >= 0 && na <= a.E;
-                ctl->tile_start[valid ? na : 0] = valid ? na : 0;
-                ctl->off[valid ? na : 0] = (valid ? na : 0) * a.B;
-                ctl->n_active = valid ? na : 0;
-                ctl->total_tiles = (na > 0 && valid) ? na : 0;
-                if (!valid) atomicCAS(&a.ctr->error, 0, DEV_BAD_LISTS);
-            }
         } else {
-            const int na = __ldcg(a.n_active);
-            // tile table: active expert i owns tiles [tile_start[i], tile_start[i+1])
-            int run = 0;
-            for (int base_i = 0; base_i < na; base_i += 32) {
-                const int i = base_i + lane;
-                int nt = 0;
-                if (i < na) nt = (__ldg(a.offsets + i + 1) - __ldg(a.offsets + i) + TN - 1) / TN;
-                int incl = nt;
+            // lists from the caller (or the selection): checked before any
+            // of their values is used as an index
+            const int na = checked_n_active(a, lane);
+            if (a.dense) {
+                // one tile per active expert; H rows of slot i start at i * B
+                for (int i = lane; i < na; i += 32) {
+                    ctl->tile_start[i] = i;
+                    ctl->act_e[i] = __ldcg(a.active + i);
+                    ctl->off[i] = i * a.B;
+                }
+                if (lane == 0) {
+                    ctl->tile_start[na] = na;
+                    ctl->off[na] = na * a.B;
+                    ctl->n_active = na;
+                    ctl->total_tiles = na;
+                }
+            } else {
+                // tile table: active expert i owns tiles [tile_start[i], tile_start[i+1])
+                int run = 0;
+                for (int base_i = 0; base_i < na; base_i += 32) {
+                    const int i = base_i + lane;
+                    int nt = 0;
+                    if (i < na) nt = (__ldcg(a.offsets + i + 1) - __ldcg(a.offsets + i) + TN - 1) / TN;
+                    int incl = nt;
 #pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const int v = __shfl_up_sync(0xffffffffu, incl, o);
-                    if (lane >= o) incl += v;
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                        if (lane >= o) incl += v;
+                    }
+                    if (i < na) {
+                        ctl->tile_start[i] = run + incl - nt;
+                        ctl->act_e[i] = __ldcg(a.active + i);
+                        ctl->off[i] = __ldcg(a.offsets + i);
+                    }
+                    run += __shfl_sync(0xffffffffu, incl, 31);
                 }
-                if (i < na) {
-                    ctl->tile_start[i] = run + incl - nt;
-                    ctl->act_e[i] = __ldg(a.active + i);
-                    ctl->off[i] = __ldg(a.offsets + i);
+                if (lane == 0) {
+                    ctl->off[na] = na > 0 ? __ldcg(a.offsets + na) : 0;
+                    ctl->tile_start[na] = run;
+                    ctl->n_active = na;
+                    ctl->total_tiles = run;
                 }
-                run += __shfl_sync(0xffffffffu, incl, 31);
-            }
-            if (lane == 0 && na >= 0 && na <= a.E) ctl->off[na] = __ldg(a.offsets + na);
-            if (lane == 0) {
-                ctl->tile_start[na >= 0 && na <= a.E ? na : 0] = run;
-                ctl->n_active = na;
-                ctl->total_tiles = (na > 0 && na <= a.E) ? run : 0;
-                if (na < 0 || na > a.E) atomicCAS(&a.ctr->error, 0, DEV_BAD_LISTS);
             }
         }
     }
@@ -901,7 +927,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 //  - the gate/up completion counts cleared (standalone path).
 struct PrepArgs {
     const float *x;
-    int B, d;
+    int B, d, k;
+    int slots;     // active-expert slots: min(E, B*k)
     uint16_t *xb;  // dense mode: x in bf16, or null
     uint16_t *xd;  // larger batches: dispatched x rows, or null
     float *y;      // zeroed when non-null
@@ -909,6 +936,7 @@ struct PrepArgs {
     const int32_t *n_active, *offsets, *tok;
     const float *w;
     float *wd;  // dense weights [slot][B] (B <= 32), or null
+    int32_t *err;  // error word for inconsistent lists, or null
 };
 
 __device__ __forceinline__ uint2 bf16x4(float4 v) {
@@ -932,10 +960,15 @@ __global__ void __launch_bounds__(256) ffn_prep_kernel(PrepArgs p) {
             if (p.y) reinterpret_cast<float4 *>(p.y)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
     }
+    // the lists may come from the caller: n_active and the offsets are
+    // clamped to the buffers they index (min(E, B*k) active slots, B*k
+    // pairs) and tokens outside the batch are skipped; the expert kernel
+    // checks the same lists and reports inconsistent ones
+    const int pairs = p.B * p.k;
     if (p.xd) {
         // one thread per 4 columns of a pair row; rows of unused pairs skipped
         const int na = *p.n_active;
-        const int total = (na > 0 && na <= 256) ? p.offsets[na] : 0;
+        const int total = (na > 0 && na <= p.slots) ? min(max(p.offsets[na], 0), pairs) : 0;
         const int q4 = p.d / 4;
         for (int i = tid; i < total * q4; i += nthreads) {
             const int pr = i / q4, c = i - pr * q4;
@@ -948,15 +981,18 @@ __global__ void __launch_bounds__(256) ffn_prep_kernel(PrepArgs p) {
     if (p.wd) {
         // wd[i][t] = weight of token t in active expert i's list, else 0:
         // one warp per active expert (its list holds at most B <= 32 pairs)
-        const int na = *p.n_active;
+        const int na0 = *p.n_active;
+        const int na = (na0 > 0 && na0 <= p.slots) ? na0 : 0;
         const int lane = threadIdx.x & 31;
         for (int i = tid >> 5; i < na; i += nthreads >> 5) {
-            const int j0 = p.offsets[i], n = p.offsets[i + 1] - j0;
+            const int j0 = min(max(p.offsets[i], 0), pairs);
+            const int n = min(max(p.offsets[i + 1], j0), pairs) - j0;
             const int t = lane < n ? p.tok[j0 + lane] : -1;
             const float wv = lane < n ? p.w[j0 + lane] : 0.0f;
             if (lane < p.B) p.wd[static_cast<size_t>(i) * p.B + lane] = 0.0f;
             __syncwarp();
-            if (t >= 0) p.wd[static_cast<size_t>(i) * p.B + t] = wv;
+            if (t >= 0 && t < p.B) p.wd[static_cast<size_t>(i) * p.B + t] = wv;
+            else if (lane < n && p.err) atomicCAS(p.err, 0, DEV_BAD_LISTS);  // pair skipped
         }
     }
     if (p.ctr && blockIdx.x == 0)
@@ -1015,6 +1051,9 @@ cudaError_t launch_ffn_prep(const float *x, const moe_dims_t &d, uint16_t *xb, u
     p.x = x;
     p.B = d.B;
     p.d = d.d;
+    p.k = d.k;
+    p.slots = active_slots(d);
+    p.err = ctr ? &ctr->error : nullptr;
     p.xb = xb;
     p.xd = xd;
     p.y = y;

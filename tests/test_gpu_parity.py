@@ -3,9 +3,10 @@ the same seeded inputs.
 
 Router and re-selection: bit-exact (logits, probabilities, indices,
 weights, lists).  Layer output: max-abs 2e-2 and relative-L2 1e-2 against
-the fp64 oracle.  Sizes run from the tiny layer (several tiles plus ragged
-tails) to the full Qwen3-30B-A3B- and Qwen3-235B-A22B-shaped layers, where
-the oracle's FFN is evaluated on sampled tokens."""
+the fp64 oracle, every row of y up to 64 tokens (sampled rows only for the
+256-token and 100-token edge layers).  Sizes run from the tiny layer
+(several tiles plus ragged tails) to the full Qwen3-30B-A3B- and
+Qwen3-235B-A22B-shaped layers."""
 import os
 
 import numpy as np
@@ -193,22 +194,22 @@ Q30_CASES = [(1, NONE, 0, 0), (1, OEA, 2, 0), (4, OEA, 4, 0), (16, NONE, 0, 0), 
 
 @pytest.mark.parametrize("B,mode,k0,budget", Q30_CASES)
 def test_layer_decode_parity_q30b(B, mode, k0, budget):
+    # every row of y against the oracle
     S, L, x, y, sel, selw, n_act = _run_layer("q30b", B, 0, mode, k0, budget)
-    rows = np.unique(np.linspace(0, B - 1, min(B, 6)).astype(np.int32))
-    sel_r, w_r, n_r, y_r = _oracle_layer(S, L, x, mode, k0, budget, rows)
+    sel_r, w_r, n_r, y_r = _oracle_layer(S, L, x, mode, k0, budget, None)
     assert np.array_equal(sel, sel_r)
     assert np.array_equal(bits(selw), bits(w_r))
     assert n_act == n_r
-    assert_close_y(y[rows], y_r, f"q30b B={B} mode={mode} k0={k0}")
+    assert_close_y(y, y_r, f"q30b B={B} mode={mode} k0={k0}")
 
 
 @pytest.mark.parametrize("budget", [24, 32, 48])
 def test_layer_decode_parity_speculative(budget):
     S, L, x, y, sel, selw, n_act = _run_layer("q30b", 32, 0, XSHARE, 0, budget, kind="spec")
-    rows = np.array([0, 5, 13, 31], np.int32)
-    sel_r, w_r, n_r, y_r = _oracle_layer(S, L, x, XSHARE, 0, budget, rows)
+    sel_r, w_r, n_r, y_r = _oracle_layer(S, L, x, XSHARE, 0, budget, None)
     assert np.array_equal(sel, sel_r) and n_act == n_r <= budget
-    assert_close_y(y[rows], y_r, f"spec budget={budget}")
+    assert np.array_equal(bits(selw), bits(w_r))
+    assert_close_y(y, y_r, f"spec budget={budget}")
 
 
 HIER_LAYER_CASES = [("q30b", 16, 4, 16), ("q30b", 16, 3, 24), ("q30b", 32, 4, 24), ("q30b", 32, 4, 32),
@@ -222,21 +223,21 @@ def test_layer_decode_parity_xshare_hier(name, B, group, budget):
     # starts early; larger batches take the dispatch path
     kind = "spec" if name == "q30b" and B % 8 == 0 else "normal"
     S, L, x, y, sel, selw, n_act = _run_layer(name, B, 0, XSHARE_HIER, 0, budget, kind=kind, group=group)
-    rows = np.unique(np.linspace(0, B - 1, min(B, 6)).astype(np.int32))
+    rows = None if B <= 64 else np.arange(0, B, 7, dtype=np.int32)
     sel_r, w_r, n_r, y_r = _oracle_layer(S, L, x, XSHARE_HIER, 0, budget, rows, group=group)
     assert np.array_equal(sel, sel_r)
     assert np.array_equal(bits(selw), bits(w_r))
     assert n_act == n_r <= budget
-    assert_close_y(y[rows], y_r, f"{name} B={B} hierarchical group={group} budget={budget}")
+    assert_close_y(y if rows is None else y[rows], y_r, f"{name} B={B} hierarchical group={group} budget={budget}")
 
 
 @pytest.mark.parametrize("B,mode,k0", [(1, OEA, 4), (16, NONE, 0), (16, OEA, 4), (64, OEA, 4)])
 def test_layer_decode_parity_q235b(B, mode, k0):
     S, L, x, y, sel, selw, n_act = _run_layer("q235b", B, 0, mode, k0)
-    rows = np.unique(np.linspace(0, B - 1, min(B, 3)).astype(np.int32))
-    sel_r, w_r, n_r, y_r = _oracle_layer(S, L, x, mode, k0, 0, rows)
+    sel_r, w_r, n_r, y_r = _oracle_layer(S, L, x, mode, k0, 0, None)
     assert np.array_equal(sel, sel_r) and n_act == n_r
-    assert_close_y(y[rows], y_r, f"q235b B={B} mode={mode}")
+    assert np.array_equal(bits(selw), bits(w_r))
+    assert_close_y(y, y_r, f"q235b B={B} mode={mode}")
 
 
 def test_expert_ffn_entry_matches_oracle():
