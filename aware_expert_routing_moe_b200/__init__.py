@@ -23,7 +23,7 @@ __all__ = [
     "Dims", "Rule", "Lists", "load_library", "library_path", "moe_workspace_bytes",
     "moe_status_string", "moe_route", "moe_reselect", "moe_expert_ffn", "moe_layer_decode",
     "moe_check_error", "moe_expert_ffn_noalloc", "new_workspace", "alloc_lists", "ABI_SYMBOLS",
-    "NOALLOC_SCRATCH_BYTES",
+    "NOALLOC_SCRATCH_BYTES", "moe_set_wait_limit_ns",
 ]
 
 MOE_RESELECT_NONE, MOE_RESELECT_OEA, MOE_RESELECT_XSHARE = 0, 1, 2
@@ -31,7 +31,8 @@ MOE_RESELECT_AFFINITY, MOE_RESELECT_XSHARE_HIER = 3, 4
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_MISALIGNED", 3: "MOE_ERR_WORKSPACE",
           4: "MOE_ERR_UNSUPPORTED", 5: "MOE_ERR_CUDA", 6: "MOE_ERR_INTERNAL"}
 ABI_SYMBOLS = ("moe_workspace_bytes", "moe_route", "moe_reselect", "moe_expert_ffn",
-               "moe_layer_decode", "moe_expert_ffn_noalloc", "moe_check_error", "moe_status_string")
+               "moe_layer_decode", "moe_expert_ffn_noalloc", "moe_check_error", "moe_status_string",
+               "moe_set_wait_limit_ns")
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -88,6 +89,8 @@ def load_library() -> ctypes.CDLL:
         lib.moe_expert_ffn_noalloc.argtypes = [P, P, P, P, Dims, Lists, P, P]
         lib.moe_check_error.restype = ctypes.c_int
         lib.moe_check_error.argtypes = [P, S, P]
+        lib.moe_set_wait_limit_ns.restype = None
+        lib.moe_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
         _lib = lib
     return _lib
 
@@ -223,6 +226,11 @@ def moe_expert_ffn_noalloc(x, Wgate, Wup, Wdown, lists: dict, k: int, y=None, st
                                                Dims(B, d, E, k, F), _lists(lists), _ptr(y), _stream(stream))
     _check(st, "moe_expert_ffn_noalloc")
     return y
+
+
+def moe_set_wait_limit_ns(ns: int) -> None:
+    """Limit of the kernels' bounded waits for later launches (0 = 1 s)."""
+    load_library().moe_set_wait_limit_ns(int(ns))
 
 
 def moe_check_error(ws, stream=None) -> int:

@@ -2,6 +2,7 @@
 // validation, workspace layout, TMA descriptor encoding and launch chaining.
 // Nothing here allocates device memory; every failure is reported as a
 // status code before anything is enqueued.
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -12,6 +13,9 @@ namespace moe {
 namespace {
 
 constexpr size_t ALIGN = 256;
+constexpr unsigned long long DEFAULT_WAIT_NS = 1000000000ull;  // 1 s
+
+std::atomic<unsigned long long> g_wait_ns{DEFAULT_WAIT_NS};
 
 size_t round_up(size_t v) { return (v + ALIGN - 1) / ALIGN * ALIGN; }
 
@@ -180,6 +184,8 @@ bool encode_router_maps(RouterMaps *m, const moe_dims_t &d, const float *x, cons
            encode_f32_lines(&m->wg, Wg, static_cast<uint64_t>(d.E), static_cast<uint64_t>(d.d), bl);
 }
 
+unsigned long long wait_limit_ns() { return g_wait_ns.load(std::memory_order_relaxed); }
+
 WsLayout ws_layout(const moe_dims_t &d) {
     WsLayout L;
     size_t o = 0;
@@ -279,7 +285,7 @@ moe_status_t moe_expert_ffn(const float *x, const uint16_t *Wgate, const uint16_
     float *wd = dense ? seg<float>(ws, L.wd) : nullptr;
     st = from_cuda(launch_ffn_prep(x, dims, dense ? xk : nullptr, dense ? nullptr : xk, y, ctr, lists, wd, false, s));
     if (st != MOE_OK) return st;
-    return from_cuda(launch_expert_ffn(maps, xk, dims, lists, y, seg<uint16_t>(ws, L.h), wd, ctr, false, 0, s));
+    return from_cuda(launch_expert_ffn(maps, xk, dims, lists, y, seg<uint16_t>(ws, L.h), wd, ctr, s));
 }
 
 moe_status_t moe_layer_decode(const float *x, const float *Wg, const float *bias, const uint16_t *Wgate,
@@ -310,22 +316,25 @@ moe_status_t moe_layer_decode(const float *x, const float *Wg, const float *bias
     int32_t *si = sel_idx ? sel_idx : seg<int32_t>(ws, L.sel_idx);
     float *sw = sel_w ? sel_w : seg<float>(ws, L.sel_w);
     const moe_lists_t lists = ws_lists(ws, L);
-    // B <= 32: the expert kernel starts streaming as soon as the router has
-    // published the activated set.  Larger batches dispatch each pair's x
-    // row once the selection has built the lists, then stream.
-    float *wd = dense ? seg<float>(ws, L.wd) : nullptr;
-    st = from_cuda(launch_layer_route(rmaps, x, bias, dims, rule, logits, probs, dense ? xk : nullptr, y, ctr, dense,
-                                      s));
-    if (st != MOE_OK) return st;
-    st = from_cuda(launch_layer_select(logits, probs, dims, rule, si, sw, lists, n_active, ctr, wd, dense, s));
-    if (st != MOE_OK) return st;
-    if (!dense) {
-        st = from_cuda(launch_ffn_prep(x, dims, nullptr, xk, nullptr, nullptr, lists, nullptr, true, s));
-        if (st != MOE_OK) return st;
+    if (dense) {
+        // B <= 32: one persistent kernel for the whole call
+        return from_cuda(launch_layer_fused(maps, rmaps, dims, rule, x, bias, logits, probs, xk, y,
+                                            seg<uint16_t>(ws, L.h), seg<float>(ws, L.wd), si, sw, lists, n_active,
+                                            ctr, s));
     }
-    return from_cuda(launch_expert_ffn(maps, xk, dims, lists, y, seg<uint16_t>(ws, L.h), wd, ctr, dense,
-                                       layer_pub_target(dims, rule), s));
+    // larger batches: router, selection (lists), the dispatch of each
+    // pair's x row, then the expert kernel, chained with programmatic
+    // dependent launch
+    st = from_cuda(launch_layer_route(rmaps, x, bias, dims, logits, y, ctr, s));
+    if (st != MOE_OK) return st;
+    st = from_cuda(launch_layer_select(logits, probs, dims, rule, si, sw, lists, n_active, s));
+    if (st != MOE_OK) return st;
+    st = from_cuda(launch_ffn_prep(x, dims, nullptr, xk, nullptr, nullptr, lists, nullptr, true, s));
+    if (st != MOE_OK) return st;
+    return from_cuda(launch_expert_ffn(maps, xk, dims, lists, y, seg<uint16_t>(ws, L.h), nullptr, ctr, s));
 }
+
+void moe_set_wait_limit_ns(uint64_t ns) { g_wait_ns.store(ns == 0 ? DEFAULT_WAIT_NS : ns, std::memory_order_relaxed); }
 
 moe_status_t moe_check_error(void *ws, size_t ws_bytes, void *stream) {
     if (!ws || ws_bytes < sizeof(Counters)) return MOE_ERR_WORKSPACE;

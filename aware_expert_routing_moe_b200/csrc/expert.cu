@@ -44,6 +44,7 @@
 #include <cuda_bf16.h>
 
 #include "internal.h"
+#include "route_dev.cuh"
 
 namespace moe {
 namespace {
@@ -85,7 +86,12 @@ static_assert(RingSmallB::SLOT_BYTES % 1024 == 0 && RingLargeB::SLOT_BYTES % 102
               "slots must keep 1 KiB alignment for 128B swizzle");
 static_assert(smem_bytes<RingSmallB>() <= 232448 && smem_bytes<RingLargeB>() <= 232448, "shared memory budget");
 
-constexpr unsigned long long WAIT_LIMIT_NS = 1000000000ull;  // 1 s
+// Bounded waits: a wait on another CTA, another kernel or a copy gives up
+// after the call's wait limit (ExpertArgs::wait_ns, 1 s unless the caller
+// set another with moe_set_wait_limit_ns), records an error code and ends
+// the CTA's work; copies already in flight into its shared memory are then
+// drained, with a fixed limit, before the CTA exits.
+constexpr unsigned long long DRAIN_LIMIT_NS = 1000000000ull;  // 1 s
 constexpr int SPLIT_TABLE_MAX = 256;  // tile counts covered by the split table
 
 enum : int { UNIT_GU = 0, UNIT_D = 1, UNIT_END = 2 };
@@ -105,6 +111,7 @@ struct UnitRec {
 constexpr int UNIT_WINDOW = 32;  // units a producer decodes at once (one per lane)
 
 struct SharedCtl {
+    unsigned long long wait_ns;  // limit of every bounded wait of this call
     unsigned long long full[MAX_STAGES];
     unsigned long long empty[MAX_STAGES];
     unsigned long long sig_full[SIG_SLOTS];
@@ -127,6 +134,11 @@ static_assert(sizeof(SharedCtl) <= CTL_BYTES, "SharedCtl does not fit its reserv
 struct ExpertArgs {
     const uint16_t *xb;
     int B, d, E, k, F;
+    unsigned long long wait_ns;  // limit of the bounded waits
+    int unit_ctas;               // CTAs the work units are dealt to (0 .. unit_ctas-1)
+    // early mode: the dense weights are ready once *lists_flag >= 1 (fused
+    // layer kernel); null: once the previous kernel has completed
+    const int32_t *lists_flag;
     // dense mode (B <= TN): every stage works on all B tokens; gate/up stages
     // load all token rows of x in one box, H is token-indexed [slot][B][d_ff]
     // and the down epilogue weighs tokens by wd[slot][B]
@@ -250,7 +262,7 @@ __device__ bool wait_phase(unsigned long long *bar, unsigned parity, SharedCtl *
     for (;;) {
         if (mbar_try_wait(bar, parity)) return true;
         if (ctl->abort_flag) return false;
-        if (global_ns() - t0 > WAIT_LIMIT_NS) {
+        if (global_ns() - t0 > ctl->wait_ns) {
             record_error(ctr, ctl, code);
             return false;
         }
@@ -360,14 +372,14 @@ __device__ __forceinline__ void decode_rec(int u, int n_units, const ExpertArgs 
 }
 
 // The j-th unit of this CTA's round-robin sequence (units blockIdx.x +
-// j * gridDim.x).  The producer's lanes decode UNIT_WINDOW units at a time
+// j * unit_ctas).  The producer's lanes decode UNIT_WINDOW units at a time
 // into shared memory; the prefetches of the unit's first stage are issued
 // here and first used when that stage is issued.
 __device__ bool fetch_unit(int j, int &win_base, int n_units, const ExpertArgs &a, SharedCtl *ctl, int lane,
                            UnitInfo &ui) {
     if (j >= win_base + UNIT_WINDOW) {
         __syncwarp();
-        decode_rec(blockIdx.x + (j + lane) * gridDim.x, n_units, a, ctl, ctl->urec[lane]);
+        decode_rec(blockIdx.x + (j + lane) * a.unit_ctas, n_units, a, ctl, ctl->urec[lane]);
         __syncwarp();
         win_base = j;
     }
@@ -450,7 +462,7 @@ __device__ void producer(const ExpertArgs &a, const ExpertMaps &m, SharedCtl *ct
                             const unsigned long long t0 = global_ns();
                             while ((v = ld_acquire(&a.ctr->gu_done[cur.i_act])) < cur.need) {
                                 if (ctl->abort_flag) { ok = false; break; }
-                                if (global_ns() - t0 > WAIT_LIMIT_NS) {
+                                if (global_ns() - t0 > a.wait_ns) {
                                     record_error(a.ctr, ctl, DEV_TIMEOUT_DEP);
                                     ok = false;
                                     break;
@@ -487,7 +499,7 @@ __device__ void producer(const ExpertArgs &a, const ExpertMaps &m, SharedCtl *ct
         for (int q = ctl->consumed; q < g; ++q) {
             const unsigned long long t0 = global_ns();
             while (!mbar_try_wait(&ctl->full[q % STAGES], (q / STAGES) & 1)) {
-                if (global_ns() - t0 > WAIT_LIMIT_NS) break;
+                if (global_ns() - t0 > DRAIN_LIMIT_NS) break;
             }
         }
     }
@@ -602,7 +614,24 @@ __device__ void consumer(const ExpertArgs &a, SharedCtl *ctl, unsigned char *slo
                 // the dense weights are the selection's last output: in early
                 // mode wait for it to complete before the first down unit
                 if (!lists_ready) {
-                    asm volatile("griddepcontrol.wait;" ::: "memory");
+                    if (a.lists_flag == nullptr) {
+                        asm volatile("griddepcontrol.wait;" ::: "memory");
+                    } else {
+                        // fused layer kernel: the selection CTA raises the flag
+                        if (ct == 0) {
+                            const unsigned long long t0 = global_ns();
+                            while (ld_acquire(a.lists_flag) < 1) {
+                                if (ctl->abort_flag) break;
+                                if (global_ns() - t0 > a.wait_ns) {
+                                    record_error(a.ctr, ctl, DEV_TIMEOUT_DEP);
+                                    break;
+                                }
+                                __nanosleep(64);
+                            }
+                        }
+                        consumer_bar();
+                        if (ctl->abort_flag) return;
+                    }
                     lists_ready = true;
                 }
 #pragma unroll
@@ -755,153 +784,172 @@ __device__ int checked_n_active(const ExpertArgs &a, int lane) {
     return bad ? 0 : na;
 }
 
+// Shared memory of an expert CTA: the ring slots, the gate/up epilogue
+// buffer and the control block, from a 1024-byte aligned base.
 template <class RG>
-__global__ void __launch_bounds__(NTHREADS, 1)
-    expert_ffn_kernel(const __grid_constant__ ExpertMaps maps, const ExpertArgs a) {
-    constexpr int STAGES = RG::STAGES;
-    extern __shared__ unsigned char smem_raw[];
-    unsigned char *base = reinterpret_cast<unsigned char *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    unsigned char *slots = base;
-    float *part = reinterpret_cast<float *>(base + STAGES * RG::SLOT_BYTES);
-    SharedCtl *ctl = reinterpret_cast<SharedCtl *>(part + PART_FLOATS);
+struct CtaSmem {
+    unsigned char *slots;
+    float *part;
+    SharedCtl *ctl;
+    __device__ explicit CtaSmem(unsigned char *raw) {
+        unsigned char *base = reinterpret_cast<unsigned char *>(
+            (reinterpret_cast<uintptr_t>(raw) + 1023) & ~static_cast<uintptr_t>(1023));
+        slots = base;
+        part = reinterpret_cast<float *>(base + RG::STAGES * RG::SLOT_BYTES);
+        ctl = reinterpret_cast<SharedCtl *>(part + PART_FLOATS);
+    }
+};
 
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&ctl->full[s], 1);
-            mbar_init(&ctl->empty[s], NCW);
-        }
-        for (int s = 0; s < SIG_SLOTS; ++s) {
-            mbar_init(&ctl->sig_full[s], 1);
-            mbar_init(&ctl->sig_empty[s], 1);
-        }
-        ctl->abort_flag = 0;
-        ctl->consumed = 0;
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+// Barriers and flags of a CTA (thread 0).
+template <class RG>
+__device__ void ctl_init(SharedCtl *ctl, unsigned long long wait_ns) {
+    for (int s = 0; s < RG::STAGES; ++s) {
+        mbar_init(&ctl->full[s], 1);
+        mbar_init(&ctl->empty[s], NCW);
     }
-    if (warp == NCW && lane == 0) {
-        prefetch_tmap(&maps.gate);
-        prefetch_tmap(&maps.up);
-        prefetch_tmap(&maps.down);
-        prefetch_tmap(&maps.h);
-        prefetch_tmap(&maps.x);
+    for (int s = 0; s < SIG_SLOTS; ++s) {
+        mbar_init(&ctl->sig_full[s], 1);
+        mbar_init(&ctl->sig_empty[s], 1);
     }
-    // everything above overlaps the selection.  Early mode: wait only until
-    // the activated set is published; otherwise until the previous kernel
-    // (selection or input preparation) has completed.
-    if (!a.early) asm volatile("griddepcontrol.wait;" ::: "memory");
+    ctl->wait_ns = wait_ns;
+    ctl->abort_flag = 0;
+    ctl->consumed = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void prefetch_expert_maps(const ExpertMaps &maps) {
+    prefetch_tmap(&maps.gate);
+    prefetch_tmap(&maps.up);
+    prefetch_tmap(&maps.down);
+    prefetch_tmap(&maps.h);
+    prefetch_tmap(&maps.x);
+}
+
+// Dense mode from an activated-set bit mask (producer warp; lane l holds
+// word l, experts 32 l .. 32 l + 31): one tile per active expert in
+// ascending expert order, the slot order the selection uses for H and the
+// dense weights; H rows of slot i start at i * B.
+__device__ void table_from_mask(const ExpertArgs &a, SharedCtl *ctl, unsigned word, int lane) {
+    if (32 * lane >= a.E) word = 0u;
+    else if (a.E - 32 * lane < 32) word &= (1u << (a.E - 32 * lane)) - 1u;
+    int incl = __popc(word);
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    int pos = incl - __popc(word);
+    while (word != 0u) {
+        const int bit = __ffs(word) - 1;
+        word &= word - 1u;
+        ctl->act_e[pos] = 32 * lane + bit;
+        ctl->tile_start[pos] = pos;
+        ctl->off[pos] = pos * a.B;
+        ++pos;
+    }
+    const int na = __shfl_sync(0xffffffffu, incl, 31);
+    if (lane == 0) {
+        ctl->tile_start[na] = na;
+        ctl->off[na] = na * a.B;
+        ctl->n_active = na;
+        ctl->total_tiles = na;
+    }
+}
+
+// Early mode: wait (bounded) until the activated set is published in the
+// CTA's copy of the publication line, then build the table from its mask.
+__device__ void table_from_publication(const ExpertArgs &a, SharedCtl *ctl, int lane) {
+    bool ok = true;
+    uint4 m0 = make_uint4(0u, 0u, 0u, 0u), m1 = m0;
+    const PubLine *pl = &a.ctr->pubs[blockIdx.x % PUB_COPIES];
+    if (lane == 0) {
+        const unsigned long long t0 = global_ns();
+        while (ld_acquire(&pl->pub) < a.pub_target) {
+            if (global_ns() - t0 > a.wait_ns) {
+                record_error(a.ctr, ctl, DEV_TIMEOUT_DEP);
+                ok = false;
+                break;
+            }
+            __nanosleep(64);
+        }
+        if (ok) {
+            m0 = __ldcg(reinterpret_cast<const uint4 *>(pl->mask));
+            m1 = __ldcg(reinterpret_cast<const uint4 *>(pl->mask) + 1);
+        }
+    }
+    const unsigned mw[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+    unsigned word = 0u;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const unsigned v = __shfl_sync(0xffffffffu, mw[i], 0);
+        if (lane == i) word = v;
+    }
+    table_from_mask(a, ctl, word, lane);
+}
+
+// Lists from the caller (or the selection kernel): checked, then the tile
+// table (producer warp).
+__device__ void table_from_lists(const ExpertArgs &a, SharedCtl *ctl, int lane) {
+    const int na = checked_n_active(a, lane);
+    if (a.dense) {
+        // one tile per active expert; H rows of slot i start at i * B
+        for (int i = lane; i < na; i += 32) {
+            ctl->tile_start[i] = i;
+            ctl->act_e[i] = __ldcg(a.active + i);
+            ctl->off[i] = i * a.B;
+        }
+        if (lane == 0) {
+            ctl->tile_start[na] = na;
+            ctl->off[na] = na * a.B;
+            ctl->n_active = na;
+            ctl->total_tiles = na;
+        }
+        return;
+    }
+    // tile table: active expert i owns tiles [tile_start[i], tile_start[i+1])
+    int run = 0;
+    for (int base_i = 0; base_i < na; base_i += 32) {
+        const int i = base_i + lane;
+        int nt = 0;
+        if (i < na) nt = (__ldcg(a.offsets + i + 1) - __ldcg(a.offsets + i) + TN - 1) / TN;
+        int incl = nt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        if (i < na) {
+            ctl->tile_start[i] = run + incl - nt;
+            ctl->act_e[i] = __ldcg(a.active + i);
+            ctl->off[i] = __ldcg(a.offsets + i);
+        }
+        run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) {
+        ctl->off[na] = na > 0 ? __ldcg(a.offsets + na) : 0;
+        ctl->tile_start[na] = run;
+        ctl->n_active = na;
+        ctl->total_tiles = run;
+    }
+}
+
+template <class RG>
+__device__ __forceinline__ void run_roles(const ExpertArgs &a, const ExpertMaps &maps, const CtaSmem<RG> &sm) {
+    const int warp = threadIdx.x >> 5;
     if (warp == NCW) {
-        if (a.early) {
-            // dense mode: one tile per active expert, taken from the published
-            // bit mask (ascending expert order, the order of the selection's
-            // active list); H rows of slot i start at i * B
-            bool ok = true;
-            uint4 m0 = make_uint4(0u, 0u, 0u, 0u), m1 = m0;
-            const PubLine *pl = &a.ctr->pubs[blockIdx.x % PUB_COPIES];
-            if (lane == 0) {
-                const unsigned long long t0 = global_ns();
-                while (ld_acquire(&pl->pub) < a.pub_target) {
-                    if (global_ns() - t0 > WAIT_LIMIT_NS) {
-                        record_error(a.ctr, ctl, DEV_TIMEOUT_DEP);
-                        ok = false;
-                        break;
-                    }
-                    __nanosleep(64);
-                }
-                if (ok) {
-                    m0 = __ldcg(reinterpret_cast<const uint4 *>(pl->mask));
-                    m1 = __ldcg(reinterpret_cast<const uint4 *>(pl->mask) + 1);
-                }
-            }
-            const unsigned mw[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
-            unsigned word = 0u;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const unsigned v = __shfl_sync(0xffffffffu, mw[i], 0);
-                if (lane == i) word = v;
-            }
-            if (32 * lane >= a.E) word = 0u;
-            else if (a.E - 32 * lane < 32) word &= (1u << (a.E - 32 * lane)) - 1u;
-            int incl = __popc(word);
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int v = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += v;
-            }
-            int pos = incl - __popc(word);
-            while (word != 0u) {
-                const int bit = __ffs(word) - 1;
-                word &= word - 1u;
-                ctl->act_e[pos] = 32 * lane + bit;
-                ctl->tile_start[pos] = pos;
-                ctl->off[pos] = pos * a.B;
-                ++pos;
-            }
-            const int na = __shfl_sync(0xffffffffu, incl, 31);
-            if (lane == 0) {
-                ctl->tile_start[na] = na;
-                ctl->off[na] = na * a.B;
-                ctl->n_active = na;
-                ctl->total_tiles = na;
-            }
-        } else {
-            // lists from the caller (or the selection): checked before any
-            // of their values is used as an index
-            const int na = checked_n_active(a, lane);
-            if (a.dense) {
-                // one tile per active expert; H rows of slot i start at i * B
-                for (int i = lane; i < na; i += 32) {
-                    ctl->tile_start[i] = i;
-                    ctl->act_e[i] = __ldcg(a.active + i);
-                    ctl->off[i] = i * a.B;
-                }
-                if (lane == 0) {
-                    ctl->tile_start[na] = na;
-                    ctl->off[na] = na * a.B;
-                    ctl->n_active = na;
-                    ctl->total_tiles = na;
-                }
-            } else {
-                // tile table: active expert i owns tiles [tile_start[i], tile_start[i+1])
-                int run = 0;
-                for (int base_i = 0; base_i < na; base_i += 32) {
-                    const int i = base_i + lane;
-                    int nt = 0;
-                    if (i < na) nt = (__ldcg(a.offsets + i + 1) - __ldcg(a.offsets + i) + TN - 1) / TN;
-                    int incl = nt;
-#pragma unroll
-                    for (int o = 1; o < 32; o <<= 1) {
-                        const int v = __shfl_up_sync(0xffffffffu, incl, o);
-                        if (lane >= o) incl += v;
-                    }
-                    if (i < na) {
-                        ctl->tile_start[i] = run + incl - nt;
-                        ctl->act_e[i] = __ldcg(a.active + i);
-                        ctl->off[i] = __ldcg(a.offsets + i);
-                    }
-                    run += __shfl_sync(0xffffffffu, incl, 31);
-                }
-                if (lane == 0) {
-                    ctl->off[na] = na > 0 ? __ldcg(a.offsets + na) : 0;
-                    ctl->tile_start[na] = run;
-                    ctl->n_active = na;
-                    ctl->total_tiles = run;
-                }
-            }
-        }
-    }
-    __syncthreads();
-    if (warp == NCW) {
-        producer<RG>(a, maps, ctl, slots);
+        producer<RG>(a, maps, sm.ctl, sm.slots);
     } else if (warp == NCW + 1) {
-        signaller(a, ctl);
+        signaller(a, sm.ctl);
     } else {
-        consumer<RG>(a, ctl, slots, part);
+        consumer<RG>(a, sm.ctl, sm.slots, sm.part);
     }
-    // The last CTA to finish puts the call's counters back to zero (every
-    // CTA has read the published set and no gate/up count is awaited any
-    // more); the next call's first kernel starts after this grid completes.
+}
+
+// The last CTA to finish puts the call's counters back to zero (every CTA
+// has passed the grid barrier, read the published set and awaits no
+// gate/up count any more); the next call's kernels start after this grid
+// completes.
+__device__ void cta_exit(const ExpertArgs &a, SharedCtl *ctl) {
     __syncthreads();
     if (threadIdx.x == 0) {
         __threadfence();
@@ -914,8 +962,215 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int i = threadIdx.x; i < PUB_COPIES * (E_MAX / 32); i += blockDim.x)
             a.ctr->pubs[i / (E_MAX / 32)].mask[i % (E_MAX / 32)] = 0u;
         if (threadIdx.x < PUB_COPIES) a.ctr->pubs[threadIdx.x].pub = 0;
-        if (threadIdx.x == 0) a.ctr->k3_exit = 0;
+        if (threadIdx.x == 0) {
+            a.ctr->k3_exit = 0;
+            a.ctr->arrive = 0;
+            a.ctr->lists_ready = 0;
+        }
     }
+}
+
+template <class RG>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    expert_ffn_kernel(const __grid_constant__ ExpertMaps maps, const ExpertArgs a) {
+    extern __shared__ unsigned char smem_raw[];
+    const CtaSmem<RG> sm(smem_raw);
+    SharedCtl *ctl = sm.ctl;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) ctl_init<RG>(ctl, a.wait_ns);
+    if (warp == NCW && lane == 0) prefetch_expert_maps(maps);
+    // everything above overlaps the previous kernel (selection or input
+    // preparation); the lists are complete once it has
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (warp == NCW) table_from_lists(a, ctl, lane);
+    __syncthreads();
+    run_roles<RG>(a, maps, sm);
+    cta_exit(a, ctl);
+}
+
+// ------------------------------------------------------ fused layer kernel --
+// One persistent grid for the whole layer call when B <= 32 (dense mode),
+// one CTA per SM, launched cooperatively so that every CTA is resident:
+//  1. router: the CTAs compute the logits in items of (epb experts) x (tpb
+//     tokens) with the router's fixed-order dot products (rows staged by
+//     TMA in the ring's shared memory); meanwhile every CTA writes its share
+//     of x in bf16 and zeroes its share of y;
+//  2. grid barrier: each CTA counts itself in (release) and waits (acquire,
+//     bounded) until all have;
+//  3. the last CTA runs the batch selection (softmax, re-selection, weights,
+//     lists, dense weights) and raises a flag when the dense weights are
+//     written; for the batch-wide rules it publishes the activated set as
+//     soon as that is fixed;
+//  4. every other CTA takes the activated set -- OEA and plain top-k: it
+//     ranks every token's first r1 experts itself (the union of the kept
+//     sets, resp. of the top-k sets, is final before any fill is chosen);
+//     the batch-wide rules: from the selection CTA's publication -- and
+//     streams its share of the activated experts' units as the standalone
+//     expert kernel does, waiting for the flag only before its first down
+//     epilogue.
+struct LayerArgs {
+    const float *x;     // [B][d] fp32
+    const float *bias;  // [E] or null
+    float *logits;      // [B][E]
+    int epb, tpb;       // experts (one warp each) and tokens per router item
+    int n_eg, n_items;  // expert groups; items = expert groups x token groups
+    int row_bytes;      // shared-memory stride of one staged row (multiple of 1024)
+    int box_lines, boxes;
+    int r1;             // first ranks per token forming the set (OEA: k0, top-k: k); 0: published
+    ReselectArgs sel;   // the selection CTA's arguments
+};
+
+template <class RG, int NI>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    layer_kernel(const __grid_constant__ ExpertMaps maps, const __grid_constant__ RouterMaps rmaps,
+                 const ExpertArgs a, const LayerArgs L) {
+    extern __shared__ unsigned char smem_raw[];
+    const CtaSmem<RG> sm(smem_raw);
+    SharedCtl *ctl = sm.ctl;
+    __shared__ __align__(8) unsigned long long s_rbar;  // router row staging
+    __shared__ unsigned s_set[E_MAX / 32];
+    __shared__ int s_ok;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        ctl_init<RG>(ctl, a.wait_ns);
+        mbar_init(&s_rbar, 1);
+        s_ok = 1;
+    }
+    if (threadIdx.x < E_MAX / 32) s_set[threadIdx.x] = 0u;
+    if (warp == NCW && lane == 0) {
+        prefetch_expert_maps(maps);
+        prefetch_tmap(&rmaps.x);
+        prefetch_tmap(&rmaps.wg);
+    }
+    __syncthreads();
+
+    // ---- 1. router items (one per CTA when there are no more items than CTAs)
+    unsigned char *wrows = sm.slots;
+    unsigned char *xrows = sm.slots + L.epb * L.row_bytes;
+    bool prepped = false;
+    int phase = 0;
+    for (int item = blockIdx.x; item < L.n_items; item += gridDim.x) {
+        const int eg = item % L.n_eg, tg = item / L.n_eg;
+        const int e0 = eg * L.epb, b0 = tg * L.tpb;
+        const int ne = min(L.epb, a.E - e0), nb = min(L.tpb, a.B - b0);
+        if (threadIdx.x == 0) {
+            mbar_expect_tx(&s_rbar, static_cast<unsigned>((ne + nb) * L.boxes * L.box_lines * 128));
+            const int lines = a.d >> 5;  // 128-byte lines per row
+            for (int r = 0; r < ne; ++r)
+                for (int bx = 0; bx < L.boxes; ++bx)
+                    tma_rows(wrows + r * L.row_bytes + bx * L.box_lines * 128, &rmaps.wg,
+                             (e0 + r) * lines + bx * L.box_lines, &s_rbar);
+            for (int r = 0; r < nb; ++r)
+                for (int bx = 0; bx < L.boxes; ++bx)
+                    tma_rows(xrows + r * L.row_bytes + bx * L.box_lines * 128, &rmaps.x,
+                             (b0 + r) * lines + bx * L.box_lines, &s_rbar);
+        }
+        if (!prepped) {
+            // x -> bf16 (read by the gate/up copies) and y = 0 (the down
+            // epilogues add into it), grid-stride: overlaps the row loads
+            layer_prep(L.x, a.B, a.d, const_cast<uint16_t *>(a.xb), a.y);
+            prepped = true;
+        }
+        // every thread waits for the rows; on expiry the rows are still
+        // awaited (drained) before the shared memory is used for anything else
+        if (!mbar_try_wait(&s_rbar, phase)) {
+            const unsigned long long t0 = global_ns();
+            bool late = false;
+            while (!mbar_try_wait(&s_rbar, phase)) {
+                const unsigned long long dt = global_ns() - t0;
+                if (!late && dt > a.wait_ns) {
+                    late = true;
+                    s_ok = 0;
+                    atomicCAS(&a.ctr->error, 0, DEV_TIMEOUT_FULL);
+                }
+                if (dt > a.wait_ns + DRAIN_LIMIT_NS) break;
+            }
+        }
+        __syncthreads();
+        if (warp < ne && s_ok) {
+            const int e = e0 + warp;
+            float acc[GEMV_TPB_MAX];
+#pragma unroll
+            for (int t = 0; t < GEMV_TPB_MAX; ++t) acc[t] = 0.0f;
+            if ((a.d & 255) == 0) gemv_rows<true>(wrows + warp * L.row_bytes, xrows, L.row_bytes, a.d, nb, lane, acc);
+            else gemv_rows<false>(wrows + warp * L.row_bytes, xrows, L.row_bytes, a.d, nb, lane, acc);
+            float mine = 0.0f;
+#pragma unroll
+            for (int t = 0; t < GEMV_TPB_MAX; ++t) {
+                const float v = warp_butterfly_sum(acc[t]);
+                if (lane == t) mine = v;
+            }
+            if (lane < nb) {
+                const float v = L.bias ? __fadd_rn(mine, __ldg(L.bias + e)) : mine;
+                L.logits[static_cast<size_t>(b0 + lane) * a.E + e] = v;
+            }
+        }
+        __syncthreads();  // the staging area is free again
+        phase ^= 1;
+    }
+    if (!prepped) layer_prep(L.x, a.B, a.d, const_cast<uint16_t *>(a.xb), a.y);
+    // x in bf16 is read by the async proxy (TMA) of other CTAs
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    __syncthreads();
+
+    // ---- 2. grid barrier
+    if (threadIdx.x == 0) {
+        __threadfence();
+        asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(&a.ctr->arrive), "r"(1) : "memory");
+        const unsigned long long t0 = global_ns();
+        while (ld_acquire(&a.ctr->arrive) < static_cast<int>(gridDim.x)) {
+            if (global_ns() - t0 > a.wait_ns) {
+                atomicCAS(&a.ctr->error, 0, DEV_TIMEOUT_DEP);
+                s_ok = 0;
+                break;
+            }
+        }
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+    }
+    __syncthreads();
+    const bool ok = s_ok != 0;
+
+    // ---- 3. the selection CTA
+    if (blockIdx.x == gridDim.x - 1) {
+        if (ok) reselect_body<NI>(L.sel, sm.slots);
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            __threadfence();
+            asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(&a.ctr->lists_ready), "r"(1) : "memory");
+        }
+        cta_exit(a, ctl);
+        return;
+    }
+
+    // ---- 4. the activated set, then the expert stream
+    if (L.r1 > 0) {
+        if (warp < NCW && ok) {
+#pragma unroll 1
+            for (int b = warp; b < a.B; b += NCW) {
+                float l[NI];
+                unsigned ord[NI];
+                load_row<NI>(L.logits + static_cast<size_t>(b) * a.E, a.E, lane, l);
+#pragma unroll
+                for (int i = 0; i < NI; ++i) ord[i] = ord_of(l[i]);
+                unsigned cand = valid_bits<NI>(a.E, lane);
+                int mye = -1;
+#pragma unroll 1
+                for (int j = 0; j < L.r1; ++j) {
+                    const int e = warp_argmax<NI>(ord, cand, lane);
+                    if (lane == j) mye = e;
+                }
+                if (lane < L.r1 && mye >= 0) atomicOr(&s_set[mye >> 5], 1u << (mye & 31));
+            }
+        }
+        __syncthreads();
+        if (warp == NCW) table_from_mask(a, ctl, lane < E_MAX / 32 ? s_set[lane] : 0u, lane);
+    } else if (warp == NCW) {
+        if (ok) table_from_publication(a, ctl, lane);
+        else table_from_mask(a, ctl, 0u, lane);
+    }
+    __syncthreads();
+    run_roles<RG>(a, maps, sm);
+    cta_exit(a, ctl);
 }
 
 // ------------------------------------------------------------------ prep --
@@ -1034,7 +1289,6 @@ int split_for_tiles(long long tiles, int gu_per_tile, int d_per_tile, int ns_gu,
 }
 
 int g_num_sms[MAX_DEVICES] = {0};
-bool g_attr_small[MAX_DEVICES] = {false}, g_attr_large[MAX_DEVICES] = {false};
 
 }  // namespace
 
@@ -1081,9 +1335,10 @@ cudaError_t launch_ffn_prep(const float *x, const moe_dims_t &d, uint16_t *xb, u
     return cudaLaunchKernelEx(&cfg, ffn_prep_kernel, p);
 }
 
-cudaError_t launch_expert_ffn(const ExpertMaps &maps, const uint16_t *xb, const moe_dims_t &d,
-                              const moe_lists_t &l, float *y, uint16_t *h, const float *wd, Counters *ctr, bool early,
-                              int pub_target, cudaStream_t s) {
+namespace {
+
+// Number of SMs of the current device (cached per device).
+cudaError_t device_sms(int *dev_out, int *sms) {
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
@@ -1094,16 +1349,24 @@ cudaError_t launch_expert_ffn(const ExpertMaps &maps, const uint16_t *xb, const 
         if (err != cudaSuccess) return err;
         g_num_sms[dev] = n;
     }
-    const bool small = d.B <= 16;
-    bool &configured = small ? g_attr_small[dev] : g_attr_large[dev];
-    if (!configured) {
-        err = small ? cudaFuncSetAttribute(expert_ffn_kernel<RingSmallB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           smem_bytes<RingSmallB>())
-                    : cudaFuncSetAttribute(expert_ffn_kernel<RingLargeB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           smem_bytes<RingLargeB>());
-        if (err != cudaSuccess) return err;
-        configured = true;
-    }
+    *dev_out = dev;
+    *sms = g_num_sms[dev];
+    return cudaSuccess;
+}
+
+// Sets the dynamic shared-memory limit of a kernel once per device.
+template <class K>
+cudaError_t configure_smem(K kernel, int bytes, int dev) {
+    static bool done[MAX_DEVICES] = {};
+    if (done[dev]) return cudaSuccess;
+    const cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (err == cudaSuccess) done[dev] = true;
+    return err;
+}
+
+// Expert-stream arguments for dims d, units dealt to `unit_ctas` CTAs.
+ExpertArgs make_expert_args(const uint16_t *xb, const moe_dims_t &d, const moe_lists_t &l, float *y, uint16_t *h,
+                            const float *wd, Counters *ctr, int unit_ctas) {
     ExpertArgs a;
     a.xb = xb;
     a.B = d.B;
@@ -1111,11 +1374,14 @@ cudaError_t launch_expert_ffn(const ExpertMaps &maps, const uint16_t *xb, const 
     a.E = d.E;
     a.k = d.k;
     a.F = d.d_ff;
+    a.wait_ns = wait_limit_ns();
+    a.unit_ctas = unit_ctas;
+    a.lists_flag = nullptr;
     a.dense = d.B <= TN ? 1 : 0;
     a.bpad = (d.B + 7) / 8 * 8;
     a.hrows = expert_ffn_h_rows(d.B);
-    a.early = (early && a.dense) ? 1 : 0;
-    a.pub_target = pub_target;
+    a.early = 0;
+    a.pub_target = 0;
     a.gu_per_tile = d.d_ff / GU_ROWS;
     a.d_per_tile = d.d / D_ROWS;
     {
@@ -1132,12 +1398,11 @@ cudaError_t launch_expert_ffn(const ExpertMaps &maps, const uint16_t *xb, const 
         static std::mutex mu;
         static int key[5] = {-1, -1, -1, -1, -1};
         static unsigned char table[SPLIT_TABLE_MAX + 1];
-        const int grid = early && g_num_sms[dev] > 1 ? g_num_sms[dev] - 1 : g_num_sms[dev];
-        const int k[5] = {a.gu_per_tile, a.d_per_tile, a.ns_gu, a.ns_d, grid};
+        const int k[5] = {a.gu_per_tile, a.d_per_tile, a.ns_gu, a.ns_d, unit_ctas};
         std::lock_guard<std::mutex> lock(mu);
         if (std::memcmp(k, key, sizeof(k)) != 0) {
             for (int t = 0; t <= SPLIT_TABLE_MAX; ++t)
-                table[t] = static_cast<unsigned char>(split_for_tiles(t, k[0], k[1], k[2], k[3], grid));
+                table[t] = static_cast<unsigned char>(split_for_tiles(t, k[0], k[1], k[2], k[3], unit_ctas));
             std::memcpy(key, k, sizeof(k));
         }
         std::memcpy(a.split_for, table, sizeof(table));
@@ -1151,12 +1416,66 @@ cudaError_t launch_expert_ffn(const ExpertMaps &maps, const uint16_t *xb, const 
     a.y = y;
     a.h = h;
     a.ctr = ctr;
+    return a;
+}
+
+// Router items of the fused layer kernel: tokens per item up to 4, experts
+// per item 4 (8 when 4 would give more items than CTAs), both cut back
+// while the staged rows exceed the ring's shared memory.
+LayerArgs make_layer_router(const moe_dims_t &d, int grid, int ring_bytes) {
+    LayerArgs L;
+    const int lines = d.d / 32;
+    L.box_lines = router_box_lines(d.d);
+    L.boxes = (lines + L.box_lines - 1) / L.box_lines;
+    L.row_bytes = (L.boxes * L.box_lines * 128 + 1023) / 1024 * 1024;
+    L.tpb = d.B < GEMV_TPB_MAX ? d.B : GEMV_TPB_MAX;
+    const int n_tg = (d.B + L.tpb - 1) / L.tpb;
+    L.epb = ((d.E + 3) / 4) * n_tg > grid ? NCW : 4;
+    while ((L.epb + L.tpb) * L.row_bytes > ring_bytes) {
+        if (L.epb > 1) --L.epb;
+        else if (L.tpb > 1) --L.tpb;
+        else break;
+    }
+    L.n_eg = (d.E + L.epb - 1) / L.epb;
+    L.n_items = L.n_eg * ((d.B + L.tpb - 1) / L.tpb);
+    return L;
+}
+
+template <class RG, int NI>
+cudaError_t launch_layer_ni(const ExpertMaps &maps, const RouterMaps &rmaps, const ExpertArgs &a,
+                            const LayerArgs &L, int grid, int dev, cudaStream_t s) {
+    cudaError_t err = configure_smem(layer_kernel<RG, NI>, smem_bytes<RG>(), dev);
+    if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
-    // early mode: one SM stays with the selection kernel, which runs beside
-    // this grid; the router blocks exit before the activated set is
-    // published, so all CTAs of this grid are resident when streaming starts
-    // (the round-robin deal assumes they start together)
-    cfg.gridDim = dim3(early && g_num_sms[dev] > 1 ? g_num_sms[dev] - 1 : g_num_sms[dev]);
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(NTHREADS);
+    cfg.dynamicSmemBytes = smem_bytes<RG>();
+    cfg.stream = s;
+    // every CTA must be resident: the CTAs wait for one another at the
+    // grid barrier
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, layer_kernel<RG, NI>, maps, rmaps, a, L);
+}
+
+}  // namespace
+
+cudaError_t launch_expert_ffn(const ExpertMaps &maps, const uint16_t *xb, const moe_dims_t &d,
+                              const moe_lists_t &l, float *y, uint16_t *h, const float *wd, Counters *ctr,
+                              cudaStream_t s) {
+    int dev = 0, sms = 0;
+    cudaError_t err = device_sms(&dev, &sms);
+    if (err != cudaSuccess) return err;
+    const bool small = d.B <= 16;
+    err = small ? configure_smem(expert_ffn_kernel<RingSmallB>, smem_bytes<RingSmallB>(), dev)
+                : configure_smem(expert_ffn_kernel<RingLargeB>, smem_bytes<RingLargeB>(), dev);
+    if (err != cudaSuccess) return err;
+    const ExpertArgs a = make_expert_args(xb, d, l, y, h, wd, ctr, sms);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(sms);
     cfg.blockDim = dim3(NTHREADS);
     cfg.dynamicSmemBytes = small ? smem_bytes<RingSmallB>() : smem_bytes<RingLargeB>();
     cfg.stream = s;
@@ -1167,6 +1486,48 @@ cudaError_t launch_expert_ffn(const ExpertMaps &maps, const uint16_t *xb, const 
     cfg.numAttrs = 1;  // always chained to the previous kernel with programmatic dependent launch
     return small ? cudaLaunchKernelEx(&cfg, expert_ffn_kernel<RingSmallB>, maps, a)
                  : cudaLaunchKernelEx(&cfg, expert_ffn_kernel<RingLargeB>, maps, a);
+}
+
+cudaError_t launch_layer_fused(const ExpertMaps &maps, const RouterMaps &rmaps, const moe_dims_t &d,
+                               const moe_reselect_t &rule, const float *x, const float *bias, float *logits,
+                               float *probs, uint16_t *xb, float *y, uint16_t *h, float *wd, int32_t *sel_idx,
+                               float *sel_w, const moe_lists_t &lists, int32_t *n_active_copy, Counters *ctr,
+                               cudaStream_t s) {
+    if (d.B > TN) return cudaErrorInvalidValue;
+    int dev = 0, sms = 0;
+    cudaError_t err = device_sms(&dev, &sms);
+    if (err != cudaSuccess) return err;
+    if (sms < 2) return cudaErrorInvalidConfiguration;
+    const bool small = d.B <= 16;
+    // the last CTA runs the selection; the others stream the experts
+    ExpertArgs a = make_expert_args(xb, d, lists, y, h, wd, ctr, sms - 1);
+    a.early = 1;
+    a.lists_flag = &ctr->lists_ready;
+    const bool batch_rule = rule.mode == MOE_RESELECT_XSHARE || rule.mode == MOE_RESELECT_AFFINITY ||
+                            rule.mode == MOE_RESELECT_XSHARE_HIER;
+    a.pub_target = 1;
+    const int ring = small ? RingSmallB::STAGES * RingSmallB::SLOT_BYTES : RingLargeB::STAGES * RingLargeB::SLOT_BYTES;
+    LayerArgs L = make_layer_router(d, sms, ring);
+    L.x = x;
+    L.bias = bias;
+    L.logits = logits;
+    L.r1 = rule.mode == MOE_RESELECT_OEA ? rule.k0 : (rule.mode == MOE_RESELECT_NONE ? d.k : 0);
+    L.sel = make_reselect_args(logits, probs, true, d, rule, sel_idx, sel_w, lists, n_active_copy);
+    L.sel.ctr = ctr;
+    L.sel.wd = wd;
+    L.sel.publish_set = batch_rule ? 1 : 0;
+    const size_t sel_smem = reselect_smem(d, rule, &L.sel.cache_rows);
+    if (sel_smem > static_cast<size_t>(ring)) return cudaErrorInvalidValue;
+    switch (ni_for(d.E)) {
+        case 1: return small ? launch_layer_ni<RingSmallB, 1>(maps, rmaps, a, L, sms, dev, s)
+                             : launch_layer_ni<RingLargeB, 1>(maps, rmaps, a, L, sms, dev, s);
+        case 2: return small ? launch_layer_ni<RingSmallB, 2>(maps, rmaps, a, L, sms, dev, s)
+                             : launch_layer_ni<RingLargeB, 2>(maps, rmaps, a, L, sms, dev, s);
+        case 4: return small ? launch_layer_ni<RingSmallB, 4>(maps, rmaps, a, L, sms, dev, s)
+                             : launch_layer_ni<RingLargeB, 4>(maps, rmaps, a, L, sms, dev, s);
+        default: return small ? launch_layer_ni<RingSmallB, 8>(maps, rmaps, a, L, sms, dev, s)
+                              : launch_layer_ni<RingLargeB, 8>(maps, rmaps, a, L, sms, dev, s);
+    }
 }
 
 }  // namespace moe

@@ -18,14 +18,10 @@ constexpr int D_MIN = 64, D_MAX = 16384;
 constexpr int F_MIN = 64, F_MAX = 8192;
 
 // Counters the kernels share inside one workspace.  They are zero between
-// calls: each user puts back what it changed (the router's last block of a
-// token group its count, the router's last group the batch-wide rules'
-// contributions; the expert kernel's last CTA everything else).
+// calls: the last CTA of the expert stream puts them back.
 // One published copy of the activated set, alone in a 128-byte line.
 struct PubLine {
-    int32_t pub;                // token groups whose first ranks are in `mask`
-                                // (+1 once the router's last group has added
-                                // a batch-wide rule's set)
+    int32_t pub;                // 1 once `mask` holds the activated set
     int32_t pad0[3];
     uint32_t mask[E_MAX / 32];  // the activated set, one bit per expert
     int32_t pad1[20];
@@ -37,19 +33,11 @@ constexpr int PUB_COPIES = 8;  // expert-kernel CTA c polls copy c % PUB_COPIES
 struct Counters {
     int32_t error;     // first error code a kernel recorded (0 = none)
     int32_t k3_exit;   // expert-kernel CTAs finished
-    int32_t pad0[30];
-    PubLine pubs[PUB_COPIES];   // layer path: the activated set, in copies
-    int32_t grp_done[B_MAX];    // router blocks finished, per token group
+    int32_t arrive;    // fused layer kernel: CTAs past the router (grid barrier)
+    int32_t lists_ready;  // fused layer kernel: the selection CTA has written the lists
+    int32_t pad0[28];
+    PubLine pubs[PUB_COPIES];   // fused layer kernel, batch-wide rules: the activated set
     int32_t gu_done[E_MAX];     // finished gate/up units per active-expert slot
-    // Batch-wide rules published by the router (XShare, hierarchical XShare,
-    // affinity binning; B <= 32): each token group's contributions, cleared
-    // by the last group
-    int32_t grp_final;                 // token groups whose contributions are in
-    uint32_t ubase_bits[E_MAX / 32];   // union of the top-k sets
-    uint32_t r0_bits[E_MAX / 32];      // every token's rank-0 expert
-    int32_t pad2[15];
-    uint32_t memb[E_MAX];              // XShare rules: tokens (bit b) whose top-k holds the expert
-    unsigned long long aff_score[E_MAX];  // affinity binning: sum of 2^bin
 };
 static_assert(sizeof(Counters) % 16 == 0, "Counters must keep 16-byte alignment");
 
@@ -108,22 +96,14 @@ cudaError_t launch_route_topk(const float *logits, const moe_dims_t &d, float *p
 cudaError_t launch_reselect(const float *logits, const float *probs, const moe_dims_t &d,
                             const moe_reselect_t &r, int32_t *sel_idx, float *sel_w,
                             const moe_lists_t &l, cudaStream_t s);
-// Layer path, first kernel: router GEMV; also writes x in bf16, zeroes y
-// and, with `early` (B <= 32), publishes the activated set in ctr->pubs for
-// the expert kernel started early (every rule: OEA and no re-selection per
-// token group, the batch-wide rules once all groups are in).
+// Layer path above 32 tokens, first kernel: router GEMV; also zeroes y.
 cudaError_t launch_layer_route(const RouterMaps &maps, const float *x, const float *bias, const moe_dims_t &d,
-                               const moe_reselect_t &rule, float *logits, float *probs, uint16_t *xb, float *y,
-                               Counters *ctr, bool early, cudaStream_t s);
-// Layer path, second kernel (chained with programmatic dependent launch):
-// softmax, selection, lists, and `wd` (B <= 32) the dense weights.  With
-// `early` the next kernel may launch at once.
+                               float *logits, float *y, Counters *ctr, cudaStream_t s);
+// Layer path above 32 tokens, second kernel (chained with programmatic
+// dependent launch): softmax, selection, lists.
 cudaError_t launch_layer_select(const float *logits, float *probs, const moe_dims_t &d, const moe_reselect_t &rule,
                                 int32_t *sel_idx, float *sel_w, const moe_lists_t &l, int32_t *n_active_copy,
-                                Counters *ctr, float *wd, bool early, cudaStream_t s);
-// Value of every ctr->pubs[c].pub once the activated set of a layer call is
-// published.
-int layer_pub_target(const moe_dims_t &d, const moe_reselect_t &rule);
+                                cudaStream_t s);
 // Input preparation of the expert kernel (all pointers may be null, each
 // step is skipped then): x -> bf16 (xb, dense mode), each pair's x row ->
 // xd (larger batches), y = 0, gate/up counts cleared and, for B <= 32, the
@@ -138,13 +118,23 @@ cudaError_t launch_ffn_prep(const float *x, const moe_dims_t &d, uint16_t *xb, u
 struct ExpertMaps {
     CUtensorMap gate, up, down, h, x;
 };
-// early (layer path, B <= 32): start when ctr->pubs[c].pub reaches
-// pub_target and take the activated set from its mask, instead of waiting for the
-// previous kernel; wd: dense weights (B <= 32).
-cudaError_t launch_expert_ffn(const ExpertMaps &maps, const uint16_t *xb,
-                              const moe_dims_t &d, const moe_lists_t &l, float *y,
-                              uint16_t *h, const float *wd, Counters *ctr, bool early, int pub_target,
+// The expert kernel alone (moe_expert_ffn): lists from the previous kernel
+// (chained with programmatic dependent launch) or the caller; wd: dense
+// weights (B <= 32).
+cudaError_t launch_expert_ffn(const ExpertMaps &maps, const uint16_t *xb, const moe_dims_t &d,
+                              const moe_lists_t &l, float *y, uint16_t *h, const float *wd, Counters *ctr,
                               cudaStream_t s);
+// The whole layer in one cooperative persistent kernel (B <= 32): router,
+// grid barrier, selection (last CTA), expert stream (the other CTAs).  xb:
+// x in bf16 (written), h: the SwiGLU scratch, wd: the dense weights.
+cudaError_t launch_layer_fused(const ExpertMaps &maps, const RouterMaps &rmaps, const moe_dims_t &d,
+                               const moe_reselect_t &rule, const float *x, const float *bias, float *logits,
+                               float *probs, uint16_t *xb, float *y, uint16_t *h, float *wd, int32_t *sel_idx,
+                               float *sel_w, const moe_lists_t &lists, int32_t *n_active_copy, Counters *ctr,
+                               cudaStream_t s);
+// Limit of every bounded wait inside the kernels launched from now on
+// (nanoseconds; moe_set_wait_limit_ns).
+unsigned long long wait_limit_ns();
 int expert_ffn_h_rows(int B);         // rows of one H box
 int expert_ffn_dense_batch(int B);    // 1 if gate/up stages load all B token rows at once
 int expert_ffn_gu_rows();             // rows of Wgate / Wup per gate-up unit

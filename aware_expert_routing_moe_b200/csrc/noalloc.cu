@@ -109,6 +109,6 @@ extern "C" moe_status_t moe_expert_ffn_noalloc(const float *x, const uint16_t *W
     if (launch_ffn_prep(x, dims, dense ? xk : nullptr, dense ? nullptr : xk, y, ctr, lists, wd, false, s) !=
         cudaSuccess)
         return MOE_ERR_CUDA;
-    if (launch_expert_ffn(maps, xk, dims, lists, y, h, wd, ctr, false, 0, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_expert_ffn(maps, xk, dims, lists, y, h, wd, ctr, s) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;
 }

@@ -14,7 +14,9 @@ every call.
 
 Printed (rank 0, one JSON line): value = algorithmic bytes of all ranks per
 second (activated experts x 3 d d_ff x 2 B + router weights + x + y), the
-roofline of the expert kernel (events around moe_expert_ffn), the oracle
+roofline of the dominant kernel (up to 32 tokens the fused layer kernel,
+which is the whole call; above, the expert kernel, timed with events
+around moe_expert_ffn), the oracle
 timed on the host cores (cpu_baseline), an end-to-end number through the
 Python API with host buffers (e2e), and the SM clocks sampled with NVML
 during the timed region.
@@ -66,7 +68,7 @@ WORKLOADS = {
 # capture of the same workload (profiles/expert_ffn_kernel_q30b_b16_oea4.md);
 # a workload without an entry reports null.  Entries are dropped whenever
 # the kernel changes.
-NCU_TRAFFIC = {"q30b_b16_oea4": 146014464}  # 141.83 MB read + 4.18 MB written
+NCU_TRAFFIC = {}
 
 
 def workload_desc(w: dict) -> str:
@@ -144,7 +146,7 @@ class ClockSampler:
                 self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
             except Exception:
                 pass
-            time.sleep(0.002)
+            time.sleep(0.001)
 
     def __enter__(self):
         if self._nv is not None:
@@ -305,13 +307,15 @@ def run_ours(args, w, rank, world, local_rank):
         barrier()
         return max_over_ranks(e0.elapsed_time(e1), world, dev)  # ms, all steps
 
-    # ---- main timed region: K graph-replayed layer calls
+    # ---- main timed region: K graph-replayed layer calls.  The clock
+    # sampler runs from the warm-up through the last leg below, so that a
+    # short timed region still gets a clock record of several samples; the
+    # GPU is busy with the same kernels throughout.
+    sampler = ClockSampler(local_rank)
+    sampler.__enter__()
     with torch.cuda.stream(s):
         replay(args.warmup)
-    sampler = ClockSampler(local_rank)
-    with sampler:
-        ms_total = timed(replay, args.steps)
-    clocks = sampler.summary()
+    ms_total = timed(replay, args.steps)
     ms_step = ms_total / args.steps
     value = aggregate_gbs(total_bytes, world, ms_step)
 
@@ -340,11 +344,25 @@ def run_ours(args, w, rank, world, local_rank):
     ms_ffn = timed(lambda n: [g_ffn.replay() for _ in range(n)], nrep) / (nrep * ROTATE)
     hbm_peak, peak_kind = measured_peaks()
     ffn_gbs = ffn_bytes / (ms_ffn * 1e-3) / 1e9
-    roofline = {"bound": "hbm", "achieved": ffn_gbs, "peak": hbm_peak, "unit": "GB/s",
-                "frac": ffn_gbs / hbm_peak, "traffic": NCU_TRAFFIC.get(args.workload),
-                "kernel": "moe_expert_ffn (input prep + grouped SwiGLU expert kernel)",
-                "peak_source": f"{peak_kind} HBM copy bandwidth",
-                "frac_of_nominal_8tbs": ffn_gbs / NOMINAL_HBM_GBS}
+    layer_gbs = total_bytes / (ms_step * 1e-3) / 1e9
+    if B <= 32:
+        # one kernel per call: the fused layer kernel is the dominant kernel,
+        # timed by the main region itself
+        roofline = {"bound": "hbm", "achieved": layer_gbs, "peak": hbm_peak, "unit": "GB/s",
+                    "frac": layer_gbs / hbm_peak, "traffic": NCU_TRAFFIC.get(args.workload),
+                    "kernel": "layer_kernel (router, grid barrier, selection, expert stream)",
+                    "bytes_per_launch": total_bytes, "us_per_launch": ms_step * 1e3,
+                    "peak_source": f"{peak_kind} HBM copy bandwidth",
+                    "frac_of_nominal_8tbs": layer_gbs / NOMINAL_HBM_GBS}
+    else:
+        roofline = {"bound": "hbm", "achieved": ffn_gbs, "peak": hbm_peak, "unit": "GB/s",
+                    "frac": ffn_gbs / hbm_peak, "traffic": NCU_TRAFFIC.get(args.workload),
+                    "kernel": "moe_expert_ffn (input prep + grouped SwiGLU expert kernel)",
+                    "bytes_per_launch": ffn_bytes, "us_per_launch": ms_ffn * 1e3,
+                    "peak_source": f"{peak_kind} HBM copy bandwidth",
+                    "frac_of_nominal_8tbs": ffn_gbs / NOMINAL_HBM_GBS}
+    expert_leg = {"kernel": "moe_expert_ffn (input prep + expert kernel, lists given)", "achieved": ffn_gbs,
+                  "unit": "GB/s", "frac": ffn_gbs / hbm_peak, "us_per_call": ms_ffn * 1e3}
 
     # ---- end to end through the Python API with pinned host buffers
     x_host = torch.from_numpy(x_np).pin_memory()
@@ -365,6 +383,9 @@ def run_ours(args, w, rank, world, local_rank):
     e2e = {"value": aggregate_gbs(total_bytes, world, ms_e2e), "unit": UNIT,
            "h2d_bytes_per_step": B * S.d * 4, "d2h_bytes_per_step": B * S.d * 4,
            "ms_per_step": ms_e2e}
+    sampler.__exit__(None, None, None)
+    clocks = sampler.summary()
+    clocks["window"] = "warm-up, timed region, launch-overhead, expert-kernel and end-to-end legs"
     if moe.moe_check_error(ws, s) != 0:
         raise RuntimeError("device error word set during the benchmark")
 
@@ -380,16 +401,18 @@ def run_ours(args, w, rank, world, local_rank):
                    "parallelism": f"replicas x{world}",
                    "l2": f"inputs larger than L2: {ROTATE} rotating copies of the layer weights "
                          f"({3 * S.E * S.d * S.F * 2 / 1e9:.2f} GB of experts + the router each)",
-                   "launch": "CUDA graph of 4 layer calls, PDL between the 3 kernels of a call"},
+                   "launch": ("CUDA graph of 4 layer calls, one cooperative kernel per call" if B <= 32 else
+                              "CUDA graph of 4 layer calls, 4 kernels per call chained with PDL")},
         "us_per_call": ms_step * 1e3,
         "frac_of_nominal_8tbs": (total_bytes / (ms_step * 1e-3) / 1e9) / NOMINAL_HBM_GBS,
         "frac_of_measured_hbm": (total_bytes / (ms_step * 1e-3) / 1e9) / hbm_peak,
         "stream_launch_us_per_call": ms_stream * 1e3,
         "roofline": roofline,
+        "expert_ffn_leg": expert_leg,
         "e2e": e2e,
-        # router, selection and expert kernels; batches above 32 tokens add
-        # the kernel that dispatches each pair's x row
-        "gpu_launches": (3 if B <= 32 else 4) * args.steps,
+        # up to 32 tokens one fused kernel per call; above, router,
+        # selection, x dispatch and expert kernels
+        "gpu_launches": (1 if B <= 32 else 4) * args.steps,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

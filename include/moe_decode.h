@@ -149,6 +149,17 @@ moe_status_t moe_route(const float *x, const float *Wg, const float *bias,
                        int32_t *topk_idx, float *topk_w, void *stream);
 
 /* Batch-aware re-selection + per-expert token lists.
+ * The rules follow "Opportunistic Expert Activation: Batch-Aware Expert
+ * Routing for Faster Decode Without Retraining" (abstract: a token keeps
+ * its most important experts and reuses experts the batch already loads),
+ * "XShare: Collaborative in-Batch Expert Sharing for Faster MoE Inference"
+ * (abstract: batch selection as a modular objective solved greedily, and
+ * its hierarchical form for speculative decoding) and "Lynx: Enabling
+ * Efficient MoE Inference through Dynamic Batch-Aware Expert Selection"
+ * (sections 2.1-2.2: confidence bins, critical experts, remapping); the
+ * pages give no formulas, so the precise rules below are this library's
+ * reading.  The lists are the expert-major dispatch the Lynx page's
+ * remapper hands to the experts (section 2.3).
  *   logits[B][E], probs[B][E] fp32 (device; as produced by moe_route);
  *   outputs (device): sel_idx[B][k] int32 (chosen experts in rank order,
  *   -1 in unused slots), sel_w[B][k] fp32 (gate weights renormalised over
@@ -172,7 +183,14 @@ moe_status_t moe_reselect(const float *logits, const float *probs,
                           int32_t *sel_idx, float *sel_w, moe_lists_t lists,
                           void *stream);
 
-/* Grouped SwiGLU expert FFN with the weighted combine.
+/* Grouped SwiGLU expert FFN with the weighted combine: every activated
+ * expert's weights are streamed from HBM once per call, which is what decode
+ * latency follows ("Lynx: Enabling Efficient MoE Inference through Dynamic
+ * Batch-Aware Expert Selection", section 1; "Opportunistic Expert
+ * Activation: Batch-Aware Expert Routing for Faster Decode Without
+ * Retraining", abstract: decode is memory-bound and its MoE latency grows
+ * with the number of activated experts).  SwiGLU is the expert type of the
+ * Qwen3 MoE models the OEA page evaluates; the pages do not restate it.
  *   x[B][d] fp32; Wgate[E][d_ff][d], Wup[E][d_ff][d], Wdown[E][d][d_ff]
  *   bf16 bits (device; nn.Linear out x in layout); lists as written by
  *   moe_reselect (device, read only);
@@ -190,7 +208,13 @@ moe_status_t moe_expert_ffn(const float *x, const uint16_t *Wgate,
 
 /* The whole layer: moe_route -> moe_reselect -> moe_expert_ffn, chained on
  * the device with no host round trip (the activated-expert count never
- * leaves the GPU).  Arguments as above; y[B][d] is overwritten.
+ * leaves the GPU): the re-routing step sits between the router and the
+ * experts and intercepts the router's output ("Lynx: Enabling Efficient MoE
+ * Inference through Dynamic Batch-Aware Expert Selection", section 2.2).
+ * Up to 32 tokens the call is one persistent kernel (router, a grid-wide
+ * barrier, selection and expert stream); above, four kernels chained with
+ * programmatic dependent launch.  Arguments as above; y[B][d] is
+ * overwritten.
  * sel_idx[B][k], sel_w[B][k] and n_active[1] are optional device outputs
  * (NULL = not returned).  ws: device workspace of at least
  * moe_workspace_bytes(dims) bytes. */
@@ -240,6 +264,19 @@ moe_status_t moe_expert_ffn_noalloc(const float *x, const uint16_t *Wgate,
                                     const uint16_t *Wup, const uint16_t *Wdown,
                                     moe_dims_t dims, moe_lists_t lists, float *y,
                                     void *stream);
+
+/* Limit of every bounded wait inside the library's kernels, for kernels
+ * launched after this call (process-wide; 0 restores the default of 1 s).
+ * A kernel waits on other CTAs (the fused layer kernel's grid barrier and
+ * its flags), on its own copies and on the previous kernel's results; when
+ * a wait runs past the limit the CTA records an error code in the
+ * workspace (reported by moe_check_error as MOE_ERR_INTERNAL), lets the
+ * copies already in flight into its shared memory land (up to a further
+ * 1 s), and ends its share of the call, so that the device stays usable.
+ * A limit shorter than the work it waits for makes calls fail on purpose
+ * (a diagnostic of the error path); the default never expires in normal
+ * operation. */
+void moe_set_wait_limit_ns(uint64_t ns);
 
 /* Synchronises `stream`, then reads and clears the error word that kernels
  * of earlier calls using this workspace may have set (a bounded wait that

@@ -110,3 +110,42 @@ def test_token_outside_batch_is_skipped_and_reported(name, B, k0):
     w2[t_bad, slot] = 0.0
     y_r = oracle.ffn(x, L["Wgate"], L["Wup"], L["Wdown"], sel, w2, threads=THREADS)
     assert_close_y(y.cpu().numpy(), y_r, "bad token skipped")
+
+
+# ------------------------------------------------------------ bounded waits --
+@pytest.mark.parametrize("path", ["layer_fused", "expert_ffn", "layer_tiled"])
+def test_bounded_waits_expire_and_report(path):
+    # With a 200 ns limit every wait on a copy, on another CTA or on a flag
+    # runs out: each CTA records the error, lets its copies in flight land,
+    # ends its share of the call and exits; the call completes and
+    # moe_check_error reports MOE_ERR_INTERNAL.  After the default limit is
+    # restored and the workspace zeroed, the same call matches the oracle.
+    name, B = ("q30b", 16) if path != "layer_tiled" else ("q30b", 64)
+    S = shape(name)
+    L = host_layer(name, 0)
+    D = device_layer(name, 0)
+    x = ms.make_tokens(S, B, 0)
+    xd = torch.from_numpy(x).cuda()
+    ws = moe.new_workspace(B, S.d, S.E, S.k, S.F)
+    logits, probs, _, _ = oracle.route(x, L["Wg"], L["bias"], S.k)
+    sel, w = oracle.reselect(logits, probs, S.k, OEA, 4, 0)
+    li = oracle.lists(sel, w, S.E)
+
+    def call():
+        if path == "expert_ffn":
+            y = moe.moe_expert_ffn(xd, D["Wgate"], D["Wup"], D["Wdown"], _device_lists(li, S.E, B, S.k), S.k, ws)
+        else:
+            y = moe.moe_layer_decode(xd, D["Wg"], D["bias"], D["Wgate"], D["Wup"], D["Wdown"], S.k, OEA, 4, ws=ws)
+        return y, moe.moe_check_error(ws)
+
+    moe.moe_set_wait_limit_ns(200)
+    try:
+        _, status = call()
+    finally:
+        moe.moe_set_wait_limit_ns(0)
+    assert status == MOE_ERR_INTERNAL
+    ws.zero_()
+    y, status = call()
+    assert status == 0
+    y_r = oracle.ffn(x, L["Wgate"], L["Wup"], L["Wdown"], sel, w, threads=THREADS)
+    assert_close_y(y.cpu().numpy(), y_r, f"{path} after expired waits")
