@@ -23,7 +23,8 @@ __all__ = [
     "Dims", "Rule", "Lists", "load_library", "library_path", "moe_workspace_bytes",
     "moe_status_string", "moe_route", "moe_reselect", "moe_expert_ffn", "moe_layer_decode",
     "moe_check_error", "moe_expert_ffn_noalloc", "new_workspace", "alloc_lists", "ABI_SYMBOLS",
-    "NOALLOC_SCRATCH_BYTES", "moe_set_wait_limit_ns",
+    "NOALLOC_SCRATCH_BYTES", "moe_set_wait_limit_ns", "moe_decode_stack", "LayerWeights",
+    "MOE_PHASE_DECODE", "MOE_PHASE_PREFILL",
 ]
 
 MOE_RESELECT_NONE, MOE_RESELECT_OEA, MOE_RESELECT_XSHARE = 0, 1, 2
@@ -32,7 +33,7 @@ STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_MISALIGNED", 3: "MO
           4: "MOE_ERR_UNSUPPORTED", 5: "MOE_ERR_CUDA", 6: "MOE_ERR_INTERNAL"}
 ABI_SYMBOLS = ("moe_workspace_bytes", "moe_route", "moe_reselect", "moe_expert_ffn",
                "moe_layer_decode", "moe_expert_ffn_noalloc", "moe_check_error", "moe_status_string",
-               "moe_set_wait_limit_ns")
+               "moe_set_wait_limit_ns", "moe_decode_stack")
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -54,6 +55,11 @@ class Dims(ctypes.Structure):
 class Rule(ctypes.Structure):
     _fields_ = [("mode", ctypes.c_int32), ("k0", ctypes.c_int32), ("budget", ctypes.c_int32),
                 ("group", ctypes.c_int32)]
+
+
+class LayerWeights(ctypes.Structure):
+    _fields_ = [("Wg", ctypes.c_void_p), ("bias", ctypes.c_void_p), ("Wgate", ctypes.c_void_p),
+                ("Wup", ctypes.c_void_p), ("Wdown", ctypes.c_void_p)]
 
 
 class Lists(ctypes.Structure):
@@ -89,6 +95,9 @@ def load_library() -> ctypes.CDLL:
         lib.moe_expert_ffn_noalloc.argtypes = [P, P, P, P, Dims, Lists, P, P]
         lib.moe_check_error.restype = ctypes.c_int
         lib.moe_check_error.argtypes = [P, S, P]
+        lib.moe_decode_stack.restype = ctypes.c_int
+        lib.moe_decode_stack.argtypes = [ctypes.POINTER(LayerWeights), ctypes.c_int32, Dims, Rule, ctypes.c_int32,
+                                         P, P, P, P, S, P]
         lib.moe_set_wait_limit_ns.restype = None
         lib.moe_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
         _lib = lib
@@ -212,6 +221,30 @@ def moe_layer_decode(x, Wg, bias, Wgate, Wup, Wdown, k: int, mode: int, k0: int 
         ws.numel() * ws.element_size(), _stream(stream))
     _check(st, "moe_layer_decode")
     return y
+
+
+MOE_PHASE_DECODE, MOE_PHASE_PREFILL = 0, 1
+
+
+def moe_decode_stack(xs, layers, k: int, mode: int, k0: int = 0, budget: int = 0, phase: int = MOE_PHASE_DECODE,
+                     ws=None, sel_idx=None, n_active=None, stream=None, group: int = 1):
+    """n_layers residual MoE layers: xs[l + 1] = xs[l] + layer_l(xs[l]).
+    ``xs``: [n_layers + 1][B][d] fp32 device tensor, xs[0] the input;
+    ``layers``: list of (Wg, bias, Wgate, Wup, Wdown) device tensors.
+    Optional device outputs sel_idx[n_layers][B][k], n_active[n_layers].
+    -> xs."""
+    n = len(layers)
+    _, B, d = xs.shape
+    E, F, _ = layers[0][2].shape
+    if ws is None:
+        ws = new_workspace(B, d, E, k, F, xs.device)
+    arr = (LayerWeights * n)(*[LayerWeights(_ptr(Wg), _ptr(bias), _ptr(g), _ptr(u), _ptr(dn))
+                               for (Wg, bias, g, u, dn) in layers])
+    st = load_library().moe_decode_stack(arr, n, Dims(B, d, E, k, F), Rule(mode, k0, budget, group), int(phase),
+                                         _ptr(xs), _ptr(sel_idx), _ptr(n_active), _ptr(ws),
+                                         ws.numel() * ws.element_size(), _stream(stream))
+    _check(st, "moe_decode_stack")
+    return xs
 
 
 def moe_expert_ffn_noalloc(x, Wgate, Wup, Wdown, lists: dict, k: int, y=None, stream=None):

@@ -157,6 +157,13 @@ moe_lists_t ws_lists(void *ws, const WsLayout &L) {
     return l;
 }
 
+// One layer call (arguments validated): up to 32 tokens the fused kernel,
+// above the four chained kernels.  residual: y = x + the experts' output;
+// chained: the layer follows the previous layer of a stack on the stream.
+moe_status_t layer_call(const float *x, const moe_layer_weights_t &w, const moe_dims_t &dims,
+                        const moe_reselect_t &rule, float *y, int32_t *sel_idx, float *sel_w, int32_t *n_active,
+                        void *ws, cudaStream_t s, bool residual, bool chained);
+
 }  // namespace
 
 bool encode_expert_maps(ExpertMaps *m, const moe_dims_t &d, const uint16_t *Wgate, const uint16_t *Wup,
@@ -207,6 +214,45 @@ WsLayout ws_layout(const moe_dims_t &d) {
     L.total = o;
     return L;
 }
+
+namespace {
+
+moe_status_t layer_call(const float *x, const moe_layer_weights_t &w, const moe_dims_t &dims,
+                        const moe_reselect_t &rule, float *y, int32_t *sel_idx, float *sel_w, int32_t *n_active,
+                        void *ws, cudaStream_t s, bool residual, bool chained) {
+    const WsLayout L = ws_layout(dims);
+    const bool dense = expert_ffn_dense_batch(dims.B) != 0;
+    // the expert kernel's x: bf16 x (B <= 32) or the dispatched pair rows
+    uint16_t *xk = dense ? seg<uint16_t>(ws, L.xb) : seg<uint16_t>(ws, L.xd);
+    ExpertMaps maps;
+    if (!encode_expert_maps(&maps, dims, w.Wgate, w.Wup, w.Wdown, seg<uint16_t>(ws, L.h), xk)) return MOE_ERR_CUDA;
+    RouterMaps rmaps;
+    if (!encode_router_maps(&rmaps, dims, x, w.Wg)) return MOE_ERR_CUDA;
+    Counters *ctr = seg<Counters>(ws, L.counters);
+    float *logits = seg<float>(ws, L.logits);
+    float *probs = seg<float>(ws, L.probs);
+    int32_t *si = sel_idx ? sel_idx : seg<int32_t>(ws, L.sel_idx);
+    float *sw = sel_w ? sel_w : seg<float>(ws, L.sel_w);
+    const moe_lists_t lists = ws_lists(ws, L);
+    if (dense) {
+        // B <= 32: one persistent kernel for the whole call
+        return from_cuda(launch_layer_fused(maps, rmaps, dims, rule, x, w.bias, logits, probs, xk, y,
+                                            seg<uint16_t>(ws, L.h), seg<float>(ws, L.wd), si, sw, lists, n_active,
+                                            ctr, residual, chained, s));
+    }
+    // larger batches: router, selection (lists), the dispatch of each
+    // pair's x row, then the expert kernel, chained with programmatic
+    // dependent launch
+    moe_status_t st = from_cuda(launch_layer_route(rmaps, x, w.bias, dims, logits, y, ctr, residual, chained, s));
+    if (st != MOE_OK) return st;
+    st = from_cuda(launch_layer_select(logits, probs, dims, rule, si, sw, lists, n_active, s));
+    if (st != MOE_OK) return st;
+    st = from_cuda(launch_ffn_prep(x, dims, nullptr, xk, nullptr, nullptr, lists, nullptr, true, s));
+    if (st != MOE_OK) return st;
+    return from_cuda(launch_expert_ffn(maps, xk, dims, lists, y, seg<uint16_t>(ws, L.h), nullptr, ctr, s));
+}
+
+}  // namespace
 
 }  // namespace moe
 
@@ -301,37 +347,39 @@ moe_status_t moe_layer_decode(const float *x, const float *Wg, const float *bias
     if (st != MOE_OK) return st;
     st = check_device();
     if (st != MOE_OK) return st;
-    const WsLayout L = ws_layout(dims);
-    const bool dense = expert_ffn_dense_batch(dims.B) != 0;
-    // the expert kernel's x: bf16 x (B <= 32) or the dispatched pair rows
-    uint16_t *xk = dense ? seg<uint16_t>(ws, L.xb) : seg<uint16_t>(ws, L.xd);
-    ExpertMaps maps;
-    if (!encode_expert_maps(&maps, dims, Wgate, Wup, Wdown, seg<uint16_t>(ws, L.h), xk)) return MOE_ERR_CUDA;
-    RouterMaps rmaps;
-    if (!encode_router_maps(&rmaps, dims, x, Wg)) return MOE_ERR_CUDA;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    Counters *ctr = seg<Counters>(ws, L.counters);
-    float *logits = seg<float>(ws, L.logits);
-    float *probs = seg<float>(ws, L.probs);
-    int32_t *si = sel_idx ? sel_idx : seg<int32_t>(ws, L.sel_idx);
-    float *sw = sel_w ? sel_w : seg<float>(ws, L.sel_w);
-    const moe_lists_t lists = ws_lists(ws, L);
-    if (dense) {
-        // B <= 32: one persistent kernel for the whole call
-        return from_cuda(launch_layer_fused(maps, rmaps, dims, rule, x, bias, logits, probs, xk, y,
-                                            seg<uint16_t>(ws, L.h), seg<float>(ws, L.wd), si, sw, lists, n_active,
-                                            ctr, s));
+    const moe_layer_weights_t w = {Wg, bias, Wgate, Wup, Wdown};
+    return layer_call(x, w, dims, rule, y, sel_idx, sel_w, n_active, ws, static_cast<cudaStream_t>(stream), false,
+                      false);
+}
+
+moe_status_t moe_decode_stack(const moe_layer_weights_t *layers, int32_t n_layers, moe_dims_t dims,
+                              moe_reselect_t rule, int32_t phase, float *xs, int32_t *sel_idx, int32_t *n_active,
+                              void *ws, size_t ws_bytes, void *stream) {
+    if (!layers || n_layers < 1 || n_layers > MOE_STACK_MAX_LAYERS || !xs) return MOE_ERR_INVALID_ARG;
+    if (phase != MOE_PHASE_DECODE && phase != MOE_PHASE_PREFILL) return MOE_ERR_INVALID_ARG;
+    // prefill bypasses the re-selection: standard top-k routing
+    const moe_reselect_t r = phase == MOE_PHASE_PREFILL ? moe_reselect_t{MOE_RESELECT_NONE, 0, 0, 1} : rule;
+    if (!dims_ok(dims) || !rule_ok(dims, r)) return MOE_ERR_INVALID_ARG;
+    if (!al16(xs) || (sel_idx && !al16(sel_idx)) || (n_active && !al16(n_active))) return MOE_ERR_MISALIGNED;
+    for (int32_t l = 0; l < n_layers; ++l) {
+        const moe_layer_weights_t &w = layers[l];
+        if (!w.Wg || !w.Wgate || !w.Wup || !w.Wdown) return MOE_ERR_INVALID_ARG;
+        if (!al16(w.Wg) || (w.bias && !al16(w.bias)) || !al16(w.Wgate) || !al16(w.Wup) || !al16(w.Wdown))
+            return MOE_ERR_MISALIGNED;
     }
-    // larger batches: router, selection (lists), the dispatch of each
-    // pair's x row, then the expert kernel, chained with programmatic
-    // dependent launch
-    st = from_cuda(launch_layer_route(rmaps, x, bias, dims, logits, y, ctr, s));
+    moe_status_t st = check_ws(dims, ws, ws_bytes);
     if (st != MOE_OK) return st;
-    st = from_cuda(launch_layer_select(logits, probs, dims, rule, si, sw, lists, n_active, s));
+    st = check_device();
     if (st != MOE_OK) return st;
-    st = from_cuda(launch_ffn_prep(x, dims, nullptr, xk, nullptr, nullptr, lists, nullptr, true, s));
-    if (st != MOE_OK) return st;
-    return from_cuda(launch_expert_ffn(maps, xk, dims, lists, y, seg<uint16_t>(ws, L.h), nullptr, ctr, s));
+    const size_t act = static_cast<size_t>(dims.B) * dims.d;
+    const size_t sel = static_cast<size_t>(dims.B) * dims.k;
+    for (int32_t l = 0; l < n_layers; ++l) {
+        st = layer_call(xs + l * act, layers[l], dims, r, xs + (l + 1) * act, sel_idx ? sel_idx + l * sel : nullptr,
+                        nullptr, n_active ? n_active + l : nullptr, ws, static_cast<cudaStream_t>(stream), true,
+                        l > 0);
+        if (st != MOE_OK) return st;
+    }
+    return MOE_OK;
 }
 
 void moe_set_wait_limit_ns(uint64_t ns) { g_wait_ns.store(ns == 0 ? DEFAULT_WAIT_NS : ns, std::memory_order_relaxed); }

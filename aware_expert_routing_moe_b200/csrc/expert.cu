@@ -177,6 +177,11 @@ __device__ __forceinline__ void mbar_expect_tx(unsigned long long *bar, unsigned
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                  : "memory");
 }
+// Adds to the transaction count of the current phase without arriving.
+__device__ __forceinline__ void mbar_add_tx(unsigned long long *bar, unsigned bytes) {
+    asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
 __device__ __forceinline__ void mbar_arrive(unsigned long long *bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
@@ -1017,6 +1022,12 @@ struct LayerArgs {
     int row_bytes;      // shared-memory stride of one staged row (multiple of 1024)
     int box_lines, boxes;
     int r1;             // first ranks per token forming the set (OEA: k0, top-k: k); 0: published
+    int residual;       // y = x + the experts' output (a layer of a residual stack) instead of y = 0 + ...
+    // launched with programmatic dependent launch after the previous layer
+    // of a stack: x (its output) and the shared workspace are read only
+    // after the previous kernel has completed; the router weights of this
+    // layer are staged before that
+    int chained;
     ReselectArgs sel;   // the selection CTA's arguments
 };
 
@@ -1044,31 +1055,47 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     __syncthreads();
 
+    // a layer of a stack may start while the previous layer's last CTAs
+    // still run: let the next layer's CTAs launch as SMs free up
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
     // ---- 1. router items (one per CTA when there are no more items than CTAs)
     unsigned char *wrows = sm.slots;
     unsigned char *xrows = sm.slots + L.epb * L.row_bytes;
     bool prepped = false;
+    bool waited = !L.chained;
     int phase = 0;
+    const int lines = a.d >> 5;  // 128-byte lines per row
     for (int item = blockIdx.x; item < L.n_items; item += gridDim.x) {
         const int eg = item % L.n_eg, tg = item / L.n_eg;
         const int e0 = eg * L.epb, b0 = tg * L.tpb;
         const int ne = min(L.epb, a.E - e0), nb = min(L.tpb, a.B - b0);
+        const unsigned wbytes = static_cast<unsigned>(ne * L.boxes * L.box_lines * 128);
+        const unsigned xbytes = static_cast<unsigned>(nb * L.boxes * L.box_lines * 128);
         if (threadIdx.x == 0) {
-            mbar_expect_tx(&s_rbar, static_cast<unsigned>((ne + nb) * L.boxes * L.box_lines * 128));
-            const int lines = a.d >> 5;  // 128-byte lines per row
+            // the router weights first: they do not depend on the previous layer
+            if (waited) mbar_expect_tx(&s_rbar, wbytes + xbytes);
+            else mbar_add_tx(&s_rbar, wbytes);
             for (int r = 0; r < ne; ++r)
                 for (int bx = 0; bx < L.boxes; ++bx)
                     tma_rows(wrows + r * L.row_bytes + bx * L.box_lines * 128, &rmaps.wg,
                              (e0 + r) * lines + bx * L.box_lines, &s_rbar);
+        }
+        if (!waited) {
+            asm volatile("griddepcontrol.wait;" ::: "memory");
+            waited = true;
+            if (threadIdx.x == 0) mbar_expect_tx(&s_rbar, xbytes);
+        }
+        if (threadIdx.x == 0) {
             for (int r = 0; r < nb; ++r)
                 for (int bx = 0; bx < L.boxes; ++bx)
                     tma_rows(xrows + r * L.row_bytes + bx * L.box_lines * 128, &rmaps.x,
                              (b0 + r) * lines + bx * L.box_lines, &s_rbar);
         }
         if (!prepped) {
-            // x -> bf16 (read by the gate/up copies) and y = 0 (the down
-            // epilogues add into it), grid-stride: overlaps the row loads
-            layer_prep(L.x, a.B, a.d, const_cast<uint16_t *>(a.xb), a.y);
+            // x -> bf16 (read by the gate/up copies) and y = 0 or x (the
+            // down epilogues add into it), grid-stride: overlaps the row loads
+            layer_prep(L.x, a.B, a.d, const_cast<uint16_t *>(a.xb), a.y, L.residual != 0);
             prepped = true;
         }
         // every thread waits for the rows; on expiry the rows are still
@@ -1108,7 +1135,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         __syncthreads();  // the staging area is free again
         phase ^= 1;
     }
-    if (!prepped) layer_prep(L.x, a.B, a.d, const_cast<uint16_t *>(a.xb), a.y);
+    if (!waited) asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (!prepped) layer_prep(L.x, a.B, a.d, const_cast<uint16_t *>(a.xb), a.y, L.residual != 0);
     // x in bf16 is read by the async proxy (TMA) of other CTAs
     asm volatile("fence.proxy.async.global;" ::: "memory");
     __syncthreads();
@@ -1452,12 +1480,15 @@ cudaError_t launch_layer_ni(const ExpertMaps &maps, const RouterMaps &rmaps, con
     cfg.dynamicSmemBytes = smem_bytes<RG>();
     cfg.stream = s;
     // every CTA must be resident: the CTAs wait for one another at the
-    // grid barrier
-    cudaLaunchAttribute attr[1];
+    // grid barrier.  A chained layer may launch before the previous one has
+    // finished (its CTAs take SMs as the previous layer's CTAs leave them).
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeCooperative;
     attr[0].val.cooperative = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = L.chained ? 2 : 1;
     return cudaLaunchKernelEx(&cfg, layer_kernel<RG, NI>, maps, rmaps, a, L);
 }
 
@@ -1492,7 +1523,7 @@ cudaError_t launch_layer_fused(const ExpertMaps &maps, const RouterMaps &rmaps, 
                                const moe_reselect_t &rule, const float *x, const float *bias, float *logits,
                                float *probs, uint16_t *xb, float *y, uint16_t *h, float *wd, int32_t *sel_idx,
                                float *sel_w, const moe_lists_t &lists, int32_t *n_active_copy, Counters *ctr,
-                               cudaStream_t s) {
+                               bool residual, bool chained, cudaStream_t s) {
     if (d.B > TN) return cudaErrorInvalidValue;
     int dev = 0, sms = 0;
     cudaError_t err = device_sms(&dev, &sms);
@@ -1512,6 +1543,8 @@ cudaError_t launch_layer_fused(const ExpertMaps &maps, const RouterMaps &rmaps, 
     L.bias = bias;
     L.logits = logits;
     L.r1 = rule.mode == MOE_RESELECT_OEA ? rule.k0 : (rule.mode == MOE_RESELECT_NONE ? d.k : 0);
+    L.residual = residual ? 1 : 0;
+    L.chained = chained ? 1 : 0;
     L.sel = make_reselect_args(logits, probs, true, d, rule, sel_idx, sel_w, lists, n_active_copy);
     L.sel.ctr = ctr;
     L.sel.wd = wd;

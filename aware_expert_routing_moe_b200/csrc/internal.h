@@ -96,9 +96,11 @@ cudaError_t launch_route_topk(const float *logits, const moe_dims_t &d, float *p
 cudaError_t launch_reselect(const float *logits, const float *probs, const moe_dims_t &d,
                             const moe_reselect_t &r, int32_t *sel_idx, float *sel_w,
                             const moe_lists_t &l, cudaStream_t s);
-// Layer path above 32 tokens, first kernel: router GEMV; also zeroes y.
+// Layer path above 32 tokens, first kernel: router GEMV; also sets y = 0
+// (y = x with residual).  chained: launched with programmatic dependent
+// launch after the previous layer of a stack.
 cudaError_t launch_layer_route(const RouterMaps &maps, const float *x, const float *bias, const moe_dims_t &d,
-                               float *logits, float *y, Counters *ctr, cudaStream_t s);
+                               float *logits, float *y, Counters *ctr, bool residual, bool chained, cudaStream_t s);
 // Layer path above 32 tokens, second kernel (chained with programmatic
 // dependent launch): softmax, selection, lists.
 cudaError_t launch_layer_select(const float *logits, float *probs, const moe_dims_t &d, const moe_reselect_t &rule,
@@ -127,11 +129,13 @@ cudaError_t launch_expert_ffn(const ExpertMaps &maps, const uint16_t *xb, const 
 // The whole layer in one cooperative persistent kernel (B <= 32): router,
 // grid barrier, selection (last CTA), expert stream (the other CTAs).  xb:
 // x in bf16 (written), h: the SwiGLU scratch, wd: the dense weights.
+// residual: y = x + the experts' output; chained: launched with
+// programmatic dependent launch after the previous layer of a stack.
 cudaError_t launch_layer_fused(const ExpertMaps &maps, const RouterMaps &rmaps, const moe_dims_t &d,
                                const moe_reselect_t &rule, const float *x, const float *bias, float *logits,
                                float *probs, uint16_t *xb, float *y, uint16_t *h, float *wd, int32_t *sel_idx,
                                float *sel_w, const moe_lists_t &lists, int32_t *n_active_copy, Counters *ctr,
-                               cudaStream_t s);
+                               bool residual, bool chained, cudaStream_t s);
 // Limit of every bounded wait inside the kernels launched from now on
 // (nanoseconds; moe_set_wait_limit_ns).
 unsigned long long wait_limit_ns();

@@ -721,9 +721,10 @@ __device__ __forceinline__ float comp(const float4 &v, int u) {
 }
 
 // Layer path: x -> bf16 copy for the expert kernel (when xb is non-null),
-// y = 0 (grid-stride over the blocks of the launch).
+// y = 0, or y = x for a residual layer whose experts add on top of its
+// input (grid-stride over the blocks of the launch).
 __device__ void layer_prep(const float *__restrict__ x, int B, int d, uint16_t *__restrict__ xb,
-                           float *__restrict__ y) {
+                           float *__restrict__ y, bool residual) {
     const int n4 = B * d / 4;
     const int nblocks = gridDim.x * gridDim.y;
     const int nthreads = nblocks * blockDim.x;
@@ -734,7 +735,7 @@ __device__ void layer_prep(const float *__restrict__ x, int B, int d, uint16_t *
         const unsigned hi = static_cast<unsigned>(__bfloat16_as_ushort(__float2bfloat16_rn(v.z))) |
                             (static_cast<unsigned>(__bfloat16_as_ushort(__float2bfloat16_rn(v.w))) << 16);
         if (xb) reinterpret_cast<uint2 *>(xb)[i] = make_uint2(lo, hi);
-        reinterpret_cast<float4 *>(y)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        reinterpret_cast<float4 *>(y)[i] = residual ? v : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 }
 

@@ -95,8 +95,10 @@ struct GemvArgs {
     int boxes;        // boxes per row
     float *logits;
     const float *x;   // layer path: the tokens (y has their shape)
-    float *y;         // layer path: zeroed (else null)
+    float *y;         // layer path: zeroed, or set to x when residual (else null)
     Counters *ctr;    // layer path: error word (else null)
+    int residual;     // layer path: y = x (the experts add on top of the layer's input)
+    int chained;      // launched with programmatic dependent launch after the previous layer
 };
 
 template <int NI>
@@ -107,6 +109,8 @@ __global__ void __launch_bounds__(32 * GEMV_EPB_MAX) route_gemv_kernel(const __g
     __shared__ int s_fail;
     // the next kernel (the selection) may become resident while this runs
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    // a layer of a stack reads the previous layer's output and workspace
+    if (g.chained) asm volatile("griddepcontrol.wait;" ::: "memory");
     unsigned char *rows = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(gemv_smem) + 1023) & ~static_cast<uintptr_t>(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -134,7 +138,7 @@ __global__ void __launch_bounds__(32 * GEMV_EPB_MAX) route_gemv_kernel(const __g
                 tma_rows(xrows + r * g.row_bytes + bx * g.box_lines * 128, &maps.x,
                          (b0 + r) * lines + bx * g.box_lines, &s_bar);
     }
-    if (g.y != nullptr) layer_prep(g.x, g.B, g.d, nullptr, g.y);  // overlaps the loads
+    if (g.y != nullptr) layer_prep(g.x, g.B, g.d, nullptr, g.y, g.residual != 0);  // overlaps the loads
     if (!bar_try_wait0(&s_bar)) {
         // bounded: past the limit the block records the error and skips its
         // dot products, but still lets the copies land (up to a further
@@ -202,7 +206,8 @@ GemvShape gemv_shape(const moe_dims_t &d) {
 }
 
 template <int NI>
-cudaError_t launch_gemv_ni(const RouterMaps &maps, const GemvArgs &g, const GemvShape &sh, cudaStream_t s) {
+cudaError_t launch_gemv_ni(const RouterMaps &maps, const GemvArgs &g, const GemvShape &sh, cudaStream_t s,
+                           bool chained) {
     // the attributes belong to the function on each device: set them once per device
     static bool configured[MAX_DEVICES] = {};
     int dev = 0;
@@ -219,17 +224,26 @@ cudaError_t launch_gemv_ni(const RouterMaps &maps, const GemvArgs &g, const Gemv
         if (err != cudaSuccess) return err;
         configured[dev] = true;
     }
-    const dim3 grid((g.E + sh.epb - 1) / sh.epb, (g.B + sh.tpb - 1) / sh.tpb);
-    route_gemv_kernel<NI><<<grid, 32 * sh.epb, sh.smem, s>>>(maps, g);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((g.E + sh.epb - 1) / sh.epb, (g.B + sh.tpb - 1) / sh.tpb);
+    cfg.blockDim = dim3(32 * sh.epb);
+    cfg.dynamicSmemBytes = sh.smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = chained ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, route_gemv_kernel<NI>, maps, g);
 }
 
-cudaError_t launch_gemv(const RouterMaps &maps, const GemvArgs &g, const GemvShape &sh, cudaStream_t s) {
+cudaError_t launch_gemv(const RouterMaps &maps, const GemvArgs &g, const GemvShape &sh, cudaStream_t s,
+                        bool chained = false) {
     switch (ni_for(g.E)) {
-        case 1: return launch_gemv_ni<1>(maps, g, sh, s);
-        case 2: return launch_gemv_ni<2>(maps, g, sh, s);
-        case 4: return launch_gemv_ni<4>(maps, g, sh, s);
-        default: return launch_gemv_ni<8>(maps, g, sh, s);
+        case 1: return launch_gemv_ni<1>(maps, g, sh, s, chained);
+        case 2: return launch_gemv_ni<2>(maps, g, sh, s, chained);
+        case 4: return launch_gemv_ni<4>(maps, g, sh, s, chained);
+        default: return launch_gemv_ni<8>(maps, g, sh, s, chained);
     }
 }
 
@@ -249,6 +263,8 @@ GemvArgs make_gemv_args(const float *bias, const moe_dims_t &d, const GemvShape 
     g.x = nullptr;
     g.y = nullptr;
     g.ctr = nullptr;
+    g.residual = 0;
+    g.chained = 0;
     return g;
 }
 
@@ -326,13 +342,15 @@ cudaError_t launch_reselect(const float *logits, const float *probs, const moe_d
 }
 
 cudaError_t launch_layer_route(const RouterMaps &maps, const float *x, const float *bias, const moe_dims_t &d,
-                               float *logits, float *y, Counters *ctr, cudaStream_t s) {
+                               float *logits, float *y, Counters *ctr, bool residual, bool chained, cudaStream_t s) {
     const GemvShape sh = gemv_shape(d);
     GemvArgs g = make_gemv_args(bias, d, sh, logits);
     g.x = x;
     g.y = y;
     g.ctr = ctr;
-    return launch_gemv(maps, g, sh, s);
+    g.residual = residual ? 1 : 0;
+    g.chained = chained ? 1 : 0;
+    return launch_gemv(maps, g, sh, s, chained);
 }
 
 cudaError_t launch_layer_select(const float *logits, float *probs, const moe_dims_t &d, const moe_reselect_t &rule,

@@ -364,6 +364,28 @@ def run_ours(args, w, rank, world, local_rank):
     expert_leg = {"kernel": "moe_expert_ffn (input prep + expert kernel, lists given)", "achieved": ffn_gbs,
                   "unit": "GB/s", "frac": ffn_gbs / hbm_peak, "us_per_call": ms_ffn * 1e3}
 
+    # ---- the same layers as a stack: the ROTATE weight copies as ROTATE
+    # consecutive residual layers, chained on the device (moe_decode_stack)
+    xs = torch.zeros(ROTATE + 1, B, S.d, dtype=torch.float32, device=dev)
+    xs[0] = x
+    stack_layers = [(c[3], bias, c[0], c[1], c[2]) for c in copies]
+    stack_ws = moe.new_workspace(B, S.d, S.E, S.k, S.F, dev)
+    with torch.cuda.stream(s):
+        moe.moe_decode_stack(xs, stack_layers, S.k, mode, k0, budget, ws=stack_ws, group=group)
+    s.synchronize()
+    g_stack = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_stack, stream=s):
+        moe.moe_decode_stack(xs, stack_layers, S.k, mode, k0, budget, ws=stack_ws, group=group)
+    nst = max(1, args.steps // ROTATE)
+    with torch.cuda.stream(s):
+        for _ in range(max(1, args.warmup // ROTATE)):
+            g_stack.replay()
+    ms_stack = timed(lambda n: [g_stack.replay() for _ in range(n)], nst) / (nst * ROTATE)
+    if moe.moe_check_error(stack_ws, s) != 0:
+        raise RuntimeError("device error word set in the stack leg")
+    stack = {"layers": ROTATE, "us_per_layer": ms_stack * 1e3,
+             "note": "residual stack of the rotating weight copies, layer l+1 chained on layer l"}
+
     # ---- end to end through the Python API with pinned host buffers
     x_host = torch.from_numpy(x_np).pin_memory()
     y_host = torch.empty(B, S.d, dtype=torch.float32).pin_memory()
@@ -385,7 +407,7 @@ def run_ours(args, w, rank, world, local_rank):
            "ms_per_step": ms_e2e}
     sampler.__exit__(None, None, None)
     clocks = sampler.summary()
-    clocks["window"] = "warm-up, timed region, launch-overhead, expert-kernel and end-to-end legs"
+    clocks["window"] = "warm-up, timed region, launch-overhead, expert-kernel, stack and end-to-end legs"
     if moe.moe_check_error(ws, s) != 0:
         raise RuntimeError("device error word set during the benchmark")
 
@@ -409,6 +431,7 @@ def run_ours(args, w, rank, world, local_rank):
         "stream_launch_us_per_call": ms_stream * 1e3,
         "roofline": roofline,
         "expert_ffn_leg": expert_leg,
+        "stack_leg": stack,
         "e2e": e2e,
         # up to 32 tokens one fused kernel per call; above, router,
         # selection, x dispatch and expert kernels
@@ -419,7 +442,7 @@ def run_ours(args, w, rank, world, local_rank):
         line["cpu_baseline"] = cpu_baseline(w, S, L, x_np)
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del g_all, g_one, g_ffn
+    del g_all, g_one, g_ffn, g_stack
     torch.cuda.synchronize(dev)
 
 

@@ -225,6 +225,54 @@ moe_status_t moe_layer_decode(const float *x, const float *Wg, const float *bias
                               float *sel_w, int32_t *n_active, void *ws,
                               size_t ws_bytes, void *stream);
 
+/* One MoE layer's weights for moe_decode_stack (device pointers, layouts as
+ * for moe_layer_decode; bias may be NULL). */
+typedef struct {
+    const float *Wg;
+    const float *bias;
+    const uint16_t *Wgate;
+    const uint16_t *Wup;
+    const uint16_t *Wdown;
+} moe_layer_weights_t;
+
+/* Phase of a stack call.  Re-selection pays only in decode, where the layer
+ * is bound by memory bandwidth; prefill is compute-bound and sensitive to
+ * which experts a token gets, so a phase-aware caller bypasses re-routing
+ * there ("Lynx: Enabling Efficient MoE Inference through Dynamic
+ * Batch-Aware Expert Selection", section 2.1 "Phase Sensitivity" and
+ * section 2.2 "Phase-Aware Optimizer"). */
+typedef enum {
+    MOE_PHASE_DECODE = 0,   /* apply the given re-selection rule */
+    MOE_PHASE_PREFILL = 1   /* prefill or chunked prefill: standard top-k (MOE_RESELECT_NONE) */
+} moe_phase_t;
+
+#define MOE_STACK_MAX_LAYERS 1024
+
+/* n_layers MoE layers back to back on a residual stream:
+ *   xs[l + 1] = xs[l] + layer_l(xs[l]),   l = 0 .. n_layers - 1,
+ * each layer_l as moe_layer_decode with layers[l]'s weights and the same
+ * dims and rule (the attention blocks between MoE layers are not part of
+ * this library).  Consecutive layers are chained on the device with no host
+ * round trip: layer l + 1 is launched with programmatic dependent launch,
+ * so its CTAs start, and stage layer l + 1's router weights, while layer
+ * l's last CTAs still stream experts; its router reads xs[l + 1] once layer
+ * l has completed ("Router Caching and Optimization", "Scheduling Router
+ * Computation": router computation for a layer partially overlapped with
+ * the previous layer's).
+ *   layers: HOST array of n_layers weight sets (1 <= n_layers <=
+ *   MOE_STACK_MAX_LAYERS); phase: moe_phase_t (PREFILL replaces `rule` by
+ *   standard top-k);
+ *   xs[n_layers + 1][B][d] fp32 (device): xs[0] is the input, read only;
+ *   xs[1 .. n_layers] are written;
+ *   sel_idx[n_layers][B][k] int32, n_active[n_layers] int32: optional
+ *   device outputs per layer (NULL = not returned);
+ *   ws: one workspace of moe_workspace_bytes(dims) bytes, reused by every
+ *   layer.
+ * Validation covers every layer before anything is enqueued. */
+moe_status_t moe_decode_stack(const moe_layer_weights_t *layers, int32_t n_layers, moe_dims_t dims,
+                              moe_reselect_t rule, int32_t phase, float *xs, int32_t *sel_idx,
+                              int32_t *n_active, void *ws, size_t ws_bytes, void *stream);
+
 /* moe_expert_ffn for callers that cannot allocate device memory.
  * (The source pages have no counterpart to this entry point; it is a
  * deployment convenience of this library.)

@@ -195,3 +195,18 @@ def test_noalloc_size_limit(lib):
     # invalid dims and misaligned buffers are reported first
     assert lib.moe_expert_ffn_noalloc(A, A, A, A, Dims(257, 2048, 128, 8, 768), lists, A, None) == INVALID
     assert lib.moe_expert_ffn_noalloc(A + 4, A, A, A, Dims(16, 2048, 128, 8, 768), lists, A, None) == MISALIGNED
+
+
+def test_stack_rejects_bad_arguments(lib):
+    # host validation only: every layer is checked before anything is enqueued
+    A = 0x10000
+    w = (moe.LayerWeights * 2)(moe.LayerWeights(A, 0, A, A, A), moe.LayerWeights(A, 0, 0, A, A))
+    d = moe.Dims(16, 2048, 128, 8, 768)
+    r = moe.Rule(1, 4, 0, 1)
+    assert lib.moe_decode_stack(w, 0, d, r, 0, A, None, None, A, 1 << 30, None) == 1  # no layers
+    assert lib.moe_decode_stack(w, 2, d, r, 0, A, None, None, A, 1 << 30, None) == 1  # layer 1 lacks Wgate
+    assert lib.moe_decode_stack(w, 1, d, r, 7, A, None, None, A, 1 << 30, None) == 1  # unknown phase
+    assert lib.moe_decode_stack(w, 1, d, moe.Rule(1, 9, 0, 1), 0, A, None, None, A, 1 << 30, None) == 1  # k0 > k
+    # prefill ignores the decode rule, so an invalid rule passes there
+    assert lib.moe_decode_stack(w, 1, d, moe.Rule(1, 9, 0, 1), 1, A + 4, None, None, A, 1 << 30, None) == 2
+    assert lib.moe_decode_stack(w, 1, d, r, 0, A + 4, None, None, A, 1 << 30, None) == 2  # misaligned xs
