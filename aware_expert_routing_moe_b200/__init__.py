@@ -24,7 +24,7 @@ __all__ = [
     "moe_status_string", "moe_route", "moe_reselect", "moe_expert_ffn", "moe_layer_decode",
     "moe_check_error", "moe_expert_ffn_noalloc", "new_workspace", "alloc_lists", "ABI_SYMBOLS",
     "NOALLOC_SCRATCH_BYTES", "moe_set_wait_limit_ns", "moe_decode_stack", "LayerWeights",
-    "MOE_PHASE_DECODE", "MOE_PHASE_PREFILL",
+    "MOE_PHASE_DECODE", "MOE_PHASE_PREFILL", "moe_down_channel_major", "moe_expert_ffn_channels",
 ]
 
 MOE_RESELECT_NONE, MOE_RESELECT_OEA, MOE_RESELECT_XSHARE = 0, 1, 2
@@ -33,7 +33,8 @@ STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_MISALIGNED", 3: "MO
           4: "MOE_ERR_UNSUPPORTED", 5: "MOE_ERR_CUDA", 6: "MOE_ERR_INTERNAL"}
 ABI_SYMBOLS = ("moe_workspace_bytes", "moe_route", "moe_reselect", "moe_expert_ffn",
                "moe_layer_decode", "moe_expert_ffn_noalloc", "moe_check_error", "moe_status_string",
-               "moe_set_wait_limit_ns", "moe_decode_stack")
+               "moe_set_wait_limit_ns", "moe_decode_stack", "moe_down_channel_major",
+               "moe_channels_workspace_bytes", "moe_expert_ffn_channels")
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -98,6 +99,12 @@ def load_library() -> ctypes.CDLL:
         lib.moe_decode_stack.restype = ctypes.c_int
         lib.moe_decode_stack.argtypes = [ctypes.POINTER(LayerWeights), ctypes.c_int32, Dims, Rule, ctypes.c_int32,
                                          P, P, P, P, S, P]
+        lib.moe_down_channel_major.restype = ctypes.c_int
+        lib.moe_down_channel_major.argtypes = [P, Dims, P, P]
+        lib.moe_channels_workspace_bytes.restype = S
+        lib.moe_channels_workspace_bytes.argtypes = [Dims]
+        lib.moe_expert_ffn_channels.restype = ctypes.c_int
+        lib.moe_expert_ffn_channels.argtypes = [P, P, P, P, Dims, P, P, P, ctypes.c_int32, P, P, P, S, P]
         lib.moe_set_wait_limit_ns.restype = None
         lib.moe_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
         _lib = lib
@@ -245,6 +252,41 @@ def moe_decode_stack(xs, layers, k: int, mode: int, k0: int = 0, budget: int = 0
                                          ws.numel() * ws.element_size(), _stream(stream))
     _check(st, "moe_decode_stack")
     return xs
+
+
+def moe_down_channel_major(Wdown, out=None, stream=None):
+    """Channel-major copy of the down weights: out[E][d_ff][d] = Wdown[E][d][d_ff]
+    transposed per expert (bf16 bits as int16/uint16 tensors)."""
+    E, d, F = Wdown.shape
+    if out is None:
+        out = torch.empty(E, F, d, dtype=Wdown.dtype, device=Wdown.device)
+    st = load_library().moe_down_channel_major(_ptr(Wdown), Dims(1, d, E, 1, F), _ptr(out), _stream(stream))
+    _check(st, "moe_down_channel_major")
+    return out
+
+
+def moe_expert_ffn_channels(x, Wgate, Wup, WdownT, sel_idx, sel_w, score, c: int, y=None, keep=None, ws=None,
+                            stream=None):
+    """Expert FFN where each (token, slot) keeps its c highest-scoring
+    channels (score[B][k][d_ff]); WdownT from moe_down_channel_major.
+    -> y[B][d] fp32.  ``keep``: optional [B][k][d_ff/32] int32 output."""
+    B, d = x.shape
+    E, F, _ = Wgate.shape
+    k = sel_idx.shape[1]
+    lib = load_library()
+    dims = Dims(B, d, E, k, F)
+    n = int(lib.moe_channels_workspace_bytes(dims))
+    if n == 0:
+        raise MoeError(4, "moe_channels_workspace_bytes")
+    if ws is None:
+        ws = torch.empty(n, dtype=torch.uint8, device=x.device)
+    if y is None:
+        y = torch.empty(B, d, dtype=torch.float32, device=x.device)
+    st = lib.moe_expert_ffn_channels(_ptr(x), _ptr(Wgate), _ptr(Wup), _ptr(WdownT), dims, _ptr(sel_idx),
+                                     _ptr(sel_w), _ptr(score), int(c), _ptr(y), _ptr(keep), _ptr(ws),
+                                     ws.numel() * ws.element_size(), _stream(stream))
+    _check(st, "moe_expert_ffn_channels")
+    return y
 
 
 def moe_expert_ffn_noalloc(x, Wgate, Wup, Wdown, lists: dict, k: int, y=None, stream=None):

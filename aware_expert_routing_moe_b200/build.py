@@ -22,7 +22,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libmoe_decode.so")
 BUILD_DIR = os.path.join(ROOT, "_build")
 
-SOURCES = ["router.cu", "expert.cu", "abi.cu", "noalloc.cu"]
+SOURCES = ["router.cu", "expert.cu", "abi.cu", "noalloc.cu", "channels.cu"]
 GENCODE = "arch=compute_100a,code=sm_100a"
 
 

@@ -382,6 +382,39 @@ moe_status_t moe_decode_stack(const moe_layer_weights_t *layers, int32_t n_layer
     return MOE_OK;
 }
 
+moe_status_t moe_down_channel_major(const uint16_t *Wdown, moe_dims_t dims, uint16_t *WdownT, void *stream) {
+    if (!dims_ok(dims) || !Wdown || !WdownT) return MOE_ERR_INVALID_ARG;
+    if (!al16(Wdown) || !al16(WdownT)) return MOE_ERR_MISALIGNED;
+    const moe_status_t st = check_device();
+    if (st != MOE_OK) return st;
+    return from_cuda(launch_down_transpose(Wdown, dims, WdownT, static_cast<cudaStream_t>(stream)));
+}
+
+size_t moe_channels_workspace_bytes(moe_dims_t dims) {
+    if (!dims_ok(dims) || dims.B > MOE_CHANNELS_B_MAX || channels_stages(dims) < 2) return 0;
+    return channels_workspace_bytes(dims);
+}
+
+moe_status_t moe_expert_ffn_channels(const float *x, const uint16_t *Wgate, const uint16_t *Wup,
+                                     const uint16_t *WdownT, moe_dims_t dims, const int32_t *sel_idx,
+                                     const float *sel_w, const float *score, int32_t c, float *y, uint32_t *keep,
+                                     void *ws, size_t ws_bytes, void *stream) {
+    if (!dims_ok(dims)) return MOE_ERR_INVALID_ARG;
+    if (!x || !Wgate || !Wup || !WdownT || !sel_idx || !sel_w || !score || !y) return MOE_ERR_INVALID_ARG;
+    if (c < 1 || c > dims.d_ff) return MOE_ERR_INVALID_ARG;
+    if (dims.B > MOE_CHANNELS_B_MAX || channels_stages(dims) < 2) return MOE_ERR_UNSUPPORTED;
+    if (!al16(x) || !al16(Wgate) || !al16(Wup) || !al16(WdownT) || !al16(sel_idx) || !al16(sel_w) ||
+        !al16(score) || !al16(y) || (keep && !al16(keep)))
+        return MOE_ERR_MISALIGNED;
+    if (!ws) return MOE_ERR_WORKSPACE;
+    if (!al256(ws)) return MOE_ERR_MISALIGNED;
+    if (ws_bytes < channels_workspace_bytes(dims)) return MOE_ERR_WORKSPACE;
+    const moe_status_t st = check_device();
+    if (st != MOE_OK) return st;
+    return from_cuda(launch_channels(x, Wgate, Wup, WdownT, dims, sel_idx, sel_w, score, c, y, keep, ws,
+                                     static_cast<cudaStream_t>(stream)));
+}
+
 void moe_set_wait_limit_ns(uint64_t ns) { g_wait_ns.store(ns == 0 ? DEFAULT_WAIT_NS : ns, std::memory_order_relaxed); }
 
 moe_status_t moe_check_error(void *ws, size_t ws_bytes, void *stream) {

@@ -136,6 +136,15 @@ cudaError_t launch_layer_fused(const ExpertMaps &maps, const RouterMaps &rmaps, 
                                float *probs, uint16_t *xb, float *y, uint16_t *h, float *wd, int32_t *sel_idx,
                                float *sel_w, const moe_lists_t &lists, int32_t *n_active_copy, Counters *ctr,
                                bool residual, bool chained, cudaStream_t s);
+// Per-token channel top-k (channels.cu): workspace bytes, ring stages of the
+// stream kernel for d (0: the dims do not fit its shared memory), the
+// channel-major copy of Wdown, and the three kernels of one call.
+size_t channels_workspace_bytes(const moe_dims_t &d);
+int channels_stages(const moe_dims_t &d);
+cudaError_t launch_down_transpose(const uint16_t *Wdown, const moe_dims_t &d, uint16_t *WdownT, cudaStream_t s);
+cudaError_t launch_channels(const float *x, const uint16_t *Wgate, const uint16_t *Wup, const uint16_t *WdownT,
+                            const moe_dims_t &d, const int32_t *sel_idx, const float *sel_w, const float *score,
+                            int c, float *y, uint32_t *keep_out, void *ws, cudaStream_t s);
 // Limit of every bounded wait inside the kernels launched from now on
 // (nanoseconds; moe_set_wait_limit_ns).
 unsigned long long wait_limit_ns();

@@ -273,6 +273,46 @@ moe_status_t moe_decode_stack(const moe_layer_weights_t *layers, int32_t n_layer
                               moe_reselect_t rule, int32_t phase, float *xs, int32_t *sel_idx,
                               int32_t *n_active, void *ws, size_t ws_bytes, void *stream);
 
+/* ---- Per-token channel top-k inside the activated experts ----------------
+ * "Channel Selection for Mixture-of-Experts Decoding Needs No Calibration
+ * Data", methodology: a channel selector is a score plus a keep rule; the
+ * top-k keep rule takes each token's c highest-scoring channels of an
+ * expert; channel f of expert e is gate row f, up row f and down column f,
+ * and only the kept channels' weights are read (counted in 32-byte
+ * sectors).  The scores come from the caller (any selector).  The down
+ * projection is read from a channel-major copy, so that a channel's down
+ * weights are one contiguous 2*d-byte row like its gate and up rows. */
+#define MOE_CHANNELS_B_MAX 8
+
+/* WdownT[E][d_ff][d] = Wdown[E][d][d_ff] transposed per expert (bf16 bits,
+ * device; done once when the weights are loaded).  d, d_ff as for the
+ * layer (multiples of 64).  Enqueued on `stream`. */
+moe_status_t moe_down_channel_major(const uint16_t *Wdown, moe_dims_t dims, uint16_t *WdownT, void *stream);
+
+/* Device workspace bytes of moe_expert_ffn_channels for dims (0 if the
+ * dims are outside its limits: B <= MOE_CHANNELS_B_MAX, 2 * B * d * 4 +
+ * 2 * 3 * d * 2 <= 200 KB of shared memory, plus the layer's limits). */
+size_t moe_channels_workspace_bytes(moe_dims_t dims);
+
+/* y[b] = sum over slots s with e = sel_idx[b][s] >= 0 of sel_w[b][s] *
+ *        sum over the kept channels f of Wdown[e][:, f] silu(g_f) u_f,
+ * g_f = Wgate[e][f] . x[b], u_f = Wup[e][f] . x[b], where (b, s) keeps the
+ * c channels with the largest score[b][s][f] (equal scores to the lower
+ * channel index).
+ *   x[B][d] fp32; Wgate, Wup [E][d_ff][d] bf16; WdownT [E][d_ff][d] bf16
+ *   (moe_down_channel_major); sel_idx[B][k] int32 (-1 = empty slot) and
+ *   sel_w[B][k] fp32, e.g. from moe_reselect; score[B][k][d_ff] fp32;
+ *   1 <= c <= d_ff; y[B][d] fp32 (overwritten); keep[B][k][d_ff / 32]
+ *   uint32 (optional output, bit f of word f / 32 = channel f kept; NULL =
+ *   not returned); ws of moe_channels_workspace_bytes(dims) bytes, 256-byte
+ *   aligned (no zero-fill needed).  Weights are read in fp32 FMAs (no
+ *   tensor cores: a handful of tokens share a channel); summation order
+ *   within a dot product is fixed per launch shape. */
+moe_status_t moe_expert_ffn_channels(const float *x, const uint16_t *Wgate, const uint16_t *Wup,
+                                     const uint16_t *WdownT, moe_dims_t dims, const int32_t *sel_idx,
+                                     const float *sel_w, const float *score, int32_t c, float *y,
+                                     uint32_t *keep, void *ws, size_t ws_bytes, void *stream);
+
 /* moe_expert_ffn for callers that cannot allocate device memory.
  * (The source pages have no counterpart to this entry point; it is a
  * deployment convenience of this library.)

@@ -210,3 +210,21 @@ def test_stack_rejects_bad_arguments(lib):
     # prefill ignores the decode rule, so an invalid rule passes there
     assert lib.moe_decode_stack(w, 1, d, moe.Rule(1, 9, 0, 1), 1, A + 4, None, None, A, 1 << 30, None) == 2
     assert lib.moe_decode_stack(w, 1, d, r, 0, A + 4, None, None, A, 1 << 30, None) == 2  # misaligned xs
+
+
+def test_channels_rejects_bad_arguments(lib):
+    A = 0x10000
+    d = moe.Dims(4, 2048, 128, 8, 768)
+    nb = lib.moe_channels_workspace_bytes(d)
+    assert nb > 0
+    assert lib.moe_channels_workspace_bytes(moe.Dims(9, 2048, 128, 8, 768)) == 0  # B above MOE_CHANNELS_B_MAX
+    assert lib.moe_channels_workspace_bytes(moe.Dims(8, 16384, 128, 8, 768)) == 0  # rows exceed shared memory
+    call = lambda dims, c, ws=A, n=nb, x=A: lib.moe_expert_ffn_channels(x, A, A, A, dims, A, A, A, c, A, None, ws, n,
+                                                                        None)
+    assert call(d, 0) == 1            # c < 1
+    assert call(d, 769) == 1          # c > d_ff
+    assert call(moe.Dims(9, 2048, 128, 8, 768), 10) == 4
+    assert call(d, 10, x=A + 4) == 2  # misaligned x
+    assert call(d, 10, ws=None) == 3
+    assert call(d, 10, n=nb - 1) == 3
+    assert lib.moe_down_channel_major(A, moe.Dims(1, 2048, 128, 8, 768), A + 8, None) == 2
