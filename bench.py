@@ -62,6 +62,12 @@ WORKLOADS = {
     "q30b_b16_affinity": dict(shape="q30b", B=16, mode=3, k0=0, budget=0, rule="Lynx affinity binning"),
     "spec_xshare_hier32": dict(shape="q30b", B=32, mode=4, k0=0, budget=32, group=4, kind="spec",
                                rule="hierarchical XShare budget=32, 4 tokens per request"),
+    # per-token channel top-k inside the activated experts (c = 13 % of
+    # d_ff, scores drawn at random per (token, slot))
+    "q30b_b1_oea4_ch13": dict(shape="q30b", B=1, mode=1, k0=4, budget=0, channels=0.13,
+                              rule="OEA k0=4, channel top-k 13 %"),
+    "q30b_b4_oea4_ch13": dict(shape="q30b", B=4, mode=1, k0=4, budget=0, channels=0.13,
+                              rule="OEA k0=4, channel top-k 13 %"),
 }
 
 # DRAM bytes (read + write) per launch of the expert kernel from an ncu
@@ -461,6 +467,97 @@ SWEEP = {
 }
 
 
+def channel_bytes(keep_bits: np.ndarray, sel: np.ndarray, d: int, F: int, B: int, k: int) -> int:
+    """Algorithmic bytes of one channel top-k call: for every activated
+    expert, the union of its pairs' kept channels, each a gate row, an up row
+    and a channel-major down row of 2 d bytes (whole 32-byte sectors, since
+    2 d is a multiple of 128); plus the scores, x and y."""
+    bits = np.unpackbits(keep_bits.view(np.uint8), bitorder="little").reshape(B, k, F)
+    weights = 0
+    for e in np.unique(sel[sel >= 0]):
+        u = np.zeros(F, bool)
+        for b, slot in zip(*np.nonzero(sel == e)):
+            u |= bits[b, slot].astype(bool)
+        weights += int(u.sum()) * 3 * 2 * d
+    return weights + B * k * F * 4 + 2 * B * d * 4
+
+
+def run_channels(args, w, rank, world, local_rank):
+    """Per-token channel top-k inside the activated experts: routing and
+    selection as for the layer (moe_route, moe_reselect), then
+    moe_expert_ffn_channels timed alone over graph replays on ROTATE weight
+    copies (each with its channel-major down copy)."""
+    import torch
+    import aware_expert_routing_moe_b200 as moe
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    S = ms.SHAPES[w["shape"]]
+    B = w["B"]
+    c = max(1, int(round(w["channels"] * S.F)))
+    L = ms.make_weights(S, 0)
+    x_np = ms.make_tokens(S, B, 0)
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    x, Wg, bias = t(x_np), t(L["Wg"]), t(L["bias"])
+    base = (t(L["Wgate"].view(np.int16)), t(L["Wup"].view(np.int16)), t(L["Wdown"].view(np.int16)))
+    copies = [base] + [tuple(a.clone() for a in base) for _ in range(ROTATE - 1)]
+    downT = [moe.moe_down_channel_major(cp[2]) for cp in copies]
+    logits, probs, _, _ = moe.moe_route(x, Wg, bias, S.k)
+    sel, sw, _ = moe.moe_reselect(logits, probs, S.k, w["mode"], w["k0"], w["budget"])
+    score = t(np.random.default_rng(1000).standard_normal((B, S.k, S.F)).astype(np.float32))
+    y = torch.empty(B, S.d, dtype=torch.float32, device=dev)
+    keep = torch.empty(B, S.k, S.F // 32, dtype=torch.int32, device=dev)
+    ws = torch.empty(moe.load_library().moe_channels_workspace_bytes(moe.Dims(B, S.d, S.E, S.k, S.F)),
+                     dtype=torch.uint8, device=dev)
+    s = torch.cuda.Stream(dev)
+
+    def call(r):
+        g, u, _ = copies[r]
+        moe.moe_expert_ffn_channels(x, g, u, downT[r], sel, sw, score, c, y=y, keep=keep, ws=ws)
+
+    with torch.cuda.stream(s):
+        for r in range(ROTATE):
+            call(r)
+    s.synchronize()
+    nbytes = channel_bytes(keep.cpu().numpy(), sel.cpu().numpy(), S.d, S.F, B, S.k)
+    g_all = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_all, stream=s):
+        for r in range(ROTATE):
+            call(r)
+    reps = max(1, args.steps // ROTATE)
+    with torch.cuda.stream(s):
+        for _ in range(max(1, args.warmup // ROTATE)):
+            g_all.replay()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local_rank)
+    with sampler, torch.cuda.stream(s):
+        e0.record(s)
+        for _ in range(reps):
+            g_all.replay()
+        e1.record(s)
+        e1.synchronize()
+    ms_call = e0.elapsed_time(e1) / (reps * ROTATE)
+    if moe.moe_check_error(ws, s) != 0:
+        raise RuntimeError("device error word set in the channel path")
+    hbm_peak, peak_kind = measured_peaks()
+    gbs = nbytes / (ms_call * 1e-3) / 1e9
+    line = {
+        "metric": "per-token channel top-k expert FFN: µs and achieved HBM GB/s of the sector-counted bytes",
+        "value": gbs, "unit": UNIT, "n_gpus": 1, "steps": reps * ROTATE, "warmup": args.warmup,
+        "ms_per_step": ms_call, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": workload_desc(w), "channels_kept": c, "bytes_per_call": nbytes,
+                   "l2": f"{ROTATE} rotating copies of the expert weights"},
+        "us_per_call": ms_call * 1e3,
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
+                     "traffic": None, "kernel": "channel_select + channel_items + channel_stream kernels",
+                     "peak_source": f"{peak_kind} HBM copy bandwidth"},
+        "gpu_launches": 3 * reps * ROTATE, "clocks": sampler.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    del g_all
+
+
 def run_sweep(args):
     """Times moe_layer_decode on every configuration of SWEEP (device time per
     call over graph replays of ROTATE calls on rotating weight copies) and
@@ -589,6 +686,10 @@ def main(argv=None):
         return run_sweep(args)
     if args.profile:
         return run_profile_case(args, w)
+    if "channels" in w and args.impl == "ours":
+        if rank == 0:
+            run_channels(args, w, rank, world, local_rank)
+        return 0
     if args.impl == "reference":
         run_reference(args, w, rank)
         return 0

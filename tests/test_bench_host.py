@@ -4,6 +4,7 @@ CPU), the workload table and the algorithmic byte count."""
 import os
 import socket
 
+import numpy as np
 import pytest
 import torch.distributed as dist
 import torch.multiprocessing as mp
@@ -88,3 +89,17 @@ def test_every_timed_configuration_passes_host_validation():
         st = lib.moe_layer_decode(A, A, A, A, A, A, dims, Rule(mode, k0, budget, group), A, None, None, None, A,
                                   nbytes, None)
         assert st == 5, (shape, B, mode, k0, budget, group, st)    # MOE_ERR_CUDA: validation passed
+
+
+def test_channel_bytes_match_the_oracle_sector_count(oracle_lib):
+    # bench.py counts the channel path's weight bytes itself (the timed code
+    # may not call the oracle); it must agree with the oracle's sector count
+    import bench
+    rng = np.random.default_rng(5)
+    B, k, E, d, F = 3, 4, 10, 256, 128
+    sel = rng.integers(-1, E, size=(B, k)).astype(np.int32)
+    keep = (rng.random((B, k, F)) < 0.2).astype(np.uint8)
+    keep[sel < 0] = 0
+    bits = np.packbits(keep, axis=-1, bitorder="little").view(np.uint32)
+    got = bench.channel_bytes(bits, sel, d, F, B, k) - (B * k * F * 4 + 2 * B * d * 4)
+    assert got == oracle_lib.channel_sector_bytes(keep, sel, E, d, down_channel_major=True)
