@@ -279,7 +279,7 @@ def moe_expert_ffn_channels(x, Wgate, Wup, WdownT, sel_idx, sel_w, score, c: int
     if n == 0:
         raise MoeError(4, "moe_channels_workspace_bytes")
     if ws is None:
-        ws = torch.empty(n, dtype=torch.uint8, device=x.device)
+        ws = torch.zeros(n, dtype=torch.uint8, device=x.device)
     if y is None:
         y = torch.empty(B, d, dtype=torch.float32, device=x.device)
     st = lib.moe_expert_ffn_channels(_ptr(x), _ptr(Wgate), _ptr(Wup), _ptr(WdownT), dims, _ptr(sel_idx),

@@ -85,7 +85,13 @@ moe_status_t check_device() {
     return cached[dev] == 1 ? MOE_OK : MOE_ERR_UNSUPPORTED;
 }
 
-moe_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+// A failed launch leaves its error as the thread's last error: clear it, so
+// that the next call's launch check does not report it again.
+moe_status_t from_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return MOE_OK;
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+}
 
 // ---------------------------------------------------------- tensor maps --
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
@@ -418,7 +424,8 @@ moe_status_t moe_expert_ffn_channels(const float *x, const uint16_t *Wgate, cons
 void moe_set_wait_limit_ns(uint64_t ns) { g_wait_ns.store(ns == 0 ? DEFAULT_WAIT_NS : ns, std::memory_order_relaxed); }
 
 moe_status_t moe_check_error(void *ws, size_t ws_bytes, void *stream) {
-    if (!ws || ws_bytes < sizeof(Counters)) return MOE_ERR_WORKSPACE;
+    // every workspace of this library starts with its error word
+    if (!ws || ws_bytes < sizeof(int32_t)) return MOE_ERR_WORKSPACE;
     if (!al256(ws)) return MOE_ERR_MISALIGNED;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     Counters *ctr = seg<Counters>(ws, 0);

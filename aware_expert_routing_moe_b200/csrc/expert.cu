@@ -1382,13 +1382,19 @@ cudaError_t device_sms(int *dev_out, int *sms) {
     return cudaSuccess;
 }
 
-// Sets the dynamic shared-memory limit of a kernel once per device.
+// Sets the dynamic shared-memory limit of a kernel once per device (keyed
+// by the kernel's address: template instances share a type).
 template <class K>
 cudaError_t configure_smem(K kernel, int bytes, int dev) {
-    static bool done[MAX_DEVICES] = {};
-    if (done[dev]) return cudaSuccess;
+    static std::mutex mu;
+    static const void *done[64][MAX_DEVICES] = {};
+    const void *key = reinterpret_cast<const void *>(kernel);
+    std::lock_guard<std::mutex> lock(mu);
+    int slot = 0;
+    for (; slot < 64 && done[slot][dev] != nullptr; ++slot)
+        if (done[slot][dev] == key) return cudaSuccess;
     const cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (err == cudaSuccess) done[dev] = true;
+    if (err == cudaSuccess && slot < 64) done[slot][dev] = key;
     return err;
 }
 

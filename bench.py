@@ -506,7 +506,7 @@ def run_channels(args, w, rank, world, local_rank):
     score = t(np.random.default_rng(1000).standard_normal((B, S.k, S.F)).astype(np.float32))
     y = torch.empty(B, S.d, dtype=torch.float32, device=dev)
     keep = torch.empty(B, S.k, S.F // 32, dtype=torch.int32, device=dev)
-    ws = torch.empty(moe.load_library().moe_channels_workspace_bytes(moe.Dims(B, S.d, S.E, S.k, S.F)),
+    ws = torch.zeros(moe.load_library().moe_channels_workspace_bytes(moe.Dims(B, S.d, S.E, S.k, S.F)),
                      dtype=torch.uint8, device=dev)
     s = torch.cuda.Stream(dev)
 

@@ -305,7 +305,8 @@ size_t moe_channels_workspace_bytes(moe_dims_t dims);
  *   1 <= c <= d_ff; y[B][d] fp32 (overwritten); keep[B][k][d_ff / 32]
  *   uint32 (optional output, bit f of word f / 32 = channel f kept; NULL =
  *   not returned); ws of moe_channels_workspace_bytes(dims) bytes, 256-byte
- *   aligned (no zero-fill needed).  Weights are read in fp32 FMAs (no
+ *   aligned, zero-filled once before its first use (its first word is the
+ *   error word moe_check_error reads and clears).  Weights are read in fp32 FMAs (no
  *   tensor cores: a handful of tokens share a channel); summation order
  *   within a dot product is fixed per launch shape. */
 moe_status_t moe_expert_ffn_channels(const float *x, const uint16_t *Wgate, const uint16_t *Wup,
@@ -368,7 +369,8 @@ void moe_set_wait_limit_ns(uint64_t ns);
 
 /* Synchronises `stream`, then reads and clears the error word that kernels
  * of earlier calls using this workspace may have set (a bounded wait that
- * ran out).  Returns MOE_OK, MOE_ERR_INTERNAL or MOE_ERR_CUDA. */
+ * ran out, or inconsistent token lists); works for the layer workspace and
+ * for the channel path's workspace alike (both start with the word).  Returns MOE_OK, MOE_ERR_INTERNAL or MOE_ERR_CUDA. */
 moe_status_t moe_check_error(void *ws, size_t ws_bytes, void *stream);
 
 /* Static description of a status code (never NULL). */

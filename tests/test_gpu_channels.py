@@ -58,20 +58,20 @@ def _run(S, B, mode, k0, c, seed, ties=False, L=None):
     y_r, keep_r = oracle.ffn_channels(x, L["Wgate"], L["Wup"], L["Wdown"], sel, w, score, c, threads=THREADS)
     t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
     dims = (B, S.d, S.E, S.k, S.F)
-    Wdn = t(L["Wdown"].view(np.int16))
+    # every device buffer stays referenced until the kernels have run
+    Wg_d, Wu_d, Wdn = (t(L[n].view(np.int16)) for n in ("Wgate", "Wup", "Wdown"))
     WdT = torch.empty(S.E, S.F, S.d, dtype=torch.int16, device="cuda")
     lib = moe.load_library()
     assert lib.moe_down_channel_major(Wdn.data_ptr(), moe.Dims(*dims), WdT.data_ptr(), None) == 0
     nbytes = lib.moe_channels_workspace_bytes(moe.Dims(*dims))
     assert nbytes > 0
-    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
     xd, seld, wd, scd = t(x), t(sel), t(w), t(score)
     y = torch.empty(B, S.d, dtype=torch.float32, device="cuda")
     keep = torch.empty(B, S.k, S.F // 32, dtype=torch.int32, device="cuda")
-    st = lib.moe_expert_ffn_channels(xd.data_ptr(), t(L["Wgate"].view(np.int16)).data_ptr(),
-                                     t(L["Wup"].view(np.int16)).data_ptr(), WdT.data_ptr(), moe.Dims(*dims),
-                                     seld.data_ptr(), wd.data_ptr(), scd.data_ptr(), c, y.data_ptr(),
-                                     keep.data_ptr(), ws.data_ptr(), nbytes, None)
+    st = lib.moe_expert_ffn_channels(xd.data_ptr(), Wg_d.data_ptr(), Wu_d.data_ptr(), WdT.data_ptr(),
+                                     moe.Dims(*dims), seld.data_ptr(), wd.data_ptr(), scd.data_ptr(), c,
+                                     y.data_ptr(), keep.data_ptr(), ws.data_ptr(), nbytes, None)
     assert st == 0
     torch.cuda.synchronize()
     assert moe.moe_check_error(ws) == 0
