@@ -163,7 +163,7 @@ moe_lists_t ws_lists(void *ws, const WsLayout &L) {
     return l;
 }
 
-// One layer call (arguments validated): up to 32 tokens the fused kernel,
+// One layer call (arguments validated): up to 64 tokens the fused kernel,
 // above the four chained kernels.  residual: y = x + the experts' output;
 // chained: the layer follows the previous layer of a stack on the stream.
 moe_status_t layer_call(const float *x, const moe_layer_weights_t &w, const moe_dims_t &dims,
@@ -176,9 +176,9 @@ bool encode_expert_maps(ExpertMaps *m, const moe_dims_t &d, const uint16_t *Wgat
                         const uint16_t *Wdown, const uint16_t *h, const uint16_t *x) {
     std::memset(m, 0, sizeof(*m));
     const uint64_t E = d.E, F = d.d_ff, D = d.d;
-    const uint32_t gu_chunks = expert_ffn_gu_chunks(d.d), d_chunks = expert_ffn_d_chunks(d.d_ff);
-    return encode_bf16_chunked(&m->gate, Wgate, E * F, D, expert_ffn_gu_rows(), gu_chunks) &&
-           encode_bf16_chunked(&m->up, Wup, E * F, D, expert_ffn_gu_rows(), gu_chunks) &&
+    const uint32_t gu_chunks = expert_ffn_gu_chunks(d.d, d.B), d_chunks = expert_ffn_d_chunks(d.d_ff);
+    return encode_bf16_chunked(&m->gate, Wgate, E * F, D, expert_ffn_gu_rows(d.B), gu_chunks) &&
+           encode_bf16_chunked(&m->up, Wup, E * F, D, expert_ffn_gu_rows(d.B), gu_chunks) &&
            encode_bf16_chunked(&m->down, Wdown, E * D, F, expert_ffn_d_rows(), d_chunks) &&
            encode_bf16_chunked(&m->h, h,
                                expert_ffn_dense_batch(d.B) ? static_cast<uint64_t>(active_slots(d)) * d.B
@@ -228,7 +228,7 @@ moe_status_t layer_call(const float *x, const moe_layer_weights_t &w, const moe_
                         void *ws, cudaStream_t s, bool residual, bool chained) {
     const WsLayout L = ws_layout(dims);
     const bool dense = expert_ffn_dense_batch(dims.B) != 0;
-    // the expert kernel's x: bf16 x (B <= 32) or the dispatched pair rows
+    // the expert kernel's x: bf16 x (B <= 64) or the dispatched pair rows
     uint16_t *xk = dense ? seg<uint16_t>(ws, L.xb) : seg<uint16_t>(ws, L.xd);
     ExpertMaps maps;
     if (!encode_expert_maps(&maps, dims, w.Wgate, w.Wup, w.Wdown, seg<uint16_t>(ws, L.h), xk)) return MOE_ERR_CUDA;
@@ -241,7 +241,7 @@ moe_status_t layer_call(const float *x, const moe_layer_weights_t &w, const moe_
     float *sw = sel_w ? sel_w : seg<float>(ws, L.sel_w);
     const moe_lists_t lists = ws_lists(ws, L);
     if (dense) {
-        // B <= 32: one persistent kernel for the whole call
+        // B <= 64: one persistent kernel for the whole call
         return from_cuda(launch_layer_fused(maps, rmaps, dims, rule, x, w.bias, logits, probs, xk, y,
                                             seg<uint16_t>(ws, L.h), seg<float>(ws, L.wd), si, sw, lists, n_active,
                                             ctr, residual, chained, s));
@@ -328,7 +328,7 @@ moe_status_t moe_expert_ffn(const float *x, const uint16_t *Wgate, const uint16_
     if (st != MOE_OK) return st;
     const WsLayout L = ws_layout(dims);
     const bool dense = expert_ffn_dense_batch(dims.B) != 0;
-    // the expert kernel's x: bf16 x (B <= 32) or the dispatched pair rows
+    // the expert kernel's x: bf16 x (B <= 64) or the dispatched pair rows
     uint16_t *xk = dense ? seg<uint16_t>(ws, L.xb) : seg<uint16_t>(ws, L.xd);
     ExpertMaps maps;
     if (!encode_expert_maps(&maps, dims, Wgate, Wup, Wdown, seg<uint16_t>(ws, L.h), xk)) return MOE_ERR_CUDA;

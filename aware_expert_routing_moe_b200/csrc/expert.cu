@@ -16,15 +16,16 @@
 // Every CTA takes all its GU units before its D units; a D unit's producer
 // waits (bounded) until its expert's GU units are published done.
 //
-// Dense mode (B <= 32): every unit works on all B tokens of the batch, so
+// Dense mode (B <= 64): every unit works on all B tokens of the batch, so
 // gate/up stages load x for all tokens in one swizzled box, H is indexed by
 // (active slot, token), and the down epilogue weighs each token by a dense
 // [slot][B] weight matrix (0 for tokens that did not choose the expert).
-// Gate/up work then needs only the activated set, which the layer path
-// publishes before the token lists exist (the router kernel: per token
-// group for OEA and plain top-k, once every group is in for the batch-wide
-// rules): the kernel is launched early,
-// reads the set from a published bit mask and starts streaming at once.
+// Gate/up work then needs only the activated set, which the fused layer
+// kernel has before the token lists exist: its CTAs rank the tokens' first
+// experts themselves (OEA, plain top-k) or read the set the selection CTA
+// publishes (the batch-wide rules), and start streaming at once.  From 33
+// to 64 tokens the gate/up units are 32 rows by 256-column stages, and the
+// consumer warps split a stage by (row tile, token tile).
 // Larger batches use tiles of up to 32 (token, expert) pairs: the input
 // preparation copies each pair's x row (bf16) into a pair-indexed buffer in
 // the lists' order, so a tile's x rows are one swizzled box like H's.
@@ -53,8 +54,14 @@ constexpr int NCW = 8;                    // consumer warps
 constexpr int NTHREADS = (NCW + 2) * 32;  // + one producer warp + one signal warp
 constexpr int SIG_SLOTS = 4;              // gate/up completions queued for the signal warp
 constexpr int TN = 32;                    // tokens per tile
+constexpr int DENSE_MAX = 64;             // dense mode (every unit takes the whole batch) up to 64 tokens
 constexpr int GU_ROWS = 16;               // rows of Wgate and of Wup per GU unit
 constexpr int GU_CHUNKS = 8;              // 64-column chunks of d per GU stage (at most)
+// wide dense mode (33..64 tokens): GU units of 32 rows, stages of 4 chunks,
+// so that a stage's weights (32 KB) and its 64 token rows (32 KB) fill a
+// slot of the large ring
+constexpr int WIDE_ROWS = 32;
+constexpr int WIDE_CHUNKS = 4;
 constexpr int D_ROWS = 64;                // rows of Wdown per D unit
 constexpr int D_CHUNKS = 4;               // 64-column chunks of d_ff per D stage (at most)
 constexpr int MAX_STAGES = 4;
@@ -78,6 +85,9 @@ constexpr int smem_bytes() {
 using RingSmallB = Ring<4, 16384>;
 using RingLargeB = Ring<3, 32768>;
 static_assert(2 * GU_ROWS * 128 * GU_CHUNKS <= W_BYTES, "gate/up tiles do not fit");
+static_assert(WIDE_ROWS * 128 * WIDE_CHUNKS == UP_OFF, "wide gate tile must end where the up tile starts");
+static_assert(DENSE_MAX * 128 * WIDE_CHUNKS <= RingLargeB::OP_BYTES, "wide x rows (64 tokens) do not fit");
+static_assert(DENSE_MAX * 128 * D_CHUNKS <= RingLargeB::OP_BYTES, "wide H tile (64 tokens) does not fit");
 static_assert(D_ROWS * 128 * D_CHUNKS <= W_BYTES, "down tile does not fit");
 static_assert(16 * GU_CHUNKS * 128 <= RingSmallB::OP_BYTES, "dense x rows (B <= 16) do not fit");
 static_assert(TN * GU_CHUNKS * 128 <= RingLargeB::OP_BYTES, "x rows (32 tokens) do not fit");
@@ -139,10 +149,15 @@ struct ExpertArgs {
     // early mode: the dense weights are ready once *lists_flag >= 1 (fused
     // layer kernel); null: once the previous kernel has completed
     const int32_t *lists_flag;
-    // dense mode (B <= TN): every stage works on all B tokens; gate/up stages
-    // load all token rows of x in one box, H is token-indexed [slot][B][d_ff]
-    // and the down epilogue weighs tokens by wd[slot][B]
+    // dense mode (B <= DENSE_MAX): every stage works on all B tokens; gate/up
+    // stages load all token rows of x in one box, H is token-indexed
+    // [slot][B][d_ff] and the down epilogue weighs tokens by wd[slot][B]
     int dense;
+    // wide dense mode (B > TN): 32-row gate/up units, and the consumer warps
+    // split each stage by (row tile, token tile) instead of by k
+    int wide;
+    int gu_rows;  // rows of Wgate / Wup per GU unit
+    int gc;       // 64-column chunks of d per GU stage
     int bpad;   // B rounded up to a multiple of 8 (dense mode)
     int hrows;  // rows of one H box (bpad in dense mode, TN otherwise)
     int early;       // start when ctr->pubs[c].pub reaches pub_target, not at the previous kernel's end
@@ -221,7 +236,6 @@ __device__ __forceinline__ void tma_load_3d_stream(void *dst, const CUtensorMap 
         "l"(reinterpret_cast<unsigned long long>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar)), "l"(policy)
         : "memory");
 }
-__device__ __forceinline__ int gu_chunks_of(int d) { return min(GU_CHUNKS, d / 64); }
 __device__ __forceinline__ int d_chunks_of(int F) { return min(D_CHUNKS, F / 64); }
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<unsigned long long>(map)) : "memory");
@@ -330,7 +344,7 @@ __device__ __forceinline__ void decode_rec(int u, int n_units, const ExpertArgs 
         const int i = div_by(v, per, gu ? a.inv_gu : a.inv_d);
         ui.type = gu ? UNIT_GU : UNIT_D;
         ui.ns = gu ? a.ns_gu : (ui.k0 > 0 || u - uc.n_gu >= uc.d_main ? 1 : a.ns_d);
-        ui.row0 = (v - i * per) * (gu ? GU_ROWS : D_ROWS);
+        ui.row0 = (v - i * per) * (gu ? a.gu_rows : D_ROWS);
         ui.i_act = i;
         ui.e = ctl->act_e[i];
         ui.p0 = i * a.B;
@@ -346,8 +360,7 @@ __device__ __forceinline__ void decode_rec(int u, int n_units, const ExpertArgs 
         ui.type = UNIT_GU;
         per = gu_per_tile;
         v = u;
-        const int gk = 64 * gu_chunks_of(a.d);
-        ui.ns = (a.d + gk - 1) / gk;
+        ui.ns = a.ns_gu;
     } else {
         ui.type = UNIT_D;
         per = d_per_tile;
@@ -427,10 +440,10 @@ __device__ void producer(const ExpertArgs &a, const ExpertMaps &m, SharedCtl *ct
             }
             unsigned char *wdst = slots + slot * RG::SLOT_BYTES;
             unsigned char *odst = wdst + W_BYTES;
-            const int gc = gu_chunks_of(a.d), dc = d_chunks_of(a.F);
+            const int gc = a.gc, dc = d_chunks_of(a.F);
             // x tile: all B token rows (dense mode) or the tile's TN pair rows
             const unsigned xbytes = static_cast<unsigned>(gc) * (a.dense ? a.bpad : TN) * 128u;
-            const unsigned bytes = cur.type == UNIT_GU ? 2u * gc * (GU_ROWS * 128) + xbytes
+            const unsigned bytes = cur.type == UNIT_GU ? 2u * gc * (a.gu_rows * 128) + xbytes
                                                        : dc * (D_ROWS * 128u) + dc * (a.hrows * 128u);
             if (lane == 0) {
                 StageHdr &h = ctl->hdr[slot];
@@ -568,11 +581,56 @@ __device__ __forceinline__ void d_stage(uint32_t wbase, uint32_t hbase, int hrow
     }
 }
 
+// Wide dense mode.  Gate/up: warp w takes rows 16 (w / 4) .. + 16 of the
+// 32-row unit and tokens 16 (w % 4) .. + 16 (two n-tiles) over every k-step
+// of the stage, so each (row, token) sum is one warp's own, in k order.
+__device__ __forceinline__ void gu_stage_wide(uint32_t wbase, uint32_t xbase, int x_tile, int kvalid, int warp,
+                                              int lane, float (&acc_g)[4][4], float (&acc_u)[4][4]) {
+    const int nks = kvalid / 16;
+    const int r = (warp >> 2) * 16 + (lane & 15);
+    const int n = (warp & 3) * 16 + (lane & 7) + ((lane >> 4) << 3);
+#pragma unroll 4
+    for (int ks = 0; ks < nks; ++ks) {
+        const int box = ks >> 2;
+        const int chunk = ((ks & 3) << 1) + (lane >> 4);
+        uint32_t g0, g1, g2, g3, u0, u1, u2, u3, b0, b1, b2, b3;
+        ldsm_x4(swz(wbase + box * (WIDE_ROWS * 128), r, chunk), g0, g1, g2, g3);
+        ldsm_x4(swz(wbase + UP_OFF + box * (WIDE_ROWS * 128), r, chunk), u0, u1, u2, u3);
+        ldsm_x4(swz(xbase + box * x_tile, n, ((ks & 3) << 1) + ((lane >> 3) & 1)), b0, b1, b2, b3);
+        mma_bf16(acc_g[0], g0, g1, g2, g3, b0, b1);
+        mma_bf16(acc_g[1], g0, g1, g2, g3, b2, b3);
+        mma_bf16(acc_u[0], u0, u1, u2, u3, b0, b1);
+        mma_bf16(acc_u[1], u0, u1, u2, u3, b2, b3);
+    }
+}
+// Down: warp w takes rows 16 (w % 4) .. + 16 of the 64-row unit and tokens
+// 32 (w / 4) .. + 32 (four n-tiles) over every k-step of the stage.
+__device__ __forceinline__ void d_stage_wide(uint32_t wbase, uint32_t hbase, int hrows, int kvalid, int warp,
+                                             int lane, float (&acc)[4][4]) {
+    const int nks = kvalid / 16;
+    const int r = (warp & 3) * 16 + (lane & 15);
+#pragma unroll 4
+    for (int ks = 0; ks < nks; ++ks) {
+        const int box = ks >> 2;
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(swz(wbase + box * (D_ROWS * 128), r, ((ks & 3) << 1) + (lane >> 4)), a0, a1, a2, a3);
+        const int hchunk = ((ks & 3) << 1) + ((lane >> 3) & 1);
+#pragma unroll
+        for (int np = 0; np < 2; ++np) {
+            const int n = (warp >> 2) * 32 + np * 16 + (lane & 7) + ((lane >> 4) << 3);
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4(swz(hbase + box * (hrows * 128), n, hchunk), b0, b1, b2, b3);
+            mma_bf16(acc[2 * np], a0, a1, a2, a3, b0, b1);
+            mma_bf16(acc[2 * np + 1], a0, a1, a2, a3, b2, b3);
+        }
+    }
+}
+
 template <int NT>
 __device__ __forceinline__ void stage_dispatch(const StageHdr &h, uint32_t wbase, uint32_t obase, const ExpertArgs &a,
                                                int warp, int lane, float (&acc_g)[4][4], float (&acc_u)[4][4]) {
     if (h.type == UNIT_GU) {
-        const int gk = 64 * gu_chunks_of(a.d);
+        const int gk = 64 * a.gc;
         gu_stage<NT>(wbase, obase, (a.dense ? a.bpad : TN) * 128, min(gk, a.d - h.k * gk), warp, lane, acc_g, acc_u);
     } else {
         const int dk = 64 * d_chunks_of(a.F);
@@ -639,11 +697,13 @@ __device__ void consumer(const ExpertArgs &a, SharedCtl *ctl, unsigned char *slo
                     }
                     lists_ready = true;
                 }
+                // wide mode: this warp's tokens start at 32 (warp / 4)
+                const int tb = a.wide ? (warp >> 2) * 32 : 0;
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
 #pragma unroll
                     for (int c = 0; c < 2; ++c) {
-                        const int t = j * 8 + col + c;
+                        const int t = tb + j * 8 + col + c;
                         tk[j][c] = t;
                         wk[j][c] = t < a.B ? __ldcg(a.wd + static_cast<size_t>(h.i_act) * a.B + t) : 0.0f;
                     }
@@ -666,12 +726,22 @@ __device__ void consumer(const ExpertArgs &a, SharedCtl *ctl, unsigned char *slo
         }
         const uint32_t wbase = smem_u32(slots + slot * RG::SLOT_BYTES);
         const uint32_t obase = wbase + W_BYTES;
-        const int nt = (h.type == UNIT_GU && a.dense) ? (a.bpad >> 3) : ((h.n + 7) >> 3);
-        switch (nt) {
-            case 1: stage_dispatch<1>(h, wbase, obase, a, warp, lane, acc_g, acc_u); break;
-            case 2: stage_dispatch<2>(h, wbase, obase, a, warp, lane, acc_g, acc_u); break;
-            case 3: stage_dispatch<3>(h, wbase, obase, a, warp, lane, acc_g, acc_u); break;
-            default: stage_dispatch<4>(h, wbase, obase, a, warp, lane, acc_g, acc_u); break;
+        const int nt = a.wide ? 4 : (h.type == UNIT_GU && a.dense) ? (a.bpad >> 3) : ((h.n + 7) >> 3);
+        if (a.wide) {
+            if (h.type == UNIT_GU) {
+                const int gk = 64 * a.gc;
+                gu_stage_wide(wbase, obase, a.bpad * 128, min(gk, a.d - h.k * gk), warp, lane, acc_g, acc_u);
+            } else {
+                const int dk = 64 * d_chunks_of(a.F);
+                d_stage_wide(wbase, obase, a.hrows, min(dk, a.F - h.k * dk), warp, lane, acc_g);
+            }
+        } else {
+            switch (nt) {
+                case 1: stage_dispatch<1>(h, wbase, obase, a, warp, lane, acc_g, acc_u); break;
+                case 2: stage_dispatch<2>(h, wbase, obase, a, warp, lane, acc_g, acc_u); break;
+                case 3: stage_dispatch<3>(h, wbase, obase, a, warp, lane, acc_g, acc_u); break;
+                default: stage_dispatch<4>(h, wbase, obase, a, warp, lane, acc_g, acc_u); break;
+            }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctl->empty[slot]);
@@ -679,15 +749,36 @@ __device__ void consumer(const ExpertArgs &a, SharedCtl *ctl, unsigned char *slo
         if (h.s != h.ns - 1) continue;
 
         // ---- unit epilogue
-        if (h.type == UNIT_D) {
-            // each warp holds a k-half of a 16-row block: both halves add into y
+        if (h.type == UNIT_GU && a.wide) {
+            // each warp owns complete sums: h = silu(g) u straight to H
+            const int r0 = h.row0 + (warp >> 2) * 16 + row;
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int t = (warp & 3) * 16 + j * 8 + col + (c & 1);
+                    if (t < a.B) {
+                        const float gs = acc_g[j][c], us = acc_u[j][c];
+                        const float hv = gs / (1.0f + __expf(-gs)) * us;
+                        a.h[static_cast<size_t>(h.p0 + t) * a.F + r0 + ((c >> 1) << 3)] =
+                            __bfloat16_as_ushort(__float2bfloat16_rn(hv));
+                    }
+                }
+            // H is read by other CTAs through TMA (the async proxy)
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+            consumer_bar();
+            if (ct == 0 && !post_signal(ctl, a.ctr, nsig++, h.i_act)) return;
+        } else if (h.type == UNIT_D) {
+            // each warp holds a k-half of a 16-row block (wide mode: all of k
+            // for 32 tokens): both halves add into y
             const int i_base = h.row0 + (warp & 3) * 16 + row;
+            const int tb = a.wide ? (warp >> 2) * 32 : 0;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 if (j >= nt) break;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    const int n = j * 8 + col + (c & 1);
+                    const int n = tb + j * 8 + col + (c & 1);
                     if (n < h.n && wk[j][c & 1] != 0.0f) {
                         const int i = i_base + ((c >> 1) << 3);
                         atomicAdd(a.y + static_cast<size_t>(tk[j][c & 1]) * a.d + i, wk[j][c & 1] * acc_g[j][c]);
@@ -994,7 +1085,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 }
 
 // ------------------------------------------------------ fused layer kernel --
-// One persistent grid for the whole layer call when B <= 32 (dense mode),
+// One persistent grid for the whole layer call when B <= 64 (dense mode),
 // one CTA per SM, launched cooperatively so that every CTA is resident:
 //  1. router: the CTAs compute the logits in items of (epb experts) x (tpb
 //     tokens) with the router's fixed-order dot products (rows staged by
@@ -1218,7 +1309,7 @@ struct PrepArgs {
     Counters *ctr; // gate/up counts cleared when non-null
     const int32_t *n_active, *offsets, *tok;
     const float *w;
-    float *wd;  // dense weights [slot][B] (B <= 32), or null
+    float *wd;  // dense weights [slot][B] (B <= 64), or null
     int32_t *err;  // error word for inconsistent lists, or null
 };
 
@@ -1263,19 +1354,20 @@ __global__ void __launch_bounds__(256) ffn_prep_kernel(PrepArgs p) {
     }
     if (p.wd) {
         // wd[i][t] = weight of token t in active expert i's list, else 0:
-        // one warp per active expert (its list holds at most B <= 32 pairs)
+        // one warp per active expert (its list holds at most B <= 64 pairs)
         const int na0 = *p.n_active;
         const int na = (na0 > 0 && na0 <= p.slots) ? na0 : 0;
         const int lane = threadIdx.x & 31;
         for (int i = tid >> 5; i < na; i += nthreads >> 5) {
             const int j0 = min(max(p.offsets[i], 0), pairs);
-            const int n = min(max(p.offsets[i + 1], j0), pairs) - j0;
-            const int t = lane < n ? p.tok[j0 + lane] : -1;
-            const float wv = lane < n ? p.w[j0 + lane] : 0.0f;
-            if (lane < p.B) p.wd[static_cast<size_t>(i) * p.B + lane] = 0.0f;
+            const int n = min(min(max(p.offsets[i + 1], j0), pairs) - j0, p.B);
+            for (int t = lane; t < p.B; t += 32) p.wd[static_cast<size_t>(i) * p.B + t] = 0.0f;
             __syncwarp();
-            if (t >= 0 && t < p.B) p.wd[static_cast<size_t>(i) * p.B + t] = wv;
-            else if (lane < n && p.err) atomicCAS(p.err, 0, DEV_BAD_LISTS);  // pair skipped
+            for (int q = lane; q < n; q += 32) {
+                const int t = p.tok[j0 + q];
+                if (t >= 0 && t < p.B) p.wd[static_cast<size_t>(i) * p.B + t] = p.w[j0 + q];
+                else if (p.err) atomicCAS(p.err, 0, DEV_BAD_LISTS);  // pair skipped
+            }
         }
     }
     if (p.ctr && blockIdx.x == 0)
@@ -1320,11 +1412,14 @@ int g_num_sms[MAX_DEVICES] = {0};
 
 }  // namespace
 
-int expert_ffn_h_rows(int B) { return B <= TN ? (B + 7) / 8 * 8 : TN; }
-int expert_ffn_dense_batch(int B) { return B <= TN ? 1 : 0; }
-int expert_ffn_gu_rows() { return GU_ROWS; }
+int expert_ffn_h_rows(int B) { return B <= DENSE_MAX ? (B + 7) / 8 * 8 : TN; }
+int expert_ffn_dense_batch(int B) { return B <= DENSE_MAX ? 1 : 0; }
+int expert_ffn_gu_rows(int B) { return B > TN && B <= DENSE_MAX ? WIDE_ROWS : GU_ROWS; }
 int expert_ffn_d_rows() { return D_ROWS; }
-int expert_ffn_gu_chunks(int d) { return d / 64 < GU_CHUNKS ? d / 64 : GU_CHUNKS; }
+int expert_ffn_gu_chunks(int d, int B) {
+    const int cap = B > TN && B <= DENSE_MAX ? WIDE_CHUNKS : GU_CHUNKS;
+    return d / 64 < cap ? d / 64 : cap;
+}
 int expert_ffn_d_chunks(int F) { return F / 64 < D_CHUNKS ? F / 64 : D_CHUNKS; }
 
 cudaError_t launch_ffn_prep(const float *x, const moe_dims_t &d, uint16_t *xb, uint16_t *xd, float *y,
@@ -1411,15 +1506,18 @@ ExpertArgs make_expert_args(const uint16_t *xb, const moe_dims_t &d, const moe_l
     a.wait_ns = wait_limit_ns();
     a.unit_ctas = unit_ctas;
     a.lists_flag = nullptr;
-    a.dense = d.B <= TN ? 1 : 0;
+    a.dense = d.B <= DENSE_MAX ? 1 : 0;
+    a.wide = d.B > TN && d.B <= DENSE_MAX ? 1 : 0;
+    a.gu_rows = expert_ffn_gu_rows(d.B);
+    a.gc = expert_ffn_gu_chunks(d.d, d.B);
     a.bpad = (d.B + 7) / 8 * 8;
     a.hrows = expert_ffn_h_rows(d.B);
     a.early = 0;
     a.pub_target = 0;
-    a.gu_per_tile = d.d_ff / GU_ROWS;
+    a.gu_per_tile = d.d_ff / a.gu_rows;
     a.d_per_tile = d.d / D_ROWS;
     {
-        const int gk = 64 * expert_ffn_gu_chunks(d.d), dk = 64 * expert_ffn_d_chunks(d.d_ff);
+        const int gk = 64 * a.gc, dk = 64 * expert_ffn_d_chunks(d.d_ff);
         a.ns_gu = (d.d + gk - 1) / gk;
         a.ns_d = (d.d_ff + dk - 1) / dk;
     }
@@ -1530,7 +1628,7 @@ cudaError_t launch_layer_fused(const ExpertMaps &maps, const RouterMaps &rmaps, 
                                float *probs, uint16_t *xb, float *y, uint16_t *h, float *wd, int32_t *sel_idx,
                                float *sel_w, const moe_lists_t &lists, int32_t *n_active_copy, Counters *ctr,
                                bool residual, bool chained, cudaStream_t s) {
-    if (d.B > TN) return cudaErrorInvalidValue;
+    if (d.B > DENSE_MAX) return cudaErrorInvalidValue;
     int dev = 0, sms = 0;
     cudaError_t err = device_sms(&dev, &sms);
     if (err != cudaSuccess) return err;

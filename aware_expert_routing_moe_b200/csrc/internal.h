@@ -60,20 +60,23 @@ struct WsLayout {
 
 // Activated-expert slots a call can have: min(E, B*k).
 inline int active_slots(const moe_dims_t &d) { return d.E < d.B * d.k ? d.E : d.B * d.k; }
+// Batches up to this many tokens run the dense mode: every unit takes the
+// whole batch (the tokens that did not choose the expert weigh 0).
+constexpr int DENSE_B_MAX = 64;
 // Bytes of the expert kernel's H scratch: token-indexed [slot][B][d_ff]
-// when the batch is small enough for dense gate/up stages (B <= 32), else
-// pair-indexed [B*k][d_ff]; bf16.
+// in dense mode (B <= 64), else pair-indexed [B*k][d_ff]; bf16.
 inline size_t h_scratch_bytes(const moe_dims_t &d) {
     const size_t F = d.d_ff;
-    return d.B <= 32 ? static_cast<size_t>(active_slots(d)) * d.B * F * 2 : static_cast<size_t>(d.B) * d.k * F * 2;
+    return d.B <= DENSE_B_MAX ? static_cast<size_t>(active_slots(d)) * d.B * F * 2
+                              : static_cast<size_t>(d.B) * d.k * F * 2;
 }
-// Bytes of the dispatched x rows [B*k][d] bf16 (B > 32 only).
+// Bytes of the dispatched x rows [B*k][d] bf16 (B > 64 only).
 inline size_t xd_bytes(const moe_dims_t &d) {
-    return d.B <= 32 ? 0 : static_cast<size_t>(d.B) * d.k * d.d * 2;
+    return d.B <= DENSE_B_MAX ? 0 : static_cast<size_t>(d.B) * d.k * d.d * 2;
 }
-// Bytes of the dense weight matrix [slot][B] fp32 (B <= 32 only).
+// Bytes of the dense weight matrix [slot][B] fp32 (B <= 64 only).
 inline size_t wd_bytes(const moe_dims_t &d) {
-    return d.B <= 32 ? static_cast<size_t>(active_slots(d)) * d.B * 4 : 0;
+    return d.B <= DENSE_B_MAX ? static_cast<size_t>(active_slots(d)) * d.B * 4 : 0;
 }
 
 WsLayout ws_layout(const moe_dims_t &d);
@@ -96,37 +99,37 @@ cudaError_t launch_route_topk(const float *logits, const moe_dims_t &d, float *p
 cudaError_t launch_reselect(const float *logits, const float *probs, const moe_dims_t &d,
                             const moe_reselect_t &r, int32_t *sel_idx, float *sel_w,
                             const moe_lists_t &l, cudaStream_t s);
-// Layer path above 32 tokens, first kernel: router GEMV; also sets y = 0
+// Layer path above 64 tokens, first kernel: router GEMV; also sets y = 0
 // (y = x with residual).  chained: launched with programmatic dependent
 // launch after the previous layer of a stack.
 cudaError_t launch_layer_route(const RouterMaps &maps, const float *x, const float *bias, const moe_dims_t &d,
                                float *logits, float *y, Counters *ctr, bool residual, bool chained, cudaStream_t s);
-// Layer path above 32 tokens, second kernel (chained with programmatic
+// Layer path above 64 tokens, second kernel (chained with programmatic
 // dependent launch): softmax, selection, lists.
 cudaError_t launch_layer_select(const float *logits, float *probs, const moe_dims_t &d, const moe_reselect_t &rule,
                                 int32_t *sel_idx, float *sel_w, const moe_lists_t &l, int32_t *n_active_copy,
                                 cudaStream_t s);
 // Input preparation of the expert kernel (all pointers may be null, each
 // step is skipped then): x -> bf16 (xb, dense mode), each pair's x row ->
-// xd (larger batches), y = 0, gate/up counts cleared and, for B <= 32, the
+// xd (larger batches), y = 0, gate/up counts cleared and, for B <= 64, the
 // dense weights built from the lists.  chained: launched with programmatic
 // dependent launch after the kernel that writes the lists.
 cudaError_t launch_ffn_prep(const float *x, const moe_dims_t &d, uint16_t *xb, uint16_t *xd, float *y,
                             Counters *ctr, const moe_lists_t &l, float *wd, bool chained, cudaStream_t s);
 
 // TMA descriptors of the expert kernel: the three weight tensors, the H
-// scratch and the bf16 x rows (xb for B <= 32, the dispatched pair rows xd
+// scratch and the bf16 x rows (xb for B <= 64, the dispatched pair rows xd
 // above) as (64-column chunk, row, chunk index) boxes.
 struct ExpertMaps {
     CUtensorMap gate, up, down, h, x;
 };
 // The expert kernel alone (moe_expert_ffn): lists from the previous kernel
 // (chained with programmatic dependent launch) or the caller; wd: dense
-// weights (B <= 32).
+// weights (B <= 64).
 cudaError_t launch_expert_ffn(const ExpertMaps &maps, const uint16_t *xb, const moe_dims_t &d,
                               const moe_lists_t &l, float *y, uint16_t *h, const float *wd, Counters *ctr,
                               cudaStream_t s);
-// The whole layer in one cooperative persistent kernel (B <= 32): router,
+// The whole layer in one cooperative persistent kernel (B <= 64): router,
 // grid barrier, selection (last CTA), expert stream (the other CTAs).  xb:
 // x in bf16 (written), h: the SwiGLU scratch, wd: the dense weights.
 // residual: y = x + the experts' output; chained: launched with
@@ -150,13 +153,13 @@ cudaError_t launch_channels(const float *x, const uint16_t *Wgate, const uint16_
 unsigned long long wait_limit_ns();
 int expert_ffn_h_rows(int B);         // rows of one H box
 int expert_ffn_dense_batch(int B);    // 1 if gate/up stages load all B token rows at once
-int expert_ffn_gu_rows();             // rows of Wgate / Wup per gate-up unit
+int expert_ffn_gu_rows(int B);        // rows of Wgate / Wup per gate-up unit
 int expert_ffn_d_rows();              // rows of Wdown per down unit
-int expert_ffn_gu_chunks(int d);      // 64-column chunks of d per gate-up stage
+int expert_ffn_gu_chunks(int d, int B);  // 64-column chunks of d per gate-up stage
 int expert_ffn_d_chunks(int d_ff);    // 64-column chunks of d_ff per down stage
 
 // Builds the expert kernel's TMA descriptors (weights, H scratch at `h`,
-// bf16 x at `x`: xb [B][d] for B <= 32, xd [B*k][d] above).
+// bf16 x at `x`: xb [B][d] for B <= 64, xd [B*k][d] above).
 bool encode_expert_maps(ExpertMaps *m, const moe_dims_t &d, const uint16_t *Wgate, const uint16_t *Wup,
                         const uint16_t *Wdown, const uint16_t *h, const uint16_t *x);
 

@@ -97,7 +97,7 @@ extern "C" moe_status_t moe_expert_ffn_noalloc(const float *x, const uint16_t *W
 
     Counters *ctr = reinterpret_cast<Counters *>(scratch + L.counters);
     const bool dense = expert_ffn_dense_batch(dims.B) != 0;
-    // the expert kernel's x: bf16 x (B <= 32) or the dispatched pair rows
+    // the expert kernel's x: bf16 x (B <= 64) or the dispatched pair rows
     uint16_t *xk = reinterpret_cast<uint16_t *>(scratch + (dense ? L.xb : L.xd));
     uint16_t *h = reinterpret_cast<uint16_t *>(scratch + L.h);
     float *wd = dense ? reinterpret_cast<float *>(scratch + L.wd) : nullptr;

@@ -2,8 +2,8 @@
 //
 //  route_gemv_kernel    : logits = x Wg^T + bias in a fixed fp32 order
 //      ("Router Caching and Optimization", "Analyzing Router Inference Cost",
-//      step 1).  In the layer path for batches above 32 tokens it also
-//      zeroes y.  (Batches up to 32 tokens run the whole layer in the fused
+//      step 1).  In the layer path for batches above 64 tokens it also
+//      zeroes y.  (Batches up to 64 tokens run the whole layer in the fused
 //      kernel of expert.cu, which uses the same dot products.)
 //  route_topk_kernel    : warp per token: softmax (step 2) + top-k (step 3)
 //      with a warp-shuffle reduction and register-resident keys.
@@ -83,7 +83,7 @@ __global__ void __launch_bounds__(1024, 1) reselect_kernel(ReselectArgs a) {
 // block's tokens over its columns, chunk by chunk, the tokens' chains
 // interleaved.
 //
-// Layer path for batches above 32 tokens (y != null): while the loads are
+// Layer path for batches above 64 tokens (y != null): while the loads are
 // in flight the blocks zero y, into which the expert kernel adds.
 struct GemvArgs {
     const float *bias;

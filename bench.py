@@ -14,7 +14,7 @@ every call.
 
 Printed (rank 0, one JSON line): value = algorithmic bytes of all ranks per
 second (activated experts x 3 d d_ff x 2 B + router weights + x + y), the
-roofline of the dominant kernel (up to 32 tokens the fused layer kernel,
+roofline of the dominant kernel (up to 64 tokens the fused layer kernel,
 which is the whole call; above, the expert kernel, timed with events
 around moe_expert_ffn), the oracle
 timed on the host cores (cpu_baseline), an end-to-end number through the
@@ -351,7 +351,7 @@ def run_ours(args, w, rank, world, local_rank):
     hbm_peak, peak_kind = measured_peaks()
     ffn_gbs = ffn_bytes / (ms_ffn * 1e-3) / 1e9
     layer_gbs = total_bytes / (ms_step * 1e-3) / 1e9
-    if B <= 32:
+    if B <= 64:
         # one kernel per call: the fused layer kernel is the dominant kernel,
         # timed by the main region itself
         roofline = {"bound": "hbm", "achieved": layer_gbs, "peak": hbm_peak, "unit": "GB/s",
@@ -429,7 +429,7 @@ def run_ours(args, w, rank, world, local_rank):
                    "parallelism": f"replicas x{world}",
                    "l2": f"inputs larger than L2: {ROTATE} rotating copies of the layer weights "
                          f"({3 * S.E * S.d * S.F * 2 / 1e9:.2f} GB of experts + the router each)",
-                   "launch": ("CUDA graph of 4 layer calls, one cooperative kernel per call" if B <= 32 else
+                   "launch": ("CUDA graph of 4 layer calls, one cooperative kernel per call" if B <= 64 else
                               "CUDA graph of 4 layer calls, 4 kernels per call chained with PDL")},
         "us_per_call": ms_step * 1e3,
         "frac_of_nominal_8tbs": (total_bytes / (ms_step * 1e-3) / 1e9) / NOMINAL_HBM_GBS,
@@ -439,9 +439,9 @@ def run_ours(args, w, rank, world, local_rank):
         "expert_ffn_leg": expert_leg,
         "stack_leg": stack,
         "e2e": e2e,
-        # up to 32 tokens one fused kernel per call; above, router,
+        # up to 64 tokens one fused kernel per call; above, router,
         # selection, x dispatch and expert kernels
-        "gpu_launches": (1 if B <= 32 else 4) * args.steps,
+        "gpu_launches": (1 if B <= 64 else 4) * args.steps,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -211,7 +211,7 @@ moe_status_t moe_expert_ffn(const float *x, const uint16_t *Wgate,
  * leaves the GPU): the re-routing step sits between the router and the
  * experts and intercepts the router's output ("Lynx: Enabling Efficient MoE
  * Inference through Dynamic Batch-Aware Expert Selection", section 2.2).
- * Up to 32 tokens the call is one persistent kernel (router, a grid-wide
+ * Up to 64 tokens the call is one persistent kernel (router, a grid-wide
  * barrier, selection and expert stream); above, four kernels chained with
  * programmatic dependent launch.  Arguments as above; y[B][d] is
  * overwritten.
@@ -331,7 +331,7 @@ moe_status_t moe_expert_ffn_channels(const float *x, const uint16_t *Wgate, cons
  * allocating routine.
  *
  *  - Size limit: the scratch must fit in MOE_NOALLOC_SCRATCH_BYTES: when
- *    B <= 32, B*d*2 bytes of bf16 x, min(E, B*k)*B*d_ff*2 bytes of SwiGLU
+ *    B <= 64, B*d*2 bytes of bf16 x, min(E, B*k)*B*d_ff*2 bytes of SwiGLU
  *    activations and min(E, B*k)*B*4 bytes of dense weights; above,
  *    B*k*d*2 bytes of per-pair x rows and B*k*d_ff*2 bytes of activations;
  *    plus about 7 KB of counters, each part rounded up to 256 bytes.  Larger

@@ -88,12 +88,14 @@ def test_status_strings(lib):
 def test_workspace_bytes(lib):
     q30 = moe.moe_workspace_bytes(16, 2048, 128, 8, 768)
     assert q30 > 0 and q30 % 256 == 0
-    # B <= 32: token-indexed activations [min(E, B*k)][B][d_ff] bf16 + dense weights
+    # B <= 64: token-indexed activations [min(E, B*k)][B][d_ff] bf16 + dense weights
     assert q30 >= 128 * 16 * 768 * 2 + 128 * 16 * 4
-    # larger batches: pair-indexed activations [B*k][d_ff] bf16
     q30_64 = moe.moe_workspace_bytes(64, 2048, 128, 8, 768)
-    assert q30_64 >= 64 * 8 * 768 * 2 + 64 * 2048 * 2
-    assert q30_64 < 128 * 64 * 768 * 2
+    assert q30_64 >= 128 * 64 * 768 * 2 + 128 * 64 * 4
+    # larger batches: pair-indexed activations [B*k][d_ff] bf16 + dispatched x rows
+    q30_65 = moe.moe_workspace_bytes(65, 2048, 128, 8, 768)
+    assert q30_65 >= 65 * 8 * 768 * 2 + 65 * 8 * 2048 * 2
+    assert q30_65 < 128 * 65 * 768 * 2
     assert moe.moe_workspace_bytes(16, 4096, 128, 8, 1536) > q30
     for bad in [(0, 2048, 128, 8, 768), (257, 2048, 128, 8, 768), (16, 2048, 128, 0, 768),
                 (16, 2048, 128, 17, 768), (16, 2048, 7, 8, 768), (16, 2048, 257, 8, 768),

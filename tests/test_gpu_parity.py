@@ -188,8 +188,12 @@ def test_layer_decode_parity_small(name, B, seed, mode, k0, budget):
 
 Q30_CASES = [(1, NONE, 0, 0), (1, OEA, 2, 0), (4, OEA, 4, 0), (16, NONE, 0, 0), (16, OEA, 2, 0),
              (16, OEA, 4, 0), (16, OEA, 6, 0), (16, OEA, 8, 0), (16, XSHARE, 0, 16), (16, AFFINITY, 0, 0),
-             (64, AFFINITY, 0, 0), (32, NONE, 0, 0),
-             (64, NONE, 0, 0), (64, OEA, 4, 0)]
+             (64, AFFINITY, 0, 0), (32, NONE, 0, 0), (17, OEA, 4, 0),
+             # 33..64 tokens: the wide dense mode (ragged token counts included)
+             (33, OEA, 4, 0), (48, NONE, 0, 0), (57, XSHARE, 0, 40),
+             (64, NONE, 0, 0), (64, OEA, 4, 0),
+             # above 64 tokens: token tiles of dispatched pairs
+             (65, OEA, 4, 0), (96, NONE, 0, 0)]
 
 
 @pytest.mark.parametrize("B,mode,k0,budget", Q30_CASES)
@@ -219,8 +223,8 @@ HIER_LAYER_CASES = [("q30b", 16, 4, 16), ("q30b", 16, 3, 24), ("q30b", 32, 4, 24
 
 @pytest.mark.parametrize("name,B,group,budget", HIER_LAYER_CASES)
 def test_layer_decode_parity_xshare_hier(name, B, group, budget):
-    # B <= 32: the router publishes the batch set and the expert kernel
-    # starts early; larger batches take the dispatch path
+    # B <= 64: the fused kernel's selection CTA publishes the batch set and
+    # the other CTAs stream from it; larger batches take the dispatch path
     kind = "spec" if name == "q30b" and B % 8 == 0 else "normal"
     S, L, x, y, sel, selw, n_act = _run_layer(name, B, 0, XSHARE_HIER, 0, budget, kind=kind, group=group)
     rows = None if B <= 64 else np.arange(0, B, 7, dtype=np.int32)
