@@ -1133,9 +1133,50 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     __shared__ unsigned s_set[E_MAX / 32];
     __shared__ int s_ok;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    unsigned char *wrows = sm.slots;
+    unsigned char *xrows = sm.slots + L.epb * L.row_bytes;
+    const int lines = a.d >> 5;  // 128-byte lines per row
+    // the router's row copies of this CTA's first item come first: they are
+    // the head of the call's critical path (the router weights do not depend
+    // on a previous layer; the token rows, in a stack, do)
+    auto issue_rows = [&](int item, bool weights, bool tokens) {
+        const int eg = item % L.n_eg, tg = item / L.n_eg;
+        const int e0 = eg * L.epb, b0 = tg * L.tpb;
+        const int ne = min(L.epb, a.E - e0), nb = min(L.tpb, a.B - b0);
+        if (weights) {
+            unsigned long long keep;
+            asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(keep));
+            for (int r = 0; r < ne; ++r)
+                for (int bx = 0; bx < L.boxes; ++bx)
+                    tma_rows_hint(wrows + r * L.row_bytes + bx * L.box_lines * 128, &rmaps.wg,
+                                  (e0 + r) * lines + bx * L.box_lines, &s_rbar, keep);
+        }
+        if (tokens)
+            for (int r = 0; r < nb; ++r)
+                for (int bx = 0; bx < L.boxes; ++bx)
+                    tma_rows(xrows + r * L.row_bytes + bx * L.box_lines * 128, &rmaps.x,
+                             (b0 + r) * lines + bx * L.box_lines, &s_rbar);
+    };
+    auto item_bytes = [&](int item, bool weights) {
+        const int eg = item % L.n_eg, tg = item / L.n_eg;
+        const int n = weights ? min(L.epb, a.E - eg * L.epb) : min(L.tpb, a.B - tg * L.tpb);
+        return static_cast<unsigned>(n * L.boxes * L.box_lines * 128);
+    };
+    bool waited = !L.chained;
     if (threadIdx.x == 0) {
-        ctl_init<RG>(ctl, a.wait_ns);
         mbar_init(&s_rbar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        if (static_cast<int>(blockIdx.x) < L.n_items) {
+            const int item = blockIdx.x;
+            if (waited) {
+                mbar_expect_tx(&s_rbar, item_bytes(item, true) + item_bytes(item, false));
+                issue_rows(item, true, true);
+            } else {
+                mbar_add_tx(&s_rbar, item_bytes(item, true));
+                issue_rows(item, true, false);
+            }
+        }
+        ctl_init<RG>(ctl, a.wait_ns);
         s_ok = 1;
     }
     if (threadIdx.x < E_MAX / 32) s_set[threadIdx.x] = 0u;
@@ -1151,37 +1192,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     // ---- 1. router items (one per CTA when there are no more items than CTAs)
-    unsigned char *wrows = sm.slots;
-    unsigned char *xrows = sm.slots + L.epb * L.row_bytes;
     bool prepped = false;
-    bool waited = !L.chained;
     int phase = 0;
-    const int lines = a.d >> 5;  // 128-byte lines per row
     for (int item = blockIdx.x; item < L.n_items; item += gridDim.x) {
         const int eg = item % L.n_eg, tg = item / L.n_eg;
         const int e0 = eg * L.epb, b0 = tg * L.tpb;
         const int ne = min(L.epb, a.E - e0), nb = min(L.tpb, a.B - b0);
-        const unsigned wbytes = static_cast<unsigned>(ne * L.boxes * L.box_lines * 128);
-        const unsigned xbytes = static_cast<unsigned>(nb * L.boxes * L.box_lines * 128);
-        if (threadIdx.x == 0) {
-            // the router weights first: they do not depend on the previous layer
-            if (waited) mbar_expect_tx(&s_rbar, wbytes + xbytes);
-            else mbar_add_tx(&s_rbar, wbytes);
-            for (int r = 0; r < ne; ++r)
-                for (int bx = 0; bx < L.boxes; ++bx)
-                    tma_rows(wrows + r * L.row_bytes + bx * L.box_lines * 128, &rmaps.wg,
-                             (e0 + r) * lines + bx * L.box_lines, &s_rbar);
+        if (item != static_cast<int>(blockIdx.x) && threadIdx.x == 0) {
+            // a later item: the staging area was freed at the end of the last one
+            mbar_expect_tx(&s_rbar, item_bytes(item, true) + item_bytes(item, false));
+            issue_rows(item, true, true);
         }
         if (!waited) {
             asm volatile("griddepcontrol.wait;" ::: "memory");
             waited = true;
-            if (threadIdx.x == 0) mbar_expect_tx(&s_rbar, xbytes);
-        }
-        if (threadIdx.x == 0) {
-            for (int r = 0; r < nb; ++r)
-                for (int bx = 0; bx < L.boxes; ++bx)
-                    tma_rows(xrows + r * L.row_bytes + bx * L.box_lines * 128, &rmaps.x,
-                             (b0 + r) * lines + bx * L.box_lines, &s_rbar);
+            if (threadIdx.x == 0) {
+                mbar_expect_tx(&s_rbar, item_bytes(item, false));
+                issue_rows(item, false, true);
+            }
         }
         if (!prepped) {
             // x -> bf16 (read by the gate/up copies) and y = 0 or x (the
@@ -1234,7 +1262,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
     // ---- 2. grid barrier
     if (threadIdx.x == 0) {
-        __threadfence();
+        // the CTA barrier above orders the CTA's writes before this thread's
+        // release, which makes them visible at gpu scope
         asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(&a.ctr->arrive), "r"(1) : "memory");
         const unsigned long long t0 = global_ns();
         while (ld_acquire(&a.ctr->arrive) < static_cast<int>(gridDim.x)) {
@@ -1253,32 +1282,41 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (blockIdx.x == gridDim.x - 1) {
         if (ok) reselect_body<NI>(L.sel, sm.slots);
         __syncthreads();
-        if (threadIdx.x == 0) {
-            __threadfence();
+        if (threadIdx.x == 0)
             asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(&a.ctr->lists_ready), "r"(1) : "memory");
-        }
         cta_exit(a, ctl);
         return;
     }
 
     // ---- 4. the activated set, then the expert stream
     if (L.r1 > 0) {
+        // two tokens per warp at a time, their arg-max rounds interleaved
+        // (independent reductions overlap); only the union is kept, so the
+        // order of a token's winners does not matter
         if (warp < NCW && ok) {
 #pragma unroll 1
-            for (int b = warp; b < a.B; b += NCW) {
-                float l[NI];
-                unsigned ord[NI];
+            for (int b = warp; b < a.B; b += 2 * NCW) {
+                const int b2 = b + NCW;
+                const bool two = b2 < a.B;
+                float l[NI], l2[NI];
+                unsigned ord[NI], ord2[NI];
                 load_row<NI>(L.logits + static_cast<size_t>(b) * a.E, a.E, lane, l);
+                load_row<NI>(L.logits + static_cast<size_t>(two ? b2 : b) * a.E, a.E, lane, l2);
 #pragma unroll
-                for (int i = 0; i < NI; ++i) ord[i] = ord_of(l[i]);
-                unsigned cand = valid_bits<NI>(a.E, lane);
-                int mye = -1;
+                for (int i = 0; i < NI; ++i) {
+                    ord[i] = ord_of(l[i]);
+                    ord2[i] = ord_of(l2[i]);
+                }
+                unsigned cand = valid_bits<NI>(a.E, lane), cand2 = cand;
+                unsigned mine = 0u;  // bit j: lane's expert-word hits (set below)
 #pragma unroll 1
                 for (int j = 0; j < L.r1; ++j) {
                     const int e = warp_argmax<NI>(ord, cand, lane);
-                    if (lane == j) mye = e;
+                    const int e2 = warp_argmax<NI>(ord2, cand2, lane);
+                    if (e >= 0 && (e >> 5) == lane) mine |= 1u << (e & 31);
+                    if (two && e2 >= 0 && (e2 >> 5) == lane) mine |= 1u << (e2 & 31);
                 }
-                if (lane < L.r1 && mye >= 0) atomicOr(&s_set[mye >> 5], 1u << (mye & 31));
+                if (lane < E_MAX / 32 && mine != 0u) atomicOr(&s_set[lane], mine);
             }
         }
         __syncthreads();

@@ -16,7 +16,7 @@ import torch
 import moe_synth as ms
 import oracle
 import aware_expert_routing_moe_b200 as moe
-from gpu_cases import assert_close_y, shape
+from gpu_cases import assert_close_y, host_layer, shape
 
 pytestmark = pytest.mark.gpu
 
@@ -80,7 +80,7 @@ def _run(S, B, mode, k0, c, seed, ties=False, L=None):
 
 def test_down_channel_major_is_the_transpose():
     S = shape("q30b")
-    L = ms.make_weights(S, 0)
+    L = host_layer("q30b", 0)
     Wdn = torch.from_numpy(L["Wdown"].view(np.int16)).cuda()
     WdT = torch.empty(S.E, S.F, S.d, dtype=torch.int16, device="cuda")
     lib = moe.load_library()
@@ -103,21 +103,21 @@ def test_channels_small_shape(B, mode, k0, c, ties):
 def test_channels_q30b(B, mode, k0, frac):
     S = shape("q30b")
     c = int(round(frac * S.F))
-    L, sel, keep, keep_r, y, y_r, _ = _run(S, B, mode, k0, c, seed=0)
+    L, sel, keep, keep_r, y, y_r, _ = _run(S, B, mode, k0, c, seed=0, L=host_layer("q30b", 0))
     assert np.array_equal(keep, _packed(keep_r) * (sel[:, :, None] >= 0))
     assert_close_y(y, y_r, f"q30b B={B} c={c}")
 
 
 def test_channels_q235b_b4():
     S = shape("q235b")
-    L, sel, keep, keep_r, y, y_r, _ = _run(S, 4, OEA, 4, 200, seed=0)
+    L, sel, keep, keep_r, y, y_r, _ = _run(S, 4, OEA, 4, 200, seed=0, L=host_layer("q235b", 0))
     assert np.array_equal(keep, _packed(keep_r) * (sel[:, :, None] >= 0))
     assert_close_y(y, y_r, "q235b B=4 c=200")
 
 
 def test_all_channels_kept_is_the_dense_ffn():
     S = shape("q30b")
-    L, sel, keep, keep_r, y, _, _ = _run(S, 2, OEA, 4, S.F, seed=3)
+    L, sel, keep, keep_r, y, _, _ = _run(S, 2, OEA, 4, S.F, seed=3, L=host_layer("q30b", 0))
     x = ms.make_tokens(S, 2, 3)
     logits, probs, _, _ = oracle.route(x, L["Wg"], L["bias"], S.k)
     s2, w2 = oracle.reselect(logits, probs, S.k, OEA, 4, 0)

@@ -282,3 +282,44 @@ def test_layer_repeatable_and_workspace_reuse():
     for yy in ys[1:]:
         # same routing; the combine's atomics may add in another order
         assert torch.allclose(yy, ys[0], rtol=1e-5, atol=1e-6)
+
+
+@pytest.mark.parametrize("name,B,mode,k0", [("q30b", 1, OEA, 4), ("q30b", 4, NONE, 0), ("q30b", 16, OEA, 4),
+                                           ("q30b", 40, OEA, 4), ("tiny", 4, OEA, 2), ("q30b", 16, XSHARE, 0)])
+def test_layer_graph_replays(name, B, mode, k0):
+    # back-to-back calls on one workspace, as a serving loop issues them: a
+    # CUDA graph of 4 calls replayed 25 times; the error word stays clear and
+    # every replay gives the single call's selection and (up to the order of
+    # the combine's atomic adds) its output, which matches the oracle
+    S = shape(name)
+    L = host_layer(name, 0)
+    D = device_layer(name, 0)
+    x = _tokens(name, B, 0)
+    xd = torch.from_numpy(x).cuda()
+    budget = 16 if mode == XSHARE else 0
+    ws = moe.new_workspace(B, S.d, S.E, S.k, S.F)
+    ys = [torch.empty(B, S.d, dtype=torch.float32, device="cuda") for _ in range(4)]
+    sels = [torch.empty(B, S.k, dtype=torch.int32, device="cuda") for _ in range(4)]
+    s = torch.cuda.Stream()
+
+    def calls():
+        for i in range(4):
+            moe.moe_layer_decode(xd, D["Wg"], D["bias"], D["Wgate"], D["Wup"], D["Wdown"], S.k, mode, k0, budget,
+                                 ws=ws, y=ys[i], sel_idx=sels[i], stream=s)
+
+    with torch.cuda.stream(s):
+        calls()
+    s.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        calls()
+    with torch.cuda.stream(s):
+        for _ in range(25):
+            g.replay()
+    s.synchronize()
+    assert moe.moe_check_error(ws, s) == 0
+    sel_r, w_r, n_r, y_r = _oracle_layer(S, L, x, mode, k0, budget, None)
+    for i in range(4):
+        assert np.array_equal(sels[i].cpu().numpy(), sel_r)
+        assert_close_y(ys[i].cpu().numpy(), y_r, f"{name} B={B} replay call {i}")
+    del g

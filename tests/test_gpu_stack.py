@@ -29,15 +29,23 @@ def _lib():
     moe.load_library()
     yield
     torch.cuda.synchronize()
+    _CACHE.clear()
+
+
+_CACHE = {}
 
 
 def _stack_layers(name, n):
+    # one set of layers per shape, grown as needed and shared by the tests
     S = shape(name)
-    host = [ms.make_weights(S, seed) for seed in range(n)]
+    host, dev = _CACHE.setdefault(name, ([], []))
     t = lambda a: torch.from_numpy(a).cuda()
-    dev = [(t(L["Wg"]), t(L["bias"]), t(L["Wgate"].view(np.int16)), t(L["Wup"].view(np.int16)),
-            t(L["Wdown"].view(np.int16))) for L in host]
-    return S, host, dev
+    while len(host) < n:
+        L = ms.make_weights(S, len(host))
+        host.append(L)
+        dev.append((t(L["Wg"]), t(L["bias"]), t(L["Wgate"].view(np.int16)), t(L["Wup"].view(np.int16)),
+                    t(L["Wdown"].view(np.int16))))
+    return S, host[:n], dev[:n]
 
 
 def _check_stack(name, B, n, mode, k0=0, budget=0, phase=moe.MOE_PHASE_DECODE, kind="normal"):
