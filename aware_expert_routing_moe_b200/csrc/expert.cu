@@ -74,6 +74,9 @@ struct Ring {
     static constexpr int STAGES = ST;
     static constexpr int OP_BYTES = OPB;
     static constexpr int SLOT_BYTES = W_BYTES + OPB;
+    // the wide dense mode (33..64 tokens) needs 32 KB operand tiles; the
+    // small ring's instances leave its code out
+    static constexpr bool WIDE_OK = OPB >= 32768;
 };
 constexpr int PART_LD = TN + 1;                        // padded row of the epilogue buffer
 constexpr int PART_FLOATS = (NCW / 2) * 2 * 16 * PART_LD;  // GU partial sums for the epilogue
@@ -698,7 +701,7 @@ __device__ void consumer(const ExpertArgs &a, SharedCtl *ctl, unsigned char *slo
                     lists_ready = true;
                 }
                 // wide mode: this warp's tokens start at 32 (warp / 4)
-                const int tb = a.wide ? (warp >> 2) * 32 : 0;
+                const int tb = (RG::WIDE_OK && a.wide) ? (warp >> 2) * 32 : 0;
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
 #pragma unroll
@@ -726,8 +729,9 @@ __device__ void consumer(const ExpertArgs &a, SharedCtl *ctl, unsigned char *slo
         }
         const uint32_t wbase = smem_u32(slots + slot * RG::SLOT_BYTES);
         const uint32_t obase = wbase + W_BYTES;
-        const int nt = a.wide ? 4 : (h.type == UNIT_GU && a.dense) ? (a.bpad >> 3) : ((h.n + 7) >> 3);
-        if (a.wide) {
+        const bool wide = RG::WIDE_OK && a.wide;
+        const int nt = wide ? 4 : (h.type == UNIT_GU && a.dense) ? (a.bpad >> 3) : ((h.n + 7) >> 3);
+        if (wide) {
             if (h.type == UNIT_GU) {
                 const int gk = 64 * a.gc;
                 gu_stage_wide(wbase, obase, a.bpad * 128, min(gk, a.d - h.k * gk), warp, lane, acc_g, acc_u);
@@ -749,7 +753,7 @@ __device__ void consumer(const ExpertArgs &a, SharedCtl *ctl, unsigned char *slo
         if (h.s != h.ns - 1) continue;
 
         // ---- unit epilogue
-        if (h.type == UNIT_GU && a.wide) {
+        if (h.type == UNIT_GU && wide) {
             // each warp owns complete sums: h = silu(g) u straight to H
             const int r0 = h.row0 + (warp >> 2) * 16 + row;
 #pragma unroll
@@ -772,7 +776,7 @@ __device__ void consumer(const ExpertArgs &a, SharedCtl *ctl, unsigned char *slo
             // each warp holds a k-half of a 16-row block (wide mode: all of k
             // for 32 tokens): both halves add into y
             const int i_base = h.row0 + (warp & 3) * 16 + row;
-            const int tb = a.wide ? (warp >> 2) * 32 : 0;
+            const int tb = wide ? (warp >> 2) * 32 : 0;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 if (j >= nt) break;
@@ -1122,6 +1126,39 @@ struct LayerArgs {
     ReselectArgs sel;   // the selection CTA's arguments
 };
 
+// OR each token's first r1 experts (r1 <= R) into s_set (bit e of word
+// e / 32): warp w takes tokens w, w + NCW, ...
+template <int NI, int R>
+__device__ __forceinline__ void rank_union(const ExpertArgs &a, const LayerArgs &L, int warp, int lane,
+                                           unsigned *s_set) {
+#pragma unroll 1
+    for (int b = warp; b < a.B; b += 2 * NCW) {
+        const int b2 = b + NCW;
+        const bool two = b2 < a.B;
+        float l[NI], l2[NI];
+        unsigned ord[NI], ord2[NI];
+        load_row<NI>(L.logits + static_cast<size_t>(b) * a.E, a.E, lane, l);
+        load_row<NI>(L.logits + static_cast<size_t>(two ? b2 : b) * a.E, a.E, lane, l2);
+#pragma unroll
+        for (int i = 0; i < NI; ++i) {
+            ord[i] = ord_of(l[i]);
+            ord2[i] = ord_of(l2[i]);
+        }
+        unsigned long long top[R], top2[R];
+        warp_top_r<NI, R>(ord, a.E, lane, top);
+        warp_top_r<NI, R>(ord2, a.E, lane, top2);
+        unsigned mine = 0u;  // bits of expert word `lane`
+#pragma unroll
+        for (int j = 0; j < R; ++j) {
+            if (j >= L.r1) break;
+            const int e = topr_expert(top[j]), e2 = topr_expert(top2[j]);
+            if (e >= 0 && (e >> 5) == lane) mine |= 1u << (e & 31);
+            if (two && e2 >= 0 && (e2 >> 5) == lane) mine |= 1u << (e2 & 31);
+        }
+        if (lane < E_MAX / 32 && mine != 0u) atomicOr(&s_set[lane], mine);
+    }
+}
+
 template <class RG, int NI>
 __global__ void __launch_bounds__(NTHREADS, 1)
     layer_kernel(const __grid_constant__ ExpertMaps maps, const __grid_constant__ RouterMaps rmaps,
@@ -1290,34 +1327,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
     // ---- 4. the activated set, then the expert stream
     if (L.r1 > 0) {
-        // two tokens per warp at a time, their arg-max rounds interleaved
-        // (independent reductions overlap); only the union is kept, so the
-        // order of a token's winners does not matter
+        // each warp ranks tokens warp, warp + NCW, ... (two at a time, their
+        // butterfly merges independent); only the union of the tokens' first
+        // r1 experts is kept, so the order within a token does not matter
         if (warp < NCW && ok) {
-#pragma unroll 1
-            for (int b = warp; b < a.B; b += 2 * NCW) {
-                const int b2 = b + NCW;
-                const bool two = b2 < a.B;
-                float l[NI], l2[NI];
-                unsigned ord[NI], ord2[NI];
-                load_row<NI>(L.logits + static_cast<size_t>(b) * a.E, a.E, lane, l);
-                load_row<NI>(L.logits + static_cast<size_t>(two ? b2 : b) * a.E, a.E, lane, l2);
-#pragma unroll
-                for (int i = 0; i < NI; ++i) {
-                    ord[i] = ord_of(l[i]);
-                    ord2[i] = ord_of(l2[i]);
-                }
-                unsigned cand = valid_bits<NI>(a.E, lane), cand2 = cand;
-                unsigned mine = 0u;  // bit j: lane's expert-word hits (set below)
-#pragma unroll 1
-                for (int j = 0; j < L.r1; ++j) {
-                    const int e = warp_argmax<NI>(ord, cand, lane);
-                    const int e2 = warp_argmax<NI>(ord2, cand2, lane);
-                    if (e >= 0 && (e >> 5) == lane) mine |= 1u << (e & 31);
-                    if (two && e2 >= 0 && (e2 >> 5) == lane) mine |= 1u << (e2 & 31);
-                }
-                if (lane < E_MAX / 32 && mine != 0u) atomicOr(&s_set[lane], mine);
-            }
+            if (L.r1 <= 4) rank_union<NI, 4>(a, L, warp, lane, s_set);
+            else if (L.r1 <= 8) rank_union<NI, 8>(a, L, warp, lane, s_set);
+            else rank_union<NI, 16>(a, L, warp, lane, s_set);
         }
         __syncthreads();
         if (warp == NCW) table_from_mask(a, ctl, lane < E_MAX / 32 ? s_set[lane] : 0u, lane);

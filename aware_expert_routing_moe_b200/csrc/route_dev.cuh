@@ -288,6 +288,97 @@ __device__ __forceinline__ int warp_argmax(const unsigned (&ord)[NI], unsigned &
     return idx;
 }
 
+// ---------------------------------------------------- warp top-R set --
+// The R largest of a token's rank keys (logit image, then lower index),
+// R a power of two: every lane ends with the same list, descending.  Each
+// lane first sorts its own keys; then, at each of five butterfly levels, a
+// lane merges its list with its partner's: the elementwise maximum of the
+// list and the reversed partner list holds the R largest of the two (a
+// bitonic sequence), which a bitonic merge sorts.  Five shuffle levels
+// instead of R dependent rounds of warp arg-max.  Key 0 = no expert.
+__device__ __forceinline__ unsigned long long topr_key(unsigned ord, int e) {
+    return (static_cast<unsigned long long>(ord) << 32) | static_cast<unsigned>(~static_cast<unsigned>(e));
+}
+__device__ __forceinline__ int topr_expert(unsigned long long key) {
+    return key == 0ull ? -1 : static_cast<int>(~static_cast<unsigned>(key & 0xffffffffull));
+}
+template <int R>
+__device__ __forceinline__ void bitonic_sort_desc(unsigned long long (&v)[R]) {
+    // v is bitonic: sort it descending
+#pragma unroll
+    for (int half = R / 2; half >= 1; half >>= 1)
+#pragma unroll
+        for (int i = 0; i < R; ++i)
+            if ((i & half) == 0) {
+                const unsigned long long a = v[i], b = v[i + half];
+                v[i] = a > b ? a : b;
+                v[i + half] = a > b ? b : a;
+            }
+}
+// top = the R largest of top and other (both descending), descending.
+template <int R>
+__device__ __forceinline__ void merge_top(unsigned long long (&top)[R], const unsigned long long (&other)[R]) {
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+        const unsigned long long b = other[R - 1 - i];
+        top[i] = top[i] > b ? top[i] : b;
+    }
+    bitonic_sort_desc<R>(top);
+}
+// v (any order) sorted descending: runs of doubling length, each made
+// bitonic by reversing its second half, then merged.
+template <int R>
+__device__ __forceinline__ void sort_desc(unsigned long long (&v)[R]) {
+#pragma unroll
+    for (int len = 2; len <= R; len <<= 1) {
+#pragma unroll
+        for (int base = 0; base < R; base += len)
+#pragma unroll
+            for (int i = 0; i < len / 4; ++i) {
+                const unsigned long long t = v[base + len / 2 + i];
+                v[base + len / 2 + i] = v[base + len - 1 - i];
+                v[base + len - 1 - i] = t;
+            }
+#pragma unroll
+        for (int half = len / 2; half >= 1; half >>= 1)
+#pragma unroll
+            for (int i = 0; i < R; ++i)
+                if ((i & half) == 0) {
+                    const unsigned long long a = v[i], b = v[i + half];
+                    v[i] = a > b ? a : b;
+                    v[i + half] = a > b ? b : a;
+                }
+    }
+}
+template <int NI, int R>
+__device__ __forceinline__ void warp_top_r(const unsigned (&ord)[NI], int E, int lane, unsigned long long (&top)[R]) {
+    // this lane's keys (e = lane + 32 i), R at a time
+#pragma unroll
+    for (int c = 0; c < (NI + R - 1) / R; ++c) {
+        unsigned long long cur[R];
+#pragma unroll
+        for (int i = 0; i < R; ++i) {
+            const int ii = c * R + i;
+            const int e = lane + 32 * ii;
+            cur[i] = (ii < NI && e < E) ? topr_key(ord[ii < NI ? ii : 0], e) : 0ull;
+        }
+        sort_desc<R>(cur);
+        if (c == 0) {
+#pragma unroll
+            for (int i = 0; i < R; ++i) top[i] = cur[i];
+        } else {
+            merge_top<R>(top, cur);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+        unsigned long long other[R];
+#pragma unroll
+        for (int i = 0; i < R; ++i) other[i] = __shfl_xor_sync(FULL, top[i], o);
+        merge_top<R>(top, other);
+    }
+}
+
 // Softmax of one token (row lane-distributed: e = lane + 32 i), max by
 // warp reduction of logit images, sum in the canonical lane/butterfly order.
 template <int NI>
