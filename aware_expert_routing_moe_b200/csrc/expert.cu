@@ -652,7 +652,11 @@ __device__ bool post_signal(SharedCtl *ctl, Counters *ctr, int q, int i) {
     return true;
 }
 
-template <class RG>
+// DNT: 0 = the token-tile count is taken per stage (the expert kernel:
+// any mode); 1..4 = dense mode with that many 8-token tiles, fixed for the
+// call; 5 = the wide dense mode.  A fixed count leaves only that path's code
+// in the consumer loop (the fused layer kernel is instantiated per count).
+template <class RG, int DNT = 0>
 __device__ void consumer(const ExpertArgs &a, SharedCtl *ctl, unsigned char *slots, float *part) {
     constexpr int STAGES = RG::STAGES;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -701,7 +705,7 @@ __device__ void consumer(const ExpertArgs &a, SharedCtl *ctl, unsigned char *slo
                     lists_ready = true;
                 }
                 // wide mode: this warp's tokens start at 32 (warp / 4)
-                const int tb = (RG::WIDE_OK && a.wide) ? (warp >> 2) * 32 : 0;
+                const int tb = (DNT == 5 || (DNT == 0 && RG::WIDE_OK && a.wide)) ? (warp >> 2) * 32 : 0;
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
 #pragma unroll
@@ -729,9 +733,13 @@ __device__ void consumer(const ExpertArgs &a, SharedCtl *ctl, unsigned char *slo
         }
         const uint32_t wbase = smem_u32(slots + slot * RG::SLOT_BYTES);
         const uint32_t obase = wbase + W_BYTES;
-        const bool wide = RG::WIDE_OK && a.wide;
-        const int nt = wide ? 4 : (h.type == UNIT_GU && a.dense) ? (a.bpad >> 3) : ((h.n + 7) >> 3);
-        if (wide) {
+        const bool wide = DNT == 5 || (DNT == 0 && RG::WIDE_OK && a.wide);
+        const int nt = (DNT >= 1 && DNT <= 4) ? DNT
+                       : wide                 ? 4
+                       : (h.type == UNIT_GU && a.dense) ? (a.bpad >> 3) : ((h.n + 7) >> 3);
+        if constexpr (DNT >= 1 && DNT <= 4) {
+            stage_dispatch<(DNT >= 1 && DNT <= 4) ? DNT : 1>(h, wbase, obase, a, warp, lane, acc_g, acc_u);
+        } else if (wide) {
             if (h.type == UNIT_GU) {
                 const int gk = 64 * a.gc;
                 gu_stage_wide(wbase, obase, a.bpad * 128, min(gk, a.d - h.k * gk), warp, lane, acc_g, acc_u);
@@ -1033,7 +1041,7 @@ __device__ void table_from_lists(const ExpertArgs &a, SharedCtl *ctl, int lane) 
     }
 }
 
-template <class RG>
+template <class RG, int DNT = 0>
 __device__ __forceinline__ void run_roles(const ExpertArgs &a, const ExpertMaps &maps, const CtaSmem<RG> &sm) {
     const int warp = threadIdx.x >> 5;
     if (warp == NCW) {
@@ -1041,7 +1049,7 @@ __device__ __forceinline__ void run_roles(const ExpertArgs &a, const ExpertMaps 
     } else if (warp == NCW + 1) {
         signaller(a, sm.ctl);
     } else {
-        consumer<RG>(a, sm.ctl, sm.slots, sm.part);
+        consumer<RG, DNT>(a, sm.ctl, sm.slots, sm.part);
     }
 }
 
@@ -1159,7 +1167,7 @@ __device__ __forceinline__ void rank_union(const ExpertArgs &a, const LayerArgs 
     }
 }
 
-template <class RG, int NI>
+template <class RG, int NI, int DNT>
 __global__ void __launch_bounds__(NTHREADS, 1)
     layer_kernel(const __grid_constant__ ExpertMaps maps, const __grid_constant__ RouterMaps rmaps,
                  const ExpertArgs a, const LayerArgs L) {
@@ -1181,12 +1189,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int e0 = eg * L.epb, b0 = tg * L.tpb;
         const int ne = min(L.epb, a.E - e0), nb = min(L.tpb, a.B - b0);
         if (weights) {
-            unsigned long long keep;
-            asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(keep));
             for (int r = 0; r < ne; ++r)
                 for (int bx = 0; bx < L.boxes; ++bx)
-                    tma_rows_hint(wrows + r * L.row_bytes + bx * L.box_lines * 128, &rmaps.wg,
-                                  (e0 + r) * lines + bx * L.box_lines, &s_rbar, keep);
+                    tma_rows(wrows + r * L.row_bytes + bx * L.box_lines * 128, &rmaps.wg,
+                                  (e0 + r) * lines + bx * L.box_lines, &s_rbar);
         }
         if (tokens)
             for (int r = 0; r < nb; ++r)
@@ -1342,7 +1348,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         else table_from_mask(a, ctl, 0u, lane);
     }
     __syncthreads();
-    run_roles<RG>(a, maps, sm);
+    run_roles<RG, DNT>(a, maps, sm);
     cta_exit(a, ctl);
 }
 
@@ -1627,10 +1633,10 @@ LayerArgs make_layer_router(const moe_dims_t &d, int grid, int ring_bytes) {
     return L;
 }
 
-template <class RG, int NI>
+template <class RG, int NI, int DNT>
 cudaError_t launch_layer_ni(const ExpertMaps &maps, const RouterMaps &rmaps, const ExpertArgs &a,
                             const LayerArgs &L, int grid, int dev, cudaStream_t s) {
-    cudaError_t err = configure_smem(layer_kernel<RG, NI>, smem_bytes<RG>(), dev);
+    cudaError_t err = configure_smem(layer_kernel<RG, NI, DNT>, smem_bytes<RG>(), dev);
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
@@ -1647,7 +1653,7 @@ cudaError_t launch_layer_ni(const ExpertMaps &maps, const RouterMaps &rmaps, con
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = L.chained ? 2 : 1;
-    return cudaLaunchKernelEx(&cfg, layer_kernel<RG, NI>, maps, rmaps, a, L);
+    return cudaLaunchKernelEx(&cfg, layer_kernel<RG, NI, DNT>, maps, rmaps, a, L);
 }
 
 }  // namespace
@@ -1709,16 +1715,22 @@ cudaError_t launch_layer_fused(const ExpertMaps &maps, const RouterMaps &rmaps, 
     L.sel.publish_set = batch_rule ? 1 : 0;
     const size_t sel_smem = reselect_smem(d, rule, &L.sel.cache_rows);
     if (sel_smem > static_cast<size_t>(ring)) return cudaErrorInvalidValue;
-    switch (ni_for(d.E)) {
-        case 1: return small ? launch_layer_ni<RingSmallB, 1>(maps, rmaps, a, L, sms, dev, s)
-                             : launch_layer_ni<RingLargeB, 1>(maps, rmaps, a, L, sms, dev, s);
-        case 2: return small ? launch_layer_ni<RingSmallB, 2>(maps, rmaps, a, L, sms, dev, s)
-                             : launch_layer_ni<RingLargeB, 2>(maps, rmaps, a, L, sms, dev, s);
-        case 4: return small ? launch_layer_ni<RingSmallB, 4>(maps, rmaps, a, L, sms, dev, s)
-                             : launch_layer_ni<RingLargeB, 4>(maps, rmaps, a, L, sms, dev, s);
-        default: return small ? launch_layer_ni<RingSmallB, 8>(maps, rmaps, a, L, sms, dev, s)
-                              : launch_layer_ni<RingLargeB, 8>(maps, rmaps, a, L, sms, dev, s);
+    // instantiated per token-tile count (small ring: 1-2 tiles of 8
+    // tokens, large ring: 3-4 tiles or the wide mode) and for logit rows of
+    // up to 128 or 256 experts per warp
+    const int dnt = d.B > TN ? 5 : (d.B + 7) / 8;
+    const bool ni8 = ni_for(d.E) > 4;
+#define MOE_LAYER_CASE(RGT, DN)                                                                        \
+    return ni8 ? launch_layer_ni<RGT, 8, DN>(maps, rmaps, a, L, sms, dev, s)                          \
+               : launch_layer_ni<RGT, 4, DN>(maps, rmaps, a, L, sms, dev, s)
+    switch (dnt) {
+        case 1: MOE_LAYER_CASE(RingSmallB, 1);
+        case 2: MOE_LAYER_CASE(RingSmallB, 2);
+        case 3: MOE_LAYER_CASE(RingLargeB, 3);
+        case 4: MOE_LAYER_CASE(RingLargeB, 4);
+        default: MOE_LAYER_CASE(RingLargeB, 5);
     }
+#undef MOE_LAYER_CASE
 }
 
 }  // namespace moe

@@ -807,16 +807,6 @@ __device__ __forceinline__ void tma_rows(void *dst, const CUtensorMap *map, int 
         "l"(reinterpret_cast<unsigned long long>(map)), "r"(0), "r"(line), "r"(smem_addr(bar))
         : "memory");
 }
-// The same with an L2 cache policy (the router weights: evict-last, so that
-// they stay resident across calls while the expert weights stream through).
-__device__ __forceinline__ void tma_rows_hint(void *dst, const CUtensorMap *map, int line, unsigned long long *bar,
-                                              unsigned long long policy) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
-        " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_addr(dst)),
-        "l"(reinterpret_cast<unsigned long long>(map)), "r"(0), "r"(line), "r"(smem_addr(bar)), "l"(policy)
-        : "memory");
-}
 __device__ __forceinline__ float comp(const float4 &v, int u) {
     return u == 0 ? v.x : u == 1 ? v.y : u == 2 ? v.z : v.w;
 }
