@@ -56,6 +56,7 @@ WORKLOADS = {
     "q30b_b16_oea4": dict(shape="q30b", B=16, mode=1, k0=4, budget=0, rule="OEA k0=4"),
     "q30b_b16_none": dict(shape="q30b", B=16, mode=0, k0=0, budget=0, rule="NONE (standard top-8)"),
     "q30b_b64_oea4": dict(shape="q30b", B=64, mode=1, k0=4, budget=0, rule="OEA k0=4"),
+    "q30b_b96_oea4": dict(shape="q30b", B=96, mode=1, k0=4, budget=0, rule="OEA k0=4"),
     "q235b_b16_oea4": dict(shape="q235b", B=16, mode=1, k0=4, budget=0, rule="OEA k0=4"),
     "spec_xshare32": dict(shape="q30b", B=32, mode=2, k0=0, budget=32, rule="XShare budget=32",
                           kind="spec"),
@@ -458,7 +459,7 @@ SWEEP = {
     # ROTATE copies); mode 4 (hierarchical XShare) takes the request size
     "tiny": [(4, 1, 2, 0, "normal"), (4, 0, 0, 0, "normal")],
     "e64": [(16, 1, 4, 0, "normal"), (16, 0, 0, 0, "normal")],
-    "q30b": [(b, m, k0, 0, "normal") for b in (1, 4, 16, 32, 64) for (m, k0) in ((0, 0), (1, 4))]
+    "q30b": [(b, m, k0, 0, "normal") for b in (1, 4, 16, 32, 48, 64, 128) for (m, k0) in ((0, 0), (1, 4))]
             + [(16, 1, k0, 0, "normal") for k0 in (2, 6, 8)]
             + [(32, 0, 0, 0, "spec")] + [(32, 2, 0, m, "spec") for m in (24, 32, 48)]
             + [(16, 3, 0, 0, "normal"), (64, 3, 0, 0, "normal"), (32, 3, 0, 0, "spec")]

@@ -285,7 +285,9 @@ def test_layer_repeatable_and_workspace_reuse():
 
 
 @pytest.mark.parametrize("name,B,mode,k0", [("q30b", 1, OEA, 4), ("q30b", 4, NONE, 0), ("q30b", 16, OEA, 4),
-                                           ("q30b", 40, OEA, 4), ("tiny", 4, OEA, 2), ("q30b", 16, XSHARE, 0)])
+                                           ("q30b", 40, OEA, 4), ("tiny", 4, OEA, 2), ("q30b", 16, XSHARE, 0),
+                                           ("q30b", 16, NONE, 0), ("q235b", 1, OEA, 4), ("q235b", 16, OEA, 4),
+                                           ("q235b", 16, NONE, 0)])
 def test_layer_graph_replays(name, B, mode, k0):
     # back-to-back calls on one workspace, as a serving loop issues them: a
     # CUDA graph of 4 calls replayed 25 times; the error word stays clear and
