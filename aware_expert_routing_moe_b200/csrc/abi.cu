@@ -177,8 +177,9 @@ bool encode_expert_maps(ExpertMaps *m, const moe_dims_t &d, const uint16_t *Wgat
     std::memset(m, 0, sizeof(*m));
     const uint64_t E = d.E, F = d.d_ff, D = d.d;
     const uint32_t gu_chunks = expert_ffn_gu_chunks(d.d, d.B), d_chunks = expert_ffn_d_chunks(d.d_ff);
-    return encode_bf16_chunked(&m->gate, Wgate, E * F, D, expert_ffn_gu_rows(d.B), gu_chunks) &&
-           encode_bf16_chunked(&m->up, Wup, E * F, D, expert_ffn_gu_rows(d.B), gu_chunks) &&
+    const uint32_t gu_box = expert_ffn_gu_box_chunks(d.d, d.B);
+    return encode_bf16_chunked(&m->gate, Wgate, E * F, D, expert_ffn_gu_rows(d.B), gu_box) &&
+           encode_bf16_chunked(&m->up, Wup, E * F, D, expert_ffn_gu_rows(d.B), gu_box) &&
            encode_bf16_chunked(&m->down, Wdown, E * D, F, expert_ffn_d_rows(), d_chunks) &&
            encode_bf16_chunked(&m->h, h,
                                expert_ffn_dense_batch(d.B) ? static_cast<uint64_t>(active_slots(d)) * d.B

@@ -8,7 +8,8 @@
 // Retraining", abstract).
 //
 // Work units, dealt round robin to persistent CTAs (one per SM):
-//   GU unit (expert e, token tile, 16-row block of d_ff):
+//   GU unit (expert e, token tile, block of d_ff rows: 32 in dense mode,
+//   16 in tile mode):
 //       g = Wgate[e][rows] x_t, u = Wup[e][rows] x_t over all of d,
 //       h = silu(g) * u -> H scratch (bf16);
 //   D unit (expert e, token tile, 64-row block of d):
@@ -23,22 +24,27 @@
 // Gate/up work then needs only the activated set, which the fused layer
 // kernel has before the token lists exist: its CTAs rank the tokens' first
 // experts themselves (OEA, plain top-k) or read the set the selection CTA
-// publishes (the batch-wide rules), and start streaming at once.  From 33
-// to 64 tokens the gate/up units are 32 rows by 256-column stages, and the
-// consumer warps split a stage by (row tile, token tile).
-// Larger batches use tiles of up to 32 (token, expert) pairs: the input
-// preparation copies each pair's x row (bf16) into a pair-indexed buffer in
-// the lists' order, so a tile's x rows are one swizzled box like H's.
+// publishes (the batch-wide rules), and start streaming at once.
+// Larger batches (tile mode) use tiles of up to 32 (token, expert) pairs:
+// the input preparation copies each pair's x row (bf16) into a pair-indexed
+// buffer in the lists' order, so a tile's x rows are one swizzled box like
+// H's.
 //
 // Per CTA: one producer warp issues TMA tensor copies (three-dimensional
 // boxes of 64-column chunks, 128-byte swizzle) into a ring of 32 KB weight
-// stages plus operand tiles, each guarded by a full/empty mbarrier pair;
-// eight consumer warps split every stage's k-steps and run mma.sync
-// m16n8k16 bf16 tiles (16 weight rows as A, tokens as B, fp32 accumulation);
-// a signal warp publishes gate/up completions.  Every wait is bounded by a
-// time limit; on expiry the CTA records an error code in the workspace,
-// drains its in-flight copies and returns.  The last CTA to finish puts the
-// workspace counters of the call back to zero.
+// stages plus operand tiles, each guarded by a full/empty mbarrier pair.
+// Dense mode runs on the 5th-generation tensor cores: one thread issues, per
+// stage, tcgen05 MMAs of 64 weight rows (a gate/up chunk is 32 gate rows and
+// the same 32 up rows) by bpad token columns into a TMEM accumulator, two
+// buffers deep so that a unit's epilogue overlaps the next unit's MMAs; the
+// MMA completion itself frees the stage; eight epilogue warps read the
+// accumulator out (silu * u -> H, or weighted atomics into y) and publish
+// gate/up completions.  Tile mode keeps eight mma.sync consumer warps that
+// split every stage's k-steps (m16n8k16 bf16, 16 weight rows as A, pairs as
+// B) and a signal warp that publishes completions.  Every wait is bounded by
+// a time limit; on expiry the CTA records an error code in the workspace,
+// drains its in-flight copies (and MMAs) and returns.  The last CTA to
+// finish puts the workspace counters of the call back to zero.
 #include <cstring>
 #include <mutex>
 
@@ -46,58 +52,85 @@
 
 #include "internal.h"
 #include "route_dev.cuh"
+#include "tcgen05.cuh"
 
 namespace moe {
 namespace {
 
-constexpr int NCW = 8;                    // consumer warps
-constexpr int NTHREADS = (NCW + 2) * 32;  // + one producer warp + one signal warp
+constexpr int NCW = 8;                    // consumer (epilogue) warps
+constexpr int NTHREADS = (NCW + 2) * 32;  // tile mode: + one producer warp + one signal warp
+// Dense mode: the MMAs are issued by NISSUE warps (one per SM sub-partition:
+// a single thread issues at most about one tcgen05.mma per 165 cycles,
+// whatever its shape, measured), each taking every NISSUE-th k-step of a
+// stage into a partial accumulator of its own.
+constexpr int NISSUE = 4;
+constexpr int NTHREADS_UM = (NCW + 1 + NISSUE) * 32;
+template <bool UM>
+constexpr int cta_threads() { return UM ? NTHREADS_UM : NTHREADS; }
 constexpr int SIG_SLOTS = 4;              // gate/up completions queued for the signal warp
-constexpr int TN = 32;                    // tokens per tile
+constexpr int TN = 32;                    // pairs per token tile (batches above 64 tokens)
 constexpr int DENSE_MAX = 64;             // dense mode (every unit takes the whole batch) up to 64 tokens
-constexpr int GU_ROWS = 16;               // rows of Wgate and of Wup per GU unit
-constexpr int GU_CHUNKS = 8;              // 64-column chunks of d per GU stage (at most)
-// wide dense mode (33..64 tokens): GU units of 32 rows, stages of 4 chunks,
-// so that a stage's weights (32 KB) and its 64 token rows (32 KB) fill a
-// slot of the large ring
-constexpr int WIDE_ROWS = 32;
-constexpr int WIDE_CHUNKS = 4;
+// Batches above 64 tokens (tile mode): GU units of 16 rows, stages of 8
+// chunks, mma.sync consumers.
+constexpr int GU_ROWS = 16;
+constexpr int GU_CHUNKS = 8;
+// Dense mode (tensor-core path): GU units of 32 gate rows and the same 32 up
+// rows; a stage holds 4 chunks of 64 columns, each chunk as the gate tile
+// [32][64] followed by the up tile [32][64], so that one chunk is a single
+// 64-row MMA operand (1 KiB row groups throughout).
+constexpr int UM_ROWS = 32;
+constexpr int UM_CHUNKS = 4;
+constexpr int UM_TILE = UM_ROWS * 128;        // one gate (or up) tile of a chunk
+constexpr int UM_CHUNK_BYTES = 2 * UM_TILE;   // gate + up tiles of a chunk
 constexpr int D_ROWS = 64;                // rows of Wdown per D unit
 constexpr int D_CHUNKS = 4;               // 64-column chunks of d_ff per D stage (at most)
-constexpr int MAX_STAGES = 4;
+constexpr int MAX_STAGES = 5;
 constexpr int W_BYTES = 32768;            // weight bytes per stage (both kinds)
-constexpr int UP_OFF = GU_ROWS * 128 * GU_CHUNKS;  // Wup tile after the Wgate tile
-// Two ring shapes: 4 stages with a 16 KB operand region (B <= 16), and 3
-// stages with 32 KB (larger batches).
-template <int ST, int OPB>
+constexpr int UP_OFF = GU_ROWS * 128 * GU_CHUNKS;  // Wup tile after the Wgate tile (tile mode)
+// Ring shapes: stages of 32 KB of weights plus an operand region for the
+// token rows (x for gate/up, H for down): bpad rows x 4 chunks in dense mode
+// (8, 16 or 32 KB for up to 16, 32 or 64 tokens), 32 pair rows x 8 chunks in
+// tile mode.
+constexpr int PART_LD = TN + 1;                        // padded row of the tile-mode epilogue buffer
+constexpr int PART_FLOATS = (NCW / 2) * 2 * 16 * PART_LD;  // GU partial sums (tile mode)
+// PARTB: bytes of the epilogue buffer (tile mode: the partial sums; dense
+// mode: the accumulator copy, [bpad tokens][64 rows] fp32)
+template <int ST, int OPB, int PARTB>
 struct Ring {
     static constexpr int STAGES = ST;
     static constexpr int OP_BYTES = OPB;
     static constexpr int SLOT_BYTES = W_BYTES + OPB;
-    // the wide dense mode (33..64 tokens) needs 32 KB operand tiles; the
-    // small ring's instances leave its code out
-    static constexpr bool WIDE_OK = OPB >= 32768;
+    static constexpr int PART_BYTES = PARTB;
 };
-constexpr int PART_LD = TN + 1;                        // padded row of the epilogue buffer
-constexpr int PART_FLOATS = (NCW / 2) * 2 * 16 * PART_LD;  // GU partial sums for the epilogue
 constexpr int CTL_BYTES = 6144;  // reserved for SharedCtl (checked below)
+// The fused layer kernel adds static shared memory of its own (router and
+// selection state, under 7 KB); the budget below keeps room for it.
+constexpr int STATIC_SMEM_RESERVE = 7168;
 template <class RG>
 constexpr int smem_bytes() {
-    return 1024 /*align slack*/ + RG::STAGES * RG::SLOT_BYTES + PART_FLOATS * 4 + CTL_BYTES;
+    return 1024 /*align slack*/ + RG::STAGES * RG::SLOT_BYTES + RG::PART_BYTES + CTL_BYTES;
 }
-using RingSmallB = Ring<4, 16384>;
-using RingLargeB = Ring<3, 32768>;
+using RingB16 = Ring<5, 8192, 16 * 64 * 4>;
+using RingB32 = Ring<4, 16384, 32 * 64 * 4>;
+using RingB64 = Ring<3, 32768, PART_FLOATS * 4>;
 static_assert(2 * GU_ROWS * 128 * GU_CHUNKS <= W_BYTES, "gate/up tiles do not fit");
-static_assert(WIDE_ROWS * 128 * WIDE_CHUNKS == UP_OFF, "wide gate tile must end where the up tile starts");
-static_assert(DENSE_MAX * 128 * WIDE_CHUNKS <= RingLargeB::OP_BYTES, "wide x rows (64 tokens) do not fit");
-static_assert(DENSE_MAX * 128 * D_CHUNKS <= RingLargeB::OP_BYTES, "wide H tile (64 tokens) does not fit");
+static_assert(UM_CHUNKS * UM_CHUNK_BYTES == W_BYTES, "dense gate/up chunks must fill the weight region");
+static_assert(2 * UM_ROWS == UMMA_M && D_ROWS == UMMA_M && D_ROWS * 128 == UM_CHUNK_BYTES,
+              "a gate/up chunk and a down chunk are one 64-row MMA operand each");
+static_assert(16 * 128 * UM_CHUNKS <= RingB16::OP_BYTES && 32 * 128 * UM_CHUNKS <= RingB32::OP_BYTES &&
+                  DENSE_MAX * 128 * UM_CHUNKS <= RingB64::OP_BYTES && DENSE_MAX * 128 * D_CHUNKS <= RingB64::OP_BYTES,
+              "dense token rows do not fit");
 static_assert(D_ROWS * 128 * D_CHUNKS <= W_BYTES, "down tile does not fit");
-static_assert(16 * GU_CHUNKS * 128 <= RingSmallB::OP_BYTES, "dense x rows (B <= 16) do not fit");
-static_assert(TN * GU_CHUNKS * 128 <= RingLargeB::OP_BYTES, "x rows (32 tokens) do not fit");
-static_assert(TN * 128 * D_CHUNKS <= RingSmallB::OP_BYTES, "H tile does not fit");
-static_assert(RingSmallB::SLOT_BYTES % 1024 == 0 && RingLargeB::SLOT_BYTES % 1024 == 0,
+static_assert(TN * GU_CHUNKS * 128 <= RingB64::OP_BYTES, "x rows (32 pairs) do not fit");
+static_assert(DENSE_MAX * 64 * 4 <= RingB64::PART_BYTES, "accumulator copy does not fit");
+static_assert(RingB16::SLOT_BYTES % 1024 == 0 && RingB32::SLOT_BYTES % 1024 == 0 && RingB64::SLOT_BYTES % 1024 == 0,
               "slots must keep 1 KiB alignment for 128B swizzle");
-static_assert(smem_bytes<RingSmallB>() <= 232448 && smem_bytes<RingLargeB>() <= 232448, "shared memory budget");
+static_assert(RingB16::STAGES <= MAX_STAGES && RingB32::STAGES <= MAX_STAGES && RingB64::STAGES <= MAX_STAGES,
+              "too many stages");
+static_assert(smem_bytes<RingB16>() + STATIC_SMEM_RESERVE <= 232448 &&
+                  smem_bytes<RingB32>() + STATIC_SMEM_RESERVE <= 232448 &&
+                  smem_bytes<RingB64>() + STATIC_SMEM_RESERVE <= 232448,
+              "shared memory budget");
 
 // Bounded waits: a wait on another CTA, another kernel or a copy gives up
 // after the call's wait limit (ExpertArgs::wait_ns, 1 s unless the caller
@@ -123,6 +156,11 @@ struct UnitRec {
 };
 constexpr int UNIT_WINDOW = 32;  // units a producer decodes at once (one per lane)
 
+// The unit an accumulator buffer holds (tensor-core path).
+struct AccHdr {
+    int type, i_act, row0, p0, n;
+};
+
 struct SharedCtl {
     unsigned long long wait_ns;  // limit of every bounded wait of this call
     unsigned long long full[MAX_STAGES];
@@ -140,6 +178,14 @@ struct SharedCtl {
     UnitRec urec[UNIT_WINDOW];  // the producer's decoded window of its own units
     int act_e[E_MAX];       // active expert ids (copied once per CTA)
     int off[E_MAX + 1];     // list offsets (copied once per CTA)
+    // tensor-core path: accumulator buffers (TMEM columns 64 b ..) full /
+    // released, completion of the MMAs issued, the unit each buffer holds
+    unsigned long long acc_full[2];
+    unsigned long long acc_empty[2];
+    unsigned long long mma_done;
+    AccHdr acc_hdr[2];
+    uint32_t tmem;  // TMEM base address of the CTA's allocation
+    volatile int epi_go, epi_lists;  // outcomes of the epilogue's waits (its thread 0)
 };
 
 static_assert(sizeof(SharedCtl) <= CTL_BYTES, "SharedCtl does not fit its reservation");
@@ -156,9 +202,6 @@ struct ExpertArgs {
     // stages load all token rows of x in one box, H is token-indexed
     // [slot][B][d_ff] and the down epilogue weighs tokens by wd[slot][B]
     int dense;
-    // wide dense mode (B > TN): 32-row gate/up units, and the consumer warps
-    // split each stage by (row tile, token tile) instead of by k
-    int wide;
     int gu_rows;  // rows of Wgate / Wup per GU unit
     int gc;       // 64-column chunks of d per GU stage
     int bpad;   // B rounded up to a multiple of 8 (dense mode)
@@ -411,7 +454,9 @@ __device__ bool fetch_unit(int j, int &win_base, int n_units, const ExpertArgs &
     return true;
 }
 
-template <class RG>
+// UM: dense tensor-core layout (a gate/up stage is UM_CHUNKS chunk copies
+// of each matrix, interleaved per chunk); otherwise the tile-mode layout.
+template <class RG, bool UM>
 __device__ void producer(const ExpertArgs &a, const ExpertMaps &m, SharedCtl *ctl, unsigned char *slots) {
     constexpr int STAGES = RG::STAGES;
     const int lane = threadIdx.x & 31;
@@ -444,10 +489,12 @@ __device__ void producer(const ExpertArgs &a, const ExpertMaps &m, SharedCtl *ct
             unsigned char *wdst = slots + slot * RG::SLOT_BYTES;
             unsigned char *odst = wdst + W_BYTES;
             const int gc = a.gc, dc = d_chunks_of(a.F);
+            // chunks of d this gate/up stage covers (the last stage may hold fewer)
+            const int gcv = min(gc, (a.d >> 6) - (cur.k0 + s) * gc);
             // x tile: all B token rows (dense mode) or the tile's TN pair rows
             const unsigned xbytes = static_cast<unsigned>(gc) * (a.dense ? a.bpad : TN) * 128u;
-            const unsigned bytes = cur.type == UNIT_GU ? 2u * gc * (a.gu_rows * 128) + xbytes
-                                                       : dc * (D_ROWS * 128u) + dc * (a.hrows * 128u);
+            const unsigned wbytes = UM ? 2u * gcv * UM_TILE : 2u * gc * (a.gu_rows * 128);
+            const unsigned bytes = cur.type == UNIT_GU ? wbytes + xbytes : dc * (D_ROWS * 128u) + dc * (a.hrows * 128u);
             if (lane == 0) {
                 StageHdr &h = ctl->hdr[slot];
                 h.type = cur.type;
@@ -464,11 +511,22 @@ __device__ void producer(const ExpertArgs &a, const ExpertMaps &m, SharedCtl *ct
             __syncwarp();
             if (cur.type == UNIT_GU) {
                 const int grow = cur.e * a.F + cur.row0;
-                if (lane == 0) tma_load_3d_stream(wdst, &m.gate, 0, grow, s * gc, &ctl->full[slot], policy);
-                if (lane == 1) tma_load_3d_stream(wdst + UP_OFF, &m.up, 0, grow, s * gc, &ctl->full[slot], policy);
-                // x rows of this column range in one swizzled box: all B
-                // tokens (dense mode) or the tile's pairs of the dispatched x
-                if (lane == 2) tma_load_3d(odst, &m.x, 0, a.dense ? 0 : cur.p0, s * gc, &ctl->full[slot]);
+                if constexpr (UM) {
+                    // chunk c: gate tile at 8 KB c, up tile 4 KB after it
+                    if (lane < gcv)
+                        tma_load_3d_stream(wdst + lane * UM_CHUNK_BYTES, &m.gate, 0, grow, s * gc + lane,
+                                           &ctl->full[slot], policy);
+                    else if (lane >= 8 && lane < 8 + gcv)
+                        tma_load_3d_stream(wdst + (lane - 8) * UM_CHUNK_BYTES + UM_TILE, &m.up, 0, grow,
+                                           s * gc + lane - 8, &ctl->full[slot], policy);
+                    // x rows of all B tokens for this column range, one swizzled box
+                    if (lane == 16) tma_load_3d(odst, &m.x, 0, 0, s * gc, &ctl->full[slot]);
+                } else {
+                    if (lane == 0) tma_load_3d_stream(wdst, &m.gate, 0, grow, s * gc, &ctl->full[slot], policy);
+                    if (lane == 1) tma_load_3d_stream(wdst + UP_OFF, &m.up, 0, grow, s * gc, &ctl->full[slot], policy);
+                    // the tile's pair rows of the dispatched x in one swizzled box
+                    if (lane == 2) tma_load_3d(odst, &m.x, 0, cur.p0, s * gc, &ctl->full[slot]);
+                }
             } else {
                 if (lane == 0)
                     tma_load_3d_stream(wdst, &m.down, 0, cur.e * a.d + cur.row0, (cur.k0 + s) * dc, &ctl->full[slot],
@@ -584,57 +642,12 @@ __device__ __forceinline__ void d_stage(uint32_t wbase, uint32_t hbase, int hrow
     }
 }
 
-// Wide dense mode.  Gate/up: warp w takes rows 16 (w / 4) .. + 16 of the
-// 32-row unit and tokens 16 (w % 4) .. + 16 (two n-tiles) over every k-step
-// of the stage, so each (row, token) sum is one warp's own, in k order.
-__device__ __forceinline__ void gu_stage_wide(uint32_t wbase, uint32_t xbase, int x_tile, int kvalid, int warp,
-                                              int lane, float (&acc_g)[4][4], float (&acc_u)[4][4]) {
-    const int nks = kvalid / 16;
-    const int r = (warp >> 2) * 16 + (lane & 15);
-    const int n = (warp & 3) * 16 + (lane & 7) + ((lane >> 4) << 3);
-#pragma unroll 4
-    for (int ks = 0; ks < nks; ++ks) {
-        const int box = ks >> 2;
-        const int chunk = ((ks & 3) << 1) + (lane >> 4);
-        uint32_t g0, g1, g2, g3, u0, u1, u2, u3, b0, b1, b2, b3;
-        ldsm_x4(swz(wbase + box * (WIDE_ROWS * 128), r, chunk), g0, g1, g2, g3);
-        ldsm_x4(swz(wbase + UP_OFF + box * (WIDE_ROWS * 128), r, chunk), u0, u1, u2, u3);
-        ldsm_x4(swz(xbase + box * x_tile, n, ((ks & 3) << 1) + ((lane >> 3) & 1)), b0, b1, b2, b3);
-        mma_bf16(acc_g[0], g0, g1, g2, g3, b0, b1);
-        mma_bf16(acc_g[1], g0, g1, g2, g3, b2, b3);
-        mma_bf16(acc_u[0], u0, u1, u2, u3, b0, b1);
-        mma_bf16(acc_u[1], u0, u1, u2, u3, b2, b3);
-    }
-}
-// Down: warp w takes rows 16 (w % 4) .. + 16 of the 64-row unit and tokens
-// 32 (w / 4) .. + 32 (four n-tiles) over every k-step of the stage.
-__device__ __forceinline__ void d_stage_wide(uint32_t wbase, uint32_t hbase, int hrows, int kvalid, int warp,
-                                             int lane, float (&acc)[4][4]) {
-    const int nks = kvalid / 16;
-    const int r = (warp & 3) * 16 + (lane & 15);
-#pragma unroll 4
-    for (int ks = 0; ks < nks; ++ks) {
-        const int box = ks >> 2;
-        uint32_t a0, a1, a2, a3;
-        ldsm_x4(swz(wbase + box * (D_ROWS * 128), r, ((ks & 3) << 1) + (lane >> 4)), a0, a1, a2, a3);
-        const int hchunk = ((ks & 3) << 1) + ((lane >> 3) & 1);
-#pragma unroll
-        for (int np = 0; np < 2; ++np) {
-            const int n = (warp >> 2) * 32 + np * 16 + (lane & 7) + ((lane >> 4) << 3);
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4(swz(hbase + box * (hrows * 128), n, hchunk), b0, b1, b2, b3);
-            mma_bf16(acc[2 * np], a0, a1, a2, a3, b0, b1);
-            mma_bf16(acc[2 * np + 1], a0, a1, a2, a3, b2, b3);
-        }
-    }
-}
-
 template <int NT>
 __device__ __forceinline__ void stage_dispatch(const StageHdr &h, uint32_t wbase, uint32_t obase, const ExpertArgs &a,
                                                int warp, int lane, float (&acc_g)[4][4], float (&acc_u)[4][4]) {
     if (h.type == UNIT_GU) {
         const int gk = 64 * a.gc;
-        gu_stage<NT>(wbase, obase, (a.dense ? a.bpad : TN) * 128, min(gk, a.d - h.k * gk), warp, lane, acc_g, acc_u);
+        gu_stage<NT>(wbase, obase, TN * 128, min(gk, a.d - h.k * gk), warp, lane, acc_g, acc_u);
     } else {
         const int dk = 64 * d_chunks_of(a.F);
         d_stage<NT>(wbase, obase, a.hrows, min(dk, a.F - h.k * dk), warp, lane, acc_g);
@@ -652,11 +665,10 @@ __device__ bool post_signal(SharedCtl *ctl, Counters *ctr, int q, int i) {
     return true;
 }
 
-// DNT: 0 = the token-tile count is taken per stage (the expert kernel:
-// any mode); 1..4 = dense mode with that many 8-token tiles, fixed for the
-// call; 5 = the wide dense mode.  A fixed count leaves only that path's code
-// in the consumer loop (the fused layer kernel is instantiated per count).
-template <class RG, int DNT = 0>
+// Tile-mode consumers (batches above 64 tokens): the eight warps split
+// every stage's k-steps (mma.sync), then reduce and apply the epilogue at
+// the unit's last stage.
+template <class RG>
 __device__ void consumer(const ExpertArgs &a, SharedCtl *ctl, unsigned char *slots, float *part) {
     constexpr int STAGES = RG::STAGES;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -665,7 +677,6 @@ __device__ void consumer(const ExpertArgs &a, SharedCtl *ctl, unsigned char *slo
     int tk[4][2];
     float wk[4][2];
     int nsig = 0;  // completions posted (thread 0)
-    bool lists_ready = !a.early;
     const int row = lane >> 2, col = (lane & 3) * 2;
     for (int g = 0;; ++g) {
         const int slot = g % STAGES;
@@ -680,41 +691,7 @@ __device__ void consumer(const ExpertArgs &a, SharedCtl *ctl, unsigned char *slo
             for (int j = 0; j < 4; ++j)
 #pragma unroll
                 for (int c = 0; c < 4; ++c) acc_g[j][c] = acc_u[j][c] = 0.0f;
-            if (h.type == UNIT_D && a.dense) {
-                // the dense weights are the selection's last output: in early
-                // mode wait for it to complete before the first down unit
-                if (!lists_ready) {
-                    if (a.lists_flag == nullptr) {
-                        asm volatile("griddepcontrol.wait;" ::: "memory");
-                    } else {
-                        // fused layer kernel: the selection CTA raises the flag
-                        if (ct == 0) {
-                            const unsigned long long t0 = global_ns();
-                            while (ld_acquire(a.lists_flag) < 1) {
-                                if (ctl->abort_flag) break;
-                                if (global_ns() - t0 > a.wait_ns) {
-                                    record_error(a.ctr, ctl, DEV_TIMEOUT_DEP);
-                                    break;
-                                }
-                                __nanosleep(64);
-                            }
-                        }
-                        consumer_bar();
-                        if (ctl->abort_flag) return;
-                    }
-                    lists_ready = true;
-                }
-                // wide mode: this warp's tokens start at 32 (warp / 4)
-                const int tb = (DNT == 5 || (DNT == 0 && RG::WIDE_OK && a.wide)) ? (warp >> 2) * 32 : 0;
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-#pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        const int t = tb + j * 8 + col + c;
-                        tk[j][c] = t;
-                        wk[j][c] = t < a.B ? __ldcg(a.wd + static_cast<size_t>(h.i_act) * a.B + t) : 0.0f;
-                    }
-            } else if (h.type == UNIT_D) {
+            if (h.type == UNIT_D) {
                 // tokens and gate weights this thread combines; used at the
                 // unit's last stage, loaded now so the latency is hidden
 #pragma unroll
@@ -733,27 +710,12 @@ __device__ void consumer(const ExpertArgs &a, SharedCtl *ctl, unsigned char *slo
         }
         const uint32_t wbase = smem_u32(slots + slot * RG::SLOT_BYTES);
         const uint32_t obase = wbase + W_BYTES;
-        const bool wide = DNT == 5 || (DNT == 0 && RG::WIDE_OK && a.wide);
-        const int nt = (DNT >= 1 && DNT <= 4) ? DNT
-                       : wide                 ? 4
-                       : (h.type == UNIT_GU && a.dense) ? (a.bpad >> 3) : ((h.n + 7) >> 3);
-        if constexpr (DNT >= 1 && DNT <= 4) {
-            stage_dispatch<(DNT >= 1 && DNT <= 4) ? DNT : 1>(h, wbase, obase, a, warp, lane, acc_g, acc_u);
-        } else if (wide) {
-            if (h.type == UNIT_GU) {
-                const int gk = 64 * a.gc;
-                gu_stage_wide(wbase, obase, a.bpad * 128, min(gk, a.d - h.k * gk), warp, lane, acc_g, acc_u);
-            } else {
-                const int dk = 64 * d_chunks_of(a.F);
-                d_stage_wide(wbase, obase, a.hrows, min(dk, a.F - h.k * dk), warp, lane, acc_g);
-            }
-        } else {
-            switch (nt) {
-                case 1: stage_dispatch<1>(h, wbase, obase, a, warp, lane, acc_g, acc_u); break;
-                case 2: stage_dispatch<2>(h, wbase, obase, a, warp, lane, acc_g, acc_u); break;
-                case 3: stage_dispatch<3>(h, wbase, obase, a, warp, lane, acc_g, acc_u); break;
-                default: stage_dispatch<4>(h, wbase, obase, a, warp, lane, acc_g, acc_u); break;
-            }
+        const int nt = (h.n + 7) >> 3;
+        switch (nt) {
+            case 1: stage_dispatch<1>(h, wbase, obase, a, warp, lane, acc_g, acc_u); break;
+            case 2: stage_dispatch<2>(h, wbase, obase, a, warp, lane, acc_g, acc_u); break;
+            case 3: stage_dispatch<3>(h, wbase, obase, a, warp, lane, acc_g, acc_u); break;
+            default: stage_dispatch<4>(h, wbase, obase, a, warp, lane, acc_g, acc_u); break;
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctl->empty[slot]);
@@ -761,36 +723,15 @@ __device__ void consumer(const ExpertArgs &a, SharedCtl *ctl, unsigned char *slo
         if (h.s != h.ns - 1) continue;
 
         // ---- unit epilogue
-        if (h.type == UNIT_GU && wide) {
-            // each warp owns complete sums: h = silu(g) u straight to H
-            const int r0 = h.row0 + (warp >> 2) * 16 + row;
-#pragma unroll
-            for (int j = 0; j < 2; ++j)
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const int t = (warp & 3) * 16 + j * 8 + col + (c & 1);
-                    if (t < a.B) {
-                        const float gs = acc_g[j][c], us = acc_u[j][c];
-                        const float hv = gs / (1.0f + __expf(-gs)) * us;
-                        a.h[static_cast<size_t>(h.p0 + t) * a.F + r0 + ((c >> 1) << 3)] =
-                            __bfloat16_as_ushort(__float2bfloat16_rn(hv));
-                    }
-                }
-            // H is read by other CTAs through TMA (the async proxy)
-            asm volatile("fence.proxy.async.global;" ::: "memory");
-            consumer_bar();
-            if (ct == 0 && !post_signal(ctl, a.ctr, nsig++, h.i_act)) return;
-        } else if (h.type == UNIT_D) {
-            // each warp holds a k-half of a 16-row block (wide mode: all of k
-            // for 32 tokens): both halves add into y
+        if (h.type == UNIT_D) {
+            // each warp holds a k-half of a 16-row block: both halves add into y
             const int i_base = h.row0 + (warp & 3) * 16 + row;
-            const int tb = wide ? (warp >> 2) * 32 : 0;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 if (j >= nt) break;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    const int n = tb + j * 8 + col + (c & 1);
+                    const int n = j * 8 + col + (c & 1);
                     if (n < h.n && wk[j][c & 1] != 0.0f) {
                         const int i = i_base + ((c >> 1) << 3);
                         atomicAdd(a.y + static_cast<size_t>(tk[j][c & 1]) * a.d + i, wk[j][c & 1] * acc_g[j][c]);
@@ -831,14 +772,13 @@ __device__ void consumer(const ExpertArgs &a, SharedCtl *ctl, unsigned char *slo
             }
             consumer_bar();
             for (int idx = ct; idx < 16 * h.n; idx += NCW * 32) {
-                // column n: token n (dense mode) or the tile's pair n; H row p0 + n
+                // column n: the tile's pair n; H row p0 + n
                 const int r = idx & 15, n = idx >> 4;
-                const int cn = n;
                 float gs = 0.0f, us = 0.0f;
 #pragma unroll
                 for (int wv = 0; wv < NCW / 2; ++wv) {
-                    gs += part[(wv * 2 + 0) * 16 * PART_LD + r * PART_LD + cn];
-                    us += part[(wv * 2 + 1) * 16 * PART_LD + r * PART_LD + cn];
+                    gs += part[(wv * 2 + 0) * 16 * PART_LD + r * PART_LD + n];
+                    us += part[(wv * 2 + 1) * 16 * PART_LD + r * PART_LD + n];
                 }
                 const float hv = gs / (1.0f + __expf(-gs)) * us;
                 a.h[static_cast<size_t>(h.p0 + n) * a.F + h.row0 + r] =
@@ -866,6 +806,197 @@ __device__ void signaller(const ExpertArgs &a, SharedCtl *ctl) {
         if (i < 0) return;
         __threadfence();
         atomicAdd(&a.ctr->gu_done[i], 1);
+    }
+}
+
+// ------------------------------------------------ tensor-core path (dense) --
+// TMEM columns of the CTA's allocation: two accumulator buffers, each
+// NISSUE partial accumulators of bpad columns (a power of two, at least 32).
+__device__ __forceinline__ int tmem_cols_for(int bpad) {
+    int c = 32;
+    while (c < 2 * NISSUE * bpad) c <<= 1;
+    return c;
+}
+
+// Issuer p (one thread of each issuer warp): for every stage it waits for
+// the copies, issues k-steps p, p + NISSUE, ... of the stage (64-row x
+// bpad-column MMAs, K = 16 each) into its partial accumulator of the unit's
+// buffer, and commits them to the stage's empty barrier (the slot is free
+// once every issuer's MMAs have read it).  At a unit's last stage it commits
+// to the buffer's full barrier as well.  A gate/up chunk is [32 gate rows]
+// [32 up rows] of 64 columns and a down chunk 64 rows of Wdown, both one
+// 8 KB operand; the token rows (x, or H) are the B operand, bpad rows per
+// chunk.  Issuer 0 also hands the unit's header to the epilogue.
+__device__ void umma_issuer(const ExpertArgs &a, SharedCtl *ctl, unsigned char *slots, int stages, int slot_bytes,
+                            uint32_t tmem, int p) {
+    const uint32_t idesc = umma_idesc_bf16(a.bpad);
+    const uint32_t b_chunk = static_cast<uint32_t>(a.bpad) * 128u;
+    const uint32_t buf_stride = static_cast<uint32_t>(tmem_cols_for(a.bpad) / 2);
+    const int gk = 64 * a.gc, dk = 64 * d_chunks_of(a.F);
+    int unit = 0;  // units started
+    for (int g = 0;; ++g) {
+        const int slot = g % stages;
+        if (!wait_phase(&ctl->full[slot], (g / stages) & 1, ctl, a.ctr, DEV_TIMEOUT_FULL)) break;
+        if (p == 0) ctl->consumed = g + 1;  // the copies have landed
+        const StageHdr h = ctl->hdr[slot];
+        const int b = unit & 1;
+        if (h.type == UNIT_END || h.s == 0) {
+            // the buffer's previous unit must have been read out
+            if (unit >= 2 && !wait_phase(&ctl->acc_empty[b], ((unit >> 1) - 1) & 1, ctl, a.ctr, DEV_TIMEOUT_EMPTY))
+                break;
+            tc_fence_after();
+            if (p == 0) {
+                AccHdr &ah = ctl->acc_hdr[b];
+                ah.type = h.type;
+                ah.i_act = h.i_act;
+                ah.row0 = h.row0;
+                ah.p0 = h.p0;
+                ah.n = h.n;
+                // the extra arrival of the buffer's phase; releases the header
+                mbar_arrive(&ctl->acc_full[b]);
+            }
+            if (h.type == UNIT_END) {
+                mbar_arrive(&ctl->acc_full[b]);
+                break;
+            }
+        }
+        const uint32_t wbase = smem_u32(slots + slot * slot_bytes);
+        const uint32_t obase = wbase + W_BYTES;
+        const int nks = (h.type == UNIT_GU ? min(gk, a.d - h.k * gk) : min(dk, a.F - h.k * dk)) >> 4;
+        const uint32_t dcol = tmem + static_cast<uint32_t>(b) * buf_stride + static_cast<uint32_t>(p * a.bpad);
+        // nks >= 4 = NISSUE (d and d_ff are multiples of 64): every issuer
+        // starts its partial sum at stage 0
+        for (int ks = p; ks < nks; ks += NISSUE) {
+            const uint32_t c = static_cast<uint32_t>(ks >> 2), kk = static_cast<uint32_t>(ks & 3) * 32u;
+            umma_bf16(dcol, umma_desc(wbase + c * UM_CHUNK_BYTES + kk), umma_desc(obase + c * b_chunk + kk), idesc,
+                      (h.s > 0 || ks >= NISSUE) ? 1u : 0u);
+        }
+        umma_commit(smem_u32(&ctl->empty[slot]));
+        if (h.s == h.ns - 1) {
+            umma_commit(smem_u32(&ctl->acc_full[b]));
+            ++unit;
+        }
+    }
+    // every MMA issued must have completed before the CTA's shared memory
+    // and tensor memory are released
+    umma_commit(smem_u32(&ctl->mma_done));
+    const unsigned long long t0 = global_ns();
+    while (!mbar_try_wait(&ctl->mma_done, 0)) {
+        if (global_ns() - t0 > DRAIN_LIMIT_NS) break;
+    }
+}
+
+// The eight epilogue warps, one accumulator buffer per unit in turn: warp w
+// reads TMEM lanes 32 (w % 4) .. (rows 16 (w % 4) ..) for the column groups
+// of 8 tokens g = w / 4, w / 4 + 2, ..., adds the issuers' partial sums in
+// issuer order, releases the buffer and copies the values to shared memory
+// as [token][64 rows]; then
+//   gate/up unit: rows 0..31 are g, rows 32..63 u: h = silu(g) u -> H
+//     (bf16, two rows per thread), and thread 0 publishes the completion;
+//   down unit:    y[t][row0 + r] += wd[slot][t] acc[t][r], four rows per
+//     vector atomic.
+__device__ void umma_epilogue(const ExpertArgs &a, SharedCtl *ctl, float *xch, uint32_t tmem) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int ct = threadIdx.x;  // 0 .. NCW*32-1
+    const int q = warp & 3, half = warp >> 2;
+    const int ncg = a.bpad >> 3;
+    const uint32_t buf_stride = static_cast<uint32_t>(tmem_cols_for(a.bpad) / 2);
+    bool lists_ready = !a.early;
+    // Thread 0 takes every wait and passes its outcome through shared
+    // memory, so that all epilogue threads leave together (none is left at a
+    // barrier): epi_go is read between the first and second barrier of a
+    // unit, epi_lists after the second.
+    for (int u = 0;; ++u) {
+        const int b = u & 1;
+        if (ct == 0) ctl->epi_go = wait_phase(&ctl->acc_full[b], (u >> 1) & 1, ctl, a.ctr, DEV_TIMEOUT_FULL) ? 1 : 0;
+        consumer_bar();  // also: the previous unit's readers of xch are done
+        if (!ctl->epi_go) return;
+        const AccHdr ah = ctl->acc_hdr[b];
+        if (ah.type == UNIT_END) return;
+        tc_fence_after();
+        // the issuers' partial accumulators, summed in issuer order
+        float v[4][8];
+        const uint32_t tb = tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(b) * buf_stride;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int cg = half + 2 * j;
+            if (cg < ncg) {
+                tmem_ld8(tb + static_cast<uint32_t>(cg * 8), v[j]);
+#pragma unroll
+                for (int pi = 1; pi < NISSUE; ++pi) {
+                    float w8[8];
+                    tmem_ld8(tb + static_cast<uint32_t>(pi * a.bpad + cg * 8), w8);
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) v[j][c] += w8[c];
+                }
+            }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->acc_empty[b]);
+        if (ah.type == UNIT_D && !lists_ready) {
+            // the dense weights are the selection's last output: in early
+            // mode wait for them before the first down epilogue
+            if (a.lists_flag == nullptr) {
+                asm volatile("griddepcontrol.wait;" ::: "memory");
+                if (ct == 0) ctl->epi_lists = 1;
+            } else if (ct == 0) {
+                int ok = 1;
+                const unsigned long long t0 = global_ns();
+                while (ld_acquire(a.lists_flag) < 1) {
+                    if (ctl->abort_flag) { ok = 0; break; }
+                    if (global_ns() - t0 > a.wait_ns) {
+                        record_error(a.ctr, ctl, DEV_TIMEOUT_DEP);
+                        ok = 0;
+                        break;
+                    }
+                    __nanosleep(64);
+                }
+                ctl->epi_lists = ok;
+            }
+            lists_ready = true;
+        }
+        if (lane < 16) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int cg = half + 2 * j;
+                if (cg < ncg) {
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) xch[(cg * 8 + c) * 64 + 16 * q + lane] = v[j][c];
+                }
+            }
+        }
+        consumer_bar();
+        if (ah.type == UNIT_GU) {
+            for (int idx = ct; idx < 16 * a.B; idx += NCW * 32) {
+                const int t = idx >> 4, r = (idx & 15) * 2;
+                const float2 gs = *reinterpret_cast<const float2 *>(xch + t * 64 + r);
+                const float2 us = *reinterpret_cast<const float2 *>(xch + t * 64 + UM_ROWS + r);
+                const float h0 = gs.x / (1.0f + __expf(-gs.x)) * us.x;
+                const float h1 = gs.y / (1.0f + __expf(-gs.y)) * us.y;
+                const unsigned packed = static_cast<unsigned>(__bfloat16_as_ushort(__float2bfloat16_rn(h0))) |
+                                        (static_cast<unsigned>(__bfloat16_as_ushort(__float2bfloat16_rn(h1))) << 16);
+                *reinterpret_cast<unsigned *>(a.h + static_cast<size_t>(ah.p0 + t) * a.F + ah.row0 + r) = packed;
+            }
+            // H is read by other CTAs through TMA (the async proxy)
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+            consumer_bar();
+            if (ct == 0) {
+                __threadfence();
+                atomicAdd(&a.ctr->gu_done[ah.i_act], 1);
+            }
+        } else {
+            if (!ctl->epi_lists) return;
+            for (int idx = ct; idx < 16 * a.B; idx += NCW * 32) {
+                const int t = idx >> 4, r = (idx & 15) * 4;
+                const float w = __ldcg(a.wd + static_cast<size_t>(ah.i_act) * a.B + t);
+                if (w != 0.0f) {
+                    const float4 s4 = *reinterpret_cast<const float4 *>(xch + t * 64 + r);
+                    atomicAdd(reinterpret_cast<float4 *>(a.y + static_cast<size_t>(t) * a.d + ah.row0 + r),
+                              make_float4(w * s4.x, w * s4.y, w * s4.z, w * s4.w));
+                }
+            }
+        }
     }
 }
 
@@ -904,17 +1035,24 @@ struct CtaSmem {
             (reinterpret_cast<uintptr_t>(raw) + 1023) & ~static_cast<uintptr_t>(1023));
         slots = base;
         part = reinterpret_cast<float *>(base + RG::STAGES * RG::SLOT_BYTES);
-        ctl = reinterpret_cast<SharedCtl *>(part + PART_FLOATS);
+        ctl = reinterpret_cast<SharedCtl *>(base + RG::STAGES * RG::SLOT_BYTES + RG::PART_BYTES);
     }
 };
 
 // Barriers and flags of a CTA (thread 0).
-template <class RG>
+// UM: the tensor-core path (a stage is released by the issuers' MMA commits).
+template <class RG, bool UM>
 __device__ void ctl_init(SharedCtl *ctl, unsigned long long wait_ns) {
     for (int s = 0; s < RG::STAGES; ++s) {
         mbar_init(&ctl->full[s], 1);
-        mbar_init(&ctl->empty[s], NCW);
+        mbar_init(&ctl->empty[s], UM ? NISSUE : NCW);  // one MMA commit per issuer
     }
+    for (int b = 0; b < 2; ++b) {
+        mbar_init(&ctl->acc_full[b], NISSUE + 1);  // the first issuer's arrive + every issuer's commit
+        mbar_init(&ctl->acc_empty[b], NCW);
+    }
+    mbar_init(&ctl->mma_done, NISSUE);
+    ctl->epi_lists = 1;
     for (int s = 0; s < SIG_SLOTS; ++s) {
         mbar_init(&ctl->sig_full[s], 1);
         mbar_init(&ctl->sig_empty[s], 1);
@@ -1041,15 +1179,43 @@ __device__ void table_from_lists(const ExpertArgs &a, SharedCtl *ctl, int lane) 
     }
 }
 
-template <class RG, int DNT = 0>
+// The roles of an expert CTA.  Tile mode: producer, signal warp, eight
+// mma.sync consumer warps.  Dense mode (UM): producer, NISSUE MMA issuer
+// warps (one thread each; the first holds the CTA's TMEM allocation), eight
+// epilogue warps.
+template <class RG, bool UM>
 __device__ __forceinline__ void run_roles(const ExpertArgs &a, const ExpertMaps &maps, const CtaSmem<RG> &sm) {
-    const int warp = threadIdx.x >> 5;
-    if (warp == NCW) {
-        producer<RG>(a, maps, sm.ctl, sm.slots);
-    } else if (warp == NCW + 1) {
-        signaller(a, sm.ctl);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if constexpr (!UM) {
+        if (warp == NCW) {
+            producer<RG, false>(a, maps, sm.ctl, sm.slots);
+        } else if (warp == NCW + 1) {
+            signaller(a, sm.ctl);
+        } else {
+            consumer<RG>(a, sm.ctl, sm.slots, sm.part);
+        }
     } else {
-        consumer<RG, DNT>(a, sm.ctl, sm.slots, sm.part);
+        const int cols = tmem_cols_for(a.bpad);
+        if (warp == NCW + 1) tmem_alloc(smem_u32(&sm.ctl->tmem), cols);
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        const uint32_t tmem = sm.ctl->tmem;
+        if (warp == NCW) {
+            producer<RG, true>(a, maps, sm.ctl, sm.slots);
+        } else if (warp > NCW) {
+            if (lane == 0) umma_issuer(a, sm.ctl, sm.slots, RG::STAGES, RG::SLOT_BYTES, tmem, warp - NCW - 1);
+        } else {
+            umma_epilogue(a, sm.ctl, sm.part, tmem);
+        }
+        // the issuers have waited for their MMAs, the epilogue for its loads
+        tc_fence_before();
+        __syncthreads();
+        if (warp == NCW + 1) {
+            __syncwarp();
+            tc_fence_after();
+            tmem_dealloc(tmem, cols);
+        }
     }
 }
 
@@ -1078,21 +1244,22 @@ __device__ void cta_exit(const ExpertArgs &a, SharedCtl *ctl) {
     }
 }
 
-template <class RG>
-__global__ void __launch_bounds__(NTHREADS, 1)
+// UM: dense mode on the tensor cores (B <= 64); otherwise tile mode.
+template <class RG, bool UM>
+__global__ void __launch_bounds__(cta_threads<UM>(), 1)
     expert_ffn_kernel(const __grid_constant__ ExpertMaps maps, const ExpertArgs a) {
     extern __shared__ unsigned char smem_raw[];
     const CtaSmem<RG> sm(smem_raw);
     SharedCtl *ctl = sm.ctl;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (threadIdx.x == 0) ctl_init<RG>(ctl, a.wait_ns);
+    if (threadIdx.x == 0) ctl_init<RG, UM>(ctl, a.wait_ns);
     if (warp == NCW && lane == 0) prefetch_expert_maps(maps);
     // everything above overlaps the previous kernel (selection or input
     // preparation); the lists are complete once it has
     asm volatile("griddepcontrol.wait;" ::: "memory");
     if (warp == NCW) table_from_lists(a, ctl, lane);
     __syncthreads();
-    run_roles<RG>(a, maps, sm);
+    run_roles<RG, UM>(a, maps, sm);
     cta_exit(a, ctl);
 }
 
@@ -1167,8 +1334,8 @@ __device__ __forceinline__ void rank_union(const ExpertArgs &a, const LayerArgs 
     }
 }
 
-template <class RG, int NI, int DNT>
-__global__ void __launch_bounds__(NTHREADS, 1)
+template <class RG, int NI>
+__global__ void __launch_bounds__(NTHREADS_UM, 1)
     layer_kernel(const __grid_constant__ ExpertMaps maps, const __grid_constant__ RouterMaps rmaps,
                  const ExpertArgs a, const LayerArgs L) {
     extern __shared__ unsigned char smem_raw[];
@@ -1219,7 +1386,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 issue_rows(item, true, false);
             }
         }
-        ctl_init<RG>(ctl, a.wait_ns);
+        ctl_init<RG, true>(ctl, a.wait_ns);
         s_ok = 1;
     }
     if (threadIdx.x < E_MAX / 32) s_set[threadIdx.x] = 0u;
@@ -1348,7 +1515,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         else table_from_mask(a, ctl, 0u, lane);
     }
     __syncthreads();
-    run_roles<RG, DNT>(a, maps, sm);
+    run_roles<RG, true>(a, maps, sm);
     cta_exit(a, ctl);
 }
 
@@ -1474,12 +1641,13 @@ int g_num_sms[MAX_DEVICES] = {0};
 
 int expert_ffn_h_rows(int B) { return B <= DENSE_MAX ? (B + 7) / 8 * 8 : TN; }
 int expert_ffn_dense_batch(int B) { return B <= DENSE_MAX ? 1 : 0; }
-int expert_ffn_gu_rows(int B) { return B > TN && B <= DENSE_MAX ? WIDE_ROWS : GU_ROWS; }
+int expert_ffn_gu_rows(int B) { return B <= DENSE_MAX ? UM_ROWS : GU_ROWS; }
 int expert_ffn_d_rows() { return D_ROWS; }
 int expert_ffn_gu_chunks(int d, int B) {
-    const int cap = B > TN && B <= DENSE_MAX ? WIDE_CHUNKS : GU_CHUNKS;
+    const int cap = B <= DENSE_MAX ? UM_CHUNKS : GU_CHUNKS;
     return d / 64 < cap ? d / 64 : cap;
 }
+int expert_ffn_gu_box_chunks(int d, int B) { return B <= DENSE_MAX ? 1 : expert_ffn_gu_chunks(d, B); }
 int expert_ffn_d_chunks(int F) { return F / 64 < D_CHUNKS ? F / 64 : D_CHUNKS; }
 
 cudaError_t launch_ffn_prep(const float *x, const moe_dims_t &d, uint16_t *xb, uint16_t *xd, float *y,
@@ -1567,7 +1735,6 @@ ExpertArgs make_expert_args(const uint16_t *xb, const moe_dims_t &d, const moe_l
     a.unit_ctas = unit_ctas;
     a.lists_flag = nullptr;
     a.dense = d.B <= DENSE_MAX ? 1 : 0;
-    a.wide = d.B > TN && d.B <= DENSE_MAX ? 1 : 0;
     a.gu_rows = expert_ffn_gu_rows(d.B);
     a.gc = expert_ffn_gu_chunks(d.d, d.B);
     a.bpad = (d.B + 7) / 8 * 8;
@@ -1633,14 +1800,14 @@ LayerArgs make_layer_router(const moe_dims_t &d, int grid, int ring_bytes) {
     return L;
 }
 
-template <class RG, int NI, int DNT>
+template <class RG, int NI>
 cudaError_t launch_layer_ni(const ExpertMaps &maps, const RouterMaps &rmaps, const ExpertArgs &a,
                             const LayerArgs &L, int grid, int dev, cudaStream_t s) {
-    cudaError_t err = configure_smem(layer_kernel<RG, NI, DNT>, smem_bytes<RG>(), dev);
+    cudaError_t err = configure_smem(layer_kernel<RG, NI>, smem_bytes<RG>(), dev);
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(NTHREADS);
+    cfg.blockDim = dim3(NTHREADS_UM);
     cfg.dynamicSmemBytes = smem_bytes<RG>();
     cfg.stream = s;
     // every CTA must be resident: the CTAs wait for one another at the
@@ -1653,9 +1820,28 @@ cudaError_t launch_layer_ni(const ExpertMaps &maps, const RouterMaps &rmaps, con
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = L.chained ? 2 : 1;
-    return cudaLaunchKernelEx(&cfg, layer_kernel<RG, NI, DNT>, maps, rmaps, a, L);
+    return cudaLaunchKernelEx(&cfg, layer_kernel<RG, NI>, maps, rmaps, a, L);
 }
 
+}  // namespace
+
+namespace {
+template <class RG, bool UM>
+cudaError_t launch_expert_ffn_rg(const ExpertMaps &maps, const ExpertArgs &a, int sms, int dev, cudaStream_t s) {
+    cudaError_t err = configure_smem(expert_ffn_kernel<RG, UM>, smem_bytes<RG>(), dev);
+    if (err != cudaSuccess) return err;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(sms);
+    cfg.blockDim = dim3(cta_threads<UM>());
+    cfg.dynamicSmemBytes = smem_bytes<RG>();
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;  // always chained to the previous kernel with programmatic dependent launch
+    return cudaLaunchKernelEx(&cfg, expert_ffn_kernel<RG, UM>, maps, a);
+}
 }  // namespace
 
 cudaError_t launch_expert_ffn(const ExpertMaps &maps, const uint16_t *xb, const moe_dims_t &d,
@@ -1664,23 +1850,12 @@ cudaError_t launch_expert_ffn(const ExpertMaps &maps, const uint16_t *xb, const 
     int dev = 0, sms = 0;
     cudaError_t err = device_sms(&dev, &sms);
     if (err != cudaSuccess) return err;
-    const bool small = d.B <= 16;
-    err = small ? configure_smem(expert_ffn_kernel<RingSmallB>, smem_bytes<RingSmallB>(), dev)
-                : configure_smem(expert_ffn_kernel<RingLargeB>, smem_bytes<RingLargeB>(), dev);
-    if (err != cudaSuccess) return err;
     const ExpertArgs a = make_expert_args(xb, d, l, y, h, wd, ctr, sms);
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(sms);
-    cfg.blockDim = dim3(NTHREADS);
-    cfg.dynamicSmemBytes = small ? smem_bytes<RingSmallB>() : smem_bytes<RingLargeB>();
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;  // always chained to the previous kernel with programmatic dependent launch
-    return small ? cudaLaunchKernelEx(&cfg, expert_ffn_kernel<RingSmallB>, maps, a)
-                 : cudaLaunchKernelEx(&cfg, expert_ffn_kernel<RingLargeB>, maps, a);
+    // dense mode on the tensor cores, the ring sized for the token rows
+    if (d.B <= 16) return launch_expert_ffn_rg<RingB16, true>(maps, a, sms, dev, s);
+    if (d.B <= 32) return launch_expert_ffn_rg<RingB32, true>(maps, a, sms, dev, s);
+    if (d.B <= DENSE_MAX) return launch_expert_ffn_rg<RingB64, true>(maps, a, sms, dev, s);
+    return launch_expert_ffn_rg<RingB64, false>(maps, a, sms, dev, s);
 }
 
 cudaError_t launch_layer_fused(const ExpertMaps &maps, const RouterMaps &rmaps, const moe_dims_t &d,
@@ -1693,7 +1868,6 @@ cudaError_t launch_layer_fused(const ExpertMaps &maps, const RouterMaps &rmaps, 
     cudaError_t err = device_sms(&dev, &sms);
     if (err != cudaSuccess) return err;
     if (sms < 2) return cudaErrorInvalidConfiguration;
-    const bool small = d.B <= 16;
     // the last CTA runs the selection; the others stream the experts
     ExpertArgs a = make_expert_args(xb, d, lists, y, h, wd, ctr, sms - 1);
     a.early = 1;
@@ -1701,7 +1875,9 @@ cudaError_t launch_layer_fused(const ExpertMaps &maps, const RouterMaps &rmaps, 
     const bool batch_rule = rule.mode == MOE_RESELECT_XSHARE || rule.mode == MOE_RESELECT_AFFINITY ||
                             rule.mode == MOE_RESELECT_XSHARE_HIER;
     a.pub_target = 1;
-    const int ring = small ? RingSmallB::STAGES * RingSmallB::SLOT_BYTES : RingLargeB::STAGES * RingLargeB::SLOT_BYTES;
+    const int ring = d.B <= 16 ? RingB16::STAGES * RingB16::SLOT_BYTES
+                     : d.B <= 32 ? RingB32::STAGES * RingB32::SLOT_BYTES
+                                 : RingB64::STAGES * RingB64::SLOT_BYTES;
     LayerArgs L = make_layer_router(d, sms, ring);
     L.x = x;
     L.bias = bias;
@@ -1715,21 +1891,15 @@ cudaError_t launch_layer_fused(const ExpertMaps &maps, const RouterMaps &rmaps, 
     L.sel.publish_set = batch_rule ? 1 : 0;
     const size_t sel_smem = reselect_smem(d, rule, &L.sel.cache_rows);
     if (sel_smem > static_cast<size_t>(ring)) return cudaErrorInvalidValue;
-    // instantiated per token-tile count (small ring: 1-2 tiles of 8
-    // tokens, large ring: 3-4 tiles or the wide mode) and for logit rows of
-    // up to 128 or 256 experts per warp
-    const int dnt = d.B > TN ? 5 : (d.B + 7) / 8;
+    // instantiated per ring (up to 16, 32 or 64 tokens) and for logit rows
+    // of up to 128 or 256 experts per warp
     const bool ni8 = ni_for(d.E) > 4;
-#define MOE_LAYER_CASE(RGT, DN)                                                                        \
-    return ni8 ? launch_layer_ni<RGT, 8, DN>(maps, rmaps, a, L, sms, dev, s)                          \
-               : launch_layer_ni<RGT, 4, DN>(maps, rmaps, a, L, sms, dev, s)
-    switch (dnt) {
-        case 1: MOE_LAYER_CASE(RingSmallB, 1);
-        case 2: MOE_LAYER_CASE(RingSmallB, 2);
-        case 3: MOE_LAYER_CASE(RingLargeB, 3);
-        case 4: MOE_LAYER_CASE(RingLargeB, 4);
-        default: MOE_LAYER_CASE(RingLargeB, 5);
-    }
+#define MOE_LAYER_CASE(RGT)                                                                            \
+    return ni8 ? launch_layer_ni<RGT, 8>(maps, rmaps, a, L, sms, dev, s)                              \
+               : launch_layer_ni<RGT, 4>(maps, rmaps, a, L, sms, dev, s)
+    if (d.B <= 16) MOE_LAYER_CASE(RingB16);
+    if (d.B <= 32) MOE_LAYER_CASE(RingB32);
+    MOE_LAYER_CASE(RingB64);
 #undef MOE_LAYER_CASE
 }
 

@@ -156,6 +156,7 @@ int expert_ffn_dense_batch(int B);    // 1 if gate/up stages load all B token ro
 int expert_ffn_gu_rows(int B);        // rows of Wgate / Wup per gate-up unit
 int expert_ffn_d_rows();              // rows of Wdown per down unit
 int expert_ffn_gu_chunks(int d, int B);  // 64-column chunks of d per gate-up stage
+int expert_ffn_gu_box_chunks(int d, int B);  // chunks per gate (or up) copy: 1 in dense mode
 int expert_ffn_d_chunks(int d_ff);    // 64-column chunks of d_ff per down stage
 
 // Builds the expert kernel's TMA descriptors (weights, H scratch at `h`,
