@@ -263,6 +263,9 @@ def run_ours(args, w, rank, world, local_rank):
     y = torch.empty(B, S.d, dtype=torch.float32, device=dev)
     nact_t = torch.zeros(4, dtype=torch.int32, device=dev)
     s = torch.cuda.Stream(dev)
+    # the copies and the zero-filled workspace were written on the default
+    # stream: the calls on s must not start before they are complete
+    s.wait_stream(torch.cuda.current_stream(dev))
 
     def layer(r):
         g, u, dn, wg = copies[r]
@@ -377,6 +380,7 @@ def run_ours(args, w, rank, world, local_rank):
     xs[0] = x
     stack_layers = [(c[3], bias, c[0], c[1], c[2]) for c in copies]
     stack_ws = moe.new_workspace(B, S.d, S.E, S.k, S.F, dev)
+    s.wait_stream(torch.cuda.current_stream(dev))
     with torch.cuda.stream(s):
         moe.moe_decode_stack(xs, stack_layers, S.k, mode, k0, budget, ws=stack_ws, group=group)
     s.synchronize()
@@ -510,6 +514,7 @@ def run_channels(args, w, rank, world, local_rank):
     ws = torch.zeros(moe.load_library().moe_channels_workspace_bytes(moe.Dims(B, S.d, S.E, S.k, S.F)),
                      dtype=torch.uint8, device=dev)
     s = torch.cuda.Stream(dev)
+    s.wait_stream(torch.cuda.current_stream(dev))
 
     def call(r):
         g, u, _ = copies[r]
@@ -588,6 +593,7 @@ def run_sweep(args):
             ws = moe.new_workspace(B, S.d, S.E, S.k, S.F, dev)
             y = torch.empty(B, S.d, dtype=torch.float32, device=dev)
             nact_t = torch.zeros(4, dtype=torch.int32, device=dev)
+            s.wait_stream(torch.cuda.current_stream(dev))
 
             def layer(r):
                 g, u, dn, wg = copies[r]

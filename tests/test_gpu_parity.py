@@ -303,6 +303,8 @@ def test_layer_graph_replays(name, B, mode, k0):
     ys = [torch.empty(B, S.d, dtype=torch.float32, device="cuda") for _ in range(4)]
     sels = [torch.empty(B, S.k, dtype=torch.int32, device="cuda") for _ in range(4)]
     s = torch.cuda.Stream()
+    # the workspace was zero-filled on the default stream
+    s.wait_stream(torch.cuda.current_stream())
 
     def calls():
         for i in range(4):
