@@ -1179,6 +1179,13 @@ __device__ void table_from_lists(const ExpertArgs &a, SharedCtl *ctl, int lane) 
     }
 }
 
+// Allocation of the CTA's TMEM columns by the first issuer warp at kernel
+// entry, off the critical path; the address is read after the CTA barrier
+// that follows (with the tcgen05 fences around it).
+__device__ __forceinline__ void tmem_alloc_cta(const ExpertArgs &a, SharedCtl *ctl) {
+    if ((threadIdx.x >> 5) == NCW + 1) tmem_alloc(smem_u32(&ctl->tmem), tmem_cols_for(a.bpad));
+}
+
 // The roles of an expert CTA.  Tile mode: producer, signal warp, eight
 // mma.sync consumer warps.  Dense mode (UM): producer, NISSUE MMA issuer
 // warps (one thread each; the first holds the CTA's TMEM allocation), eight
@@ -1195,11 +1202,8 @@ __device__ __forceinline__ void run_roles(const ExpertArgs &a, const ExpertMaps 
             consumer<RG>(a, sm.ctl, sm.slots, sm.part);
         }
     } else {
+        // the TMEM columns were allocated at kernel entry (tmem_alloc_cta)
         const int cols = tmem_cols_for(a.bpad);
-        if (warp == NCW + 1) tmem_alloc(smem_u32(&sm.ctl->tmem), cols);
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
         const uint32_t tmem = sm.ctl->tmem;
         if (warp == NCW) {
             producer<RG, true>(a, maps, sm.ctl, sm.slots);
@@ -1254,11 +1258,14 @@ __global__ void __launch_bounds__(cta_threads<UM>(), 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) ctl_init<RG, UM>(ctl, a.wait_ns);
     if (warp == NCW && lane == 0) prefetch_expert_maps(maps);
+    if constexpr (UM) tmem_alloc_cta(a, ctl);
     // everything above overlaps the previous kernel (selection or input
     // preparation); the lists are complete once it has
     asm volatile("griddepcontrol.wait;" ::: "memory");
     if (warp == NCW) table_from_lists(a, ctl, lane);
+    if constexpr (UM) tc_fence_before();
     __syncthreads();
+    if constexpr (UM) tc_fence_after();
     run_roles<RG, UM>(a, maps, sm);
     cta_exit(a, ctl);
 }
@@ -1395,7 +1402,11 @@ __global__ void __launch_bounds__(NTHREADS_UM, 1)
         prefetch_tmap(&rmaps.x);
         prefetch_tmap(&rmaps.wg);
     }
+    // the expert CTAs' TMEM columns (the selection CTA runs no MMAs)
+    if (blockIdx.x != gridDim.x - 1) tmem_alloc_cta(a, ctl);
+    tc_fence_before();
     __syncthreads();
+    tc_fence_after();
 
     // a layer of a stack may start while the previous layer's last CTAs
     // still run: let the next layer's CTAs launch as SMs free up
@@ -1514,7 +1525,8 @@ __global__ void __launch_bounds__(NTHREADS_UM, 1)
         if (ok) table_from_publication(a, ctl, lane);
         else table_from_mask(a, ctl, 0u, lane);
     }
-    __syncthreads();
+    // only the producer warp, which built it, reads the unit table: the
+    // other roles start at once
     run_roles<RG, true>(a, maps, sm);
     cta_exit(a, ctl);
 }
