@@ -8,8 +8,7 @@
 // Retraining", abstract).
 //
 // Work units, dealt round robin to persistent CTAs (one per SM):
-//   GU unit (expert e, token tile, block of d_ff rows: 32 in dense mode,
-//   16 in tile mode):
+//   GU unit (expert e, token tile, 32 rows of d_ff):
 //       g = Wgate[e][rows] x_t, u = Wup[e][rows] x_t over all of d,
 //       h = silu(g) * u -> H scratch (bf16);
 //   D unit (expert e, token tile, 64-row block of d):
@@ -28,23 +27,22 @@
 // Larger batches (tile mode) use tiles of up to 32 (token, expert) pairs:
 // the input preparation copies each pair's x row (bf16) into a pair-indexed
 // buffer in the lists' order, so a tile's x rows are one swizzled box like
-// H's.
+// H's, and the down epilogue weighs each pair by its list weight.
 //
 // Per CTA: one producer warp issues TMA tensor copies (three-dimensional
 // boxes of 64-column chunks, 128-byte swizzle) into a ring of 32 KB weight
 // stages plus operand tiles, each guarded by a full/empty mbarrier pair.
-// Dense mode runs on the 5th-generation tensor cores: one thread issues, per
-// stage, tcgen05 MMAs of 64 weight rows (a gate/up chunk is 32 gate rows and
-// the same 32 up rows) by bpad token columns into a TMEM accumulator, two
-// buffers deep so that a unit's epilogue overlaps the next unit's MMAs; the
-// MMA completion itself frees the stage; eight epilogue warps read the
-// accumulator out (silu * u -> H, or weighted atomics into y) and publish
-// gate/up completions.  Tile mode keeps eight mma.sync consumer warps that
-// split every stage's k-steps (m16n8k16 bf16, 16 weight rows as A, pairs as
-// B) and a signal warp that publishes completions.  Every wait is bounded by
-// a time limit; on expiry the CTA records an error code in the workspace,
-// drains its in-flight copies (and MMAs) and returns.  The last CTA to
-// finish puts the workspace counters of the call back to zero.
+// The math runs on the 5th-generation tensor cores: four issuer warps
+// (one thread each) issue, per stage, tcgen05 MMAs of 64 weight rows (a
+// gate/up chunk is 32 gate rows and the same 32 up rows) by the tile's
+// token columns into partial TMEM accumulators, two buffers deep so that a
+// unit's epilogue overlaps the next unit's MMAs; the MMA completion itself
+// frees the stage.  Eight epilogue warps read the accumulators out (silu *
+// u -> H, or weighted atomics into y) and publish gate/up completions.
+// Every wait is bounded by a time limit; on expiry the CTA records an error
+// code in the workspace, drains its in-flight copies and MMAs and returns.
+// The last CTA to finish puts the workspace counters of the call back to
+// zero.
 #include <cstring>
 #include <mutex>
 
@@ -57,44 +55,31 @@
 namespace moe {
 namespace {
 
-constexpr int NCW = 8;                    // consumer (epilogue) warps
-constexpr int NTHREADS = (NCW + 2) * 32;  // tile mode: + one producer warp + one signal warp
-// Dense mode: the MMAs are issued by NISSUE warps (one per SM sub-partition:
-// a single thread issues at most about one tcgen05.mma per 165 cycles,
-// whatever its shape, measured), each taking every NISSUE-th k-step of a
-// stage into a partial accumulator of its own.
+constexpr int NCW = 8;  // epilogue warps
+// The MMAs are issued by NISSUE warps (one per SM sub-partition: a single
+// thread issues at most about one tcgen05.mma per 165 cycles, whatever its
+// shape, measured), each taking every NISSUE-th k-step of a stage into a
+// partial accumulator of its own.
 constexpr int NISSUE = 4;
-constexpr int NTHREADS_UM = (NCW + 1 + NISSUE) * 32;
-template <bool UM>
-constexpr int cta_threads() { return UM ? NTHREADS_UM : NTHREADS; }
-constexpr int SIG_SLOTS = 4;              // gate/up completions queued for the signal warp
-constexpr int TN = 32;                    // pairs per token tile (batches above 64 tokens)
-constexpr int DENSE_MAX = 64;             // dense mode (every unit takes the whole batch) up to 64 tokens
-// Batches above 64 tokens (tile mode): GU units of 16 rows, stages of 8
-// chunks, mma.sync consumers.
-constexpr int GU_ROWS = 16;
-constexpr int GU_CHUNKS = 8;
-// Dense mode (tensor-core path): GU units of 32 gate rows and the same 32 up
-// rows; a stage holds 4 chunks of 64 columns, each chunk as the gate tile
-// [32][64] followed by the up tile [32][64], so that one chunk is a single
-// 64-row MMA operand (1 KiB row groups throughout).
+constexpr int NTHREADS = (NCW + 1 + NISSUE) * 32;  // + one producer warp
+constexpr int TN = 32;         // pairs per token tile (batches above 64 tokens)
+constexpr int DENSE_MAX = 64;  // dense mode (every unit takes the whole batch) up to 64 tokens
+// GU units of 32 gate rows and the same 32 up rows; a stage holds 4 chunks
+// of 64 columns, each chunk as the gate tile [32][64] followed by the up
+// tile [32][64], so that one chunk is a single 64-row MMA operand (1 KiB row
+// groups throughout).
 constexpr int UM_ROWS = 32;
 constexpr int UM_CHUNKS = 4;
-constexpr int UM_TILE = UM_ROWS * 128;        // one gate (or up) tile of a chunk
-constexpr int UM_CHUNK_BYTES = 2 * UM_TILE;   // gate + up tiles of a chunk
-constexpr int D_ROWS = 64;                // rows of Wdown per D unit
-constexpr int D_CHUNKS = 4;               // 64-column chunks of d_ff per D stage (at most)
+constexpr int UM_TILE = UM_ROWS * 128;       // one gate (or up) tile of a chunk
+constexpr int UM_CHUNK_BYTES = 2 * UM_TILE;  // gate + up tiles of a chunk
+constexpr int D_ROWS = 64;                   // rows of Wdown per D unit
+constexpr int D_CHUNKS = 4;                  // 64-column chunks of d_ff per D stage (at most)
 constexpr int MAX_STAGES = 5;
-constexpr int W_BYTES = 32768;            // weight bytes per stage (both kinds)
-constexpr int UP_OFF = GU_ROWS * 128 * GU_CHUNKS;  // Wup tile after the Wgate tile (tile mode)
+constexpr int W_BYTES = 32768;               // weight bytes per stage (both kinds)
 // Ring shapes: stages of 32 KB of weights plus an operand region for the
-// token rows (x for gate/up, H for down): bpad rows x 4 chunks in dense mode
-// (8, 16 or 32 KB for up to 16, 32 or 64 tokens), 32 pair rows x 8 chunks in
-// tile mode.
-constexpr int PART_LD = TN + 1;                        // padded row of the tile-mode epilogue buffer
-constexpr int PART_FLOATS = (NCW / 2) * 2 * 16 * PART_LD;  // GU partial sums (tile mode)
-// PARTB: bytes of the epilogue buffer (tile mode: the partial sums; dense
-// mode: the accumulator copy, [bpad tokens][64 rows] fp32)
+// token rows of 4 chunks (x for gate/up, H for down): bpad rows in dense
+// mode (8, 16 or 32 KB for up to 16, 32 or 64 tokens), 32 pair rows in tile
+// mode; PARTB: the epilogue's accumulator copy, [rows][64] fp32.
 template <int ST, int OPB, int PARTB>
 struct Ring {
     static constexpr int STAGES = ST;
@@ -112,16 +97,15 @@ constexpr int smem_bytes() {
 }
 using RingB16 = Ring<5, 8192, 16 * 64 * 4>;
 using RingB32 = Ring<4, 16384, 32 * 64 * 4>;
-using RingB64 = Ring<3, 32768, PART_FLOATS * 4>;
-static_assert(2 * GU_ROWS * 128 * GU_CHUNKS <= W_BYTES, "gate/up tiles do not fit");
-static_assert(UM_CHUNKS * UM_CHUNK_BYTES == W_BYTES, "dense gate/up chunks must fill the weight region");
+using RingB64 = Ring<3, 32768, 64 * 64 * 4>;
+static_assert(UM_CHUNKS * UM_CHUNK_BYTES == W_BYTES, "gate/up chunks must fill the weight region");
 static_assert(2 * UM_ROWS == UMMA_M && D_ROWS == UMMA_M && D_ROWS * 128 == UM_CHUNK_BYTES,
               "a gate/up chunk and a down chunk are one 64-row MMA operand each");
 static_assert(16 * 128 * UM_CHUNKS <= RingB16::OP_BYTES && 32 * 128 * UM_CHUNKS <= RingB32::OP_BYTES &&
                   DENSE_MAX * 128 * UM_CHUNKS <= RingB64::OP_BYTES && DENSE_MAX * 128 * D_CHUNKS <= RingB64::OP_BYTES,
-              "dense token rows do not fit");
+              "token rows do not fit");
+static_assert(TN == 32, "tile mode uses the 32-row ring");
 static_assert(D_ROWS * 128 * D_CHUNKS <= W_BYTES, "down tile does not fit");
-static_assert(TN * GU_CHUNKS * 128 <= RingB64::OP_BYTES, "x rows (32 pairs) do not fit");
 static_assert(DENSE_MAX * 64 * 4 <= RingB64::PART_BYTES, "accumulator copy does not fit");
 static_assert(RingB16::SLOT_BYTES % 1024 == 0 && RingB32::SLOT_BYTES % 1024 == 0 && RingB64::SLOT_BYTES % 1024 == 0,
               "slots must keep 1 KiB alignment for 128B swizzle");
@@ -165,9 +149,6 @@ struct SharedCtl {
     unsigned long long wait_ns;  // limit of every bounded wait of this call
     unsigned long long full[MAX_STAGES];
     unsigned long long empty[MAX_STAGES];
-    unsigned long long sig_full[SIG_SLOTS];
-    unsigned long long sig_empty[SIG_SLOTS];
-    int sig_iact[SIG_SLOTS];
     StageHdr hdr[MAX_STAGES];
     volatile int abort_flag;
     volatile int consumed;
@@ -286,32 +267,12 @@ __device__ __forceinline__ int d_chunks_of(int F) { return min(D_CHUNKS, F / 64)
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<unsigned long long>(map)) : "memory");
 }
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
-                                        uint32_t &r3) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-                 : "r"(addr));
-}
-__device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                         uint32_t a3, uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
-        "{%8, %9}, {%0, %1, %2, %3};"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
 __device__ __forceinline__ int ld_acquire(const int *p) {
     int v;
     asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
 __device__ __forceinline__ void consumer_bar() { asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory"); }
-static_assert(NCW == 8, "the stage split below assumes eight consumer warps");
-
-// address of (row r, 16-byte chunk c) in a 128B-swizzled box with 128-byte rows
-__device__ __forceinline__ uint32_t swz(uint32_t base, int r, int c) {
-    return base + r * 128 + ((c ^ (r & 7)) << 4);
-}
 
 __device__ void record_error(Counters *ctr, SharedCtl *ctl, int code) {
     atomicCAS(&ctr->error, 0, code);
@@ -367,6 +328,9 @@ __device__ __forceinline__ UnitCounts unit_counts(const ExpertArgs &a, int total
     c.total = c.n_gu + c.d_main + split * a.ns_d;
     return c;
 }
+// DENSE: dense mode known at compile time (the fused layer kernel), which
+// leaves the tile-mode code out of the persistent kernel.
+template <bool DENSE>
 __device__ __forceinline__ void decode_rec(int u, int n_units, const ExpertArgs &a, const SharedCtl *ctl,
                                            UnitRec &ui) {
     if (u >= n_units) {
@@ -382,7 +346,7 @@ __device__ __forceinline__ void decode_rec(int u, int n_units, const ExpertArgs 
         ui.k0 = j - q * a.ns_d;
         u = uc.n_gu + uc.d_main + q;
     }
-    if (a.dense) {
+    if (DENSE || a.dense) {
         // one tile per active expert: slot i's units are consecutive
         const bool gu = u < uc.n_gu;
         const int v = gu ? u : u - uc.n_gu;
@@ -398,8 +362,7 @@ __device__ __forceinline__ void decode_rec(int u, int n_units, const ExpertArgs 
         ui.need = a.gu_per_tile;
         return;
     }
-    const int gu_per_tile = a.F / GU_ROWS;
-    const int d_per_tile = a.d / D_ROWS;
+    const int gu_per_tile = a.gu_per_tile;
     const int n_gu = ctl->total_tiles * gu_per_tile;
     int per, v;
     if (u < n_gu) {
@@ -409,7 +372,7 @@ __device__ __forceinline__ void decode_rec(int u, int n_units, const ExpertArgs 
         ui.ns = a.ns_gu;
     } else {
         ui.type = UNIT_D;
-        per = d_per_tile;
+        per = a.d_per_tile;
         v = u - n_gu;
         ui.ns = v >= uc.d_main ? 1 : a.ns_d;
     }
@@ -427,7 +390,7 @@ __device__ __forceinline__ void decode_rec(int u, int n_units, const ExpertArgs 
     const int local = v - ctl->tile_start[i] * per;
     const int blk = local / nt_i;
     const int tt = local - blk * nt_i;
-    ui.row0 = blk * (ui.type == UNIT_GU ? GU_ROWS : D_ROWS);
+    ui.row0 = blk * (ui.type == UNIT_GU ? a.gu_rows : D_ROWS);
     ui.i_act = i;
     ui.e = ctl->act_e[i];
     ui.p0 = ctl->off[i] + tt * TN;
@@ -439,11 +402,12 @@ __device__ __forceinline__ void decode_rec(int u, int n_units, const ExpertArgs 
 // j * unit_ctas).  The producer's lanes decode UNIT_WINDOW units at a time
 // into shared memory; the prefetches of the unit's first stage are issued
 // here and first used when that stage is issued.
+template <bool DENSE>
 __device__ bool fetch_unit(int j, int &win_base, int n_units, const ExpertArgs &a, SharedCtl *ctl, int lane,
                            UnitInfo &ui) {
     if (j >= win_base + UNIT_WINDOW) {
         __syncwarp();
-        decode_rec(blockIdx.x + (j + lane) * a.unit_ctas, n_units, a, ctl, ctl->urec[lane]);
+        decode_rec<DENSE>(blockIdx.x + (j + lane) * a.unit_ctas, n_units, a, ctl, ctl->urec[lane]);
         __syncwarp();
         win_base = j;
     }
@@ -454,9 +418,9 @@ __device__ bool fetch_unit(int j, int &win_base, int n_units, const ExpertArgs &
     return true;
 }
 
-// UM: dense tensor-core layout (a gate/up stage is UM_CHUNKS chunk copies
-// of each matrix, interleaved per chunk); otherwise the tile-mode layout.
-template <class RG, bool UM>
+// A gate/up stage is UM_CHUNKS chunk copies of each matrix, interleaved
+// per chunk (the tensor-core operand layout).
+template <class RG, bool DENSE>
 __device__ void producer(const ExpertArgs &a, const ExpertMaps &m, SharedCtl *ctl, unsigned char *slots) {
     constexpr int STAGES = RG::STAGES;
     const int lane = threadIdx.x & 31;
@@ -473,7 +437,7 @@ __device__ void producer(const ExpertArgs &a, const ExpertMaps &m, SharedCtl *ct
     // precedes every down unit in each CTA's sequence)
     int j_next = 0, win_base = -UNIT_WINDOW;
     UnitInfo cur;
-    bool have = fetch_unit(j_next++, win_base, n_units, a, ctl, lane, cur);
+    bool have = fetch_unit<DENSE>(j_next++, win_base, n_units, a, ctl, lane, cur);
     int g = 0;  // stages issued
     bool ok = true;
     while (have && ok) {
@@ -493,7 +457,7 @@ __device__ void producer(const ExpertArgs &a, const ExpertMaps &m, SharedCtl *ct
             const int gcv = min(gc, (a.d >> 6) - (cur.k0 + s) * gc);
             // x tile: all B token rows (dense mode) or the tile's TN pair rows
             const unsigned xbytes = static_cast<unsigned>(gc) * (a.dense ? a.bpad : TN) * 128u;
-            const unsigned wbytes = UM ? 2u * gcv * UM_TILE : 2u * gc * (a.gu_rows * 128);
+            const unsigned wbytes = 2u * gcv * UM_TILE;
             const unsigned bytes = cur.type == UNIT_GU ? wbytes + xbytes : dc * (D_ROWS * 128u) + dc * (a.hrows * 128u);
             if (lane == 0) {
                 StageHdr &h = ctl->hdr[slot];
@@ -511,22 +475,16 @@ __device__ void producer(const ExpertArgs &a, const ExpertMaps &m, SharedCtl *ct
             __syncwarp();
             if (cur.type == UNIT_GU) {
                 const int grow = cur.e * a.F + cur.row0;
-                if constexpr (UM) {
-                    // chunk c: gate tile at 8 KB c, up tile 4 KB after it
-                    if (lane < gcv)
-                        tma_load_3d_stream(wdst + lane * UM_CHUNK_BYTES, &m.gate, 0, grow, s * gc + lane,
-                                           &ctl->full[slot], policy);
-                    else if (lane >= 8 && lane < 8 + gcv)
-                        tma_load_3d_stream(wdst + (lane - 8) * UM_CHUNK_BYTES + UM_TILE, &m.up, 0, grow,
-                                           s * gc + lane - 8, &ctl->full[slot], policy);
-                    // x rows of all B tokens for this column range, one swizzled box
-                    if (lane == 16) tma_load_3d(odst, &m.x, 0, 0, s * gc, &ctl->full[slot]);
-                } else {
-                    if (lane == 0) tma_load_3d_stream(wdst, &m.gate, 0, grow, s * gc, &ctl->full[slot], policy);
-                    if (lane == 1) tma_load_3d_stream(wdst + UP_OFF, &m.up, 0, grow, s * gc, &ctl->full[slot], policy);
-                    // the tile's pair rows of the dispatched x in one swizzled box
-                    if (lane == 2) tma_load_3d(odst, &m.x, 0, cur.p0, s * gc, &ctl->full[slot]);
-                }
+                // chunk c: gate tile at 8 KB c, up tile 4 KB after it
+                if (lane < gcv)
+                    tma_load_3d_stream(wdst + lane * UM_CHUNK_BYTES, &m.gate, 0, grow, s * gc + lane,
+                                       &ctl->full[slot], policy);
+                else if (lane >= 8 && lane < 8 + gcv)
+                    tma_load_3d_stream(wdst + (lane - 8) * UM_CHUNK_BYTES + UM_TILE, &m.up, 0, grow,
+                                       s * gc + lane - 8, &ctl->full[slot], policy);
+                // x rows for this column range, one swizzled box: all B
+                // tokens (dense mode) or the tile's pairs of the dispatched x
+                if (lane == 16) tma_load_3d(odst, &m.x, 0, (DENSE || a.dense) ? 0 : cur.p0, s * gc, &ctl->full[slot]);
             } else {
                 if (lane == 0)
                     tma_load_3d_stream(wdst, &m.down, 0, cur.e * a.d + cur.row0, (cur.k0 + s) * dc, &ctl->full[slot],
@@ -558,7 +516,7 @@ __device__ void producer(const ExpertArgs &a, const ExpertMaps &m, SharedCtl *ct
             }
             ++g;
             if (!ok) break;
-            if (s == 0) have_nxt = fetch_unit(j_next++, win_base, n_units, a, ctl, lane, nxt);
+            if (s == 0) have_nxt = fetch_unit<DENSE>(j_next++, win_base, n_units, a, ctl, lane, nxt);
         }
         cur = nxt;
         have = have_nxt;
@@ -584,231 +542,6 @@ __device__ void producer(const ExpertArgs &a, const ExpertMaps &m, SharedCtl *ct
     }
 }
 
-// ------------------------------------------------------------ consumers --
-// B operand rows: a 128B-swizzled tile per 64 columns, x_tile bytes apart
-// ([rows][64] per chunk): token t in dense mode, the tile's pair n otherwise.
-template <int NT>
-__device__ __forceinline__ void gu_stage(uint32_t wbase, uint32_t xbase, int x_tile, int kvalid, int warp, int lane,
-                                         float (&acc_g)[4][4], float (&acc_u)[4][4]) {
-    const int nks = kvalid / 16;
-#pragma unroll
-    for (int q = 0; q < (GU_CHUNKS * 4) / NCW; ++q) {
-        const int ks = warp + NCW * q;
-        if (ks >= nks) break;
-        const int box = ks >> 2;
-        const int chunk = ((ks & 3) << 1) + (lane >> 4);
-        const int r = lane & 15;
-        uint32_t g0, g1, g2, g3, u0, u1, u2, u3;
-        ldsm_x4(swz(wbase + box * (GU_ROWS * 128), r, chunk), g0, g1, g2, g3);
-        ldsm_x4(swz(wbase + UP_OFF + box * (GU_ROWS * 128), r, chunk), u0, u1, u2, u3);
-        const int xchunk = ((ks & 3) << 1) + ((lane >> 3) & 1);
-#pragma unroll
-        for (int np = 0; np < (NT + 1) / 2; ++np) {
-            const int n = np * 16 + (lane & 7) + ((lane >> 4) << 3);
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4(swz(xbase + box * x_tile, n, xchunk), b0, b1, b2, b3);
-            mma_bf16(acc_g[2 * np], g0, g1, g2, g3, b0, b1);
-            mma_bf16(acc_u[2 * np], u0, u1, u2, u3, b0, b1);
-            if (2 * np + 1 < NT) {
-                mma_bf16(acc_g[2 * np + 1], g0, g1, g2, g3, b2, b3);
-                mma_bf16(acc_u[2 * np + 1], u0, u1, u2, u3, b2, b3);
-            }
-        }
-    }
-}
-
-template <int NT>
-__device__ __forceinline__ void d_stage(uint32_t wbase, uint32_t hbase, int hrows, int kvalid, int warp, int lane,
-                                        float (&acc)[4][4]) {
-    const int nks = kvalid / 16;
-#pragma unroll
-    for (int q = 0; q < (D_CHUNKS * 4) / 2; ++q) {
-        const int ks = (warp >> 2) * ((D_CHUNKS * 4) / 2) + q;
-        if (ks >= nks) break;
-        const int box = ks >> 2;
-        const int r = (warp & 3) * 16 + (lane & 15);
-        const int chunk = ((ks & 3) << 1) + (lane >> 4);
-        uint32_t a0, a1, a2, a3;
-        ldsm_x4(swz(wbase + box * (D_ROWS * 128), r, chunk), a0, a1, a2, a3);
-        const int hchunk = ((ks & 3) << 1) + ((lane >> 3) & 1);
-#pragma unroll
-        for (int np = 0; np < (NT + 1) / 2; ++np) {
-            const int n = np * 16 + (lane & 7) + ((lane >> 4) << 3);
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4(swz(hbase + box * (hrows * 128), n, hchunk), b0, b1, b2, b3);
-            mma_bf16(acc[2 * np], a0, a1, a2, a3, b0, b1);
-            if (2 * np + 1 < NT) mma_bf16(acc[2 * np + 1], a0, a1, a2, a3, b2, b3);
-        }
-    }
-}
-
-template <int NT>
-__device__ __forceinline__ void stage_dispatch(const StageHdr &h, uint32_t wbase, uint32_t obase, const ExpertArgs &a,
-                                               int warp, int lane, float (&acc_g)[4][4], float (&acc_u)[4][4]) {
-    if (h.type == UNIT_GU) {
-        const int gk = 64 * a.gc;
-        gu_stage<NT>(wbase, obase, TN * 128, min(gk, a.d - h.k * gk), warp, lane, acc_g, acc_u);
-    } else {
-        const int dk = 64 * d_chunks_of(a.F);
-        d_stage<NT>(wbase, obase, a.hrows, min(dk, a.F - h.k * dk), warp, lane, acc_g);
-    }
-}
-
-// Queue one gate/up completion (i >= 0) or the end marker (i < 0) for the
-// signal warp.  False if the CTA aborted.
-__device__ bool post_signal(SharedCtl *ctl, Counters *ctr, int q, int i) {
-    const int slot = q % SIG_SLOTS;
-    if (q >= SIG_SLOTS && !wait_phase(&ctl->sig_empty[slot], ((q / SIG_SLOTS) - 1) & 1, ctl, ctr, DEV_TIMEOUT_EMPTY))
-        return false;
-    ctl->sig_iact[slot] = i;
-    mbar_arrive(&ctl->sig_full[slot]);
-    return true;
-}
-
-// Tile-mode consumers (batches above 64 tokens): the eight warps split
-// every stage's k-steps (mma.sync), then reduce and apply the epilogue at
-// the unit's last stage.
-template <class RG>
-__device__ void consumer(const ExpertArgs &a, SharedCtl *ctl, unsigned char *slots, float *part) {
-    constexpr int STAGES = RG::STAGES;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int ct = threadIdx.x;  // 0 .. NCW*32-1
-    float acc_g[4][4], acc_u[4][4];
-    int tk[4][2];
-    float wk[4][2];
-    int nsig = 0;  // completions posted (thread 0)
-    const int row = lane >> 2, col = (lane & 3) * 2;
-    for (int g = 0;; ++g) {
-        const int slot = g % STAGES;
-        if (!wait_phase(&ctl->full[slot], (g / STAGES) & 1, ctl, a.ctr, DEV_TIMEOUT_FULL)) return;
-        const StageHdr h = ctl->hdr[slot];
-        if (h.type == UNIT_END) {
-            if (ct == 0) post_signal(ctl, a.ctr, nsig, -1);
-            return;
-        }
-        if (h.s == 0) {
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-#pragma unroll
-                for (int c = 0; c < 4; ++c) acc_g[j][c] = acc_u[j][c] = 0.0f;
-            if (h.type == UNIT_D) {
-                // tokens and gate weights this thread combines; used at the
-                // unit's last stage, loaded now so the latency is hidden
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-#pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        const int n = j * 8 + col + c;
-                        const int t = n < h.n ? __ldg(a.tok + h.p0 + n) : 0;
-                        // a token outside the batch is skipped (and reported)
-                        const bool v = n < h.n && t >= 0 && t < a.B;
-                        if (n < h.n && !v) atomicCAS(&a.ctr->error, 0, DEV_BAD_LISTS);
-                        tk[j][c] = v ? t : 0;
-                        wk[j][c] = v ? __ldg(a.w + h.p0 + n) : 0.0f;
-                    }
-            }
-        }
-        const uint32_t wbase = smem_u32(slots + slot * RG::SLOT_BYTES);
-        const uint32_t obase = wbase + W_BYTES;
-        const int nt = (h.n + 7) >> 3;
-        switch (nt) {
-            case 1: stage_dispatch<1>(h, wbase, obase, a, warp, lane, acc_g, acc_u); break;
-            case 2: stage_dispatch<2>(h, wbase, obase, a, warp, lane, acc_g, acc_u); break;
-            case 3: stage_dispatch<3>(h, wbase, obase, a, warp, lane, acc_g, acc_u); break;
-            default: stage_dispatch<4>(h, wbase, obase, a, warp, lane, acc_g, acc_u); break;
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&ctl->empty[slot]);
-        if (ct == 0) ctl->consumed = g + 1;
-        if (h.s != h.ns - 1) continue;
-
-        // ---- unit epilogue
-        if (h.type == UNIT_D) {
-            // each warp holds a k-half of a 16-row block: both halves add into y
-            const int i_base = h.row0 + (warp & 3) * 16 + row;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                if (j >= nt) break;
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const int n = j * 8 + col + (c & 1);
-                    if (n < h.n && wk[j][c & 1] != 0.0f) {
-                        const int i = i_base + ((c >> 1) << 3);
-                        atomicAdd(a.y + static_cast<size_t>(tk[j][c & 1]) * a.d + i, wk[j][c & 1] * acc_g[j][c]);
-                    }
-                }
-            }
-        } else {
-            // reduce the eight warps' k-slices in a fixed order (warp w + 4
-            // into warp w, then the four sums) and apply silu(g) * u
-            float *pg = part + ((warp & 3) * 2 + 0) * 16 * PART_LD;
-            float *pu = part + ((warp & 3) * 2 + 1) * 16 * PART_LD;
-            if (warp >= 4) {
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    if (j >= nt) break;
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const int r = row + ((c >> 1) << 3);
-                        const int n = j * 8 + col + (c & 1);
-                        pg[r * PART_LD + n] = acc_g[j][c];
-                        pu[r * PART_LD + n] = acc_u[j][c];
-                    }
-                }
-            }
-            consumer_bar();
-            if (warp < 4) {
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    if (j >= nt) break;
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const int r = row + ((c >> 1) << 3);
-                        const int n = j * 8 + col + (c & 1);
-                        pg[r * PART_LD + n] = acc_g[j][c] + pg[r * PART_LD + n];
-                        pu[r * PART_LD + n] = acc_u[j][c] + pu[r * PART_LD + n];
-                    }
-                }
-            }
-            consumer_bar();
-            for (int idx = ct; idx < 16 * h.n; idx += NCW * 32) {
-                // column n: the tile's pair n; H row p0 + n
-                const int r = idx & 15, n = idx >> 4;
-                float gs = 0.0f, us = 0.0f;
-#pragma unroll
-                for (int wv = 0; wv < NCW / 2; ++wv) {
-                    gs += part[(wv * 2 + 0) * 16 * PART_LD + r * PART_LD + n];
-                    us += part[(wv * 2 + 1) * 16 * PART_LD + r * PART_LD + n];
-                }
-                const float hv = gs / (1.0f + __expf(-gs)) * us;
-                a.h[static_cast<size_t>(h.p0 + n) * a.F + h.row0 + r] =
-                    __bfloat16_as_ushort(__float2bfloat16_rn(hv));
-            }
-            // H is read by other CTAs through TMA (the async proxy)
-            asm volatile("fence.proxy.async.global;" ::: "memory");
-            consumer_bar();
-            // the signal warp publishes the completion (fence + counter), so
-            // the consumers do not wait for it
-            if (ct == 0 && !post_signal(ctl, a.ctr, nsig++, h.i_act)) return;
-        }
-    }
-}
-
-// Signal warp: turns queued gate/up completions into gu_done increments
-// visible to the whole GPU.
-__device__ void signaller(const ExpertArgs &a, SharedCtl *ctl) {
-    if ((threadIdx.x & 31) != 0) return;
-    for (int q = 0;; ++q) {
-        const int slot = q % SIG_SLOTS;
-        if (!wait_phase(&ctl->sig_full[slot], (q / SIG_SLOTS) & 1, ctl, a.ctr, DEV_TIMEOUT_FULL)) return;
-        const int i = ctl->sig_iact[slot];
-        mbar_arrive(&ctl->sig_empty[slot]);
-        if (i < 0) return;
-        __threadfence();
-        atomicAdd(&a.ctr->gu_done[i], 1);
-    }
-}
-
 // ------------------------------------------------ tensor-core path (dense) --
 // TMEM columns of the CTA's allocation: two accumulator buffers, each
 // NISSUE partial accumulators of bpad columns (a power of two, at least 32).
@@ -829,9 +562,9 @@ __device__ __forceinline__ int tmem_cols_for(int bpad) {
 // chunk.  Issuer 0 also hands the unit's header to the epilogue.
 __device__ void umma_issuer(const ExpertArgs &a, SharedCtl *ctl, unsigned char *slots, int stages, int slot_bytes,
                             uint32_t tmem, int p) {
-    const uint32_t idesc = umma_idesc_bf16(a.bpad);
-    const uint32_t b_chunk = static_cast<uint32_t>(a.bpad) * 128u;
-    const uint32_t buf_stride = static_cast<uint32_t>(tmem_cols_for(a.bpad) / 2);
+    const uint32_t idesc = umma_idesc_bf16(a.hrows);
+    const uint32_t b_chunk = static_cast<uint32_t>(a.hrows) * 128u;
+    const uint32_t buf_stride = static_cast<uint32_t>(tmem_cols_for(a.hrows) / 2);
     const int gk = 64 * a.gc, dk = 64 * d_chunks_of(a.F);
     int unit = 0;  // units started
     for (int g = 0;; ++g) {
@@ -863,7 +596,7 @@ __device__ void umma_issuer(const ExpertArgs &a, SharedCtl *ctl, unsigned char *
         const uint32_t wbase = smem_u32(slots + slot * slot_bytes);
         const uint32_t obase = wbase + W_BYTES;
         const int nks = (h.type == UNIT_GU ? min(gk, a.d - h.k * gk) : min(dk, a.F - h.k * dk)) >> 4;
-        const uint32_t dcol = tmem + static_cast<uint32_t>(b) * buf_stride + static_cast<uint32_t>(p * a.bpad);
+        const uint32_t dcol = tmem + static_cast<uint32_t>(b) * buf_stride + static_cast<uint32_t>(p * a.hrows);
         // nks >= 4 = NISSUE (d and d_ff are multiples of 64): every issuer
         // starts its partial sum at stage 0
         for (int ks = p; ks < nks; ks += NISSUE) {
@@ -895,12 +628,13 @@ __device__ void umma_issuer(const ExpertArgs &a, SharedCtl *ctl, unsigned char *
 //     (bf16, two rows per thread), and thread 0 publishes the completion;
 //   down unit:    y[t][row0 + r] += wd[slot][t] acc[t][r], four rows per
 //     vector atomic.
+template <bool DENSE>
 __device__ void umma_epilogue(const ExpertArgs &a, SharedCtl *ctl, float *xch, uint32_t tmem) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int ct = threadIdx.x;  // 0 .. NCW*32-1
     const int q = warp & 3, half = warp >> 2;
-    const int ncg = a.bpad >> 3;
-    const uint32_t buf_stride = static_cast<uint32_t>(tmem_cols_for(a.bpad) / 2);
+    const int ncg = a.hrows >> 3;
+    const uint32_t buf_stride = static_cast<uint32_t>(tmem_cols_for(a.hrows) / 2);
     bool lists_ready = !a.early;
     // Thread 0 takes every wait and passes its outcome through shared
     // memory, so that all epilogue threads leave together (none is left at a
@@ -925,7 +659,7 @@ __device__ void umma_epilogue(const ExpertArgs &a, SharedCtl *ctl, float *xch, u
 #pragma unroll
                 for (int pi = 1; pi < NISSUE; ++pi) {
                     float w8[8];
-                    tmem_ld8(tb + static_cast<uint32_t>(pi * a.bpad + cg * 8), w8);
+                    tmem_ld8(tb + static_cast<uint32_t>(pi * a.hrows + cg * 8), w8);
 #pragma unroll
                     for (int c = 0; c < 8; ++c) v[j][c] += w8[c];
                 }
@@ -968,7 +702,8 @@ __device__ void umma_epilogue(const ExpertArgs &a, SharedCtl *ctl, float *xch, u
         }
         consumer_bar();
         if (ah.type == UNIT_GU) {
-            for (int idx = ct; idx < 16 * a.B; idx += NCW * 32) {
+            // column t: token t (dense mode) or the tile's pair t; H row p0 + t
+            for (int idx = ct; idx < 16 * ah.n; idx += NCW * 32) {
                 const int t = idx >> 4, r = (idx & 15) * 2;
                 const float2 gs = *reinterpret_cast<const float2 *>(xch + t * 64 + r);
                 const float2 us = *reinterpret_cast<const float2 *>(xch + t * 64 + UM_ROWS + r);
@@ -987,11 +722,23 @@ __device__ void umma_epilogue(const ExpertArgs &a, SharedCtl *ctl, float *xch, u
             }
         } else {
             if (!ctl->epi_lists) return;
-            for (int idx = ct; idx < 16 * a.B; idx += NCW * 32) {
-                const int t = idx >> 4, r = (idx & 15) * 4;
-                const float w = __ldcg(a.wd + static_cast<size_t>(ah.i_act) * a.B + t);
+            for (int idx = ct; idx < 16 * ah.n; idx += NCW * 32) {
+                const int n = idx >> 4, r = (idx & 15) * 4;
+                // dense mode: token n, weight wd[slot][n]; tile mode: the
+                // pair's token and weight from the lists (a token outside the
+                // batch is skipped and reported)
+                int t = n;
+                float w;
+                if (DENSE || a.dense) {
+                    w = __ldcg(a.wd + static_cast<size_t>(ah.i_act) * a.B + n);
+                } else {
+                    t = __ldg(a.tok + ah.p0 + n);
+                    const bool v = t >= 0 && t < a.B;
+                    if (!v && r == 0) atomicCAS(&a.ctr->error, 0, DEV_BAD_LISTS);
+                    w = v ? __ldg(a.w + ah.p0 + n) : 0.0f;
+                }
                 if (w != 0.0f) {
-                    const float4 s4 = *reinterpret_cast<const float4 *>(xch + t * 64 + r);
+                    const float4 s4 = *reinterpret_cast<const float4 *>(xch + n * 64 + r);
                     atomicAdd(reinterpret_cast<float4 *>(a.y + static_cast<size_t>(t) * a.d + ah.row0 + r),
                               make_float4(w * s4.x, w * s4.y, w * s4.z, w * s4.w));
                 }
@@ -1039,13 +786,13 @@ struct CtaSmem {
     }
 };
 
-// Barriers and flags of a CTA (thread 0).
-// UM: the tensor-core path (a stage is released by the issuers' MMA commits).
-template <class RG, bool UM>
+// Barriers and flags of a CTA (thread 0).  A stage is released by the
+// issuers' MMA commits.
+template <class RG>
 __device__ void ctl_init(SharedCtl *ctl, unsigned long long wait_ns) {
     for (int s = 0; s < RG::STAGES; ++s) {
         mbar_init(&ctl->full[s], 1);
-        mbar_init(&ctl->empty[s], UM ? NISSUE : NCW);  // one MMA commit per issuer
+        mbar_init(&ctl->empty[s], NISSUE);  // one MMA commit per issuer
     }
     for (int b = 0; b < 2; ++b) {
         mbar_init(&ctl->acc_full[b], NISSUE + 1);  // the first issuer's arrive + every issuer's commit
@@ -1053,10 +800,6 @@ __device__ void ctl_init(SharedCtl *ctl, unsigned long long wait_ns) {
     }
     mbar_init(&ctl->mma_done, NISSUE);
     ctl->epi_lists = 1;
-    for (int s = 0; s < SIG_SLOTS; ++s) {
-        mbar_init(&ctl->sig_full[s], 1);
-        mbar_init(&ctl->sig_empty[s], 1);
-    }
     ctl->wait_ns = wait_ns;
     ctl->abort_flag = 0;
     ctl->consumed = 0;
@@ -1183,43 +926,32 @@ __device__ void table_from_lists(const ExpertArgs &a, SharedCtl *ctl, int lane) 
 // entry, off the critical path; the address is read after the CTA barrier
 // that follows (with the tcgen05 fences around it).
 __device__ __forceinline__ void tmem_alloc_cta(const ExpertArgs &a, SharedCtl *ctl) {
-    if ((threadIdx.x >> 5) == NCW + 1) tmem_alloc(smem_u32(&ctl->tmem), tmem_cols_for(a.bpad));
+    if ((threadIdx.x >> 5) == NCW + 1) tmem_alloc(smem_u32(&ctl->tmem), tmem_cols_for(a.hrows));
 }
 
-// The roles of an expert CTA.  Tile mode: producer, signal warp, eight
-// mma.sync consumer warps.  Dense mode (UM): producer, NISSUE MMA issuer
-// warps (one thread each; the first holds the CTA's TMEM allocation), eight
+// The roles of an expert CTA: the producer, NISSUE MMA issuer warps (one
+// thread each; the first holds the CTA's TMEM allocation) and eight
 // epilogue warps.
-template <class RG, bool UM>
+template <class RG, bool DENSE>
 __device__ __forceinline__ void run_roles(const ExpertArgs &a, const ExpertMaps &maps, const CtaSmem<RG> &sm) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if constexpr (!UM) {
-        if (warp == NCW) {
-            producer<RG, false>(a, maps, sm.ctl, sm.slots);
-        } else if (warp == NCW + 1) {
-            signaller(a, sm.ctl);
-        } else {
-            consumer<RG>(a, sm.ctl, sm.slots, sm.part);
-        }
+    // the TMEM columns were allocated at kernel entry (tmem_alloc_cta)
+    const int cols = tmem_cols_for(a.hrows);
+    const uint32_t tmem = sm.ctl->tmem;
+    if (warp == NCW) {
+        producer<RG, DENSE>(a, maps, sm.ctl, sm.slots);
+    } else if (warp > NCW) {
+        if (lane == 0) umma_issuer(a, sm.ctl, sm.slots, RG::STAGES, RG::SLOT_BYTES, tmem, warp - NCW - 1);
     } else {
-        // the TMEM columns were allocated at kernel entry (tmem_alloc_cta)
-        const int cols = tmem_cols_for(a.bpad);
-        const uint32_t tmem = sm.ctl->tmem;
-        if (warp == NCW) {
-            producer<RG, true>(a, maps, sm.ctl, sm.slots);
-        } else if (warp > NCW) {
-            if (lane == 0) umma_issuer(a, sm.ctl, sm.slots, RG::STAGES, RG::SLOT_BYTES, tmem, warp - NCW - 1);
-        } else {
-            umma_epilogue(a, sm.ctl, sm.part, tmem);
-        }
-        // the issuers have waited for their MMAs, the epilogue for its loads
-        tc_fence_before();
-        __syncthreads();
-        if (warp == NCW + 1) {
-            __syncwarp();
-            tc_fence_after();
-            tmem_dealloc(tmem, cols);
-        }
+        umma_epilogue<DENSE>(a, sm.ctl, sm.part, tmem);
+    }
+    // the issuers have waited for their MMAs, the epilogue for its loads
+    tc_fence_before();
+    __syncthreads();
+    if (warp == NCW + 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, cols);
     }
 }
 
@@ -1248,25 +980,24 @@ __device__ void cta_exit(const ExpertArgs &a, SharedCtl *ctl) {
     }
 }
 
-// UM: dense mode on the tensor cores (B <= 64); otherwise tile mode.
-template <class RG, bool UM>
-__global__ void __launch_bounds__(cta_threads<UM>(), 1)
+template <class RG>
+__global__ void __launch_bounds__(NTHREADS, 1)
     expert_ffn_kernel(const __grid_constant__ ExpertMaps maps, const ExpertArgs a) {
     extern __shared__ unsigned char smem_raw[];
     const CtaSmem<RG> sm(smem_raw);
     SharedCtl *ctl = sm.ctl;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (threadIdx.x == 0) ctl_init<RG, UM>(ctl, a.wait_ns);
+    if (threadIdx.x == 0) ctl_init<RG>(ctl, a.wait_ns);
     if (warp == NCW && lane == 0) prefetch_expert_maps(maps);
-    if constexpr (UM) tmem_alloc_cta(a, ctl);
+    tmem_alloc_cta(a, ctl);
     // everything above overlaps the previous kernel (selection or input
     // preparation); the lists are complete once it has
     asm volatile("griddepcontrol.wait;" ::: "memory");
     if (warp == NCW) table_from_lists(a, ctl, lane);
-    if constexpr (UM) tc_fence_before();
+    tc_fence_before();
     __syncthreads();
-    if constexpr (UM) tc_fence_after();
-    run_roles<RG, UM>(a, maps, sm);
+    tc_fence_after();
+    run_roles<RG, false>(a, maps, sm);
     cta_exit(a, ctl);
 }
 
@@ -1342,7 +1073,7 @@ __device__ __forceinline__ void rank_union(const ExpertArgs &a, const LayerArgs 
 }
 
 template <class RG, int NI>
-__global__ void __launch_bounds__(NTHREADS_UM, 1)
+__global__ void __launch_bounds__(NTHREADS, 1)
     layer_kernel(const __grid_constant__ ExpertMaps maps, const __grid_constant__ RouterMaps rmaps,
                  const ExpertArgs a, const LayerArgs L) {
     extern __shared__ unsigned char smem_raw[];
@@ -1393,7 +1124,7 @@ __global__ void __launch_bounds__(NTHREADS_UM, 1)
                 issue_rows(item, true, false);
             }
         }
-        ctl_init<RG, true>(ctl, a.wait_ns);
+        ctl_init<RG>(ctl, a.wait_ns);
         s_ok = 1;
     }
     if (threadIdx.x < E_MAX / 32) s_set[threadIdx.x] = 0u;
@@ -1653,13 +1384,13 @@ int g_num_sms[MAX_DEVICES] = {0};
 
 int expert_ffn_h_rows(int B) { return B <= DENSE_MAX ? (B + 7) / 8 * 8 : TN; }
 int expert_ffn_dense_batch(int B) { return B <= DENSE_MAX ? 1 : 0; }
-int expert_ffn_gu_rows(int B) { return B <= DENSE_MAX ? UM_ROWS : GU_ROWS; }
+int expert_ffn_gu_rows(int) { return UM_ROWS; }
 int expert_ffn_d_rows() { return D_ROWS; }
 int expert_ffn_gu_chunks(int d, int B) {
-    const int cap = B <= DENSE_MAX ? UM_CHUNKS : GU_CHUNKS;
-    return d / 64 < cap ? d / 64 : cap;
+    (void)B;
+    return d / 64 < UM_CHUNKS ? d / 64 : UM_CHUNKS;
 }
-int expert_ffn_gu_box_chunks(int d, int B) { return B <= DENSE_MAX ? 1 : expert_ffn_gu_chunks(d, B); }
+int expert_ffn_gu_box_chunks(int, int) { return 1; }
 int expert_ffn_d_chunks(int F) { return F / 64 < D_CHUNKS ? F / 64 : D_CHUNKS; }
 
 cudaError_t launch_ffn_prep(const float *x, const moe_dims_t &d, uint16_t *xb, uint16_t *xd, float *y,
@@ -1819,7 +1550,7 @@ cudaError_t launch_layer_ni(const ExpertMaps &maps, const RouterMaps &rmaps, con
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(NTHREADS_UM);
+    cfg.blockDim = dim3(NTHREADS);
     cfg.dynamicSmemBytes = smem_bytes<RG>();
     cfg.stream = s;
     // every CTA must be resident: the CTAs wait for one another at the
@@ -1838,13 +1569,13 @@ cudaError_t launch_layer_ni(const ExpertMaps &maps, const RouterMaps &rmaps, con
 }  // namespace
 
 namespace {
-template <class RG, bool UM>
+template <class RG>
 cudaError_t launch_expert_ffn_rg(const ExpertMaps &maps, const ExpertArgs &a, int sms, int dev, cudaStream_t s) {
-    cudaError_t err = configure_smem(expert_ffn_kernel<RG, UM>, smem_bytes<RG>(), dev);
+    cudaError_t err = configure_smem(expert_ffn_kernel<RG>, smem_bytes<RG>(), dev);
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(sms);
-    cfg.blockDim = dim3(cta_threads<UM>());
+    cfg.blockDim = dim3(NTHREADS);
     cfg.dynamicSmemBytes = smem_bytes<RG>();
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
@@ -1852,7 +1583,7 @@ cudaError_t launch_expert_ffn_rg(const ExpertMaps &maps, const ExpertArgs &a, in
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;  // always chained to the previous kernel with programmatic dependent launch
-    return cudaLaunchKernelEx(&cfg, expert_ffn_kernel<RG, UM>, maps, a);
+    return cudaLaunchKernelEx(&cfg, expert_ffn_kernel<RG>, maps, a);
 }
 }  // namespace
 
@@ -1863,11 +1594,11 @@ cudaError_t launch_expert_ffn(const ExpertMaps &maps, const uint16_t *xb, const 
     cudaError_t err = device_sms(&dev, &sms);
     if (err != cudaSuccess) return err;
     const ExpertArgs a = make_expert_args(xb, d, l, y, h, wd, ctr, sms);
-    // dense mode on the tensor cores, the ring sized for the token rows
-    if (d.B <= 16) return launch_expert_ffn_rg<RingB16, true>(maps, a, sms, dev, s);
-    if (d.B <= 32) return launch_expert_ffn_rg<RingB32, true>(maps, a, sms, dev, s);
-    if (d.B <= DENSE_MAX) return launch_expert_ffn_rg<RingB64, true>(maps, a, sms, dev, s);
-    return launch_expert_ffn_rg<RingB64, false>(maps, a, sms, dev, s);
+    // the ring sized for the token rows: dense mode up to 16, 32 or 64
+    // tokens, tile mode (32 pair rows) above
+    if (d.B <= 16) return launch_expert_ffn_rg<RingB16>(maps, a, sms, dev, s);
+    if (d.B <= 32 || d.B > DENSE_MAX) return launch_expert_ffn_rg<RingB32>(maps, a, sms, dev, s);
+    return launch_expert_ffn_rg<RingB64>(maps, a, sms, dev, s);
 }
 
 cudaError_t launch_layer_fused(const ExpertMaps &maps, const RouterMaps &rmaps, const moe_dims_t &d,

@@ -59,8 +59,9 @@ def _ffn(name, x, dl, ws):
     return y, moe.moe_check_error(ws)
 
 
-# tiny (B = 4): dense mode; ragged (B = 37): token tiles of the dispatched pairs
-@pytest.mark.parametrize("name,B,k0", [("tiny", 4, 2), ("ragged", 37, 2)])
+# tiny (B = 4), ragged (B = 37): dense mode; ragged (B = 70): token tiles of
+# the dispatched pairs
+@pytest.mark.parametrize("name,B,k0", [("tiny", 4, 2), ("ragged", 37, 2), ("ragged", 70, 2)])
 @pytest.mark.parametrize("damage", ["n_active_above_E", "n_active_negative", "active_id_out_of_range",
                                     "offsets_decreasing", "offsets_past_pairs"])
 def test_inconsistent_lists_are_reported_and_contained(name, B, k0, damage):
@@ -90,7 +91,7 @@ def test_inconsistent_lists_are_reported_and_contained(name, B, k0, damage):
     assert_close_y(y2.cpu().numpy(), y_r, f"{name} after {damage}")
 
 
-@pytest.mark.parametrize("name,B,k0", [("tiny", 4, 2), ("ragged", 37, 2)])
+@pytest.mark.parametrize("name,B,k0", [("tiny", 4, 2), ("ragged", 37, 2), ("ragged", 70, 2)])
 def test_token_outside_batch_is_skipped_and_reported(name, B, k0):
     # one list entry names token B + 5; that pair is skipped, the other
     # pairs are combined as usual (dense mode: the preparation leaves its
@@ -120,7 +121,8 @@ def test_bounded_waits_expire_and_report(path):
     # ends its share of the call and exits; the call completes and
     # moe_check_error reports MOE_ERR_INTERNAL.  After the default limit is
     # restored and the workspace zeroed, the same call matches the oracle.
-    name, B = ("q30b", 16) if path != "layer_tiled" else ("q30b", 64)
+    # the four-kernel path starts above 64 tokens
+    name, B = ("q30b", 16) if path != "layer_tiled" else ("q30b", 96)
     S = shape(name)
     L = host_layer(name, 0)
     D = device_layer(name, 0)

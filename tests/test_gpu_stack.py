@@ -80,8 +80,13 @@ def test_stack_of_four_q30b_b16(mode, k0, budget):
     _check_stack("q30b", 16, 4, mode, k0, budget)
 
 
-def test_stack_tiled_path_q30b_b64():
+def test_stack_fused_path_q30b_b64():
     _check_stack("q30b", 64, 2, OEA, 4)
+
+
+def test_stack_tiled_path_q30b_b96():
+    # above 64 tokens: the four chained kernels per layer
+    _check_stack("q30b", 96, 2, OEA, 4)
 
 
 def test_stack_small_shapes():
