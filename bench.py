@@ -71,11 +71,19 @@ WORKLOADS = {
                               rule="OEA k0=4, channel top-k 13 %"),
 }
 
-# DRAM bytes (read + write) per launch of the expert kernel from an ncu
-# capture of the same workload (profiles/expert_ffn_kernel_q30b_b16_oea4.md);
+# DRAM bytes (read + write) per launch of the dominant kernel (the fused
+# layer kernel up to 64 tokens) from an ncu capture of the same workload on
+# one weight copy (profiles/layer_kernel_q30b_b16_oea4.md, ..._b64_...);
 # a workload without an entry reports null.  Entries are dropped whenever
 # the kernel changes.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    "q30b_b16_oea4": 142876928 + 3602944,
+    "q30b_b64_oea4": 284828672 + 5148672,
+    # channel top-k workloads: channel_stream_kernel, which moves the weights
+    # (profiles/channel_stream_kernel_q30b_oea4_ch13.md)
+    "q30b_b1_oea4_ch13": 4967936,
+    "q30b_b4_oea4_ch13": 33602560,
+}
 
 
 def workload_desc(w: dict) -> str:
@@ -556,7 +564,8 @@ def run_channels(args, w, rank, world, local_rank):
                    "l2": f"{ROTATE} rotating copies of the expert weights"},
         "us_per_call": ms_call * 1e3,
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
-                     "traffic": None, "kernel": "channel_select + channel_items + channel_stream kernels",
+                     "traffic": NCU_TRAFFIC.get(args.workload),
+                     "kernel": "channel_select + channel_items + channel_stream kernels (traffic: channel_stream)",
                      "peak_source": f"{peak_kind} HBM copy bandwidth"},
         "gpu_launches": 3 * reps * ROTATE, "clocks": sampler.summary(),
     }
@@ -649,16 +658,35 @@ def run_sweep(args):
 def run_profile_case(args, w):
     """A small case for ncu captures: one weight copy (about 1.2 GB for the
     Qwen3-30B shape, so the activated experts still exceed L2), `warmup`
-    layer calls, then `steps` more, launched from the stream, no timing."""
+    layer calls, then `steps` more, launched from the stream, no timing.
+    Channel workloads: routing and selection once, then the channel top-k
+    calls; the sector-counted bytes of one call are printed."""
     import torch
     import aware_expert_routing_moe_b200 as moe
     S = ms.SHAPES[w["shape"]]
     B = w["B"]
     L = ms.make_weights(S, 0)
-    t = lambda a: torch.from_numpy(a).cuda()
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
     x = t(ms.make_tokens(S, B, 0, kind=w.get("kind", "normal")))
     Wg, bias = t(L["Wg"]), t(L["bias"])
     g, u, dn = (t(L[n].view(np.int16)) for n in ("Wgate", "Wup", "Wdown"))
+    if "channels" in w:
+        c = max(1, int(round(w["channels"] * S.F)))
+        downT = moe.moe_down_channel_major(dn)
+        logits, probs, _, _ = moe.moe_route(x, Wg, bias, S.k)
+        sel, sw, _ = moe.moe_reselect(logits, probs, S.k, w["mode"], w["k0"], w["budget"])
+        score = t(np.random.default_rng(1000).standard_normal((B, S.k, S.F)).astype(np.float32))
+        keep = torch.empty(B, S.k, S.F // 32, dtype=torch.int32, device="cuda")
+        cws = torch.zeros(moe.load_library().moe_channels_workspace_bytes(moe.Dims(B, S.d, S.E, S.k, S.F)),
+                          dtype=torch.uint8, device="cuda")
+        for _ in range(args.warmup + args.steps):
+            moe.moe_expert_ffn_channels(x, g, u, downT, sel, sw, score, c, keep=keep, ws=cws)
+        torch.cuda.synchronize()
+        status = moe.moe_check_error(cws)
+        nbytes = channel_bytes(keep.cpu().numpy(), sel.cpu().numpy(), S.d, S.F, B, S.k)
+        print(f"profile case {args.workload}: {args.warmup}+{args.steps} channel calls, status {status}, "
+              f"sector-counted bytes per call {nbytes}")
+        return 0 if status == 0 else 1
     ws = moe.new_workspace(B, S.d, S.E, S.k, S.F)
     for _ in range(args.warmup + args.steps):
         moe.moe_layer_decode(x, Wg, bias, g, u, dn, S.k, w["mode"], w["k0"], w["budget"], ws=ws,
