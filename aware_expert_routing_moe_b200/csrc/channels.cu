@@ -96,6 +96,8 @@ struct SelectArgs {
 __global__ void __launch_bounds__(CH_THREADS) channel_select_kernel(SelectArgs a) {
     __shared__ unsigned hist[CH_WARPS][256];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // the union kernel may launch now; it waits for this grid before reading
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     // y = 0 (the stream kernel adds into it)
     const int n4 = a.B * a.d / 4;
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += gridDim.x * blockDim.x)
@@ -172,6 +174,10 @@ __global__ void __launch_bounds__(CH_THREADS) channel_items_kernel(ItemsArgs a) 
     const int t = threadIdx.x;
     const int pairs = a.B * a.k, words = a.F / 32;
     if (t < E_MAX / 32) s_emask[t] = 0u;
+    // launched early (programmatic dependent launch): the keep masks are
+    // complete once the selection grid has finished
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     __syncthreads();
     for (int p = t; p < pairs; p += blockDim.x) {
         const int e = a.sel_idx[p];
@@ -307,6 +313,10 @@ __global__ void __launch_bounds__(CH_THREADS, 1) channel_stream_kernel(StreamArg
         xs[i] = __ldg(a.x + i);
         ys[i] = 0.0f;
     }
+    // everything above overlaps the union kernel (programmatic dependent
+    // launch); the items, the slots and y = 0 are complete once it (and the
+    // selection before it) has finished
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     __syncthreads();
     const int n_items = a.ctr_ro->n_items;
     unsigned long long policy;
@@ -510,8 +520,16 @@ cudaError_t launch_channels(const float *x, const uint16_t *Wgate, const uint16_
     ia.slot_np = reinterpret_cast<int32_t *>(w + L.slot_np);
     ia.slot_pairs = reinterpret_cast<int32_t *>(w + L.slot_pairs);
     ia.items = reinterpret_cast<int32_t *>(w + L.items);
-    channel_items_kernel<<<1, CH_THREADS, 0, s>>>(ia);
-    err = cudaGetLastError();
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1);
+    cfg.blockDim = dim3(CH_THREADS);
+    cfg.stream = s;
+    cfg.attrs = pdl;
+    cfg.numAttrs = 1;
+    err = cudaLaunchKernelEx(&cfg, channel_items_kernel, ia);
     if (err != cudaSuccess) return err;
     StreamArgs ta;
     ta.x = x;
@@ -541,8 +559,9 @@ cudaError_t launch_channels(const float *x, const uint16_t *Wgate, const uint16_
         if (err != cudaSuccess) return err;
         configured[dev] = true;
     }
-    channel_stream_kernel<<<g_ch_sms[dev], CH_THREADS, smem, s>>>(ta);
-    return cudaGetLastError();
+    cfg.gridDim = dim3(g_ch_sms[dev]);
+    cfg.dynamicSmemBytes = smem;
+    return cudaLaunchKernelEx(&cfg, channel_stream_kernel, ta);
 }
 
 }  // namespace moe

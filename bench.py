@@ -79,10 +79,6 @@ WORKLOADS = {
 NCU_TRAFFIC = {
     "q30b_b16_oea4": 142876928 + 3602944,
     "q30b_b64_oea4": 284828672 + 5148672,
-    # channel top-k workloads: channel_stream_kernel, which moves the weights
-    # (profiles/channel_stream_kernel_q30b_oea4_ch13.md)
-    "q30b_b1_oea4_ch13": 4967936,
-    "q30b_b4_oea4_ch13": 33602560,
 }
 
 
