@@ -24,7 +24,7 @@
 // kernel has before the token lists exist: its CTAs rank the tokens' first
 // experts themselves (OEA, plain top-k) or read the set the selection CTA
 // publishes (the batch-wide rules), and start streaming at once.
-// Larger batches (tile mode) use tiles of up to 32 (token, expert) pairs:
+// Larger batches (tile mode) use tiles of up to 64 (token, expert) pairs:
 // the input preparation copies each pair's x row (bf16) into a pair-indexed
 // buffer in the lists' order, so a tile's x rows are one swizzled box like
 // H's, and the down epilogue weighs each pair by its list weight.
@@ -62,7 +62,7 @@ constexpr int NCW = 8;  // epilogue warps
 // partial accumulator of its own.
 constexpr int NISSUE = 4;
 constexpr int NTHREADS = (NCW + 1 + NISSUE) * 32;  // + one producer warp
-constexpr int TN = 32;         // pairs per token tile (batches above 64 tokens)
+constexpr int TN = 64;         // pairs per token tile (batches above 64 tokens)
 constexpr int DENSE_MAX = 64;  // dense mode (every unit takes the whole batch) up to 64 tokens
 // GU units of 32 gate rows and the same 32 up rows; a stage holds 4 chunks
 // of 64 columns, each chunk as the gate tile [32][64] followed by the up
@@ -78,7 +78,7 @@ constexpr int MAX_STAGES = 5;
 constexpr int W_BYTES = 32768;               // weight bytes per stage (both kinds)
 // Ring shapes: stages of 32 KB of weights plus an operand region for the
 // token rows of 4 chunks (x for gate/up, H for down): bpad rows in dense
-// mode (8, 16 or 32 KB for up to 16, 32 or 64 tokens), 32 pair rows in tile
+// mode (8, 16 or 32 KB for up to 16, 32 or 64 tokens), 64 pair rows in tile
 // mode; PARTB: the epilogue's accumulator copy, [rows][64] fp32.
 template <int ST, int OPB, int PARTB>
 struct Ring {
@@ -104,7 +104,8 @@ static_assert(2 * UM_ROWS == UMMA_M && D_ROWS == UMMA_M && D_ROWS * 128 == UM_CH
 static_assert(16 * 128 * UM_CHUNKS <= RingB16::OP_BYTES && 32 * 128 * UM_CHUNKS <= RingB32::OP_BYTES &&
                   DENSE_MAX * 128 * UM_CHUNKS <= RingB64::OP_BYTES && DENSE_MAX * 128 * D_CHUNKS <= RingB64::OP_BYTES,
               "token rows do not fit");
-static_assert(TN == 32, "tile mode uses the 32-row ring");
+static_assert(TN * 128 * UM_CHUNKS <= RingB64::OP_BYTES && TN * 64 * 4 <= RingB64::PART_BYTES,
+              "tile mode uses the 64-row ring");
 static_assert(D_ROWS * 128 * D_CHUNKS <= W_BYTES, "down tile does not fit");
 static_assert(DENSE_MAX * 64 * 4 <= RingB64::PART_BYTES, "accumulator copy does not fit");
 static_assert(RingB16::SLOT_BYTES % 1024 == 0 && RingB32::SLOT_BYTES % 1024 == 0 && RingB64::SLOT_BYTES % 1024 == 0,
@@ -1595,9 +1596,9 @@ cudaError_t launch_expert_ffn(const ExpertMaps &maps, const uint16_t *xb, const 
     if (err != cudaSuccess) return err;
     const ExpertArgs a = make_expert_args(xb, d, l, y, h, wd, ctr, sms);
     // the ring sized for the token rows: dense mode up to 16, 32 or 64
-    // tokens, tile mode (32 pair rows) above
+    // tokens, tile mode (64 pair rows) above
     if (d.B <= 16) return launch_expert_ffn_rg<RingB16>(maps, a, sms, dev, s);
-    if (d.B <= 32 || d.B > DENSE_MAX) return launch_expert_ffn_rg<RingB32>(maps, a, sms, dev, s);
+    if (d.B <= 32) return launch_expert_ffn_rg<RingB32>(maps, a, sms, dev, s);
     return launch_expert_ffn_rg<RingB64>(maps, a, sms, dev, s);
 }
 
