@@ -523,7 +523,7 @@ __device__ void producer(const ExpertArgs &a, const ExpertMaps &m, SharedCtl *ct
         have = have_nxt;
     }
     if (ok) {
-        // end marker for the consumers
+        // end marker for the issuers (and, through them, the epilogue)
         const int slot = g % STAGES;
         if (g >= STAGES && !wait_phase(&ctl->empty[slot], ((g / STAGES) - 1) & 1, ctl, a.ctr, DEV_TIMEOUT_EMPTY))
             ok = false;

@@ -77,8 +77,12 @@ WORKLOADS = {
 # a workload without an entry reports null.  Entries are dropped whenever
 # the kernel changes.
 NCU_TRAFFIC = {
-    "q30b_b16_oea4": 142876928 + 3602944,
-    "q30b_b64_oea4": 284828672 + 5148672,
+    "q30b_b16_oea4": 142883072 + 3001856,
+    "q30b_b64_oea4": 284835840 + 3391232,
+    # channel top-k workloads: channel_stream_kernel, which moves the weights
+    # (profiles/channel_stream_kernel_q30b_oea4_ch13.md)
+    "q30b_b1_oea4_ch13": 4969984,
+    "q30b_b4_oea4_ch13": 33603328,
 }
 
 

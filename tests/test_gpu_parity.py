@@ -189,11 +189,12 @@ def test_layer_decode_parity_small(name, B, seed, mode, k0, budget):
 Q30_CASES = [(1, NONE, 0, 0), (1, OEA, 2, 0), (4, OEA, 4, 0), (16, NONE, 0, 0), (16, OEA, 2, 0),
              (16, OEA, 4, 0), (16, OEA, 6, 0), (16, OEA, 8, 0), (16, XSHARE, 0, 16), (16, AFFINITY, 0, 0),
              (64, AFFINITY, 0, 0), (32, NONE, 0, 0), (17, OEA, 4, 0),
-             # 33..64 tokens: the wide dense mode (ragged token counts included)
+             # 33..64 tokens: the 64-row ring (ragged token counts included)
              (33, OEA, 4, 0), (48, NONE, 0, 0), (57, XSHARE, 0, 40),
              (64, NONE, 0, 0), (64, OEA, 4, 0),
-             # above 64 tokens: token tiles of dispatched pairs
-             (65, OEA, 4, 0), (96, NONE, 0, 0)]
+             # above 64 tokens: tiles of up to 64 dispatched pairs (several
+             # tiles per expert at 256 tokens)
+             (65, OEA, 4, 0), (96, NONE, 0, 0), (128, OEA, 4, 0), (256, NONE, 0, 0)]
 
 
 @pytest.mark.parametrize("B,mode,k0,budget", Q30_CASES)
