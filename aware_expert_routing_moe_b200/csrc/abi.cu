@@ -163,6 +163,18 @@ moe_lists_t ws_lists(void *ws, const WsLayout &L) {
     return l;
 }
 
+// The most experts a call under `rule` can activate: the union of every
+// token's candidates (OEA: its first k0; top-k and the affinity rule: its
+// k), at most the budget for the XShare rules, at most E.
+int max_activated(const moe_dims_t &d, const moe_reselect_t &rule) {
+    int per_token = d.k;
+    if (rule.mode == MOE_RESELECT_OEA) per_token = rule.k0;
+    long long n = static_cast<long long>(d.B) * per_token;
+    if ((rule.mode == MOE_RESELECT_XSHARE || rule.mode == MOE_RESELECT_XSHARE_HIER) && rule.budget < n)
+        n = rule.budget;
+    return static_cast<int>(n < d.E ? n : d.E);
+}
+
 // One layer call (arguments validated): up to 64 tokens the fused kernel,
 // above the four chained kernels.  residual: y = x + the experts' output;
 // chained: the layer follows the previous layer of a stack on the stream.
@@ -173,13 +185,13 @@ moe_status_t layer_call(const float *x, const moe_layer_weights_t &w, const moe_
 }  // namespace
 
 bool encode_expert_maps(ExpertMaps *m, const moe_dims_t &d, const uint16_t *Wgate, const uint16_t *Wup,
-                        const uint16_t *Wdown, const uint16_t *h, const uint16_t *x) {
+                        const uint16_t *Wdown, const uint16_t *h, const uint16_t *x, int wm) {
     std::memset(m, 0, sizeof(*m));
     const uint64_t E = d.E, F = d.d_ff, D = d.d;
-    const uint32_t gu_chunks = expert_ffn_gu_chunks(d.d, d.B), d_chunks = expert_ffn_d_chunks(d.d_ff);
-    const uint32_t gu_box = expert_ffn_gu_box_chunks(d.d, d.B);
-    return encode_bf16_chunked(&m->gate, Wgate, E * F, D, expert_ffn_gu_rows(d.B), gu_box) &&
-           encode_bf16_chunked(&m->up, Wup, E * F, D, expert_ffn_gu_rows(d.B), gu_box) &&
+    const uint32_t gu_chunks = expert_ffn_gu_chunks(d.d, wm), d_chunks = expert_ffn_d_chunks(d.d_ff);
+    const uint32_t gu_box = expert_ffn_gu_box_chunks(d.d, wm);
+    return encode_bf16_chunked(&m->gate, Wgate, E * F, D, expert_ffn_gu_rows(wm), gu_box) &&
+           encode_bf16_chunked(&m->up, Wup, E * F, D, expert_ffn_gu_rows(wm), gu_box) &&
            encode_bf16_chunked(&m->down, Wdown, E * D, F, expert_ffn_d_rows(), d_chunks) &&
            encode_bf16_chunked(&m->h, h,
                                expert_ffn_dense_batch(d.B) ? static_cast<uint64_t>(active_slots(d)) * d.B
@@ -231,8 +243,10 @@ moe_status_t layer_call(const float *x, const moe_layer_weights_t &w, const moe_
     const bool dense = expert_ffn_dense_batch(dims.B) != 0;
     // the expert kernel's x: bf16 x (B <= 64) or the dispatched pair rows
     uint16_t *xk = dense ? seg<uint16_t>(ws, L.xb) : seg<uint16_t>(ws, L.xd);
+    const int wm = expert_ffn_warp_mma(dims, max_activated(dims, rule));
     ExpertMaps maps;
-    if (!encode_expert_maps(&maps, dims, w.Wgate, w.Wup, w.Wdown, seg<uint16_t>(ws, L.h), xk)) return MOE_ERR_CUDA;
+    if (!encode_expert_maps(&maps, dims, w.Wgate, w.Wup, w.Wdown, seg<uint16_t>(ws, L.h), xk, wm))
+        return MOE_ERR_CUDA;
     RouterMaps rmaps;
     if (!encode_router_maps(&rmaps, dims, x, w.Wg)) return MOE_ERR_CUDA;
     Counters *ctr = seg<Counters>(ws, L.counters);
@@ -245,7 +259,7 @@ moe_status_t layer_call(const float *x, const moe_layer_weights_t &w, const moe_
         // B <= 64: one persistent kernel for the whole call
         return from_cuda(launch_layer_fused(maps, rmaps, dims, rule, x, w.bias, logits, probs, xk, y,
                                             seg<uint16_t>(ws, L.h), seg<float>(ws, L.wd), si, sw, lists, n_active,
-                                            ctr, residual, chained, s));
+                                            ctr, wm, residual, chained, s));
     }
     // larger batches: router, selection (lists), the dispatch of each
     // pair's x row, then the expert kernel, chained with programmatic
@@ -256,7 +270,7 @@ moe_status_t layer_call(const float *x, const moe_layer_weights_t &w, const moe_
     if (st != MOE_OK) return st;
     st = from_cuda(launch_ffn_prep(x, dims, nullptr, xk, nullptr, nullptr, lists, nullptr, true, s));
     if (st != MOE_OK) return st;
-    return from_cuda(launch_expert_ffn(maps, xk, dims, lists, y, seg<uint16_t>(ws, L.h), nullptr, ctr, s));
+    return from_cuda(launch_expert_ffn(maps, xk, dims, lists, y, seg<uint16_t>(ws, L.h), nullptr, ctr, wm, s));
 }
 
 }  // namespace
@@ -331,14 +345,16 @@ moe_status_t moe_expert_ffn(const float *x, const uint16_t *Wgate, const uint16_
     const bool dense = expert_ffn_dense_batch(dims.B) != 0;
     // the expert kernel's x: bf16 x (B <= 64) or the dispatched pair rows
     uint16_t *xk = dense ? seg<uint16_t>(ws, L.xb) : seg<uint16_t>(ws, L.xd);
+    // caller-supplied lists: any union of the tokens' k choices
+    const int wm = expert_ffn_warp_mma(dims, dims.B * dims.k);
     ExpertMaps maps;
-    if (!encode_expert_maps(&maps, dims, Wgate, Wup, Wdown, seg<uint16_t>(ws, L.h), xk)) return MOE_ERR_CUDA;
+    if (!encode_expert_maps(&maps, dims, Wgate, Wup, Wdown, seg<uint16_t>(ws, L.h), xk, wm)) return MOE_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     Counters *ctr = seg<Counters>(ws, L.counters);
     float *wd = dense ? seg<float>(ws, L.wd) : nullptr;
     st = from_cuda(launch_ffn_prep(x, dims, dense ? xk : nullptr, dense ? nullptr : xk, y, ctr, lists, wd, false, s));
     if (st != MOE_OK) return st;
-    return from_cuda(launch_expert_ffn(maps, xk, dims, lists, y, seg<uint16_t>(ws, L.h), wd, ctr, s));
+    return from_cuda(launch_expert_ffn(maps, xk, dims, lists, y, seg<uint16_t>(ws, L.h), wd, ctr, wm, s));
 }
 
 moe_status_t moe_layer_decode(const float *x, const float *Wg, const float *bias, const uint16_t *Wgate,

@@ -39,6 +39,9 @@
 // unit's epilogue overlaps the next unit's MMAs; the MMA completion itself
 // frees the stage.  Eight epilogue warps read the accumulators out (silu *
 // u -> H, or weighted atomics into y) and publish gate/up completions.
+// Batches of up to 8 tokens run the warp-MMA variant of the same roles
+// instead: 16-row gate/up units, and eight consumer warps that do each
+// stage's math with mma.sync and the epilogues themselves.
 // Every wait is bounded by a time limit; on expiry the CTA records an error
 // code in the workspace, drains its in-flight copies and MMAs and returns.
 // The last CTA to finish puts the workspace counters of the call back to
@@ -98,6 +101,26 @@ constexpr int smem_bytes() {
 using RingB16 = Ring<5, 8192, 16 * 64 * 4>;
 using RingB32 = Ring<4, 16384, 32 * 64 * 4>;
 using RingB64 = Ring<3, 32768, 64 * 64 * 4>;
+// Batches of up to WM_MAX tokens that activate at most WM_ACTIVE_MAX
+// experts take the warp-MMA path instead (mma.sync m16n8k16, the tokens one
+// 8-column tile): its gate/up units are 16 rows, a stage the gate box
+// [WM_CHUNKS][16 rows][64 cols] and the up box after it.  With so few
+// tokens the work per weight byte is small enough for the warps, and the
+// finer units spread the few activated experts over more CTAs; a 64-row
+// tensor-core MMA cannot take a 16-row unit without reading rows it does
+// not use.  With more experts the stream is long enough for 32-row units,
+// and those are cheaper per byte (measured: at Qwen3-30B shape, 8 tokens,
+// top-8 the warp-MMA path took 54 us against 51 us; with OEA k0 = 4, at
+// most 32 experts, 35 us against 36 us).
+constexpr int WM_MAX = 8;
+constexpr int WM_ACTIVE_MAX = 32;
+constexpr int WM_ROWS = 16;
+constexpr int WM_CHUNKS = 8;
+constexpr int WM_UP_OFF = WM_ROWS * 128 * WM_CHUNKS;  // the up box after the gate box
+constexpr int SIG_SLOTS = 4;  // gate/up completions queued for the signal warp (warp-MMA path)
+static_assert(2 * WM_UP_OFF == W_BYTES, "warp-MMA gate/up boxes must fill the weight region");
+static_assert(WM_MAX * 128 * WM_CHUNKS <= RingB16::OP_BYTES, "warp-MMA x rows do not fit");
+static_assert(4 * 2 * WM_ROWS * WM_MAX * 4 <= RingB16::PART_BYTES, "warp-MMA gate/up partial sums do not fit");
 static_assert(UM_CHUNKS * UM_CHUNK_BYTES == W_BYTES, "gate/up chunks must fill the weight region");
 static_assert(2 * UM_ROWS == UMMA_M && D_ROWS == UMMA_M && D_ROWS * 128 == UM_CHUNK_BYTES,
               "a gate/up chunk and a down chunk are one 64-row MMA operand each");
@@ -168,6 +191,12 @@ struct SharedCtl {
     AccHdr acc_hdr[2];
     uint32_t tmem;  // TMEM base address of the CTA's allocation
     volatile int epi_go, epi_lists;  // outcomes of the epilogue's waits (its thread 0)
+    // warp-MMA path: outcome of a stage's wait (by stage parity); the
+    // queue of gate/up completions the signal warp publishes
+    volatile int wm_go[2];
+    unsigned long long sig_full[SIG_SLOTS];
+    unsigned long long sig_empty[SIG_SLOTS];
+    int sig_iact[SIG_SLOTS];
 };
 
 static_assert(sizeof(SharedCtl) <= CTL_BYTES, "SharedCtl does not fit its reservation");
@@ -420,8 +449,9 @@ __device__ bool fetch_unit(int j, int &win_base, int n_units, const ExpertArgs &
 }
 
 // A gate/up stage is UM_CHUNKS chunk copies of each matrix, interleaved
-// per chunk (the tensor-core operand layout).
-template <class RG, bool DENSE>
+// per chunk (the tensor-core operand layout), or on the warp-MMA path (WM)
+// one gate box and one up box of gc chunks each.
+template <class RG, bool DENSE, bool WM>
 __device__ void producer(const ExpertArgs &a, const ExpertMaps &m, SharedCtl *ctl, unsigned char *slots) {
     constexpr int STAGES = RG::STAGES;
     const int lane = threadIdx.x & 31;
@@ -458,7 +488,8 @@ __device__ void producer(const ExpertArgs &a, const ExpertMaps &m, SharedCtl *ct
             const int gcv = min(gc, (a.d >> 6) - (cur.k0 + s) * gc);
             // x tile: all B token rows (dense mode) or the tile's TN pair rows
             const unsigned xbytes = static_cast<unsigned>(gc) * (a.dense ? a.bpad : TN) * 128u;
-            const unsigned wbytes = 2u * gcv * UM_TILE;
+            // (the warp-MMA boxes always hold gc chunks; the tail of d reads as zeros)
+            const unsigned wbytes = WM ? 2u * gc * (WM_ROWS * 128u) : 2u * gcv * UM_TILE;
             const unsigned bytes = cur.type == UNIT_GU ? wbytes + xbytes : dc * (D_ROWS * 128u) + dc * (a.hrows * 128u);
             if (lane == 0) {
                 StageHdr &h = ctl->hdr[slot];
@@ -476,13 +507,21 @@ __device__ void producer(const ExpertArgs &a, const ExpertMaps &m, SharedCtl *ct
             __syncwarp();
             if (cur.type == UNIT_GU) {
                 const int grow = cur.e * a.F + cur.row0;
-                // chunk c: gate tile at 8 KB c, up tile 4 KB after it
-                if (lane < gcv)
-                    tma_load_3d_stream(wdst + lane * UM_CHUNK_BYTES, &m.gate, 0, grow, s * gc + lane,
-                                       &ctl->full[slot], policy);
-                else if (lane >= 8 && lane < 8 + gcv)
-                    tma_load_3d_stream(wdst + (lane - 8) * UM_CHUNK_BYTES + UM_TILE, &m.up, 0, grow,
-                                       s * gc + lane - 8, &ctl->full[slot], policy);
+                if constexpr (WM) {
+                    // the gate box of gc chunks, the up box after it
+                    if (lane == 0)
+                        tma_load_3d_stream(wdst, &m.gate, 0, grow, s * gc, &ctl->full[slot], policy);
+                    else if (lane == 8)
+                        tma_load_3d_stream(wdst + WM_UP_OFF, &m.up, 0, grow, s * gc, &ctl->full[slot], policy);
+                } else {
+                    // chunk c: gate tile at 8 KB c, up tile 4 KB after it
+                    if (lane < gcv)
+                        tma_load_3d_stream(wdst + lane * UM_CHUNK_BYTES, &m.gate, 0, grow, s * gc + lane,
+                                           &ctl->full[slot], policy);
+                    else if (lane >= 8 && lane < 8 + gcv)
+                        tma_load_3d_stream(wdst + (lane - 8) * UM_CHUNK_BYTES + UM_TILE, &m.up, 0, grow,
+                                           s * gc + lane - 8, &ctl->full[slot], policy);
+                }
                 // x rows for this column range, one swizzled box: all B
                 // tokens (dense mode) or the tile's pairs of the dispatched x
                 if (lane == 16) tma_load_3d(odst, &m.x, 0, (DENSE || a.dense) ? 0 : cur.p0, s * gc, &ctl->full[slot]);
@@ -523,7 +562,8 @@ __device__ void producer(const ExpertArgs &a, const ExpertMaps &m, SharedCtl *ct
         have = have_nxt;
     }
     if (ok) {
-        // end marker for the issuers (and, through them, the epilogue)
+        // end marker for the issuers (and, through them, the epilogue) or
+        // the warp-MMA consumers
         const int slot = g % STAGES;
         if (g >= STAGES && !wait_phase(&ctl->empty[slot], ((g / STAGES) - 1) & 1, ctl, a.ctr, DEV_TIMEOUT_EMPTY))
             ok = false;
@@ -748,6 +788,222 @@ __device__ void umma_epilogue(const ExpertArgs &a, SharedCtl *ctl, float *xch, u
     }
 }
 
+// ------------------------------------------------ warp-MMA path (B <= 8) --
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t &r0, uint32_t &r1) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
+}
+// c += A (16 x 16, row-major fragments a0..a3) * B (16 x 8, column fragments b0, b1), fp32 accumulate
+__device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// Address of (row r, 16-byte column group c) in a 128B-swizzled tile of
+// 128-byte rows whose base is 1 KiB aligned (the TMA's swizzle pattern).
+__device__ __forceinline__ uint32_t swz(uint32_t base, int r, int c) {
+    return base + r * 128 + ((c ^ (r & 7)) << 4);
+}
+// The B operand fragment of k-step ks (16 columns) of an [8 rows][64 cols]
+// token tile: lanes 0..7 address the rows' first 8 columns, lanes 8..15
+// the next 8.
+__device__ __forceinline__ void wm_b_frag(uint32_t tile, int ks, int lane, uint32_t &b0, uint32_t &b1) {
+    ldsm_x2(swz(tile, lane & 7, ((ks & 3) << 1) + ((lane >> 3) & 1)), b0, b1);
+}
+
+// Gate/up stage: warp w takes k-steps w, w + NCW, ... (16 columns each) of
+// the stage's 16 gate and 16 up rows against the 8 token columns.
+__device__ __forceinline__ void wm_gu_stage(uint32_t wbase, uint32_t xbase, int nks, int warp, int lane,
+                                            float (&cg)[4], float (&cu)[4]) {
+#pragma unroll 4
+    for (int ks = warp; ks < nks; ks += NCW) {
+        const int c = ks >> 2;  // 64-column chunk
+        const int col = ((ks & 3) << 1) + (lane >> 4);
+        uint32_t g0, g1, g2, g3, u0, u1, u2, u3, b0, b1;
+        ldsm_x4(swz(wbase + c * (WM_ROWS * 128), lane & 15, col), g0, g1, g2, g3);
+        ldsm_x4(swz(wbase + WM_UP_OFF + c * (WM_ROWS * 128), lane & 15, col), u0, u1, u2, u3);
+        wm_b_frag(xbase + c * (WM_MAX * 128), ks, lane, b0, b1);
+        mma_bf16(cg, g0, g1, g2, g3, b0, b1);
+        mma_bf16(cu, u0, u1, u2, u3, b0, b1);
+    }
+}
+// Down stage: warp w takes rows 16 (w % 4) .. + 16 of the 64-row unit over
+// the k-steps of its half of the stage, (w / 4) * 2 D_CHUNKS ...
+__device__ __forceinline__ void wm_d_stage(uint32_t wbase, uint32_t hbase, int nks, int warp, int lane,
+                                           float (&acc)[4]) {
+    const int r = (warp & 3) * 16 + (lane & 15);
+    const int k0 = (warp >> 2) * (2 * D_CHUNKS);
+    const int k1 = min(nks, k0 + 2 * D_CHUNKS);
+#pragma unroll 4
+    for (int ks = k0; ks < k1; ++ks) {
+        const int c = ks >> 2;
+        uint32_t a0, a1, a2, a3, b0, b1;
+        ldsm_x4(swz(wbase + c * (D_ROWS * 128), r, ((ks & 3) << 1) + (lane >> 4)), a0, a1, a2, a3);
+        wm_b_frag(hbase + c * (WM_MAX * 128), ks, lane, b0, b1);
+        mma_bf16(acc, a0, a1, a2, a3, b0, b1);
+    }
+}
+
+// Queue one gate/up completion (i >= 0) or the end marker (i < 0) for the
+// signal warp (consumer thread 0).  A wait that expires has recorded the
+// error and raised the abort flag, which ends the consumers at their next
+// stage.
+__device__ void wm_post(SharedCtl *ctl, Counters *ctr, int q, int i) {
+    const int slot = q % SIG_SLOTS;
+    if (q >= SIG_SLOTS && !wait_phase(&ctl->sig_empty[slot], ((q / SIG_SLOTS) - 1) & 1, ctl, ctr, DEV_TIMEOUT_EMPTY))
+        return;
+    ctl->sig_iact[slot] = i;
+    mbar_arrive(&ctl->sig_full[slot]);
+}
+// Signal warp (one thread): turns the queued completions into gate/up
+// counts visible to the whole GPU.  The consumers wrote H and passed a CTA
+// barrier before the completion was queued; this thread's fence is
+// cumulative over those writes, so the count is raised after H is visible.
+__device__ void wm_signaller(const ExpertArgs &a, SharedCtl *ctl) {
+    for (int q = 0;; ++q) {
+        const int slot = q % SIG_SLOTS;
+        if (!wait_phase(&ctl->sig_full[slot], (q / SIG_SLOTS) & 1, ctl, a.ctr, DEV_TIMEOUT_FULL)) return;
+        const int i = ctl->sig_iact[slot];
+        mbar_arrive(&ctl->sig_empty[slot]);
+        if (i < 0) return;
+        __threadfence();
+        atomicAdd(&a.ctr->gu_done[i], 1);
+    }
+}
+
+// The eight consumer warps of the warp-MMA path (dense mode, B <= WM_MAX):
+// every stage's math and, at a unit's last stage, its epilogue
+//   gate/up: the warps' k-slices are summed in a fixed order (warp w + 4
+//     into warp w, then the four sums), h = silu(g) u -> H (bf16), and the
+//     completion is queued for the signal warp, so that no consumer waits
+//     for the GPU-wide fence;
+//   down:    y[t][row] += wd[slot][t] acc[t][row], each warp its k-half.
+// Thread 0 takes every wait and passes the outcome on through shared
+// memory (by stage parity), so all consumer threads leave together.
+template <class RG>
+__device__ void wm_consumer(const ExpertArgs &a, SharedCtl *ctl, unsigned char *slots, float *part) {
+    constexpr int STAGES = RG::STAGES;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int ct = threadIdx.x;  // 0 .. NCW*32-1
+    const int row = lane >> 2, col = (lane & 3) * 2;
+    const int gk = 64 * a.gc, dk = 64 * d_chunks_of(a.F);
+    float acc_g[4], acc_u[4], wk[2] = {0.0f, 0.0f};
+    bool lists_ready = !a.early;
+    int nsig = 0;  // completions queued (thread 0)
+    for (int g = 0;; ++g) {
+        const int slot = g % STAGES;
+        const unsigned parity = (g / STAGES) & 1;
+        if (ct == 0) ctl->wm_go[g & 1] = wait_phase(&ctl->full[slot], parity, ctl, a.ctr, DEV_TIMEOUT_FULL) ? 1 : 0;
+        consumer_bar();
+        if (!ctl->wm_go[g & 1]) return;
+        // the phase is complete: this thread's own observation of it orders
+        // the copies' data before its reads
+        (void)mbar_try_wait(&ctl->full[slot], parity);
+        if (ct == 0) ctl->consumed = g + 1;
+        const StageHdr h = ctl->hdr[slot];
+        if (h.type == UNIT_END) {
+            if (ct == 0) wm_post(ctl, a.ctr, nsig, -1);
+            return;
+        }
+        if (h.s == 0) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) acc_g[c] = acc_u[c] = 0.0f;
+            if (h.type == UNIT_D) {
+                if (!lists_ready) {
+                    // the dense weights are the selection's last output: in
+                    // early mode wait for them before the first down unit
+                    if (a.lists_flag == nullptr) {
+                        asm volatile("griddepcontrol.wait;" ::: "memory");
+                    } else if (ct == 0) {
+                        int ok = 1;
+                        const unsigned long long t0 = global_ns();
+                        while (ld_acquire(a.lists_flag) < 1) {
+                            if (ctl->abort_flag) { ok = 0; break; }
+                            if (global_ns() - t0 > a.wait_ns) {
+                                record_error(a.ctr, ctl, DEV_TIMEOUT_DEP);
+                                ok = 0;
+                                break;
+                            }
+                            __nanosleep(64);
+                        }
+                        ctl->epi_lists = ok;
+                    }
+                    consumer_bar();
+                    if (!ctl->epi_lists) return;
+                    lists_ready = true;
+                }
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    const int t = col + c;
+                    wk[c] = t < a.B ? __ldcg(a.wd + static_cast<size_t>(h.i_act) * a.B + t) : 0.0f;
+                }
+            }
+        }
+        const uint32_t wbase = smem_u32(slots + slot * RG::SLOT_BYTES);
+        const uint32_t obase = wbase + W_BYTES;
+        if (h.type == UNIT_GU) wm_gu_stage(wbase, obase, min(gk, a.d - h.k * gk) >> 4, warp, lane, acc_g, acc_u);
+        else wm_d_stage(wbase, obase, min(dk, a.F - h.k * dk) >> 4, warp, lane, acc_g);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->empty[slot]);
+        if (h.s != h.ns - 1) continue;
+
+        // ---- unit epilogue (accumulator c: row lane/4 + 8 (c/2), token 2 (lane%4) + c%2)
+        if (h.type == UNIT_D) {
+            const int i_base = h.row0 + (warp & 3) * 16 + row;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int t = col + (c & 1);
+                if (t < a.B && wk[c & 1] != 0.0f)
+                    atomicAdd(a.y + static_cast<size_t>(t) * a.d + i_base + ((c >> 1) << 3), wk[c & 1] * acc_g[c]);
+            }
+            continue;
+        }
+        // gate/up: part holds, per warp pair (w, w + 4), g then u as [16 rows][8 tokens]
+        float *pg = part + (warp & 3) * (2 * WM_ROWS * WM_MAX);
+        float *pu = pg + WM_ROWS * WM_MAX;
+        if (warp >= 4) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int o = (row + ((c >> 1) << 3)) * WM_MAX + col + (c & 1);
+                pg[o] = acc_g[c];
+                pu[o] = acc_u[c];
+            }
+        }
+        consumer_bar();
+        if (warp < 4) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int o = (row + ((c >> 1) << 3)) * WM_MAX + col + (c & 1);
+                pg[o] = acc_g[c] + pg[o];
+                pu[o] = acc_u[c] + pu[o];
+            }
+        }
+        consumer_bar();
+        for (int idx = ct; idx < WM_ROWS * h.n; idx += NCW * 32) {
+            const int r = idx & (WM_ROWS - 1), t = idx >> 4;
+            float gs = 0.0f, us = 0.0f;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                gs += part[q * (2 * WM_ROWS * WM_MAX) + r * WM_MAX + t];
+                us += part[q * (2 * WM_ROWS * WM_MAX) + WM_ROWS * WM_MAX + r * WM_MAX + t];
+            }
+            const float hv = gs / (1.0f + __expf(-gs)) * us;
+            a.h[static_cast<size_t>(h.p0 + t) * a.F + h.row0 + r] = __bfloat16_as_ushort(__float2bfloat16_rn(hv));
+        }
+        // H is read by other CTAs through TMA (the async proxy)
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        consumer_bar();
+        if (ct == 0) wm_post(ctl, a.ctr, nsig++, h.i_act);
+    }
+}
+
 // n_active of caller-supplied lists, checked by the producer warp before
 // any list value is used as an index: 0 <= n_active <= min(E, B*k) (the H
 // and dense-weight slots), every active id an expert, and offsets
@@ -788,16 +1044,22 @@ struct CtaSmem {
 };
 
 // Barriers and flags of a CTA (thread 0).  A stage is released by the
-// issuers' MMA commits.
-template <class RG>
+// issuers' MMA commits (warp-MMA path: by the consumer warps).
+template <class RG, bool WM>
 __device__ void ctl_init(SharedCtl *ctl, unsigned long long wait_ns) {
     for (int s = 0; s < RG::STAGES; ++s) {
         mbar_init(&ctl->full[s], 1);
-        mbar_init(&ctl->empty[s], NISSUE);  // one MMA commit per issuer
+        mbar_init(&ctl->empty[s], WM ? NCW : NISSUE);  // one MMA commit per issuer, or one arrival per warp
     }
     for (int b = 0; b < 2; ++b) {
         mbar_init(&ctl->acc_full[b], NISSUE + 1);  // the first issuer's arrive + every issuer's commit
         mbar_init(&ctl->acc_empty[b], NCW);
+    }
+    if (WM) {
+        for (int q = 0; q < SIG_SLOTS; ++q) {
+            mbar_init(&ctl->sig_full[q], 1);
+            mbar_init(&ctl->sig_empty[q], 1);
+        }
     }
     mbar_init(&ctl->mma_done, NISSUE);
     ctl->epi_lists = 1;
@@ -932,15 +1194,23 @@ __device__ __forceinline__ void tmem_alloc_cta(const ExpertArgs &a, SharedCtl *c
 
 // The roles of an expert CTA: the producer, NISSUE MMA issuer warps (one
 // thread each; the first holds the CTA's TMEM allocation) and eight
-// epilogue warps.
-template <class RG, bool DENSE>
+// epilogue warps; on the warp-MMA path (WM) the producer, eight consumer
+// warps and a signal warp (the other issuer warps idle).
+template <class RG, bool DENSE, bool WM>
 __device__ __forceinline__ void run_roles(const ExpertArgs &a, const ExpertMaps &maps, const CtaSmem<RG> &sm) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if constexpr (WM) {
+        if (warp == NCW) producer<RG, DENSE, true>(a, maps, sm.ctl, sm.slots);
+        else if (warp < NCW) wm_consumer<RG>(a, sm.ctl, sm.slots, sm.part);
+        else if (warp == NCW + 1 && lane == 0) wm_signaller(a, sm.ctl);
+        __syncthreads();
+        return;
+    }
     // the TMEM columns were allocated at kernel entry (tmem_alloc_cta)
     const int cols = tmem_cols_for(a.hrows);
     const uint32_t tmem = sm.ctl->tmem;
     if (warp == NCW) {
-        producer<RG, DENSE>(a, maps, sm.ctl, sm.slots);
+        producer<RG, DENSE, false>(a, maps, sm.ctl, sm.slots);
     } else if (warp > NCW) {
         if (lane == 0) umma_issuer(a, sm.ctl, sm.slots, RG::STAGES, RG::SLOT_BYTES, tmem, warp - NCW - 1);
     } else {
@@ -981,16 +1251,16 @@ __device__ void cta_exit(const ExpertArgs &a, SharedCtl *ctl) {
     }
 }
 
-template <class RG>
+template <class RG, bool WM>
 __global__ void __launch_bounds__(NTHREADS, 1)
     expert_ffn_kernel(const __grid_constant__ ExpertMaps maps, const ExpertArgs a) {
     extern __shared__ unsigned char smem_raw[];
     const CtaSmem<RG> sm(smem_raw);
     SharedCtl *ctl = sm.ctl;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (threadIdx.x == 0) ctl_init<RG>(ctl, a.wait_ns);
+    if (threadIdx.x == 0) ctl_init<RG, WM>(ctl, a.wait_ns);
     if (warp == NCW && lane == 0) prefetch_expert_maps(maps);
-    tmem_alloc_cta(a, ctl);
+    if (!WM) tmem_alloc_cta(a, ctl);
     // everything above overlaps the previous kernel (selection or input
     // preparation); the lists are complete once it has
     asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -998,7 +1268,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    run_roles<RG, false>(a, maps, sm);
+    run_roles<RG, false, WM>(a, maps, sm);
     cta_exit(a, ctl);
 }
 
@@ -1073,7 +1343,7 @@ __device__ __forceinline__ void rank_union(const ExpertArgs &a, const LayerArgs 
     }
 }
 
-template <class RG, int NI>
+template <class RG, int NI, bool WM>
 __global__ void __launch_bounds__(NTHREADS, 1)
     layer_kernel(const __grid_constant__ ExpertMaps maps, const __grid_constant__ RouterMaps rmaps,
                  const ExpertArgs a, const LayerArgs L) {
@@ -1125,7 +1395,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 issue_rows(item, true, false);
             }
         }
-        ctl_init<RG>(ctl, a.wait_ns);
+        ctl_init<RG, WM>(ctl, a.wait_ns);
         s_ok = 1;
     }
     if (threadIdx.x < E_MAX / 32) s_set[threadIdx.x] = 0u;
@@ -1134,8 +1404,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         prefetch_tmap(&rmaps.x);
         prefetch_tmap(&rmaps.wg);
     }
-    // the expert CTAs' TMEM columns (the selection CTA runs no MMAs)
-    if (blockIdx.x != gridDim.x - 1) tmem_alloc_cta(a, ctl);
+    // the expert CTAs' TMEM columns (the selection CTA runs no MMAs, the
+    // warp-MMA path none on the tensor-core pipe)
+    if (!WM && blockIdx.x != gridDim.x - 1) tmem_alloc_cta(a, ctl);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -1259,7 +1530,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     // only the producer warp, which built it, reads the unit table: the
     // other roles start at once
-    run_roles<RG, true>(a, maps, sm);
+    run_roles<RG, true, WM>(a, maps, sm);
     cta_exit(a, ctl);
 }
 
@@ -1385,13 +1656,16 @@ int g_num_sms[MAX_DEVICES] = {0};
 
 int expert_ffn_h_rows(int B) { return B <= DENSE_MAX ? (B + 7) / 8 * 8 : TN; }
 int expert_ffn_dense_batch(int B) { return B <= DENSE_MAX ? 1 : 0; }
-int expert_ffn_gu_rows(int) { return UM_ROWS; }
-int expert_ffn_d_rows() { return D_ROWS; }
-int expert_ffn_gu_chunks(int d, int B) {
-    (void)B;
-    return d / 64 < UM_CHUNKS ? d / 64 : UM_CHUNKS;
+int expert_ffn_warp_mma(const moe_dims_t &d, int max_active) {
+    return d.B <= WM_MAX && max_active <= WM_ACTIVE_MAX ? 1 : 0;
 }
-int expert_ffn_gu_box_chunks(int, int) { return 1; }
+int expert_ffn_gu_rows(int wm) { return wm ? WM_ROWS : UM_ROWS; }
+int expert_ffn_d_rows() { return D_ROWS; }
+int expert_ffn_gu_chunks(int d, int wm) {
+    const int c = wm ? WM_CHUNKS : UM_CHUNKS;
+    return d / 64 < c ? d / 64 : c;
+}
+int expert_ffn_gu_box_chunks(int d, int wm) { return wm ? expert_ffn_gu_chunks(d, wm) : 1; }
 int expert_ffn_d_chunks(int F) { return F / 64 < D_CHUNKS ? F / 64 : D_CHUNKS; }
 
 cudaError_t launch_ffn_prep(const float *x, const moe_dims_t &d, uint16_t *xb, uint16_t *xd, float *y,
@@ -1467,7 +1741,7 @@ cudaError_t configure_smem(K kernel, int bytes, int dev) {
 
 // Expert-stream arguments for dims d, units dealt to `unit_ctas` CTAs.
 ExpertArgs make_expert_args(const uint16_t *xb, const moe_dims_t &d, const moe_lists_t &l, float *y, uint16_t *h,
-                            const float *wd, Counters *ctr, int unit_ctas) {
+                            const float *wd, Counters *ctr, int unit_ctas, int wm) {
     ExpertArgs a;
     a.xb = xb;
     a.B = d.B;
@@ -1479,8 +1753,8 @@ ExpertArgs make_expert_args(const uint16_t *xb, const moe_dims_t &d, const moe_l
     a.unit_ctas = unit_ctas;
     a.lists_flag = nullptr;
     a.dense = d.B <= DENSE_MAX ? 1 : 0;
-    a.gu_rows = expert_ffn_gu_rows(d.B);
-    a.gc = expert_ffn_gu_chunks(d.d, d.B);
+    a.gu_rows = expert_ffn_gu_rows(wm);
+    a.gc = expert_ffn_gu_chunks(d.d, wm);
     a.bpad = (d.B + 7) / 8 * 8;
     a.hrows = expert_ffn_h_rows(d.B);
     a.early = 0;
@@ -1544,10 +1818,10 @@ LayerArgs make_layer_router(const moe_dims_t &d, int grid, int ring_bytes) {
     return L;
 }
 
-template <class RG, int NI>
+template <class RG, int NI, bool WM>
 cudaError_t launch_layer_ni(const ExpertMaps &maps, const RouterMaps &rmaps, const ExpertArgs &a,
                             const LayerArgs &L, int grid, int dev, cudaStream_t s) {
-    cudaError_t err = configure_smem(layer_kernel<RG, NI>, smem_bytes<RG>(), dev);
+    cudaError_t err = configure_smem(layer_kernel<RG, NI, WM>, smem_bytes<RG>(), dev);
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
@@ -1564,15 +1838,15 @@ cudaError_t launch_layer_ni(const ExpertMaps &maps, const RouterMaps &rmaps, con
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = L.chained ? 2 : 1;
-    return cudaLaunchKernelEx(&cfg, layer_kernel<RG, NI>, maps, rmaps, a, L);
+    return cudaLaunchKernelEx(&cfg, layer_kernel<RG, NI, WM>, maps, rmaps, a, L);
 }
 
 }  // namespace
 
 namespace {
-template <class RG>
+template <class RG, bool WM>
 cudaError_t launch_expert_ffn_rg(const ExpertMaps &maps, const ExpertArgs &a, int sms, int dev, cudaStream_t s) {
-    cudaError_t err = configure_smem(expert_ffn_kernel<RG>, smem_bytes<RG>(), dev);
+    cudaError_t err = configure_smem(expert_ffn_kernel<RG, WM>, smem_bytes<RG>(), dev);
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(sms);
@@ -1584,36 +1858,38 @@ cudaError_t launch_expert_ffn_rg(const ExpertMaps &maps, const ExpertArgs &a, in
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;  // always chained to the previous kernel with programmatic dependent launch
-    return cudaLaunchKernelEx(&cfg, expert_ffn_kernel<RG>, maps, a);
+    return cudaLaunchKernelEx(&cfg, expert_ffn_kernel<RG, WM>, maps, a);
 }
 }  // namespace
 
 cudaError_t launch_expert_ffn(const ExpertMaps &maps, const uint16_t *xb, const moe_dims_t &d,
-                              const moe_lists_t &l, float *y, uint16_t *h, const float *wd, Counters *ctr,
+                              const moe_lists_t &l, float *y, uint16_t *h, const float *wd, Counters *ctr, int wm,
                               cudaStream_t s) {
+    if (wm && d.B > WM_MAX) return cudaErrorInvalidValue;
     int dev = 0, sms = 0;
     cudaError_t err = device_sms(&dev, &sms);
     if (err != cudaSuccess) return err;
-    const ExpertArgs a = make_expert_args(xb, d, l, y, h, wd, ctr, sms);
-    // the ring sized for the token rows: dense mode up to 16, 32 or 64
-    // tokens, tile mode (64 pair rows) above
-    if (d.B <= 16) return launch_expert_ffn_rg<RingB16>(maps, a, sms, dev, s);
-    if (d.B <= 32) return launch_expert_ffn_rg<RingB32>(maps, a, sms, dev, s);
-    return launch_expert_ffn_rg<RingB64>(maps, a, sms, dev, s);
+    const ExpertArgs a = make_expert_args(xb, d, l, y, h, wd, ctr, sms, wm);
+    // the warp-MMA path, or the ring sized for the token rows: dense mode
+    // up to 16, 32 or 64 tokens, tile mode (64 pair rows) above
+    if (wm) return launch_expert_ffn_rg<RingB16, true>(maps, a, sms, dev, s);
+    if (d.B <= 16) return launch_expert_ffn_rg<RingB16, false>(maps, a, sms, dev, s);
+    if (d.B <= 32) return launch_expert_ffn_rg<RingB32, false>(maps, a, sms, dev, s);
+    return launch_expert_ffn_rg<RingB64, false>(maps, a, sms, dev, s);
 }
 
 cudaError_t launch_layer_fused(const ExpertMaps &maps, const RouterMaps &rmaps, const moe_dims_t &d,
                                const moe_reselect_t &rule, const float *x, const float *bias, float *logits,
                                float *probs, uint16_t *xb, float *y, uint16_t *h, float *wd, int32_t *sel_idx,
                                float *sel_w, const moe_lists_t &lists, int32_t *n_active_copy, Counters *ctr,
-                               bool residual, bool chained, cudaStream_t s) {
-    if (d.B > DENSE_MAX) return cudaErrorInvalidValue;
+                               int wm, bool residual, bool chained, cudaStream_t s) {
+    if (d.B > DENSE_MAX || (wm && d.B > WM_MAX)) return cudaErrorInvalidValue;
     int dev = 0, sms = 0;
     cudaError_t err = device_sms(&dev, &sms);
     if (err != cudaSuccess) return err;
     if (sms < 2) return cudaErrorInvalidConfiguration;
     // the last CTA runs the selection; the others stream the experts
-    ExpertArgs a = make_expert_args(xb, d, lists, y, h, wd, ctr, sms - 1);
+    ExpertArgs a = make_expert_args(xb, d, lists, y, h, wd, ctr, sms - 1, wm);
     a.early = 1;
     a.lists_flag = &ctr->lists_ready;
     const bool batch_rule = rule.mode == MOE_RESELECT_XSHARE || rule.mode == MOE_RESELECT_AFFINITY ||
@@ -1635,15 +1911,17 @@ cudaError_t launch_layer_fused(const ExpertMaps &maps, const RouterMaps &rmaps, 
     L.sel.publish_set = batch_rule ? 1 : 0;
     const size_t sel_smem = reselect_smem(d, rule, &L.sel.cache_rows);
     if (sel_smem > static_cast<size_t>(ring)) return cudaErrorInvalidValue;
-    // instantiated per ring (up to 16, 32 or 64 tokens) and for logit rows
-    // of up to 128 or 256 experts per warp
+    // instantiated for the warp-MMA path (up to WM_MAX tokens) and per ring
+    // (up to 16, 32 or 64 tokens), and for logit rows of up to 128 or 256
+    // experts per warp
     const bool ni8 = ni_for(d.E) > 4;
-#define MOE_LAYER_CASE(RGT)                                                                            \
-    return ni8 ? launch_layer_ni<RGT, 8>(maps, rmaps, a, L, sms, dev, s)                              \
-               : launch_layer_ni<RGT, 4>(maps, rmaps, a, L, sms, dev, s)
-    if (d.B <= 16) MOE_LAYER_CASE(RingB16);
-    if (d.B <= 32) MOE_LAYER_CASE(RingB32);
-    MOE_LAYER_CASE(RingB64);
+#define MOE_LAYER_CASE(RGT, WMV)                                                                       \
+    return ni8 ? launch_layer_ni<RGT, 8, WMV>(maps, rmaps, a, L, sms, dev, s)                         \
+               : launch_layer_ni<RGT, 4, WMV>(maps, rmaps, a, L, sms, dev, s)
+    if (wm) MOE_LAYER_CASE(RingB16, true);
+    if (d.B <= 16) MOE_LAYER_CASE(RingB16, false);
+    if (d.B <= 32) MOE_LAYER_CASE(RingB32, false);
+    MOE_LAYER_CASE(RingB64, false);
 #undef MOE_LAYER_CASE
 }
 

@@ -127,18 +127,19 @@ struct ExpertMaps {
 // (chained with programmatic dependent launch) or the caller; wd: dense
 // weights (B <= 64).
 cudaError_t launch_expert_ffn(const ExpertMaps &maps, const uint16_t *xb, const moe_dims_t &d,
-                              const moe_lists_t &l, float *y, uint16_t *h, const float *wd, Counters *ctr,
+                              const moe_lists_t &l, float *y, uint16_t *h, const float *wd, Counters *ctr, int wm,
                               cudaStream_t s);
 // The whole layer in one cooperative persistent kernel (B <= 64): router,
 // grid barrier, selection (last CTA), expert stream (the other CTAs).  xb:
 // x in bf16 (written), h: the SwiGLU scratch, wd: the dense weights.
-// residual: y = x + the experts' output; chained: launched with
-// programmatic dependent launch after the previous layer of a stack.
+// wm: the warp-MMA expert stream (expert_ffn_warp_mma); residual: y = x +
+// the experts' output; chained: launched with programmatic dependent launch
+// after the previous layer of a stack.
 cudaError_t launch_layer_fused(const ExpertMaps &maps, const RouterMaps &rmaps, const moe_dims_t &d,
                                const moe_reselect_t &rule, const float *x, const float *bias, float *logits,
                                float *probs, uint16_t *xb, float *y, uint16_t *h, float *wd, int32_t *sel_idx,
                                float *sel_w, const moe_lists_t &lists, int32_t *n_active_copy, Counters *ctr,
-                               bool residual, bool chained, cudaStream_t s);
+                               int wm, bool residual, bool chained, cudaStream_t s);
 // Per-token channel top-k (channels.cu): workspace bytes, ring stages of the
 // stream kernel for d (0: the dims do not fit its shared memory), the
 // channel-major copy of Wdown, and the three kernels of one call.
@@ -153,15 +154,20 @@ cudaError_t launch_channels(const float *x, const uint16_t *Wgate, const uint16_
 unsigned long long wait_limit_ns();
 int expert_ffn_h_rows(int B);         // rows of one H box
 int expert_ffn_dense_batch(int B);    // 1 if gate/up stages load all B token rows at once
-int expert_ffn_gu_rows(int B);        // rows of Wgate / Wup per gate-up unit
+// 1 if the expert stream of a call runs on warp-level MMAs (16-row gate/up
+// units): at most 8 tokens and at most 32 activated experts (max_active:
+// the most the call's rule can activate)
+int expert_ffn_warp_mma(const moe_dims_t &d, int max_active);
+int expert_ffn_gu_rows(int wm);       // rows of Wgate / Wup per gate-up unit
 int expert_ffn_d_rows();              // rows of Wdown per down unit
-int expert_ffn_gu_chunks(int d, int B);  // 64-column chunks of d per gate-up stage
-int expert_ffn_gu_box_chunks(int d, int B);  // chunks per gate (or up) copy: 1 in dense mode
+int expert_ffn_gu_chunks(int d, int wm);  // 64-column chunks of d per gate-up stage
+int expert_ffn_gu_box_chunks(int d, int wm);  // chunks per gate (or up) copy: 1, or a stage's on the warp-MMA path
 int expert_ffn_d_chunks(int d_ff);    // 64-column chunks of d_ff per down stage
 
 // Builds the expert kernel's TMA descriptors (weights, H scratch at `h`,
-// bf16 x at `x`: xb [B][d] for B <= 64, xd [B*k][d] above).
+// bf16 x at `x`: xb [B][d] for B <= 64, xd [B*k][d] above); wm: the
+// gate/up boxes of the warp-MMA path.
 bool encode_expert_maps(ExpertMaps *m, const moe_dims_t &d, const uint16_t *Wgate, const uint16_t *Wup,
-                        const uint16_t *Wdown, const uint16_t *h, const uint16_t *x);
+                        const uint16_t *Wdown, const uint16_t *h, const uint16_t *x, int wm);
 
 }  // namespace moe

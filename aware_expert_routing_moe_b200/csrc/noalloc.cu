@@ -101,14 +101,16 @@ extern "C" moe_status_t moe_expert_ffn_noalloc(const float *x, const uint16_t *W
     uint16_t *xk = reinterpret_cast<uint16_t *>(scratch + (dense ? L.xb : L.xd));
     uint16_t *h = reinterpret_cast<uint16_t *>(scratch + L.h);
     float *wd = dense ? reinterpret_cast<float *>(scratch + L.wd) : nullptr;
+    // caller-supplied lists: any union of the tokens' k choices
+    const int wm = expert_ffn_warp_mma(dims, dims.B * dims.k);
     ExpertMaps maps;
-    if (!encode_expert_maps(&maps, dims, Wgate, Wup, Wdown, h, xk)) return MOE_ERR_CUDA;
+    if (!encode_expert_maps(&maps, dims, Wgate, Wup, Wdown, h, xk, wm)) return MOE_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     // the prep kernel clears the per-expert counters the expert kernel needs
     // at zero and rebuilds x, the dense weights and (in the kernel) H
     if (launch_ffn_prep(x, dims, dense ? xk : nullptr, dense ? nullptr : xk, y, ctr, lists, wd, false, s) !=
         cudaSuccess)
         return MOE_ERR_CUDA;
-    if (launch_expert_ffn(maps, xk, dims, lists, y, h, wd, ctr, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_expert_ffn(maps, xk, dims, lists, y, h, wd, ctr, wm, s) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;
 }

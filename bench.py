@@ -54,6 +54,8 @@ ROTATE = 4
 
 WORKLOADS = {
     "q30b_b16_oea4": dict(shape="q30b", B=16, mode=1, k0=4, budget=0, rule="OEA k0=4"),
+    # up to 8 tokens and 32 activated experts: the warp-MMA expert stream
+    "q30b_b4_oea4": dict(shape="q30b", B=4, mode=1, k0=4, budget=0, rule="OEA k0=4"),
     "q30b_b16_none": dict(shape="q30b", B=16, mode=0, k0=0, budget=0, rule="NONE (standard top-8)"),
     "q30b_b64_oea4": dict(shape="q30b", B=64, mode=1, k0=4, budget=0, rule="OEA k0=4"),
     "q30b_b96_oea4": dict(shape="q30b", B=96, mode=1, k0=4, budget=0, rule="OEA k0=4"),
@@ -73,12 +75,13 @@ WORKLOADS = {
 
 # DRAM bytes (read + write) per launch of the dominant kernel (the fused
 # layer kernel up to 64 tokens) from an ncu capture of the same workload on
-# one weight copy (profiles/layer_kernel_q30b_b16_oea4.md, ..._b64_...);
-# a workload without an entry reports null.  Entries are dropped whenever
-# the kernel changes.
+# one weight copy (profiles/layer_kernel_q30b_b16_oea4.md, ..._b64_...,
+# ..._b4_...); a workload without an entry reports null.  Entries are
+# dropped whenever the kernel changes.
 NCU_TRAFFIC = {
-    "q30b_b16_oea4": 142883072 + 3001856,
-    "q30b_b64_oea4": 284835840 + 3391232,
+    "q30b_b16_oea4": 142884608 + 3348480,
+    "q30b_b64_oea4": 284837120 + 5679104,
+    "q30b_b4_oea4": 105041664 + 2753280,
     # channel top-k workloads: channel_stream_kernel, which moves the weights
     # (profiles/channel_stream_kernel_q30b_oea4_ch13.md)
     "q30b_b1_oea4_ch13": 4969984,
@@ -471,7 +474,7 @@ SWEEP = {
     # ROTATE copies); mode 4 (hierarchical XShare) takes the request size
     "tiny": [(4, 1, 2, 0, "normal"), (4, 0, 0, 0, "normal")],
     "e64": [(16, 1, 4, 0, "normal"), (16, 0, 0, 0, "normal")],
-    "q30b": [(b, m, k0, 0, "normal") for b in (1, 4, 16, 32, 48, 64, 128) for (m, k0) in ((0, 0), (1, 4))]
+    "q30b": [(b, m, k0, 0, "normal") for b in (1, 4, 8, 16, 32, 48, 64, 128) for (m, k0) in ((0, 0), (1, 4))]
             + [(16, 1, k0, 0, "normal") for k0 in (2, 6, 8)]
             + [(32, 0, 0, 0, "spec")] + [(32, 2, 0, m, "spec") for m in (24, 32, 48)]
             + [(16, 3, 0, 0, "normal"), (64, 3, 0, 0, "normal"), (32, 3, 0, 0, "spec")]

@@ -172,6 +172,7 @@ LAYER_CASES = [
     ("maxek", 256, 0, NONE, 0, 0), ("maxek", 256, 0, OEA, 8, 0), ("maxek", 100, 0, XSHARE, 0, 40),
     ("tiny", 4, 1, AFFINITY, 0, 0), ("ragged", 37, 0, AFFINITY, 0, 0), ("maxek", 256, 0, AFFINITY, 0, 0),
     ("e64", 16, 0, NONE, 0, 0), ("e64", 16, 0, OEA, 4, 0),
+    ("ragged", 6, 0, OEA, 2, 0), ("ragged", 8, 0, XSHARE, 0, 10),
 ]
 
 
@@ -186,7 +187,12 @@ def test_layer_decode_parity_small(name, B, seed, mode, k0, budget):
     assert_close_y(y if rows is None else y[rows], y_r, f"{name} B={B} mode={mode}")
 
 
-Q30_CASES = [(1, NONE, 0, 0), (1, OEA, 2, 0), (4, OEA, 4, 0), (16, NONE, 0, 0), (16, OEA, 2, 0),
+Q30_CASES = [(1, NONE, 0, 0), (1, OEA, 2, 0), (4, OEA, 4, 0),
+             # up to 8 tokens and at most 32 activated experts: warp-level
+             # MMAs on 16-row gate/up units; 8 tokens top-8 and 9 tokens:
+             # the tensor-core stream
+             (5, XSHARE, 0, 12), (8, NONE, 0, 0), (8, OEA, 4, 0), (9, OEA, 4, 0),
+             (16, NONE, 0, 0), (16, OEA, 2, 0),
              (16, OEA, 4, 0), (16, OEA, 6, 0), (16, OEA, 8, 0), (16, XSHARE, 0, 16), (16, AFFINITY, 0, 0),
              (64, AFFINITY, 0, 0), (32, NONE, 0, 0), (17, OEA, 4, 0),
              # 33..64 tokens: the 64-row ring (ragged token counts included)
@@ -236,7 +242,7 @@ def test_layer_decode_parity_xshare_hier(name, B, group, budget):
     assert_close_y(y if rows is None else y[rows], y_r, f"{name} B={B} hierarchical group={group} budget={budget}")
 
 
-@pytest.mark.parametrize("B,mode,k0", [(1, OEA, 4), (16, NONE, 0), (16, OEA, 4), (64, OEA, 4)])
+@pytest.mark.parametrize("B,mode,k0", [(1, OEA, 4), (8, OEA, 4), (16, NONE, 0), (16, OEA, 4), (64, OEA, 4)])
 def test_layer_decode_parity_q235b(B, mode, k0):
     S, L, x, y, sel, selw, n_act = _run_layer("q235b", B, 0, mode, k0)
     sel_r, w_r, n_r, y_r = _oracle_layer(S, L, x, mode, k0, 0, None)
@@ -245,9 +251,11 @@ def test_layer_decode_parity_q235b(B, mode, k0):
     assert_close_y(y, y_r, f"q235b B={B} mode={mode}")
 
 
-def test_expert_ffn_entry_matches_oracle():
-    # the FFN stage alone, fed the oracle's own lists
-    name, B = "q30b", 16
+@pytest.mark.parametrize("B", [4, 16])
+def test_expert_ffn_entry_matches_oracle(B):
+    # the FFN stage alone, fed the oracle's own lists (4 tokens: warp-level
+    # MMAs, 16: the tensor cores)
+    name = "q30b"
     S = shape(name)
     L = host_layer(name, 0)
     D = device_layer(name, 0)

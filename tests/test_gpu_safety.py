@@ -59,9 +59,10 @@ def _ffn(name, x, dl, ws):
     return y, moe.moe_check_error(ws)
 
 
-# tiny (B = 4), ragged (B = 37): dense mode; ragged (B = 70): token tiles of
-# the dispatched pairs
-@pytest.mark.parametrize("name,B,k0", [("tiny", 4, 2), ("ragged", 37, 2), ("ragged", 70, 2)])
+# tiny (B = 4): dense mode on warp-level MMAs; ragged (B = 9, 37): dense
+# mode on the tensor cores; ragged (B = 70): token tiles of the dispatched
+# pairs
+@pytest.mark.parametrize("name,B,k0", [("tiny", 4, 2), ("ragged", 37, 2), ("ragged", 70, 2), ("ragged", 9, 2)])
 @pytest.mark.parametrize("damage", ["n_active_above_E", "n_active_negative", "active_id_out_of_range",
                                     "offsets_decreasing", "offsets_past_pairs"])
 def test_inconsistent_lists_are_reported_and_contained(name, B, k0, damage):
@@ -114,15 +115,17 @@ def test_token_outside_batch_is_skipped_and_reported(name, B, k0):
 
 
 # ------------------------------------------------------------ bounded waits --
-@pytest.mark.parametrize("path", ["layer_fused", "expert_ffn", "layer_tiled"])
+@pytest.mark.parametrize("path", ["layer_fused", "expert_ffn", "layer_tiled", "layer_fused_b4", "expert_ffn_b4"])
 def test_bounded_waits_expire_and_report(path):
     # With a 200 ns limit every wait on a copy, on another CTA or on a flag
     # runs out: each CTA records the error, lets its copies in flight land,
     # ends its share of the call and exits; the call completes and
     # moe_check_error reports MOE_ERR_INTERNAL.  After the default limit is
     # restored and the workspace zeroed, the same call matches the oracle.
-    # the four-kernel path starts above 64 tokens
-    name, B = ("q30b", 16) if path != "layer_tiled" else ("q30b", 96)
+    # the four-kernel path starts above 64 tokens; up to 8 tokens the expert
+    # stream runs on warp-level MMAs
+    name, B = {"layer_tiled": ("q30b", 96), "layer_fused_b4": ("q30b", 4),
+               "expert_ffn_b4": ("q30b", 4)}.get(path, ("q30b", 16))
     S = shape(name)
     L = host_layer(name, 0)
     D = device_layer(name, 0)
@@ -134,7 +137,7 @@ def test_bounded_waits_expire_and_report(path):
     li = oracle.lists(sel, w, S.E)
 
     def call():
-        if path == "expert_ffn":
+        if path.startswith("expert_ffn"):
             y = moe.moe_expert_ffn(xd, D["Wgate"], D["Wup"], D["Wdown"], _device_lists(li, S.E, B, S.k), S.k, ws)
         else:
             y = moe.moe_layer_decode(xd, D["Wg"], D["bias"], D["Wgate"], D["Wup"], D["Wdown"], S.k, OEA, 4, ws=ws)
