@@ -119,9 +119,16 @@ cudaError_t launch_ffn_prep(const float *x, const moe_dims_t &d, uint16_t *xb, u
 
 // TMA descriptors of the expert kernel: the three weight tensors, the H
 // scratch and the bf16 x rows (xb for B <= 64, the dispatched pair rows xd
-// above) as (64-column chunk, row, chunk index) boxes.
+// above) as (64-column chunk, row, chunk index) boxes.  gu: Wgate and Wup
+// as one 4-D tensor whose matrix dimension steps from the lower of the two
+// buffers to the higher, so that one box holds a whole gate/up stage in
+// the tensor-core stage's layout; gu_mode 0: not used (the warp-MMA
+// path) or not encodable (the buffers coincide, or their distance is no
+// valid TMA stride), the stage takes per-matrix boxes; 1: Wgate is the
+// lower buffer; 2: Wup is (gate and up halves swapped in shared memory).
 struct ExpertMaps {
-    CUtensorMap gate, up, down, h, x;
+    CUtensorMap gate, up, down, h, x, gu;
+    int gu_mode;
 };
 // The expert kernel alone (moe_expert_ffn): lists from the previous kernel
 // (chained with programmatic dependent launch) or the caller; wd: dense

@@ -75,13 +75,12 @@ WORKLOADS = {
 
 # DRAM bytes (read + write) per launch of the dominant kernel (the fused
 # layer kernel up to 64 tokens) from an ncu capture of the same workload on
-# one weight copy (profiles/layer_kernel_q30b_b16_oea4.md, ..._b64_...,
-# ..._b4_...); a workload without an entry reports null.  Entries are
-# dropped whenever the kernel changes.
+# one weight copy (profiles/layer_kernel_q30b_b16_oea4.md, ..._b64_...);
+# a workload without an entry reports null.  Entries are dropped whenever
+# the kernel changes.
 NCU_TRAFFIC = {
-    "q30b_b16_oea4": 142884608 + 3348480,
-    "q30b_b64_oea4": 284837120 + 5679104,
-    "q30b_b4_oea4": 105041664 + 2753280,
+    "q30b_b16_oea4": 142883840 + 3248896,
+    "q30b_b64_oea4": 284837120 + 4763904,
     # channel top-k workloads: channel_stream_kernel, which moves the weights
     # (profiles/channel_stream_kernel_q30b_oea4_ch13.md)
     "q30b_b1_oea4_ch13": 4969984,

@@ -252,6 +252,51 @@ def test_layer_decode_parity_q235b(B, mode, k0):
 
 
 @pytest.mark.parametrize("B", [4, 16])
+@pytest.mark.parametrize("layout", ["up_below_gate", "gate_is_up"])
+def test_gate_up_buffer_layouts(B, layout):
+    # A gate/up stage is copied as one box of Wgate and Wup seen as a single
+    # tensor whose matrix dimension steps from the lower buffer to the
+    # higher; when Wup lies below Wgate the two halves swap, and when both
+    # arguments are the same buffer the stage falls back to one box per
+    # matrix.  Both cases must give the oracle's layer (4 tokens: warp-level
+    # MMAs, 16: the tensor cores), through the fused layer and the expert
+    # entry point.
+    name = "q30b"
+    S = shape(name)
+    L = host_layer(name, 0)
+    D = device_layer(name, 0)
+    x = _tokens(name, B, 0)
+    xd = torch.from_numpy(x).cuda()
+    if layout == "up_below_gate":
+        both = torch.empty((2,) + tuple(D["Wgate"].shape), dtype=D["Wgate"].dtype, device="cuda")
+        both[0].copy_(D["Wup"])
+        both[1].copy_(D["Wgate"])
+        wgate, wup, up_host = both[1], both[0], L["Wup"]
+        assert wup.data_ptr() < wgate.data_ptr()
+    else:
+        wgate, wup, up_host = D["Wgate"], D["Wgate"], L["Wgate"]
+    ws = moe.new_workspace(B, S.d, S.E, S.k, S.F)
+    sel = torch.empty(B, S.k, dtype=torch.int32, device="cuda")
+    selw = torch.empty(B, S.k, dtype=torch.float32, device="cuda")
+    y = moe.moe_layer_decode(xd, D["Wg"], D["bias"], wgate, wup, D["Wdown"], S.k, OEA, 4, ws=ws, sel_idx=sel,
+                             sel_w=selw)
+    assert moe.moe_check_error(ws) == 0
+    logits, probs, _, _ = oracle.route(x, L["Wg"], L["bias"], S.k)
+    sel_r, w_r = oracle.reselect(logits, probs, S.k, OEA, 4, 0)
+    assert np.array_equal(sel.cpu().numpy(), sel_r)
+    y_r = oracle.ffn(x, L["Wgate"], up_host, L["Wdown"], sel_r, w_r, threads=THREADS)
+    assert_close_y(y.cpu().numpy(), y_r, f"layer, {layout}, B={B}")
+    li = oracle.lists(sel_r, w_r, S.E)
+    dl = {"n_active": torch.tensor([li["n_active"], 0, 0, 0], dtype=torch.int32).cuda(),
+          "active": torch.from_numpy(li["active"]).cuda(), "offsets": torch.from_numpy(li["offsets"]).cuda(),
+          "tok": torch.from_numpy(li["tok"]).cuda(), "w": torch.from_numpy(li["w"]).cuda()}
+    ws.zero_()
+    y2 = moe.moe_expert_ffn(xd, wgate, wup, D["Wdown"], dl, S.k, ws)
+    assert moe.moe_check_error(ws) == 0
+    assert_close_y(y2.cpu().numpy(), y_r, f"moe_expert_ffn, {layout}, B={B}")
+
+
+@pytest.mark.parametrize("B", [4, 16])
 def test_expert_ffn_entry_matches_oracle(B):
     # the FFN stage alone, fed the oracle's own lists (4 tokens: warp-level
     # MMAs, 16: the tensor cores)
