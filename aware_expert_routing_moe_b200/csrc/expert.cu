@@ -8,7 +8,7 @@
 // Retraining", abstract).
 //
 // Work units, dealt round robin to persistent CTAs (one per SM):
-//   GU unit (expert e, token tile, 32 rows of d_ff):
+//   GU unit (expert e, token tile, 32 rows of d_ff; 16 on the warp-MMA path):
 //       g = Wgate[e][rows] x_t, u = Wup[e][rows] x_t over all of d,
 //       h = silu(g) * u -> H scratch (bf16);
 //   D unit (expert e, token tile, 64-row block of d):
