@@ -103,3 +103,28 @@ def test_channel_bytes_match_the_oracle_sector_count(oracle_lib):
     bits = np.packbits(keep, axis=-1, bitorder="little").view(np.uint32)
     got = bench.channel_bytes(bits, sel, d, F, B, k) - (B * k * F * 4 + 2 * B * d * 4)
     assert got == oracle_lib.channel_sector_bytes(keep, sel, E, d, down_channel_major=True)
+
+
+def test_recorded_layer_traffic_matches_the_algorithmic_bytes():
+    # Each ncu traffic entry of the fused layer kernel (DRAM bytes read +
+    # written per launch, from the capture of that workload) must cover the
+    # call's algorithmic bytes and exceed them by at most 3 %: every
+    # activated expert's weights read once, the rest small writes (y, H,
+    # logits, the selection's outputs).  The activated count comes from the
+    # oracle's routing of the workload's own seeded inputs.
+    import oracle
+    checked = 0
+    for name, traffic in bench.NCU_TRAFFIC.items():
+        w = bench.WORKLOADS[name]
+        if "channels" in w:
+            continue  # sector-counted bytes, checked against the oracle above
+        S = ms.SHAPES[w["shape"]]
+        L = ms.make_weights(S, 0, experts=False)
+        x = ms.make_tokens(S, w["B"], 0, kind=w.get("kind", "normal"))
+        logits, probs, _, _ = oracle.route(x, L["Wg"], L["bias"], S.k)
+        sel, wt = oracle.reselect(logits, probs, S.k, w["mode"], w["k0"], w["budget"], w.get("group", 1))
+        n_active = oracle.lists(sel, wt, S.E)["n_active"]
+        total, _ = bench.algorithmic_bytes(S, w["B"], n_active)
+        assert total <= traffic <= 1.03 * total, (name, n_active, total, traffic)
+        checked += 1
+    assert checked >= 1
